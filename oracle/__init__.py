@@ -1,0 +1,289 @@
+"""Oracle for the single-device Megatron-style tensor-parallel layer.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package.  The product library
+never calls into it, and it shares no code with the CUDA path: the arithmetic
+lives in ``tpl_oracle.c`` (plain fp64 loops), this module only marshals numpy
+arrays through ctypes.
+
+Every function cites the page passage it follows, by page title and section:
+
+* "Tensor parallel scaling curves", section "What tensor parallelism actually
+  splits" -- head-wise column split of Q/K/V, local attention on owned heads,
+  row split of the output projection, gate/up column split, down row split,
+  partial sums added (two per layer, 2L per pass).
+* "Tensor Parallelism Fundamentals", sections "Mechanics of Matrix Slicing" and
+  "Memory Overhead and Communication Bottlenecks" -- column-then-row slicing,
+  weights divided by t, the per-GPU KV formula.
+
+Parity status: every function here is pinned by ``tests/test_oracle.py``
+(closed forms, exact integer identities, the pages' worked numbers and an
+independent numpy float64 evaluation).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "tpl_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+
+NORM = 1
+RESIDUAL = 2
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle (gcc, -O2, no fast-math, no FP contraction)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
+               "-std=c11", "-o", _LIB_PATH + ".tmp", _SRC, "-lm"]
+        subprocess.check_call(cmd)
+        os.replace(_LIB_PATH + ".tmp", _LIB_PATH)
+    return _LIB_PATH
+
+
+class _Dims(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int32), ("n_q_heads", ctypes.c_int32),
+                ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("ffn", ctypes.c_int32), ("eps", ctypes.c_double), ("flags", ctypes.c_uint32)]
+
+
+class _Weights(ctypes.Structure):
+    _fields_ = [("wq", ctypes.c_void_p), ("wk", ctypes.c_void_p), ("wv", ctypes.c_void_p),
+                ("wo", ctypes.c_void_p), ("wg", ctypes.c_void_p), ("wu", ctypes.c_void_p),
+                ("wd", ctypes.c_void_p), ("gamma_attn", ctypes.c_void_p),
+                ("gamma_mlp", ctypes.c_void_p), ("wtype", ctypes.c_int32)]
+
+
+class _Trace(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("k_new", ctypes.c_void_p), ("v_new", ctypes.c_void_p),
+                ("attn", ctypes.c_void_p), ("h", ctypes.c_void_p), ("act", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        L = _lib
+        L.orc_decode_layer.restype = ctypes.c_int
+        L.orc_prefill_layer.restype = ctypes.c_int
+        L.orc_mlp_sharded.restype = ctypes.c_int
+        L.orc_attn_sharded.restype = ctypes.c_int
+        L.orc_plan_maps.restype = ctypes.c_int
+        L.orc_kv_bytes_per_shard.restype = ctypes.c_longlong
+        L.orc_kv_bytes_per_shard.argtypes = [ctypes.c_longlong] * 7
+        L.orc_layer_params_per_shard.restype = ctypes.c_longlong
+        L.orc_reductions_per_pass.restype = ctypes.c_longlong
+        L.orc_reductions_per_pass.argtypes = [ctypes.c_longlong]
+        L.orc_silu.restype = ctypes.c_double
+        L.orc_silu.argtypes = [ctypes.c_double]
+        L.orc_get_threads.restype = ctypes.c_int
+        L.orc_set_threads.argtypes = [ctypes.c_int]
+    return _lib
+
+
+def set_threads(n: int) -> None:
+    lib().orc_set_threads(int(n))
+
+
+def get_threads() -> int:
+    return int(lib().orc_get_threads())
+
+
+@dataclass
+class Dims:
+    hidden: int
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    ffn: int
+    eps: float = 1e-5
+    flags: int = NORM | RESIDUAL
+
+    def c(self) -> _Dims:
+        return _Dims(self.hidden, self.n_q_heads, self.n_kv_heads, self.head_dim, self.ffn,
+                     float(self.eps), int(self.flags))
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _weights_struct(w: dict):
+    """w: numpy arrays in nn.Linear orientation: wq, wk, wv, wo, wg, wu, wd as
+    uint16 (raw bf16 bits) or float32; optional gamma_attn, gamma_mlp float32."""
+    keep = {}
+    wtype = None
+    for k in ("wq", "wk", "wv", "wo", "wg", "wu", "wd"):
+        a = w.get(k)
+        if a is None:
+            keep[k] = None
+            continue
+        a = np.ascontiguousarray(a)
+        t = 0 if a.dtype == np.uint16 else 1
+        if a.dtype not in (np.uint16, np.float32):
+            raise TypeError(f"{k}: weights must be uint16 (bf16 bits) or float32, got {a.dtype}")
+        if wtype is None:
+            wtype = t
+        elif wtype != t:
+            raise TypeError("all weights must share one dtype")
+        keep[k] = a
+    for k in ("gamma_attn", "gamma_mlp"):
+        a = w.get(k)
+        keep[k] = None if a is None else np.ascontiguousarray(a, dtype=np.float32)
+    s = _Weights(*[_p(keep[k]) for k in ("wq", "wk", "wv", "wo", "wg", "wu", "wd",
+                                          "gamma_attn", "gamma_mlp")], wtype or 0)
+    return s, keep
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact widening of raw bf16 bit patterns to float64."""
+    u = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    return u.view(np.float32).astype(np.float64)
+
+
+def decode_layer(dims: Dims, w: dict, x: np.ndarray, kc: np.ndarray, vc: np.ndarray, S: int,
+                 trace: bool = False):
+    """Unsharded decode layer ("Tensor parallel scaling curves", "What tensor
+    parallelism actually splits", read unsharded).  x [B][H] float64; kc/vc
+    uint16 [B][n_kv][S_cap][d]; S cached tokens.  Returns y [B][H] (float64)
+    and, if trace, a dict of q, k_new, v_new, attn, h, act."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    B, H = x.shape
+    kc = np.ascontiguousarray(kc, dtype=np.uint16)
+    vc = np.ascontiguousarray(vc, dtype=np.uint16)
+    S_cap = kc.shape[2]
+    y = np.empty((B, H), np.float64)
+    ws, keep = _weights_struct(w)
+    tr = None
+    tr_arrays = {}
+    if trace:
+        nqd = dims.n_q_heads * dims.head_dim
+        nkd = dims.n_kv_heads * dims.head_dim
+        tr_arrays = {"q": np.empty((B, nqd)), "k_new": np.empty((B, nkd)),
+                     "v_new": np.empty((B, nkd)), "attn": np.empty((B, nqd)),
+                     "h": np.empty((B, H)), "act": np.empty((B, dims.ffn))}
+        tr = _Trace(*[_p(tr_arrays[k]) for k in ("q", "k_new", "v_new", "attn", "h", "act")])
+    rc = lib().orc_decode_layer(ctypes.byref(dims.c()), ctypes.byref(ws), ctypes.c_long(B), _p(x),
+                                _p(kc), _p(vc), ctypes.c_long(S_cap), ctypes.c_long(S), _p(y),
+                                ctypes.byref(tr) if tr is not None else None)
+    if rc != 0:
+        raise ValueError(f"orc_decode_layer failed ({rc})")
+    return (y, tr_arrays) if trace else y
+
+
+def prefill_layer(dims: Dims, w: dict, x: np.ndarray, trace: bool = False):
+    """Unsharded prefill layer over a chunk starting at position 0, causal
+    inside the chunk ("Tensor parallel scaling curves", "Prefill vs decode").
+    Returns y [T][H], k [T][n_kv*d], v [T][n_kv*d] (and a trace dict)."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    T, H = x.shape
+    nkd = dims.n_kv_heads * dims.head_dim
+    y = np.empty((T, H))
+    k = np.empty((T, nkd))
+    v = np.empty((T, nkd))
+    ws, keep = _weights_struct(w)
+    tr = None
+    tr_arrays = {}
+    if trace:
+        nqd = dims.n_q_heads * dims.head_dim
+        tr_arrays = {"q": np.empty((T, nqd)), "attn": np.empty((T, nqd)), "h": np.empty((T, H)),
+                     "act": np.empty((T, dims.ffn))}
+        tr = _Trace(_p(tr_arrays["q"]), None, None, _p(tr_arrays["attn"]), _p(tr_arrays["h"]),
+                    _p(tr_arrays["act"]))
+    rc = lib().orc_prefill_layer(ctypes.byref(dims.c()), ctypes.byref(ws), ctypes.c_long(T), _p(x),
+                                 _p(y), _p(k), _p(v), ctypes.byref(tr) if tr is not None else None)
+    if rc != 0:
+        raise ValueError(f"orc_prefill_layer failed ({rc})")
+    return (y, k, v, tr_arrays) if trace else (y, k, v)
+
+
+def mlp_sharded(dims: Dims, w: dict, t: int, x: np.ndarray, partials: bool = False):
+    """MLP pair sharded t ways, partials summed in ascending shard order
+    ("Tensor Parallelism Fundamentals", "Mechanics of Matrix Slicing")."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    B, H = x.shape
+    y = np.empty((B, H))
+    parts = np.empty((t, B, H)) if partials else None
+    ws, keep = _weights_struct(w)
+    rc = lib().orc_mlp_sharded(ctypes.byref(dims.c()), ctypes.byref(ws), ctypes.c_int32(t),
+                               ctypes.c_long(B), _p(x), _p(y), _p(parts))
+    if rc != 0:
+        raise ValueError(f"orc_mlp_sharded failed ({rc})")
+    return (y, parts) if partials else y
+
+
+def attn_sharded(dims: Dims, w: dict, t: int, x: np.ndarray, a: np.ndarray, kc, vc, S: int,
+                 partials: bool = False):
+    """Attention block sharded t ways by whole heads ("Tensor parallel scaling
+    curves", "What tensor parallelism actually splits"): h = x + sum_s
+    partial_s in ascending s (residual only if flagged)."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    a = np.ascontiguousarray(a, dtype=np.float64)
+    B, H = x.shape
+    kc = np.ascontiguousarray(kc, dtype=np.uint16)
+    vc = np.ascontiguousarray(vc, dtype=np.uint16)
+    h = np.empty((B, H))
+    parts = np.empty((t, B, H)) if partials else None
+    ws, keep = _weights_struct(w)
+    rc = lib().orc_attn_sharded(ctypes.byref(dims.c()), ctypes.byref(ws), ctypes.c_int32(t),
+                                ctypes.c_long(B), _p(x), _p(a), _p(kc), _p(vc),
+                                ctypes.c_long(kc.shape[2]), ctypes.c_long(S), _p(h), _p(parts))
+    if rc != 0:
+        raise ValueError(f"orc_attn_sharded failed ({rc})")
+    return (h, parts) if partials else h
+
+
+def plan_maps(dims: Dims, t: int):
+    """Shard maps from the ownership rule heads[rank*h_per_gpu:(rank+1)*h_per_gpu]
+    ("Tensor parallel scaling curves", "What tensor parallelism actually
+    splits").  Returns None when t is not admissible."""
+    q_shard = np.empty(dims.n_q_heads, np.int32)
+    q_local = np.empty(dims.n_q_heads, np.int32)
+    kv_shard = np.empty(dims.n_kv_heads, np.int32)
+    ffn_shard = np.empty(dims.ffn, np.int32)
+    rc = lib().orc_plan_maps(ctypes.byref(dims.c()), ctypes.c_int32(t), _p(q_shard), _p(q_local),
+                             _p(kv_shard), _p(ffn_shard))
+    if rc != 0:
+        return None
+    return {"q_shard": q_shard, "q_local": q_local, "kv_shard": kv_shard, "ffn_shard": ffn_shard}
+
+
+def kv_bytes_per_shard(layers, kv_heads, head_dim, seq, bytes_per_elem, batch, t) -> int:
+    """Per-GPU KV bytes ("Tensor Parallelism Fundamentals", "Memory Overhead and
+    Communication Bottlenecks")."""
+    return int(lib().orc_kv_bytes_per_shard(layers, kv_heads, head_dim, seq, bytes_per_elem, batch, t))
+
+
+def layer_params_per_shard(dims: Dims, t: int) -> int:
+    return int(lib().orc_layer_params_per_shard(ctypes.byref(dims.c()), ctypes.c_int32(t)))
+
+
+def reductions_per_pass(layers: int) -> int:
+    """2L sums per forward pass ("Tensor parallel scaling curves")."""
+    return int(lib().orc_reductions_per_pass(layers))
+
+
+def silu(z: float) -> float:
+    return float(lib().orc_silu(float(z)))
+
+
+def rmsnorm(x: np.ndarray, gamma, eps: float) -> np.ndarray:
+    """RMSNorm of one vector: x * gamma / sqrt(mean(x^2) + eps) (pre-norm reading
+    of the Llama-shaped layer the pages size; the pages do not name the norm)."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    out = np.empty_like(x)
+    g = None if gamma is None else np.ascontiguousarray(gamma, dtype=np.float32)
+    L = lib()
+    L.orc_rmsnorm.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_long, ctypes.c_double,
+                              ctypes.c_void_p]
+    L.orc_rmsnorm(_p(x), _p(g), x.size, float(eps), _p(out))
+    return out

@@ -1,0 +1,84 @@
+"""An independent float64 evaluation of the layer with numpy's library
+routines (matmul, exp), used only to cross-check the C oracle on small cases.
+It shares no code with the oracle or the CUDA path."""
+import numpy as np
+
+
+def _widen(a):
+    a = np.asarray(a)
+    if a.dtype == np.uint16:
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return a.astype(np.float64)
+
+
+def _norm(x, gamma, eps):
+    r = np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    g = 1.0 if gamma is None else np.asarray(gamma, np.float64)
+    return x / r * g
+
+
+def _softmax(z):
+    z = z - z.max(axis=-1, keepdims=True)
+    e = np.exp(z)
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+def decode_layer(H, nq, nkv, d, F, eps, norm, residual, w, x, kc, vc, S):
+    W = {k: _widen(w[k]) for k in ("wq", "wk", "wv", "wo", "wg", "wu", "wd")}
+    x = np.asarray(x, np.float64)
+    B = x.shape[0]
+    g = nq // nkv
+    a = _norm(x, w.get("gamma_attn"), eps) if norm else x
+    q = a @ W["wq"].T
+    k = a @ W["wk"].T
+    v = a @ W["wv"].T
+    Kc = _widen(kc)[:, :, :S, :]
+    Vc = _widen(vc)[:, :, :S, :]
+    o = np.zeros((B, nq * d))
+    for b in range(B):
+        for h in range(nq):
+            j = h // g
+            keys = np.concatenate([Kc[b, j], k[b, j * d:(j + 1) * d][None]], axis=0)
+            vals = np.concatenate([Vc[b, j], v[b, j * d:(j + 1) * d][None]], axis=0)
+            p = _softmax(keys @ q[b, h * d:(h + 1) * d] / np.sqrt(d))
+            o[b, h * d:(h + 1) * d] = p @ vals
+    hh = o @ W["wo"].T
+    if residual:
+        hh = x + hh
+    m = _norm(hh, w.get("gamma_mlp"), eps) if norm else hh
+    gg = m @ W["wg"].T
+    uu = m @ W["wu"].T
+    act = gg / (1.0 + np.exp(-gg)) * uu
+    y = act @ W["wd"].T
+    if residual:
+        y = hh + y
+    return y, {"q": q, "k_new": k, "v_new": v, "attn": o, "h": hh, "act": act}
+
+
+def prefill_layer(H, nq, nkv, d, F, eps, norm, residual, w, x):
+    W = {k: _widen(w[k]) for k in ("wq", "wk", "wv", "wo", "wg", "wu", "wd")}
+    x = np.asarray(x, np.float64)
+    T = x.shape[0]
+    g = nq // nkv
+    a = _norm(x, w.get("gamma_attn"), eps) if norm else x
+    q = a @ W["wq"].T
+    k = a @ W["wk"].T
+    v = a @ W["wv"].T
+    o = np.zeros((T, nq * d))
+    mask = np.tril(np.ones((T, T), bool))
+    for h in range(nq):
+        j = h // g
+        s = q[:, h * d:(h + 1) * d] @ k[:, j * d:(j + 1) * d].T / np.sqrt(d)
+        s = np.where(mask, s, -np.inf)
+        o[:, h * d:(h + 1) * d] = _softmax(s) @ v[:, j * d:(j + 1) * d]
+    hh = o @ W["wo"].T
+    if residual:
+        hh = x + hh
+    m = _norm(hh, w.get("gamma_mlp"), eps) if norm else hh
+    gg = m @ W["wg"].T
+    uu = m @ W["wu"].T
+    act = gg / (1.0 + np.exp(-gg)) * uu
+    y = act @ W["wd"].T
+    if residual:
+        y = hh + y
+    return y, k, v

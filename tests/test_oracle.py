@@ -1,0 +1,445 @@
+"""Pins for the oracle: what the pages and the mathematics fix, independent of
+the oracle's own code.  CPU only.
+
+Each test is chosen so that a plausible mistake in the oracle (a dropped term,
+a wrong sign, a transposed operand, a wrong head mapping, a wrong softmax
+scale, a wrong summation) fails at least one of them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from tests import np_reference
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def f32(a):
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def rng(seed=0):
+    return np.random.default_rng(seed)
+
+
+def rand_bf16_bits(r, shape, std):
+    """Random values rounded to bf16 (truncation of float32 bits is fine for a
+    test input: the result is some bf16 value), returned as raw bits."""
+    a = (r.standard_normal(shape) * std).astype(np.float32)
+    return (a.view(np.uint32) >> 16).astype(np.uint16)
+
+
+def small_layer(r, H=32, nq=4, nkv=2, d=8, F=48, std=0.2, bf16=True):
+    shapes = {"wq": (nq * d, H), "wk": (nkv * d, H), "wv": (nkv * d, H), "wo": (H, nq * d),
+              "wg": (F, H), "wu": (F, H), "wd": (H, F)}
+    if bf16:
+        w = {k: rand_bf16_bits(r, s, std) for k, s in shapes.items()}
+    else:
+        w = {k: f32(r.standard_normal(s) * std) for k, s in shapes.items()}
+    w["gamma_attn"] = f32(1 + 0.1 * r.standard_normal(H))
+    w["gamma_mlp"] = f32(1 + 0.1 * r.standard_normal(H))
+    return w
+
+
+# --------------------------------------------------------------------------
+# The pages' worked numbers
+# --------------------------------------------------------------------------
+
+def test_kv_formula_worked_example():
+    g = golden("kv_footprint.json")
+    per_seq = oracle.kv_bytes_per_shard(g["layers"], g["kv_heads"], g["head_dim"], g["seq"],
+                                        g["bytes_per_elem"], 1, 1)
+    assert per_seq == g["bytes_per_sequence"]
+    assert per_seq // g["bytes_per_elem"] == g["elements_per_sequence"]
+    assert oracle.kv_bytes_per_shard(g["layers"], g["kv_heads"], g["head_dim"], g["seq"],
+                                     g["bytes_per_elem"], g["batch"], 1) == g["bytes_batch"]
+    assert oracle.kv_bytes_per_shard(g["layers"], g["kv_heads"], g["head_dim"], g["seq"],
+                                     g["bytes_per_elem"], g["batch"], g["t"]) == g["bytes_per_gpu"]
+    # the page's rounded figures are binary gigabytes
+    assert g["bytes_per_sequence"] == 2.5 * 2**30
+    assert g["bytes_batch"] == 40 * 2**30
+    assert g["bytes_per_gpu"] == 10 * 2**30
+
+
+def test_reductions_per_pass():
+    g = golden("reductions.json")
+    assert oracle.reductions_per_pass(g["layers"]) == g["per_pass"]
+    assert oracle.reductions_per_pass(1) == g["per_layer"]
+    assert 8192 * 2 == g["message_bytes_per_token"]
+
+
+def test_weight_footprint_70b():
+    g = golden("weights_footprint.json")
+    d = oracle.Dims(8192, 64, 8, 128, 28672)
+    per_shard = oracle.layer_params_per_shard(d, g["t"])
+    full = oracle.layer_params_per_shard(d, 1)
+    assert full == 4 * per_shard  # weights divide exactly by t
+    total_gb = 80 * full * 2 / 1e9
+    per_gpu_gb = 80 * per_shard * 2 / 1e9
+    assert abs(total_gb - g["approx_total_GB"]) / g["approx_total_GB"] < g["rel_tolerance"]
+    assert abs(per_gpu_gb - g["approx_per_gpu_GB_t4"]) / g["approx_per_gpu_GB_t4"] < g["rel_tolerance"]
+    # hand count of the Llama-3.1-70B-shaped layer: q 8192x8192, k/v 1024x8192,
+    # o 8192x8192, gate/up 28672x8192, down 8192x28672
+    assert full == 8192 * 8192 * 2 + 1024 * 8192 * 2 + 28672 * 8192 * 3
+
+
+# --------------------------------------------------------------------------
+# Shard maps: the ownership rule and its consequences
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dims", [(8192, 64, 8, 128, 28672), (4096, 32, 32, 128, 11008),
+                                  (256, 4, 2, 64, 688)])
+@pytest.mark.parametrize("t", [1, 2, 4, 8])
+def test_plan_maps_invariants(dims, t):
+    d = oracle.Dims(*dims)
+    m = oracle.plan_maps(d, t)
+    H, nq, nkv, hd, F = dims
+    if nq % t or nkv % t or F % t:
+        assert m is None
+        return
+    g = nq // nkv
+    # every shard owns the same number of whole heads, contiguously
+    for s in range(t):
+        owned = np.nonzero(m["q_shard"] == s)[0]
+        assert len(owned) == nq // t
+        assert np.all(np.diff(owned) == 1)
+        assert list(m["q_local"][owned]) == list(range(nq // t))
+    # local attention needs no communication: the kv head a query head reads
+    # lives on the same shard
+    for h in range(nq):
+        assert m["kv_shard"][h // g] == m["q_shard"][h]
+    assert np.all(np.bincount(m["ffn_shard"], minlength=t) == F // t)
+    assert np.all(np.diff(m["ffn_shard"]) >= 0)
+
+
+@pytest.mark.parametrize("t", [0, 3, 5, 16, -1])
+def test_plan_maps_rejects_bad_degree(t):
+    assert oracle.plan_maps(oracle.Dims(256, 8, 8, 32, 64), t) is None
+
+
+def test_plan_maps_rejects_indivisible():
+    assert oracle.plan_maps(oracle.Dims(256, 4, 2, 64, 688), 4) is None  # 2 kv heads, t = 4
+    assert oracle.plan_maps(oracle.Dims(256, 8, 8, 32, 100), 8) is None  # F = 100, t = 8
+
+
+# --------------------------------------------------------------------------
+# Closed forms
+# --------------------------------------------------------------------------
+
+def test_silu_known_values():
+    assert oracle.silu(0.0) == 0.0
+    assert oracle.silu(1.0) == pytest.approx(0.7310585786300049, abs=1e-16)
+    assert oracle.silu(-1.0) == pytest.approx(-0.2689414213699951, abs=1e-16)
+    assert oracle.silu(50.0) == 50.0
+    assert abs(oracle.silu(-50.0)) < 1e-20
+
+
+@pytest.mark.parametrize("c", [0.5, 3.0, -2.0])
+def test_rmsnorm_constant_vector(c):
+    n, eps = 16, 1e-5
+    gamma = f32(np.linspace(0.5, 1.5, n))
+    out = oracle.rmsnorm(np.full(n, c), gamma, eps)
+    expect = gamma.astype(np.float64) * c / math.sqrt(c * c + eps)
+    np.testing.assert_allclose(out, expect, rtol=1e-15, atol=0)
+
+
+def _eye_bits(n, m=None):
+    m = n if m is None else m
+    e = np.zeros((n, m), np.float32)
+    e[np.arange(min(n, m)), np.arange(min(n, m))] = 1
+    return (e.view(np.uint32) >> 16).astype(np.uint16)
+
+
+def _bits(a):
+    return (f32(a).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def test_single_key_returns_new_value():
+    """S = 0: one key, softmax weight exactly 1, so attention output = v_new."""
+    r = rng(1)
+    H, nq, nkv, d, F = 32, 4, 2, 8, 48
+    w = small_layer(r, H, nq, nkv, d, F)
+    dims = oracle.Dims(H, nq, nkv, d, F)
+    x = r.standard_normal((3, H))
+    kc = np.zeros((3, nkv, 4, d), np.uint16)
+    y, tr = oracle.decode_layer(dims, w, x, kc, kc, 0, trace=True)
+    g = nq // nkv
+    for h in range(nq):
+        j = h // g
+        np.testing.assert_array_equal(tr["attn"][:, h * d:(h + 1) * d], tr["v_new"][:, j * d:(j + 1) * d])
+
+
+def test_uniform_logits_give_mean_and_gqa_mapping():
+    """Wq = 0 makes every logit 0, so each head averages its kv head's S+1
+    values.  Constant, head-specific cache values pin the GQA map h -> h//g."""
+    H, nq, nkv, d, F, S = 16, 8, 2, 4, 8, 5
+    r = rng(2)
+    w = small_layer(r, H, nq, nkv, d, F)
+    w["wq"] = np.zeros_like(w["wq"])
+    w["wv"] = np.zeros_like(w["wv"])           # new value = 0
+    dims = oracle.Dims(H, nq, nkv, d, F, flags=0)
+    B = 2
+    vc = np.zeros((B, nkv, S + 3, d), np.float32)
+    consts = {0: 1.5, 1: -3.0}
+    for j, c in consts.items():
+        vc[:, j, :S, :] = c
+    kc = _bits(r.standard_normal((B, nkv, S + 3, d)))
+    x = r.standard_normal((B, H))
+    _, tr = oracle.decode_layer(dims, w, x, kc, _bits(vc), S, trace=True)
+    g = nq // nkv
+    for h in range(nq):
+        np.testing.assert_allclose(tr["attn"][:, h * d:(h + 1) * d], consts[h // g] * S / (S + 1),
+                                   rtol=1e-14)
+
+
+def test_softmax_scale_is_inverse_sqrt_head_dim():
+    """Two keys: logits (alpha*beta/sqrt(d), 0); the weight of key 0 is the
+    logistic of alpha*beta/sqrt(d)."""
+    d = 16
+    H, nq, nkv, F = d, 1, 1, 8
+    w = {"wq": _eye_bits(d), "wk": np.zeros((d, d), np.uint16), "wv": np.zeros((d, d), np.uint16),
+         "wo": _eye_bits(d), "wg": np.zeros((F, H), np.uint16), "wu": np.zeros((F, H), np.uint16),
+         "wd": np.zeros((H, F), np.uint16)}
+    dims = oracle.Dims(H, nq, nkv, d, F, flags=0)
+    alpha, beta = 2.0, 3.0
+    x = np.zeros((1, H))
+    x[0, 0] = beta
+    kc = np.zeros((1, 1, 2, d), np.float32)
+    vc = np.zeros((1, 1, 2, d), np.float32)
+    kc[0, 0, 0, 0] = alpha
+    vc[0, 0, 0, 1] = 1.0
+    _, tr = oracle.decode_layer(dims, w, x, _bits(kc), _bits(vc), 1, trace=True)
+    p0 = 1.0 / (1.0 + math.exp(-alpha * beta / math.sqrt(d)))
+    assert tr["attn"][0, 1] == pytest.approx(p0, rel=1e-15)
+    # Wo = I and no residual: h is the attention output itself
+    np.testing.assert_array_equal(tr["h"], tr["attn"])
+
+
+def test_projection_orientation_with_shift_permutations():
+    """nn.Linear orientation: y = W x with W[out][in].  With cyclic-shift
+    matrices a transposed product would shift the other way."""
+    n = 8
+    H = F = n
+    d, nq, nkv = n, 1, 1
+    P = np.zeros((n, n), np.float32)
+    P[np.arange(n), (np.arange(n) + 1) % n] = 1      # (P x)[i] = x[i+1]
+    Pb = _bits(P)
+    big = _bits(np.eye(n) * 64.0)                     # gate = 64 x: silu(64 x) = 64 x for x >= 1
+    w = {"wq": np.zeros((n, n), np.uint16), "wk": np.zeros((n, n), np.uint16), "wv": Pb,
+         "wo": Pb, "wg": big, "wu": _eye_bits(n), "wd": Pb}
+    dims = oracle.Dims(H, nq, nkv, d, F, flags=oracle.RESIDUAL)
+    x = np.arange(1, n + 1, dtype=np.float64)[None] * 1.0
+    y, tr = oracle.decode_layer(dims, w, x, np.zeros((1, 1, 1, d), np.uint16),
+                                np.zeros((1, 1, 1, d), np.uint16), 0, trace=True)
+    sh = lambda v, k: np.roll(v, -k, axis=-1)
+    np.testing.assert_array_equal(tr["v_new"], sh(x, 1))          # Wv x
+    np.testing.assert_array_equal(tr["attn"], sh(x, 1))           # single key
+    np.testing.assert_array_equal(tr["h"], x + sh(x, 2))          # x + Wo attn
+    m = tr["h"]
+    act = (64.0 * m) * m                                           # silu(64 m) * m
+    np.testing.assert_allclose(y, m + sh(act, 1), rtol=1e-15)
+
+
+def test_swiglu_identity_weights():
+    """Wg = Wu = Wd = I, Wo = 0, no norm: h = x and y = x + silu(x) * x."""
+    n = 16
+    w = {"wq": np.zeros((n, n), np.uint16), "wk": np.zeros((n, n), np.uint16),
+         "wv": np.zeros((n, n), np.uint16), "wo": np.zeros((n, n), np.uint16),
+         "wg": _eye_bits(n), "wu": _eye_bits(n), "wd": _eye_bits(n)}
+    dims = oracle.Dims(n, 1, 1, n, n, flags=oracle.RESIDUAL)
+    x = np.linspace(-4, 4, n)[None]
+    y, tr = oracle.decode_layer(dims, w, x, np.zeros((1, 1, 1, n), np.uint16),
+                                np.zeros((1, 1, 1, n), np.uint16), 0, trace=True)
+    np.testing.assert_array_equal(tr["h"], x)
+    np.testing.assert_allclose(tr["act"][0], x[0] * x[0] / (1 + np.exp(-x[0])), rtol=1e-15)
+    np.testing.assert_allclose(y[0], x[0] + x[0] * x[0] / (1 + np.exp(-x[0])), rtol=1e-15)
+
+
+def test_residuals_with_zero_branches():
+    r = rng(3)
+    H, nq, nkv, d, F = 16, 2, 1, 8, 24
+    w = small_layer(r, H, nq, nkv, d, F)
+    w["wo"] = np.zeros_like(w["wo"])
+    w["wg"] = np.zeros_like(w["wg"])
+    x = r.standard_normal((2, H))
+    dims = oracle.Dims(H, nq, nkv, d, F)
+    kc = rand_bf16_bits(r, (2, nkv, 5, d), 1.0)
+    y, tr = oracle.decode_layer(dims, w, x, kc, kc, 3, trace=True)
+    np.testing.assert_array_equal(tr["h"], x)
+    np.testing.assert_array_equal(y, x)
+
+
+# --------------------------------------------------------------------------
+# Exact row-split / column-split identities (integer data, every sum exact)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("t", [1, 2, 4, 8])
+def test_mlp_row_split_identity_exact(t):
+    """Sum of the t row-split partials equals the unsharded MLP bit for bit.
+    Gate inputs are >= 40 so silu(g) == g exactly in float64 and every value
+    is an integer."""
+    r = rng(10 + t)
+    H, F, B = 8, 16, 3
+    x = r.integers(5, 9, (B, H)).astype(np.float64)
+    wg = f32(r.integers(1, 9, (F, H)))
+    wu = f32(r.integers(-8, 9, (F, H)))
+    wd = f32(r.integers(-8, 9, (H, F)))
+    z = np.zeros((4, H), np.float32)
+    w = {"wq": z, "wk": z, "wv": z, "wo": f32(np.zeros((H, 4))), "wg": wg, "wu": wu, "wd": wd}
+    dims = oracle.Dims(H, 1, 1, 4, F, flags=oracle.RESIDUAL)
+    kc = np.zeros((B, 1, 1, 4), np.uint16)
+    # wo = 0 makes h = x, so the layer is x + MLP(x); every value is an integer
+    y_full = oracle.decode_layer(dims, w, x, kc, kc, 0) - x
+    y_sh, parts = oracle.mlp_sharded(dims, w, t, x, partials=True)
+    np.testing.assert_array_equal(y_sh, y_full)
+    np.testing.assert_array_equal(parts.sum(axis=0), y_full)
+    # and against exact integer arithmetic
+    g = x @ wg.T.astype(np.float64)
+    assert np.all(g >= 40)
+    exact = (g * (x @ wu.T.astype(np.float64))) @ wd.T.astype(np.float64)
+    np.testing.assert_array_equal(y_full, exact)
+
+
+@pytest.mark.parametrize("t", [1, 2, 4, 8])
+def test_attention_head_split_identity_exact(t):
+    """S = 0 and integer data: attention output = v exactly; the head-wise
+    column split plus row-split O projection sums to the unsharded h."""
+    r = rng(20 + t)
+    H, nq, nkv, d, B = 16, 8, 8, 4, 2
+    w = {"wq": f32(r.integers(-8, 9, (nq * d, H))), "wk": f32(r.integers(-8, 9, (nkv * d, H))),
+         "wv": f32(r.integers(-8, 9, (nkv * d, H))), "wo": f32(r.integers(-8, 9, (H, nq * d))),
+         "wg": f32(np.zeros((4, H))), "wu": f32(np.zeros((4, H))), "wd": f32(np.zeros((H, 4)))}
+    dims = oracle.Dims(H, nq, nkv, d, 4, flags=oracle.RESIDUAL)
+    x = r.integers(-8, 9, (B, H)).astype(np.float64)
+    kc = np.zeros((B, nkv, 2, d), np.uint16)
+    _, tr = oracle.decode_layer(dims, w, x, kc, kc, 0, trace=True)
+    h_sh, parts = oracle.attn_sharded(dims, w, t, x, x, kc, kc, 0, partials=True)
+    np.testing.assert_array_equal(h_sh, tr["h"])
+    exact = x + (x @ w["wv"].T.astype(np.float64)) @ w["wo"].T.astype(np.float64)
+    np.testing.assert_array_equal(tr["h"], exact)
+
+
+@pytest.mark.parametrize("t", [1, 2, 4])
+def test_attention_head_split_identity_gqa(t):
+    """GQA with a real cache: sharded and unsharded agree to rounding."""
+    r = rng(30 + t)
+    H, nq, nkv, d, F, B, S = 32, 8, 4, 8, 16, 2, 7
+    w = small_layer(r, H, nq, nkv, d, F)
+    dims = oracle.Dims(H, nq, nkv, d, F, flags=oracle.NORM | oracle.RESIDUAL)
+    x = r.standard_normal((B, H))
+    kc = rand_bf16_bits(r, (B, nkv, S + 2, d), 1.0)
+    vc = rand_bf16_bits(r, (B, nkv, S + 2, d), 1.0)
+    _, tr = oracle.decode_layer(dims, w, x, kc, vc, S, trace=True)
+    a = np.stack([oracle.rmsnorm(x[b], w["gamma_attn"], dims.eps) for b in range(B)])
+    h_sh = oracle.attn_sharded(dims, w, t, x, a, kc, vc, S)
+    np.testing.assert_allclose(h_sh, tr["h"], rtol=1e-12, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# Independent evaluation with numpy's library routines
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("case", [
+    dict(H=256, nq=4, nkv=2, d=64, F=688, B=1, S=0, flags=0),          # MLP-shaped tiny case
+    dict(H=64, nq=4, nkv=4, d=16, F=96, B=3, S=9, flags=3),             # MHA, g = 1
+    dict(H=64, nq=8, nkv=2, d=16, F=80, B=2, S=33, flags=3),            # GQA, g = 4
+    dict(H=32, nq=4, nkv=1, d=8, F=40, B=2, S=5, flags=1),              # norm only
+])
+def test_decode_matches_numpy(case):
+    r = rng(40)
+    H, nq, nkv, d, F, B, S = (case[k] for k in ("H", "nq", "nkv", "d", "F", "B", "S"))
+    w = small_layer(r, H, nq, nkv, d, F, std=0.1)
+    dims = oracle.Dims(H, nq, nkv, d, F, flags=case["flags"])
+    x = r.standard_normal((B, H))
+    kc = rand_bf16_bits(r, (B, nkv, S + 4, d), 1.0)
+    vc = rand_bf16_bits(r, (B, nkv, S + 4, d), 1.0)
+    y, tr = oracle.decode_layer(dims, w, x, kc, vc, S, trace=True)
+    y_np, tr_np = np_reference.decode_layer(H, nq, nkv, d, F, dims.eps, bool(dims.flags & 1),
+                                            bool(dims.flags & 2), w, x, kc, vc, S)
+    scale = np.abs(y_np).max()
+    np.testing.assert_allclose(y, y_np, rtol=1e-12, atol=1e-12 * scale)
+    for k in tr:
+        s = max(np.abs(tr_np[k]).max(), 1e-300)
+        np.testing.assert_allclose(tr[k], tr_np[k], rtol=1e-12, atol=1e-12 * s)
+
+
+def test_decode_fp32_weights_match_numpy():
+    r = rng(41)
+    H, nq, nkv, d, F, B, S = 64, 8, 2, 16, 80, 2, 12
+    w = small_layer(r, H, nq, nkv, d, F, std=0.1, bf16=False)
+    dims = oracle.Dims(H, nq, nkv, d, F)
+    x = r.standard_normal((B, H))
+    kc = rand_bf16_bits(r, (B, nkv, S + 1, d), 1.0)
+    vc = rand_bf16_bits(r, (B, nkv, S + 1, d), 1.0)
+    y = oracle.decode_layer(dims, w, x, kc, vc, S)
+    y_np, _ = np_reference.decode_layer(H, nq, nkv, d, F, dims.eps, True, True, w, x, kc, vc, S)
+    np.testing.assert_allclose(y, y_np, rtol=1e-12, atol=1e-12 * np.abs(y_np).max())
+
+
+def test_prefill_matches_numpy():
+    r = rng(42)
+    H, nq, nkv, d, F, T = 64, 8, 2, 16, 80, 13
+    w = small_layer(r, H, nq, nkv, d, F, std=0.1)
+    dims = oracle.Dims(H, nq, nkv, d, F)
+    x = r.standard_normal((T, H))
+    y, k, v = oracle.prefill_layer(dims, w, x)
+    y_np, k_np, v_np = np_reference.prefill_layer(H, nq, nkv, d, F, dims.eps, True, True, w, x)
+    np.testing.assert_allclose(y, y_np, rtol=1e-12, atol=1e-12 * np.abs(y_np).max())
+    np.testing.assert_allclose(k, k_np, rtol=1e-12, atol=1e-12 * np.abs(k_np).max())
+
+
+def test_prefill_is_causal_and_agrees_with_decode():
+    """Token i of a prefill chunk sees only tokens 0..i: changing later tokens
+    leaves earlier outputs unchanged, and with bf16-exact keys/values the last
+    token equals one decode step over a cache holding the earlier tokens."""
+    r = rng(43)
+    H, nq, nkv, d, F, T = 16, 4, 2, 8, 12, 6
+    w = {k: f32(r.integers(-2, 3, s)) for k, s in
+         {"wq": (nq * d, H), "wk": (nkv * d, H), "wv": (nkv * d, H), "wo": (H, nq * d),
+          "wg": (F, H), "wu": (F, H), "wd": (H, F)}.items()}
+    w["wq"] = f32(w["wq"] * 0.125)
+    dims = oracle.Dims(H, nq, nkv, d, F, flags=oracle.RESIDUAL)
+    x = r.integers(-2, 3, (T, H)).astype(np.float64)
+    y, k, v = oracle.prefill_layer(dims, w, x)
+    x2 = x.copy()
+    x2[-1] += 1.0
+    y2, _, _ = oracle.prefill_layer(dims, w, x2)
+    np.testing.assert_array_equal(y[:-1], y2[:-1])
+    assert not np.array_equal(y[-1], y2[-1])
+    # keys and values are small integers: exact in bf16
+    S = T - 1
+    kc = np.zeros((1, nkv, T, d), np.float32)
+    vc = np.zeros((1, nkv, T, d), np.float32)
+    for j in range(nkv):
+        kc[0, j, :S] = k[:S, j * d:(j + 1) * d]
+        vc[0, j, :S] = v[:S, j * d:(j + 1) * d]
+    assert np.array_equal(_bits(kc).astype(np.uint32) << 16, kc.view(np.uint32))
+    yd = oracle.decode_layer(dims, w, x[-1:], _bits(kc), _bits(vc), S)
+    np.testing.assert_allclose(yd[0], y[-1], rtol=1e-13, atol=1e-13)
+    # token 0 of the chunk is a decode step over an empty cache
+    y0 = oracle.decode_layer(dims, w, x[:1], np.zeros((1, nkv, 1, d), np.uint16),
+                             np.zeros((1, nkv, 1, d), np.uint16), 0)
+    np.testing.assert_allclose(y0[0], y[0], rtol=1e-14, atol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# Planted mistakes must be caught (a check of the checks, done on the CPU)
+# --------------------------------------------------------------------------
+
+def test_planted_transposed_wo_is_caught():
+    """A transposed O projection in a reference would fail the orientation
+    pin: emulate it with numpy and confirm the pinned values differ."""
+    n = 8
+    P = np.zeros((n, n))
+    P[np.arange(n), (np.arange(n) + 1) % n] = 1
+    o = np.arange(1, n + 1, dtype=np.float64)
+    assert not np.array_equal(P @ o, P.T @ o)

@@ -1,0 +1,381 @@
+#!/usr/bin/env python
+"""Decode throughput of the 70B-shaped 80-layer stack in the t = 8 shard
+layout on one GPU (batch 4, KV length 4096), through the C-ABI library.
+
+One step = one decode token for each of the B sequences through all 80
+layers: per layer the column-parallel QKV, the owned-head attention, the
+row-parallel O projection with its fused shard sum, the column-parallel
+gate/up with SwiGLU and the row-parallel down projection with its fused
+shard sum (160 reduction points per step).  Weights (137 GB) and KV caches
+(5.4 GB) are seeded synthetic tensors resident in HBM; every step reads all
+of them, so the working set is far larger than L2 and no flush is needed.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (under torchrun) every rank runs an independent replica of the
+stack on its own GPU (the path has no cross-GPU exchange in this build);
+value = all tokens / the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode tokens/s (70B-shaped layer stack, 1 GPU); achieved HBM GB/s vs peak"
+H, NQ, NKV, D, F, L = 8192, 64, 8, 128, 28672, 80
+T_SHARDS, BATCH, KV_LEN = 8, 4, 4096
+WORKLOAD = "70B-shaped 80-layer decode stack, t=8 shard layout"
+
+
+def config_dict():
+    return {"workload": WORKLOAD, "hidden": H, "n_q_heads": NQ, "n_kv_heads": NKV, "head_dim": D, "ffn": F,
+            "layers": L, "t": T_SHARDS, "batch": BATCH, "kv_len": KV_LEN, "reduce": "fused",
+            "reductions_per_step": 2 * L,
+            "l2": "no flush: every step streams 142 GB of weights and KV, far above the 126 MB L2"}
+
+
+def algorithmic_bytes_per_step():
+    w = (NQ + 2 * NKV) * D * H + H * NQ * D + 2 * F * H + H * F  # params per layer
+    per_layer = (w * 2                                   # every weight once (bf16)
+                 + BATCH * 2 * NKV * KV_LEN * D * 2      # K and V cache read
+                 + BATCH * 2 * NKV * D * 2               # new K/V written and read back
+                 + BATCH * H * 2 * 2)                    # x in, y out
+    return L * per_layer
+
+
+def gate_up_bytes_per_launch():
+    return 2 * F * H * 2 + BATCH * H * 4 + BATCH * F * 2  # weights + h (fp32) + act (bf16)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "megatron_tensor_transformer_plan_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h", ".cpp")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode())
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """dram bytes per gate/up launch from the committed ncu summary, valid only
+    while the kernel sources are unchanged since the capture."""
+    p = os.path.join(ROOT, "profiles", "gemv_gate_up_stack.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        j = json.load(f)
+    if j.get("source_hash") != kernel_source_hash():
+        return None
+    return j.get("dram_bytes_per_launch")
+
+
+class Clocks:
+    """nvidia-smi sampled every 200 ms during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.gpu_index)],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_init():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def run_reference(args, ws, rank):
+    """The oracle (plain fp64 C, as it stands) on the host cores, on a bounded
+    sample of the same workload: one decoder layer of the stack per step,
+    scaled to the 80-layer stack's tokens/s."""
+    if rank != 0:
+        return 0
+    import numpy as np
+    import torch
+    import oracle
+    from megatron_tensor_transformer_plan_b200 import synth
+    threads = os.cpu_count() or 1
+    oracle.set_threads(threads)
+    dims = oracle.Dims(H, NQ, NKV, D, F)
+    w = synth.layer_weights(H, NQ, NKV, D, F, seed=0, layer=0, dtype=torch.bfloat16, device="cpu")
+    wb = {k: synth.bits(v) for k, v in w.items()}
+    x = synth.activations(BATCH, H, seed=0, dtype=torch.bfloat16).float().numpy().astype(np.float64)
+    kl, vl = synth.kv_cache((BATCH, NKV, KV_LEN + 1, D), seed=0)
+    kb, vb = synth.bits(kl), synth.bits(vl)
+    for _ in range(args.warmup):
+        oracle.decode_layer(dims, wb, x, kb, vb, KV_LEN)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.decode_layer(dims, wb, x, kb, vb, KV_LEN)
+        times.append(time.perf_counter() - t0)
+    t_layer = sum(times) / len(times)
+    step_s = t_layer * L
+    value = BATCH / step_s
+    cpu = {"value": value, "unit": "tokens/s", "cores": oracle.get_threads(), "kind": "oracle",
+           "sample": f"one decoder layer (B={BATCH}, KV {KV_LEN}) per step, fp64, x{L} layers extrapolated"}
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config_dict(),
+            "cpu_baseline": cpu,
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def build_stack(plan, tpl, synth, torch, dev, seed=0):
+    packed, kvs, keep = [], [], []
+    nkv_s = NKV // T_SHARDS
+    for l in range(L):
+        w = synth.layer_weights(H, NQ, NKV, D, F, seed=seed, layer=l, dtype=torch.bfloat16, device=dev)
+        packed.append(plan.pack_layer(w))
+        del w
+        k, v = synth.kv_cache((T_SHARDS, BATCH, nkv_s, KV_LEN + 1, D), seed=seed, layer=l, device=dev)
+        keep.append((k, v))
+        kvs.append(tpl.Plan.kv(k, v, BATCH, KV_LEN + 1))
+    torch.cuda.synchronize()
+    return packed, kvs, keep
+
+
+def run_ours(args, ws, rank, local):
+    import torch
+    from megatron_tensor_transformer_plan_b200 import build
+    build.build()
+    from megatron_tensor_transformer_plan_b200 import synth, tpl
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=dev)
+
+    dims = tpl.make_dims(H, NQ, NKV, D, F, L, 1e-5, tpl.TPL_NORM | tpl.TPL_RESIDUAL)
+    plan = tpl.Plan(dims, T_SHARDS)
+    packed, kvs, keep = build_stack(plan, tpl, synth, torch, dev)
+    x = synth.activations(BATCH, H, seed=0, dtype=torch.bfloat16, device=dev)
+    y = torch.empty_like(x)
+    wsb = plan.workspace(BATCH, KV_LEN, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    arr = (ctypes.c_void_p * L)(*[p.data_ptr() for p in packed])
+    kva = (tpl.tpl_kv * L)(*kvs)
+
+    def step(xin, yout):
+        tpl.check(tpl.tpl_decode_stack(plan.handle, arr, kva, xin.data_ptr(), BATCH, KV_LEN, yout.data_ptr(), None,
+                                       wsb.data_ptr(), wsb.numel(), tpl.TPL_REDUCE_FUSED, stream.cuda_stream),
+                  "tpl_decode_stack")
+
+    def barrier():
+        if ws > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    # ---- device-resident throughput ----
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step(x, y)
+    torch.cuda.synchronize()
+    assert plan.last_device_error() == tpl.TPL_OK
+    plan.reset_counters()
+    clocks = Clocks(local)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step(x, y)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    reductions = plan.reduction_count()
+    if ws > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    tokens_per_s = ws * BATCH / (ms / 1e3)
+
+    # ---- end to end: pinned host x in, y back to the host, every step ----
+    xh = x.cpu().pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    xd = torch.empty_like(x)
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            xd.copy_(xh, non_blocking=True)
+            step(xd, y)
+            yh.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    e2e_steps = max(3, args.steps // 4)
+    with torch.cuda.stream(stream):
+        for _ in range(e2e_steps):
+            xd.copy_(xh, non_blocking=True)
+            step(xd, y)
+            yh.copy_(y, non_blocking=True)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = f0.elapsed_time(f1) / e2e_steps
+    if ws > 1:
+        import torch.distributed as dist
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    # ---- the dominant kernel (gate/up) timed alone, one launch per layer ----
+    act = torch.empty((BATCH, F), dtype=torch.bfloat16, device=dev)
+    hbuf = torch.randn((BATCH, H), dtype=torch.float32, device=dev)
+    with torch.cuda.stream(stream):
+        for l in range(3):
+            plan.gate_up(packed[l], hbuf, act, wsb)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L)]
+    with torch.cuda.stream(stream):
+        for l in range(L):
+            evs[l][0].record(stream)
+            plan.gate_up(packed[l], hbuf, act, wsb)
+            evs[l][1].record(stream)
+    torch.cuda.synchronize()
+    gu_ms = sum(a.elapsed_time(b) for a, b in evs) / L
+    peak, peak_kind = load_peaks()
+    gu_gbs = gate_up_bytes_per_launch() / (gu_ms / 1e3) / 1e9
+    step_gbs = algorithmic_bytes_per_step() / (ms / 1e3) / 1e9
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,0.02) weights, N(0,1) x/KV)",
+                "config": dict(config_dict(), step_hbm_gbs=step_gbs, step_hbm_frac=step_gbs / peak,
+                               algorithmic_bytes_per_step=algorithmic_bytes_per_step(),
+                               reductions_counted=reductions // max(1, args.steps)),
+                "roofline": {"bound": "hbm", "kernel": "gemv_kernel<0> (gate/up + SwiGLU)", "achieved": gu_gbs,
+                             "peak": peak, "peak_kind": peak_kind + " (burst copy, kernel timed alone)",
+                             "unit": "GB/s", "frac": gu_gbs / peak, "traffic": recorded_traffic(),
+                             "algorithmic_bytes_per_launch": gate_up_bytes_per_launch(), "launch_ms": gu_ms},
+                "e2e": {"value": ws * BATCH / (e2e_ms / 1e3), "unit": "tokens/s",
+                        "h2d_bytes_per_step": x.numel() * 2, "d2h_bytes_per_step": y.numel() * 2},
+                "gpu_launches": 5 * L * args.steps,
+                "clocks": clk}
+        if ws == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline_sample()
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def cpu_baseline_sample():
+    """The oracle as it stands on the host cores: one layer of the stack
+    (batch 4, KV 4096), about 10-30 s of CPU work, scaled to the stack."""
+    import numpy as np
+    import torch
+    import oracle
+    from megatron_tensor_transformer_plan_b200 import synth
+    threads = os.cpu_count() or 1
+    oracle.set_threads(threads)
+    dims = oracle.Dims(H, NQ, NKV, D, F)
+    w = synth.layer_weights(H, NQ, NKV, D, F, seed=0, layer=0, dtype=torch.bfloat16, device="cpu")
+    wb = {k: synth.bits(v) for k, v in w.items()}
+    x = synth.activations(BATCH, H, seed=0, dtype=torch.bfloat16).float().numpy().astype(np.float64)
+    kl, vl = synth.kv_cache((BATCH, NKV, KV_LEN + 1, D), seed=0)
+    kb, vb = synth.bits(kl), synth.bits(vl)
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        oracle.decode_layer(dims, wb, x, kb, vb, KV_LEN)
+        n += 1
+        if time.perf_counter() - t0 > 10.0 or n >= 5:
+            break
+    t_layer = (time.perf_counter() - t0) / n
+    return {"value": BATCH / (t_layer * L), "unit": "tokens/s", "cores": oracle.get_threads(), "kind": "oracle",
+            "sample": f"{n} run(s) of one decoder layer (B={BATCH}, KV {KV_LEN}), fp64; x{L} layers extrapolated"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    ws, rank, local = dist_init()
+    if args.impl == "reference":
+        return run_reference(args, ws, rank)
+    return run_ours(args, ws, rank, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,277 @@
+/*
+ * tpl -- a single-device Megatron-style tensor-parallel transformer layer.
+ *
+ * The problem, as the pages state it: an input x, a shard degree t and the
+ * layer dimensions go in; the output equals that of the unsharded layer.
+ * Inside, the layer is computed the tensor-parallel way:
+ *   - Q/K/V and gate/up projections are split by output columns into t
+ *     shards, Q/K/V by whole attention heads ("Tensor parallel scaling
+ *     curves", section "What tensor parallelism actually splits"; the
+ *     ownership rule heads[rank*h_per_gpu:(rank+1)*h_per_gpu]);
+ *   - each shard attends over its own heads only, with no exchange (same
+ *     section, "local attention on owned heads");
+ *   - the O and down projections are split by input rows, so each shard
+ *     yields a full-size partial sum, and the t partials are added -- the
+ *     arithmetic of the all-reduce, two per layer, 2L per forward pass (same
+ *     section; "Tensor Parallelism Fundamentals", section "Mechanics of
+ *     Matrix Slicing").
+ * All t shards live in one device's memory: a shard is a weight and KV-cache
+ * layout, and the partial-sum reduction runs on the device, fused into the
+ * epilogue of the row-parallel kernels (TPL_REDUCE_FUSED) or as a separate
+ * ordered reduction (TPL_REDUCE_SEPARATE, kept for comparison).  The two
+ * modes produce bitwise identical results.
+ *
+ * Conventions for every call:
+ *   - Device pointers are plain CUDA device addresses; host pointers are
+ *     marked "host".  The caller owns every buffer (weights, packed weights,
+ *     KV caches, activations, workspace); the library never allocates device
+ *     memory and owns only the host-side plan.
+ *   - `stream` is a cudaStream_t passed as void*.  Calls only enqueue work on
+ *     it and return; nothing synchronises except tpl_last_device_error.
+ *   - Calls return a status (TPL_OK or a TPL_E* code).  Arguments are
+ *     validated on the host before anything is launched; on an error nothing
+ *     is launched.  No C++ exception crosses this interface.
+ *   - Activations use the "activation type": bf16 by default, fp32 when the
+ *     plan's flags contain TPL_FP32_WEIGHTS.  The KV cache is always bf16.
+ *   - Weights use the nn.Linear orientation W[out][in], row-major.
+ */
+#ifndef TPL_H
+#define TPL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+#if defined(__GNUC__)
+#pragma GCC visibility push(default)
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+#define TPL_OK 0
+#define TPL_EINVAL 1        /* null pointer, negative size, bad enum value      */
+#define TPL_EINDIVISIBLE 2  /* t not in {1,2,4,8}, or t does not divide n_q_heads,
+                               n_kv_heads or ffn                                 */
+#define TPL_EWORKSPACE 3    /* workspace smaller than tpl_workspace_size()       */
+#define TPL_ENOMEM 4        /* a caller-provided capacity is too small (packed
+                               buffer, KV capacity)                              */
+#define TPL_ECUDA 5         /* a CUDA call or kernel launch failed               */
+#define TPL_EDEVICE 6       /* a kernel reported an inconsistency (device error
+                               word, read by tpl_last_device_error)              */
+#define TPL_EUNSUPPORTED 7  /* valid dimensions this build does not implement
+                               (head_dim != 128, group size > 16, dims not a
+                               multiple of 8)                                    */
+
+/* ---- flags ------------------------------------------------------------- */
+#define TPL_NORM 1u          /* pre-RMSNorm before QKV and before gate/up       */
+#define TPL_RESIDUAL 2u      /* residual adds after O and after down            */
+#define TPL_FP32_WEIGHTS 4u  /* fp32 weights and activations (KV stays bf16)    */
+
+#define TPL_REDUCE_FUSED 0    /* t-way sum inside the row-parallel epilogue     */
+#define TPL_REDUCE_SEPARATE 1 /* partials to memory, then tpl_reduce_partials   */
+
+typedef void *tpl_stream; /* a cudaStream_t */
+
+/* Layer dimensions.  head_dim must be 128; hidden and ffn/t multiples of 8. */
+typedef struct {
+    int32_t hidden, n_q_heads, n_kv_heads, head_dim, ffn, n_layers;
+    float rms_eps;
+    uint32_t flags; /* TPL_NORM | TPL_RESIDUAL | TPL_FP32_WEIGHTS */
+} tpl_dims;
+
+typedef struct tpl_plan tpl_plan; /* opaque, host-owned by the library */
+
+/* Footprints of a plan.  All sizes are per layer unless stated. */
+typedef struct {
+    int32_t t;
+    int32_t q_heads_per_shard, kv_heads_per_shard, ffn_per_shard, group_size;
+    int32_t qkv_rows_per_shard;        /* (n_q/t + 2 n_kv/t) * head_dim          */
+    int32_t elem_bytes;                /* weight/activation element size: 2 or 4 */
+    int64_t layer_params_per_shard;    /* Wq,Wk,Wv rows + Wo cols + Wg,Wu rows + Wd cols */
+    int64_t layer_weight_bytes_per_shard;
+    int64_t packed_layer_bytes;        /* bytes tpl_pack_layer writes (all shards + gains) */
+    int64_t reductions_per_step;       /* 2 * n_layers                             */
+} tpl_plan_info;
+
+/* Unsharded weights of one layer on the device, nn.Linear orientation, in the
+ * activation type: wq [n_q*d][H], wk/wv [n_kv*d][H], wo [H][n_q*d],
+ * wg/wu [F][H], wd [H][F].  gamma_* are fp32 [H]; NULL means all ones.
+ * For an MLP-only plan (n_q_heads used only for sizing) wq..wo may be NULL. */
+typedef struct {
+    const void *wq, *wk, *wv, *wo, *wg, *wu, *wd;
+    const float *gamma_attn, *gamma_mlp;
+} tpl_layer_weights;
+
+/* The KV cache of one layer, all shards, bf16, shard-major:
+ *   k, v: [t][batch_cap][n_kv/t][seq_cap][head_dim]
+ * (shard s's part is a contiguous block, as it would be on its own GPU; the
+ * per-GPU size is the formula of "Tensor Parallelism Fundamentals", section
+ * "Memory Overhead and Communication Bottlenecks"). */
+typedef struct {
+    void *k, *v;
+    int32_t batch_cap;
+    int64_t seq_cap;
+} tpl_kv;
+
+/* ---- planning (host only; no GPU needed) -------------------------------- */
+
+/* Create a plan for dims `*dims` and degree t.  Validates the shard maps of
+ * "Tensor parallel scaling curves" ("What tensor parallelism actually
+ * splits"): t in {1,2,4,8} ("Tensor Parallelism" docs: the size is 1, 2, 4 or
+ * 8), t | n_q_heads, t | n_kv_heads, t | ffn, n_kv_heads | n_q_heads.
+ * *out receives a plan to be released with tpl_plan_destroy. */
+int tpl_plan_create(const tpl_dims *dims, int32_t t, tpl_plan **out);
+void tpl_plan_destroy(tpl_plan *plan);
+
+/* Plan options (host).  TPL_OPT_GEMV_MODE selects the inner product of the
+ * bf16 matrix-vector kernels: 0 = tensor cores (mma.sync, the default),
+ * 2 = FFMA on the CUDA cores (kept to measure against).  fp32 plans always
+ * use FFMA.  Returns TPL_EINVAL for an unknown option or value. */
+#define TPL_OPT_GEMV_MODE 1
+int tpl_plan_set_option(tpl_plan *plan, int32_t option, int32_t value);
+
+/* Footprints (host) -- see tpl_plan_info. */
+int tpl_plan_info_get(const tpl_plan *plan, tpl_plan_info *out);
+
+/* Shard maps (host arrays, each may be NULL):
+ *   q_shard[n_q], q_local[n_q]: shard and local index of query head h;
+ *   kv_shard[n_kv]: shard of kv head j;
+ *   ffn_shard[ffn]: shard of ffn column c;
+ *   packed_offsets[4*t + 2]: byte offsets inside a packed layer of the blocks
+ *     Wqkv[s], Wo[s], Wgu[s], Wd[s] (s = 0..t-1, in that order) followed by
+ *     gamma_attn and gamma_mlp. */
+int tpl_plan_maps(const tpl_plan *plan, int32_t *q_shard, int32_t *q_local, int32_t *kv_shard,
+                  int32_t *ffn_shard, int64_t *packed_offsets);
+
+/* Per-GPU KV bytes of the whole model: 2*n_layers*n_kv*head_dim*seq*
+ * bytes_per_elem*batch / t ("Tensor Parallelism Fundamentals", "Memory
+ * Overhead and Communication Bottlenecks").  Returns -1 on invalid input or
+ * when t does not divide the total. */
+int64_t tpl_kv_bytes(const tpl_dims *dims, int32_t t, int64_t batch, int64_t seq,
+                     int32_t bytes_per_elem);
+
+/* Bytes of one layer's K (or V) buffer for tpl_kv with the given capacities. */
+int64_t tpl_kv_layer_bytes(const tpl_plan *plan, int32_t batch_cap, int64_t seq_cap);
+
+/* Workspace bytes needed by the decode calls for batch B and cached length S
+ * (both reduce modes), and by tpl_prefill_layer for T tokens when B = T. */
+int tpl_workspace_size(const tpl_plan *plan, int32_t batch, int64_t seq, size_t *out);
+
+/* ---- device calls ------------------------------------------------------- */
+
+/* Zero the workspace's bookkeeping words (cross-block arrival counters).
+ * Call once after allocating a workspace (or zero the whole buffer); kernels
+ * leave the counters at zero afterwards. */
+int tpl_workspace_init(const tpl_plan *plan, void *ws, size_t ws_bytes, tpl_stream stream);
+
+/* Rearrange one layer's unsharded weights into the plan's packed shard
+ * layout (`packed`, packed_bytes >= info.packed_layer_bytes):
+ *   Wqkv[s] = rows [q heads of s | k heads of s | v heads of s] of Wq/Wk/Wv
+ *   Wo[s]   = Wo[:, s*(n_q/t)*d : (s+1)*(n_q/t)*d]           (row split)
+ *   Wgu[s]  = rows Wg[c], Wu[c] interleaved for c in shard s's ffn columns
+ *   Wd[s]   = Wd[:, s*F/t : (s+1)*F/t]                        (row split)
+ * then gamma_attn, gamma_mlp (fp32).  "Tensor parallel scaling curves",
+ * "What tensor parallelism actually splits". */
+int tpl_pack_layer(const tpl_plan *plan, const tpl_layer_weights *w, void *packed,
+                   size_t packed_bytes, tpl_stream stream);
+
+/* Copy an unsharded cache [batch_cap][n_kv][seq_cap][d] (bf16) into the
+ * shard-major layout of tpl_kv (both device buffers, same byte size). */
+int tpl_pack_kv(const tpl_plan *plan, const void *unsharded, void *sharded, int32_t batch_cap,
+                int64_t seq_cap, tpl_stream stream);
+
+/* One decode step of one layer for B sequences with S cached tokens each
+ * (the new token is position S; requires S < kv->seq_cap, B <= batch_cap):
+ *   a = RMSNorm(x)            [TPL_NORM]
+ *   q|k|v = column-parallel projection of a, k/v written to slot S
+ *   o = owned-head GQA attention over the S+1 positions
+ *   h = x + sum_s o_s Wo[s]^T  (reduction point 1)   [+x if TPL_RESIDUAL]
+ *   m = RMSNorm(h)            [TPL_NORM]
+ *   y = h + sum_s (silu(m Wg_s^T) * (m Wu_s^T)) Wd[s]^T (reduction point 2)
+ * x, y: [B][hidden] activation type; y32: fp32 [B][hidden] or NULL.
+ * reduce_mode: TPL_REDUCE_FUSED or TPL_REDUCE_SEPARATE. */
+int tpl_decode_layer(tpl_plan *plan, const void *packed, const tpl_kv *kv, const void *x,
+                     int32_t B, int64_t S, void *y, float *y32, void *ws, size_t ws_bytes,
+                     int32_t reduce_mode, tpl_stream stream);
+
+/* n_layers decode steps: layer l reads layer l-1's output.  packed_per_layer
+ * and kv_per_layer are host arrays of n_layers entries.  Adds 2 * n_layers to
+ * the plan's reduction counter ("Tensor parallel scaling curves": 2L
+ * all-reduce points per forward pass). */
+int tpl_decode_stack(tpl_plan *plan, const void *const *packed_per_layer, const tpl_kv *kv_per_layer,
+                     const void *x, int32_t B, int64_t S, void *y, float *y32, void *ws,
+                     size_t ws_bytes, int32_t reduce_mode, tpl_stream stream);
+
+/* Prefill of one layer over T tokens of one sequence starting at position 0
+ * (causal inside the chunk: token i sees positions 0..i), writing K/V cache
+ * slots 0..T-1 of batch row 0.  x, y: [T][hidden] activation type. */
+int tpl_prefill_layer(tpl_plan *plan, const void *packed, const tpl_kv *kv, const void *x,
+                      int32_t T, void *y, float *y32, void *ws, size_t ws_bytes,
+                      int32_t reduce_mode, tpl_stream stream);
+
+/* ---- the individual steps (each is one kernel launch, except where noted;
+ *      the decode calls above are these in order) --------------------------- */
+
+/* Column-parallel QKV: q [B][n_q][d] fp32; k/v of the new token to slot S. */
+int tpl_qkv(tpl_plan *plan, const void *packed, const tpl_kv *kv, const void *x, int32_t B,
+            int64_t S, float *q, void *ws, size_t ws_bytes, tpl_stream stream);
+
+/* Owned-head GQA decode attention over positions 0..S (split over the key
+ * range, partial results combined in a fixed order).  o [B][n_q*d]
+ * activation type.  Uses the workspace for the split partials. */
+int tpl_attn_decode(tpl_plan *plan, const tpl_kv *kv, const float *q, int32_t B, int64_t S,
+                    void *o, void *ws, size_t ws_bytes, tpl_stream stream);
+
+/* Row-parallel O projection.  partials == NULL: fused, h = x + sum_s o_s
+ * Wo[s]^T (fp32 [B][H]); partials != NULL: writes P[s] = o_s Wo[s]^T
+ * (fp32 [t][B][H]) and leaves h untouched. */
+int tpl_o_proj(tpl_plan *plan, const void *packed, const void *o, const void *x, int32_t B, float *h,
+               float *partials, void *ws, size_t ws_bytes, tpl_stream stream);
+
+/* Column-parallel gate/up with SwiGLU: act [B][F] = silu(m Wg^T) * (m Wu^T),
+ * m = RMSNorm(h) [TPL_NORM] or h.  h: fp32 [B][H], or the activation type
+ * when h_is_act != 0. */
+int tpl_gate_up(tpl_plan *plan, const void *packed, const void *h, int32_t h_is_act, int32_t B,
+                void *act, void *ws, size_t ws_bytes, tpl_stream stream);
+
+/* Row-parallel down projection, like tpl_o_proj: fused y = h + sum_s act_s
+ * Wd[s]^T (y activation type, y32 fp32 or NULL), or partials. */
+int tpl_down_proj(tpl_plan *plan, const void *packed, const void *act, const float *h, int32_t B,
+                  void *y, float *y32, float *partials, void *ws, size_t ws_bytes, tpl_stream stream);
+
+/* The separate reduction: out = resid + P[0] + P[1] + ... + P[t-1] in that
+ * order (resid NULL: no residual).  P fp32 [t][B][H]; resid is fp32 when
+ * resid_is_f32, else the activation type; out32 fp32 (may be NULL), out_act
+ * activation type (may be NULL).  Counts one reduction point. */
+int tpl_reduce_partials(tpl_plan *plan, const float *P, const void *resid, int32_t resid_is_f32,
+                        int32_t B, float *out32, void *out_act, tpl_stream stream);
+
+/* The MLP pair alone (gate/up column-split, down row-split; flags decide the
+ * norm and the residual): y = [x +] sum_s (silu(a Wg_s^T) * (a Wu_s^T)) Wd[s]^T,
+ * a = RMSNorm(x) [TPL_NORM] or x.  "Tensor Parallelism Fundamentals",
+ * "Mechanics of Matrix Slicing" (the feed-forward example). */
+int tpl_mlp_block(tpl_plan *plan, const void *packed, const void *x, int32_t B, void *y, float *y32,
+                  void *ws, size_t ws_bytes, int32_t reduce_mode, tpl_stream stream);
+
+/* ---- diagnostics -------------------------------------------------------- */
+
+/* Reduction points launched through this plan since creation/reset. */
+int64_t tpl_reduction_count(const tpl_plan *plan);
+void tpl_reset_counters(tpl_plan *plan);
+
+/* Synchronise `stream`, read and clear the device error word of the current
+ * device.  TPL_OK, TPL_EDEVICE (a kernel recorded an inconsistency) or
+ * TPL_ECUDA (the stream reported an error). */
+int tpl_last_device_error(const tpl_plan *plan, tpl_stream stream);
+
+/* Static description of a status code. */
+const char *tpl_status_string(int status);
+
+#if defined(__GNUC__)
+#pragma GCC visibility pop
+#endif
+#ifdef __cplusplus
+}
+#endif
+#endif /* TPL_H */

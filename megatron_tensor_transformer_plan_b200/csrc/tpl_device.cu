@@ -1,0 +1,525 @@
+// Kernels and C-ABI entry points of libtpl (one translation unit, so the
+// device error word is a plain __device__ variable).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstring>
+
+#include "tpl_attn.cuh"
+#include "tpl_common.cuh"
+#include "tpl_gemv.cuh"
+#include "tpl_internal.h"
+
+namespace tpl {
+
+// out = resid + ((P[0] + P[1]) + ... + P[t-1]), the separate form of the
+// row-split sum ("Tensor parallel scaling curves": the all-reduce after the
+// output and down projections).  Same order and operations as the fused
+// epilogue of gemv_kernel, hence identical bits.
+__global__ void reduce_partials_kernel(const float *__restrict__ P, int t, int64_t n, const void *resid,
+                                       int resid_f32, float *out32, void *out_act, int act_f32) {
+    pdl_wait();
+    pdl_trigger();
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        float acc = P[i];
+        for (int s = 1; s < t; ++s) acc = acc + P[(int64_t)s * n + i];
+        if (resid) acc = load_act(resid, resid_f32, i) + acc;
+        if (out32) out32[i] = acc;
+        if (out_act) store_act(out_act, act_f32, i, acc);
+    }
+}
+
+__global__ void fill_f32_kernel(float *p, int64_t n, float v) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        p[i] = v;
+}
+
+namespace {
+
+// Launch with programmatic dependent launch enabled: the kernel may start
+// while the previous kernel on the stream drains; every kernel here waits
+// (griddepcontrol.wait) before touching data a previous kernel wrote.
+template <typename... KA, typename... A>
+cudaError_t launch_pdl(void (*kern)(KA...), int grid, int block, size_t smem, cudaStream_t st, A &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...);
+}
+
+bool g_attr_done[64][3];
+
+int prepare_gemv(int mode) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return TPL_ECUDA;
+    if (!g_attr_done[dev][mode]) {
+        cudaError_t e;
+        const int maxb = 227 * 1024;
+        if (mode == 0) e = cudaFuncSetAttribute(gemv_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxb);
+        else if (mode == 1) e = cudaFuncSetAttribute(gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxb);
+        else e = cudaFuncSetAttribute(gemv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxb);
+        if (e != cudaSuccess) return TPL_ECUDA;
+        g_attr_done[dev][mode] = true;
+    }
+    return TPL_OK;
+}
+
+int cuda_rc(cudaError_t e) { return e == cudaSuccess ? TPL_OK : TPL_ECUDA; }
+
+bool al16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+struct Ctx {
+    tpl_plan *p;
+    char *ws;
+    WsLayout L;
+    cudaStream_t st;
+    int B;
+    int64_t S;
+};
+
+int make_ctx(tpl_plan *p, void *ws, size_t ws_bytes, int B, int64_t S, tpl_stream stream, Ctx *c) {
+    if (!p || !ws || !al16(ws)) return TPL_EINVAL;
+    if (B < 1 || B > 16 || S < 0) return B > 16 ? TPL_EUNSUPPORTED : TPL_EINVAL;
+    int rc = ws_layout(p, B, S, &c->L);
+    if (rc != TPL_OK) return rc;
+    if (ws_bytes < c->L.total) return TPL_EWORKSPACE;
+    c->p = p;
+    c->ws = static_cast<char *>(ws);
+    c->st = static_cast<cudaStream_t>(stream);
+    c->B = B;
+    c->S = S;
+    return TPL_OK;
+}
+
+int check_kv(const tpl_kv *kv, int B, int64_t S) {
+    if (!kv || !kv->k || !kv->v || !al16(kv->k) || !al16(kv->v)) return TPL_EINVAL;
+    if (kv->batch_cap < B || kv->seq_cap <= S || S < 0) return TPL_ENOMEM;
+    return TPL_OK;
+}
+
+int gemv_launch(Ctx &c, GemvArgs &a, int N, int nseg, int Kseg, int op) {
+    tpl_plan *p = c.p;
+    const int sms = num_sms_current();
+    if (sms <= 0) return TPL_ECUDA;
+    int rc = gemv_geom(N, nseg, Kseg, c.B, p->f32 ? 4 : 2, sms, &a.g);
+    if (rc != TPL_OK) return rc;
+    const int mode = p->f32 ? 1 : (p->gemv_mode == 2 ? 2 : 0);
+    rc = prepare_gemv(mode);
+    if (rc != TPL_OK) return rc;
+    a.B = c.B;
+    a.gp = reinterpret_cast<float *>(c.ws + c.L.gp);
+    a.tickets = reinterpret_cast<unsigned *>(c.ws + c.L.tickets) + kTicketGemv + 512 * op;
+    const int grid = a.g.rb * a.g.ksplit;
+    cudaError_t e;
+    if (mode == 0) e = launch_pdl(gemv_kernel<0>, grid, kGemvThreads, a.g.smem, c.st, a);
+    else if (mode == 1) e = launch_pdl(gemv_kernel<1>, grid, kGemvThreads, a.g.smem, c.st, a);
+    else e = launch_pdl(gemv_kernel<2>, grid, kGemvThreads, a.g.smem, c.st, a);
+    return cuda_rc(e);
+}
+
+GemvArgs base_args(const tpl_plan *p) {
+    GemvArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.act_f32 = p->f32 ? 1 : 0;
+    a.eps = p->d.rms_eps;
+    a.hd = p->d.head_dim;
+    return a;
+}
+
+int run_qkv(Ctx &c, const char *packed, const tpl_kv *kv, const void *x, float *q) {
+    tpl_plan *p = c.p;
+    GemvArgs a = base_args(p);
+    a.W = packed + p->off_qkv;
+    a.blk_r = p->blk_qkv;
+    a.rps = p->qkv_rows_s;
+    a.ldw = p->d.hidden;
+    a.x = x;
+    a.x_f32 = p->f32;
+    a.ldx = p->d.hidden;
+    a.norm = (p->d.flags & TPL_NORM) ? 1 : 0;
+    a.gamma = reinterpret_cast<const float *>(packed + p->off_g1);
+    a.epi = EPI_QKV;
+    a.q = q;
+    a.kc = static_cast<__nv_bfloat16 *>(kv->k);
+    a.vc = static_cast<__nv_bfloat16 *>(kv->v);
+    a.nq = p->d.n_q_heads;
+    a.nq_s = p->nq_s;
+    a.nkv_s = p->nkv_s;
+    a.batch_cap = kv->batch_cap;
+    a.S = c.S;
+    a.seq_cap = kv->seq_cap;
+    return gemv_launch(c, a, p->t * p->qkv_rows_s, 1, p->d.hidden, OP_QKV);
+}
+
+int run_attn(Ctx &c, const tpl_kv *kv, const float *q, void *o) {
+    tpl_plan *p = c.p;
+    AttnGeom g;
+    attn_geom(c.B, p->d.n_kv_heads, c.S, &g);
+    if (g.pairs > kMaxPairs) return TPL_EUNSUPPORTED;
+    AttnArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.q = q;
+    a.kc = static_cast<const __nv_bfloat16 *>(kv->k);
+    a.vc = static_cast<const __nv_bfloat16 *>(kv->v);
+    a.seq_cap = kv->seq_cap;
+    a.batch_cap = kv->batch_cap;
+    a.B = c.B;
+    a.nq = p->d.n_q_heads;
+    a.nkv_s = p->nkv_s;
+    a.g = p->g;
+    a.keys = c.S + 1;
+    a.nsplit = g.nsplit;
+    a.kps = g.kps;
+    a.scale_log2 = 1.4426950408889634f / sqrtf((float)p->d.head_dim);
+    a.part_o = reinterpret_cast<float *>(c.ws + c.L.part_o);
+    a.part_ml = reinterpret_cast<float *>(c.ws + c.L.part_ml);
+    a.tickets = reinterpret_cast<unsigned *>(c.ws + c.L.tickets) + kTicketAttn;
+    a.o = o;
+    a.o_f32 = p->f32;
+    const int grid = g.pairs * (g.nsplit / kAttnWarps);
+    return cuda_rc(launch_pdl(attn_decode_kernel, grid, kAttnWarps * 32, 0, c.st, a));
+}
+
+// Row-parallel O projection: fused (partials == NULL) or partial output.
+int run_o(Ctx &c, const char *packed, const void *o, const void *resid, float *h, float *partials) {
+    tpl_plan *p = c.p;
+    GemvArgs a = base_args(p);
+    a.W = packed + p->off_o;
+    a.blk_s = p->blk_o;
+    a.rps = p->d.hidden;
+    a.ldw = p->nq_s * p->d.head_dim;
+    a.x = o;
+    a.x_f32 = p->f32;
+    a.ldx = p->d.n_q_heads * p->d.head_dim;
+    if (partials) {
+        a.epi = EPI_ROW_PARTIAL;
+        a.partials = partials;
+    } else {
+        a.epi = EPI_ROW;
+        a.resid = resid;
+        a.resid_f32 = p->f32;
+        a.out32 = h;
+    }
+    int rc = gemv_launch(c, a, p->d.hidden, p->t, p->nq_s * p->d.head_dim, OP_O);
+    if (rc == TPL_OK && !partials) p->reductions.fetch_add(1);
+    return rc;
+}
+
+int run_gu(Ctx &c, const char *packed, const void *h, int h_is_act, void *act) {
+    tpl_plan *p = c.p;
+    GemvArgs a = base_args(p);
+    a.W = packed + p->off_gu;
+    a.blk_r = p->blk_gu;
+    a.rps = 2 * p->F_s;
+    a.ldw = p->d.hidden;
+    a.x = h;
+    a.x_f32 = h_is_act ? p->f32 : 1;
+    a.ldx = p->d.hidden;
+    a.norm = (p->d.flags & TPL_NORM) ? 1 : 0;
+    a.gamma = reinterpret_cast<const float *>(packed + p->off_g2);
+    a.epi = EPI_GU;
+    a.out_act = act;
+    return gemv_launch(c, a, p->t * 2 * p->F_s, 1, p->d.hidden, OP_GU);
+}
+
+int run_down(Ctx &c, const char *packed, const void *act, const void *resid, int resid_f32, void *y, float *y32,
+             float *partials) {
+    tpl_plan *p = c.p;
+    GemvArgs a = base_args(p);
+    a.W = packed + p->off_d;
+    a.blk_s = p->blk_d;
+    a.rps = p->d.hidden;
+    a.ldw = p->F_s;
+    a.x = act;
+    a.x_f32 = p->f32;
+    a.ldx = p->d.ffn;
+    if (partials) {
+        a.epi = EPI_ROW_PARTIAL;
+        a.partials = partials;
+    } else {
+        a.epi = EPI_ROW;
+        a.resid = resid;
+        a.resid_f32 = resid_f32;
+        a.out32 = y32;
+        a.out_act = y;
+    }
+    int rc = gemv_launch(c, a, p->d.hidden, p->t, p->F_s, OP_DOWN);
+    if (rc == TPL_OK && !partials) p->reductions.fetch_add(1);
+    return rc;
+}
+
+int run_reduce(tpl_plan *p, cudaStream_t st, const float *P, const void *resid, int resid_f32, int B, float *out32,
+               void *out_act) {
+    const int64_t n = (int64_t)B * p->d.hidden;
+    const int grid = (int)std::min<int64_t>((n + 255) / 256, 4 * 148);
+    int rc = cuda_rc(launch_pdl(reduce_partials_kernel, grid, 256, 0, st, P, p->t, n, resid, resid_f32, out32, out_act,
+                                p->f32 ? 1 : 0));
+    if (rc == TPL_OK) p->reductions.fetch_add(1);
+    return rc;
+}
+
+// One decode layer: x (activation type) -> y (activation type) [+ y32].
+int decode_layer(Ctx &c, const char *packed, const tpl_kv *kv, const void *x, void *y, float *y32, int mode) {
+    tpl_plan *p = c.p;
+    const bool resid = (p->d.flags & TPL_RESIDUAL) != 0;
+    float *q = reinterpret_cast<float *>(c.ws + c.L.q);
+    void *o = c.ws + c.L.o;
+    float *h = reinterpret_cast<float *>(c.ws + c.L.h);
+    void *act = c.ws + c.L.act;
+    float *P = reinterpret_cast<float *>(c.ws + c.L.P);
+    int rc = run_qkv(c, packed, kv, x, q);
+    if (rc == TPL_OK) rc = run_attn(c, kv, q, o);
+    if (rc == TPL_OK) {
+        if (mode == TPL_REDUCE_FUSED) {
+            rc = run_o(c, packed, o, resid ? x : nullptr, h, nullptr);
+        } else {
+            rc = run_o(c, packed, o, nullptr, nullptr, P);
+            if (rc == TPL_OK) rc = run_reduce(p, c.st, P, resid ? x : nullptr, p->f32, c.B, h, nullptr);
+        }
+    }
+    if (rc == TPL_OK) rc = run_gu(c, packed, h, 0, act);
+    if (rc == TPL_OK) {
+        if (mode == TPL_REDUCE_FUSED) {
+            rc = run_down(c, packed, act, resid ? h : nullptr, 1, y, y32, nullptr);
+        } else {
+            rc = run_down(c, packed, act, nullptr, 1, nullptr, nullptr, P);
+            if (rc == TPL_OK) rc = run_reduce(p, c.st, P, resid ? h : nullptr, 1, c.B, y32, y);
+        }
+    }
+    return rc;
+}
+
+}  // namespace
+}  // namespace tpl
+
+using namespace tpl;
+
+extern "C" {
+
+int tpl_workspace_init(const tpl_plan *plan, void *ws, size_t ws_bytes, tpl_stream stream) {
+    if (!plan || !ws) return TPL_EINVAL;
+    if (ws_bytes < sizeof(uint32_t) * kTicketSlots) return TPL_EWORKSPACE;
+    return cuda_rc(cudaMemsetAsync(ws, 0, sizeof(uint32_t) * kTicketSlots, static_cast<cudaStream_t>(stream)));
+}
+
+int tpl_pack_layer(const tpl_plan *p, const tpl_layer_weights *w, void *packed, size_t packed_bytes,
+                   tpl_stream stream) {
+    if (!p || !w || !packed || !al16(packed)) return TPL_EINVAL;
+    if ((int64_t)packed_bytes < p->packed_bytes) return TPL_ENOMEM;
+    if (!w->wg || !w->wu || !w->wd) return TPL_EINVAL;
+    const bool attn = w->wq && w->wk && w->wv && w->wo;
+    if (!attn && (w->wq || w->wk || w->wv || w->wo)) return TPL_EINVAL;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const tpl_dims &d = p->d;
+    const int64_t es = p->esize, H = d.hidden, hd = d.head_dim, F = d.ffn;
+    const int64_t Ks = (int64_t)p->nq_s * hd;
+    char *P = static_cast<char *>(packed);
+    const char *wq = static_cast<const char *>(w->wq), *wk = static_cast<const char *>(w->wk);
+    const char *wv = static_cast<const char *>(w->wv), *wo = static_cast<const char *>(w->wo);
+    const char *wg = static_cast<const char *>(w->wg), *wu = static_cast<const char *>(w->wu);
+    const char *wd = static_cast<const char *>(w->wd);
+    cudaError_t e = cudaSuccess;
+    auto ok = [&](cudaError_t r) {
+        if (e == cudaSuccess) e = r;
+    };
+    for (int s = 0; s < p->t; ++s) {
+        if (attn) {
+            char *dq = P + p->off_qkv + s * p->blk_qkv;
+            const int64_t qb = (int64_t)p->nq_s * hd * H * es, kb = (int64_t)p->nkv_s * hd * H * es;
+            ok(cudaMemcpyAsync(dq, wq + s * qb, qb, cudaMemcpyDeviceToDevice, st));
+            ok(cudaMemcpyAsync(dq + qb, wk + s * kb, kb, cudaMemcpyDeviceToDevice, st));
+            ok(cudaMemcpyAsync(dq + qb + kb, wv + s * kb, kb, cudaMemcpyDeviceToDevice, st));
+            ok(cudaMemcpy2DAsync(P + p->off_o + s * p->blk_o, Ks * es, wo + s * Ks * es, (int64_t)d.n_q_heads * hd * es,
+                                 Ks * es, H, cudaMemcpyDeviceToDevice, st));
+        }
+        char *dgu = P + p->off_gu + s * p->blk_gu;
+        ok(cudaMemcpy2DAsync(dgu, 2 * H * es, wg + (int64_t)s * p->F_s * H * es, H * es, H * es, p->F_s,
+                             cudaMemcpyDeviceToDevice, st));
+        ok(cudaMemcpy2DAsync(dgu + H * es, 2 * H * es, wu + (int64_t)s * p->F_s * H * es, H * es, H * es, p->F_s,
+                             cudaMemcpyDeviceToDevice, st));
+        ok(cudaMemcpy2DAsync(P + p->off_d + s * p->blk_d, (int64_t)p->F_s * es, wd + (int64_t)s * p->F_s * es, F * es,
+                             (int64_t)p->F_s * es, H, cudaMemcpyDeviceToDevice, st));
+    }
+    float *g1 = reinterpret_cast<float *>(P + p->off_g1), *g2 = reinterpret_cast<float *>(P + p->off_g2);
+    if (w->gamma_attn) ok(cudaMemcpyAsync(g1, w->gamma_attn, H * 4, cudaMemcpyDeviceToDevice, st));
+    else {
+        fill_f32_kernel<<<(int)((H + 255) / 256), 256, 0, st>>>(g1, H, 1.0f);
+        ok(cudaGetLastError());
+    }
+    if (w->gamma_mlp) ok(cudaMemcpyAsync(g2, w->gamma_mlp, H * 4, cudaMemcpyDeviceToDevice, st));
+    else {
+        fill_f32_kernel<<<(int)((H + 255) / 256), 256, 0, st>>>(g2, H, 1.0f);
+        ok(cudaGetLastError());
+    }
+    return cuda_rc(e);
+}
+
+int tpl_pack_kv(const tpl_plan *p, const void *unsharded, void *sharded, int32_t batch_cap, int64_t seq_cap,
+                tpl_stream stream) {
+    if (!p || !unsharded || !sharded || batch_cap < 0 || seq_cap < 0) return TPL_EINVAL;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t row = seq_cap * p->d.head_dim * 2;  // one head's cache bytes
+    cudaError_t e = cudaSuccess;
+    for (int s = 0; s < p->t && e == cudaSuccess; ++s) {
+        const char *src = static_cast<const char *>(unsharded) + (int64_t)s * p->nkv_s * row;
+        char *dst = static_cast<char *>(sharded) + (int64_t)s * batch_cap * p->nkv_s * row;
+        e = cudaMemcpy2DAsync(dst, p->nkv_s * row, src, (int64_t)p->d.n_kv_heads * row, p->nkv_s * row, batch_cap,
+                              cudaMemcpyDeviceToDevice, st);
+    }
+    return cuda_rc(e);
+}
+
+int tpl_qkv(tpl_plan *p, const void *packed, const tpl_kv *kv, const void *x, int32_t B, int64_t S, float *q,
+            void *ws, size_t ws_bytes, tpl_stream stream) {
+    if (B == 0) return TPL_OK;
+    Ctx c;
+    int rc = make_ctx(p, ws, ws_bytes, B, S, stream, &c);
+    if (rc != TPL_OK) return rc;
+    if (!packed || !x || !q || !al16(x) || !al16(packed)) return TPL_EINVAL;
+    if ((rc = check_kv(kv, B, S)) != TPL_OK) return rc;
+    return run_qkv(c, static_cast<const char *>(packed), kv, x, q);
+}
+
+int tpl_attn_decode(tpl_plan *p, const tpl_kv *kv, const float *q, int32_t B, int64_t S, void *o, void *ws,
+                    size_t ws_bytes, tpl_stream stream) {
+    if (B == 0) return TPL_OK;
+    Ctx c;
+    int rc = make_ctx(p, ws, ws_bytes, B, S, stream, &c);
+    if (rc != TPL_OK) return rc;
+    if (!q || !o || !al16(q)) return TPL_EINVAL;
+    if ((rc = check_kv(kv, B, S)) != TPL_OK) return rc;
+    return run_attn(c, kv, q, o);
+}
+
+int tpl_o_proj(tpl_plan *p, const void *packed, const void *o, const void *x, int32_t B, float *h, float *partials,
+               void *ws, size_t ws_bytes, tpl_stream stream) {
+    if (B == 0) return TPL_OK;
+    Ctx c;
+    int rc = make_ctx(p, ws, ws_bytes, B, 0, stream, &c);
+    if (rc != TPL_OK) return rc;
+    if (!packed || !o || !al16(o) || (!partials && !h)) return TPL_EINVAL;
+    const bool resid = (p->d.flags & TPL_RESIDUAL) != 0;
+    if (resid && !partials && !x) return TPL_EINVAL;
+    return run_o(c, static_cast<const char *>(packed), o, resid ? x : nullptr, h, partials);
+}
+
+int tpl_gate_up(tpl_plan *p, const void *packed, const void *h, int32_t h_is_act, int32_t B, void *act, void *ws,
+                size_t ws_bytes, tpl_stream stream) {
+    if (B == 0) return TPL_OK;
+    Ctx c;
+    int rc = make_ctx(p, ws, ws_bytes, B, 0, stream, &c);
+    if (rc != TPL_OK) return rc;
+    if (!packed || !h || !act || !al16(h)) return TPL_EINVAL;
+    return run_gu(c, static_cast<const char *>(packed), h, h_is_act ? 1 : 0, act);
+}
+
+int tpl_down_proj(tpl_plan *p, const void *packed, const void *act, const float *h, int32_t B, void *y, float *y32,
+                  float *partials, void *ws, size_t ws_bytes, tpl_stream stream) {
+    if (B == 0) return TPL_OK;
+    Ctx c;
+    int rc = make_ctx(p, ws, ws_bytes, B, 0, stream, &c);
+    if (rc != TPL_OK) return rc;
+    if (!packed || !act || !al16(act) || (!partials && !y && !y32)) return TPL_EINVAL;
+    const bool resid = (p->d.flags & TPL_RESIDUAL) != 0;
+    if (resid && !partials && !h) return TPL_EINVAL;
+    return run_down(c, static_cast<const char *>(packed), act, resid ? h : nullptr, 1, y, y32, partials);
+}
+
+int tpl_reduce_partials(tpl_plan *p, const float *P, const void *resid, int32_t resid_is_f32, int32_t B, float *out32,
+                        void *out_act, tpl_stream stream) {
+    if (!p || !P || B < 0 || (!out32 && !out_act)) return TPL_EINVAL;
+    if (B == 0) return TPL_OK;
+    return run_reduce(p, static_cast<cudaStream_t>(stream), P, resid, resid_is_f32 ? 1 : 0, B, out32, out_act);
+}
+
+int tpl_mlp_block(tpl_plan *p, const void *packed, const void *x, int32_t B, void *y, float *y32, void *ws,
+                  size_t ws_bytes, int32_t reduce_mode, tpl_stream stream) {
+    if (B == 0) return TPL_OK;
+    if (reduce_mode != TPL_REDUCE_FUSED && reduce_mode != TPL_REDUCE_SEPARATE) return TPL_EINVAL;
+    Ctx c;
+    int rc = make_ctx(p, ws, ws_bytes, B, 0, stream, &c);
+    if (rc != TPL_OK) return rc;
+    if (!packed || !x || !al16(x) || (!y && !y32)) return TPL_EINVAL;
+    const char *pk = static_cast<const char *>(packed);
+    const bool resid = (p->d.flags & TPL_RESIDUAL) != 0;
+    void *act = c.ws + c.L.act;
+    float *P = reinterpret_cast<float *>(c.ws + c.L.P);
+    rc = run_gu(c, pk, x, 1, act);
+    if (rc != TPL_OK) return rc;
+    if (reduce_mode == TPL_REDUCE_FUSED) return run_down(c, pk, act, resid ? x : nullptr, p->f32, y, y32, nullptr);
+    rc = run_down(c, pk, act, nullptr, 0, nullptr, nullptr, P);
+    if (rc != TPL_OK) return rc;
+    return run_reduce(p, c.st, P, resid ? x : nullptr, p->f32, B, y32, y);
+}
+
+int tpl_decode_layer(tpl_plan *p, const void *packed, const tpl_kv *kv, const void *x, int32_t B, int64_t S, void *y,
+                     float *y32, void *ws, size_t ws_bytes, int32_t reduce_mode, tpl_stream stream) {
+    if (B == 0) return TPL_OK;
+    if (reduce_mode != TPL_REDUCE_FUSED && reduce_mode != TPL_REDUCE_SEPARATE) return TPL_EINVAL;
+    Ctx c;
+    int rc = make_ctx(p, ws, ws_bytes, B, S, stream, &c);
+    if (rc != TPL_OK) return rc;
+    if (!packed || !x || !al16(x) || !al16(packed) || (!y && !y32)) return TPL_EINVAL;
+    if ((rc = check_kv(kv, B, S)) != TPL_OK) return rc;
+    return decode_layer(c, static_cast<const char *>(packed), kv, x, y, y32, reduce_mode);
+}
+
+int tpl_decode_stack(tpl_plan *p, const void *const *packed_per_layer, const tpl_kv *kv_per_layer, const void *x,
+                     int32_t B, int64_t S, void *y, float *y32, void *ws, size_t ws_bytes, int32_t reduce_mode,
+                     tpl_stream stream) {
+    if (B == 0) return TPL_OK;
+    if (reduce_mode != TPL_REDUCE_FUSED && reduce_mode != TPL_REDUCE_SEPARATE) return TPL_EINVAL;
+    Ctx c;
+    int rc = make_ctx(p, ws, ws_bytes, B, S, stream, &c);
+    if (rc != TPL_OK) return rc;
+    if (!packed_per_layer || !kv_per_layer || !x || !al16(x) || (!y && !y32)) return TPL_EINVAL;
+    const int L = p->d.n_layers;
+    for (int l = 0; l < L; ++l) {
+        if (!packed_per_layer[l] || !al16(packed_per_layer[l])) return TPL_EINVAL;
+        if ((rc = check_kv(&kv_per_layer[l], B, S)) != TPL_OK) return rc;
+    }
+    void *buf[2] = {c.ws + c.L.ybuf0, c.ws + c.L.ybuf1};
+    const void *cur = x;
+    for (int l = 0; l < L; ++l) {
+        const bool last = l == L - 1;
+        void *out = last ? y : buf[l & 1];
+        float *out32 = last ? y32 : nullptr;
+        if (last && !y) out = buf[l & 1];
+        rc = decode_layer(c, static_cast<const char *>(packed_per_layer[l]), &kv_per_layer[l], cur, out, out32,
+                          reduce_mode);
+        if (rc != TPL_OK) return rc;
+        cur = out;
+    }
+    return TPL_OK;
+}
+
+int tpl_prefill_layer(tpl_plan *p, const void *packed, const tpl_kv *kv, const void *x, int32_t T, void *y,
+                      float *y32, void *ws, size_t ws_bytes, int32_t reduce_mode, tpl_stream stream) {
+    (void)p; (void)packed; (void)kv; (void)x; (void)T; (void)y; (void)y32; (void)ws; (void)ws_bytes;
+    (void)reduce_mode; (void)stream;
+    return TPL_EUNSUPPORTED;
+}
+
+int tpl_last_device_error(const tpl_plan *p, tpl_stream stream) {
+    (void)p;
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return TPL_ECUDA;
+    unsigned v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_err_word, sizeof(v)) != cudaSuccess) return TPL_ECUDA;
+    if (v) {
+        const unsigned z = 0;
+        if (cudaMemcpyToSymbol(g_err_word, &z, sizeof(z)) != cudaSuccess) return TPL_ECUDA;
+        return TPL_EDEVICE;
+    }
+    return TPL_OK;
+}
+
+}  // extern "C"

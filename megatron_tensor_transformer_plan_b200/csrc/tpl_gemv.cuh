@@ -1,0 +1,443 @@
+// Matrix-vector kernels for the decode projections (B <= 16 tokens).
+//
+// One CTA per SM (512 threads).  The grid is rb row blocks x ksplit K-splits.
+// Inside a CTA the 16 warps form wk K-groups x wr row slots; a warp streams
+// 8-row groups of the weight matrix over its K-group's 128-column blocks with
+// 16-byte loads, double-buffered in registers, against the activation slice
+// the CTA staged (normalised, rounded to the activation type) in shared
+// memory.  Partial sums per (K-group, row, token) land in shared memory and
+// are added in a fixed order per segment (shard) at the end of each round of
+// row groups; split-K CTAs hand their per-segment partials to the last CTA of
+// the row block to arrive (an arrival counter, no waiting), which adds them
+// in order.  The per-segment sums p_s are the shard partials of the row-split
+// projections ("Tensor parallel scaling curves", "What tensor parallelism
+// actually splits"): the fused epilogue adds them in ascending shard order,
+// the separate mode writes them out for tpl_reduce_partials, which adds them
+// in the same order -- so both modes give identical bits.
+//
+// Inner product modes:
+//   MODE 0 -- bf16 weights on the tensor cores (mma.sync m16n8k16): the
+//             activation tile is the A operand (tokens as rows), 8 weight rows
+//             the B operand; the k index of each 16-wide step is permuted so
+//             that every lane's operands are 16-byte contiguous in memory.
+//   MODE 1 -- fp32 weights with fp32 FFMA (exact-arithmetic comparison mode).
+//   MODE 2 -- bf16 weights with FFMA on the CUDA cores (kept to measure
+//             against MODE 0).
+#pragma once
+
+#include "tpl_common.cuh"
+#include "tpl_internal.h"
+
+namespace tpl {
+
+enum { EPI_QKV = 0, EPI_GU = 1, EPI_ROW = 2, EPI_ROW_PARTIAL = 3 };
+
+struct GemvArgs {
+    const char *W;   // first weight block
+    int64_t blk_r;   // bytes between row blocks (column-parallel shards)
+    int64_t blk_s;   // bytes between K segments (row-parallel shards)
+    int rps;         // rows per row block
+    int ldw;         // elements per weight row inside a block
+    GemvGeom g;
+    int B;
+    const void *x;   // activation source [B][ldx]; column seg*Kseg + k
+    int x_f32, ldx;
+    int norm;
+    const float *gamma;
+    float eps;
+    int epi;
+    float *out32;
+    void *out_act;
+    int act_f32;
+    const void *resid;
+    int resid_f32;
+    float *partials;  // [nseg][B][N]
+    float *q;
+    __nv_bfloat16 *kc, *vc;
+    int nq, nq_s, nkv_s, hd, batch_cap;
+    int64_t S, seq_cap;
+    float *gp;
+    unsigned *tickets;
+};
+
+template <int MODE>
+struct GemvTraits;
+template <>
+struct GemvTraits<0> {  // bf16 weights, bf16 staged x, tensor cores
+    static constexpr int WES = 2, XES = 2, NBI = 2, LPM = 1;
+};
+template <>
+struct GemvTraits<1> {  // fp32 weights, fp32 staged x, FFMA
+    static constexpr int WES = 4, XES = 4, NBI = 1, LPM = 2;
+};
+template <>
+struct GemvTraits<2> {  // bf16 weights, bf16 staged x, FFMA
+    static constexpr int WES = 2, XES = 2, NBI = 2, LPM = 1;
+};
+
+// Segment sums and the final write for one (row, token).
+struct SegSums {
+    float p[8];
+};
+
+__device__ __forceinline__ void gemv_final_row(const GemvArgs &a, int row, int tok, const SegSums &ss) {
+    const int N = a.g.N, B = a.B;
+    if (a.epi == EPI_QKV) {
+        const float v = ss.p[0];
+        const int s = row / a.rps, l = row % a.rps;
+        const int qd = a.nq_s * a.hd, kd = a.nkv_s * a.hd;
+        if (l < qd) {
+            const int head = s * a.nq_s + l / a.hd, dim = l % a.hd;
+            a.q[((int64_t)tok * a.nq + head) * a.hd + dim] = v;
+        } else {
+            const bool isk = l < qd + kd;
+            const int ll = isk ? l - qd : l - qd - kd;
+            const int kvl = ll / a.hd, dim = ll % a.hd;
+            __nv_bfloat16 *c = isk ? a.kc : a.vc;
+            c[((((int64_t)s * a.batch_cap + tok) * a.nkv_s + kvl) * a.seq_cap + a.S) * a.hd + dim] =
+                __float2bfloat16_rn(v);
+        }
+    } else if (a.epi == EPI_ROW) {
+        float acc = ss.p[0];
+        for (int s = 1; s < a.g.nseg; ++s) acc = acc + ss.p[s];
+        if (a.resid) acc = load_act(a.resid, a.resid_f32, (int64_t)tok * N + row) + acc;
+        if (a.out32) a.out32[(int64_t)tok * N + row] = acc;
+        if (a.out_act) store_act(a.out_act, a.act_f32, (int64_t)tok * N + row, acc);
+    } else {  // EPI_ROW_PARTIAL
+        for (int s = 0; s < a.g.nseg; ++s) a.partials[((int64_t)s * B + tok) * N + row] = ss.p[s];
+    }
+}
+
+__device__ __forceinline__ void gemv_final_pair(const GemvArgs &a, int pair, int tok, float gsum, float usum) {
+    store_act(a.out_act, a.act_f32, (int64_t)tok * (a.g.N / 2) + pair, silu(gsum) * usum);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_constant__ GemvArgs a) {
+    using T = GemvTraits<MODE>;
+    extern __shared__ __align__(128) unsigned char smem[];
+    const GemvGeom &g = a.g;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int gid = lane >> 2, c = lane & 3;
+    const int B = a.B;
+    const int rb = blockIdx.x / g.ksplit, ks = blockIdx.x % g.ksplit;
+    const int rg0 = (int)((int64_t)rb * g.ng / g.rb), rg1 = (int)((int64_t)(rb + 1) * g.ng / g.rb);
+    const int kgl = warp % g.wk, wslot = warp / g.wk;
+
+    // K-group -> segment and block range.
+    const int KG = g.ksplit * g.wk;
+    const int kpseg = KG / g.nseg;
+    const int Gk = ks * g.wk + kgl;
+    const int seg = Gk / kpseg, piece = Gk % kpseg;
+    const int kb_lo = (int)((int64_t)piece * g.nb / kpseg), kb_hi = (int)((int64_t)(piece + 1) * g.nb / kpseg);
+    // CTA's staged span.
+    const int seg_lo = (ks * g.wk) / kpseg;
+    int cblk_lo = 0, nbc = g.nb;
+    if (g.ksplit > g.nseg) {
+        const int per = g.pieces, pi = ks % per;
+        cblk_lo = (int)((int64_t)pi * g.nb / per);
+        nbc = (int)((int64_t)(pi + 1) * g.nb / per) - cblk_lo;
+    }
+    const int kpc = g.wk / g.segs_per_cta;  // K-groups per segment inside the CTA
+
+    unsigned char *xs = smem;
+    float *part = reinterpret_cast<float *>(smem + (size_t)B * g.x_stride);
+    const int prows = g.wr * g.rgc * 8;  // rows per round
+    float *s_inv = part + (size_t)g.wk * prows * B;
+    int *s_flag = reinterpret_cast<int *>(s_inv + 16);
+
+    // Warp's work: row groups rg0 + wslot + k*wr, items of NBI blocks.
+    const int nrg_w = rg1 - rg0 > wslot ? (rg1 - rg0 - wslot + g.wr - 1) / g.wr : 0;
+    const int nblk = kb_hi - kb_lo;
+    const int nit = nblk > 0 ? (nblk + T::NBI - 1) / T::NBI : 1;
+    const int nitems = nrg_w * nit;
+
+    constexpr int NW = T::NBI * 4 * T::LPM;  // uint4 per item per lane
+    uint4 wa[NW], wb[NW];
+
+    auto load_item = [&](uint4 (&w)[NW], int f) {
+        const int k = f / nit, it = f % nit;
+        const int rg = rg0 + wslot + k * g.wr;
+        const int row = rg * 8 + gid;
+        const bool row_ok = row < g.N;
+        const char *rp = a.W + (int64_t)(row / a.rps) * a.blk_r + (int64_t)seg * a.blk_s +
+                         (int64_t)(row % a.rps) * a.ldw * T::WES;
+#pragma unroll
+        for (int bi = 0; bi < T::NBI; ++bi) {
+            const int blk = kb_lo + it * T::NBI + bi;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int col = blk * 128 + 32 * m + 8 * c;
+                const bool ok = row_ok && blk < kb_hi && col < g.Kseg;
+#pragma unroll
+                for (int l = 0; l < T::LPM; ++l) {
+                    w[(bi * 4 + m) * T::LPM + l] =
+                        ok ? ldg_stream(rp + (int64_t)col * T::WES + 16 * l) : make_uint4(0, 0, 0, 0);
+                }
+            }
+        }
+    };
+
+    // Issue the first weight loads before waiting on the previous kernel.
+    if (nitems > 0) load_item(wa, 0);
+    pdl_wait();
+    pdl_trigger();
+
+    // ---- stage the activation slice (normalised if requested) ----
+    if (a.norm) {
+        // inverse RMS over the full row of each token, fixed-order reduction
+        float *s_red = part;  // scratch, [16 warps][B]
+        for (int tok = 0; tok < B; ++tok) {
+            float ss = 0.f;
+            for (int i = tid * 8; i < a.ldx; i += kGemvThreads * 8) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    float v = load_act(a.x, a.x_f32, (int64_t)tok * a.ldx + i + e);
+                    ss += v * v;
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            if (lane == 0) s_red[warp * B + tok] = ss;
+        }
+        __syncthreads();
+        if (tid < B) {
+            float ss = 0.f;
+            for (int w = 0; w < kGemvWarps; ++w) ss += s_red[w * B + tid];
+            s_inv[tid] = 1.0f / sqrtf(ss / (float)a.ldx + a.eps);
+        }
+        __syncthreads();
+    }
+    {
+        const int chunks_per_tok = g.segs_per_cta * nbc * 16;  // 8-element chunks
+        for (int u = tid; u < B * chunks_per_tok; u += kGemvThreads) {
+            const int tok = u / chunks_per_tok, r = u % chunks_per_tok;
+            const int sl = r / (nbc * 16), rr = r % (nbc * 16);
+            const int blk = cblk_lo + rr / 16, j = rr % 16;
+            const int k = blk * 128 + j * 8;
+            const int sg = seg_lo + sl;
+            float v[8];
+            if (k < g.Kseg) {
+                const int64_t src = (int64_t)tok * a.ldx + (int64_t)sg * g.Kseg + k;
+                if (a.x_f32) {
+                    const float4 *p4 = reinterpret_cast<const float4 *>(static_cast<const float *>(a.x) + src);
+                    float4 x0 = p4[0], x1 = p4[1];
+                    v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w;
+                    v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
+                } else {
+                    uint4 r4 = *reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(a.x) + src);
+                    v[0] = bf16lo(r4.x); v[1] = bf16hi(r4.x); v[2] = bf16lo(r4.y); v[3] = bf16hi(r4.y);
+                    v[4] = bf16lo(r4.z); v[5] = bf16hi(r4.z); v[6] = bf16lo(r4.w); v[7] = bf16hi(r4.w);
+                }
+                if (a.norm) {
+                    const float inv = s_inv[tok];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) v[e] = v[e] * inv * (a.gamma ? a.gamma[k + e] : 1.0f);
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v[e] = 0.f;
+            }
+            unsigned char *dst = xs + (size_t)tok * g.x_stride + (size_t)((sl * nbc + (blk - cblk_lo)) * 128 + j * 8) * T::XES;
+            if (T::XES == 2) {
+                uint4 o;
+                o.x = pack_bf16x2(v[0], v[1]); o.y = pack_bf16x2(v[2], v[3]);
+                o.z = pack_bf16x2(v[4], v[5]); o.w = pack_bf16x2(v[6], v[7]);
+                *reinterpret_cast<uint4 *>(dst) = o;
+            } else {
+                reinterpret_cast<float4 *>(dst)[0] = make_float4(v[0], v[1], v[2], v[3]);
+                reinterpret_cast<float4 *>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
+            }
+        }
+    }
+    __syncthreads();
+
+    // ---- main loop ----
+    const int rg_cta = rg1 - rg0;
+    const int rounds = (((rg_cta + g.wr - 1) / g.wr) + g.rgc - 1) / g.rgc;
+    const int sl_mine = seg - seg_lo;  // this warp's segment inside the CTA
+    float acc[MODE == 0 ? 4 : 16];
+#pragma unroll
+    for (int i = 0; i < (MODE == 0 ? 4 : 16); ++i) acc[i] = 0.f;
+
+    int f = 0;
+    for (int r = 0; r < rounds; ++r) {
+        const int k_end = min((r + 1) * g.rgc, nrg_w);
+        const int f_end = k_end * nit;
+        for (; f < f_end; ++f) {
+            if (f + 1 < nitems) load_item(wb, f + 1);
+            const int k = f / nit, it = f % nit;
+#pragma unroll
+            for (int bi = 0; bi < T::NBI; ++bi) {
+                const int blk = kb_lo + it * T::NBI + bi;
+                if (blk < kb_hi) {
+                    const int xcol = (sl_mine * nbc + (blk - cblk_lo)) * 128;
+                    if constexpr (MODE == 0) {
+#pragma unroll
+                        for (int m = 0; m < 4; ++m) {
+                            const size_t off = (size_t)(xcol + 32 * m + 8 * c) * 2;
+                            uint4 xa = gid < B ? lds128(xs + (size_t)gid * g.x_stride + off) : make_uint4(0, 0, 0, 0);
+                            uint4 xb = gid + 8 < B ? lds128(xs + (size_t)(gid + 8) * g.x_stride + off)
+                                                   : make_uint4(0, 0, 0, 0);
+                            const uint4 w = wa[bi * 4 + m];
+                            mma_bf16_16816(acc, xa.x, xb.x, xa.y, xb.y, w.x, w.y);
+                            mma_bf16_16816(acc, xa.z, xb.z, xa.w, xb.w, w.z, w.w);
+                        }
+                    } else {
+#pragma unroll
+                        for (int m = 0; m < 4; ++m) {
+                            float wv[8];
+                            if constexpr (T::WES == 4) {
+                                const uint4 w0 = wa[(bi * 4 + m) * 2], w1 = wa[(bi * 4 + m) * 2 + 1];
+                                wv[0] = __uint_as_float(w0.x); wv[1] = __uint_as_float(w0.y);
+                                wv[2] = __uint_as_float(w0.z); wv[3] = __uint_as_float(w0.w);
+                                wv[4] = __uint_as_float(w1.x); wv[5] = __uint_as_float(w1.y);
+                                wv[6] = __uint_as_float(w1.z); wv[7] = __uint_as_float(w1.w);
+                            } else {
+                                const uint4 w0 = wa[bi * 4 + m];
+                                wv[0] = bf16lo(w0.x); wv[1] = bf16hi(w0.x); wv[2] = bf16lo(w0.y); wv[3] = bf16hi(w0.y);
+                                wv[4] = bf16lo(w0.z); wv[5] = bf16hi(w0.z); wv[6] = bf16lo(w0.w); wv[7] = bf16hi(w0.w);
+                            }
+                            const size_t off = (size_t)(xcol + 32 * m + 8 * c) * T::XES;
+#pragma unroll
+                            for (int tok = 0; tok < 16; ++tok) {
+                                if (tok < B) {
+                                    float xv[8];
+                                    const unsigned char *xp = xs + (size_t)tok * g.x_stride + off;
+                                    if constexpr (T::XES == 4) {
+                                        const uint4 x0 = lds128(xp), x1 = lds128(xp + 16);
+                                        xv[0] = __uint_as_float(x0.x); xv[1] = __uint_as_float(x0.y);
+                                        xv[2] = __uint_as_float(x0.z); xv[3] = __uint_as_float(x0.w);
+                                        xv[4] = __uint_as_float(x1.x); xv[5] = __uint_as_float(x1.y);
+                                        xv[6] = __uint_as_float(x1.z); xv[7] = __uint_as_float(x1.w);
+                                    } else {
+                                        const uint4 x0 = lds128(xp);
+                                        xv[0] = bf16lo(x0.x); xv[1] = bf16hi(x0.x); xv[2] = bf16lo(x0.y); xv[3] = bf16hi(x0.y);
+                                        xv[4] = bf16lo(x0.z); xv[5] = bf16hi(x0.z); xv[6] = bf16lo(x0.w); xv[7] = bf16hi(x0.w);
+                                    }
+                                    float s = acc[tok];
+#pragma unroll
+                                    for (int e = 0; e < 8; ++e) s = fmaf(wv[e], xv[e], s);
+                                    acc[tok] = s;
+                                }
+                            }
+                        }
+                    }
+                }
+            }
+            if (it == nit - 1) {
+                // row group done: write its partial sums for this K-group
+                const int pr = (wslot + (k - r * g.rgc) * g.wr) * 8;
+                float *pp = part + ((size_t)kgl * prows + pr) * B;
+                if constexpr (MODE == 0) {
+                    if (gid < B) {
+                        pp[(2 * c) * B + gid] = acc[0];
+                        pp[(2 * c + 1) * B + gid] = acc[1];
+                    }
+                    if (gid + 8 < B) {
+                        pp[(2 * c) * B + gid + 8] = acc[2];
+                        pp[(2 * c + 1) * B + gid + 8] = acc[3];
+                    }
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) acc[i] = 0.f;
+                } else {
+#pragma unroll
+                    for (int tok = 0; tok < 16; ++tok) {
+                        float s = acc[tok];
+                        s += __shfl_xor_sync(0xffffffffu, s, 1);
+                        s += __shfl_xor_sync(0xffffffffu, s, 2);
+                        if (tok < B && (tok & 3) == c) pp[gid * B + tok] = s;
+                        acc[tok] = 0.f;
+                    }
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < NW; ++i) wa[i] = wb[i];
+        }
+        __syncthreads();
+        // ---- round epilogue: fixed-order sums over K-groups per segment ----
+        const int rbase = (rg0 + r * g.wr * g.rgc) * 8;
+        const int nrows = min(prows, min(rg1 * 8, g.N) - rbase);
+        if (nrows > 0) {
+            const int pr_ok = g.ksplit == 1;
+            const int pc = g.ksplit > g.nseg ? ks % g.pieces : 0;
+            if (a.epi == EPI_GU) {
+                for (int u = tid; u < (nrows / 2) * B; u += kGemvThreads) {
+                    const int pp = u / B, tok = u % B;
+                    float gs = 0.f, us = 0.f;
+                    for (int kg = 0; kg < g.wk; ++kg) {
+                        gs += part[((size_t)kg * prows + 2 * pp) * B + tok];
+                        us += part[((size_t)kg * prows + 2 * pp + 1) * B + tok];
+                    }
+                    const int row = rbase + 2 * pp;
+                    if (pr_ok) {
+                        gemv_final_pair(a, row / 2, tok, gs, us);
+                    } else {
+                        a.gp[(((int64_t)0 * g.pieces + pc) * g.N + row) * B + tok] = gs;
+                        a.gp[(((int64_t)0 * g.pieces + pc) * g.N + row + 1) * B + tok] = us;
+                    }
+                }
+            } else {
+                for (int u = tid; u < nrows * B; u += kGemvThreads) {
+                    const int prow = u / B, tok = u % B;
+                    const int row = rbase + prow;
+                    SegSums ss;
+                    for (int sl = 0; sl < g.segs_per_cta; ++sl) {
+                        float s = 0.f;
+                        for (int kg = sl * kpc; kg < (sl + 1) * kpc; ++kg) s += part[((size_t)kg * prows + prow) * B + tok];
+                        ss.p[sl] = s;
+                    }
+                    if (pr_ok) {
+                        gemv_final_row(a, row, tok, ss);
+                    } else {
+                        for (int sl = 0; sl < g.segs_per_cta; ++sl)
+                            a.gp[(((int64_t)(seg_lo + sl) * g.pieces + pc) * g.N + row) * B + tok] = ss.p[sl];
+                    }
+                }
+            }
+        }
+        __syncthreads();
+    }
+
+    // ---- split-K: the last CTA of the row block adds the partials in order ----
+    if (g.ksplit > 1) {
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) {
+            const unsigned prev = atomicAdd(&a.tickets[rb], 1u);
+            *s_flag = prev == (unsigned)(g.ksplit - 1);
+            if (prev >= (unsigned)g.ksplit) record_error(1u);
+        }
+        __syncthreads();
+        if (*s_flag) {
+            __threadfence();
+            const int row0 = rg0 * 8, row1 = min(rg1 * 8, g.N);
+            if (a.epi == EPI_GU) {
+                for (int u = tid; u < ((row1 - row0) / 2) * B; u += kGemvThreads) {
+                    const int row = row0 + 2 * (u / B), tok = u % B;
+                    float gs = 0.f, us = 0.f;
+                    for (int pc = 0; pc < g.pieces; ++pc) {
+                        gs += __ldcg(&a.gp[(((int64_t)pc) * g.N + row) * B + tok]);
+                        us += __ldcg(&a.gp[(((int64_t)pc) * g.N + row + 1) * B + tok]);
+                    }
+                    gemv_final_pair(a, row / 2, tok, gs, us);
+                }
+            } else {
+                for (int u = tid; u < (row1 - row0) * B; u += kGemvThreads) {
+                    const int row = row0 + u / B, tok = u % B;
+                    SegSums ss;
+                    for (int s = 0; s < g.nseg; ++s) {
+                        float v = 0.f;
+                        for (int pc = 0; pc < g.pieces; ++pc)
+                            v += __ldcg(&a.gp[(((int64_t)s * g.pieces + pc) * g.N + row) * B + tok]);
+                        ss.p[s] = v;
+                    }
+                    gemv_final_row(a, row, tok, ss);
+                }
+            }
+            if (tid == 0) atomicExch(&a.tickets[rb], 0u);
+        }
+    }
+}
+
+}  // namespace tpl

@@ -1,0 +1,80 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <atomic>
+#include <cstddef>
+#include <cstdint>
+
+#include "tpl.h"
+
+#ifdef __CUDACC__
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#endif
+
+namespace tpl {
+
+constexpr int kGemvThreads = 512;          // 16 warps, one CTA per SM
+constexpr int kGemvWarps = kGemvThreads / 32;
+constexpr size_t kXSmemMax = 140 * 1024;   // activation slice staged per CTA
+constexpr size_t kPartSmemMax = 64 * 1024; // per-round partial sums
+constexpr int kAttnWarps = 4;              // warps per attention CTA
+constexpr int kAttnTargetWarps = 2048;     // key-range splits across all (b, kv head) pairs
+constexpr int kTicketSlots = 4096;         // uint32 arrival counters at the workspace start
+constexpr int kTicketAttn = 0;             // [0, 1024): attention pairs
+constexpr int kTicketGemv = 1024;          // + 512 * op
+constexpr int kMaxPairs = 1024;
+constexpr int kMaxRowBlocks = 512;
+
+enum GemvOp { OP_QKV = 0, OP_O = 1, OP_GU = 2, OP_DOWN = 3 };
+
+}  // namespace tpl
+
+struct tpl_plan {
+    tpl_dims d;
+    int t;
+    int nq_s, nkv_s, F_s, g, qkv_rows_s, esize;
+    bool f32;
+    int64_t blk_qkv, blk_o, blk_gu, blk_d;  // byte stride between shard blocks
+    int64_t off_qkv, off_o, off_gu, off_d, off_g1, off_g2, packed_bytes;
+    std::atomic<long long> reductions;
+    int gemv_mode;  // 0: tensor-core fragments (bf16); 1: fp32 FFMA; 2: bf16 FFMA
+};
+
+namespace tpl {
+
+// Geometry of one matrix-vector launch (rows split across CTAs, the K
+// dimension split into segments (shards), split-K CTAs and K-groups of warps).
+struct GemvGeom {
+    int N;       // output rows
+    int nseg;    // segments along K (t for row-parallel, 1 for column-parallel)
+    int Kseg;    // columns per segment
+    int nb;      // 128-column blocks per segment (last one ragged)
+    int ksplit;  // CTAs along K per row block
+    int wk, wr;  // warps: K-groups x row slots (wk * wr == 16)
+    int rb;      // row blocks (grid = rb * ksplit)
+    int ng;      // 8-row groups = ceil(N / 8)
+    int cta_blocks;   // 128-column blocks of x staged per CTA (per segment span)
+    int segs_per_cta; // whole segments per CTA (1 when a CTA holds part of one)
+    int pieces;       // partial results per segment across split-K CTAs
+    int rgc;          // row groups per warp per round
+    int x_stride;     // bytes per token row of staged x
+    size_t smem;      // dynamic shared memory bytes
+    size_t gp_floats; // cross-CTA partial floats (0 when ksplit == 1)
+};
+
+int gemv_geom(int N, int nseg, int Kseg, int B, int xbytes, int num_sms, GemvGeom *g);
+
+struct AttnGeom {
+    int pairs, nsplit, kps;  // pairs = B * n_kv; splits per pair; keys per split
+};
+void attn_geom(int B, int nkv, int64_t S, AttnGeom *a);
+
+struct WsLayout {
+    size_t tickets, q, o, h, act, ybuf0, ybuf1, P, part_o, part_ml, gp, total;
+};
+int ws_layout(const tpl_plan *p, int B, int64_t S, WsLayout *w);
+
+int num_sms_current();  // multiprocessor count of the current device (cached)
+
+}  // namespace tpl

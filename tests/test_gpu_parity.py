@@ -49,7 +49,7 @@ def _check_layer(L, ref_y, tr, mode_both=True):
 SMALL = [
     # H, nq, nkv, F, t, B, S, gamma_std
     (512, 8, 2, 1376, 2, 3, 37, 0.0),       # ragged batch, short cache
-    (256, 4, 4, 688, 4, 1, 0, 0.0),         # MHA (g = 1), S = 0: one key
+    (256, 4, 4, 704, 4, 1, 0, 0.0),         # MHA (g = 1), S = 0: one key
     (1024, 16, 8, 2816, 8, 16, 300, 0.02),  # B = 16, t = 8, non-unit gains
     (768, 12, 4, 1056, 4, 5, 129, 0.0),     # F/t = 264 (ragged 128-column block), g = 3
     (512, 16, 1, 512, 1, 2, 1000, 0.0),     # g = 16

@@ -213,15 +213,49 @@ int tpl_prefill_layer(tpl_plan *plan, const void *packed, const tpl_kv *kv, cons
 /* ---- the individual steps (each is one kernel launch, except where noted;
  *      the decode calls above are these in order) --------------------------- */
 
-/* Column-parallel QKV: q [B][n_q][d] fp32; k/v of the new token to slot S. */
+/* Column-parallel QKV: q [B][n_q][d] fp32; the new token's k/v go to cache
+ * slot S (bf16) and, when k_new/v_new are not NULL, also to k_new/v_new
+ * [B][n_kv][d] fp32 (both or neither). */
 int tpl_qkv(tpl_plan *plan, const void *packed, const tpl_kv *kv, const void *x, int32_t B,
-            int64_t S, float *q, void *ws, size_t ws_bytes, tpl_stream stream);
+            int64_t S, float *q, float *k_new, float *v_new, void *ws, size_t ws_bytes,
+            tpl_stream stream);
 
-/* Owned-head GQA decode attention over positions 0..S (split over the key
- * range, partial results combined in a fixed order).  o [B][n_q*d]
+/* Owned-head GQA decode attention over positions 0..S ("Tensor parallel
+ * scaling curves": local attention on owned heads).  The S cached keys are
+ * split over key ranges whose partial results are combined in a fixed
+ * order; the new token (position S) is taken from k_new/v_new [B][n_kv][d]
+ * fp32 when given (both or neither), else from cache slot S.  o [B][n_q*d]
  * activation type.  Uses the workspace for the split partials. */
-int tpl_attn_decode(tpl_plan *plan, const tpl_kv *kv, const float *q, int32_t B, int64_t S,
-                    void *o, void *ws, size_t ws_bytes, tpl_stream stream);
+int tpl_attn_decode(tpl_plan *plan, const tpl_kv *kv, const float *q, const float *k_new,
+                    const float *v_new, int32_t B, int64_t S, void *o, void *ws, size_t ws_bytes,
+                    tpl_stream stream);
+
+/* Allocation-free variant of tpl_attn_decode.  The pages have no counterpart
+ * for this call; it exists for callers that cannot allocate device memory
+ * themselves -- for example a plugin inside a host application whose memory
+ * manager owns the whole device budget, or a latency-critical serving loop
+ * that must never enter the allocator.  It takes no workspace: the split
+ * partials and arrival counters live in one array of fixed size,
+ * TPL_ATTN_STATIC_SCRATCH_BYTES, held in the library's static device memory
+ * on every device that loads the library, until the process exits.
+ *   - Same arguments and result as tpl_attn_decode, minus the workspace.
+ *   - Returns TPL_ENOMEM, before launching anything, when the problem needs
+ *     more scratch than that: the 256-byte-rounded sum of 4*pairs
+ *     (counters), 8*pairs*n*g and 512*pairs*n*g bytes, pairs = B*n_kv, n the
+ *     blocks per pair (a quarter of the key-range split count, which is
+ *     about 1024/pairs rounded up to a multiple of 4, with at least 128 keys
+ *     per split).
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - Every call uses the same array, and it keeps the previous call's
+ *     contents; the call clears the counters it needs on `stream` first.
+ *     Calls that may overlap on the GPU (other streams, other threads) race
+ *     on the array and must be serialised by the caller.
+ *   - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library
+ *     routine. */
+#define TPL_ATTN_STATIC_SCRATCH_BYTES (4u * 1024u * 1024u)
+int tpl_attn_decode_static(tpl_plan *plan, const tpl_kv *kv, const float *q, const float *k_new,
+                           const float *v_new, int32_t B, int64_t S, void *o, tpl_stream stream);
 
 /* Row-parallel O projection.  partials == NULL: fused, h = x + sum_s o_s
  * Wo[s]^T (fp32 [B][H]); partials != NULL: writes P[s] = o_s Wo[s]^T

@@ -1,14 +1,19 @@
 // Owned-head GQA decode attention ("Tensor parallel scaling curves", "What
 // tensor parallelism actually splits": attention runs on the heads a shard
 // owns, with no exchange).  One (shard, sequence, kv head) pair is split over
-// its S+1 keys into `nsplit` ranges; each warp handles one range with an
-// online softmax and writes (max, sum, unnormalised output); the last CTA of
-// the pair to arrive (an arrival counter, no waiting) combines the ranges in
-// ascending order.
+// its S cached keys into `nsplit` ranges; each warp handles one range with an
+// online softmax, the CTA's warps merge their (max, sum, unnormalised output)
+// in shared memory, and the last CTA of the pair to arrive (an arrival
+// counter, no waiting) combines the CTA partials in ascending order and then
+// the new token's key/value in fp32, as the
+// projection produced them (when they are not given, position S is read from
+// the cache like the others).
 //
 // Per warp, 16 keys per step on the tensor cores (mma.sync m16n8k16, bf16):
-//   S = Q K^T  -- A = the g query heads of the kv head (rows, zero-padded to
-//                 16), B = 8 keys; the head_dim index of each 16-wide step is
+//   S = Q K^T  -- A = the g query heads of the kv head (rows), B = 8 keys;
+//                 q and P are each carried as two bf16 parts (hi + lo), in
+//                 the otherwise-empty rows 8-15 when g <= 8; the head_dim
+//                 index of each 16-wide step is
 //                 permuted so that a lane's K operands are the 64 contiguous
 //                 bytes K[key][32m + 8c .. +8), m = 0..3;
 //   O += P V   -- A = P from the S accumulators (register reuse), B = V with
@@ -28,16 +33,18 @@ struct AttnArgs {
     int64_t seq_cap;
     int batch_cap;
     int B, nq, nkv_s, g;
-    int64_t keys;  // S + 1
+    int64_t keys;  // keys covered by the splits: S (new key given separately) or S + 1
+    const float *k_new, *v_new;  // [B][n_kv][128] fp32 of the new token, or NULL
     int nsplit, kps;
     float scale_log2;  // log2(e) / sqrt(head_dim)
-    float *part_o;     // [pairs][nsplit][g][128]
-    float *part_ml;    // [pairs][nsplit][g][2]
+    float *part_o;     // [pairs][CTAs per pair][g][128]
+    float *part_ml;    // [pairs][CTAs per pair][g][2]
     unsigned *tickets; // [pairs]
     void *o;           // [B][nq*128] activation type
     int o_f32;
 };
 
+template <bool PACKED>  // PACKED: g <= 8, q/P low parts in rows 8-15
 __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const __grid_constant__ AttnArgs a) {
     constexpr int D = 128;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -59,33 +66,33 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const __gr
     pdl_wait();
     pdl_trigger();
 
-    // Q fragments: rows gid (and gid+8) = query heads j*g + row, bf16.
-    uint32_t qa[16], qb[16];  // [m*4 + {0..3}]: bf16x2 of q cols 32m+8c+{0,1},{2,3},{4,5},{6,7}
+    // Q operands.  Each query value is carried as a bf16 pair hi + lo
+    // (lo = q - hi), so the logits keep ~16 mantissa bits.  With g <= 8 the
+    // hi parts fill A rows 0-7 and the lo parts rows 8-15 of the same mma
+    // (the rows that would otherwise be zero padding); with g > 8 rows 0-15
+    // are heads and hi/lo take two mma.
+    constexpr bool packed_rows = PACKED;
+    uint32_t qh0[16], ql0[16], qh1[16], ql1[16];  // [m*4 + i]: cols 32m+8c+2i, +1
 #pragma unroll
-    for (int i = 0; i < 16; ++i) { qa[i] = 0u; qb[i] = 0u; }
-    if (gid < a.g) {
-        const float *qp = a.q + ((int64_t)b * a.nq + (int64_t)j * a.g + gid) * D;
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const float4 x0 = *reinterpret_cast<const float4 *>(qp + 32 * m + 8 * c);
-            const float4 x1 = *reinterpret_cast<const float4 *>(qp + 32 * m + 8 * c + 4);
-            qa[m * 4 + 0] = pack_bf16x2(x0.x, x0.y);
-            qa[m * 4 + 1] = pack_bf16x2(x0.z, x0.w);
-            qa[m * 4 + 2] = pack_bf16x2(x1.x, x1.y);
-            qa[m * 4 + 3] = pack_bf16x2(x1.z, x1.w);
-        }
-    }
-    if (gid + 8 < a.g) {
-        const float *qp = a.q + ((int64_t)b * a.nq + (int64_t)j * a.g + gid + 8) * D;
+    for (int i = 0; i < 16; ++i) qh0[i] = ql0[i] = qh1[i] = ql1[i] = 0u;
+    auto load_q = [&](int row, uint32_t *hi, uint32_t *lo) {
+        const float *qp = a.q + ((int64_t)b * a.nq + (int64_t)j * a.g + row) * D;
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
             const float4 x0 = *reinterpret_cast<const float4 *>(qp + 32 * m + 8 * c);
             const float4 x1 = *reinterpret_cast<const float4 *>(qp + 32 * m + 8 * c + 4);
-            qb[m * 4 + 0] = pack_bf16x2(x0.x, x0.y);
-            qb[m * 4 + 1] = pack_bf16x2(x0.z, x0.w);
-            qb[m * 4 + 2] = pack_bf16x2(x1.x, x1.y);
-            qb[m * 4 + 3] = pack_bf16x2(x1.z, x1.w);
+            const float v[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint32_t h = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+                hi[m * 4 + i] = h;
+                lo[m * 4 + i] = pack_bf16x2(v[2 * i] - bf16lo(h), v[2 * i + 1] - bf16hi(h));
+            }
         }
+    };
+    if (gid < a.g) load_q(gid, qh0, ql0);
+    if constexpr (!PACKED) {
+        if (gid + 8 < a.g) load_q(gid + 8, qh1, ql1);
     }
 
     float o[16][4];
@@ -118,33 +125,55 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const __gr
                 vd[h] = kd < k1 ? ldg_stream(Vp + kd * D + col) : make_uint4(0, 0, 0, 0);
             }
         }
-        // ---- scores ----
+        // ---- scores: s0 keys kb+2c, +1 (tile 0), s1 keys kb+8+2c, +1 (tile 1) ----
         float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+        if constexpr (PACKED) {
+            // rows gid: hi . K, rows gid+8: lo . K (same head)
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            mma_bf16_16816(s0, qa[m * 4 + 0], qb[m * 4 + 0], qa[m * 4 + 1], qb[m * 4 + 1], kt0[m].x, kt0[m].y);
-            mma_bf16_16816(s0, qa[m * 4 + 2], qb[m * 4 + 2], qa[m * 4 + 3], qb[m * 4 + 3], kt0[m].z, kt0[m].w);
-            mma_bf16_16816(s1, qa[m * 4 + 0], qb[m * 4 + 0], qa[m * 4 + 1], qb[m * 4 + 1], kt1[m].x, kt1[m].y);
-            mma_bf16_16816(s1, qa[m * 4 + 2], qb[m * 4 + 2], qa[m * 4 + 3], qb[m * 4 + 3], kt1[m].z, kt1[m].w);
+            for (int m = 0; m < 4; ++m) {
+                mma_bf16_16816(s0, qh0[m * 4 + 0], ql0[m * 4 + 0], qh0[m * 4 + 1], ql0[m * 4 + 1], kt0[m].x, kt0[m].y);
+                mma_bf16_16816(s0, qh0[m * 4 + 2], ql0[m * 4 + 2], qh0[m * 4 + 3], ql0[m * 4 + 3], kt0[m].z, kt0[m].w);
+                mma_bf16_16816(s1, qh0[m * 4 + 0], ql0[m * 4 + 0], qh0[m * 4 + 1], ql0[m * 4 + 1], kt1[m].x, kt1[m].y);
+                mma_bf16_16816(s1, qh0[m * 4 + 2], ql0[m * 4 + 2], qh0[m * 4 + 3], ql0[m * 4 + 3], kt1[m].z, kt1[m].w);
+            }
+            s0[0] += s0[2];
+            s0[1] += s0[3];
+            s1[0] += s1[2];
+            s1[1] += s1[3];
+            s0[2] = s0[0];
+            s0[3] = s0[1];
+            s1[2] = s1[0];
+            s1[3] = s1[1];
+        } else {
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                mma_bf16_16816(s0, qh0[m * 4 + 0], qh1[m * 4 + 0], qh0[m * 4 + 1], qh1[m * 4 + 1], kt0[m].x, kt0[m].y);
+                mma_bf16_16816(s0, qh0[m * 4 + 2], qh1[m * 4 + 2], qh0[m * 4 + 3], qh1[m * 4 + 3], kt0[m].z, kt0[m].w);
+                mma_bf16_16816(s1, qh0[m * 4 + 0], qh1[m * 4 + 0], qh0[m * 4 + 1], qh1[m * 4 + 1], kt1[m].x, kt1[m].y);
+                mma_bf16_16816(s1, qh0[m * 4 + 2], qh1[m * 4 + 2], qh0[m * 4 + 3], qh1[m * 4 + 3], kt1[m].z, kt1[m].w);
+                mma_bf16_16816(s0, ql0[m * 4 + 0], ql1[m * 4 + 0], ql0[m * 4 + 1], ql1[m * 4 + 1], kt0[m].x, kt0[m].y);
+                mma_bf16_16816(s0, ql0[m * 4 + 2], ql1[m * 4 + 2], ql0[m * 4 + 3], ql1[m * 4 + 3], kt0[m].z, kt0[m].w);
+                mma_bf16_16816(s1, ql0[m * 4 + 0], ql1[m * 4 + 0], ql0[m * 4 + 1], ql1[m * 4 + 1], kt1[m].x, kt1[m].y);
+                mma_bf16_16816(s1, ql0[m * 4 + 2], ql1[m * 4 + 2], ql0[m * 4 + 3], ql1[m * 4 + 3], kt1[m].z, kt1[m].w);
+            }
         }
-        // s0: [row gid][keys kb+2c, +1], [row gid+8][...]; s1: keys kb+8+2c, +1
         const int64_t kk = kb + 2 * c;
-        float x0 = kk < k1 ? s0[0] * a.scale_log2 : -INFINITY;
-        float x1 = kk + 1 < k1 ? s0[1] * a.scale_log2 : -INFINITY;
-        float x2 = kk + 8 < k1 ? s1[0] * a.scale_log2 : -INFINITY;
-        float x3 = kk + 9 < k1 ? s1[1] * a.scale_log2 : -INFINITY;
-        float y0 = kk < k1 ? s0[2] * a.scale_log2 : -INFINITY;
-        float y1 = kk + 1 < k1 ? s0[3] * a.scale_log2 : -INFINITY;
-        float y2 = kk + 8 < k1 ? s1[2] * a.scale_log2 : -INFINITY;
-        float y3 = kk + 9 < k1 ? s1[3] * a.scale_log2 : -INFINITY;
+        const float x0 = kk < k1 ? s0[0] * a.scale_log2 : -INFINITY;
+        const float x1 = kk + 1 < k1 ? s0[1] * a.scale_log2 : -INFINITY;
+        const float x2 = kk + 8 < k1 ? s1[0] * a.scale_log2 : -INFINITY;
+        const float x3 = kk + 9 < k1 ? s1[1] * a.scale_log2 : -INFINITY;
+        const float y0 = kk < k1 ? s0[2] * a.scale_log2 : -INFINITY;
+        const float y1 = kk + 1 < k1 ? s0[3] * a.scale_log2 : -INFINITY;
+        const float y2 = kk + 8 < k1 ? s1[2] * a.scale_log2 : -INFINITY;
+        const float y3 = kk + 9 < k1 ? s1[3] * a.scale_log2 : -INFINITY;
         float mxa = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
         float mxb = fmaxf(fmaxf(y0, y1), fmaxf(y2, y3));
         mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 1));
         mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 2));
         mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 1));
         mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 2));
+        // finite: the first key of every step is in range
         const float mna = fmaxf(m_a, mxa), mnb = fmaxf(m_b, mxb);
-        // mna is finite: the first key of every step is in range
         const float alpha_a = exp2f(m_a - mna), alpha_b = exp2f(m_b - mnb);
         m_a = mna;
         m_b = mnb;
@@ -159,8 +188,15 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const __gr
             o[t][2] *= alpha_b;
             o[t][3] *= alpha_b;
         }
-        const uint32_t pa0 = pack_bf16x2(p0, p1), pa1 = pack_bf16x2(r0, r1);
-        const uint32_t pa2 = pack_bf16x2(p2, p3), pa3 = pack_bf16x2(r2, r3);
+        // P as bf16 hi + lo.  Packed rows: rows gid carry P_hi, rows gid+8
+        // P_lo of the same head (summed at the end).  Otherwise rows are
+        // heads and P_lo is a second mma into the same accumulator.
+        const uint32_t ph0 = pack_bf16x2(p0, p1), ph2 = pack_bf16x2(p2, p3);
+        const uint32_t pl0 = pack_bf16x2(p0 - bf16lo(ph0), p1 - bf16hi(ph0));
+        const uint32_t pl2 = pack_bf16x2(p2 - bf16lo(ph2), p3 - bf16hi(ph2));
+        const uint32_t rh0 = pack_bf16x2(r0, r1), rh2 = pack_bf16x2(r2, r3);
+        const uint32_t rl0 = pack_bf16x2(r0 - bf16lo(rh0), r1 - bf16hi(rh0));
+        const uint32_t rl2 = pack_bf16x2(r2 - bf16lo(rh2), r3 - bf16hi(rh2));
         // ---- O += P V over 16 output tiles (head_dim 16n + t) ----
 #pragma unroll
         for (int t = 0; t < 16; ++t) {
@@ -170,68 +206,138 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const __gr
             const uint32_t wb_ = comp == 0 ? vb[h].x : comp == 1 ? vb[h].y : comp == 2 ? vb[h].z : vb[h].w;
             const uint32_t wc_ = comp == 0 ? vc2[h].x : comp == 1 ? vc2[h].y : comp == 2 ? vc2[h].z : vc2[h].w;
             const uint32_t wd_ = comp == 0 ? vd[h].x : comp == 1 ? vd[h].y : comp == 2 ? vd[h].z : vd[h].w;
-            mma_bf16_16816(o[t], pa0, pa1, pa2, pa3, prmt(wa_, wb_, sel), prmt(wc_, wd_, sel));
+            const uint32_t vb0 = prmt(wa_, wb_, sel), vb1 = prmt(wc_, wd_, sel);
+            if constexpr (PACKED) {
+                mma_bf16_16816(o[t], ph0, pl0, ph2, pl2, vb0, vb1);
+            } else {
+                mma_bf16_16816(o[t], ph0, rh0, ph2, rh2, vb0, vb1);
+                mma_bf16_16816(o[t], pl0, rl0, pl2, rl2, vb0, vb1);
+            }
+        }
+    }
+    if constexpr (PACKED) {
+        // rows gid+8 held the P_lo . V half of the same head
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+            o[t][0] += o[t][2];
+            o[t][1] += o[t][3];
         }
     }
 
-    // ---- write this split's partial result ----
+    // ---- combine the CTA's warps in shared memory (ascending warp order) ----
     l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
     l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
     l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
     l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
-    const int64_t pbase = ((int64_t)pair * a.nsplit + split) * a.g;
+    __shared__ float s_o[kAttnWarps][16][D];   // unnormalised outputs per warp and head
+    __shared__ float s_ml[kAttnWarps][16][2];  // (max, sum) per warp and head
     // o[t][0] -> (row gid, dim 32c + t); o[t][1] -> (row gid, dim 32c + 16 + t); [2],[3]: row gid+8
     if (gid < a.g) {
-        float *dst = a.part_o + (pbase + gid) * D + 32 * c;
 #pragma unroll
-        for (int t = 0; t < 16; t += 4) {
-            *reinterpret_cast<float4 *>(dst + t) = make_float4(o[t][0], o[t + 1][0], o[t + 2][0], o[t + 3][0]);
-            *reinterpret_cast<float4 *>(dst + 16 + t) = make_float4(o[t][1], o[t + 1][1], o[t + 2][1], o[t + 3][1]);
+        for (int t = 0; t < 16; ++t) {
+            s_o[warp][gid][32 * c + t] = o[t][0];
+            s_o[warp][gid][32 * c + 16 + t] = o[t][1];
         }
         if (c == 0) {
-            a.part_ml[(pbase + gid) * 2 + 0] = m_a;
-            a.part_ml[(pbase + gid) * 2 + 1] = l_a;
+            s_ml[warp][gid][0] = m_a;
+            s_ml[warp][gid][1] = l_a;
         }
     }
-    if (gid + 8 < a.g) {
-        float *dst = a.part_o + (pbase + gid + 8) * D + 32 * c;
+    if (!packed_rows && gid + 8 < a.g) {
 #pragma unroll
-        for (int t = 0; t < 16; t += 4) {
-            *reinterpret_cast<float4 *>(dst + t) = make_float4(o[t][2], o[t + 1][2], o[t + 2][2], o[t + 3][2]);
-            *reinterpret_cast<float4 *>(dst + 16 + t) = make_float4(o[t][3], o[t + 1][3], o[t + 2][3], o[t + 3][3]);
+        for (int t = 0; t < 16; ++t) {
+            s_o[warp][gid + 8][32 * c + t] = o[t][2];
+            s_o[warp][gid + 8][32 * c + 16 + t] = o[t][3];
         }
         if (c == 0) {
-            a.part_ml[(pbase + gid + 8) * 2 + 0] = m_b;
-            a.part_ml[(pbase + gid + 8) * 2 + 1] = l_b;
+            s_ml[warp][gid + 8][0] = m_b;
+            s_ml[warp][gid + 8][1] = l_b;
+        }
+    }
+    __syncthreads();
+    const int dim = threadIdx.x;  // 128 threads, one head_dim column each
+    const int cpp_ = cpp;
+    const int64_t cbase = ((int64_t)pair * cpp_ + chunk) * a.g;  // this CTA's partial
+    for (int hrow = 0; hrow < a.g; ++hrow) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, s_ml[w][hrow][0]);
+        float num = 0.f, den = 0.f;
+#pragma unroll
+        for (int w = 0; w < kAttnWarps; ++w) {
+            const float mi = s_ml[w][hrow][0];
+            const float wt = mi == -INFINITY ? 0.f : exp2f(mi - M);
+            num += wt * s_o[w][hrow][dim];
+            den += wt * s_ml[w][hrow][1];
+        }
+        a.part_o[(cbase + hrow) * D + dim] = num;
+        if (dim == 0) {
+            a.part_ml[(cbase + hrow) * 2 + 0] = M;
+            a.part_ml[(cbase + hrow) * 2 + 1] = den;
         }
     }
 
-    // ---- the last CTA of the pair combines all splits in ascending order ----
+    // ---- the last CTA of the pair combines the CTA partials in ascending order ----
     __shared__ int s_last;
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) {
         const unsigned prev = atomicAdd(&a.tickets[pair], 1u);
-        s_last = prev == (unsigned)(cpp - 1);
-        if (prev >= (unsigned)cpp) record_error(2u);
+        s_last = prev == (unsigned)(cpp_ - 1);
+        if (prev >= (unsigned)cpp_) record_error(2u);
     }
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    const int dim = threadIdx.x;  // 128 threads, one head_dim column each
-    for (int hrow = 0; hrow < a.g; ++hrow) {
-        float M = -INFINITY;
-        for (int sp = 0; sp < a.nsplit; ++sp)
-            M = fmaxf(M, __ldcg(&a.part_ml[(((int64_t)pair * a.nsplit + sp) * a.g + hrow) * 2]));
-        float num = 0.f, den = 0.f;
-        for (int sp = 0; sp < a.nsplit; ++sp) {
-            const int64_t pb = ((int64_t)pair * a.nsplit + sp) * a.g + hrow;
-            const float mi = __ldcg(&a.part_ml[pb * 2]);
-            const float w = mi == -INFINITY ? 0.f : exp2f(mi - M);
-            num += w * __ldcg(&a.part_o[pb * D + dim]);
-            den += w * __ldcg(&a.part_ml[pb * 2 + 1]);
+    // stage every CTA partial's (max, sum) for this pair
+    __shared__ float s_w[64][16];  // weights exp2(m_i - M) per CTA partial and head
+    __shared__ float s_M[16], s_den[16], s_new[16];
+    const bool has_new = a.k_new != nullptr;
+    float *s_mlp = &s_o[0][0][0];  // reuse: [cpp][g][2] (cpp <= 64)
+    for (int i = threadIdx.x; i < cpp_ * a.g * 2; i += blockDim.x)
+        s_mlp[i] = __ldcg(&a.part_ml[(int64_t)pair * cpp_ * a.g * 2 + i]);
+    if (has_new) {
+        // logits of the new token for the g heads, fp32, fixed-order reduction
+        __shared__ float s_red[kAttnWarps][16];
+        const float kd = a.k_new[((int64_t)b * (a.nq / a.g) + j) * D + dim];
+        for (int hrow = 0; hrow < a.g; ++hrow) {
+            float v = a.q[((int64_t)b * a.nq + (int64_t)j * a.g + hrow) * D + dim] * kd;
+#pragma unroll
+            for (int o2 = 16; o2 > 0; o2 >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o2);
+            if (lane == 0) s_red[warp][hrow] = v;
         }
-        store_act(a.o, a.o_f32, ((int64_t)b * a.nq + (int64_t)j * a.g + hrow) * D + dim, num / den);
+        __syncthreads();
+        if (threadIdx.x < a.g) {
+            float v = 0.f;
+#pragma unroll
+            for (int w = 0; w < kAttnWarps; ++w) v += s_red[w][threadIdx.x];
+            s_new[threadIdx.x] = v * a.scale_log2;
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < a.g) {
+        const int hrow = threadIdx.x;
+        float M = has_new ? s_new[hrow] : -INFINITY;
+        for (int i = 0; i < cpp_; ++i) M = fmaxf(M, s_mlp[(i * a.g + hrow) * 2]);
+        float den = 0.f;
+        for (int i = 0; i < cpp_; ++i) {
+            const float mi = s_mlp[(i * a.g + hrow) * 2];
+            const float wt = mi == -INFINITY ? 0.f : exp2f(mi - M);
+            s_w[i][hrow] = wt;
+            den += wt * s_mlp[(i * a.g + hrow) * 2 + 1];
+        }
+        if (has_new) den += exp2f(s_new[hrow] - M);
+        s_M[hrow] = M;
+        s_den[hrow] = den;
+    }
+    __syncthreads();
+    for (int hrow = 0; hrow < a.g; ++hrow) {
+        float num = 0.f;
+        const float *po = a.part_o + ((int64_t)pair * cpp_ * a.g + hrow) * D + dim;
+#pragma unroll 8
+        for (int i = 0; i < cpp_; ++i) num += s_w[i][hrow] * __ldcg(po + (int64_t)i * a.g * D);
+        if (has_new) num += exp2f(s_new[hrow] - s_M[hrow]) * a.v_new[((int64_t)b * (a.nq / a.g) + j) * D + dim];
+        store_act(a.o, a.o_f32, ((int64_t)b * a.nq + (int64_t)j * a.g + hrow) * D + dim, num / s_den[hrow]);
     }
     if (threadIdx.x == 0) atomicExch(&a.tickets[pair], 0u);
 }

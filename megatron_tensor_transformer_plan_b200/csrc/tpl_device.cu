@@ -55,7 +55,7 @@ cudaError_t launch_pdl(void (*kern)(KA...), int grid, int block, size_t smem, cu
     return cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...);
 }
 
-bool g_attr_done[64][3];
+bool g_attr_done[64][4];
 
 int prepare_gemv(int mode) {
     int dev = 0;
@@ -65,7 +65,8 @@ int prepare_gemv(int mode) {
         const int maxb = 227 * 1024;
         if (mode == 0) e = cudaFuncSetAttribute(gemv_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxb);
         else if (mode == 1) e = cudaFuncSetAttribute(gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxb);
-        else e = cudaFuncSetAttribute(gemv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxb);
+        else if (mode == 2) e = cudaFuncSetAttribute(gemv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxb);
+        else e = cudaFuncSetAttribute(gemv_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxb);
         if (e != cudaSuccess) return TPL_ECUDA;
         g_attr_done[dev][mode] = true;
     }
@@ -109,9 +110,11 @@ int gemv_launch(Ctx &c, GemvArgs &a, int N, int nseg, int Kseg, int op) {
     tpl_plan *p = c.p;
     const int sms = num_sms_current();
     if (sms <= 0) return TPL_ECUDA;
-    int rc = gemv_geom(N, nseg, Kseg, c.B, p->f32 ? 4 : 2, sms, &a.g);
+    // The Q projection feeds a softmax and gate/up feeds SwiGLU: carry their
+    // normalised activations as bf16 hi + lo.
+    const int mode = p->f32 ? 1 : (p->gemv_mode == 2 ? 2 : ((op == OP_QKV || op == OP_GU) ? 3 : 0));
+    int rc = gemv_geom(N, nseg, Kseg, c.B, p->f32 ? 4 : 2, sms, &a.g, mode == 3 ? 2 : 1);
     if (rc != TPL_OK) return rc;
-    const int mode = p->f32 ? 1 : (p->gemv_mode == 2 ? 2 : 0);
     rc = prepare_gemv(mode);
     if (rc != TPL_OK) return rc;
     a.B = c.B;
@@ -121,7 +124,8 @@ int gemv_launch(Ctx &c, GemvArgs &a, int N, int nseg, int Kseg, int op) {
     cudaError_t e;
     if (mode == 0) e = launch_pdl(gemv_kernel<0>, grid, kGemvThreads, a.g.smem, c.st, a);
     else if (mode == 1) e = launch_pdl(gemv_kernel<1>, grid, kGemvThreads, a.g.smem, c.st, a);
-    else e = launch_pdl(gemv_kernel<2>, grid, kGemvThreads, a.g.smem, c.st, a);
+    else if (mode == 2) e = launch_pdl(gemv_kernel<2>, grid, kGemvThreads, a.g.smem, c.st, a);
+    else e = launch_pdl(gemv_kernel<3>, grid, kGemvThreads, a.g.smem, c.st, a);
     return cuda_rc(e);
 }
 
@@ -134,7 +138,7 @@ GemvArgs base_args(const tpl_plan *p) {
     return a;
 }
 
-int run_qkv(Ctx &c, const char *packed, const tpl_kv *kv, const void *x, float *q) {
+int run_qkv(Ctx &c, const char *packed, const tpl_kv *kv, const void *x, float *q, float *knew, float *vnew) {
     tpl_plan *p = c.p;
     GemvArgs a = base_args(p);
     a.W = packed + p->off_qkv;
@@ -148,6 +152,8 @@ int run_qkv(Ctx &c, const char *packed, const tpl_kv *kv, const void *x, float *
     a.gamma = reinterpret_cast<const float *>(packed + p->off_g1);
     a.epi = EPI_QKV;
     a.q = q;
+    a.knew = knew;
+    a.vnew = vnew;
     a.kc = static_cast<__nv_bfloat16 *>(kv->k);
     a.vc = static_cast<__nv_bfloat16 *>(kv->v);
     a.nq = p->d.n_q_heads;
@@ -159,10 +165,11 @@ int run_qkv(Ctx &c, const char *packed, const tpl_kv *kv, const void *x, float *
     return gemv_launch(c, a, p->t * p->qkv_rows_s, 1, p->d.hidden, OP_QKV);
 }
 
-int run_attn(Ctx &c, const tpl_kv *kv, const float *q, void *o) {
+int run_attn(Ctx &c, const tpl_kv *kv, const float *q, const float *knew, const float *vnew, void *o) {
     tpl_plan *p = c.p;
+    const int64_t keys = knew ? c.S : c.S + 1;
     AttnGeom g;
-    attn_geom(c.B, p->d.n_kv_heads, c.S, &g);
+    attn_geom(c.B, p->d.n_kv_heads, keys, &g);
     if (g.pairs > kMaxPairs) return TPL_EUNSUPPORTED;
     AttnArgs a;
     std::memset(&a, 0, sizeof(a));
@@ -175,7 +182,9 @@ int run_attn(Ctx &c, const tpl_kv *kv, const float *q, void *o) {
     a.nq = p->d.n_q_heads;
     a.nkv_s = p->nkv_s;
     a.g = p->g;
-    a.keys = c.S + 1;
+    a.keys = keys;
+    a.k_new = knew;
+    a.v_new = vnew;
     a.nsplit = g.nsplit;
     a.kps = g.kps;
     a.scale_log2 = 1.4426950408889634f / sqrtf((float)p->d.head_dim);
@@ -185,7 +194,8 @@ int run_attn(Ctx &c, const tpl_kv *kv, const float *q, void *o) {
     a.o = o;
     a.o_f32 = p->f32;
     const int grid = g.pairs * (g.nsplit / kAttnWarps);
-    return cuda_rc(launch_pdl(attn_decode_kernel, grid, kAttnWarps * 32, 0, c.st, a));
+    return cuda_rc(p->g <= 8 ? launch_pdl(attn_decode_kernel<true>, grid, kAttnWarps * 32, 0, c.st, a)
+                              : launch_pdl(attn_decode_kernel<false>, grid, kAttnWarps * 32, 0, c.st, a));
 }
 
 // Row-parallel O projection: fused (partials == NULL) or partial output.
@@ -275,8 +285,10 @@ int decode_layer(Ctx &c, const char *packed, const tpl_kv *kv, const void *x, vo
     float *h = reinterpret_cast<float *>(c.ws + c.L.h);
     void *act = c.ws + c.L.act;
     float *P = reinterpret_cast<float *>(c.ws + c.L.P);
-    int rc = run_qkv(c, packed, kv, x, q);
-    if (rc == TPL_OK) rc = run_attn(c, kv, q, o);
+    float *knew = reinterpret_cast<float *>(c.ws + c.L.knew);
+    float *vnew = reinterpret_cast<float *>(c.ws + c.L.vnew);
+    int rc = run_qkv(c, packed, kv, x, q, knew, vnew);
+    if (rc == TPL_OK) rc = run_attn(c, kv, q, knew, vnew, o);
     if (rc == TPL_OK) {
         if (mode == TPL_REDUCE_FUSED) {
             rc = run_o(c, packed, o, resid ? x : nullptr, h, nullptr);
@@ -378,25 +390,26 @@ int tpl_pack_kv(const tpl_plan *p, const void *unsharded, void *sharded, int32_t
 }
 
 int tpl_qkv(tpl_plan *p, const void *packed, const tpl_kv *kv, const void *x, int32_t B, int64_t S, float *q,
-            void *ws, size_t ws_bytes, tpl_stream stream) {
+            float *k_new, float *v_new, void *ws, size_t ws_bytes, tpl_stream stream) {
     if (B == 0) return TPL_OK;
     Ctx c;
     int rc = make_ctx(p, ws, ws_bytes, B, S, stream, &c);
     if (rc != TPL_OK) return rc;
     if (!packed || !x || !q || !al16(x) || !al16(packed)) return TPL_EINVAL;
     if ((rc = check_kv(kv, B, S)) != TPL_OK) return rc;
-    return run_qkv(c, static_cast<const char *>(packed), kv, x, q);
+    if ((k_new && !al16(k_new)) || (v_new && !al16(v_new)) || (!k_new != !v_new)) return TPL_EINVAL;
+    return run_qkv(c, static_cast<const char *>(packed), kv, x, q, k_new, v_new);
 }
 
-int tpl_attn_decode(tpl_plan *p, const tpl_kv *kv, const float *q, int32_t B, int64_t S, void *o, void *ws,
-                    size_t ws_bytes, tpl_stream stream) {
+int tpl_attn_decode(tpl_plan *p, const tpl_kv *kv, const float *q, const float *k_new, const float *v_new, int32_t B,
+                    int64_t S, void *o, void *ws, size_t ws_bytes, tpl_stream stream) {
     if (B == 0) return TPL_OK;
     Ctx c;
     int rc = make_ctx(p, ws, ws_bytes, B, S, stream, &c);
     if (rc != TPL_OK) return rc;
-    if (!q || !o || !al16(q)) return TPL_EINVAL;
+    if (!q || !o || !al16(q) || (!k_new != !v_new)) return TPL_EINVAL;
     if ((rc = check_kv(kv, B, S)) != TPL_OK) return rc;
-    return run_attn(c, kv, q, o);
+    return run_attn(c, kv, q, k_new, v_new, o);
 }
 
 int tpl_o_proj(tpl_plan *p, const void *packed, const void *o, const void *x, int32_t B, float *h, float *partials,
@@ -523,3 +536,77 @@ int tpl_last_device_error(const tpl_plan *p, tpl_stream stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of tpl_attn_decode.  For callers that cannot
+// allocate device memory (a plugin whose host application owns the device
+// budget, a serving loop that must stay out of the allocator): the split
+// partials and arrival counters live in this fixed array of static device
+// memory instead of a caller-provided workspace.  Every device that loads the
+// library holds the array until the process exits.  Calls share it and it
+// keeps the previous call's contents, so each call clears the counters it
+// uses first; calls that overlap on the GPU race on it.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_attn_scratch[TPL_ATTN_STATIC_SCRATCH_BYTES];
+
+namespace {
+std::atomic<void *> g_attn_scratch_addr[64];  // device address of g_attn_scratch, per device
+
+size_t round256(size_t v) { return (v + 255) / 256 * 256; }
+}  // namespace
+
+extern "C" int tpl_attn_decode_static(tpl_plan *p, const tpl_kv *kv, const float *q, const float *k_new,
+                                      const float *v_new, int32_t B, int64_t S, void *o, tpl_stream stream) {
+    if (!p || !q || !o || !al16(q) || B < 0 || S < 0 || (!k_new != !v_new)) return TPL_EINVAL;
+    if (B == 0) return TPL_OK;
+    if (B > 16) return TPL_EUNSUPPORTED;
+    int rc = check_kv(kv, B, S);
+    if (rc != TPL_OK) return rc;
+    const int64_t keys = k_new ? S : S + 1;
+    AttnGeom g;
+    attn_geom(B, p->d.n_kv_heads, keys, &g);
+    if (g.pairs > kMaxPairs) return TPL_EUNSUPPORTED;
+    const size_t off_ml = round256((size_t)g.pairs * sizeof(unsigned));
+    const size_t cpp = (size_t)g.nsplit / kAttnWarps;  // partials are per CTA
+    const size_t off_o = off_ml + round256((size_t)g.pairs * cpp * p->g * 2 * sizeof(float));
+    const size_t need = off_o + round256((size_t)g.pairs * cpp * p->g * p->d.head_dim * sizeof(float));
+    if (need > TPL_ATTN_STATIC_SCRATCH_BYTES) return TPL_ENOMEM;
+    // Set-up, once per device with that device current: the array's device
+    // address (in host code its name is only a host-side stand-in).
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return TPL_ECUDA;
+    void *base = g_attn_scratch_addr[dev].load();
+    if (!base) {
+        if (cudaGetSymbolAddress(&base, g_attn_scratch) != cudaSuccess || !base) return TPL_ECUDA;
+        g_attn_scratch_addr[dev].store(base);
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char *scratch = static_cast<char *>(base);
+    // The arrival counters must start at zero.
+    if (cudaMemsetAsync(scratch, 0, (size_t)g.pairs * sizeof(unsigned), st) != cudaSuccess) return TPL_ECUDA;
+    AttnArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.q = q;
+    a.kc = static_cast<const __nv_bfloat16 *>(kv->k);
+    a.vc = static_cast<const __nv_bfloat16 *>(kv->v);
+    a.seq_cap = kv->seq_cap;
+    a.batch_cap = kv->batch_cap;
+    a.B = B;
+    a.nq = p->d.n_q_heads;
+    a.nkv_s = p->nkv_s;
+    a.g = p->g;
+    a.keys = keys;
+    a.k_new = k_new;
+    a.v_new = v_new;
+    a.nsplit = g.nsplit;
+    a.kps = g.kps;
+    a.scale_log2 = 1.4426950408889634f / sqrtf((float)p->d.head_dim);
+    a.tickets = reinterpret_cast<unsigned *>(scratch);
+    a.part_ml = reinterpret_cast<float *>(scratch + off_ml);
+    a.part_o = reinterpret_cast<float *>(scratch + off_o);
+    a.o = o;
+    a.o_f32 = p->f32;
+    const int grid = g.pairs * (g.nsplit / kAttnWarps);
+    return cuda_rc(p->g <= 8 ? launch_pdl(attn_decode_kernel<true>, grid, kAttnWarps * 32, 0, st, a)
+                              : launch_pdl(attn_decode_kernel<false>, grid, kAttnWarps * 32, 0, st, a));
+}

@@ -23,6 +23,11 @@
 //   MODE 1 -- fp32 weights with fp32 FFMA (exact-arithmetic comparison mode).
 //   MODE 2 -- bf16 weights with FFMA on the CUDA cores (kept to measure
 //             against MODE 0).
+//   MODE 3 -- MODE 0 with each activation value carried as two bf16 parts
+//             (hi = bf16(v), lo = bf16(v - hi)), staged as token rows B..2B-1;
+//             for B <= 8 the lo parts ride in the otherwise-zero A rows 8-15
+//             of the same mma, for B > 8 they take a second mma.  Used where
+//             the result feeds a softmax (the Q projection).
 #pragma once
 
 #include "tpl_common.cuh"
@@ -53,6 +58,7 @@ struct GemvArgs {
     int resid_f32;
     float *partials;  // [nseg][B][N]
     float *q;
+    float *knew, *vnew;  // [B][n_kv][hd] fp32 copies of the new k/v, or NULL
     __nv_bfloat16 *kc, *vc;
     int nq, nq_s, nkv_s, hd, batch_cap;
     int64_t S, seq_cap;
@@ -72,6 +78,10 @@ struct GemvTraits<1> {  // fp32 weights, fp32 staged x, FFMA
 };
 template <>
 struct GemvTraits<2> {  // bf16 weights, bf16 staged x, FFMA
+    static constexpr int WES = 2, XES = 2, NBI = 2, LPM = 1;
+};
+template <>
+struct GemvTraits<3> {  // MODE 0 with the activation carried as bf16 hi + lo
     static constexpr int WES = 2, XES = 2, NBI = 2, LPM = 1;
 };
 
@@ -96,6 +106,8 @@ __device__ __forceinline__ void gemv_final_row(const GemvArgs &a, int row, int t
             __nv_bfloat16 *c = isk ? a.kc : a.vc;
             c[((((int64_t)s * a.batch_cap + tok) * a.nkv_s + kvl) * a.seq_cap + a.S) * a.hd + dim] =
                 __float2bfloat16_rn(v);
+            float *f = isk ? a.knew : a.vnew;
+            if (f) f[((int64_t)tok * (a.nkv_s * (a.nq / a.nq_s)) + s * a.nkv_s + kvl) * a.hd + dim] = v;
         }
     } else if (a.epi == EPI_ROW) {
         float acc = ss.p[0];
@@ -115,6 +127,8 @@ __device__ __forceinline__ void gemv_final_pair(const GemvArgs &a, int pair, int
 template <int MODE>
 __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_constant__ GemvArgs a) {
     using T = GemvTraits<MODE>;
+    constexpr bool XSPLIT = MODE == 3;
+    constexpr bool MMA = MODE == 0 || MODE == 3;
     extern __shared__ __align__(128) unsigned char smem[];
     const GemvGeom &g = a.g;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -141,7 +155,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
     const int kpc = g.wk / g.segs_per_cta;  // K-groups per segment inside the CTA
 
     unsigned char *xs = smem;
-    float *part = reinterpret_cast<float *>(smem + (size_t)B * g.x_stride);
+    float *part = reinterpret_cast<float *>(smem + (size_t)(XSPLIT ? 2 : 1) * B * g.x_stride);
     const int prows = g.wr * g.rgc * 8;  // rows per round
     float *s_inv = part + (size_t)g.wk * prows * B;
     int *s_flag = reinterpret_cast<int *>(s_inv + 16);
@@ -244,6 +258,14 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
                 o.x = pack_bf16x2(v[0], v[1]); o.y = pack_bf16x2(v[2], v[3]);
                 o.z = pack_bf16x2(v[4], v[5]); o.w = pack_bf16x2(v[6], v[7]);
                 *reinterpret_cast<uint4 *>(dst) = o;
+                if constexpr (XSPLIT) {
+                    uint4 l;
+                    l.x = pack_bf16x2(v[0] - bf16lo(o.x), v[1] - bf16hi(o.x));
+                    l.y = pack_bf16x2(v[2] - bf16lo(o.y), v[3] - bf16hi(o.y));
+                    l.z = pack_bf16x2(v[4] - bf16lo(o.z), v[5] - bf16hi(o.z));
+                    l.w = pack_bf16x2(v[6] - bf16lo(o.w), v[7] - bf16hi(o.w));
+                    *reinterpret_cast<uint4 *>(dst + (size_t)B * g.x_stride) = l;
+                }
             } else {
                 reinterpret_cast<float4 *>(dst)[0] = make_float4(v[0], v[1], v[2], v[3]);
                 reinterpret_cast<float4 *>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
@@ -256,9 +278,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
     const int rg_cta = rg1 - rg0;
     const int rounds = (((rg_cta + g.wr - 1) / g.wr) + g.rgc - 1) / g.rgc;
     const int sl_mine = seg - seg_lo;  // this warp's segment inside the CTA
-    float acc[MODE == 0 ? 4 : 16];
+    float acc[MMA ? 4 : 16];
 #pragma unroll
-    for (int i = 0; i < (MODE == 0 ? 4 : 16); ++i) acc[i] = 0.f;
+    for (int i = 0; i < (MMA ? 4 : 16); ++i) acc[i] = 0.f;
 
     int f = 0;
     for (int r = 0; r < rounds; ++r) {
@@ -282,6 +304,33 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
                             const uint4 w = wa[bi * 4 + m];
                             mma_bf16_16816(acc, xa.x, xb.x, xa.y, xb.y, w.x, w.y);
                             mma_bf16_16816(acc, xa.z, xb.z, xa.w, xb.w, w.z, w.w);
+                        }
+                    } else if constexpr (MODE == 3) {
+                        const size_t lo_off = (size_t)B * g.x_stride;
+#pragma unroll
+                        for (int m = 0; m < 4; ++m) {
+                            const size_t off = (size_t)(xcol + 32 * m + 8 * c) * 2;
+                            const uint4 w = wa[bi * 4 + m];
+                            if (B <= 8) {
+                                // rows gid: hi of token gid, rows gid+8: lo of token gid
+                                uint4 xa = make_uint4(0, 0, 0, 0), xb = make_uint4(0, 0, 0, 0);
+                                if (gid < B) {
+                                    xa = lds128(xs + (size_t)gid * g.x_stride + off);
+                                    xb = lds128(xs + lo_off + (size_t)gid * g.x_stride + off);
+                                }
+                                mma_bf16_16816(acc, xa.x, xb.x, xa.y, xb.y, w.x, w.y);
+                                mma_bf16_16816(acc, xa.z, xb.z, xa.w, xb.w, w.z, w.w);
+                            } else {
+#pragma unroll
+                                for (int part_i = 0; part_i < 2; ++part_i) {
+                                    const size_t po = part_i ? lo_off : 0;
+                                    uint4 xa = lds128(xs + po + (size_t)gid * g.x_stride + off);
+                                    uint4 xb = gid + 8 < B ? lds128(xs + po + (size_t)(gid + 8) * g.x_stride + off)
+                                                           : make_uint4(0, 0, 0, 0);
+                                    mma_bf16_16816(acc, xa.x, xb.x, xa.y, xb.y, w.x, w.y);
+                                    mma_bf16_16816(acc, xa.z, xb.z, xa.w, xb.w, w.z, w.w);
+                                }
+                            }
                         }
                     } else {
 #pragma unroll
@@ -329,7 +378,13 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
                 // row group done: write its partial sums for this K-group
                 const int pr = (wslot + (k - r * g.rgc) * g.wr) * 8;
                 float *pp = part + ((size_t)kgl * prows + pr) * B;
-                if constexpr (MODE == 0) {
+                if constexpr (MMA) {
+                    if (XSPLIT && B <= 8) {
+                        // hi and lo halves of the same token
+                        acc[0] += acc[2];
+                        acc[1] += acc[3];
+                        acc[2] = acc[3] = 0.f;
+                    }
                     if (gid < B) {
                         pp[(2 * c) * B + gid] = acc[0];
                         pp[(2 * c + 1) * B + gid] = acc[1];

@@ -19,7 +19,9 @@ constexpr int kGemvWarps = kGemvThreads / 32;
 constexpr size_t kXSmemMax = 140 * 1024;   // activation slice staged per CTA
 constexpr size_t kPartSmemMax = 64 * 1024; // per-round partial sums
 constexpr int kAttnWarps = 4;              // warps per attention CTA
-constexpr int kAttnTargetWarps = 2048;     // key-range splits across all (b, kv head) pairs
+constexpr int kAttnTargetWarps = 1024;     // key-range splits across all (b, kv head) pairs
+constexpr int kAttnMinKeys = 128;          // keys per split at least (when there are that many)
+constexpr int kAttnMaxCtasPerPair = 64;
 constexpr int kTicketSlots = 4096;         // uint32 arrival counters at the workspace start
 constexpr int kTicketAttn = 0;             // [0, 1024): attention pairs
 constexpr int kTicketGemv = 1024;          // + 512 * op
@@ -63,15 +65,18 @@ struct GemvGeom {
     size_t gp_floats; // cross-CTA partial floats (0 when ksplit == 1)
 };
 
-int gemv_geom(int N, int nseg, int Kseg, int B, int xbytes, int num_sms, GemvGeom *g);
+// xparts: 1, or 2 when the activation is staged as bf16 hi + lo rows.
+int gemv_geom(int N, int nseg, int Kseg, int B, int xbytes, int num_sms, GemvGeom *g, int xparts = 1);
 
 struct AttnGeom {
     int pairs, nsplit, kps;  // pairs = B * n_kv; splits per pair; keys per split
 };
-void attn_geom(int B, int nkv, int64_t S, AttnGeom *a);
+// keys: keys covered by the splits (S when the new token is added in the
+// combine, S + 1 when it is read from the cache).
+void attn_geom(int B, int nkv, int64_t keys, AttnGeom *a);
 
 struct WsLayout {
-    size_t tickets, q, o, h, act, ybuf0, ybuf1, P, part_o, part_ml, gp, total;
+    size_t tickets, q, o, h, act, ybuf0, ybuf1, P, knew, vnew, part_o, part_ml, gp, total;
 };
 int ws_layout(const tpl_plan *p, int B, int64_t S, WsLayout *w);
 

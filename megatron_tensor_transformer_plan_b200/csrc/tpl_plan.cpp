@@ -40,7 +40,7 @@ int validate(const tpl_dims *d, int32_t t) {
 
 namespace tpl {
 
-int gemv_geom(int N, int nseg, int Kseg, int B, int xbytes, int num_sms, GemvGeom *g) {
+int gemv_geom(int N, int nseg, int Kseg, int B, int xbytes, int num_sms, GemvGeom *g, int xparts) {
     if (N <= 0 || nseg <= 0 || Kseg <= 0 || B <= 0 || num_sms <= 0) return TPL_EINVAL;
     std::memset(g, 0, sizeof(*g));
     g->N = N;
@@ -52,13 +52,13 @@ int gemv_geom(int N, int nseg, int Kseg, int B, int xbytes, int num_sms, GemvGeo
         if (ksplit > 64) return TPL_EUNSUPPORTED;
         if (ksplit <= nseg) {
             blocks = g->nb;  // per segment, nseg/ksplit whole segments
-            int64_t bytes = (int64_t)B * ((int64_t)(nseg / ksplit) * blocks * 128 * xbytes + 64);
+            int64_t bytes = (int64_t)xparts * B * ((int64_t)(nseg / ksplit) * blocks * 128 * xbytes + 64);
             if (bytes <= (int64_t)kXSmemMax) break;
         } else {
             int per = ksplit / nseg;
             if (per > g->nb) return TPL_EUNSUPPORTED;
             blocks = (g->nb + per - 1) / per;
-            int64_t bytes = (int64_t)B * ((int64_t)blocks * 128 * xbytes + 64);
+            int64_t bytes = (int64_t)xparts * B * ((int64_t)blocks * 128 * xbytes + 64);
             if (bytes <= (int64_t)kXSmemMax) break;
         }
     }
@@ -83,17 +83,22 @@ int gemv_geom(int N, int nseg, int Kseg, int B, int xbytes, int num_sms, GemvGeo
     g->rgc = std::max(1, std::min(rg_warp, rgc_cap));
     g->x_stride = m * blocks * 128 * xbytes + 64;
     size_t part = (size_t)kGemvWarps * g->rgc * 8 * B * 4;
-    g->smem = (size_t)B * g->x_stride + part + 128;
+    g->smem = (size_t)xparts * B * g->x_stride + part + 128;
     g->gp_floats = ksplit > 1 ? (size_t)nseg * g->pieces * N * B : 0;
     return TPL_OK;
 }
 
-void attn_geom(int B, int nkv, int64_t S, AttnGeom *a) {
-    int64_t keys = S + 1;
+void attn_geom(int B, int nkv, int64_t keys, AttnGeom *a) {
     a->pairs = B * nkv;
+    if (keys <= 0) {  // nothing in the cache: the splits are empty
+        a->nsplit = kAttnWarps;
+        a->kps = 16;
+        return;
+    }
     int64_t ns = (kAttnTargetWarps + a->pairs - 1) / a->pairs;
     ns = std::max<int64_t>(ns, 1);
-    ns = std::min<int64_t>(ns, (keys + 31) / 32);
+    ns = std::min<int64_t>(ns, (keys + kAttnMinKeys - 1) / kAttnMinKeys);
+    ns = std::min<int64_t>(ns, (int64_t)kAttnMaxCtasPerPair * kAttnWarps);
     ns = std::max<int64_t>(ns, 1);
     int64_t kps = (keys + ns - 1) / ns;
     kps = (kps + 15) / 16 * 16;
@@ -122,18 +127,24 @@ int ws_layout(const tpl_plan *p, int B, int64_t S, WsLayout *w) {
     w->ybuf0 = take((size_t)B * H * es);
     w->ybuf1 = take((size_t)B * H * es);
     w->P = take((size_t)p->t * B * H * 4);
-    AttnGeom ag;
+    w->knew = take((size_t)B * d.n_kv_heads * d.head_dim * 4);
+    w->vnew = take((size_t)B * d.n_kv_heads * d.head_dim * 4);
+    AttnGeom ag, ag1;  // splits over S keys (new key apart) or S + 1 keys
     attn_geom(B, d.n_kv_heads, S, &ag);
-    w->part_o = take((size_t)ag.pairs * ag.nsplit * p->g * d.head_dim * 4);
-    w->part_ml = take((size_t)ag.pairs * ag.nsplit * p->g * 2 * 4);
+    attn_geom(B, d.n_kv_heads, S + 1, &ag1);
+    const size_t nsp = (size_t)std::max(ag.nsplit, ag1.nsplit);
+    w->part_o = take((size_t)ag.pairs * (nsp / kAttnWarps) * p->g * d.head_dim * 4);
+    w->part_ml = take((size_t)ag.pairs * (nsp / kAttnWarps) * p->g * 2 * 4);
     // cross-CTA partials: the largest over the four matrix-vector steps
     size_t gp = 0;
     GemvGeom gg;
     const int xb = p->f32 ? 4 : 2;
     const int sms = 148;  // only the split-K factor matters here, not the SM count
-    if (gemv_geom(p->t * p->qkv_rows_s, 1, (int)H, B, xb, sms, &gg) == TPL_OK) gp = std::max(gp, gg.gp_floats);
+    if (gemv_geom(p->t * p->qkv_rows_s, 1, (int)H, B, xb, sms, &gg, p->f32 ? 1 : 2) == TPL_OK)
+        gp = std::max(gp, gg.gp_floats);
     if (gemv_geom((int)H, p->t, p->nq_s * d.head_dim, B, xb, sms, &gg) == TPL_OK) gp = std::max(gp, gg.gp_floats);
-    if (gemv_geom(p->t * 2 * p->F_s, 1, (int)H, B, xb, sms, &gg) == TPL_OK) gp = std::max(gp, gg.gp_floats);
+    if (gemv_geom(p->t * 2 * p->F_s, 1, (int)H, B, xb, sms, &gg, p->f32 ? 1 : 2) == TPL_OK)
+        gp = std::max(gp, gg.gp_floats);
     if (gemv_geom((int)H, p->t, p->F_s, B, xb, sms, &gg) == TPL_OK) gp = std::max(gp, gg.gp_floats);
     w->gp = take(gp * 4 + 4);
     w->total = off;

@@ -24,6 +24,7 @@ TPL_OK, TPL_EINVAL, TPL_EINDIVISIBLE, TPL_EWORKSPACE, TPL_ENOMEM, TPL_ECUDA, TPL
 TPL_NORM, TPL_RESIDUAL, TPL_FP32_WEIGHTS = 1, 2, 4
 TPL_REDUCE_FUSED, TPL_REDUCE_SEPARATE = 0, 1
 TPL_OPT_GEMV_MODE = 1
+TPL_ATTN_STATIC_SCRATCH_BYTES = 4 * 1024 * 1024
 
 c_int32, c_int64, c_size_t, c_void_p, c_uint32 = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_uint32
 P = ctypes.POINTER
@@ -78,9 +79,11 @@ _sig("tpl_decode_stack", ctypes.c_int, _plan_p, P(c_void_p), P(tpl_kv), c_void_p
 _sig("tpl_prefill_layer", ctypes.c_int, _plan_p, c_void_p, P(tpl_kv), c_void_p, c_int32, c_void_p, c_void_p,
      c_void_p, c_size_t, c_int32, c_void_p)
 _sig("tpl_qkv", ctypes.c_int, _plan_p, c_void_p, P(tpl_kv), c_void_p, c_int32, c_int64, c_void_p, c_void_p,
-     c_size_t, c_void_p)
-_sig("tpl_attn_decode", ctypes.c_int, _plan_p, P(tpl_kv), c_void_p, c_int32, c_int64, c_void_p, c_void_p,
-     c_size_t, c_void_p)
+     c_void_p, c_void_p, c_size_t, c_void_p)
+_sig("tpl_attn_decode", ctypes.c_int, _plan_p, P(tpl_kv), c_void_p, c_void_p, c_void_p, c_int32, c_int64, c_void_p,
+     c_void_p, c_size_t, c_void_p)
+_sig("tpl_attn_decode_static", ctypes.c_int, _plan_p, P(tpl_kv), c_void_p, c_void_p, c_void_p, c_int32, c_int64,
+     c_void_p, c_void_p)
 _sig("tpl_o_proj", ctypes.c_int, _plan_p, c_void_p, c_void_p, c_void_p, c_int32, c_void_p, c_void_p, c_void_p,
      c_size_t, c_void_p)
 _sig("tpl_gate_up", ctypes.c_int, _plan_p, c_void_p, c_void_p, c_int32, c_int32, c_void_p, c_void_p, c_size_t,
@@ -233,13 +236,13 @@ class Plan:
         check(tpl_decode_stack(self.handle, arr, kvs, x.data_ptr(), B, S, _ptr(y), _ptr(y32), ws.data_ptr(),
                                ws.numel(), mode, _stream()), "tpl_decode_stack")
 
-    def qkv(self, packed, kv: tpl_kv, x, S: int, q, ws):
+    def qkv(self, packed, kv: tpl_kv, x, S: int, q, ws, k_new=None, v_new=None):
         check(tpl_qkv(self.handle, packed.data_ptr(), ctypes.byref(kv), x.data_ptr(), x.shape[0], S, q.data_ptr(),
-                      ws.data_ptr(), ws.numel(), _stream()), "tpl_qkv")
+                      _ptr(k_new), _ptr(v_new), ws.data_ptr(), ws.numel(), _stream()), "tpl_qkv")
 
-    def attn_decode(self, kv: tpl_kv, q, S: int, o, ws):
-        check(tpl_attn_decode(self.handle, ctypes.byref(kv), q.data_ptr(), q.shape[0], S, o.data_ptr(),
-                              ws.data_ptr(), ws.numel(), _stream()), "tpl_attn_decode")
+    def attn_decode(self, kv: tpl_kv, q, S: int, o, ws, k_new=None, v_new=None):
+        check(tpl_attn_decode(self.handle, ctypes.byref(kv), q.data_ptr(), _ptr(k_new), _ptr(v_new), q.shape[0], S,
+                              o.data_ptr(), ws.data_ptr(), ws.numel(), _stream()), "tpl_attn_decode")
 
     def o_proj(self, packed, o, x, h=None, partials=None, ws=None):
         check(tpl_o_proj(self.handle, packed.data_ptr(), o.data_ptr(), _ptr(x), o.shape[0], _ptr(h), _ptr(partials),

@@ -111,8 +111,10 @@ def run_steps(L: Layer, mode=tpl.TPL_REDUCE_FUSED):
     y = torch.empty((B, H), dtype=dt, device=dev)
     y32 = torch.empty((B, H), dtype=torch.float32, device=dev)
     resid = bool(d.flags & tpl.TPL_RESIDUAL)
-    p.qkv(L.packed, L.kv, L.x, L.S, q, L.ws)
-    p.attn_decode(L.kv, q, L.S, o, L.ws)
+    kn = torch.empty((B, d.n_kv_heads, d.head_dim), dtype=torch.float32, device=dev)
+    vn = torch.empty_like(kn)
+    p.qkv(L.packed, L.kv, L.x, L.S, q, L.ws, kn, vn)
+    p.attn_decode(L.kv, q, L.S, o, L.ws, kn, vn)
     if mode == tpl.TPL_REDUCE_FUSED:
         p.o_proj(L.packed, o, L.x, h=h, ws=L.ws)
     else:
@@ -128,7 +130,8 @@ def run_steps(L: Layer, mode=tpl.TPL_REDUCE_FUSED):
         p.down_proj(L.packed, act, None, partials=P2, ws=L.ws)
         p.reduce_partials(P2, h if resid else None, True, out32=y32, out_act=y)
     torch.cuda.synchronize()
-    return {"q": q, "attn": o, "h": h, "act": act, "y": y, "y32": y32, "down_partials": P2}
+    return {"q": q, "k_new": kn, "v_new": vn, "attn": o, "h": h, "act": act, "y": y, "y32": y32,
+            "down_partials": P2}
 
 
 def new_kv_slot(L: Layer):

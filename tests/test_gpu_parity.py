@@ -22,8 +22,12 @@ def _check_layer(L, ref_y, tr, mode_both=True):
     d = L.dims
     assert_close_rel(to_np(steps["q"]).reshape(L.B, -1), tr["q"], what="q")
     kk, vv = new_kv_slot(L)
-    assert_close_rel(to_np(kk), tr["k_new"], what="k_new")
-    assert_close_rel(to_np(vv), tr["v_new"], what="v_new")
+    assert_close_rel(to_np(kk), tr["k_new"], what="k_new (cache slot S)")
+    assert_close_rel(to_np(vv), tr["v_new"], what="v_new (cache slot S)")
+    assert_close_rel(to_np(steps["k_new"]).reshape(L.B, -1), tr["k_new"], what="k_new fp32")
+    assert_close_rel(to_np(steps["v_new"]).reshape(L.B, -1), tr["v_new"], what="v_new fp32")
+    # the cache holds the bf16 rounding of the fp32 values
+    assert torch.equal(kk, steps["k_new"].reshape(L.B, -1).bfloat16())
     assert_close_rel(to_np(steps["attn"]), tr["attn"], what="attention output")
     assert_close_rel(to_np(steps["h"]), tr["h"], what="h")
     assert_close_rel(to_np(steps["act"]), tr["act"], what="act")
@@ -62,6 +66,17 @@ def test_decode_layer_small(gpu, case):
     L = make_layer(H, nq, nkv, 128, F, t, B, S, gamma_std=gs, S_cap=S + 3)
     ref_y, tr = oracle_decode(L)
     _check_layer(L, ref_y, tr)
+
+
+def test_empty_cache_attention_is_new_value(gpu):
+    """S = 0: one key, weight exactly 1, so the attention output is v_new
+    (exactly, up to the output's bf16 rounding)."""
+    L = make_layer(1024, 16, 4, 128, 2816, 4, 3, 0)
+    st = run_steps(L)
+    g = 16 // 4
+    v = st["v_new"]  # [B][n_kv][d]
+    expect = v.repeat_interleave(g, dim=1).reshape(L.B, -1).bfloat16()
+    assert torch.equal(st["attn"], expect)
 
 
 def test_kv_cache_only_slot_s_changes(gpu):

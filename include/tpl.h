@@ -166,7 +166,8 @@ int tpl_workspace_size(const tpl_plan *plan, int32_t batch, int64_t seq, size_t 
 int tpl_workspace_init(const tpl_plan *plan, void *ws, size_t ws_bytes, tpl_stream stream);
 
 /* Rearrange one layer's unsharded weights into the plan's packed shard
- * layout (`packed`, packed_bytes >= info.packed_layer_bytes):
+ * layout (`packed`, packed_bytes >= info.packed_layer_bytes), every row
+ * zero-padded to a whole number of 128-column blocks:
  *   Wqkv[s] = rows [q heads of s | k heads of s | v heads of s] of Wq/Wk/Wv
  *   Wo[s]   = Wo[:, s*(n_q/t)*d : (s+1)*(n_q/t)*d]           (row split)
  *   Wgu[s]  = rows Wg[c], Wu[c] interleaved for c in shard s's ffn columns

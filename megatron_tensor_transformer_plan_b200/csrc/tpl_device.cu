@@ -55,20 +55,31 @@ cudaError_t launch_pdl(void (*kern)(KA...), int grid, int block, size_t smem, cu
     return cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...);
 }
 
-bool g_attr_done[64][4];
+bool g_attr_done[64][8];
 
-int prepare_gemv(int mode) {
+template <int MODE, bool BIG>
+cudaError_t set_smem_attr() {
+    return cudaFuncSetAttribute(gemv_kernel<MODE, BIG>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+}
+
+int prepare_gemv(int mode, bool big) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return TPL_ECUDA;
-    if (!g_attr_done[dev][mode]) {
+    const int slot = mode * 2 + (big ? 1 : 0);
+    if (!g_attr_done[dev][slot]) {
         cudaError_t e;
-        const int maxb = 227 * 1024;
-        if (mode == 0) e = cudaFuncSetAttribute(gemv_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxb);
-        else if (mode == 1) e = cudaFuncSetAttribute(gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxb);
-        else if (mode == 2) e = cudaFuncSetAttribute(gemv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxb);
-        else e = cudaFuncSetAttribute(gemv_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxb);
+        switch (slot) {
+            case 0: e = set_smem_attr<0, false>(); break;
+            case 1: e = set_smem_attr<0, true>(); break;
+            case 2: e = set_smem_attr<1, false>(); break;
+            case 3: e = set_smem_attr<1, true>(); break;
+            case 4: e = set_smem_attr<2, false>(); break;
+            case 5: e = set_smem_attr<2, true>(); break;
+            case 6: e = set_smem_attr<3, false>(); break;
+            default: e = set_smem_attr<3, true>(); break;
+        }
         if (e != cudaSuccess) return TPL_ECUDA;
-        g_attr_done[dev][mode] = true;
+        g_attr_done[dev][slot] = true;
     }
     return TPL_OK;
 }
@@ -115,17 +126,25 @@ int gemv_launch(Ctx &c, GemvArgs &a, int N, int nseg, int Kseg, int op) {
     const int mode = p->f32 ? 1 : (p->gemv_mode == 2 ? 2 : ((op == OP_QKV || op == OP_GU) ? 3 : 0));
     int rc = gemv_geom(N, nseg, Kseg, c.B, p->f32 ? 4 : 2, sms, &a.g, mode == 3 ? 2 : 1);
     if (rc != TPL_OK) return rc;
-    rc = prepare_gemv(mode);
+    const bool big = c.B > 8;
+    rc = prepare_gemv(mode, big);
     if (rc != TPL_OK) return rc;
     a.B = c.B;
     a.gp = reinterpret_cast<float *>(c.ws + c.L.gp);
     a.tickets = reinterpret_cast<unsigned *>(c.ws + c.L.tickets) + kTicketGemv + 512 * op;
     const int grid = a.g.rb * a.g.ksplit;
+    const size_t sm = a.g.smem;
     cudaError_t e;
-    if (mode == 0) e = launch_pdl(gemv_kernel<0>, grid, kGemvThreads, a.g.smem, c.st, a);
-    else if (mode == 1) e = launch_pdl(gemv_kernel<1>, grid, kGemvThreads, a.g.smem, c.st, a);
-    else if (mode == 2) e = launch_pdl(gemv_kernel<2>, grid, kGemvThreads, a.g.smem, c.st, a);
-    else e = launch_pdl(gemv_kernel<3>, grid, kGemvThreads, a.g.smem, c.st, a);
+    switch (mode * 2 + (big ? 1 : 0)) {
+        case 0: e = launch_pdl(gemv_kernel<0, false>, grid, kGemvThreads, sm, c.st, a); break;
+        case 1: e = launch_pdl(gemv_kernel<0, true>, grid, kGemvThreads, sm, c.st, a); break;
+        case 2: e = launch_pdl(gemv_kernel<1, false>, grid, kGemvThreads, sm, c.st, a); break;
+        case 3: e = launch_pdl(gemv_kernel<1, true>, grid, kGemvThreads, sm, c.st, a); break;
+        case 4: e = launch_pdl(gemv_kernel<2, false>, grid, kGemvThreads, sm, c.st, a); break;
+        case 5: e = launch_pdl(gemv_kernel<2, true>, grid, kGemvThreads, sm, c.st, a); break;
+        case 6: e = launch_pdl(gemv_kernel<3, false>, grid, kGemvThreads, sm, c.st, a); break;
+        default: e = launch_pdl(gemv_kernel<3, true>, grid, kGemvThreads, sm, c.st, a); break;
+    }
     return cuda_rc(e);
 }
 
@@ -144,7 +163,7 @@ int run_qkv(Ctx &c, const char *packed, const tpl_kv *kv, const void *x, float *
     a.W = packed + p->off_qkv;
     a.blk_r = p->blk_qkv;
     a.rps = p->qkv_rows_s;
-    a.ldw = p->d.hidden;
+    a.ldw = p->ld_h;
     a.x = x;
     a.x_f32 = p->f32;
     a.ldx = p->d.hidden;
@@ -205,7 +224,7 @@ int run_o(Ctx &c, const char *packed, const void *o, const void *resid, float *h
     a.W = packed + p->off_o;
     a.blk_s = p->blk_o;
     a.rps = p->d.hidden;
-    a.ldw = p->nq_s * p->d.head_dim;
+    a.ldw = p->ld_o;
     a.x = o;
     a.x_f32 = p->f32;
     a.ldx = p->d.n_q_heads * p->d.head_dim;
@@ -229,7 +248,7 @@ int run_gu(Ctx &c, const char *packed, const void *h, int h_is_act, void *act) {
     a.W = packed + p->off_gu;
     a.blk_r = p->blk_gu;
     a.rps = 2 * p->F_s;
-    a.ldw = p->d.hidden;
+    a.ldw = p->ld_h;
     a.x = h;
     a.x_f32 = h_is_act ? p->f32 : 1;
     a.ldx = p->d.hidden;
@@ -247,7 +266,7 @@ int run_down(Ctx &c, const char *packed, const void *act, const void *resid, int
     a.W = packed + p->off_d;
     a.blk_s = p->blk_d;
     a.rps = p->d.hidden;
-    a.ldw = p->F_s;
+    a.ldw = p->ld_f;
     a.x = act;
     a.x_f32 = p->f32;
     a.ldx = p->d.ffn;
@@ -342,22 +361,27 @@ int tpl_pack_layer(const tpl_plan *p, const tpl_layer_weights *w, void *packed, 
     auto ok = [&](cudaError_t r) {
         if (e == cudaSuccess) e = r;
     };
+    // padding columns must read as zero
+    ok(cudaMemsetAsync(P, 0, (size_t)p->off_g1, st));
+    const int64_t lh = (int64_t)p->ld_h * es, lo = (int64_t)p->ld_o * es, lf = (int64_t)p->ld_f * es;
     for (int s = 0; s < p->t; ++s) {
         if (attn) {
             char *dq = P + p->off_qkv + s * p->blk_qkv;
-            const int64_t qb = (int64_t)p->nq_s * hd * H * es, kb = (int64_t)p->nkv_s * hd * H * es;
-            ok(cudaMemcpyAsync(dq, wq + s * qb, qb, cudaMemcpyDeviceToDevice, st));
-            ok(cudaMemcpyAsync(dq + qb, wk + s * kb, kb, cudaMemcpyDeviceToDevice, st));
-            ok(cudaMemcpyAsync(dq + qb + kb, wv + s * kb, kb, cudaMemcpyDeviceToDevice, st));
-            ok(cudaMemcpy2DAsync(P + p->off_o + s * p->blk_o, Ks * es, wo + s * Ks * es, (int64_t)d.n_q_heads * hd * es,
+            const int64_t qr = (int64_t)p->nq_s * hd, kr = (int64_t)p->nkv_s * hd;  // rows
+            ok(cudaMemcpy2DAsync(dq, lh, wq + s * qr * H * es, H * es, H * es, qr, cudaMemcpyDeviceToDevice, st));
+            ok(cudaMemcpy2DAsync(dq + qr * lh, lh, wk + s * kr * H * es, H * es, H * es, kr, cudaMemcpyDeviceToDevice,
+                                 st));
+            ok(cudaMemcpy2DAsync(dq + (qr + kr) * lh, lh, wv + s * kr * H * es, H * es, H * es, kr,
+                                 cudaMemcpyDeviceToDevice, st));
+            ok(cudaMemcpy2DAsync(P + p->off_o + s * p->blk_o, lo, wo + s * Ks * es, (int64_t)d.n_q_heads * hd * es,
                                  Ks * es, H, cudaMemcpyDeviceToDevice, st));
         }
         char *dgu = P + p->off_gu + s * p->blk_gu;
-        ok(cudaMemcpy2DAsync(dgu, 2 * H * es, wg + (int64_t)s * p->F_s * H * es, H * es, H * es, p->F_s,
+        ok(cudaMemcpy2DAsync(dgu, 2 * lh, wg + (int64_t)s * p->F_s * H * es, H * es, H * es, p->F_s,
                              cudaMemcpyDeviceToDevice, st));
-        ok(cudaMemcpy2DAsync(dgu + H * es, 2 * H * es, wu + (int64_t)s * p->F_s * H * es, H * es, H * es, p->F_s,
+        ok(cudaMemcpy2DAsync(dgu + lh, 2 * lh, wu + (int64_t)s * p->F_s * H * es, H * es, H * es, p->F_s,
                              cudaMemcpyDeviceToDevice, st));
-        ok(cudaMemcpy2DAsync(P + p->off_d + s * p->blk_d, (int64_t)p->F_s * es, wd + (int64_t)s * p->F_s * es, F * es,
+        ok(cudaMemcpy2DAsync(P + p->off_d + s * p->blk_d, lf, wd + (int64_t)s * p->F_s * es, F * es,
                              (int64_t)p->F_s * es, H, cudaMemcpyDeviceToDevice, st));
     }
     float *g1 = reinterpret_cast<float *>(P + p->off_g1), *g2 = reinterpret_cast<float *>(P + p->off_g2);

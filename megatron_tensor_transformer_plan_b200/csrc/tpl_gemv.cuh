@@ -16,6 +16,9 @@
 // in the same order -- so both modes give identical bits.
 //
 // Inner product modes:
+// Weight rows are padded to whole 128-column blocks in the packed layout, and
+// each warp keeps four blocks of loads in flight in a register ring.
+//
 //   MODE 0 -- bf16 weights on the tensor cores (mma.sync m16n8k16): the
 //             activation tile is the A operand (tokens as rows), 8 weight rows
 //             the B operand; the k index of each 16-wide step is permuted so
@@ -68,21 +71,23 @@ struct GemvArgs {
 
 template <int MODE>
 struct GemvTraits;
+// WES / XES: weight / staged-activation element bytes; LPM: 16-byte loads per
+// lane per 32-column step.
 template <>
 struct GemvTraits<0> {  // bf16 weights, bf16 staged x, tensor cores
-    static constexpr int WES = 2, XES = 2, NBI = 2, LPM = 1;
+    static constexpr int WES = 2, XES = 2, LPM = 1;
 };
 template <>
 struct GemvTraits<1> {  // fp32 weights, fp32 staged x, FFMA
-    static constexpr int WES = 4, XES = 4, NBI = 1, LPM = 2;
+    static constexpr int WES = 4, XES = 4, LPM = 2;
 };
 template <>
 struct GemvTraits<2> {  // bf16 weights, bf16 staged x, FFMA
-    static constexpr int WES = 2, XES = 2, NBI = 2, LPM = 1;
+    static constexpr int WES = 2, XES = 2, LPM = 1;
 };
 template <>
 struct GemvTraits<3> {  // MODE 0 with the activation carried as bf16 hi + lo
-    static constexpr int WES = 2, XES = 2, NBI = 2, LPM = 1;
+    static constexpr int WES = 2, XES = 2, LPM = 1;
 };
 
 // Segment sums and the final write for one (row, token).
@@ -124,11 +129,14 @@ __device__ __forceinline__ void gemv_final_pair(const GemvArgs &a, int pair, int
     store_act(a.out_act, a.act_f32, (int64_t)tok * (a.g.N / 2) + pair, silu(gsum) * usum);
 }
 
-template <int MODE>
+template <int MODE, bool BIG>  // BIG: more than 8 tokens (tokens 8..15 in A rows 8-15)
 __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_constant__ GemvArgs a) {
     using T = GemvTraits<MODE>;
     constexpr bool XSPLIT = MODE == 3;
     constexpr bool MMA = MODE == 0 || MODE == 3;
+    constexpr int D = MODE == 1 ? 2 : 4;       // blocks in flight per warp (register ring)
+    constexpr int NW = 4 * T::LPM;             // uint4 per block per lane
+    constexpr int BLK_BYTES = 128 * T::WES;    // one 128-column block of one row
     extern __shared__ __align__(128) unsigned char smem[];
     const GemvGeom &g = a.g;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -155,45 +163,43 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
     const int kpc = g.wk / g.segs_per_cta;  // K-groups per segment inside the CTA
 
     unsigned char *xs = smem;
+    const size_t lo_off = (size_t)B * g.x_stride;  // hi+lo staging: lo rows follow the hi rows
     float *part = reinterpret_cast<float *>(smem + (size_t)(XSPLIT ? 2 : 1) * B * g.x_stride);
     const int prows = g.wr * g.rgc * 8;  // rows per round
     float *s_inv = part + (size_t)g.wk * prows * B;
     int *s_flag = reinterpret_cast<int *>(s_inv + 16);
 
-    // Warp's work: row groups rg0 + wslot + k*wr, items of NBI blocks.
+    // Warp's work: row groups r = 0..nrg_w-1 (rg = rg0 + wslot + r*wr), each
+    // nblk blocks of its K-group; T blocks in all, streamed in that order.
     const int nrg_w = rg1 - rg0 > wslot ? (rg1 - rg0 - wslot + g.wr - 1) / g.wr : 0;
     const int nblk = kb_hi - kb_lo;
-    const int nit = nblk > 0 ? (nblk + T::NBI - 1) / T::NBI : 1;
-    const int nitems = nrg_w * nit;
-
-    constexpr int NW = T::NBI * 4 * T::LPM;  // uint4 per item per lane
-    uint4 wa[NW], wb[NW];
-
-    auto load_item = [&](uint4 (&w)[NW], int f) {
-        const int k = f / nit, it = f % nit;
-        const int rg = rg0 + wslot + k * g.wr;
-        const int row = rg * 8 + gid;
-        const bool row_ok = row < g.N;
-        const char *rp = a.W + (int64_t)(row / a.rps) * a.blk_r + (int64_t)seg * a.blk_s +
-                         (int64_t)(row % a.rps) * a.ldw * T::WES;
+    const int T_blocks = nrg_w * nblk;
+    // weights are padded to whole 128-column blocks and N is a multiple of 8:
+    // every load below is in range without a predicate.
+    auto rowptr = [&](int r) -> const char * {
+        const int row = (rg0 + wslot + r * g.wr) * 8 + gid;
+        return a.W + (int64_t)(row / a.rps) * a.blk_r + (int64_t)seg * a.blk_s +
+               ((int64_t)(row % a.rps) * a.ldw + (int64_t)kb_lo * 128 + 8 * c) * T::WES;
+    };
+    uint4 ring[D][NW];
+    int lr = 0, lj = 0;
+    const char *lptr = nrg_w > 0 ? rowptr(0) : a.W;
+    auto load_next = [&](uint4 (&w)[NW]) {
 #pragma unroll
-        for (int bi = 0; bi < T::NBI; ++bi) {
-            const int blk = kb_lo + it * T::NBI + bi;
+        for (int m = 0; m < 4; ++m)
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const int col = blk * 128 + 32 * m + 8 * c;
-                const bool ok = row_ok && blk < kb_hi && col < g.Kseg;
-#pragma unroll
-                for (int l = 0; l < T::LPM; ++l) {
-                    w[(bi * 4 + m) * T::LPM + l] =
-                        ok ? ldg_stream(rp + (int64_t)col * T::WES + 16 * l) : make_uint4(0, 0, 0, 0);
-                }
-            }
+            for (int l = 0; l < T::LPM; ++l) w[m * T::LPM + l] = ldg_stream(lptr + m * 32 * T::WES + 16 * l);
+        if (++lj == nblk) {
+            lj = 0;
+            if (++lr < nrg_w) lptr = rowptr(lr);
+        } else {
+            lptr += BLK_BYTES;
         }
     };
-
     // Issue the first weight loads before waiting on the previous kernel.
-    if (nitems > 0) load_item(wa, 0);
+#pragma unroll
+    for (int d = 0; d < D; ++d)
+        if (d < T_blocks) load_next(ring[d]);
     pdl_wait();
     pdl_trigger();
 
@@ -201,14 +207,24 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
     if (a.norm) {
         // inverse RMS over the full row of each token, fixed-order reduction
         float *s_red = part;  // scratch, [16 warps][B]
+        const int nch = a.ldx / 8;
         for (int tok = 0; tok < B; ++tok) {
             float ss = 0.f;
-            for (int i = tid * 8; i < a.ldx; i += kGemvThreads * 8) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    float v = load_act(a.x, a.x_f32, (int64_t)tok * a.ldx + i + e);
-                    ss += v * v;
+            for (int i = tid; i < nch; i += kGemvThreads) {
+                float v[8];
+                const int64_t src = (int64_t)tok * a.ldx + (int64_t)i * 8;
+                if (a.x_f32) {
+                    const float4 *p4 = reinterpret_cast<const float4 *>(static_cast<const float *>(a.x) + src);
+                    const float4 x0 = p4[0], x1 = p4[1];
+                    v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w;
+                    v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
+                } else {
+                    const uint4 r4 = *reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(a.x) + src);
+                    v[0] = bf16lo(r4.x); v[1] = bf16hi(r4.x); v[2] = bf16lo(r4.y); v[3] = bf16hi(r4.y);
+                    v[4] = bf16lo(r4.z); v[5] = bf16hi(r4.z); v[6] = bf16lo(r4.w); v[7] = bf16hi(r4.w);
                 }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) ss += v[e] * v[e];
             }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
@@ -245,8 +261,11 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
                 }
                 if (a.norm) {
                     const float inv = s_inv[tok];
+                    const float4 g0 = reinterpret_cast<const float4 *>(a.gamma + k)[0];
+                    const float4 g1 = reinterpret_cast<const float4 *>(a.gamma + k)[1];
+                    const float gm[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) v[e] = v[e] * inv * (a.gamma ? a.gamma[k + e] : 1.0f);
+                    for (int e = 0; e < 8; ++e) v[e] = v[e] * inv * gm[e];
                 }
             } else {
 #pragma unroll
@@ -264,7 +283,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
                     l.y = pack_bf16x2(v[2] - bf16lo(o.y), v[3] - bf16hi(o.y));
                     l.z = pack_bf16x2(v[4] - bf16lo(o.z), v[5] - bf16hi(o.z));
                     l.w = pack_bf16x2(v[6] - bf16lo(o.w), v[7] - bf16hi(o.w));
-                    *reinterpret_cast<uint4 *>(dst + (size_t)B * g.x_stride) = l;
+                    *reinterpret_cast<uint4 *>(dst + lo_off) = l;
                 }
             } else {
                 reinterpret_cast<float4 *>(dst)[0] = make_float4(v[0], v[1], v[2], v[3]);
@@ -278,136 +297,147 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
     const int rg_cta = rg1 - rg0;
     const int rounds = (((rg_cta + g.wr - 1) / g.wr) + g.rgc - 1) / g.rgc;
     const int sl_mine = seg - seg_lo;  // this warp's segment inside the CTA
+    // this lane's activation bytes for block j of the K-group: xlane + j * 128 * XES
+    const unsigned char *xlane =
+        xs + (size_t)gid * g.x_stride + ((size_t)(sl_mine * nbc + kb_lo - cblk_lo) * 128 + 8 * c) * T::XES;
     float acc[MMA ? 4 : 16];
 #pragma unroll
     for (int i = 0; i < (MMA ? 4 : 16); ++i) acc[i] = 0.f;
 
-    int f = 0;
-    for (int r = 0; r < rounds; ++r) {
-        const int k_end = min((r + 1) * g.rgc, nrg_w);
-        const int f_end = k_end * nit;
-        for (; f < f_end; ++f) {
-            if (f + 1 < nitems) load_item(wb, f + 1);
-            const int k = f / nit, it = f % nit;
+    // one block (8 rows x 128 columns) against the staged activations
+    auto compute = [&](const uint4 (&w)[NW], int j) {
+        const unsigned char *xp = xlane + (size_t)j * 128 * T::XES;
+        if constexpr (MODE == 0) {
 #pragma unroll
-            for (int bi = 0; bi < T::NBI; ++bi) {
-                const int blk = kb_lo + it * T::NBI + bi;
-                if (blk < kb_hi) {
-                    const int xcol = (sl_mine * nbc + (blk - cblk_lo)) * 128;
-                    if constexpr (MODE == 0) {
-#pragma unroll
-                        for (int m = 0; m < 4; ++m) {
-                            const size_t off = (size_t)(xcol + 32 * m + 8 * c) * 2;
-                            uint4 xa = gid < B ? lds128(xs + (size_t)gid * g.x_stride + off) : make_uint4(0, 0, 0, 0);
-                            uint4 xb = gid + 8 < B ? lds128(xs + (size_t)(gid + 8) * g.x_stride + off)
-                                                   : make_uint4(0, 0, 0, 0);
-                            const uint4 w = wa[bi * 4 + m];
-                            mma_bf16_16816(acc, xa.x, xb.x, xa.y, xb.y, w.x, w.y);
-                            mma_bf16_16816(acc, xa.z, xb.z, xa.w, xb.w, w.z, w.w);
-                        }
-                    } else if constexpr (MODE == 3) {
-                        const size_t lo_off = (size_t)B * g.x_stride;
-#pragma unroll
-                        for (int m = 0; m < 4; ++m) {
-                            const size_t off = (size_t)(xcol + 32 * m + 8 * c) * 2;
-                            const uint4 w = wa[bi * 4 + m];
-                            if (B <= 8) {
-                                // rows gid: hi of token gid, rows gid+8: lo of token gid
-                                uint4 xa = make_uint4(0, 0, 0, 0), xb = make_uint4(0, 0, 0, 0);
-                                if (gid < B) {
-                                    xa = lds128(xs + (size_t)gid * g.x_stride + off);
-                                    xb = lds128(xs + lo_off + (size_t)gid * g.x_stride + off);
-                                }
-                                mma_bf16_16816(acc, xa.x, xb.x, xa.y, xb.y, w.x, w.y);
-                                mma_bf16_16816(acc, xa.z, xb.z, xa.w, xb.w, w.z, w.w);
-                            } else {
-#pragma unroll
-                                for (int part_i = 0; part_i < 2; ++part_i) {
-                                    const size_t po = part_i ? lo_off : 0;
-                                    uint4 xa = lds128(xs + po + (size_t)gid * g.x_stride + off);
-                                    uint4 xb = gid + 8 < B ? lds128(xs + po + (size_t)(gid + 8) * g.x_stride + off)
-                                                           : make_uint4(0, 0, 0, 0);
-                                    mma_bf16_16816(acc, xa.x, xb.x, xa.y, xb.y, w.x, w.y);
-                                    mma_bf16_16816(acc, xa.z, xb.z, xa.w, xb.w, w.z, w.w);
-                                }
-                            }
-                        }
-                    } else {
-#pragma unroll
-                        for (int m = 0; m < 4; ++m) {
-                            float wv[8];
-                            if constexpr (T::WES == 4) {
-                                const uint4 w0 = wa[(bi * 4 + m) * 2], w1 = wa[(bi * 4 + m) * 2 + 1];
-                                wv[0] = __uint_as_float(w0.x); wv[1] = __uint_as_float(w0.y);
-                                wv[2] = __uint_as_float(w0.z); wv[3] = __uint_as_float(w0.w);
-                                wv[4] = __uint_as_float(w1.x); wv[5] = __uint_as_float(w1.y);
-                                wv[6] = __uint_as_float(w1.z); wv[7] = __uint_as_float(w1.w);
-                            } else {
-                                const uint4 w0 = wa[bi * 4 + m];
-                                wv[0] = bf16lo(w0.x); wv[1] = bf16hi(w0.x); wv[2] = bf16lo(w0.y); wv[3] = bf16hi(w0.y);
-                                wv[4] = bf16lo(w0.z); wv[5] = bf16hi(w0.z); wv[6] = bf16lo(w0.w); wv[7] = bf16hi(w0.w);
-                            }
-                            const size_t off = (size_t)(xcol + 32 * m + 8 * c) * T::XES;
-#pragma unroll
-                            for (int tok = 0; tok < 16; ++tok) {
-                                if (tok < B) {
-                                    float xv[8];
-                                    const unsigned char *xp = xs + (size_t)tok * g.x_stride + off;
-                                    if constexpr (T::XES == 4) {
-                                        const uint4 x0 = lds128(xp), x1 = lds128(xp + 16);
-                                        xv[0] = __uint_as_float(x0.x); xv[1] = __uint_as_float(x0.y);
-                                        xv[2] = __uint_as_float(x0.z); xv[3] = __uint_as_float(x0.w);
-                                        xv[4] = __uint_as_float(x1.x); xv[5] = __uint_as_float(x1.y);
-                                        xv[6] = __uint_as_float(x1.z); xv[7] = __uint_as_float(x1.w);
-                                    } else {
-                                        const uint4 x0 = lds128(xp);
-                                        xv[0] = bf16lo(x0.x); xv[1] = bf16hi(x0.x); xv[2] = bf16lo(x0.y); xv[3] = bf16hi(x0.y);
-                                        xv[4] = bf16lo(x0.z); xv[5] = bf16hi(x0.z); xv[6] = bf16lo(x0.w); xv[7] = bf16hi(x0.w);
-                                    }
-                                    float s = acc[tok];
-#pragma unroll
-                                    for (int e = 0; e < 8; ++e) s = fmaf(wv[e], xv[e], s);
-                                    acc[tok] = s;
-                                }
-                            }
-                        }
-                    }
-                }
+            for (int m = 0; m < 4; ++m) {
+                const uint4 xa = (BIG || gid < B) ? lds128(xp + 64 * m) : make_uint4(0, 0, 0, 0);
+                const uint4 xb = (BIG && gid + 8 < B) ? lds128(xp + 8 * g.x_stride + 64 * m) : make_uint4(0, 0, 0, 0);
+                mma_bf16_16816(acc, xa.x, xb.x, xa.y, xb.y, w[m].x, w[m].y);
+                mma_bf16_16816(acc, xa.z, xb.z, xa.w, xb.w, w[m].z, w[m].w);
             }
-            if (it == nit - 1) {
-                // row group done: write its partial sums for this K-group
-                const int pr = (wslot + (k - r * g.rgc) * g.wr) * 8;
-                float *pp = part + ((size_t)kgl * prows + pr) * B;
-                if constexpr (MMA) {
-                    if (XSPLIT && B <= 8) {
-                        // hi and lo halves of the same token
-                        acc[0] += acc[2];
-                        acc[1] += acc[3];
-                        acc[2] = acc[3] = 0.f;
-                    }
-                    if (gid < B) {
-                        pp[(2 * c) * B + gid] = acc[0];
-                        pp[(2 * c + 1) * B + gid] = acc[1];
-                    }
-                    if (gid + 8 < B) {
-                        pp[(2 * c) * B + gid + 8] = acc[2];
-                        pp[(2 * c + 1) * B + gid + 8] = acc[3];
-                    }
+        } else if constexpr (MODE == 3) {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) acc[i] = 0.f;
+            for (int m = 0; m < 4; ++m) {
+                if constexpr (!BIG) {
+                    // rows gid: hi of token gid, rows gid+8: lo of token gid
+                    uint4 xa = make_uint4(0, 0, 0, 0), xb = make_uint4(0, 0, 0, 0);
+                    if (gid < B) {
+                        xa = lds128(xp + 64 * m);
+                        xb = lds128(xp + lo_off + 64 * m);
+                    }
+                    mma_bf16_16816(acc, xa.x, xb.x, xa.y, xb.y, w[m].x, w[m].y);
+                    mma_bf16_16816(acc, xa.z, xb.z, xa.w, xb.w, w[m].z, w[m].w);
                 } else {
 #pragma unroll
-                    for (int tok = 0; tok < 16; ++tok) {
-                        float s = acc[tok];
-                        s += __shfl_xor_sync(0xffffffffu, s, 1);
-                        s += __shfl_xor_sync(0xffffffffu, s, 2);
-                        if (tok < B && (tok & 3) == c) pp[gid * B + tok] = s;
-                        acc[tok] = 0.f;
+                    for (int part_i = 0; part_i < 2; ++part_i) {
+                        const unsigned char *pp = xp + (part_i ? lo_off : 0) + 64 * m;
+                        const uint4 xa = lds128(pp);
+                        const uint4 xb = gid + 8 < B ? lds128(pp + 8 * g.x_stride) : make_uint4(0, 0, 0, 0);
+                        mma_bf16_16816(acc, xa.x, xb.x, xa.y, xb.y, w[m].x, w[m].y);
+                        mma_bf16_16816(acc, xa.z, xb.z, xa.w, xb.w, w[m].z, w[m].w);
                     }
                 }
             }
+        } else {
+            // FFMA: lane (gid, c) owns row gid, columns 32m + 8c .. +8
+            const unsigned char *xt = xp - (size_t)gid * g.x_stride;  // token rows start here
 #pragma unroll
-            for (int i = 0; i < NW; ++i) wa[i] = wb[i];
+            for (int m = 0; m < 4; ++m) {
+                float wv[8];
+                if constexpr (T::WES == 4) {
+                    const uint4 w0 = w[m * 2], w1 = w[m * 2 + 1];
+                    wv[0] = __uint_as_float(w0.x); wv[1] = __uint_as_float(w0.y);
+                    wv[2] = __uint_as_float(w0.z); wv[3] = __uint_as_float(w0.w);
+                    wv[4] = __uint_as_float(w1.x); wv[5] = __uint_as_float(w1.y);
+                    wv[6] = __uint_as_float(w1.z); wv[7] = __uint_as_float(w1.w);
+                } else {
+                    const uint4 w0 = w[m];
+                    wv[0] = bf16lo(w0.x); wv[1] = bf16hi(w0.x); wv[2] = bf16lo(w0.y); wv[3] = bf16hi(w0.y);
+                    wv[4] = bf16lo(w0.z); wv[5] = bf16hi(w0.z); wv[6] = bf16lo(w0.w); wv[7] = bf16hi(w0.w);
+                }
+#pragma unroll
+                for (int tok = 0; tok < 16; ++tok) {
+                    if (tok < B) {
+                        float xv[8];
+                        const unsigned char *xq = xt + (size_t)tok * g.x_stride + 32 * m * T::XES;
+                        if constexpr (T::XES == 4) {
+                            const uint4 x0 = lds128(xq), x1 = lds128(xq + 16);
+                            xv[0] = __uint_as_float(x0.x); xv[1] = __uint_as_float(x0.y);
+                            xv[2] = __uint_as_float(x0.z); xv[3] = __uint_as_float(x0.w);
+                            xv[4] = __uint_as_float(x1.x); xv[5] = __uint_as_float(x1.y);
+                            xv[6] = __uint_as_float(x1.z); xv[7] = __uint_as_float(x1.w);
+                        } else {
+                            const uint4 x0 = lds128(xq);
+                            xv[0] = bf16lo(x0.x); xv[1] = bf16hi(x0.x); xv[2] = bf16lo(x0.y); xv[3] = bf16hi(x0.y);
+                            xv[4] = bf16lo(x0.z); xv[5] = bf16hi(x0.z); xv[6] = bf16lo(x0.w); xv[7] = bf16hi(x0.w);
+                        }
+                        float sacc = acc[tok];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) sacc = fmaf(wv[e], xv[e], sacc);
+                        acc[tok] = sacc;
+                    }
+                }
+            }
+        }
+    };
+
+    // partial sums of one finished row group for this K-group
+    auto write_part = [&](int r, int k) {
+        const int pr = (wslot + (k - r * g.rgc) * g.wr) * 8;
+        float *pp = part + ((size_t)kgl * prows + pr) * B;
+        if constexpr (MMA) {
+            if (XSPLIT && !BIG) {
+                // hi and lo halves of the same token
+                acc[0] += acc[2];
+                acc[1] += acc[3];
+                acc[2] = acc[3] = 0.f;
+            }
+            if (gid < B) {
+                pp[(2 * c) * B + gid] = acc[0];
+                pp[(2 * c + 1) * B + gid] = acc[1];
+            }
+            if (BIG && gid + 8 < B) {
+                pp[(2 * c) * B + gid + 8] = acc[2];
+                pp[(2 * c + 1) * B + gid + 8] = acc[3];
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[i] = 0.f;
+        } else {
+#pragma unroll
+            for (int tok = 0; tok < 16; ++tok) {
+                float sacc = acc[tok];
+                sacc += __shfl_xor_sync(0xffffffffu, sacc, 1);
+                sacc += __shfl_xor_sync(0xffffffffu, sacc, 2);
+                if (tok < B && (tok & 3) == c) pp[gid * B + tok] = sacc;
+                acc[tok] = 0.f;
+            }
+        }
+    };
+
+    int i = 0;          // next block to consume
+    int cr = 0, cj = 0; // its row group and block within the K-group
+    for (int r = 0; r < rounds; ++r) {
+        const int k_end = min((r + 1) * g.rgc, nrg_w);
+        if (nblk == 0) {
+            // an empty K-group contributes zeros
+            for (int k = r * g.rgc; k < k_end; ++k) write_part(r, k);
+        }
+        const int i_end = k_end * nblk;
+        // rounds hold a multiple of D blocks (rgc is a multiple of 4), so the
+        // ring slot of block i is always i % D
+        for (; i < i_end; i += D) {
+#pragma unroll
+            for (int d = 0; d < D; ++d) {
+                if (i + d < i_end) {
+                    compute(ring[d], cj);
+                    if (i + d + D < T_blocks) load_next(ring[d]);
+                    if (++cj == nblk) {
+                        write_part(r, cr);
+                        cj = 0;
+                        ++cr;
+                    }
+                }
+            }
         }
         __syncthreads();
         // ---- round epilogue: fixed-order sums over K-groups per segment ----
@@ -438,9 +468,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
                     const int row = rbase + prow;
                     SegSums ss;
                     for (int sl = 0; sl < g.segs_per_cta; ++sl) {
-                        float s = 0.f;
-                        for (int kg = sl * kpc; kg < (sl + 1) * kpc; ++kg) s += part[((size_t)kg * prows + prow) * B + tok];
-                        ss.p[sl] = s;
+                        float sv = 0.f;
+                        for (int kg = sl * kpc; kg < (sl + 1) * kpc; ++kg) sv += part[((size_t)kg * prows + prow) * B + tok];
+                        ss.p[sl] = sv;
                     }
                     if (pr_ok) {
                         gemv_final_row(a, row, tok, ss);

@@ -37,6 +37,7 @@ struct tpl_plan {
     int t;
     int nq_s, nkv_s, F_s, g, qkv_rows_s, esize;
     bool f32;
+    int ld_h, ld_o, ld_f;                   // padded row lengths: hidden, n_q*d/t, ffn/t
     int64_t blk_qkv, blk_o, blk_gu, blk_d;  // byte stride between shard blocks
     int64_t off_qkv, off_o, off_gu, off_d, off_g1, off_g2, packed_bytes;
     std::atomic<long long> reductions;

@@ -79,8 +79,11 @@ int gemv_geom(int N, int nseg, int Kseg, int B, int xbytes, int num_sms, GemvGeo
     g->rb = rb;
     int rg_cta = (g->ng + rb - 1) / rb;
     int rg_warp = (rg_cta + g->wr - 1) / g->wr;
+    // Rounds of row groups per warp: one round when the partial sums fit,
+    // else a multiple of 4 (the kernel's register ring holds 4 blocks and a
+    // round must hold a multiple of that).
     int rgc_cap = (int)(kPartSmemMax / ((size_t)kGemvWarps * 8 * B * 4));
-    g->rgc = std::max(1, std::min(rg_warp, rgc_cap));
+    g->rgc = rg_warp <= rgc_cap ? std::max(1, rg_warp) : std::max(4, rgc_cap / 4 * 4);
     g->x_stride = m * blocks * 128 * xbytes + 64;
     size_t part = (size_t)kGemvWarps * g->rgc * 8 * B * 4;
     g->smem = (size_t)xparts * B * g->x_stride + part + 128;
@@ -185,10 +188,14 @@ int tpl_plan_create(const tpl_dims *dims, int32_t t, tpl_plan **out) {
     p->esize = p->f32 ? 4 : 2;
     p->gemv_mode = p->f32 ? 1 : 0;
     const int64_t H = dims->hidden, es = p->esize;
-    p->blk_qkv = align_up((int64_t)p->qkv_rows_s * H * es, 256);
-    p->blk_o = align_up(H * p->nq_s * dims->head_dim * es, 256);
-    p->blk_gu = align_up((int64_t)2 * p->F_s * H * es, 256);
-    p->blk_d = align_up(H * p->F_s * es, 256);
+    // rows padded with zeros to whole 128-column blocks
+    p->ld_h = (int)align_up(H, 128);
+    p->ld_o = (int)align_up((int64_t)p->nq_s * dims->head_dim, 128);
+    p->ld_f = (int)align_up(p->F_s, 128);
+    p->blk_qkv = align_up((int64_t)p->qkv_rows_s * p->ld_h * es, 256);
+    p->blk_o = align_up(H * p->ld_o * es, 256);
+    p->blk_gu = align_up((int64_t)2 * p->F_s * p->ld_h * es, 256);
+    p->blk_d = align_up(H * p->ld_f * es, 256);
     int64_t off = 0;
     p->off_qkv = off;
     off += t * p->blk_qkv;

@@ -19,7 +19,8 @@
 //   O += P V   -- A = P from the S accumulators (register reuse), B = V with
 //                 output column n of tile t mapped to head_dim 16n + t, so a
 //                 lane's V operands are 32 contiguous bytes per key.
-// K and V are streamed straight from HBM with 16-byte loads.
+// K and V are streamed straight from HBM with 16-byte loads, double-buffered:
+// the next 16 keys load while the current 16 are processed.
 #pragma once
 
 #include "tpl_common.cuh"
@@ -101,30 +102,31 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const __gr
     float m_a = -INFINITY, m_b = -INFINITY;  // running max of rows gid, gid+8 (log2 domain)
     float l_a = 0.f, l_b = 0.f;              // lane-partial running sums
 
-    for (int64_t kb = k0; kb < k1; kb += 16) {
-        // ---- K operands: keys kb+gid (tile 0) and kb+8+gid (tile 1) ----
-        uint4 kt0[4], kt1[4];
-        {
-            const int64_t key0 = kb + gid, key1 = kb + 8 + gid;
+    // K/V operands of 16 keys: K rows kb+gid (tile 0) and kb+8+gid (tile 1),
+    // V rows kb+2c, kb+2c+1, kb+8+2c, kb+9+2c at head_dim 16*gid .. +16.
+    struct KV16 {
+        uint4 kt0[4], kt1[4], va[2], vb[2], vc2[2], vd[2];
+    };
+    auto load16 = [&](KV16 &f, int64_t kb) {
+        const int64_t key0 = kb + gid, key1 = kb + 8 + gid;
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                kt0[m] = key0 < k1 ? ldg_stream(Kp + key0 * D + 32 * m + 8 * c) : make_uint4(0, 0, 0, 0);
-                kt1[m] = key1 < k1 ? ldg_stream(Kp + key1 * D + 32 * m + 8 * c) : make_uint4(0, 0, 0, 0);
-            }
+        for (int m = 0; m < 4; ++m) {
+            f.kt0[m] = key0 < k1 ? ldg_stream(Kp + key0 * D + 32 * m + 8 * c) : make_uint4(0, 0, 0, 0);
+            f.kt1[m] = key1 < k1 ? ldg_stream(Kp + key1 * D + 32 * m + 8 * c) : make_uint4(0, 0, 0, 0);
         }
-        // ---- V operands: keys kb+2c, kb+2c+1, kb+8+2c, kb+9+2c; head_dim 16*gid .. +16 ----
-        uint4 va[2], vb[2], vc2[2], vd[2];
-        {
-            const int64_t ka = kb + 2 * c, kbb = ka + 1, kc_ = ka + 8, kd = ka + 9;
+        const int64_t ka = kb + 2 * c, kbb = ka + 1, kc_ = ka + 8, kd = ka + 9;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int col = 16 * gid + 8 * h;
-                va[h] = ka < k1 ? ldg_stream(Vp + ka * D + col) : make_uint4(0, 0, 0, 0);
-                vb[h] = kbb < k1 ? ldg_stream(Vp + kbb * D + col) : make_uint4(0, 0, 0, 0);
-                vc2[h] = kc_ < k1 ? ldg_stream(Vp + kc_ * D + col) : make_uint4(0, 0, 0, 0);
-                vd[h] = kd < k1 ? ldg_stream(Vp + kd * D + col) : make_uint4(0, 0, 0, 0);
-            }
+        for (int h = 0; h < 2; ++h) {
+            const int col = 16 * gid + 8 * h;
+            f.va[h] = ka < k1 ? ldg_stream(Vp + ka * D + col) : make_uint4(0, 0, 0, 0);
+            f.vb[h] = kbb < k1 ? ldg_stream(Vp + kbb * D + col) : make_uint4(0, 0, 0, 0);
+            f.vc2[h] = kc_ < k1 ? ldg_stream(Vp + kc_ * D + col) : make_uint4(0, 0, 0, 0);
+            f.vd[h] = kd < k1 ? ldg_stream(Vp + kd * D + col) : make_uint4(0, 0, 0, 0);
         }
+    };
+    auto process = [&](const KV16 &f, int64_t kb) {
+        const uint4 *kt0 = f.kt0, *kt1 = f.kt1;
+        const uint4 *va = f.va, *vb = f.vb, *vc2 = f.vc2, *vd = f.vd;
         // ---- scores: s0 keys kb+2c, +1 (tile 0), s1 keys kb+8+2c, +1 (tile 1) ----
         float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
         if constexpr (PACKED) {
@@ -214,6 +216,16 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const __gr
                 mma_bf16_16816(o[t], pl0, rl0, pl2, rl2, vb0, vb1);
             }
         }
+    };
+    // two buffers: the next 16 keys load while the current 16 are processed
+    KV16 bufA, bufB;
+    if (k0 < k1) load16(bufA, k0);
+    for (int64_t kb = k0; kb < k1; kb += 32) {
+        if (kb + 16 < k1) load16(bufB, kb + 16);
+        process(bufA, kb);
+        if (kb + 16 >= k1) break;
+        if (kb + 32 < k1) load16(bufA, kb + 32);
+        process(bufB, kb + 16);
     }
     if constexpr (PACKED) {
         // rows gid+8 held the P_lo . V half of the same head

@@ -28,6 +28,8 @@ __device__ __forceinline__ uint4 ldg_stream(const void *p) {
     return r;
 }
 
+__device__ __forceinline__ void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+
 __device__ __forceinline__ uint4 lds128(const void *p) {
     uint4 r;
     unsigned a = (unsigned)__cvta_generic_to_shared(p);

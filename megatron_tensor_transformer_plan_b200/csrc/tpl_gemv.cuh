@@ -17,7 +17,8 @@
 //
 // Inner product modes:
 // Weight rows are padded to whole 128-column blocks in the packed layout, and
-// each warp keeps four blocks of loads in flight in a register ring.
+// each warp keeps two blocks of loads in flight in a register ring (deeper
+// rings measured slower: register pressure).
 //
 //   MODE 0 -- bf16 weights on the tensor cores (mma.sync m16n8k16): the
 //             activation tile is the A operand (tokens as rows), 8 weight rows
@@ -39,6 +40,8 @@
 namespace tpl {
 
 enum { EPI_QKV = 0, EPI_GU = 1, EPI_ROW = 2, EPI_ROW_PARTIAL = 3 };
+
+constexpr int kPrefetchBlocks = 8;  // blocks per warp prefetched into L2 before the dependency wait
 
 struct GemvArgs {
     const char *W;   // first weight block
@@ -134,7 +137,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
     using T = GemvTraits<MODE>;
     constexpr bool XSPLIT = MODE == 3;
     constexpr bool MMA = MODE == 0 || MODE == 3;
-    constexpr int D = MODE == 1 ? 2 : 4;       // blocks in flight per warp (register ring)
+    constexpr int D = 2;                       // blocks in flight per warp (register ring)
     constexpr int NW = 4 * T::LPM;             // uint4 per block per lane
     constexpr int BLK_BYTES = 128 * T::WES;    // one 128-column block of one row
     extern __shared__ __align__(128) unsigned char smem[];
@@ -196,39 +199,100 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
             lptr += BLK_BYTES;
         }
     };
-    // Issue the first weight loads before waiting on the previous kernel.
+    // Issue the first weight loads before waiting on the previous kernel, and
+    // prefetch the next kPrefetchBlocks blocks of this warp's stream into L2
+    // (each block: 8 rows x 128 columns; lanes with c == 0 cover both 128-byte
+    // lines of their row).
 #pragma unroll
     for (int d = 0; d < D; ++d)
         if (d < T_blocks) load_next(ring[d]);
+    {
+        int pr = lr, pj = lj;
+        const char *pp = lptr;
+        for (int q = 0; q < kPrefetchBlocks && pr < nrg_w && D + q < T_blocks; ++q) {
+            if (c == 0) {
+                prefetch_l2(pp);
+                prefetch_l2(pp + 64 * T::WES);
+                if (T::WES == 4) {
+                    prefetch_l2(pp + 128 * 2);
+                    prefetch_l2(pp + 128 * 3);
+                }
+            }
+            if (++pj == nblk) {
+                pj = 0;
+                if (++pr < nrg_w) pp = rowptr(pr);
+            } else {
+                pp += BLK_BYTES;
+            }
+        }
+    }
     pdl_wait();
     pdl_trigger();
 
     // ---- stage the activation slice (normalised if requested) ----
+    // Loads are issued in batches of 8 independent 8-element chunks per
+    // thread, so each pass costs about one L2 round trip.
+    auto load8 = [&](int64_t src, float (&v)[8]) {
+        if (a.x_f32) {
+            const float4 *p4 = reinterpret_cast<const float4 *>(static_cast<const float *>(a.x) + src);
+            const float4 x0 = p4[0], x1 = p4[1];
+            v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w;
+            v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
+        } else {
+            const uint4 r4 = *reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(a.x) + src);
+            v[0] = bf16lo(r4.x); v[1] = bf16hi(r4.x); v[2] = bf16lo(r4.y); v[3] = bf16hi(r4.y);
+            v[4] = bf16lo(r4.z); v[5] = bf16hi(r4.z); v[6] = bf16lo(r4.w); v[7] = bf16hi(r4.w);
+        }
+    };
     if (a.norm) {
-        // inverse RMS over the full row of each token, fixed-order reduction
-        float *s_red = part;  // scratch, [16 warps][B]
-        const int nch = a.ldx / 8;
-        for (int tok = 0; tok < B; ++tok) {
-            float ss = 0.f;
-            for (int i = tid; i < nch; i += kGemvThreads) {
-                float v[8];
-                const int64_t src = (int64_t)tok * a.ldx + (int64_t)i * 8;
-                if (a.x_f32) {
-                    const float4 *p4 = reinterpret_cast<const float4 *>(static_cast<const float *>(a.x) + src);
-                    const float4 x0 = p4[0], x1 = p4[1];
-                    v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w;
-                    v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
-                } else {
-                    const uint4 r4 = *reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(a.x) + src);
-                    v[0] = bf16lo(r4.x); v[1] = bf16hi(r4.x); v[2] = bf16lo(r4.y); v[3] = bf16hi(r4.y);
-                    v[4] = bf16lo(r4.z); v[5] = bf16hi(r4.z); v[6] = bf16lo(r4.w); v[7] = bf16hi(r4.w);
+        // inverse RMS over the full row of each token, fixed-order reduction:
+        // chunk u = tid + 512*k of token u / cpt; with cpt a multiple of 32 a
+        // warp's chunk k belongs to one token.
+        const int cpt = a.ldx / 8;
+        float *s_red = part;  // scratch: [16 warps][B] per-warp sums
+        if ((cpt & 31) == 0) {
+            for (int i = tid; i < kGemvWarps * B; i += kGemvThreads) s_red[i] = 0.f;
+            __syncthreads();
+            const int total = B * cpt;
+            for (int u0 = 0; u0 < total; u0 += 8 * kGemvThreads) {
+                float sq[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const int u = u0 + k * kGemvThreads + tid;
+                    float v[8];
+                    if (u < total) {
+                        load8((int64_t)(u / cpt) * a.ldx + (int64_t)(u % cpt) * 8, v);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) v[e] = 0.f;
+                    }
+                    float acc2 = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) acc2 += v[e] * v[e];
+                    sq[k] = acc2;
                 }
 #pragma unroll
-                for (int e = 0; e < 8; ++e) ss += v[e] * v[e];
-            }
+                for (int k = 0; k < 8; ++k) {
+                    float v = sq[k];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-            if (lane == 0) s_red[warp * B + tok] = ss;
+                    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                    const int u = u0 + k * kGemvThreads + warp * 32;
+                    if (lane == 0 && u < total) s_red[warp * B + u / cpt] += v;  // one writer per (warp, token)
+                }
+            }
+        } else {
+            for (int tok = 0; tok < B; ++tok) {
+                float ss = 0.f;
+                for (int i = tid; i < cpt; i += kGemvThreads) {
+                    float v[8];
+                    load8((int64_t)tok * a.ldx + (int64_t)i * 8, v);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) ss += v[e] * v[e];
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+                if (lane == 0) s_red[warp * B + tok] = ss;
+            }
         }
         __syncthreads();
         if (tid < B) {
@@ -240,54 +304,63 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
     }
     {
         const int chunks_per_tok = g.segs_per_cta * nbc * 16;  // 8-element chunks
-        for (int u = tid; u < B * chunks_per_tok; u += kGemvThreads) {
-            const int tok = u / chunks_per_tok, r = u % chunks_per_tok;
-            const int sl = r / (nbc * 16), rr = r % (nbc * 16);
-            const int blk = cblk_lo + rr / 16, j = rr % 16;
-            const int k = blk * 128 + j * 8;
-            const int sg = seg_lo + sl;
-            float v[8];
-            if (k < g.Kseg) {
-                const int64_t src = (int64_t)tok * a.ldx + (int64_t)sg * g.Kseg + k;
-                if (a.x_f32) {
-                    const float4 *p4 = reinterpret_cast<const float4 *>(static_cast<const float *>(a.x) + src);
-                    float4 x0 = p4[0], x1 = p4[1];
-                    v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w;
-                    v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
-                } else {
-                    uint4 r4 = *reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(a.x) + src);
-                    v[0] = bf16lo(r4.x); v[1] = bf16hi(r4.x); v[2] = bf16lo(r4.y); v[3] = bf16hi(r4.y);
-                    v[4] = bf16lo(r4.z); v[5] = bf16hi(r4.z); v[6] = bf16lo(r4.w); v[7] = bf16hi(r4.w);
+        const int total = B * chunks_per_tok;
+        for (int u0 = 0; u0 < total; u0 += 4 * kGemvThreads) {
+            float v[4][8];
+            int uu[4], kk[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int u = u0 + q * kGemvThreads + tid;
+                uu[q] = u;
+                kk[q] = -1;
+                if (u < total) {
+                    const int tok = u / chunks_per_tok, r = u % chunks_per_tok;
+                    const int sl = r / (nbc * 16), rr = r % (nbc * 16);
+                    const int k = (cblk_lo + rr / 16) * 128 + (rr % 16) * 8;
+                    if (k < g.Kseg) {
+                        load8((int64_t)tok * a.ldx + (int64_t)(seg_lo + sl) * g.Kseg + k, v[q]);
+                        kk[q] = k;
+                    }
                 }
-                if (a.norm) {
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int u = uu[q];
+                if (u >= total) continue;
+                const int tok = u / chunks_per_tok, r = u % chunks_per_tok;
+                const int sl = r / (nbc * 16), rr = r % (nbc * 16);
+                const int blk = cblk_lo + rr / 16, j = rr % 16;
+                const int k = kk[q];
+                if (k < 0) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) v[q][e] = 0.f;
+                } else if (a.norm) {
                     const float inv = s_inv[tok];
                     const float4 g0 = reinterpret_cast<const float4 *>(a.gamma + k)[0];
                     const float4 g1 = reinterpret_cast<const float4 *>(a.gamma + k)[1];
                     const float gm[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) v[e] = v[e] * inv * gm[e];
+                    for (int e = 0; e < 8; ++e) v[q][e] = v[q][e] * inv * gm[e];
                 }
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) v[e] = 0.f;
-            }
-            unsigned char *dst = xs + (size_t)tok * g.x_stride + (size_t)((sl * nbc + (blk - cblk_lo)) * 128 + j * 8) * T::XES;
-            if (T::XES == 2) {
-                uint4 o;
-                o.x = pack_bf16x2(v[0], v[1]); o.y = pack_bf16x2(v[2], v[3]);
-                o.z = pack_bf16x2(v[4], v[5]); o.w = pack_bf16x2(v[6], v[7]);
-                *reinterpret_cast<uint4 *>(dst) = o;
-                if constexpr (XSPLIT) {
-                    uint4 l;
-                    l.x = pack_bf16x2(v[0] - bf16lo(o.x), v[1] - bf16hi(o.x));
-                    l.y = pack_bf16x2(v[2] - bf16lo(o.y), v[3] - bf16hi(o.y));
-                    l.z = pack_bf16x2(v[4] - bf16lo(o.z), v[5] - bf16hi(o.z));
-                    l.w = pack_bf16x2(v[6] - bf16lo(o.w), v[7] - bf16hi(o.w));
-                    *reinterpret_cast<uint4 *>(dst + lo_off) = l;
+                unsigned char *dst =
+                    xs + (size_t)tok * g.x_stride + (size_t)((sl * nbc + (blk - cblk_lo)) * 128 + j * 8) * T::XES;
+                if (T::XES == 2) {
+                    uint4 o;
+                    o.x = pack_bf16x2(v[q][0], v[q][1]); o.y = pack_bf16x2(v[q][2], v[q][3]);
+                    o.z = pack_bf16x2(v[q][4], v[q][5]); o.w = pack_bf16x2(v[q][6], v[q][7]);
+                    *reinterpret_cast<uint4 *>(dst) = o;
+                    if constexpr (XSPLIT) {
+                        uint4 l;
+                        l.x = pack_bf16x2(v[q][0] - bf16lo(o.x), v[q][1] - bf16hi(o.x));
+                        l.y = pack_bf16x2(v[q][2] - bf16lo(o.y), v[q][3] - bf16hi(o.y));
+                        l.z = pack_bf16x2(v[q][4] - bf16lo(o.z), v[q][5] - bf16hi(o.z));
+                        l.w = pack_bf16x2(v[q][6] - bf16lo(o.w), v[q][7] - bf16hi(o.w));
+                        *reinterpret_cast<uint4 *>(dst + lo_off) = l;
+                    }
+                } else {
+                    reinterpret_cast<float4 *>(dst)[0] = make_float4(v[q][0], v[q][1], v[q][2], v[q][3]);
+                    reinterpret_cast<float4 *>(dst)[1] = make_float4(v[q][4], v[q][5], v[q][6], v[q][7]);
                 }
-            } else {
-                reinterpret_cast<float4 *>(dst)[0] = make_float4(v[0], v[1], v[2], v[3]);
-                reinterpret_cast<float4 *>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
             }
         }
     }

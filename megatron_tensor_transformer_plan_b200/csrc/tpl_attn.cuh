@@ -64,8 +64,10 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const __gr
     const int64_t k0 = (int64_t)split * a.kps;
     const int64_t k1 = min(a.keys, k0 + a.kps);
 
-    pdl_wait();
-    pdl_trigger();
+    // With the new token given separately the splits read cache positions
+    // 0..S-1 only, which the preceding kernel (it writes position S) does not
+    // touch: start streaming them before waiting on it.
+    const bool early = a.k_new != nullptr;
 
     // Q operands.  Each query value is carried as a bf16 pair hi + lo
     // (lo = q - hi), so the logits keep ~16 mantissa bits.  With g <= 8 the
@@ -91,17 +93,6 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const __gr
             }
         }
     };
-    if (gid < a.g) load_q(gid, qh0, ql0);
-    if constexpr (!PACKED) {
-        if (gid + 8 < a.g) load_q(gid + 8, qh1, ql1);
-    }
-
-    float o[16][4];
-#pragma unroll
-    for (int t = 0; t < 16; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
-    float m_a = -INFINITY, m_b = -INFINITY;  // running max of rows gid, gid+8 (log2 domain)
-    float l_a = 0.f, l_b = 0.f;              // lane-partial running sums
-
     // K/V operands of 16 keys: K rows kb+gid (tile 0) and kb+8+gid (tile 1),
     // V rows kb+2c, kb+2c+1, kb+8+2c, kb+9+2c at head_dim 16*gid .. +16.
     struct KV16 {
@@ -124,6 +115,23 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const __gr
             f.vd[h] = kd < k1 ? ldg_stream(Vp + kd * D + col) : make_uint4(0, 0, 0, 0);
         }
     };
+    KV16 bufA, bufB;
+    if (early && k0 < k1) load16(bufA, k0);
+    pdl_wait();
+    pdl_trigger();
+    if (!early && k0 < k1) load16(bufA, k0);
+
+    if (gid < a.g) load_q(gid, qh0, ql0);
+    if constexpr (!PACKED) {
+        if (gid + 8 < a.g) load_q(gid + 8, qh1, ql1);
+    }
+
+    float o[16][4];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
+    float m_a = -INFINITY, m_b = -INFINITY;  // running max of rows gid, gid+8 (log2 domain)
+    float l_a = 0.f, l_b = 0.f;              // lane-partial running sums
+
     auto process = [&](const KV16 &f, int64_t kb) {
         const uint4 *kt0 = f.kt0, *kt1 = f.kt1;
         const uint4 *va = f.va, *vb = f.vb, *vc2 = f.vc2, *vd = f.vd;
@@ -218,8 +226,6 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const __gr
         }
     };
     // two buffers: the next 16 keys load while the current 16 are processed
-    KV16 bufA, bufB;
-    if (k0 < k1) load16(bufA, k0);
     for (int64_t kb = k0; kb < k1; kb += 32) {
         if (kb + 16 < k1) load16(bufB, kb + 16);
         process(bufA, kb);

@@ -230,8 +230,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
     pdl_trigger();
 
     // ---- stage the activation slice (normalised if requested) ----
-    // Loads are issued in batches of 8 independent 8-element chunks per
-    // thread, so each pass costs about one L2 round trip.
+    // Each token gets a power-of-two group of tpt threads (512 / next pow2 of
+    // B), so chunk coordinates are shifts and masks.  A chunk is 8 elements.
     auto load8 = [&](int64_t src, float (&v)[8]) {
         if (a.x_f32) {
             const float4 *p4 = reinterpret_cast<const float4 *>(static_cast<const float *>(a.x) + src);
@@ -244,122 +244,162 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
             v[4] = bf16lo(r4.z); v[5] = bf16hi(r4.z); v[6] = bf16lo(r4.w); v[7] = bf16hi(r4.w);
         }
     };
-    if (a.norm) {
-        // inverse RMS over the full row of each token, fixed-order reduction:
-        // chunk u = tid + 512*k of token u / cpt; with cpt a multiple of 32 a
-        // warp's chunk k belongs to one token.
-        const int cpt = a.ldx / 8;
-        float *s_red = part;  // scratch: [16 warps][B] per-warp sums
-        if ((cpt & 31) == 0) {
-            for (int i = tid; i < kGemvWarps * B; i += kGemvThreads) s_red[i] = 0.f;
-            __syncthreads();
-            const int total = B * cpt;
-            for (int u0 = 0; u0 < total; u0 += 8 * kGemvThreads) {
-                float sq[8];
+    // store one normalised chunk (tok, smem column col) as bf16 (+ lo part) or fp32
+    auto store8 = [&](int tok, int col, const float (&v)[8]) {
+        unsigned char *dst = xs + (size_t)tok * g.x_stride + (size_t)col * T::XES;
+        if (T::XES == 2) {
+            uint4 o;
+            o.x = pack_bf16x2(v[0], v[1]); o.y = pack_bf16x2(v[2], v[3]);
+            o.z = pack_bf16x2(v[4], v[5]); o.w = pack_bf16x2(v[6], v[7]);
+            *reinterpret_cast<uint4 *>(dst) = o;
+            if constexpr (XSPLIT) {
+                uint4 l;
+                l.x = pack_bf16x2(v[0] - bf16lo(o.x), v[1] - bf16hi(o.x));
+                l.y = pack_bf16x2(v[2] - bf16lo(o.y), v[3] - bf16hi(o.y));
+                l.z = pack_bf16x2(v[4] - bf16lo(o.z), v[5] - bf16hi(o.z));
+                l.w = pack_bf16x2(v[6] - bf16lo(o.w), v[7] - bf16hi(o.w));
+                *reinterpret_cast<uint4 *>(dst + lo_off) = l;
+            }
+        } else {
+            reinterpret_cast<float4 *>(dst)[0] = make_float4(v[0], v[1], v[2], v[3]);
+            reinterpret_cast<float4 *>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
+        }
+    };
+    auto scale8 = [&](int k, float inv, float (&v)[8]) {
+        const float4 g0 = __ldg(reinterpret_cast<const float4 *>(a.gamma + k));
+        const float4 g1 = __ldg(reinterpret_cast<const float4 *>(a.gamma + k) + 1);
+        v[0] *= inv * g0.x; v[1] *= inv * g0.y; v[2] *= inv * g0.z; v[3] *= inv * g0.w;
+        v[4] *= inv * g1.x; v[5] *= inv * g1.y; v[6] *= inv * g1.z; v[7] *= inv * g1.w;
+    };
+    const int lgBp = B <= 1 ? 0 : 32 - __clz(B - 1);  // log2 of the next power of two >= B
+    const int lg_tpt = 9 - lgBp;                       // kGemvThreads = 512 = 2^9
+    const int tpt = 1 << lg_tpt, tok_me = tid >> lg_tpt, lt = tid & (tpt - 1);
+    const bool tok_ok = tok_me < B;
+    const int64_t xrow = (int64_t)tok_me * a.ldx;
+    const int chunks_seg = nbc * 16;                   // staged chunks per segment
+    float *s_red = part;                               // scratch: per-warp sums of squares
+    const int wpt = tpt >> 5;                          // warps per token
+    // full-row, one-pass case: column-parallel, whole row staged, the raw
+    // loads held in 32 registers (8 bf16 chunks or 4 fp32 chunks per thread)
+    const int cpt_full = a.ldx >> 3;
+    const int hold = a.x_f32 ? 4 : 8;
+    const bool one_pass = a.norm && g.nseg == 1 && g.ksplit == 1 && cpt_full <= hold * tpt;
+    if (one_pass) {
+        uint4 raw[8];  // bf16: 8 chunks; fp32: 4 chunks as pairs (raw[2q], raw[2q+1])
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const int u = u0 + k * kGemvThreads + tid;
-                    float v[8];
-                    if (u < total) {
-                        load8((int64_t)(u / cpt) * a.ldx + (int64_t)(u % cpt) * 8, v);
-                    } else {
+        for (int q = 0; q < 8; ++q) raw[q] = make_uint4(0, 0, 0, 0);
+        if (a.x_f32) {
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) v[e] = 0.f;
-                    }
-                    float acc2 = 0.f;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) acc2 += v[e] * v[e];
-                    sq[k] = acc2;
-                }
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    float v = sq[k];
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                    const int u = u0 + k * kGemvThreads + warp * 32;
-                    if (lane == 0 && u < total) s_red[warp * B + u / cpt] += v;  // one writer per (warp, token)
+            for (int q = 0; q < 4; ++q) {
+                const int c16 = lt + q * tpt;
+                if (tok_ok && c16 < cpt_full) {
+                    const uint4 *p4 = reinterpret_cast<const uint4 *>(static_cast<const float *>(a.x) + xrow + (int64_t)c16 * 8);
+                    raw[2 * q] = p4[0];
+                    raw[2 * q + 1] = p4[1];
                 }
             }
         } else {
-            for (int tok = 0; tok < B; ++tok) {
-                float ss = 0.f;
-                for (int i = tid; i < cpt; i += kGemvThreads) {
-                    float v[8];
-                    load8((int64_t)tok * a.ldx + (int64_t)i * 8, v);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) ss += v[e] * v[e];
-                }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-                if (lane == 0) s_red[warp * B + tok] = ss;
+            for (int q = 0; q < 8; ++q) {
+                const int c16 = lt + q * tpt;
+                if (tok_ok && c16 < cpt_full)
+                    raw[q] = *reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(a.x) + xrow + (int64_t)c16 * 8);
             }
         }
+        auto unpack = [&](int q, float (&v)[8]) {
+            if (a.x_f32) {
+                const uint4 r0 = raw[2 * q], r1 = raw[2 * q + 1];
+                v[0] = __uint_as_float(r0.x); v[1] = __uint_as_float(r0.y); v[2] = __uint_as_float(r0.z); v[3] = __uint_as_float(r0.w);
+                v[4] = __uint_as_float(r1.x); v[5] = __uint_as_float(r1.y); v[6] = __uint_as_float(r1.z); v[7] = __uint_as_float(r1.w);
+            } else {
+                const uint4 r4 = raw[q];
+                v[0] = bf16lo(r4.x); v[1] = bf16hi(r4.x); v[2] = bf16lo(r4.y); v[3] = bf16hi(r4.y);
+                v[4] = bf16lo(r4.z); v[5] = bf16hi(r4.z); v[6] = bf16lo(r4.w); v[7] = bf16hi(r4.w);
+            }
+        };
+        float ss = 0.f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            if (q < hold) {
+                float v[8];
+                unpack(q, v);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) ss += v[e] * v[e];
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        if (lane == 0) s_red[warp] = ss;
         __syncthreads();
-        if (tid < B) {
+        float tot = 0.f;
+        for (int w = 0; w < wpt; ++w) tot += s_red[tok_me * wpt + w];  // fixed order
+        const float inv = 1.0f / sqrtf(tot / (float)a.ldx + a.eps);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int c16 = lt + q * tpt;
+            if (q < hold && tok_ok && c16 < nbc * 16) {
+                float v[8];
+                unpack(q, v);  // zeros past the row end
+                if (c16 < cpt_full) scale8(c16 * 8, inv, v);
+                store8(tok_me, c16 * 8, v);
+            }
+        }
+        // padding chunks not covered above (only when the row is padded)
+        for (int c16 = lt + hold * tpt; tok_ok && c16 < nbc * 16; c16 += tpt) {
+            float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            store8(tok_me, c16 * 8, z);
+        }
+    } else {
+        float inv = 1.f;
+        if (a.norm) {
             float ss = 0.f;
-            for (int w = 0; w < kGemvWarps; ++w) ss += s_red[w * B + tid];
-            s_inv[tid] = 1.0f / sqrtf(ss / (float)a.ldx + a.eps);
-        }
-        __syncthreads();
-    }
-    {
-        const int chunks_per_tok = g.segs_per_cta * nbc * 16;  // 8-element chunks
-        const int total = B * chunks_per_tok;
-        for (int u0 = 0; u0 < total; u0 += 4 * kGemvThreads) {
-            float v[4][8];
-            int uu[4], kk[4];
+            for (int c0 = lt; c0 < cpt_full; c0 += 4 * tpt) {
+                float v[4][8];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int u = u0 + q * kGemvThreads + tid;
-                uu[q] = u;
-                kk[q] = -1;
-                if (u < total) {
-                    const int tok = u / chunks_per_tok, r = u % chunks_per_tok;
-                    const int sl = r / (nbc * 16), rr = r % (nbc * 16);
-                    const int k = (cblk_lo + rr / 16) * 128 + (rr % 16) * 8;
-                    if (k < g.Kseg) {
-                        load8((int64_t)tok * a.ldx + (int64_t)(seg_lo + sl) * g.Kseg + k, v[q]);
-                        kk[q] = k;
+                for (int q = 0; q < 4; ++q) {
+                    const int c16 = c0 + q * tpt;
+                    if (tok_ok && c16 < cpt_full) load8(xrow + (int64_t)c16 * 8, v[q]);
+                    else {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) v[q][e] = 0.f;
                     }
                 }
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) ss += v[q][e] * v[q][e];
             }
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int u = uu[q];
-                if (u >= total) continue;
-                const int tok = u / chunks_per_tok, r = u % chunks_per_tok;
-                const int sl = r / (nbc * 16), rr = r % (nbc * 16);
-                const int blk = cblk_lo + rr / 16, j = rr % 16;
-                const int k = kk[q];
-                if (k < 0) {
+            for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            if (lane == 0) s_red[warp] = ss;
+            __syncthreads();
+            float tot = 0.f;
+            for (int w = 0; w < wpt; ++w) tot += s_red[tok_me * wpt + w];
+            inv = 1.0f / sqrtf(tot / (float)a.ldx + a.eps);
+        }
+        if (tok_ok) {
+            for (int sl = 0; sl < g.segs_per_cta; ++sl) {
+                const int64_t srow = xrow + (int64_t)(seg_lo + sl) * g.Kseg + (int64_t)cblk_lo * 128;
+                const int kbase = cblk_lo * 128;
+                for (int c0 = lt; c0 < chunks_seg; c0 += 4 * tpt) {
+                    float v[4][8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) v[q][e] = 0.f;
-                } else if (a.norm) {
-                    const float inv = s_inv[tok];
-                    const float4 g0 = reinterpret_cast<const float4 *>(a.gamma + k)[0];
-                    const float4 g1 = reinterpret_cast<const float4 *>(a.gamma + k)[1];
-                    const float gm[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+                    for (int q = 0; q < 4; ++q) {
+                        const int c16 = c0 + q * tpt;
+                        if (c16 < chunks_seg && kbase + c16 * 8 < g.Kseg) load8(srow + (int64_t)c16 * 8, v[q]);
+                        else {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) v[q][e] = v[q][e] * inv * gm[e];
-                }
-                unsigned char *dst =
-                    xs + (size_t)tok * g.x_stride + (size_t)((sl * nbc + (blk - cblk_lo)) * 128 + j * 8) * T::XES;
-                if (T::XES == 2) {
-                    uint4 o;
-                    o.x = pack_bf16x2(v[q][0], v[q][1]); o.y = pack_bf16x2(v[q][2], v[q][3]);
-                    o.z = pack_bf16x2(v[q][4], v[q][5]); o.w = pack_bf16x2(v[q][6], v[q][7]);
-                    *reinterpret_cast<uint4 *>(dst) = o;
-                    if constexpr (XSPLIT) {
-                        uint4 l;
-                        l.x = pack_bf16x2(v[q][0] - bf16lo(o.x), v[q][1] - bf16hi(o.x));
-                        l.y = pack_bf16x2(v[q][2] - bf16lo(o.y), v[q][3] - bf16hi(o.y));
-                        l.z = pack_bf16x2(v[q][4] - bf16lo(o.z), v[q][5] - bf16hi(o.z));
-                        l.w = pack_bf16x2(v[q][6] - bf16lo(o.w), v[q][7] - bf16hi(o.w));
-                        *reinterpret_cast<uint4 *>(dst + lo_off) = l;
+                            for (int e = 0; e < 8; ++e) v[q][e] = 0.f;
+                        }
                     }
-                } else {
-                    reinterpret_cast<float4 *>(dst)[0] = make_float4(v[q][0], v[q][1], v[q][2], v[q][3]);
-                    reinterpret_cast<float4 *>(dst)[1] = make_float4(v[q][4], v[q][5], v[q][6], v[q][7]);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int c16 = c0 + q * tpt;
+                        if (c16 < chunks_seg) {
+                            if (a.norm && kbase + c16 * 8 < g.Kseg) scale8(kbase + c16 * 8, inv, v[q]);
+                            store8(tok_me, sl * chunks_seg * 8 + c16 * 8, v[q]);
+                        }
+                    }
                 }
             }
         }

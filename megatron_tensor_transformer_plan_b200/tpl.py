@@ -143,8 +143,9 @@ class Plan:
 
     def __del__(self):
         h = getattr(self, "handle", None)
-        if h is not None and h.value:
-            tpl_plan_destroy(h)
+        destroy = globals().get("tpl_plan_destroy")
+        if h is not None and h.value and destroy is not None:
+            destroy(h)
             self.handle = None
 
     # ---- host queries ----

@@ -155,8 +155,23 @@ int64_t tpl_kv_bytes(const tpl_dims *dims, int32_t t, int64_t batch, int64_t seq
 int64_t tpl_kv_layer_bytes(const tpl_plan *plan, int32_t batch_cap, int64_t seq_cap);
 
 /* Workspace bytes needed by the decode calls for batch B and cached length S
- * (both reduce modes), and by tpl_prefill_layer for T tokens when B = T. */
+ * (both reduce modes). */
 int tpl_workspace_size(const tpl_plan *plan, int32_t batch, int64_t seq, size_t *out);
+
+/* Workspace bytes needed by tpl_prefill_layer for a chunk of T tokens (both
+ * reduce modes; the separate mode's t partial sums [t][T][hidden] fp32 are
+ * the largest part).  TPL_EINVAL for T <= 0. */
+int tpl_prefill_workspace_size(const tpl_plan *plan, int32_t T, size_t *out);
+
+/* Byte offsets, inside a prefill workspace for T tokens, of the
+ * intermediates the last tpl_prefill_layer call on it left behind:
+ *   offsets[0]  q    fp32 [T][n_q][d]
+ *   offsets[1]  o    attention output, bf16 [T][n_q*d]
+ *   offsets[2]  h    fp32 [T][hidden] (after the first reduction)
+ *   offsets[3]  act  SwiGLU output, bf16 [T][ffn]
+ * (for inspection and tests; the pages define these as the layer's
+ * intermediate values).  offsets: host array of 4. */
+int tpl_prefill_intermediates(const tpl_plan *plan, int32_t T, size_t *offsets);
 
 /* ---- device calls ------------------------------------------------------- */
 
@@ -206,7 +221,22 @@ int tpl_decode_stack(tpl_plan *plan, const void *const *packed_per_layer, const 
 
 /* Prefill of one layer over T tokens of one sequence starting at position 0
  * (causal inside the chunk: token i sees positions 0..i), writing K/V cache
- * slots 0..T-1 of batch row 0.  x, y: [T][hidden] activation type. */
+ * slots 0..T-1 of batch row 0 ("Tensor parallel scaling curves", sections
+ * "What tensor parallelism actually splits" and "Prefill vs decode:
+ * different curves": the same splits as decode, over many tokens, so every
+ * projection is a matrix product):
+ *   a = RMSNorm(x); q|k|v = a Wqkv[s]^T per shard; causal attention on owned
+ *   heads; h = x + sum_s o_s Wo[s]^T; m = RMSNorm(h);
+ *   y = h + sum_s (silu(m Wg_s^T) * (m Wu_s^T)) Wd[s]^T.
+ * The projections run on the tensor cores (bf16 operands, fp32 accumulation;
+ * the normalised activations feeding QKV and gate/up as bf16 hi + lo).  The
+ * row-split sums add the t shard partials in ascending shard order in both
+ * reduce modes, so the two modes give identical bits.
+ * x, y: [T][hidden] bf16 (16-byte aligned); y32: fp32 [T][hidden] or NULL
+ * (at least one of y, y32).  Requires bf16 weights (TPL_EUNSUPPORTED with
+ * TPL_FP32_WEIGHTS), T <= kv->seq_cap and kv->batch_cap >= 1 (TPL_ENOMEM),
+ * ws_bytes >= tpl_prefill_workspace_size(T) (TPL_EWORKSPACE).  T = 0 does
+ * nothing.  Adds 2 to the plan's reduction counter. */
 int tpl_prefill_layer(tpl_plan *plan, const void *packed, const tpl_kv *kv, const void *x,
                       int32_t T, void *y, float *y32, void *ws, size_t ws_bytes,
                       int32_t reduce_mode, tpl_stream stream);

@@ -331,6 +331,9 @@ int decode_layer(Ctx &c, const char *packed, const tpl_kv *kv, const void *x, vo
 }  // namespace
 }  // namespace tpl
 
+// The prefill path: its kernels and host orchestration use the helpers above.
+#include "tpl_prefill.cuh"
+
 using namespace tpl;
 
 extern "C" {
@@ -540,9 +543,19 @@ int tpl_decode_stack(tpl_plan *p, const void *const *packed_per_layer, const tpl
 
 int tpl_prefill_layer(tpl_plan *p, const void *packed, const tpl_kv *kv, const void *x, int32_t T, void *y,
                       float *y32, void *ws, size_t ws_bytes, int32_t reduce_mode, tpl_stream stream) {
-    (void)p; (void)packed; (void)kv; (void)x; (void)T; (void)y; (void)y32; (void)ws; (void)ws_bytes;
-    (void)reduce_mode; (void)stream;
-    return TPL_EUNSUPPORTED;
+    if (!p || T < 0) return TPL_EINVAL;
+    if (reduce_mode != TPL_REDUCE_FUSED && reduce_mode != TPL_REDUCE_SEPARATE) return TPL_EINVAL;
+    if (T == 0) return TPL_OK;
+    if (p->f32) return TPL_EUNSUPPORTED;
+    if (!packed || !x || !ws || !al16(packed) || !al16(x) || !al16(ws) || (!y && !y32)) return TPL_EINVAL;
+    if ((y && !al16(y)) || (y32 && !al16(y32))) return TPL_EINVAL;
+    int rc = check_kv(kv, 1, (int64_t)T - 1);
+    if (rc != TPL_OK) return rc;
+    PrefillWs L;
+    if ((rc = prefill_ws_layout(p, T, &L)) != TPL_OK) return rc;
+    if (ws_bytes < L.total) return TPL_EWORKSPACE;
+    return prefill_layer(p, static_cast<const char *>(packed), kv, x, T, y, y32, static_cast<char *>(ws), L,
+                         reduce_mode, static_cast<cudaStream_t>(stream));
 }
 
 int tpl_last_device_error(const tpl_plan *p, tpl_stream stream) {

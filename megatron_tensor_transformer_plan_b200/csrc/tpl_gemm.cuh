@@ -1,0 +1,441 @@
+// Prefill projections on the 5th-generation tensor cores (tcgen05, TMEM).
+//
+// C[M tile of 128 tokens][N tile] = A[tokens][K] . W[N][K]^T, bf16 in, fp32
+// accumulate in tensor memory.  One CTA per output tile, 192 threads:
+//   warp 0     TMA producer (one elected thread): A and W tiles of 64
+//              columns, 128-byte swizzle, into an NS-stage shared-memory ring
+//              (no multicast; every CTA loads its own tiles);
+//   warp 1     allocates TMEM and issues tcgen05.mma (one thread), K-major
+//              shared-memory descriptors, 4 MMAs of K = 16 per stage; a
+//              tcgen05.commit per stage frees the stage, one at the end
+//              hands the accumulators to the epilogue;
+//   warps 2-5  epilogue: tcgen05.ld of their 32-lane quarter, the fused
+//              epilogue, stores.
+// Row-parallel projections ("Tensor parallel scaling curves", "What tensor
+// parallelism actually splits") keep one accumulator per shard (the shard's
+// K-slice), and the epilogue adds them in ascending shard order, so the fused
+// result equals the separate per-shard partials summed by tpl_reduce_partials
+// bit for bit.  With SPLIT_A the activation comes as bf16 hi + lo tiles and
+// each K step is two MMAs into the same accumulator.
+//
+// Every mbarrier wait is bounded; a wait that runs out records an error in
+// the device error word and the kernel winds down (TMEM is released).
+#pragma once
+
+#include <cuda.h>
+
+#include "tpl_common.cuh"
+#include "tpl_internal.h"
+
+namespace tpl {
+
+constexpr int kGemmThreads = 192;
+constexpr int kGemmMTile = 128;
+constexpr int kGemmKTile = 64;  // 128 bytes of bf16: one swizzle row
+constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s: far above any healthy wait
+
+enum { GEPI_F32 = 0, GEPI_QKV = 1, GEPI_GU = 2, GEPI_ROW = 3, GEPI_PARTIAL = 4 };
+
+struct GemmArgs {
+    CUtensorMap tm_a;   // A hi: [M][K] bf16 (2-D)
+    CUtensorMap tm_a2;  // A lo (SPLIT_A)
+    CUtensorMap tm_w;   // W: 2-D [N][K_pad] or 3-D [t][N][K_pad] (row-parallel)
+    int M, N;           // output rows (tokens), output columns
+    int k_blocks;       // 64-column blocks per accumulator segment
+    int nacc;           // accumulators (shards) this CTA adds up
+    int acc_shard0;     // first shard index (separate mode: one shard per CTA)
+    int a_col_stride;   // A column offset between shard segments (row-parallel), in elements
+    int w3d;            // weights are the 3-D per-shard map
+    int n_tiles;        // N / N_TILE
+    int epi;
+    // epilogue outputs
+    float *out32;       // GEPI_F32 / GEPI_ROW: [M][N]; GEPI_PARTIAL: [shards][M][N]
+    void *out_act;      // GEPI_ROW: activation-type copy; GEPI_GU: act [M][N/2]
+    int act_f32;
+    const void *resid;  // GEPI_ROW
+    int resid_f32;
+    // QKV mapping: q fp32 [M][nq][hd]; k/v rounded to bf16 into the cache
+    // (batch row 0, slot = token) and their rounding remainders into klo/vlo
+    // [M][nkv][hd] bf16
+    float *q32;
+    __nv_bfloat16 *klo, *vlo;
+    __nv_bfloat16 *kc, *vc;
+    int rps, nq, nq_s, nkv_s, hd, batch_cap;
+    int64_t seq_cap;
+};
+
+__device__ __forceinline__ unsigned smem_u32(const void *p) { return (unsigned)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, unsigned count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, unsigned bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait for the phase of parity `parity`; false once kWaitNs have
+// passed without it.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, unsigned parity) {
+    const unsigned a = smem_u32(bar);
+    unsigned long long t0 = 0;
+    for (unsigned it = 0;; ++it) {
+        unsigned done;
+        asm volatile(
+            "{ .reg .pred P; mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2; selp.u32 %0, 1, 0, P; }"
+            : "=r"(done)
+            : "r"(a), "r"(parity)
+            : "memory");
+        if (done) return true;
+        if ((it & 255u) == 255u) {
+            const unsigned long long now = global_ns();
+            if (t0 == 0) t0 = now;
+            else if (now - t0 > kWaitNs) return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *tm, int x, int y, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+            "r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *tm, int x, int y, int z, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::
+            "r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// K-major, 128-byte-swizzle shared-memory matrix descriptor: rows of 128 B,
+// 8-row groups 1024 B apart.
+__device__ __forceinline__ uint64_t umma_desc(unsigned saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+    d |= (uint64_t)1 << 16;            // leading byte offset (16 B; unused for swizzled K-major)
+    d |= (uint64_t)(1024 >> 4) << 32;  // stride byte offset: 8 rows x 128 B
+    d |= (uint64_t)1 << 46;            // descriptor version
+    d |= (uint64_t)2 << 61;            // 128-byte swizzle
+    return d;
+}
+
+// Instruction descriptor: bf16 x bf16 -> f32, both K-major, M x N.
+__host__ __device__ constexpr uint32_t umma_idesc(int M, int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{ .reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(tmem_d),
+        "l"(da), "l"(db), "r"(idesc), "r"(acc));
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+template <int N_TILE, bool SPLIT_A>
+struct GemmSmem {
+    static constexpr int A_BYTES = kGemmMTile * kGemmKTile * 2;  // 16 KB
+    static constexpr int W_BYTES = N_TILE * kGemmKTile * 2;
+    static constexpr int STAGE = A_BYTES * (SPLIT_A ? 2 : 1) + W_BYTES;
+    static constexpr int NS = (200 * 1024) / STAGE;
+    static constexpr int BYTES = NS * STAGE + 1024 /* alignment */ + 256 /* barriers */;
+};
+
+// 16 consecutive values of a row: activation-type or fp32 source.
+__device__ __forceinline__ void load16(const void *p, int is_f32, int64_t i, float (&v)[16]) {
+    if (is_f32) {
+        const float4 *q = reinterpret_cast<const float4 *>(static_cast<const float *>(p) + i);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float4 f = q[k];
+            v[4 * k] = f.x; v[4 * k + 1] = f.y; v[4 * k + 2] = f.z; v[4 * k + 3] = f.w;
+        }
+    } else {
+        const uint4 *q = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p) + i);
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const uint4 u = q[k];
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                v[8 * k + 2 * e] = bf16lo(w[e]);
+                v[8 * k + 2 * e + 1] = bf16hi(w[e]);
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void store16_f32(float *dst, const float (&v)[16]) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+        reinterpret_cast<float4 *>(dst)[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+}
+
+__device__ __forceinline__ void store16_bf16(__nv_bfloat16 *dst, const float (&v)[16]) {
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+        reinterpret_cast<uint4 *>(dst)[k] =
+            make_uint4(pack_bf16x2(v[8 * k], v[8 * k + 1]), pack_bf16x2(v[8 * k + 2], v[8 * k + 3]),
+                       pack_bf16x2(v[8 * k + 4], v[8 * k + 5]), pack_bf16x2(v[8 * k + 6], v[8 * k + 7]));
+}
+
+template <int N_TILE, int NACC, bool SPLIT_A>
+__global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_constant__ GemmArgs a) {
+    using SM = GemmSmem<N_TILE, SPLIT_A>;
+    constexpr int NS = SM::NS;
+    constexpr int TMEM_COLS = N_TILE * NACC <= 32 ? 32 : N_TILE * NACC <= 64 ? 64 : N_TILE * NACC <= 128 ? 128
+                              : N_TILE * NACC <= 256 ? 256 : 512;
+    static_assert(N_TILE * NACC <= 512, "accumulators exceed tensor memory");
+    static_assert(N_TILE % 16 == 0 && N_TILE >= 16 && N_TILE <= 256, "M=128 MMA needs N in [16, 256], N % 16 == 0");
+    extern __shared__ __align__(1024) unsigned char gsm_raw[];
+    unsigned char *gsm = reinterpret_cast<unsigned char *>(((uintptr_t)gsm_raw + 1023) & ~(uintptr_t)1023);
+    uint64_t *full = reinterpret_cast<uint64_t *>(gsm + NS * SM::STAGE);
+    uint64_t *empty = full + NS;
+    uint64_t *accb = empty + NS;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accb + 1);
+    int *s_fail = reinterpret_cast<int *>(tmem_slot + 1);
+    int *s_issued = s_fail + 1;    // stages the producer filled
+    int *s_consumed = s_fail + 2;  // stages the MMA issuer took
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // tiles: consecutive CTAs share a weight tile (m fastest), separate mode adds a shard index
+    const int mt_count = (a.M + kGemmMTile - 1) / kGemmMTile;
+    int bid = blockIdx.x;
+    const int m_t = bid % mt_count;
+    bid /= mt_count;
+    const int n_t = bid % a.n_tiles;
+    const int shard_extra = bid / a.n_tiles;  // separate mode: shard offset
+    const int m0 = m_t * kGemmMTile, n0 = n_t * N_TILE;
+    const int shard0 = a.acc_shard0 + shard_extra;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(accb, 1);
+        *s_fail = 0;
+        *s_issued = 0;
+        *s_consumed = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = *tmem_slot;
+    const int iters = a.nacc * a.k_blocks;
+
+    pdl_wait();
+    pdl_trigger();
+
+    if (warp == 0) {
+        if (lane == 0) {
+            constexpr unsigned TX = SM::A_BYTES * (SPLIT_A ? 2 : 1) + SM::W_BYTES;
+            int it = 0;
+            for (; it < iters; ++it) {
+                const int s = it % NS;
+                const unsigned ph = (unsigned)(it / NS) & 1u;
+                if (!mbar_wait(&empty[s], ph ^ 1u)) {
+                    atomicOr(s_fail, 1);
+                    break;
+                }
+                const int acc = it / a.k_blocks, kb = it % a.k_blocks;
+                const int sh = shard0 + acc;
+                unsigned char *st = gsm + s * SM::STAGE;
+                mbar_expect_tx(&full[s], TX);
+                const int ax = sh * a.a_col_stride + kb * kGemmKTile;
+                tma_load_2d(st, &a.tm_a, ax, m0, &full[s]);
+                if (SPLIT_A) tma_load_2d(st + SM::A_BYTES, &a.tm_a2, ax, m0, &full[s]);
+                unsigned char *wdst = st + SM::A_BYTES * (SPLIT_A ? 2 : 1);
+                if (a.w3d) tma_load_3d(wdst, &a.tm_w, kb * kGemmKTile, n0, sh, &full[s]);
+                else tma_load_2d(wdst, &a.tm_w, kb * kGemmKTile, n0, &full[s]);
+            }
+            *s_issued = it;
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t IDESC = umma_idesc(kGemmMTile, N_TILE);
+            int it = 0;
+            for (; it < iters; ++it) {
+                const int s = it % NS;
+                const unsigned ph = (unsigned)(it / NS) & 1u;
+                if (!mbar_wait(&full[s], ph)) {
+                    atomicOr(s_fail, 1);
+                    break;
+                }
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                const int acc = it / a.k_blocks, kb = it % a.k_blocks;
+                const uint32_t dcol = tmem + (uint32_t)(acc * N_TILE);
+                const unsigned sa = smem_u32(gsm + s * SM::STAGE);
+                const unsigned sw = sa + SM::A_BYTES * (SPLIT_A ? 2 : 1);
+#pragma unroll
+                for (int k = 0; k < kGemmKTile / 16; ++k) {
+                    const uint64_t db = umma_desc(sw + 32 * k);
+                    umma(dcol, umma_desc(sa + 32 * k), db, IDESC, (kb > 0 || k > 0) ? 1u : 0u);
+                    if (SPLIT_A) umma(dcol, umma_desc(sa + SM::A_BYTES + 32 * k), db, IDESC, 1u);
+                }
+                umma_commit(&empty[s]);  // stage free once these MMAs complete
+            }
+            *s_consumed = it;
+            umma_commit(accb);  // all issued MMAs complete
+        }
+    } else {
+        // ---- epilogue: warps 2..5 read TMEM lanes 32*(warp % 4) .. +31 ----
+        const int q = warp & 3;
+        const int row = m0 + 32 * q + lane;
+        const bool ok = mbar_wait(accb, 0);
+        if (!ok) atomicOr(s_fail, 1);
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        if (ok) {
+            const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16);
+            const bool rok = row < a.M;
+            for (int c0 = 0; c0 < N_TILE; c0 += 16) {
+                const int col = n0 + c0;
+                if (col >= a.N) break;                // warp-uniform
+                const bool full16 = col + 16 <= a.N;  // ragged last chunk: scalar stores
+                float v[16];
+                tmem_ld16(lane_addr + (uint32_t)c0, v);
+                if (a.epi == GEPI_PARTIAL) {
+                    // one accumulator per CTA (separate mode): the shard's partial
+                    if (rok) {
+                        float *dst = a.out32 + ((int64_t)shard0 * a.M + row) * a.N + col;
+                        if (full16) store16_f32(dst, v);
+                        else
+#pragma unroll
+                            for (int i = 0; i < 16; ++i)
+                                if (col + i < a.N) dst[i] = v[i];
+                    }
+                } else if (a.epi == GEPI_ROW) {
+                    for (int acc = 1; acc < NACC; ++acc) {  // shard partials in ascending order
+                        float w[16];
+                        tmem_ld16(lane_addr + (uint32_t)(acc * N_TILE + c0), w);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) v[i] = v[i] + w[i];
+                    }
+                    if (rok) {
+                        const int64_t base = (int64_t)row * a.N + col;
+                        if (full16) {
+                            if (a.resid) {
+                                float r[16];
+                                load16(a.resid, a.resid_f32, base, r);
+#pragma unroll
+                                for (int i = 0; i < 16; ++i) v[i] = r[i] + v[i];
+                            }
+                            if (a.out32) store16_f32(a.out32 + base, v);
+                            if (a.out_act) {
+                                if (a.act_f32) store16_f32(static_cast<float *>(a.out_act) + base, v);
+                                else store16_bf16(static_cast<__nv_bfloat16 *>(a.out_act) + base, v);
+                            }
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                if (col + i >= a.N) continue;
+                                float o = v[i];
+                                if (a.resid) o = load_act(a.resid, a.resid_f32, base + i) + o;
+                                if (a.out32) a.out32[base + i] = o;
+                                if (a.out_act) store_act(a.out_act, a.act_f32, base + i, o);
+                            }
+                        }
+                    }
+                } else if (a.epi == GEPI_F32) {
+                    if (rok) {
+                        float *dst = a.out32 + (int64_t)row * a.N + col;
+                        if (full16) store16_f32(dst, v);
+                        else
+#pragma unroll
+                            for (int i = 0; i < 16; ++i)
+                                if (col + i < a.N) dst[i] = v[i];
+                    }
+                } else if (a.epi == GEPI_GU) {
+                    // rows interleave gate and up: (g, u) pairs -> silu(g) * u
+                    if (rok) {
+                        const int Fh = a.N / 2;
+                        const int64_t base = (int64_t)row * Fh + col / 2;
+                        if (full16 && !a.act_f32) {
+                            const uint4 u = make_uint4(pack_bf16x2(silu(v[0]) * v[1], silu(v[2]) * v[3]),
+                                                       pack_bf16x2(silu(v[4]) * v[5], silu(v[6]) * v[7]),
+                                                       pack_bf16x2(silu(v[8]) * v[9], silu(v[10]) * v[11]),
+                                                       pack_bf16x2(silu(v[12]) * v[13], silu(v[14]) * v[15]));
+                            *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out_act) + base) = u;
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 16; i += 2)
+                                if (col + i + 1 < a.N) store_act(a.out_act, a.act_f32, base + i / 2, silu(v[i]) * v[i + 1]);
+                        }
+                    }
+                } else {  // GEPI_QKV: a 16-column chunk never straddles a head
+                    if (rok) {
+                        const int s = col / a.rps, l = col % a.rps;
+                        const int qd = a.nq_s * a.hd, kd = a.nkv_s * a.hd;
+                        if (l < qd) {
+                            const int head = s * a.nq_s + l / a.hd, dim = l % a.hd;
+                            store16_f32(a.q32 + ((int64_t)row * a.nq + head) * a.hd + dim, v);
+                        } else {
+                            const bool isk = l < qd + kd;
+                            const int ll = isk ? l - qd : l - qd - kd;
+                            const int kvl = ll / a.hd, dim = ll % a.hd;
+                            const int nkv = a.nkv_s * (a.nq / a.nq_s);
+                            float hi[16], lo[16];
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                hi[i] = __bfloat162float(__float2bfloat16_rn(v[i]));
+                                lo[i] = v[i] - hi[i];
+                            }
+                            __nv_bfloat16 *cc = isk ? a.kc : a.vc;
+                            store16_bf16(cc + (((int64_t)s * a.batch_cap) * a.nkv_s + kvl) * a.seq_cap * a.hd +
+                                             (int64_t)row * a.hd + dim,
+                                         hi);
+                            __nv_bfloat16 *fl = isk ? a.klo : a.vlo;
+                            store16_bf16(fl + ((int64_t)row * nkv + s * a.nkv_s + kvl) * a.hd + dim, lo);
+                        }
+                    }
+                }
+            }
+        }
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (*s_fail && threadIdx.x == 0) {
+        record_error(4u);
+        // let copies that were issued but never consumed land before the
+        // shared memory goes away (bounded as well)
+        for (int it = *s_consumed; it < *s_issued; ++it) mbar_wait(&full[it % NS], (unsigned)(it / NS) & 1u);
+    }
+    __syncthreads();
+    if (warp == 1) {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+    }
+}
+
+}  // namespace tpl

@@ -81,6 +81,19 @@ struct WsLayout {
 };
 int ws_layout(const tpl_plan *p, int B, int64_t S, WsLayout *w);
 
+// Workspace of a prefill call over T tokens (byte offsets).
+struct PrefillWs {
+    size_t a_hi, a_lo;  // normalised activation, bf16 hi + lo [T][hidden] (reused for the MLP)
+    size_t q;           // fp32 [T][n_q][d]
+    size_t klo, vlo;    // bf16 rounding remainders of the new k/v [T][n_kv][d]
+    size_t o;           // attention output, bf16 [T][n_q*d]
+    size_t h;           // fp32 [T][hidden]
+    size_t act;         // SwiGLU output, bf16 [T][ffn]
+    size_t P;           // fp32 shard partials [t][T][hidden] (separate reduce mode)
+    size_t total;
+};
+int prefill_ws_layout(const tpl_plan *p, int64_t T, PrefillWs *w);
+
 int num_sms_current();  // multiprocessor count of the current device (cached)
 
 }  // namespace tpl

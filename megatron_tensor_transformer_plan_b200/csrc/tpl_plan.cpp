@@ -154,6 +154,29 @@ int ws_layout(const tpl_plan *p, int B, int64_t S, WsLayout *w) {
     return TPL_OK;
 }
 
+int prefill_ws_layout(const tpl_plan *p, int64_t T, PrefillWs *w) {
+    if (T <= 0) return TPL_EINVAL;
+    const tpl_dims &d = p->d;
+    const int64_t H = d.hidden, nqd = (int64_t)d.n_q_heads * d.head_dim, nkvd = (int64_t)d.n_kv_heads * d.head_dim;
+    size_t off = 0;
+    auto take = [&](int64_t bytes) {
+        size_t o = off;
+        off = (size_t)align_up((int64_t)off + bytes, 256);
+        return o;
+    };
+    w->a_hi = take(T * H * 2);
+    w->a_lo = take(T * H * 2);
+    w->q = take(T * nqd * 4);
+    w->klo = take(T * nkvd * 2);
+    w->vlo = take(T * nkvd * 2);
+    w->o = take(T * nqd * 2);
+    w->h = take(T * H * 4);
+    w->act = take(T * (int64_t)d.ffn * 2);
+    w->P = take((int64_t)p->t * T * H * 4);
+    w->total = off;
+    return TPL_OK;
+}
+
 int num_sms_current() {
     static int cache[64] = {0};
     int dev = 0;
@@ -290,6 +313,27 @@ int tpl_workspace_size(const tpl_plan *p, int32_t batch, int64_t seq, size_t *ou
     int rc = tpl::ws_layout(p, batch, seq, &w);
     if (rc != TPL_OK) return rc;
     *out = w.total;
+    return TPL_OK;
+}
+
+int tpl_prefill_workspace_size(const tpl_plan *p, int32_t T, size_t *out) {
+    if (!p || !out || T <= 0) return TPL_EINVAL;
+    tpl::PrefillWs w;
+    int rc = tpl::prefill_ws_layout(p, T, &w);
+    if (rc != TPL_OK) return rc;
+    *out = w.total;
+    return TPL_OK;
+}
+
+int tpl_prefill_intermediates(const tpl_plan *p, int32_t T, size_t *offsets) {
+    if (!p || !offsets || T <= 0) return TPL_EINVAL;
+    tpl::PrefillWs w;
+    int rc = tpl::prefill_ws_layout(p, T, &w);
+    if (rc != TPL_OK) return rc;
+    offsets[0] = w.q;
+    offsets[1] = w.o;
+    offsets[2] = w.h;
+    offsets[3] = w.act;
     return TPL_OK;
 }
 

@@ -70,6 +70,8 @@ _sig("tpl_kv_bytes", c_int64, P(tpl_dims), c_int32, c_int64, c_int64, c_int32)
 _sig("tpl_kv_layer_bytes", c_int64, _plan_p, c_int32, c_int64)
 _sig("tpl_workspace_size", ctypes.c_int, _plan_p, c_int32, c_int64, P(c_size_t))
 _sig("tpl_workspace_init", ctypes.c_int, _plan_p, c_void_p, c_size_t, c_void_p)
+_sig("tpl_prefill_workspace_size", ctypes.c_int, _plan_p, c_int32, P(c_size_t))
+_sig("tpl_prefill_intermediates", ctypes.c_int, _plan_p, c_int32, P(c_size_t))
 _sig("tpl_pack_layer", ctypes.c_int, _plan_p, P(tpl_layer_weights), c_void_p, c_size_t, c_void_p)
 _sig("tpl_pack_kv", ctypes.c_int, _plan_p, c_void_p, c_void_p, c_int32, c_int64, c_void_p)
 _sig("tpl_decode_layer", ctypes.c_int, _plan_p, c_void_p, P(tpl_kv), c_void_p, c_int32, c_int64, c_void_p, c_void_p,
@@ -172,6 +174,17 @@ class Plan:
         check(tpl_workspace_size(self.handle, B, S, ctypes.byref(out)), "tpl_workspace_size")
         return out.value
 
+    def prefill_workspace_size(self, T: int) -> int:
+        out = c_size_t()
+        check(tpl_prefill_workspace_size(self.handle, T, ctypes.byref(out)), "tpl_prefill_workspace_size")
+        return out.value
+
+    def prefill_intermediates(self, T: int) -> dict:
+        """Byte offsets of q, o, h, act inside a prefill workspace for T tokens."""
+        offs = (c_size_t * 4)()
+        check(tpl_prefill_intermediates(self.handle, T, offs), "tpl_prefill_intermediates")
+        return dict(zip(("q", "o", "h", "act"), list(offs)))
+
     def kv_layer_bytes(self, batch_cap: int, seq_cap: int) -> int:
         return tpl_kv_layer_bytes(self.handle, batch_cap, seq_cap)
 
@@ -228,6 +241,15 @@ class Plan:
         B = x.shape[0]
         check(tpl_decode_layer(self.handle, packed.data_ptr(), ctypes.byref(kv), x.data_ptr(), B, S, _ptr(y),
                                _ptr(y32), ws.data_ptr(), ws.numel(), mode, _stream()), "tpl_decode_layer")
+
+    def prefill_workspace(self, T: int, device="cuda"):
+        import torch
+        return torch.empty(self.prefill_workspace_size(T), dtype=torch.uint8, device=device)
+
+    def prefill_layer(self, packed, kv: tpl_kv, x, y, y32=None, ws=None, mode=TPL_REDUCE_FUSED):
+        T = x.shape[0]
+        check(tpl_prefill_layer(self.handle, packed.data_ptr(), ctypes.byref(kv), x.data_ptr(), T, _ptr(y),
+                                _ptr(y32), ws.data_ptr(), ws.numel(), mode, _stream()), "tpl_prefill_layer")
 
     def decode_stack(self, packed_list, kv_list, x, S: int, y, y32=None, ws=None, mode=TPL_REDUCE_FUSED):
         L = len(packed_list)

@@ -206,6 +206,37 @@ def prefill_layer(dims: Dims, w: dict, x: np.ndarray, trace: bool = False):
     return (y, k, v, tr_arrays) if trace else (y, k, v)
 
 
+def prefill_rows(dims: Dims, w: dict, x: np.ndarray, rows, trace: bool = False):
+    """The prefill layer's outputs at the listed token rows only (keys and
+    values for every token up to the last listed row).  Returns y
+    [len(rows)][H], k and v [max(rows)+1][n_kv*d] (and a trace dict with
+    q, attn, h, act at the listed rows)."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    T, H = x.shape
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    n = len(r)
+    R = int(r.max()) + 1 if n else 0
+    nkd = dims.n_kv_heads * dims.head_dim
+    y = np.empty((n, H))
+    k = np.empty((R, nkd))
+    v = np.empty((R, nkd))
+    ws, keep = _weights_struct(w)
+    tr = None
+    tr_arrays = {}
+    if trace:
+        nqd = dims.n_q_heads * dims.head_dim
+        tr_arrays = {"q": np.empty((n, nqd)), "attn": np.empty((n, nqd)), "h": np.empty((n, H)),
+                     "act": np.empty((n, dims.ffn))}
+        tr = _Trace(_p(tr_arrays["q"]), None, None, _p(tr_arrays["attn"]), _p(tr_arrays["h"]),
+                    _p(tr_arrays["act"]))
+    rc = lib().orc_prefill_rows(ctypes.byref(dims.c()), ctypes.byref(ws), ctypes.c_long(T), _p(x),
+                                ctypes.c_long(n), r.ctypes.data_as(ctypes.POINTER(ctypes.c_long)), _p(y), _p(k),
+                                _p(v), ctypes.byref(tr) if tr is not None else None)
+    if rc != 0:
+        raise ValueError(f"orc_prefill_rows failed ({rc})")
+    return (y, k, v, tr_arrays) if trace else (y, k, v)
+
+
 def mlp_sharded(dims: Dims, w: dict, t: int, x: np.ndarray, partials: bool = False):
     """MLP pair sharded t ways, partials summed in ascending shard order
     ("Tensor Parallelism Fundamentals", "Mechanics of Matrix Slicing")."""

@@ -237,66 +237,84 @@ int orc_decode_layer(const orc_dims *dm, const orc_weights *w, long B, const dou
 }
 
 /* One unsharded prefill layer over a chunk of T tokens starting at position
- * 0 of empty caches: token i attends keys 0..i of the chunk (causal).
- * x [T][H]; y [T][H]; k_out/v_out [T][n_kv*d] receive the new keys/values
- * (these are what the cache slots 0..T-1 hold afterwards). */
-int orc_prefill_layer(const orc_dims *dm, const orc_weights *w, long T, const double *x, double *y,
-                      double *k_out, double *v_out, const orc_trace *tr) {
+ * 0 of empty caches: token i attends keys 0..i of the chunk (causal).  The
+ * layer's outputs are produced for the `nrows` token rows listed in `rows`
+ * (each in [0, T)); the keys and values of every token up to the largest
+ * listed row are computed, since those rows attend to them.
+ *   x [T][H]; y [nrows][H] (row r of y is token rows[r]);
+ *   k_out/v_out [R][n_kv*d], R = max(rows) + 1: the new keys/values, which
+ *   are what cache slots 0..R-1 hold afterwards;
+ *   trace (optional): q/attn [nrows][nq*d], h [nrows][H], act [nrows][F].
+ * Per token the steps are those of orc_decode_layer with the chunk's own
+ * keys 0..i in place of the cache ("Tensor parallel scaling curves",
+ * "Prefill vs decode: different curves"). */
+int orc_prefill_rows(const orc_dims *dm, const orc_weights *w, long T, const double *x, long nrows,
+                     const long *rows, double *y, double *k_out, double *v_out, const orc_trace *tr) {
     const long H = dm->hidden, nq = dm->n_q_heads, nkv = dm->n_kv_heads, d = dm->head_dim,
                F = dm->ffn;
-    if (H <= 0 || nq <= 0 || nkv <= 0 || d <= 0 || F <= 0 || nq % nkv != 0 || T < 0) return 1;
+    if (H <= 0 || nq <= 0 || nkv <= 0 || d <= 0 || F <= 0 || nq % nkv != 0 || T < 0 || nrows < 0)
+        return 1;
+    long R = 0;
+    for (long r = 0; r < nrows; ++r) {
+        if (rows[r] < 0 || rows[r] >= T) return 1;
+        if (rows[r] + 1 > R) R = rows[r] + 1;
+    }
     const long g = nq / nkv;
     const double scale = 1.0 / sqrt((double)d);
     double *a = malloc(sizeof(double) * (size_t)H);
-    double *Q = malloc(sizeof(double) * (size_t)(T * nq * d + 1));
-    double *K = malloc(sizeof(double) * (size_t)(T * nkv * d + 1));
-    double *V = malloc(sizeof(double) * (size_t)(T * nkv * d + 1));
-    double *O = malloc(sizeof(double) * (size_t)(T * nq * d + 1));
+    double *q = malloc(sizeof(double) * (size_t)(nq * d));
+    double *K = malloc(sizeof(double) * (size_t)(R * nkv * d + 1));
+    double *V = malloc(sizeof(double) * (size_t)(R * nkv * d + 1));
+    double *o = malloc(sizeof(double) * (size_t)(nq * d));
     double *hh = malloc(sizeof(double) * (size_t)H);
     double *m = malloc(sizeof(double) * (size_t)H);
     double *gg = malloc(sizeof(double) * (size_t)F);
     double *uu = malloc(sizeof(double) * (size_t)F);
     double *act = malloc(sizeof(double) * (size_t)F);
     double *dn = malloc(sizeof(double) * (size_t)H);
-    for (long i = 0; i < T; ++i) {
+    /* keys and values of tokens 0..R-1 */
+    for (long p = 0; p < R; ++p) {
+        const double *xp = x + (size_t)p * H;
+        if (dm->flags & ORC_NORM) orc_rmsnorm(xp, w->gamma_attn, H, dm->eps, a);
+        else memcpy(a, xp, sizeof(double) * (size_t)H);
+        linear_block(w->wk, w->wtype, (size_t)H, 0, nkv * d, 0, H, a, K + (size_t)p * nkv * d);
+        linear_block(w->wv, w->wtype, (size_t)H, 0, nkv * d, 0, H, a, V + (size_t)p * nkv * d);
+    }
+    for (long r = 0; r < nrows; ++r) {
+        const long i = rows[r];
         const double *xi = x + (size_t)i * H;
         if (dm->flags & ORC_NORM) orc_rmsnorm(xi, w->gamma_attn, H, dm->eps, a);
         else memcpy(a, xi, sizeof(double) * (size_t)H);
-        linear_block(w->wq, w->wtype, (size_t)H, 0, nq * d, 0, H, a, Q + (size_t)i * nq * d);
-        linear_block(w->wk, w->wtype, (size_t)H, 0, nkv * d, 0, H, a, K + (size_t)i * nkv * d);
-        linear_block(w->wv, w->wtype, (size_t)H, 0, nkv * d, 0, H, a, V + (size_t)i * nkv * d);
-    }
-    long ih;
-#pragma omp parallel for schedule(dynamic, 4)
-    for (ih = 0; ih < T * nq; ++ih) {
-        long i = ih / nq, h = ih % nq, j = h / g;
-        const double *q = Q + (size_t)i * nq * d + (size_t)h * d;
-        double *out = O + (size_t)i * nq * d + (size_t)h * d;
-        double *logit = malloc(sizeof(double) * (size_t)(i + 1));
-        double mx = -INFINITY;
-        for (long p = 0; p <= i; ++p) {
-            const double *kp = K + (size_t)p * nkv * d + (size_t)j * d;
-            double s = 0.0;
-            for (long e = 0; e < d; ++e) s += q[e] * kp[e];
-            logit[p] = s * scale;
-            if (logit[p] > mx) mx = logit[p];
+        linear_block(w->wq, w->wtype, (size_t)H, 0, nq * d, 0, H, a, q);
+        long h;
+#pragma omp parallel for schedule(static)
+        for (h = 0; h < nq; ++h) {
+            const long j = h / g;
+            const double *qh = q + (size_t)h * d;
+            double *out = o + (size_t)h * d;
+            double *logit = malloc(sizeof(double) * (size_t)(i + 1));
+            double mx = -INFINITY;
+            for (long p = 0; p <= i; ++p) {
+                const double *kp = K + (size_t)p * nkv * d + (size_t)j * d;
+                double s = 0.0;
+                for (long e = 0; e < d; ++e) s += qh[e] * kp[e];
+                logit[p] = s * scale;
+                if (logit[p] > mx) mx = logit[p];
+            }
+            double den = 0.0;
+            for (long p = 0; p <= i; ++p) {
+                logit[p] = exp(logit[p] - mx);
+                den += logit[p];
+            }
+            for (long e = 0; e < d; ++e) out[e] = 0.0;
+            for (long p = 0; p <= i; ++p) {
+                const double *vp = V + (size_t)p * nkv * d + (size_t)j * d;
+                const double pr = logit[p] / den;
+                for (long e = 0; e < d; ++e) out[e] += pr * vp[e];
+            }
+            free(logit);
         }
-        double den = 0.0;
-        for (long p = 0; p <= i; ++p) {
-            logit[p] = exp(logit[p] - mx);
-            den += logit[p];
-        }
-        for (long e = 0; e < d; ++e) out[e] = 0.0;
-        for (long p = 0; p <= i; ++p) {
-            const double *vp = V + (size_t)p * nkv * d + (size_t)j * d;
-            double pr = logit[p] / den;
-            for (long e = 0; e < d; ++e) out[e] += pr * vp[e];
-        }
-        free(logit);
-    }
-    for (long i = 0; i < T; ++i) {
-        const double *xi = x + (size_t)i * H;
-        linear_block(w->wo, w->wtype, (size_t)(nq * d), 0, H, 0, nq * d, O + (size_t)i * nq * d, hh);
+        linear_block(w->wo, w->wtype, (size_t)(nq * d), 0, H, 0, nq * d, o, hh);
         if (dm->flags & ORC_RESIDUAL)
             for (long c = 0; c < H; ++c) hh[c] = xi[c] + hh[c];
         if (dm->flags & ORC_NORM) orc_rmsnorm(hh, w->gamma_mlp, H, dm->eps, m);
@@ -305,22 +323,32 @@ int orc_prefill_layer(const orc_dims *dm, const orc_weights *w, long T, const do
         linear_block(w->wu, w->wtype, (size_t)H, 0, F, 0, H, m, uu);
         for (long c = 0; c < F; ++c) act[c] = orc_silu(gg[c]) * uu[c];
         linear_block(w->wd, w->wtype, (size_t)F, 0, H, 0, F, act, dn);
-        double *yi = y + (size_t)i * H;
-        for (long c = 0; c < H; ++c) yi[c] = (dm->flags & ORC_RESIDUAL) ? hh[c] + dn[c] : dn[c];
+        double *yr = y + (size_t)r * H;
+        for (long c = 0; c < H; ++c) yr[c] = (dm->flags & ORC_RESIDUAL) ? hh[c] + dn[c] : dn[c];
         if (tr) {
-            if (tr->h) memcpy(tr->h + (size_t)i * H, hh, sizeof(double) * (size_t)H);
-            if (tr->act) memcpy(tr->act + (size_t)i * F, act, sizeof(double) * (size_t)F);
+            if (tr->q) memcpy(tr->q + (size_t)r * nq * d, q, sizeof(double) * (size_t)(nq * d));
+            if (tr->attn) memcpy(tr->attn + (size_t)r * nq * d, o, sizeof(double) * (size_t)(nq * d));
+            if (tr->h) memcpy(tr->h + (size_t)r * H, hh, sizeof(double) * (size_t)H);
+            if (tr->act) memcpy(tr->act + (size_t)r * F, act, sizeof(double) * (size_t)F);
         }
     }
-    if (k_out) memcpy(k_out, K, sizeof(double) * (size_t)(T * nkv * d));
-    if (v_out) memcpy(v_out, V, sizeof(double) * (size_t)(T * nkv * d));
-    if (tr) {
-        if (tr->q) memcpy(tr->q, Q, sizeof(double) * (size_t)(T * nq * d));
-        if (tr->attn) memcpy(tr->attn, O, sizeof(double) * (size_t)(T * nq * d));
-    }
-    free(a); free(Q); free(K); free(V); free(O); free(hh); free(m);
+    if (k_out) memcpy(k_out, K, sizeof(double) * (size_t)(R * nkv * d));
+    if (v_out) memcpy(v_out, V, sizeof(double) * (size_t)(R * nkv * d));
+    free(a); free(q); free(K); free(V); free(o); free(hh); free(m);
     free(gg); free(uu); free(act); free(dn);
     return 0;
+}
+
+/* The whole chunk: every row 0..T-1.  x [T][H]; y [T][H]; k_out/v_out
+ * [T][n_kv*d]. */
+int orc_prefill_layer(const orc_dims *dm, const orc_weights *w, long T, const double *x, double *y,
+                      double *k_out, double *v_out, const orc_trace *tr) {
+    if (T < 0) return 1;
+    long *rows = malloc(sizeof(long) * (size_t)(T > 0 ? T : 1));
+    for (long i = 0; i < T; ++i) rows[i] = i;
+    int rc = orc_prefill_rows(dm, w, T, x, T, rows, y, k_out, v_out, tr);
+    free(rows);
+    return rc;
 }
 
 /* ---------------------------------------------------------------------------

@@ -443,3 +443,23 @@ def test_planted_transposed_wo_is_caught():
     P[np.arange(n), (np.arange(n) + 1) % n] = 1
     o = np.arange(1, n + 1, dtype=np.float64)
     assert not np.array_equal(P @ o, P.T @ o)
+
+
+def test_prefill_rows_match_the_whole_chunk():
+    """The sampled-row form gives, at each listed row (any order, repeats
+    allowed), the whole chunk's row; keys/values up to the last listed row."""
+    r = rng(47)
+    H, nq, nkv, d, F, T = 32, 4, 2, 8, 24, 9
+    w = small_layer(r, H, nq, nkv, d, F)
+    dims = oracle.Dims(H, nq, nkv, d, F)
+    x = r.normal(0, 1, (T, H))
+    y, k, v, tr = oracle.prefill_layer(dims, w, x, trace=True)
+    rows = [6, 0, 3, 6]
+    ys, ks, vs, trs = oracle.prefill_rows(dims, w, x, rows, trace=True)
+    np.testing.assert_array_equal(ys, y[rows])
+    np.testing.assert_array_equal(ks, k[:7])
+    np.testing.assert_array_equal(vs, v[:7])
+    for name in ("q", "attn", "h", "act"):
+        np.testing.assert_array_equal(trs[name], tr[name][rows])
+    with pytest.raises(ValueError):
+        oracle.prefill_rows(dims, w, x, [T])

@@ -165,12 +165,13 @@ int tpl_prefill_workspace_size(const tpl_plan *plan, int32_t T, size_t *out);
 
 /* Byte offsets, inside a prefill workspace for T tokens, of the
  * intermediates the last tpl_prefill_layer call on it left behind:
- *   offsets[0]  q    fp32 [T][n_q][d]
- *   offsets[1]  o    attention output, bf16 [T][n_q*d]
- *   offsets[2]  h    fp32 [T][hidden] (after the first reduction)
- *   offsets[3]  act  SwiGLU output, bf16 [T][ffn]
+ *   offsets[0]  q     fp32 [T][n_q][d]
+ *   offsets[1]  o     attention output, bf16 high part [T][n_q*d]
+ *   offsets[2]  h     fp32 [T][hidden] (after the first reduction)
+ *   offsets[3]  act   SwiGLU output, bf16 [T][ffn]
+ *   offsets[4]  o_lo  attention output, bf16 remainder: o = o + o_lo
  * (for inspection and tests; the pages define these as the layer's
- * intermediate values).  offsets: host array of 4. */
+ * intermediate values).  offsets: host array of 5. */
 int tpl_prefill_intermediates(const tpl_plan *plan, int32_t T, size_t *offsets);
 
 /* ---- device calls ------------------------------------------------------- */

@@ -33,8 +33,7 @@ struct AttnPrefillArgs {
     int T, nq, nkv, nkv_s, g;
     int gc, wpc;                      // chunks per query group, heads (warps) per chunk
     float scale_log2;
-    void *o;                          // [T][nq*128] activation type
-    int o_f32;
+    __nv_bfloat16 *o_hi, *o_lo;       // [T][nq*128]: output as bf16 hi + lo (the O projection's split operand)
 };
 
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
@@ -233,13 +232,17 @@ __global__ void __launch_bounds__(kApMaxWarps * 32) attn_prefill_kernel(const __
         const int dcol = 8 * t + 2 * c;
         if (ra < a.T) {
             const int64_t base = (int64_t)ra * a.nq * D + (int64_t)head * D + dcol;
-            store_act(a.o, a.o_f32, base, o[t][0] * ia);
-            store_act(a.o, a.o_f32, base + 1, o[t][1] * ia);
+            const float v0 = o[t][0] * ia, v1 = o[t][1] * ia;
+            const uint32_t h = pack_bf16x2(v0, v1);
+            *reinterpret_cast<uint32_t *>(a.o_hi + base) = h;
+            *reinterpret_cast<uint32_t *>(a.o_lo + base) = pack_bf16x2(v0 - bf16lo(h), v1 - bf16hi(h));
         }
         if (rb_ < a.T) {
             const int64_t base = (int64_t)rb_ * a.nq * D + (int64_t)head * D + dcol;
-            store_act(a.o, a.o_f32, base, o[t][2] * ib);
-            store_act(a.o, a.o_f32, base + 1, o[t][3] * ib);
+            const float v0 = o[t][2] * ib, v1 = o[t][3] * ib;
+            const uint32_t h = pack_bf16x2(v0, v1);
+            *reinterpret_cast<uint32_t *>(a.o_hi + base) = h;
+            *reinterpret_cast<uint32_t *>(a.o_lo + base) = pack_bf16x2(v0 - bf16lo(h), v1 - bf16hi(h));
         }
     }
 }

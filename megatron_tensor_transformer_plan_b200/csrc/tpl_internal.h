@@ -86,7 +86,7 @@ struct PrefillWs {
     size_t a_hi, a_lo;  // normalised activation, bf16 hi + lo [T][hidden] (reused for the MLP)
     size_t q;           // fp32 [T][n_q][d]
     size_t klo, vlo;    // bf16 rounding remainders of the new k/v [T][n_kv][d]
-    size_t o;           // attention output, bf16 [T][n_q*d]
+    size_t o, o_lo;     // attention output as bf16 hi + lo [T][n_q*d]
     size_t h;           // fp32 [T][hidden]
     size_t act;         // SwiGLU output, bf16 [T][ffn]
     size_t P;           // fp32 shard partials [t][T][hidden] (separate reduce mode)

@@ -170,6 +170,7 @@ int prefill_ws_layout(const tpl_plan *p, int64_t T, PrefillWs *w) {
     w->klo = take(T * nkvd * 2);
     w->vlo = take(T * nkvd * 2);
     w->o = take(T * nqd * 2);
+    w->o_lo = take(T * nqd * 2);
     w->h = take(T * H * 4);
     w->act = take(T * (int64_t)d.ffn * 2);
     w->P = take((int64_t)p->t * T * H * 4);
@@ -334,6 +335,7 @@ int tpl_prefill_intermediates(const tpl_plan *p, int32_t T, size_t *offsets) {
     offsets[1] = w.o;
     offsets[2] = w.h;
     offsets[3] = w.act;
+    offsets[4] = w.o_lo;
     return TPL_OK;
 }
 

@@ -5,8 +5,10 @@
 //
 //   norm_split   a = RMSNorm(x) as bf16 hi + lo                 (HBM bound)
 //   gemm QKV     column-parallel, fused scatter to q / cache / k,v remainders
-//   attention    causal, owned heads, mma.sync with hi + lo operands
-//   gemm O       row-parallel, t TMEM accumulators summed in shard order + x
+//   attention    causal, owned heads, mma.sync with hi + lo operands; writes
+//                its output as bf16 hi + lo
+//   gemm O       row-parallel on o as bf16 hi + lo, t TMEM accumulators summed
+//                in shard order, + x
 //   norm_split   m = RMSNorm(h) as bf16 hi + lo
 //   gemm GU      column-parallel, SwiGLU in the epilogue
 //   gemm down    row-parallel, t accumulators summed in shard order + h
@@ -130,7 +132,7 @@ int make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uin
 
 // ---- GEMM launches ---------------------------------------------------------
 
-bool g_gemm_attr[64][8];
+bool g_gemm_attr[64][8];  // per device: dynamic shared memory attribute set, per instantiation slot
 
 template <int NT, int NA, bool SA>
 int gemm_prepare(int slot) {
@@ -172,17 +174,19 @@ int gemm_column(GemmArgs &a, const void *a_hi, const void *a_lo, int64_t K, cons
 }
 
 // Row-parallel projection: A [T][t*Ks] bf16 (shard s owns columns
-// [s*Ks, (s+1)*Ks)), W the shards' blocks [t][N][ld] (3-D).  Fused: one TMEM
-// accumulator per shard, summed in order in the epilogue (GEPI_ROW).
-// Separate: one CTA per (tile, shard) writing the shard's partial
-// (GEPI_PARTIAL).
-int gemm_row(GemmArgs &a, const tpl_plan *p, const void *A, int64_t Ks, const void *W, int64_t ld, int64_t blk,
-             bool fused, cudaStream_t st) {
+// [s*Ks, (s+1)*Ks)), optionally with its bf16 remainder A_lo, W the shards'
+// blocks [t][N][ld] (3-D).  Fused: one TMEM accumulator per shard, summed in
+// order in the epilogue (GEPI_ROW).  Separate: one CTA per (tile, shard)
+// writing the shard's partial (GEPI_PARTIAL).
+int gemm_row(GemmArgs &a, const tpl_plan *p, const void *A, const void *A_lo, int64_t Ks, const void *W, int64_t ld,
+             int64_t blk, bool fused, cudaStream_t st) {
     const int t = p->t;
     const int64_t H = p->d.hidden;
     int nt = 256;
     if (fused) nt = t <= 2 ? 256 : t == 4 ? 128 : 64;
     int rc = make_map(&a.tm_a, A, (uint64_t)t * Ks, a.M, (uint64_t)t * Ks * 2, kGemmKTile, kGemmMTile);
+    if (rc == TPL_OK && A_lo)
+        rc = make_map(&a.tm_a2, A_lo, (uint64_t)t * Ks, a.M, (uint64_t)t * Ks * 2, kGemmKTile, kGemmMTile);
     if (rc == TPL_OK) rc = make_map(&a.tm_w, W, ld, H, ld * 2, kGemmKTile, nt, t, blk);
     if (rc != TPL_OK) return rc;
     a.N = (int)H;
@@ -193,10 +197,18 @@ int gemm_row(GemmArgs &a, const tpl_plan *p, const void *A, int64_t Ks, const vo
     if (!fused) {
         a.nacc = 1;
         a.epi = GEPI_PARTIAL;
-        return gemm_go<256, 1, false>(1, a, t, st);
+        return A_lo ? gemm_go<256, 1, true>(0, a, t, st) : gemm_go<256, 1, false>(1, a, t, st);
     }
     a.nacc = t;
     a.epi = GEPI_ROW;
+    if (A_lo) {
+        switch (t) {
+            case 1: return gemm_go<256, 1, true>(0, a, 1, st);
+            case 2: return gemm_go<256, 2, true>(5, a, 1, st);
+            case 4: return gemm_go<128, 4, true>(6, a, 1, st);
+            default: return gemm_go<64, 8, true>(7, a, 1, st);
+        }
+    }
     switch (t) {
         case 1: return gemm_go<256, 1, false>(1, a, 1, st);
         case 2: return gemm_go<256, 2, false>(2, a, 1, st);
@@ -222,7 +234,7 @@ int run_norm_split(const tpl_plan *p, const void *x, int x_f32, const float *gam
 bool g_ap_attr[64];
 
 int run_attn_prefill(const tpl_plan *p, const tpl_kv *kv, const float *q, const __nv_bfloat16 *klo,
-                     const __nv_bfloat16 *vlo, int T, void *o, cudaStream_t st) {
+                     const __nv_bfloat16 *vlo, int T, __nv_bfloat16 *o_hi, __nv_bfloat16 *o_lo, cudaStream_t st) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return TPL_ECUDA;
     if (!g_ap_attr[dev]) {
@@ -250,8 +262,8 @@ int run_attn_prefill(const tpl_plan *p, const tpl_kv *kv, const float *q, const 
     a.gc = gc;
     a.wpc = p->g / gc;
     a.scale_log2 = 1.4426950408889634f / sqrtf((float)p->d.head_dim);
-    a.o = o;
-    a.o_f32 = 0;
+    a.o_hi = o_hi;
+    a.o_lo = o_lo;
     const int64_t grid = (int64_t)((T + 15) / 16) * a.nkv * gc;
     if (grid > 0x7fffffff) return TPL_EUNSUPPORTED;
     return cuda_rc(launch_pdl(attn_prefill_kernel, (int)grid, a.wpc * 32, kApSmem, st, a));
@@ -266,7 +278,8 @@ int prefill_layer(tpl_plan *p, const char *packed, const tpl_kv *kv, const void 
     auto *q = reinterpret_cast<float *>(ws + L.q);
     auto *klo = reinterpret_cast<__nv_bfloat16 *>(ws + L.klo);
     auto *vlo = reinterpret_cast<__nv_bfloat16 *>(ws + L.vlo);
-    void *o = ws + L.o;
+    auto *o = reinterpret_cast<__nv_bfloat16 *>(ws + L.o);
+    auto *o_lo = reinterpret_cast<__nv_bfloat16 *>(ws + L.o_lo);
     auto *h = reinterpret_cast<float *>(ws + L.h);
     void *act = ws + L.act;
     auto *P = reinterpret_cast<float *>(ws + L.P);
@@ -292,7 +305,7 @@ int prefill_layer(tpl_plan *p, const char *packed, const tpl_kv *kv, const void 
         rc = gemm_column(a, a_hi, a_lo, H, packed + p->off_qkv, (int64_t)p->t * p->qkv_rows_s, p->ld_h, st);
         if (rc != TPL_OK) return rc;
     }
-    rc = run_attn_prefill(p, kv, q, klo, vlo, T, o, st);
+    rc = run_attn_prefill(p, kv, q, klo, vlo, T, o, o_lo, st);
     if (rc != TPL_OK) return rc;
     {  // O: h = x + sum_s o_s Wo[s]^T
         GemmArgs a = gemm_args(T);
@@ -303,7 +316,7 @@ int prefill_layer(tpl_plan *p, const char *packed, const tpl_kv *kv, const void 
         } else {
             a.out32 = P;
         }
-        rc = gemm_row(a, p, o, (int64_t)p->nq_s * hd, packed + p->off_o, p->ld_o, p->blk_o, fused, st);
+        rc = gemm_row(a, p, o, o_lo, (int64_t)p->nq_s * hd, packed + p->off_o, p->ld_o, p->blk_o, fused, st);
         if (rc != TPL_OK) return rc;
         if (fused) p->reductions.fetch_add(1);
         else if ((rc = run_reduce(p, st, P, resid ? x : nullptr, 0, T, h, nullptr)) != TPL_OK) return rc;
@@ -329,7 +342,7 @@ int prefill_layer(tpl_plan *p, const char *packed, const tpl_kv *kv, const void 
         } else {
             a.out32 = P;
         }
-        rc = gemm_row(a, p, act, p->F_s, packed + p->off_d, p->ld_f, p->blk_d, fused, st);
+        rc = gemm_row(a, p, act, nullptr, p->F_s, packed + p->off_d, p->ld_f, p->blk_d, fused, st);
         if (rc != TPL_OK) return rc;
         if (fused) p->reductions.fetch_add(1);
         else if ((rc = run_reduce(p, st, P, resid ? h : nullptr, 1, T, y32, y)) != TPL_OK) return rc;

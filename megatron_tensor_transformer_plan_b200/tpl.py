@@ -180,10 +180,11 @@ class Plan:
         return out.value
 
     def prefill_intermediates(self, T: int) -> dict:
-        """Byte offsets of q, o, h, act inside a prefill workspace for T tokens."""
-        offs = (c_size_t * 4)()
+        """Byte offsets of q, o (high part), h, act, o_lo inside a prefill
+        workspace for T tokens."""
+        offs = (c_size_t * 5)()
         check(tpl_prefill_intermediates(self.handle, T, offs), "tpl_prefill_intermediates")
-        return dict(zip(("q", "o", "h", "act"), list(offs)))
+        return dict(zip(("q", "o", "h", "act", "o_lo"), list(offs)))
 
     def kv_layer_bytes(self, batch_cap: int, seq_cap: int) -> int:
         return tpl_kv_layer_bytes(self.handle, batch_cap, seq_cap)

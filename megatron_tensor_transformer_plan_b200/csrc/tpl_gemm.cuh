@@ -1,25 +1,31 @@
 // Prefill projections on the 5th-generation tensor cores (tcgen05, TMEM).
 //
-// C[M tile of 128 tokens][N tile] = A[tokens][K] . W[N][K]^T, bf16 in, fp32
-// accumulate in tensor memory.  One CTA per output tile, 192 threads:
-//   warp 0     TMA producer (one elected thread): A and W tiles of 64
-//              columns, 128-byte swizzle, into an NS-stage shared-memory ring
-//              (no multicast; every CTA loads its own tiles);
-//   warp 1     allocates TMEM and issues tcgen05.mma (one thread), K-major
-//              shared-memory descriptors, 4 MMAs of K = 16 per stage; a
-//              tcgen05.commit per stage frees the stage, one at the end
-//              hands the accumulators to the epilogue;
-//   warps 2-5  epilogue: tcgen05.ld of their 32-lane quarter, the fused
-//              epilogue, stores.
-// Row-parallel projections ("Tensor parallel scaling curves", "What tensor
-// parallelism actually splits") keep one accumulator per shard (the shard's
-// K-slice), and the epilogue adds them in ascending shard order, so the fused
-// result equals the separate per-shard partials summed by tpl_reduce_partials
-// bit for bit.  With SPLIT_A the activation comes as bf16 hi + lo tiles and
-// each K step is two MMAs into the same accumulator.
+// C[128-token tile][256-column tile] = A[tokens][K] . W[N][K]^T, bf16 in,
+// fp32 accumulation in tensor memory.  Persistent: one CTA per SM walks a
+// static list of output tiles.  320 threads:
+//   warp 0     TMA producer (one thread): A and W tiles of 64 columns, 128-byte
+//              swizzle, into an NS-stage shared-memory ring (no multicast;
+//              every CTA loads its own tiles);
+//   warp 1     allocates all 512 TMEM columns (two 256-column accumulators)
+//              and issues tcgen05.mma (one thread): K-major shared-memory
+//              descriptors, 4 MMAs of K = 16 per stage, a tcgen05.commit per
+//              stage frees the stage, one per accumulation segment hands the
+//              accumulator to the epilogue;
+//   warps 2-9  epilogue: each reads its 32-lane quarter of TMEM (the lanes its
+//              warp may access) for one 128-column half of the tile.
+// An output tile is built from `nseg` accumulation segments.  Column-parallel
+// projections have one.  The fused row-parallel projection ("Tensor parallel
+// scaling curves", "What tensor parallelism actually splits") has one per
+// shard (that shard's K slice): the epilogue keeps a running sum in
+// registers, adding the shard partials in ascending shard order, so the result
+// equals the separate partials summed by tpl_reduce_partials bit for bit.
+// The two accumulators alternate, so the epilogue of one segment overlaps the
+// MMAs of the next.  With SPLIT_A the activation comes as bf16 hi + lo tiles
+// and each K step is two MMAs into the same accumulator.
 //
 // Every mbarrier wait is bounded; a wait that runs out records an error in
-// the device error word and the kernel winds down (TMEM is released).
+// the device error word, every role stops, copies already issued are waited
+// for (bounded as well) and TMEM is released.
 #pragma once
 
 #include <cuda.h>
@@ -29,8 +35,10 @@
 
 namespace tpl {
 
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 320;
+constexpr int kGemmEpiWarps = 8;
 constexpr int kGemmMTile = 128;
+constexpr int kGemmNTile = 256;
 constexpr int kGemmKTile = 64;  // 128 bytes of bf16: one swizzle row
 constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s: far above any healthy wait
 
@@ -41,12 +49,12 @@ struct GemmArgs {
     CUtensorMap tm_a2;  // A lo (SPLIT_A)
     CUtensorMap tm_w;   // W: 2-D [N][K_pad] or 3-D [t][N][K_pad] (row-parallel)
     int M, N;           // output rows (tokens), output columns
-    int k_blocks;       // 64-column blocks per accumulator segment
-    int nacc;           // accumulators (shards) this CTA adds up
-    int acc_shard0;     // first shard index (separate mode: one shard per CTA)
-    int a_col_stride;   // A column offset between shard segments (row-parallel), in elements
+    int k_blocks;       // 64-column blocks per accumulation segment
+    int nseg;           // segments per output tile (t for the fused row split, else 1)
+    int a_col_stride;   // A column offset between shards (row-parallel), in elements
     int w3d;            // weights are the 3-D per-shard map
-    int n_tiles;        // N / N_TILE
+    int m_tiles, n_tiles;
+    int units;          // m_tiles * n_tiles (* t in the separate row mode: one unit per shard)
     int epi;
     // epilogue outputs
     float *out32;       // GEPI_F32 / GEPI_ROW: [M][N]; GEPI_PARTIAL: [shards][M][N]
@@ -157,15 +165,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-template <int N_TILE, bool SPLIT_A>
-struct GemmSmem {
-    static constexpr int A_BYTES = kGemmMTile * kGemmKTile * 2;  // 16 KB
-    static constexpr int W_BYTES = N_TILE * kGemmKTile * 2;
-    static constexpr int STAGE = A_BYTES * (SPLIT_A ? 2 : 1) + W_BYTES;
-    static constexpr int NS = (200 * 1024) / STAGE;
-    static constexpr int BYTES = NS * STAGE + 1024 /* alignment */ + 256 /* barriers */;
-};
-
 // 16 consecutive values of a row: activation-type or fp32 source.
 __device__ __forceinline__ void load16(const void *p, int is_f32, int64_t i, float (&v)[16]) {
     if (is_f32) {
@@ -204,41 +203,135 @@ __device__ __forceinline__ void store16_bf16(__nv_bfloat16 *dst, const float (&v
                        pack_bf16x2(v[8 * k + 4], v[8 * k + 5]), pack_bf16x2(v[8 * k + 6], v[8 * k + 7]));
 }
 
-template <int N_TILE, int NACC, bool SPLIT_A>
+template <bool SPLIT_A>
+struct GemmSmem {
+    static constexpr int A_BYTES = kGemmMTile * kGemmKTile * 2;  // 16 KB
+    static constexpr int W_BYTES = kGemmNTile * kGemmKTile * 2;  // 32 KB
+    static constexpr int STAGE = A_BYTES * (SPLIT_A ? 2 : 1) + W_BYTES;
+    static constexpr int NS = (200 * 1024) / STAGE;
+    static constexpr int BYTES = NS * STAGE + 1024 /* alignment */ + 256 /* barriers */;
+};
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Unit u -> tile origin and the shard of a separate-mode unit.
+__device__ __forceinline__ void gemm_unit(const GemmArgs &a, int u, int &m0, int &n0, int &shard) {
+    const int mt = u % a.m_tiles;
+    const int r = u / a.m_tiles;
+    m0 = mt * kGemmMTile;
+    n0 = (r % a.n_tiles) * kGemmNTile;
+    shard = r / a.n_tiles;
+}
+
+// Epilogue of one 16-column chunk of a single-segment tile.
+__device__ __forceinline__ void gemm_epi_chunk(const GemmArgs &a, const float (&v)[16], int row, int col, int shard) {
+    if (row >= a.M || col >= a.N) return;
+    const bool full16 = col + 16 <= a.N;  // ragged last chunk: scalar stores
+    if (a.epi == GEPI_PARTIAL || a.epi == GEPI_F32) {
+        float *dst = a.out32 + ((int64_t)(a.epi == GEPI_PARTIAL ? shard : 0) * a.M + row) * a.N + col;
+        if (full16) store16_f32(dst, v);
+        else
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                if (col + i < a.N) dst[i] = v[i];
+    } else if (a.epi == GEPI_GU) {
+        // rows interleave gate and up: (g, u) pairs -> silu(g) * u
+        const int64_t base = (int64_t)row * (a.N / 2) + col / 2;
+        if (full16 && !a.act_f32) {
+            const uint4 u = make_uint4(pack_bf16x2(silu(v[0]) * v[1], silu(v[2]) * v[3]),
+                                       pack_bf16x2(silu(v[4]) * v[5], silu(v[6]) * v[7]),
+                                       pack_bf16x2(silu(v[8]) * v[9], silu(v[10]) * v[11]),
+                                       pack_bf16x2(silu(v[12]) * v[13], silu(v[14]) * v[15]));
+            *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out_act) + base) = u;
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; i += 2)
+                if (col + i + 1 < a.N) store_act(a.out_act, a.act_f32, base + i / 2, silu(v[i]) * v[i + 1]);
+        }
+    } else if (a.epi == GEPI_QKV) {  // a 16-column chunk never straddles a head
+        const int s = col / a.rps, l = col % a.rps;
+        const int qd = a.nq_s * a.hd, kd = a.nkv_s * a.hd;
+        if (l < qd) {
+            const int head = s * a.nq_s + l / a.hd, dim = l % a.hd;
+            store16_f32(a.q32 + ((int64_t)row * a.nq + head) * a.hd + dim, v);
+        } else {
+            const bool isk = l < qd + kd;
+            const int ll = isk ? l - qd : l - qd - kd;
+            const int kvl = ll / a.hd, dim = ll % a.hd;
+            const int nkv = a.nkv_s * (a.nq / a.nq_s);
+            float hi[16], lo[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                hi[i] = __bfloat162float(__float2bfloat16_rn(v[i]));
+                lo[i] = v[i] - hi[i];
+            }
+            __nv_bfloat16 *cc = isk ? a.kc : a.vc;
+            store16_bf16(cc + (((int64_t)s * a.batch_cap) * a.nkv_s + kvl) * a.seq_cap * a.hd + (int64_t)row * a.hd + dim,
+                         hi);
+            __nv_bfloat16 *fl = isk ? a.klo : a.vlo;
+            store16_bf16(fl + ((int64_t)row * nkv + s * a.nkv_s + kvl) * a.hd + dim, lo);
+        }
+    }
+}
+
+// Final store of a summed row-split chunk: out = resid + sum.
+__device__ __forceinline__ void gemm_row_store(const GemmArgs &a, float (&v)[16], int row, int col) {
+    if (row >= a.M || col >= a.N) return;
+    const int64_t base = (int64_t)row * a.N + col;
+    if (col + 16 <= a.N) {
+        if (a.resid) {
+            float r[16];
+            load16(a.resid, a.resid_f32, base, r);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] = r[i] + v[i];
+        }
+        if (a.out32) store16_f32(a.out32 + base, v);
+        if (a.out_act) {
+            if (a.act_f32) store16_f32(static_cast<float *>(a.out_act) + base, v);
+            else store16_bf16(static_cast<__nv_bfloat16 *>(a.out_act) + base, v);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if (col + i >= a.N) continue;
+            float o = v[i];
+            if (a.resid) o = load_act(a.resid, a.resid_f32, base + i) + o;
+            if (a.out32) a.out32[base + i] = o;
+            if (a.out_act) store_act(a.out_act, a.act_f32, base + i, o);
+        }
+    }
+}
+
+template <bool SPLIT_A, bool ROWSUM>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_constant__ GemmArgs a) {
-    using SM = GemmSmem<N_TILE, SPLIT_A>;
+    using SM = GemmSmem<SPLIT_A>;
     constexpr int NS = SM::NS;
-    constexpr int TMEM_COLS = N_TILE * NACC <= 32 ? 32 : N_TILE * NACC <= 64 ? 64 : N_TILE * NACC <= 128 ? 128
-                              : N_TILE * NACC <= 256 ? 256 : 512;
-    static_assert(N_TILE * NACC <= 512, "accumulators exceed tensor memory");
-    static_assert(N_TILE % 16 == 0 && N_TILE >= 16 && N_TILE <= 256, "M=128 MMA needs N in [16, 256], N % 16 == 0");
+    constexpr int TMEM_COLS = 2 * kGemmNTile;
     extern __shared__ __align__(1024) unsigned char gsm_raw[];
     unsigned char *gsm = reinterpret_cast<unsigned char *>(((uintptr_t)gsm_raw + 1023) & ~(uintptr_t)1023);
     uint64_t *full = reinterpret_cast<uint64_t *>(gsm + NS * SM::STAGE);
     uint64_t *empty = full + NS;
-    uint64_t *accb = empty + NS;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accb + 1);
-    int *s_fail = reinterpret_cast<int *>(tmem_slot + 1);
-    int *s_issued = s_fail + 1;    // stages the producer filled
-    int *s_consumed = s_fail + 2;  // stages the MMA issuer took
+    uint64_t *acc_full = empty + NS;  // [2]
+    uint64_t *acc_empty = acc_full + 2;  // [2]
+    uint64_t *fin = acc_empty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(fin + 1);
+    volatile int *s_fail = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    int *s_issued = const_cast<int *>(s_fail) + 1;    // stages the producer filled
+    int *s_consumed = const_cast<int *>(s_fail) + 2;  // stages the MMA issuer took
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // tiles: consecutive CTAs share a weight tile (m fastest), separate mode adds a shard index
-    const int mt_count = (a.M + kGemmMTile - 1) / kGemmMTile;
-    int bid = blockIdx.x;
-    const int m_t = bid % mt_count;
-    bid /= mt_count;
-    const int n_t = bid % a.n_tiles;
-    const int shard_extra = bid / a.n_tiles;  // separate mode: shard offset
-    const int m0 = m_t * kGemmMTile, n0 = n_t * N_TILE;
-    const int shard0 = a.acc_shard0 + shard_extra;
-
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(accb, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], kGemmEpiWarps);
+        }
+        mbar_init(fin, 1);
         *s_fail = 0;
         *s_issued = 0;
         *s_consumed = 0;
@@ -253,7 +346,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = *tmem_slot;
-    const int iters = a.nacc * a.k_blocks;
 
     pdl_wait();
     pdl_trigger();
@@ -262,163 +354,126 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
         if (lane == 0) {
             constexpr unsigned TX = SM::A_BYTES * (SPLIT_A ? 2 : 1) + SM::W_BYTES;
             int it = 0;
-            for (; it < iters; ++it) {
-                const int s = it % NS;
-                const unsigned ph = (unsigned)(it / NS) & 1u;
-                if (!mbar_wait(&empty[s], ph ^ 1u)) {
-                    atomicOr(s_fail, 1);
-                    break;
+            for (int u = blockIdx.x; u < a.units && !*s_fail; u += gridDim.x) {
+                int m0, n0, su;
+                gemm_unit(a, u, m0, n0, su);
+                for (int seg = 0; seg < a.nseg && !*s_fail; ++seg) {
+                    const int sh = su + seg;
+                    for (int kb = 0; kb < a.k_blocks; ++kb, ++it) {
+                        const int s = it % NS;
+                        const unsigned ph = (unsigned)(it / NS) & 1u;
+                        if (*s_fail || !mbar_wait(&empty[s], ph ^ 1u)) {
+                            *s_fail = 1;
+                            break;
+                        }
+                        unsigned char *st = gsm + s * SM::STAGE;
+                        mbar_expect_tx(&full[s], TX);
+                        const int ax = sh * a.a_col_stride + kb * kGemmKTile;
+                        tma_load_2d(st, &a.tm_a, ax, m0, &full[s]);
+                        if (SPLIT_A) tma_load_2d(st + SM::A_BYTES, &a.tm_a2, ax, m0, &full[s]);
+                        unsigned char *wdst = st + SM::A_BYTES * (SPLIT_A ? 2 : 1);
+                        if (a.w3d) tma_load_3d(wdst, &a.tm_w, kb * kGemmKTile, n0, sh, &full[s]);
+                        else tma_load_2d(wdst, &a.tm_w, kb * kGemmKTile, n0, &full[s]);
+                    }
                 }
-                const int acc = it / a.k_blocks, kb = it % a.k_blocks;
-                const int sh = shard0 + acc;
-                unsigned char *st = gsm + s * SM::STAGE;
-                mbar_expect_tx(&full[s], TX);
-                const int ax = sh * a.a_col_stride + kb * kGemmKTile;
-                tma_load_2d(st, &a.tm_a, ax, m0, &full[s]);
-                if (SPLIT_A) tma_load_2d(st + SM::A_BYTES, &a.tm_a2, ax, m0, &full[s]);
-                unsigned char *wdst = st + SM::A_BYTES * (SPLIT_A ? 2 : 1);
-                if (a.w3d) tma_load_3d(wdst, &a.tm_w, kb * kGemmKTile, n0, sh, &full[s]);
-                else tma_load_2d(wdst, &a.tm_w, kb * kGemmKTile, n0, &full[s]);
             }
             *s_issued = it;
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            constexpr uint32_t IDESC = umma_idesc(kGemmMTile, N_TILE);
-            int it = 0;
-            for (; it < iters; ++it) {
-                const int s = it % NS;
-                const unsigned ph = (unsigned)(it / NS) & 1u;
-                if (!mbar_wait(&full[s], ph)) {
-                    atomicOr(s_fail, 1);
+            constexpr uint32_t IDESC = umma_idesc(kGemmMTile, kGemmNTile);
+            int it = 0, c = 0;
+            for (int u = blockIdx.x; u < a.units && !*s_fail; u += gridDim.x) {
+                for (int seg = 0; seg < a.nseg && !*s_fail; ++seg, ++c) {
+                    const int b = c & 1;
+                    const unsigned use = (unsigned)(c >> 1);
+                    if (*s_fail || !mbar_wait(&acc_empty[b], (use & 1u) ^ 1u)) {
+                        *s_fail = 1;
+                        break;
+                    }
+                    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                    const uint32_t dcol = tmem + (uint32_t)(b * kGemmNTile);
+                    bool ok = true;
+                    for (int kb = 0; kb < a.k_blocks; ++kb, ++it) {
+                        const int s = it % NS;
+                        const unsigned ph = (unsigned)(it / NS) & 1u;
+                        if (*s_fail || !mbar_wait(&full[s], ph)) {
+                            *s_fail = 1;
+                            ok = false;
+                            break;
+                        }
+                        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                        const unsigned sa = smem_u32(gsm + s * SM::STAGE);
+                        const unsigned sw = sa + SM::A_BYTES * (SPLIT_A ? 2 : 1);
+#pragma unroll
+                        for (int k = 0; k < kGemmKTile / 16; ++k) {
+                            const uint64_t db = umma_desc(sw + 32 * k);
+                            umma(dcol, umma_desc(sa + 32 * k), db, IDESC, (kb > 0 || k > 0) ? 1u : 0u);
+                            if (SPLIT_A) umma(dcol, umma_desc(sa + SM::A_BYTES + 32 * k), db, IDESC, 1u);
+                        }
+                        umma_commit(&empty[s]);  // stage free once these MMAs complete
+                    }
+                    if (!ok) break;
+                    umma_commit(&acc_full[b]);  // accumulator b holds this segment
+                }
+            }
+            *s_consumed = it;
+            // every MMA this thread issued has completed once `fin` flips
+            umma_commit(fin);
+            if (!mbar_wait(fin, 0)) *s_fail = 1;
+        }
+    } else {
+        // ---- epilogue: warp w reads TMEM lanes 32*(w % 4).. (its accessible
+        // quarter) for columns [128*h, 128*h + 128) of the tile ----
+        const int q = warp & 3, hf = (warp - 2) >> 2;
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(hf * 128);
+        int c = 0;
+        for (int u = blockIdx.x; u < a.units && !*s_fail; u += gridDim.x) {
+            int m0, n0, su;
+            gemm_unit(a, u, m0, n0, su);
+            const int row = m0 + 32 * q + lane;
+            const int cb = n0 + hf * 128;
+            float sum[ROWSUM ? 128 : 1];  // running sum of the shard partials (fused row split)
+            bool ok = true;
+            for (int seg = 0; seg < a.nseg; ++seg, ++c) {
+                const int b = c & 1;
+                const unsigned use = (unsigned)(c >> 1);
+                if (*s_fail || !mbar_wait(&acc_full[b], use & 1u)) {
+                    *s_fail = 1;
+                    ok = false;
                     break;
                 }
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-                const int acc = it / a.k_blocks, kb = it % a.k_blocks;
-                const uint32_t dcol = tmem + (uint32_t)(acc * N_TILE);
-                const unsigned sa = smem_u32(gsm + s * SM::STAGE);
-                const unsigned sw = sa + SM::A_BYTES * (SPLIT_A ? 2 : 1);
+                const uint32_t taddr = lane_base + (uint32_t)(b * kGemmNTile);
+                if constexpr (ROWSUM) {
 #pragma unroll
-                for (int k = 0; k < kGemmKTile / 16; ++k) {
-                    const uint64_t db = umma_desc(sw + 32 * k);
-                    umma(dcol, umma_desc(sa + 32 * k), db, IDESC, (kb > 0 || k > 0) ? 1u : 0u);
-                    if (SPLIT_A) umma(dcol, umma_desc(sa + SM::A_BYTES + 32 * k), db, IDESC, 1u);
+                    for (int j = 0; j < 8; ++j) {
+                        float v[16];
+                        tmem_ld16(taddr + 16 * j, v);
+#pragma unroll
+                        // -0 is the additive identity (x + -0 == x for every x,
+                        // +-0 included): segment 0 stores its partial unchanged
+                        for (int i = 0; i < 16; ++i) sum[16 * j + i] = (seg == 0 ? -0.f : sum[16 * j + i]) + v[i];
+                    }
+                } else {
+                    for (int j = 0; j < 8; ++j) {
+                        float v[16];
+                        tmem_ld16(taddr + 16 * j, v);
+                        gemm_epi_chunk(a, v, row, cb + 16 * j, su);
+                    }
                 }
-                umma_commit(&empty[s]);  // stage free once these MMAs complete
+                asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[b]);
             }
-            *s_consumed = it;
-            umma_commit(accb);  // all issued MMAs complete
-        }
-    } else {
-        // ---- epilogue: warps 2..5 read TMEM lanes 32*(warp % 4) .. +31 ----
-        const int q = warp & 3;
-        const int row = m0 + 32 * q + lane;
-        const bool ok = mbar_wait(accb, 0);
-        if (!ok) atomicOr(s_fail, 1);
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        if (ok) {
-            const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16);
-            const bool rok = row < a.M;
-            for (int c0 = 0; c0 < N_TILE; c0 += 16) {
-                const int col = n0 + c0;
-                if (col >= a.N) break;                // warp-uniform
-                const bool full16 = col + 16 <= a.N;  // ragged last chunk: scalar stores
-                float v[16];
-                tmem_ld16(lane_addr + (uint32_t)c0, v);
-                if (a.epi == GEPI_PARTIAL) {
-                    // one accumulator per CTA (separate mode): the shard's partial
-                    if (rok) {
-                        float *dst = a.out32 + ((int64_t)shard0 * a.M + row) * a.N + col;
-                        if (full16) store16_f32(dst, v);
-                        else
+            if (!ok) break;
+            if constexpr (ROWSUM) {
 #pragma unroll
-                            for (int i = 0; i < 16; ++i)
-                                if (col + i < a.N) dst[i] = v[i];
-                    }
-                } else if (a.epi == GEPI_ROW) {
-                    for (int acc = 1; acc < NACC; ++acc) {  // shard partials in ascending order
-                        float w[16];
-                        tmem_ld16(lane_addr + (uint32_t)(acc * N_TILE + c0), w);
+                for (int j = 0; j < 8; ++j) {
+                    float v[16];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) v[i] = v[i] + w[i];
-                    }
-                    if (rok) {
-                        const int64_t base = (int64_t)row * a.N + col;
-                        if (full16) {
-                            if (a.resid) {
-                                float r[16];
-                                load16(a.resid, a.resid_f32, base, r);
-#pragma unroll
-                                for (int i = 0; i < 16; ++i) v[i] = r[i] + v[i];
-                            }
-                            if (a.out32) store16_f32(a.out32 + base, v);
-                            if (a.out_act) {
-                                if (a.act_f32) store16_f32(static_cast<float *>(a.out_act) + base, v);
-                                else store16_bf16(static_cast<__nv_bfloat16 *>(a.out_act) + base, v);
-                            }
-                        } else {
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                if (col + i >= a.N) continue;
-                                float o = v[i];
-                                if (a.resid) o = load_act(a.resid, a.resid_f32, base + i) + o;
-                                if (a.out32) a.out32[base + i] = o;
-                                if (a.out_act) store_act(a.out_act, a.act_f32, base + i, o);
-                            }
-                        }
-                    }
-                } else if (a.epi == GEPI_F32) {
-                    if (rok) {
-                        float *dst = a.out32 + (int64_t)row * a.N + col;
-                        if (full16) store16_f32(dst, v);
-                        else
-#pragma unroll
-                            for (int i = 0; i < 16; ++i)
-                                if (col + i < a.N) dst[i] = v[i];
-                    }
-                } else if (a.epi == GEPI_GU) {
-                    // rows interleave gate and up: (g, u) pairs -> silu(g) * u
-                    if (rok) {
-                        const int Fh = a.N / 2;
-                        const int64_t base = (int64_t)row * Fh + col / 2;
-                        if (full16 && !a.act_f32) {
-                            const uint4 u = make_uint4(pack_bf16x2(silu(v[0]) * v[1], silu(v[2]) * v[3]),
-                                                       pack_bf16x2(silu(v[4]) * v[5], silu(v[6]) * v[7]),
-                                                       pack_bf16x2(silu(v[8]) * v[9], silu(v[10]) * v[11]),
-                                                       pack_bf16x2(silu(v[12]) * v[13], silu(v[14]) * v[15]));
-                            *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out_act) + base) = u;
-                        } else {
-#pragma unroll
-                            for (int i = 0; i < 16; i += 2)
-                                if (col + i + 1 < a.N) store_act(a.out_act, a.act_f32, base + i / 2, silu(v[i]) * v[i + 1]);
-                        }
-                    }
-                } else {  // GEPI_QKV: a 16-column chunk never straddles a head
-                    if (rok) {
-                        const int s = col / a.rps, l = col % a.rps;
-                        const int qd = a.nq_s * a.hd, kd = a.nkv_s * a.hd;
-                        if (l < qd) {
-                            const int head = s * a.nq_s + l / a.hd, dim = l % a.hd;
-                            store16_f32(a.q32 + ((int64_t)row * a.nq + head) * a.hd + dim, v);
-                        } else {
-                            const bool isk = l < qd + kd;
-                            const int ll = isk ? l - qd : l - qd - kd;
-                            const int kvl = ll / a.hd, dim = ll % a.hd;
-                            const int nkv = a.nkv_s * (a.nq / a.nq_s);
-                            float hi[16], lo[16];
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                hi[i] = __bfloat162float(__float2bfloat16_rn(v[i]));
-                                lo[i] = v[i] - hi[i];
-                            }
-                            __nv_bfloat16 *cc = isk ? a.kc : a.vc;
-                            store16_bf16(cc + (((int64_t)s * a.batch_cap) * a.nkv_s + kvl) * a.seq_cap * a.hd +
-                                             (int64_t)row * a.hd + dim,
-                                         hi);
-                            __nv_bfloat16 *fl = isk ? a.klo : a.vlo;
-                            store16_bf16(fl + ((int64_t)row * nkv + s * a.nkv_s + kvl) * a.hd + dim, lo);
-                        }
-                    }
+                    for (int i = 0; i < 16; ++i) v[i] = sum[16 * j + i];
+                    gemm_row_store(a, v, row, cb + 16 * j);
                 }
             }
         }

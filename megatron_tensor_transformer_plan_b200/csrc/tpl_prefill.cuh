@@ -132,89 +132,71 @@ int make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uin
 
 // ---- GEMM launches ---------------------------------------------------------
 
-bool g_gemm_attr[64][8];  // per device: dynamic shared memory attribute set, per instantiation slot
+bool g_gemm_attr[64][4];  // per device: dynamic shared memory attribute set, per instantiation
 
-template <int NT, int NA, bool SA>
-int gemm_prepare(int slot) {
+template <bool SA, bool RS>
+int gemm_go(int slot, GemmArgs &a, int shard_units, cudaStream_t st) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return TPL_ECUDA;
     if (!g_gemm_attr[dev][slot]) {
-        if (cudaFuncSetAttribute(gemm_tc_kernel<NT, NA, SA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 GemmSmem<NT, SA>::BYTES) != cudaSuccess)
+        if (cudaFuncSetAttribute(gemm_tc_kernel<SA, RS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 GemmSmem<SA>::BYTES) != cudaSuccess)
             return TPL_ECUDA;
         g_gemm_attr[dev][slot] = true;
     }
-    return TPL_OK;
-}
-
-template <int NT, int NA, bool SA>
-int gemm_go(int slot, GemmArgs &a, int grid, cudaStream_t st) {
-    int rc = gemm_prepare<NT, NA, SA>(slot);
-    if (rc != TPL_OK) return rc;
-    a.n_tiles = (a.N + NT - 1) / NT;
-    const int g = ((a.M + kGemmMTile - 1) / kGemmMTile) * a.n_tiles * grid;
-    return cuda_rc(launch_pdl(gemm_tc_kernel<NT, NA, SA>, g, kGemmThreads, (size_t)GemmSmem<NT, SA>::BYTES, st, a));
+    const int sms = num_sms_current();
+    if (sms <= 0) return TPL_ECUDA;
+    a.m_tiles = (a.M + kGemmMTile - 1) / kGemmMTile;
+    a.n_tiles = (a.N + kGemmNTile - 1) / kGemmNTile;
+    const int64_t units = (int64_t)a.m_tiles * a.n_tiles * shard_units;
+    if (units > 0x7fffffff) return TPL_EUNSUPPORTED;
+    a.units = (int)units;
+    const int grid = (int)std::min<int64_t>(units, sms);
+    return cuda_rc(launch_pdl(gemm_tc_kernel<SA, RS>, grid, kGemmThreads, (size_t)GemmSmem<SA>::BYTES, st, a));
 }
 
 // Column-parallel projection: A = bf16 hi + lo [T][K] activations, W the
-// shards' stacked rows [N][ld] (2-D), N_TILE 256.
+// shards' stacked rows [N][ld] (2-D).
 int gemm_column(GemmArgs &a, const void *a_hi, const void *a_lo, int64_t K, const void *W, int64_t N, int64_t ld,
                 cudaStream_t st) {
     int rc = make_map(&a.tm_a, a_hi, K, a.M, K * 2, kGemmKTile, kGemmMTile);
     if (rc == TPL_OK) rc = make_map(&a.tm_a2, a_lo, K, a.M, K * 2, kGemmKTile, kGemmMTile);
-    if (rc == TPL_OK) rc = make_map(&a.tm_w, W, ld, N, ld * 2, kGemmKTile, 256);
+    if (rc == TPL_OK) rc = make_map(&a.tm_w, W, ld, N, ld * 2, kGemmKTile, kGemmNTile);
     if (rc != TPL_OK) return rc;
     a.N = (int)N;
     a.k_blocks = (int)(ld / kGemmKTile);
-    a.nacc = 1;
-    a.acc_shard0 = 0;
+    a.nseg = 1;
     a.a_col_stride = 0;
     a.w3d = 0;
-    return gemm_go<256, 1, true>(0, a, 1, st);
+    return gemm_go<true, false>(0, a, 1, st);
 }
 
 // Row-parallel projection: A [T][t*Ks] bf16 (shard s owns columns
 // [s*Ks, (s+1)*Ks)), optionally with its bf16 remainder A_lo, W the shards'
-// blocks [t][N][ld] (3-D).  Fused: one TMEM accumulator per shard, summed in
-// order in the epilogue (GEPI_ROW).  Separate: one CTA per (tile, shard)
-// writing the shard's partial (GEPI_PARTIAL).
+// blocks [t][N][ld] (3-D).  Fused: one accumulation segment per shard, summed
+// in ascending shard order in the epilogue (GEPI_ROW).  Separate: one unit
+// per (tile, shard) writing the shard's partial (GEPI_PARTIAL).
 int gemm_row(GemmArgs &a, const tpl_plan *p, const void *A, const void *A_lo, int64_t Ks, const void *W, int64_t ld,
              int64_t blk, bool fused, cudaStream_t st) {
     const int t = p->t;
     const int64_t H = p->d.hidden;
-    int nt = 256;
-    if (fused) nt = t <= 2 ? 256 : t == 4 ? 128 : 64;
     int rc = make_map(&a.tm_a, A, (uint64_t)t * Ks, a.M, (uint64_t)t * Ks * 2, kGemmKTile, kGemmMTile);
     if (rc == TPL_OK && A_lo)
         rc = make_map(&a.tm_a2, A_lo, (uint64_t)t * Ks, a.M, (uint64_t)t * Ks * 2, kGemmKTile, kGemmMTile);
-    if (rc == TPL_OK) rc = make_map(&a.tm_w, W, ld, H, ld * 2, kGemmKTile, nt, t, blk);
+    if (rc == TPL_OK) rc = make_map(&a.tm_w, W, ld, H, ld * 2, kGemmKTile, kGemmNTile, t, blk);
     if (rc != TPL_OK) return rc;
     a.N = (int)H;
     a.k_blocks = (int)(ld / kGemmKTile);
     a.a_col_stride = (int)Ks;
     a.w3d = 1;
-    a.acc_shard0 = 0;
     if (!fused) {
-        a.nacc = 1;
+        a.nseg = 1;
         a.epi = GEPI_PARTIAL;
-        return A_lo ? gemm_go<256, 1, true>(0, a, t, st) : gemm_go<256, 1, false>(1, a, t, st);
+        return A_lo ? gemm_go<true, false>(0, a, t, st) : gemm_go<false, false>(1, a, t, st);
     }
-    a.nacc = t;
+    a.nseg = t;
     a.epi = GEPI_ROW;
-    if (A_lo) {
-        switch (t) {
-            case 1: return gemm_go<256, 1, true>(0, a, 1, st);
-            case 2: return gemm_go<256, 2, true>(5, a, 1, st);
-            case 4: return gemm_go<128, 4, true>(6, a, 1, st);
-            default: return gemm_go<64, 8, true>(7, a, 1, st);
-        }
-    }
-    switch (t) {
-        case 1: return gemm_go<256, 1, false>(1, a, 1, st);
-        case 2: return gemm_go<256, 2, false>(2, a, 1, st);
-        case 4: return gemm_go<128, 4, false>(3, a, 1, st);
-        default: return gemm_go<64, 8, false>(4, a, 1, st);
-    }
+    return A_lo ? gemm_go<true, true>(2, a, 1, st) : gemm_go<false, true>(3, a, 1, st);
 }
 
 GemmArgs gemm_args(int M) {

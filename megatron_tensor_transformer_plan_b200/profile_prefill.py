@@ -42,7 +42,9 @@ def main() -> None:
     plan = tpl.Plan(tpl.make_dims(H, NQ, NKV, D, F, 1), TP)
     w = synth.layer_weights(H, NQ, NKV, D, F, seed=0, device=dev)
     packed = plan.pack_layer(w)
+    torch.cuda.synchronize()
     del w
+    torch.cuda.empty_cache()
     n = NKV * T * D
     k = torch.zeros(n, dtype=torch.bfloat16, device=dev)
     v = torch.zeros(n, dtype=torch.bfloat16, device=dev)

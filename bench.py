@@ -67,14 +67,39 @@ def load_peaks():
     return 6650.0, "fallback"
 
 
+def load_tensor_peak():
+    """Dense bf16 TFLOP/s for a kernel sequence timed on its own (burst)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        if "bf16_tflops" in j:
+            return float(j["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
+PREFILL_T = 2048
+
+
+def prefill_flops(T=PREFILL_T):
+    """Algorithmic FLOP of one layer prefill over T tokens: 2*T per weight of
+    the four projections, plus 4*d per (query head, key) pair the causal mask
+    keeps (QK^T and PV)."""
+    params = (NQ + 2 * NKV) * D * H + H * NQ * D + 3 * F * H
+    return 2.0 * T * params + 4.0 * D * NQ * (T * (T + 1) // 2)
+
+
+# the sources the decode gate/up kernel and its launch are built from
+DECODE_SOURCES = ("tpl_common.cuh", "tpl_device.cu", "tpl_gemv.cuh", "tpl_internal.h", "tpl_plan.cpp")
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "megatron_tensor_transformer_plan_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h", ".cpp")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode())
-                h.update(f.read())
+    for name in DECODE_SOURCES:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
@@ -308,6 +333,30 @@ def run_ours(args, ws, rank, local):
             evs[l][1].record(stream)
     torch.cuda.synchronize()
     gu_ms = sum(a.elapsed_time(b) for a, b in evs) / L
+    # ---- the prefill row: one 70B layer over a 2048-token chunk (layer 0's
+    # weights, its cache rows 0..2047 of sequence 0), timed alone ----
+    xp = synth.activations(PREFILL_T, H, seed=0, layer=1000, dtype=torch.bfloat16, device=dev)
+    yp = torch.empty_like(xp)
+    wsp = plan.prefill_workspace(PREFILL_T, device=dev)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            plan.prefill_layer(packed[0], kvs[0], xp, yp, None, wsp)
+    torch.cuda.synchronize()
+    pf_times = []
+    with torch.cuda.stream(stream):
+        for _ in range(10):
+            a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a_.record(stream)
+            plan.prefill_layer(packed[0], kvs[0], xp, yp, None, wsp)
+            b_.record(stream)
+            pf_times.append((a_, b_))
+    torch.cuda.synchronize()
+    assert plan.last_device_error() == tpl.TPL_OK
+    pf_ms = max_over_ranks(statistics.median(a_.elapsed_time(b_) for a_, b_ in pf_times), ws, dev)
+    tpeak, tpeak_kind = load_tensor_peak()
+    pf_tflops = prefill_flops() / (pf_ms / 1e3) / 1e12
+    del wsp, xp, yp
+
     peak, peak_kind = load_peaks()
     gu_gbs = gate_up_bytes_per_launch() / (gu_ms / 1e3) / 1e9
     step_gbs = algorithmic_bytes_per_step() / (ms / 1e3) / 1e9
@@ -326,7 +375,13 @@ def run_ours(args, ws, rank, local):
                 "e2e": {"value": ws * BATCH / (e2e_ms / 1e3), "unit": "tokens/s",
                         "h2d_bytes_per_step": x.numel() * 2, "d2h_bytes_per_step": y.numel() * 2},
                 "gpu_launches": 5 * L * args.steps,
-                "clocks": clk}
+                "clocks": clk,
+                "prefill": {"workload": f"70B-shaped layer prefill, t={T_SHARDS}, {PREFILL_T} tokens, causal in chunk",
+                            "ms_per_layer": pf_ms, "tokens_per_s": ws * PREFILL_T / (pf_ms / 1e3),
+                            "flop_per_layer": prefill_flops(), "achieved_tflops": pf_tflops,
+                            "peak_tflops": tpeak, "peak_kind": tpeak_kind + " (dense bf16 burst)",
+                            "frac": pf_tflops / tpeak, "timing": "median of 10 calls, CUDA events, after 3 warm-ups",
+                            "kernels_per_layer": 7}}
         if ws == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline_sample()
         print(json.dumps(line), flush=True)

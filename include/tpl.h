@@ -127,8 +127,12 @@ void tpl_plan_destroy(tpl_plan *plan);
 /* Plan options (host).  TPL_OPT_GEMV_MODE selects the inner product of the
  * bf16 matrix-vector kernels: 0 = tensor cores (mma.sync, the default),
  * 2 = FFMA on the CUDA cores (kept to measure against).  fp32 plans always
- * use FFMA.  Returns TPL_EINVAL for an unknown option or value. */
+ * use FFMA.  TPL_OPT_PREFILL_ATTN selects the prefill attention kernel:
+ * 0 = 5th-generation tensor cores (tcgen05, TMEM; the default when the
+ * query group size is a power of two), 1 = mma.sync (any group size; kept to
+ * measure against).  Returns TPL_EINVAL for an unknown option or value. */
 #define TPL_OPT_GEMV_MODE 1
+#define TPL_OPT_PREFILL_ATTN 2
 int tpl_plan_set_option(tpl_plan *plan, int32_t option, int32_t value);
 
 /* Footprints (host) -- see tpl_plan_info. */

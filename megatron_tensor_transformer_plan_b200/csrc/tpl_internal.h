@@ -42,6 +42,7 @@ struct tpl_plan {
     int64_t off_qkv, off_o, off_gu, off_d, off_g1, off_g2, packed_bytes;
     std::atomic<long long> reductions;
     int gemv_mode;  // 0: tensor-core fragments (bf16); 1: fp32 FFMA; 2: bf16 FFMA
+    int attn_prefill_mode;  // 0: tcgen05 (power-of-two group sizes); 1: mma.sync
 };
 
 namespace tpl {

@@ -211,6 +211,7 @@ int tpl_plan_create(const tpl_dims *dims, int32_t t, tpl_plan **out) {
     p->f32 = (dims->flags & TPL_FP32_WEIGHTS) != 0;
     p->esize = p->f32 ? 4 : 2;
     p->gemv_mode = p->f32 ? 1 : 0;
+    p->attn_prefill_mode = 0;
     const int64_t H = dims->hidden, es = p->esize;
     // rows padded with zeros to whole 128-column blocks
     p->ld_h = (int)align_up(H, 128);
@@ -247,6 +248,11 @@ int tpl_plan_set_option(tpl_plan *p, int32_t option, int32_t value) {
         if (value != 0 && value != 2) return TPL_EINVAL;
         if (p->f32) return value == 0 ? TPL_OK : TPL_EINVAL;
         p->gemv_mode = value;
+        return TPL_OK;
+    }
+    if (option == TPL_OPT_PREFILL_ATTN) {
+        if (value != 0 && value != 1) return TPL_EINVAL;
+        p->attn_prefill_mode = value;
         return TPL_OK;
     }
     return TPL_EINVAL;

@@ -20,6 +20,7 @@
 #include <cuda.h>
 
 #include "tpl_attn_prefill.cuh"
+#include "tpl_attn_tc.cuh"
 #include "tpl_gemm.cuh"
 
 namespace tpl {
@@ -115,13 +116,13 @@ EncodeTiledFn encode_fn() {
 // `planes` of them `plane_bytes` apart); boxes of box_cols x box_rows with the
 // 128-byte swizzle the MMA descriptors expect; out-of-range elements read 0.
 int make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint64_t row_bytes, uint32_t box_cols,
-             uint32_t box_rows, uint64_t planes = 0, uint64_t plane_bytes = 0) {
+             uint32_t box_rows, uint64_t planes = 0, uint64_t plane_bytes = 0, uint32_t box_planes = 1) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return TPL_ECUDA;
     if (((uintptr_t)base & 15u) || (row_bytes & 15u) || (plane_bytes & 15u)) return TPL_EINVAL;
     const cuuint64_t gdim[3] = {cols, rows, planes};
     const cuuint64_t gstr[2] = {row_bytes, plane_bytes};
-    const cuuint32_t box[3] = {box_cols, box_rows, 1};
+    const cuuint32_t box[3] = {box_cols, box_rows, box_planes};
     const cuuint32_t es[3] = {1, 1, 1};
     const cuuint32_t rank = planes ? 3 : 2;
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), gdim, gstr, box, es,
@@ -214,11 +215,53 @@ int run_norm_split(const tpl_plan *p, const void *x, int x_f32, const float *gam
 }
 
 bool g_ap_attr[64];
+bool g_at_attr[64];
+
+// Tensor-core attention: 128 rows per CTA = (128 / g) tokens x the g heads of
+// a kv head, so g must be a power of two.
+int run_attn_prefill_tc(const tpl_plan *p, const tpl_kv *kv, const float *q, const __nv_bfloat16 *klo,
+                        const __nv_bfloat16 *vlo, int T, __nv_bfloat16 *o_hi, __nv_bfloat16 *o_lo, cudaStream_t st,
+                        int dev) {
+    if (!g_at_attr[dev]) {
+        if (cudaFuncSetAttribute(attn_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAtSmem) !=
+            cudaSuccess)
+            return TPL_ECUDA;
+        g_at_attr[dev] = true;
+    }
+    AttnTcArgs a;
+    std::memset(&a, 0, sizeof(a));
+    const int nkv = p->d.n_kv_heads;
+    const uint64_t head_blocks = (uint64_t)p->t * kv->batch_cap * p->nkv_s;
+    // cache planes: [head blocks][keys < T][128]; keys past the chunk read as 0
+    int rc = make_map(&a.tm_khi, kv->k, 128, (uint64_t)T, 256, 64, kAtKeys, head_blocks, (uint64_t)kv->seq_cap * 256);
+    if (rc == TPL_OK)
+        rc = make_map(&a.tm_vhi, kv->v, 128, (uint64_t)T, 256, 64, kAtKeys, head_blocks, (uint64_t)kv->seq_cap * 256);
+    // remainder planes: [T][nkv][128]
+    if (rc == TPL_OK) rc = make_map(&a.tm_klo, klo, 128, nkv, 256, 64, 1, (uint64_t)T, (uint64_t)nkv * 256, kAtKeys);
+    if (rc == TPL_OK) rc = make_map(&a.tm_vlo, vlo, 128, nkv, 256, 64, 1, (uint64_t)T, (uint64_t)nkv * 256, kAtKeys);
+    if (rc != TPL_OK) return rc;
+    a.q32 = q;
+    a.o_hi = o_hi;
+    a.o_lo = o_lo;
+    a.T = T;
+    a.nq = p->d.n_q_heads;
+    a.nkv = nkv;
+    a.nkv_s = p->nkv_s;
+    a.g = p->g;
+    a.tb = 128 / p->g;
+    a.batch_cap = kv->batch_cap;
+    a.scale_log2 = 1.4426950408889634f / sqrtf((float)p->d.head_dim);
+    const int64_t grid = (int64_t)((T + a.tb - 1) / a.tb) * nkv;
+    if (grid > 0x7fffffff) return TPL_EUNSUPPORTED;
+    return cuda_rc(launch_pdl(attn_prefill_tc_kernel, (int)grid, kAtThreads, kAtSmem, st, a));
+}
 
 int run_attn_prefill(const tpl_plan *p, const tpl_kv *kv, const float *q, const __nv_bfloat16 *klo,
                      const __nv_bfloat16 *vlo, int T, __nv_bfloat16 *o_hi, __nv_bfloat16 *o_lo, cudaStream_t st) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return TPL_ECUDA;
+    if ((p->g & (p->g - 1)) == 0 && p->attn_prefill_mode == 0)
+        return run_attn_prefill_tc(p, kv, q, klo, vlo, T, o_hi, o_lo, st, dev);
     if (!g_ap_attr[dev]) {
         if (cudaFuncSetAttribute(attn_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kApSmem) !=
             cudaSuccess)

@@ -20,10 +20,11 @@ SENTINEL = 0x3F80  # bf16 1.0: cache slots past the chunk must keep it
 
 class Prefill:
     def __init__(self, H, nq, nkv, F, t, T, *, seed=0, layer=0, gamma_std=0.0, S_cap=None,
-                 flags=None):
+                 flags=None, attn_mode=0):
         flags = tpl.TPL_NORM | tpl.TPL_RESIDUAL if flags is None else flags
         self.dims = tpl.make_dims(H, nq, nkv, 128, F, 1, 1e-5, flags)
         self.plan = tpl.Plan(self.dims, t)
+        self.plan.set_option(tpl.TPL_OPT_PREFILL_ATTN, attn_mode)
         self.t, self.T = t, T
         self.S_cap = S_cap or T + 5
         self.w = synth.layer_weights(H, nq, nkv, 128, F, seed=seed, layer=layer, dtype=torch.bfloat16,
@@ -124,6 +125,24 @@ SMALL = [
 def test_prefill_small(gpu, case):
     H, nq, nkv, F, t, T = case
     check_prefill(Prefill(H, nq, nkv, F, t, T, gamma_std=0.02 if T > 100 else 0.0))
+
+
+@pytest.mark.parametrize("case", [(1024, 16, 4, 2816, 4, 200), (512, 16, 1, 512, 1, 64)])
+def test_prefill_mma_sync_attention(gpu, case):
+    """The mma.sync attention kernel (kept to measure against) on group sizes
+    the tensor-core kernel also takes."""
+    H, nq, nkv, F, t, T = case
+    check_prefill(Prefill(H, nq, nkv, F, t, T, attn_mode=1))
+
+
+def test_prefill_attention_kernels_agree(gpu):
+    """Both attention kernels against each other on the same chunk."""
+    outs = []
+    for mode in (0, 1):
+        P = Prefill(1024, 16, 2, 1408, 2, 300, attn_mode=mode)
+        P.run()
+        outs.append(P.intermediates()["attn"].clone())
+    assert_close_rel(to_np(outs[0]), to_np(outs[1]).astype(np.float64), tol=2e-3, what="tcgen05 vs mma.sync")
 
 
 def test_prefill_first_token_is_decode_of_empty_cache(gpu):

@@ -1,8 +1,10 @@
-"""Run one decode layer of the 70B-shaped stack (t = 8, batch 4, KV length
-4096) a few times through the C-ABI: a small, self-contained workload for
-profilers (about 2 GB on the device, five kernels per call).
+"""Run one 70B-shaped decode layer a few times through the C-ABI: a small,
+self-contained workload for profilers (2-3 GB on the device, five kernels per
+call).  Defaults: the stack's shape (t = 8, batch 4, KV length 4096); the
+70B single-layer workload is --t 4 --batch 16 --kv 8192.
 
     python -m megatron_tensor_transformer_plan_b200.profile_layer [--calls N] [--mode fused|separate]
+        [--t T] [--batch B] [--kv S]
 """
 from __future__ import annotations
 
@@ -12,14 +14,18 @@ import torch
 
 from megatron_tensor_transformer_plan_b200 import build, synth
 
-H, NQ, NKV, D, F, T, B, S = 8192, 64, 8, 128, 28672, 8, 4, 4096
+H, NQ, NKV, D, F = 8192, 64, 8, 128, 28672
 
 
 def main() -> None:
     ap = argparse.ArgumentParser()
     ap.add_argument("--calls", type=int, default=4)
     ap.add_argument("--mode", default="fused", choices=["fused", "separate"])
+    ap.add_argument("--t", type=int, default=8)
+    ap.add_argument("--batch", type=int, default=4)
+    ap.add_argument("--kv", type=int, default=4096)
     args = ap.parse_args()
+    T, B, S = args.t, args.batch, args.kv
     build.build()
     from megatron_tensor_transformer_plan_b200 import tpl
     dev = torch.device("cuda")

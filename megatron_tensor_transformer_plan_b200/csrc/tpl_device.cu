@@ -9,7 +9,10 @@
 #include "tpl_attn.cuh"
 #include "tpl_common.cuh"
 #include "tpl_gemv.cuh"
+#include "tpl_gemv_tc.cuh"
 #include "tpl_internal.h"
+#include "tpl_norm.cuh"
+#include "tpl_tma.h"
 
 namespace tpl {
 
@@ -157,8 +160,141 @@ GemvArgs base_args(const tpl_plan *p) {
     return a;
 }
 
+// ---- tensor-core decode projections (TPL_OPT_GEMV_MODE 3) -----------------
+
+bool g_gt_attr[64][3];
+
+template <int NX, bool SPLIT>
+int gt_go(int slot, GemvTcArgs &a, cudaStream_t st) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return TPL_ECUDA;
+    if (!g_gt_attr[dev][slot]) {
+        if (cudaFuncSetAttribute(gemv_tc_kernel<NX, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 GemvTcSmem<NX>::BYTES) != cudaSuccess)
+            return TPL_ECUDA;
+        g_gt_attr[dev][slot] = true;
+    }
+    const int sms = num_sms_current();
+    if (sms <= 0) return TPL_ECUDA;
+    const int64_t G = std::min<int64_t>(std::min<int64_t>(sms, a.U), kGemvTcMaxCtas);
+    return cuda_rc(launch_pdl(gemv_tc_kernel<NX, SPLIT>, (int)G, kGtThreads, (size_t)GemvTcSmem<NX>::BYTES, st, a));
+}
+
+// MMA N: the B token rows (and with a split activation their lo rows), at
+// least 16 and a multiple of 16.
+int gt_nx(int B, bool split) { return split ? (B <= 8 ? 16 : 32) : 16; }
+
+// Fill the geometry, the weight map (2-D column-parallel rows or 3-D per-shard
+// blocks) and the activation map, then launch.
+int gemv_tc_run(Ctx &c, GemvTcArgs &a, int op, bool split, const void *W, int64_t ld, int64_t N, int nseg,
+                int64_t blk, const void *X, int64_t Kx, int64_t x_rows, int x_seg_stride) {
+    tpl_plan *p = c.p;
+    (void)p;
+    if (c.B > kGtMaxB) return TPL_EUNSUPPORTED;
+    const int nx = gt_nx(c.B, split);
+    a.B = c.B;
+    a.N = (int)N;
+    a.tiles = (int)((N + kGtRows - 1) / kGtRows);
+    if (a.tiles > kGemvTcMaxTiles) return TPL_EUNSUPPORTED;
+    a.nseg = nseg;
+    a.kbs = (int)(ld / kGtK);
+    a.U = (int64_t)a.tiles * a.nseg * a.kbs;
+    a.x_seg_stride = x_seg_stride;
+    a.w3d = nseg > 1 ? 1 : 0;
+    int rc = a.w3d ? make_map(&a.tm_w, W, ld, N, ld * 2, kGtK, kGtRows, nseg, blk)
+                   : make_map(&a.tm_w, W, ld, N, ld * 2, kGtK, kGtRows);
+    if (rc == TPL_OK) rc = make_map(&a.tm_x, X, Kx, x_rows, Kx * 2, kGtK, nx);
+    if (rc != TPL_OK) return rc;
+    a.gpart = reinterpret_cast<float *>(c.ws + c.L.gpart);
+    a.tickets = reinterpret_cast<unsigned *>(c.ws + c.L.tickets) + kTicketGemv + 512 * op;
+    if (split) return nx == 16 ? gt_go<16, true>(0, a, c.st) : gt_go<32, true>(1, a, c.st);
+    return gt_go<16, false>(2, a, c.st);
+}
+
+GemvTcArgs gt_args(const tpl_plan *p) {
+    GemvTcArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.hd = p->d.head_dim;
+    return a;
+}
+
+// RMSNorm (or a copy without TPL_NORM) of B rows into the workspace's
+// activation operand [NX][hidden]: bf16 hi rows 0..B-1, lo rows NX/2..NX/2+B-1,
+// zero rows elsewhere.
+int run_norm_rows(Ctx &c, const void *x, int x_f32, const float *gamma) {
+    tpl_plan *p = c.p;
+    auto *xs = reinterpret_cast<__nv_bfloat16 *>(c.ws + c.L.xs);
+    const int half = gt_nx(c.B, true) / 2;
+    const int norm = (p->d.flags & TPL_NORM) ? 1 : 0;
+    return cuda_rc(launch_pdl(norm_split_kernel, half, 256, 0, c.st, x, x_f32, gamma, p->d.rms_eps, norm,
+                              p->d.hidden, xs, xs + (int64_t)half * p->d.hidden, c.B));
+}
+
+int run_qkv_tc(Ctx &c, const char *packed, const tpl_kv *kv, const void *x, float *q, float *knew, float *vnew) {
+    tpl_plan *p = c.p;
+    int rc = run_norm_rows(c, x, 0, reinterpret_cast<const float *>(packed + p->off_g1));
+    if (rc != TPL_OK) return rc;
+    GemvTcArgs a = gt_args(p);
+    a.epi = GT_QKV;
+    a.q = q;
+    a.knew = knew;
+    a.vnew = vnew;
+    a.kc = static_cast<__nv_bfloat16 *>(kv->k);
+    a.vc = static_cast<__nv_bfloat16 *>(kv->v);
+    a.rps = p->qkv_rows_s;
+    a.nq = p->d.n_q_heads;
+    a.nq_s = p->nq_s;
+    a.nkv_s = p->nkv_s;
+    a.batch_cap = kv->batch_cap;
+    a.S = c.S;
+    a.seq_cap = kv->seq_cap;
+    const int64_t H = p->d.hidden;
+    return gemv_tc_run(c, a, OP_QKV, true, packed + p->off_qkv, p->ld_h, (int64_t)p->t * p->qkv_rows_s, 1, 0,
+                       c.ws + c.L.xs, H, gt_nx(c.B, true), 0);
+}
+
+int run_gu_tc(Ctx &c, const char *packed, const void *h, int h_is_act, void *act) {
+    tpl_plan *p = c.p;
+    int rc = run_norm_rows(c, h, h_is_act ? 0 : 1, reinterpret_cast<const float *>(packed + p->off_g2));
+    if (rc != TPL_OK) return rc;
+    GemvTcArgs a = gt_args(p);
+    a.epi = GT_GU;
+    a.out_act = act;
+    const int64_t H = p->d.hidden;
+    return gemv_tc_run(c, a, OP_GU, true, packed + p->off_gu, p->ld_h, (int64_t)p->t * 2 * p->F_s, 1, 0,
+                       c.ws + c.L.xs, H, gt_nx(c.B, true), 0);
+}
+
+// Row-parallel O (K slice of shard s: columns s*nq_s*d of o) or down (s*F_s of act).
+int run_row_tc(Ctx &c, const char *packed, int op, const void *x, const void *resid, int resid_f32, float *out32,
+               void *out_act, float *partials) {
+    tpl_plan *p = c.p;
+    GemvTcArgs a = gt_args(p);
+    if (partials) {
+        a.epi = GT_ROW_PARTIAL;
+        a.partials = partials;
+    } else {
+        a.epi = GT_ROW;
+        a.resid = resid;
+        a.resid_f32 = resid_f32;
+        a.out32 = out32;
+        a.out_act = out_act;
+    }
+    const bool is_o = op == OP_O;
+    const int64_t Ks = is_o ? (int64_t)p->nq_s * p->d.head_dim : p->F_s;
+    const int64_t ld = is_o ? p->ld_o : p->ld_f;
+    const int64_t blk = is_o ? p->blk_o : p->blk_d;
+    const char *W = packed + (is_o ? p->off_o : p->off_d);
+    if (p->t == 1) {
+        // one shard: a single 2-D block
+        return gemv_tc_run(c, a, op, false, W, ld, p->d.hidden, 1, 0, x, Ks, c.B, 0);
+    }
+    return gemv_tc_run(c, a, op, false, W, ld, p->d.hidden, p->t, blk, x, (int64_t)p->t * Ks, c.B, (int)Ks);
+}
+
 int run_qkv(Ctx &c, const char *packed, const tpl_kv *kv, const void *x, float *q, float *knew, float *vnew) {
     tpl_plan *p = c.p;
+    if (p->gemv_mode == 3) return run_qkv_tc(c, packed, kv, x, q, knew, vnew);
     GemvArgs a = base_args(p);
     a.W = packed + p->off_qkv;
     a.blk_r = p->blk_qkv;
@@ -220,6 +356,11 @@ int run_attn(Ctx &c, const tpl_kv *kv, const float *q, const float *knew, const 
 // Row-parallel O projection: fused (partials == NULL) or partial output.
 int run_o(Ctx &c, const char *packed, const void *o, const void *resid, float *h, float *partials) {
     tpl_plan *p = c.p;
+    if (p->gemv_mode == 3) {
+        int rc = run_row_tc(c, packed, OP_O, o, resid, 0, h, nullptr, partials);
+        if (rc == TPL_OK && !partials) p->reductions.fetch_add(1);
+        return rc;
+    }
     GemvArgs a = base_args(p);
     a.W = packed + p->off_o;
     a.blk_s = p->blk_o;
@@ -244,6 +385,7 @@ int run_o(Ctx &c, const char *packed, const void *o, const void *resid, float *h
 
 int run_gu(Ctx &c, const char *packed, const void *h, int h_is_act, void *act) {
     tpl_plan *p = c.p;
+    if (p->gemv_mode == 3) return run_gu_tc(c, packed, h, h_is_act, act);
     GemvArgs a = base_args(p);
     a.W = packed + p->off_gu;
     a.blk_r = p->blk_gu;
@@ -262,6 +404,11 @@ int run_gu(Ctx &c, const char *packed, const void *h, int h_is_act, void *act) {
 int run_down(Ctx &c, const char *packed, const void *act, const void *resid, int resid_f32, void *y, float *y32,
              float *partials) {
     tpl_plan *p = c.p;
+    if (p->gemv_mode == 3) {
+        int rc = run_row_tc(c, packed, OP_DOWN, act, resid, resid_f32, y32, y, partials);
+        if (rc == TPL_OK && !partials) p->reductions.fetch_add(1);
+        return rc;
+    }
     GemvArgs a = base_args(p);
     a.W = packed + p->off_d;
     a.blk_s = p->blk_d;

@@ -1,0 +1,424 @@
+// Decode projections (B <= 16 tokens) on the 5th-generation tensor cores.
+//
+// D[128 weight rows][NX columns] = W[128][K] . X[NX][K]^T in TMEM, where X
+// holds the B tokens' activation rows (bf16; with SPLIT, hi parts in rows
+// 0..B-1 and lo parts in rows NX/2..NX/2+B-1, the rest zero).  The kernel is bound by
+// streaming the weights from HBM: TMA brings 128-row x 64-column weight tiles
+// (16 KB, 128-byte swizzle) and the matching activation tile into a ~10-stage
+// shared-memory ring, one thread issues four M=128, N=NX, K=16 tcgen05.mma per
+// stage, and the tensor pipe idles most of the time.  192 threads: warp 0 TMA
+// producer, warp 1 TMEM owner and MMA issuer, warps 2-5 epilogue (one TMEM
+// lane = one weight row each).
+//
+// Work division ("stream-K"): the k-blocks of every (row tile, segment) are
+// laid end to end, tile-major then segment then k, and each CTA takes one
+// contiguous range, so every SM streams the same number of weight bytes.
+// A run of k-blocks of one (tile, segment) inside a CTA is one MMA chain (a
+// "piece").  Segments are the row-parallel shards ("Tensor parallel scaling
+// curves", "What tensor parallelism actually splits"); column-parallel
+// projections have one.  Order of the sums, fixed for a given SM count:
+//   segment sum = pieces in k order;  tile sum = segment sums in shard order.
+// A tile whose k-blocks all lie in one CTA is finished in registers.  A tile
+// split across CTAs has each CTA store its pieces to the workspace and add its
+// k-block count to the tile's arrival counter; the CTA that completes the
+// count adds all pieces in the fixed order (no CTA waits for another) and
+// resets the counter.  The fused and separate row-split modes run the same
+// pieces and sums, so they agree bit for bit.
+//
+// Weight tiles for the first stages are requested before the dependency wait
+// (programmatic dependent launch): weights never depend on the previous
+// kernel.  Every wait is bounded (2 s); a timeout sets the error word, stops
+// every role, waits (bounded) for copies in flight and releases TMEM.
+#pragma once
+
+#include <cuda.h>
+
+#include "tpl_common.cuh"
+#include "tpl_gemm.cuh"
+
+namespace tpl {
+
+constexpr int kGtThreads = 192;
+constexpr int kGtRows = 128;     // weight rows per tile (MMA M)
+constexpr int kGtK = 64;         // columns per k-block
+constexpr int kGtWBytes = kGtRows * kGtK * 2;  // 16 KB
+constexpr int kGtBufs = 4;       // TMEM accumulators in flight
+constexpr int kGtMaxB = 16;
+constexpr int kGtBarBytes = 512;  // mbarriers and flags after the stage ring
+
+template <int NX>
+struct GemvTcSmem {
+    static constexpr int XBYTES = NX * kGtK * 2;
+    static constexpr int STAGE = kGtWBytes + XBYTES;
+    static constexpr int NS = (200 * 1024) / STAGE;
+    static constexpr int BYTES = NS * STAGE + 1024 + kGtBarBytes;
+};
+
+enum { GT_QKV = 0, GT_GU = 1, GT_ROW = 2, GT_ROW_PARTIAL = 3 };
+
+struct GemvTcArgs {
+    CUtensorMap tm_w;   // column ops: 2-D [N][ld]; row ops: 3-D [t][N][ld]
+    CUtensorMap tm_x;   // [rows_x][K_x] bf16, box {64, NX}
+    int N;              // output rows
+    int B;              // tokens
+    int tiles, nseg, kbs;  // row tiles, segments per tile, k-blocks per segment
+    int64_t U;          // tiles * nseg * kbs
+    int x_seg_stride;   // X column offset between segments (row ops), elements
+    int w3d;
+    int epi;
+    // outputs
+    float *out32;       // GT_ROW
+    void *out_act;      // GT_ROW / GT_GU (bf16)
+    const void *resid;  // GT_ROW
+    int resid_f32;
+    float *partials;    // GT_ROW_PARTIAL: [nseg][B][N]
+    // QKV scatter (as the matrix-vector kernel)
+    float *q;
+    float *knew, *vnew;
+    __nv_bfloat16 *kc, *vc;
+    int rps, nq, nq_s, nkv_s, hd, batch_cap;
+    int64_t S, seq_cap;
+    // cross-CTA pieces and arrival counters
+    float *gpart;       // [G][2][nseg][128][B]
+    unsigned *tickets;  // [tiles]
+};
+
+template <int NX>
+__device__ __forceinline__ void tmem_ld_nx(uint32_t taddr, float (&v)[NX]) {
+    if constexpr (NX == 16) {
+        float t[16];
+        tmem_ld16(taddr, t);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = t[i];
+    } else {
+        float t0[16], t1[16];
+        tmem_ld16(taddr, t0);
+        tmem_ld16(taddr + 16, t1);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            v[i] = t0[i];
+            v[16 + i] = t1[i];
+        }
+    }
+}
+
+// CTA c's unit range [u0, u1) of U units over G CTAs.
+__device__ __forceinline__ int64_t gt_start(int64_t U, int G, int c) { return U * c / G; }
+
+// Final write of one output row for all tokens (fused sums or column ops).
+__device__ __forceinline__ void gt_final(const GemvTcArgs &a, int row, const float (&v)[kGtMaxB], int lane) {
+    const int B = a.B;
+    if (a.epi == GT_GU) {
+        // rows interleave gate and up: the even lane pairs with its odd neighbour
+#pragma unroll
+        for (int b = 0; b < kGtMaxB; ++b) {
+            const float u = __shfl_down_sync(0xffffffffu, v[b], 1);
+            if (b < B && !(lane & 1) && row + 1 < a.N)
+                static_cast<__nv_bfloat16 *>(a.out_act)[(int64_t)b * (a.N / 2) + row / 2] =
+                    __float2bfloat16_rn(silu(v[b]) * u);
+        }
+        return;
+    }
+    if (row >= a.N) return;
+    if (a.epi == GT_QKV) {
+        const int s = row / a.rps, l = row % a.rps;
+        const int qd = a.nq_s * a.hd, kd = a.nkv_s * a.hd;
+#pragma unroll
+        for (int b = 0; b < kGtMaxB; ++b) {
+            if (b >= B) continue;
+            if (l < qd) {
+                const int head = s * a.nq_s + l / a.hd, dim = l % a.hd;
+                a.q[((int64_t)b * a.nq + head) * a.hd + dim] = v[b];
+            } else {
+                const bool isk = l < qd + kd;
+                const int ll = isk ? l - qd : l - qd - kd;
+                const int kvl = ll / a.hd, dim = ll % a.hd;
+                __nv_bfloat16 *c = isk ? a.kc : a.vc;
+                c[((((int64_t)s * a.batch_cap + b) * a.nkv_s + kvl) * a.seq_cap + a.S) * a.hd + dim] =
+                    __float2bfloat16_rn(v[b]);
+                float *f = isk ? a.knew : a.vnew;
+                if (f) f[((int64_t)b * (a.nkv_s * (a.nq / a.nq_s)) + s * a.nkv_s + kvl) * a.hd + dim] = v[b];
+            }
+        }
+        return;
+    }
+    // GT_ROW: out = resid + sum
+#pragma unroll
+    for (int b = 0; b < kGtMaxB; ++b) {
+        if (b >= B) continue;
+        const int64_t i = (int64_t)b * a.N + row;
+        float o = v[b];
+        if (a.resid) o = load_act(a.resid, a.resid_f32, i) + o;
+        if (a.out32) a.out32[i] = o;
+        if (a.out_act) static_cast<__nv_bfloat16 *>(a.out_act)[i] = __float2bfloat16_rn(o);
+    }
+}
+
+template <int NX, bool SPLIT>
+__global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_constant__ GemvTcArgs a) {
+    constexpr int STAGE = GemvTcSmem<NX>::STAGE;
+    constexpr int NS = GemvTcSmem<NX>::NS;
+    static_assert(2 * NS * 8 + 2 * kGtBufs * 8 + 8 + 4 + 16 <= kGtBarBytes, "barrier area");
+    constexpr int TMEM_COLS = kGtBufs * NX <= 32 ? 32 : kGtBufs * NX <= 64 ? 64 : 128;
+    static_assert(kGtBufs * NX <= 128, "accumulators");
+    extern __shared__ __align__(1024) unsigned char gv_raw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>(((uintptr_t)gv_raw + 1023) & ~(uintptr_t)1023);
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + NS * STAGE);
+    uint64_t *empty = full + NS;
+    uint64_t *acc_full = empty + NS;       // [kGtBufs]
+    uint64_t *acc_empty = acc_full + kGtBufs;  // [kGtBufs]
+    uint64_t *fin = acc_empty + kGtBufs;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(fin + 1);
+    volatile int *s_fail = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    int *s_issued = const_cast<int *>(s_fail) + 1;
+    int *s_consumed = const_cast<int *>(s_fail) + 2;
+    volatile int *s_last = const_cast<int *>(s_fail) + 3;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = gridDim.x, cta = blockIdx.x;
+    const int64_t u0 = gt_start(a.U, G, cta), u1 = gt_start(a.U, G, cta + 1);
+    const int64_t per_tile = (int64_t)a.nseg * a.kbs;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < kGtBufs; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 4);
+        }
+        mbar_init(fin, 1);
+        *s_fail = 0;
+        *s_issued = 0;
+        *s_consumed = 0;
+        *s_last = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // weight tiles of the first stages before the dependency wait
+            const int64_t pre = (u1 - u0) < (int64_t)NS ? (u1 - u0) : (int64_t)NS;
+            auto coords = [&](int64_t u, int &tile, int &seg, int &kb) {
+                tile = (int)(u / per_tile);
+                const int64_t w = u % per_tile;
+                seg = (int)(w / a.kbs);
+                kb = (int)(w % a.kbs);
+            };
+            for (int64_t i = 0; i < pre; ++i) {
+                int tile, seg, kb;
+                coords(u0 + i, tile, seg, kb);
+                unsigned char *st = sm + i * STAGE;
+                mbar_expect_tx(&full[i], STAGE);
+                if (a.w3d) tma_load_3d(st, &a.tm_w, kb * kGtK, tile * kGtRows, seg, &full[i]);
+                else tma_load_2d(st, &a.tm_w, kb * kGtK, tile * kGtRows, &full[i]);
+            }
+            pdl_wait();
+            pdl_trigger();
+            int it = 0;
+            for (int64_t u = u0; u < u1; ++u, ++it) {
+                int tile, seg, kb;
+                coords(u, tile, seg, kb);
+                const int s = it % NS;
+                unsigned char *st = sm + s * STAGE;
+                if (it >= pre) {
+                    const unsigned ph = (unsigned)(it / NS) & 1u;
+                    if (*s_fail || !mbar_wait(&empty[s], ph ^ 1u)) {
+                        *s_fail = 1;
+                        break;
+                    }
+                    mbar_expect_tx(&full[s], STAGE);
+                    if (a.w3d) tma_load_3d(st, &a.tm_w, kb * kGtK, tile * kGtRows, seg, &full[s]);
+                    else tma_load_2d(st, &a.tm_w, kb * kGtK, tile * kGtRows, &full[s]);
+                }
+                tma_load_2d(st + kGtWBytes, &a.tm_x, seg * a.x_seg_stride + kb * kGtK, 0, &full[s]);
+            }
+            *s_issued = it;
+        }
+    } else if (warp == 1) {
+        pdl_wait();
+        pdl_trigger();
+        if (lane == 0) {
+            constexpr uint32_t IDESC = umma_idesc(kGtRows, NX);
+            int it = 0, c = 0;
+            bool ok = true;
+            for (int64_t u = u0; ok && u < u1; ++c) {
+                // one piece: the run of k-blocks of one (tile, segment)
+                const int64_t seg_end = (u / a.kbs + 1) * a.kbs;  // segments are kbs-aligned in u
+                const int64_t pe = min(u1, seg_end);
+                const int b = c % kGtBufs;
+                const unsigned use = (unsigned)(c / kGtBufs);
+                if (*s_fail || !mbar_wait(&acc_empty[b], (use & 1u) ^ 1u)) {
+                    ok = false;
+                    break;
+                }
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                const uint32_t d = tmem + (uint32_t)(b * NX);
+                for (int64_t v = u; v < pe; ++v, ++it) {
+                    const int s = it % NS;
+                    if (*s_fail || !mbar_wait(&full[s], (unsigned)(it / NS) & 1u)) {
+                        ok = false;
+                        break;
+                    }
+                    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                    const unsigned sw = smem_u32(sm + s * STAGE);
+                    const unsigned sx = sw + kGtWBytes;
+#pragma unroll
+                    for (int k = 0; k < kGtK / 16; ++k)
+                        umma(d, umma_desc(sw + 32 * k), umma_desc(sx + 32 * k), IDESC, (v > u || k > 0) ? 1u : 0u);
+                    umma_commit(&empty[s]);
+                }
+                if (!ok) break;
+                umma_commit(&acc_full[b]);
+                u = pe;
+            }
+            if (!ok) *s_fail = 1;
+            *s_consumed = it;
+            umma_commit(fin);
+            if (!mbar_wait(fin, 0)) *s_fail = 1;
+        }
+    } else {
+        pdl_wait();
+        pdl_trigger();
+        // ---- epilogue: thread = weight row 32*(warp%4) + lane of the tile ----
+        // A warp whose wait runs out keeps walking the same pieces with the
+        // work suppressed (`dead`), so the named barriers below still meet.
+        const int q = warp & 3;
+        const int r = 32 * q + lane;
+        const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+        const int B = a.B;
+        const int ep_tid = threadIdx.x - 64;  // 0..127
+        float seg_sum[kGtMaxB], tile_sum[kGtMaxB];
+        int c = 0;
+        bool dead = false;
+        int64_t u = u0;
+        while (u < u1) {
+            const int tile = (int)(u / per_tile);
+            const int64_t t_beg = (int64_t)tile * per_tile, t_end = t_beg + per_tile;
+            const bool local = t_beg >= u0 && t_end <= u1;
+            const int slot = (tile == (int)(u0 / per_tile)) ? 0 : 1;
+            const int64_t stop = min(u1, t_end);
+            while (u < stop) {
+                const int seg = (int)((u % per_tile) / a.kbs);
+                const int64_t pe = min(stop, (u / a.kbs + 1) * a.kbs);
+                const int b = c % kGtBufs;
+                ++c;
+                u = pe;
+                if (!dead)
+                    dead = !__all_sync(0xffffffffu,
+                                       !*s_fail && mbar_wait(&acc_full[b], (unsigned)((c - 1) / kGtBufs) & 1u));
+                if (dead) {
+                    *s_fail = 1;
+                    continue;
+                }
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                float d[NX];
+                tmem_ld_nx<NX>(tmem + lane_off + (uint32_t)(b * NX), d);
+                asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[b]);
+                // token t: hi part in column t, lo part in column NX/2 + t
+                float pv[kGtMaxB];
+#pragma unroll
+                for (int t = 0; t < kGtMaxB; ++t) {
+                    if constexpr (SPLIT) pv[t] = t < NX / 2 ? d[t] + d[NX / 2 + t] : 0.f;
+                    else pv[t] = t < NX ? d[t] : 0.f;
+                }
+                if (local) {
+                    // every segment of a tile inside this CTA is one piece
+#pragma unroll
+                    for (int t = 0; t < kGtMaxB; ++t) tile_sum[t] = (seg == 0 ? -0.f : tile_sum[t]) + pv[t];
+                    if (a.epi == GT_ROW_PARTIAL) {
+                        const int row = tile * kGtRows + r;
+                        if (row < a.N)
+#pragma unroll
+                            for (int t = 0; t < kGtMaxB; ++t)
+                                if (t < B) a.partials[((int64_t)seg * B + t) * a.N + row] = pv[t];
+                    }
+                } else {
+                    float *dst = a.gpart + ((((int64_t)cta * 2 + slot) * a.nseg + seg) * kGtRows + r) * B;
+#pragma unroll
+                    for (int t = 0; t < kGtMaxB; ++t)
+                        if (t < B) dst[t] = pv[t];
+                }
+            }
+            const int row = tile * kGtRows + r;
+            if (local) {
+                if (!dead && a.epi != GT_ROW_PARTIAL) gt_final(a, row, tile_sum, lane);
+                continue;
+            }
+            // shared tile: publish the pieces; the CTA completing the tile adds them
+            __threadfence();
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (ep_tid == 0) {
+                bool last = false;
+                if (!*s_fail) {
+                    const unsigned mine = (unsigned)(stop - max(u0, t_beg));
+                    const unsigned prev = atomicAdd(&a.tickets[tile], mine);
+                    last = prev + mine == (unsigned)per_tile;
+                    if (prev + mine > (unsigned)per_tile) record_error(16u);
+                    if (last) atomicExch(&a.tickets[tile], 0u);
+                }
+                *s_last = last ? 1 : 0;
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (!*s_last) continue;
+            __threadfence();
+            // CTAs covering this tile, in order; each stored its part in slot 0
+            // if the tile is its first, else in slot 1
+            int cf = (int)((t_beg * G) / a.U);
+            while (cf > 0 && gt_start(a.U, G, cf) > t_beg) --cf;
+            while (gt_start(a.U, G, cf + 1) <= t_beg) ++cf;
+#pragma unroll
+            for (int t = 0; t < kGtMaxB; ++t) tile_sum[t] = -0.f;
+            for (int s = 0; s < a.nseg; ++s) {
+                const int64_t sb = t_beg + (int64_t)s * a.kbs, se = sb + a.kbs;
+#pragma unroll
+                for (int t = 0; t < kGtMaxB; ++t) seg_sum[t] = -0.f;
+                for (int cc = cf; cc < G; ++cc) {
+                    const int64_t c0 = gt_start(a.U, G, cc), c1 = gt_start(a.U, G, cc + 1);
+                    if (c0 >= t_end) break;
+                    if (c1 <= sb || c0 >= se) continue;  // no piece of this segment
+                    const int sl = (tile == (int)(c0 / per_tile)) ? 0 : 1;
+                    const float *src = a.gpart + ((((int64_t)cc * 2 + sl) * a.nseg + s) * kGtRows + r) * B;
+#pragma unroll
+                    for (int t = 0; t < kGtMaxB; ++t)
+                        if (t < B) seg_sum[t] = seg_sum[t] + __ldcg(src + t);
+                }
+                if (a.epi == GT_ROW_PARTIAL) {
+                    if (row < a.N)
+#pragma unroll
+                        for (int t = 0; t < kGtMaxB; ++t)
+                            if (t < B) a.partials[((int64_t)s * B + t) * a.N + row] = seg_sum[t];
+                } else {
+#pragma unroll
+                    for (int t = 0; t < kGtMaxB; ++t) tile_sum[t] = tile_sum[t] + seg_sum[t];
+                }
+            }
+            if (a.epi != GT_ROW_PARTIAL) gt_final(a, row, tile_sum, lane);
+        }
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (*s_fail && threadIdx.x == 0) {
+        record_error(4u);
+        for (int it = *s_consumed; it < *s_issued; ++it) mbar_wait(&full[it % NS], (unsigned)(it / NS) & 1u);
+    }
+    __syncthreads();
+    if (warp == 1) {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+    }
+}
+
+}  // namespace tpl

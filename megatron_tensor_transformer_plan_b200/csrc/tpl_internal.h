@@ -27,6 +27,8 @@ constexpr int kTicketAttn = 0;             // [0, 1024): attention pairs
 constexpr int kTicketGemv = 1024;          // + 512 * op
 constexpr int kMaxPairs = 1024;
 constexpr int kMaxRowBlocks = 512;
+constexpr int kGemvTcMaxCtas = 256;        // CTAs of one tensor-core decode projection at most
+constexpr int kGemvTcMaxTiles = 512;       // 128-row tiles per projection (one arrival counter each)
 
 enum GemvOp { OP_QKV = 0, OP_O = 1, OP_GU = 2, OP_DOWN = 3 };
 
@@ -41,7 +43,7 @@ struct tpl_plan {
     int64_t blk_qkv, blk_o, blk_gu, blk_d;  // byte stride between shard blocks
     int64_t off_qkv, off_o, off_gu, off_d, off_g1, off_g2, packed_bytes;
     std::atomic<long long> reductions;
-    int gemv_mode;  // 0: tensor-core fragments (bf16); 1: fp32 FFMA; 2: bf16 FFMA
+    int gemv_mode;  // 0: mma.sync fragments (bf16); 1: fp32 FFMA; 2: bf16 FFMA; 3: tcgen05 + TMA (bf16)
     int attn_prefill_mode;  // 0: tcgen05 (power-of-two group sizes); 1: mma.sync
 };
 
@@ -78,7 +80,10 @@ struct AttnGeom {
 void attn_geom(int B, int nkv, int64_t keys, AttnGeom *a);
 
 struct WsLayout {
-    size_t tickets, q, o, h, act, ybuf0, ybuf1, P, knew, vnew, part_o, part_ml, gp, total;
+    size_t tickets, q, o, h, act, ybuf0, ybuf1, P, knew, vnew, part_o, part_ml, gp;
+    size_t xs;     // normalised activation as bf16 hi + lo rows [2B][hidden] (tcgen05 projections)
+    size_t gpart;  // cross-CTA pieces of the tcgen05 projections
+    size_t total;
 };
 int ws_layout(const tpl_plan *p, int B, int64_t S, WsLayout *w);
 

@@ -150,6 +150,8 @@ int ws_layout(const tpl_plan *p, int B, int64_t S, WsLayout *w) {
         gp = std::max(gp, gg.gp_floats);
     if (gemv_geom((int)H, p->t, p->F_s, B, xb, sms, &gg) == TPL_OK) gp = std::max(gp, gg.gp_floats);
     w->gp = take(gp * 4 + 4);
+    w->xs = take((size_t)32 * H * 2);  // [NX <= 32][hidden] bf16
+    w->gpart = take((size_t)kGemvTcMaxCtas * 2 * p->t * 128 * B * 4);
     w->total = off;
     return TPL_OK;
 }
@@ -245,7 +247,7 @@ void tpl_plan_destroy(tpl_plan *plan) { delete plan; }
 int tpl_plan_set_option(tpl_plan *p, int32_t option, int32_t value) {
     if (!p) return TPL_EINVAL;
     if (option == TPL_OPT_GEMV_MODE) {
-        if (value != 0 && value != 2) return TPL_EINVAL;
+        if (value != 0 && value != 2 && value != 3) return TPL_EINVAL;
         if (p->f32) return value == 0 ? TPL_OK : TPL_EINVAL;
         p->gemv_mode = value;
         return TPL_OK;

@@ -22,114 +22,12 @@
 #include "tpl_attn_prefill.cuh"
 #include "tpl_attn_tc.cuh"
 #include "tpl_gemm.cuh"
+#include "tpl_norm.cuh"
+#include "tpl_tma.h"
 
 namespace tpl {
 
-// a = x * gamma / sqrt(mean(x^2) + eps) (or a = x without TPL_NORM), split
-// into bf16 hi = rn(a) and lo = rn(a - hi).  One CTA per token row.
-__global__ void __launch_bounds__(256) norm_split_kernel(const void *x, int x_f32, const float *gamma, float eps,
-                                                         int norm, int H, __nv_bfloat16 *hi, __nv_bfloat16 *lo) {
-    __shared__ float s_red[8];
-    pdl_wait();
-    pdl_trigger();
-    const int64_t row = blockIdx.x;
-    const int n8 = H / 8;
-    float ss = 0.f;
-    for (int c = threadIdx.x; c < n8; c += blockDim.x) {
-        float v[8];
-        if (x_f32) {
-            const float4 *p = reinterpret_cast<const float4 *>(static_cast<const float *>(x) + row * H + 8 * c);
-            const float4 u0 = p[0], u1 = p[1];
-            v[0] = u0.x; v[1] = u0.y; v[2] = u0.z; v[3] = u0.w; v[4] = u1.x; v[5] = u1.y; v[6] = u1.z; v[7] = u1.w;
-        } else {
-            const uint4 u = *reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(x) + row * H + 8 * c);
-            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-            for (int e = 0; e < 4; ++e) {
-                v[2 * e] = bf16lo(w[e]);
-                v[2 * e + 1] = bf16hi(w[e]);
-            }
-        }
-        for (int e = 0; e < 8; ++e) ss += v[e] * v[e];
-    }
-    float inv = 1.f;
-    if (norm) {
-        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = ss;
-        __syncthreads();
-        float tot = 0.f;
-        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += s_red[w];
-        inv = 1.0f / sqrtf(tot / (float)H + eps);
-    }
-    for (int c = threadIdx.x; c < n8; c += blockDim.x) {
-        float v[8];
-        if (x_f32) {
-            const float4 *p = reinterpret_cast<const float4 *>(static_cast<const float *>(x) + row * H + 8 * c);
-            const float4 u0 = p[0], u1 = p[1];
-            v[0] = u0.x; v[1] = u0.y; v[2] = u0.z; v[3] = u0.w; v[4] = u1.x; v[5] = u1.y; v[6] = u1.z; v[7] = u1.w;
-        } else {
-            const uint4 u = *reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(x) + row * H + 8 * c);
-            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-            for (int e = 0; e < 4; ++e) {
-                v[2 * e] = bf16lo(w[e]);
-                v[2 * e + 1] = bf16hi(w[e]);
-            }
-        }
-        uint32_t h4[4], l4[4];
-        for (int e = 0; e < 4; ++e) {
-            float a0 = v[2 * e], a1 = v[2 * e + 1];
-            if (norm) {
-                a0 = a0 * inv * gamma[8 * c + 2 * e];
-                a1 = a1 * inv * gamma[8 * c + 2 * e + 1];
-            }
-            h4[e] = pack_bf16x2(a0, a1);
-            l4[e] = pack_bf16x2(a0 - bf16lo(h4[e]), a1 - bf16hi(h4[e]));
-        }
-        *reinterpret_cast<uint4 *>(hi + row * H + 8 * c) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
-        *reinterpret_cast<uint4 *>(lo + row * H + 8 * c) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
-    }
-}
-
 namespace {
-
-// ---- tensor maps (driver entry point fetched through the runtime) ---------
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-std::atomic<EncodeTiledFn> g_encode{nullptr};
-
-EncodeTiledFn encode_fn() {
-    EncodeTiledFn f = g_encode.load();
-    if (f) return f;
-    void *p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess || !p)
-        return nullptr;
-    f = reinterpret_cast<EncodeTiledFn>(p);
-    g_encode.store(f);
-    return f;
-}
-
-// bf16 matrix [rows][cols] with `row_bytes` between rows (and, for 3-D,
-// `planes` of them `plane_bytes` apart); boxes of box_cols x box_rows with the
-// 128-byte swizzle the MMA descriptors expect; out-of-range elements read 0.
-int make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint64_t row_bytes, uint32_t box_cols,
-             uint32_t box_rows, uint64_t planes = 0, uint64_t plane_bytes = 0, uint32_t box_planes = 1) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return TPL_ECUDA;
-    if (((uintptr_t)base & 15u) || (row_bytes & 15u) || (plane_bytes & 15u)) return TPL_EINVAL;
-    const cuuint64_t gdim[3] = {cols, rows, planes};
-    const cuuint64_t gstr[2] = {row_bytes, plane_bytes};
-    const cuuint32_t box[3] = {box_cols, box_rows, box_planes};
-    const cuuint32_t es[3] = {1, 1, 1};
-    const cuuint32_t rank = planes ? 3 : 2;
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), gdim, gstr, box, es,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? TPL_OK : TPL_EINVAL;
-}
 
 // ---- GEMM launches ---------------------------------------------------------
 
@@ -211,7 +109,7 @@ int run_norm_split(const tpl_plan *p, const void *x, int x_f32, const float *gam
                    __nv_bfloat16 *lo, cudaStream_t st) {
     const int norm = (p->d.flags & TPL_NORM) ? 1 : 0;
     return cuda_rc(launch_pdl(norm_split_kernel, T, 256, 0, st, x, x_f32, gamma, p->d.rms_eps, norm, p->d.hidden, hi,
-                              lo));
+                              lo, T));
 }
 
 bool g_ap_attr[64];

@@ -125,12 +125,15 @@ int tpl_plan_create(const tpl_dims *dims, int32_t t, tpl_plan **out);
 void tpl_plan_destroy(tpl_plan *plan);
 
 /* Plan options (host).  TPL_OPT_GEMV_MODE selects the kernels of the bf16
- * decode projections: 0 = register-streamed weights on mma.sync (the
- * default), 2 = FFMA on the CUDA cores (kept to measure against), 3 = weights
- * streamed by TMA into a shared-memory ring and multiplied on the
- * 5th-generation tensor cores (tcgen05, accumulators in TMEM), the normalised
- * activation computed once per step by a small RMSNorm kernel.  fp32 plans
- * always use FFMA.  TPL_OPT_PREFILL_ATTN selects the prefill attention kernel:
+ * decode projections: 0 = register-streamed weights on mma.sync, 2 = FFMA on
+ * the CUDA cores (kept to measure against), 3 = weights streamed by TMA into
+ * a shared-memory ring and multiplied on the 5th-generation tensor cores
+ * (tcgen05, accumulators in TMEM; the normalised activation is computed by a
+ * small RMSNorm kernel), 4 = the default: the tcgen05 kernels for every
+ * projection of layers with at least 1 GiB of weights when more than 8
+ * tokens are decoded, mma.sync otherwise (the choice that measured faster on
+ * B200; layers mixing the two families measured slower than either).  fp32
+ * plans always use FFMA.  TPL_OPT_PREFILL_ATTN selects the prefill attention kernel:
  * 0 = 5th-generation tensor cores (tcgen05, TMEM; the default when the
  * query group size is a power of two), 1 = mma.sync (any group size; kept to
  * measure against).  Returns TPL_EINVAL for an unknown option or value. */

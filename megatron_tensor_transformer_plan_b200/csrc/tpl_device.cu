@@ -126,7 +126,7 @@ int gemv_launch(Ctx &c, GemvArgs &a, int N, int nseg, int Kseg, int op) {
     if (sms <= 0) return TPL_ECUDA;
     // The Q projection feeds a softmax and gate/up feeds SwiGLU: carry their
     // normalised activations as bf16 hi + lo.
-    const int mode = p->f32 ? 1 : (p->gemv_mode == 2 ? 2 : ((op == OP_QKV || op == OP_GU) ? 3 : 0));
+    const int mode = p->f32 ? 1 : (p->gemv_mode == 2 ? 2 : ((op == OP_QKV || op == OP_GU) ? 3 : 0));  // modes 0, 4
     int rc = gemv_geom(N, nseg, Kseg, c.B, p->f32 ? 4 : 2, sms, &a.g, mode == 3 ? 2 : 1);
     if (rc != TPL_OK) return rc;
     const bool big = c.B > 8;
@@ -209,6 +209,23 @@ int gemv_tc_run(Ctx &c, GemvTcArgs &a, int op, bool split, const void *W, int64_
     a.tickets = reinterpret_cast<unsigned *>(c.ws + c.L.tickets) + kTicketGemv + 512 * op;
     if (split) return nx == 16 ? gt_go<16, true>(0, a, c.st) : gt_go<32, true>(1, a, c.st);
     return gt_go<16, false>(2, a, c.st);
+}
+
+// TPL_OPT_GEMV_MODE 4 (the default for bf16 plans): one kernel family for all
+// four projections of a layer, the one that measured faster on B200.  The
+// tcgen05 kernel streams large matrices closer to the copy bandwidth, but the
+// mma.sync kernel overlaps consecutive launches better (programmatic
+// dependent launch), and layers that mix the two families measured slower
+// than either.  So: tcgen05 with more than 8 tokens on layers of at least
+// 1 GiB of weights, mma.sync otherwise.
+bool use_tc(const tpl_plan *p, int op, int B) {
+    (void)op;
+    if (p->gemv_mode == 3) return B <= kGtMaxB;
+    if (p->gemv_mode != 4 || B > kGtMaxB) return false;
+    const tpl_dims &d = p->d;
+    const int64_t layer_params = (int64_t)(d.n_q_heads + 2 * d.n_kv_heads) * d.head_dim * d.hidden +
+                                 (int64_t)d.hidden * d.n_q_heads * d.head_dim + 3 * (int64_t)d.ffn * d.hidden;
+    return B > 8 && layer_params * 2 >= (1ll << 30);
 }
 
 GemvTcArgs gt_args(const tpl_plan *p) {
@@ -294,7 +311,7 @@ int run_row_tc(Ctx &c, const char *packed, int op, const void *x, const void *re
 
 int run_qkv(Ctx &c, const char *packed, const tpl_kv *kv, const void *x, float *q, float *knew, float *vnew) {
     tpl_plan *p = c.p;
-    if (p->gemv_mode == 3) return run_qkv_tc(c, packed, kv, x, q, knew, vnew);
+    if (use_tc(p, OP_QKV, c.B)) return run_qkv_tc(c, packed, kv, x, q, knew, vnew);
     GemvArgs a = base_args(p);
     a.W = packed + p->off_qkv;
     a.blk_r = p->blk_qkv;
@@ -356,7 +373,7 @@ int run_attn(Ctx &c, const tpl_kv *kv, const float *q, const float *knew, const 
 // Row-parallel O projection: fused (partials == NULL) or partial output.
 int run_o(Ctx &c, const char *packed, const void *o, const void *resid, float *h, float *partials) {
     tpl_plan *p = c.p;
-    if (p->gemv_mode == 3) {
+    if (use_tc(p, OP_O, c.B)) {
         int rc = run_row_tc(c, packed, OP_O, o, resid, 0, h, nullptr, partials);
         if (rc == TPL_OK && !partials) p->reductions.fetch_add(1);
         return rc;
@@ -385,7 +402,7 @@ int run_o(Ctx &c, const char *packed, const void *o, const void *resid, float *h
 
 int run_gu(Ctx &c, const char *packed, const void *h, int h_is_act, void *act) {
     tpl_plan *p = c.p;
-    if (p->gemv_mode == 3) return run_gu_tc(c, packed, h, h_is_act, act);
+    if (use_tc(p, OP_GU, c.B)) return run_gu_tc(c, packed, h, h_is_act, act);
     GemvArgs a = base_args(p);
     a.W = packed + p->off_gu;
     a.blk_r = p->blk_gu;
@@ -404,7 +421,7 @@ int run_gu(Ctx &c, const char *packed, const void *h, int h_is_act, void *act) {
 int run_down(Ctx &c, const char *packed, const void *act, const void *resid, int resid_f32, void *y, float *y32,
              float *partials) {
     tpl_plan *p = c.p;
-    if (p->gemv_mode == 3) {
+    if (use_tc(p, OP_DOWN, c.B)) {
         int rc = run_row_tc(c, packed, OP_DOWN, act, resid, resid_f32, y32, y, partials);
         if (rc == TPL_OK && !partials) p->reductions.fetch_add(1);
         return rc;

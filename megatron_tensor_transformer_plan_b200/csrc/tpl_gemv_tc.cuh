@@ -4,8 +4,8 @@
 // holds the B tokens' activation rows (bf16; with SPLIT, hi parts in rows
 // 0..B-1 and lo parts in rows NX/2..NX/2+B-1, the rest zero).  The kernel is bound by
 // streaming the weights from HBM: TMA brings 128-row x 64-column weight tiles
-// (16 KB, 128-byte swizzle) and the matching activation tile into a ~10-stage
-// shared-memory ring, one thread issues four M=128, N=NX, K=16 tcgen05.mma per
+// (16 KB, 128-byte swizzle) and the matching activation tile into a 10-11
+// stage shared-memory ring, one thread issues four M=128, N=NX, K=16 tcgen05.mma per
 // stage, and the tensor pipe idles most of the time.  192 threads: warp 0 TMA
 // producer, warp 1 TMEM owner and MMA issuer, warps 2-5 epilogue (one TMEM
 // lane = one weight row each).
@@ -44,7 +44,8 @@ constexpr int kGtK = 64;         // columns per k-block
 constexpr int kGtWBytes = kGtRows * kGtK * 2;  // 16 KB
 constexpr int kGtBufs = 4;       // TMEM accumulators in flight
 constexpr int kGtMaxB = 16;
-constexpr int kGtBarBytes = 512;  // mbarriers and flags after the stage ring
+constexpr int kGtList = 120;      // piece list entries per combine chunk
+constexpr int kGtBarBytes = 1024;  // mbarriers, flags and the piece list after the stage ring
 
 template <int NX>
 struct GemvTcSmem {
@@ -79,7 +80,7 @@ struct GemvTcArgs {
     int rps, nq, nq_s, nkv_s, hd, batch_cap;
     int64_t S, seq_cap;
     // cross-CTA pieces and arrival counters
-    float *gpart;       // [G][2][nseg][128][B]
+    float *gpart;       // [G][2][nseg][128][16]
     unsigned *tickets;  // [tiles]
 };
 
@@ -158,7 +159,7 @@ template <int NX, bool SPLIT>
 __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_constant__ GemvTcArgs a) {
     constexpr int STAGE = GemvTcSmem<NX>::STAGE;
     constexpr int NS = GemvTcSmem<NX>::NS;
-    static_assert(2 * NS * 8 + 2 * kGtBufs * 8 + 8 + 4 + 16 <= kGtBarBytes, "barrier area");
+    static_assert(2 * NS * 8 + 2 * kGtBufs * 8 + 8 + 4 + 32 + 4 * kGtList <= kGtBarBytes, "barrier area");
     constexpr int TMEM_COLS = kGtBufs * NX <= 32 ? 32 : kGtBufs * NX <= 64 ? 64 : 128;
     static_assert(kGtBufs * NX <= 128, "accumulators");
     extern __shared__ __align__(1024) unsigned char gv_raw[];
@@ -173,6 +174,9 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
     int *s_issued = const_cast<int *>(s_fail) + 1;
     int *s_consumed = const_cast<int *>(s_fail) + 2;
     volatile int *s_last = const_cast<int *>(s_fail) + 3;
+    volatile int *s_nlist = const_cast<int *>(s_fail) + 4;
+    volatile int *s_more = const_cast<int *>(s_fail) + 5;
+    volatile int *s_list = const_cast<int *>(s_fail) + 8;  // [kGtList]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = gridDim.x, cta = blockIdx.x;
@@ -204,31 +208,39 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = *tmem_slot;
+    // every thread lets the next kernel be scheduled; only what this kernel
+    // reads from earlier kernels (the activations) waits for them
+    pdl_trigger();
 
     if (warp == 0) {
         if (lane == 0) {
+            // (tile, segment, k-block) of unit u0, then stepped without divisions
+            int tile0 = (int)(u0 / per_tile);
+            const int w0 = (int)(u0 - (int64_t)tile0 * per_tile);
+            const int seg0 = w0 / a.kbs, kb0 = w0 - seg0 * a.kbs;
+            const int n = (int)(u1 - u0);
+            const int pre = n < NS ? n : NS;
             // weight tiles of the first stages before the dependency wait
-            const int64_t pre = (u1 - u0) < (int64_t)NS ? (u1 - u0) : (int64_t)NS;
-            auto coords = [&](int64_t u, int &tile, int &seg, int &kb) {
-                tile = (int)(u / per_tile);
-                const int64_t w = u % per_tile;
-                seg = (int)(w / a.kbs);
-                kb = (int)(w % a.kbs);
-            };
-            for (int64_t i = 0; i < pre; ++i) {
-                int tile, seg, kb;
-                coords(u0 + i, tile, seg, kb);
-                unsigned char *st = sm + i * STAGE;
-                mbar_expect_tx(&full[i], STAGE);
-                if (a.w3d) tma_load_3d(st, &a.tm_w, kb * kGtK, tile * kGtRows, seg, &full[i]);
-                else tma_load_2d(st, &a.tm_w, kb * kGtK, tile * kGtRows, &full[i]);
+            {
+                int tile = tile0, seg = seg0, kb = kb0;
+                for (int i = 0; i < pre; ++i) {
+                    unsigned char *st = sm + i * STAGE;
+                    mbar_expect_tx(&full[i], STAGE);
+                    if (a.w3d) tma_load_3d(st, &a.tm_w, kb * kGtK, tile * kGtRows, seg, &full[i]);
+                    else tma_load_2d(st, &a.tm_w, kb * kGtK, tile * kGtRows, &full[i]);
+                    if (++kb == a.kbs) {
+                        kb = 0;
+                        if (++seg == a.nseg) {
+                            seg = 0;
+                            ++tile;
+                        }
+                    }
+                }
             }
             pdl_wait();
-            pdl_trigger();
+            int tile = tile0, seg = seg0, kb = kb0;
             int it = 0;
-            for (int64_t u = u0; u < u1; ++u, ++it) {
-                int tile, seg, kb;
-                coords(u, tile, seg, kb);
+            for (; it < n; ++it) {
                 const int s = it % NS;
                 unsigned char *st = sm + s * STAGE;
                 if (it >= pre) {
@@ -242,12 +254,18 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
                     else tma_load_2d(st, &a.tm_w, kb * kGtK, tile * kGtRows, &full[s]);
                 }
                 tma_load_2d(st + kGtWBytes, &a.tm_x, seg * a.x_seg_stride + kb * kGtK, 0, &full[s]);
+                if (++kb == a.kbs) {
+                    kb = 0;
+                    if (++seg == a.nseg) {
+                        seg = 0;
+                        ++tile;
+                    }
+                }
             }
             *s_issued = it;
         }
     } else if (warp == 1) {
         pdl_wait();
-        pdl_trigger();
         if (lane == 0) {
             constexpr uint32_t IDESC = umma_idesc(kGtRows, NX);
             int it = 0, c = 0;
@@ -289,7 +307,6 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
         }
     } else {
         pdl_wait();
-        pdl_trigger();
         // ---- epilogue: thread = weight row 32*(warp%4) + lane of the tile ----
         // A warp whose wait runs out keeps walking the same pieces with the
         // work suppressed (`dead`), so the named barriers below still meet.
@@ -346,10 +363,11 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
                                 if (t < B) a.partials[((int64_t)seg * B + t) * a.N + row] = pv[t];
                     }
                 } else {
-                    float *dst = a.gpart + ((((int64_t)cta * 2 + slot) * a.nseg + seg) * kGtRows + r) * B;
+                    float4 *dst = reinterpret_cast<float4 *>(
+                        a.gpart + ((((int64_t)cta * 2 + slot) * a.nseg + seg) * kGtRows + r) * kGtMaxB);
 #pragma unroll
-                    for (int t = 0; t < kGtMaxB; ++t)
-                        if (t < B) dst[t] = pv[t];
+                    for (int t = 0; t < kGtMaxB; t += 4)
+                        if (t < B) dst[t / 4] = make_float4(pv[t], pv[t + 1], pv[t + 2], pv[t + 3]);
                 }
             }
             const int row = tile * kGtRows + r;
@@ -374,36 +392,90 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
             asm volatile("bar.sync 1, 128;" ::: "memory");
             if (!*s_last) continue;
             __threadfence();
-            // CTAs covering this tile, in order; each stored its part in slot 0
-            // if the tile is its first, else in slot 1
-            int cf = (int)((t_beg * G) / a.U);
-            while (cf > 0 && gt_start(a.U, G, cf) > t_beg) --cf;
-            while (gt_start(a.U, G, cf + 1) <= t_beg) ++cf;
+            // The tile's pieces in order (segment, then CTA), listed by one
+            // thread in shared memory in chunks, then loaded four at a time.
+            // Each CTA stored its part in slot 0 if the tile is its first,
+            // else in slot 1.
 #pragma unroll
-            for (int t = 0; t < kGtMaxB; ++t) tile_sum[t] = -0.f;
-            for (int s = 0; s < a.nseg; ++s) {
-                const int64_t sb = t_beg + (int64_t)s * a.kbs, se = sb + a.kbs;
-#pragma unroll
-                for (int t = 0; t < kGtMaxB; ++t) seg_sum[t] = -0.f;
-                for (int cc = cf; cc < G; ++cc) {
-                    const int64_t c0 = gt_start(a.U, G, cc), c1 = gt_start(a.U, G, cc + 1);
-                    if (c0 >= t_end) break;
-                    if (c1 <= sb || c0 >= se) continue;  // no piece of this segment
-                    const int sl = (tile == (int)(c0 / per_tile)) ? 0 : 1;
-                    const float *src = a.gpart + ((((int64_t)cc * 2 + sl) * a.nseg + s) * kGtRows + r) * B;
-#pragma unroll
-                    for (int t = 0; t < kGtMaxB; ++t)
-                        if (t < B) seg_sum[t] = seg_sum[t] + __ldcg(src + t);
+            for (int t = 0; t < kGtMaxB; ++t) {
+                tile_sum[t] = -0.f;
+                seg_sum[t] = -0.f;
+            }
+            int g_s = 0, g_cc = 0;  // generator position (thread 0)
+            if (ep_tid == 0) {
+                int cf = (int)((t_beg * G) / a.U);
+                while (cf > 0 && gt_start(a.U, G, cf) > t_beg) --cf;
+                while (gt_start(a.U, G, cf + 1) <= t_beg) ++cf;
+                g_cc = cf;
+            }
+            for (;;) {
+                if (ep_tid == 0) {
+                    int n = 0;
+                    while (n < kGtList && g_s < a.nseg) {
+                        const int64_t sb = t_beg + (int64_t)g_s * a.kbs, se = sb + a.kbs;
+                        const int64_t c0 = gt_start(a.U, G, g_cc), c1 = gt_start(a.U, G, g_cc + 1);
+                        if (c1 > sb && c0 < se) {
+                            const int sl = (tile == (int)(c0 / per_tile)) ? 0 : 1;
+                            const bool seg_last = c1 >= se;
+                            s_list[n++] = (((g_cc * 2 + sl) * a.nseg + g_s) << 5) | (g_s << 1) | (seg_last ? 1 : 0);
+                        }
+                        if (c1 >= se) {
+                            ++g_s;  // next segment starts in this same CTA
+                        } else {
+                            ++g_cc;
+                        }
+                    }
+                    *s_nlist = n;
                 }
-                if (a.epi == GT_ROW_PARTIAL) {
-                    if (row < a.N)
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                const int n = *s_nlist;
+                for (int e0 = 0; e0 < n; e0 += 4) {
+                    float4 v[4][kGtMaxB / 4];
 #pragma unroll
-                        for (int t = 0; t < kGtMaxB; ++t)
-                            if (t < B) a.partials[((int64_t)s * B + t) * a.N + row] = seg_sum[t];
-                } else {
+                    for (int j = 0; j < 4; ++j)
 #pragma unroll
-                    for (int t = 0; t < kGtMaxB; ++t) tile_sum[t] = tile_sum[t] + seg_sum[t];
+                        for (int q4 = 0; q4 < kGtMaxB / 4; ++q4) v[j][q4] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        if (e0 + j < n) {
+                            const int ent = s_list[e0 + j];
+                            const float4 *src = reinterpret_cast<const float4 *>(
+                                a.gpart + ((int64_t)(ent >> 5) * kGtRows + r) * kGtMaxB);
+#pragma unroll
+                            for (int q4 = 0; q4 < kGtMaxB / 4; ++q4)
+                                if (4 * q4 < B) v[j][q4] = __ldcg(src + q4);
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        if (e0 + j >= n) break;
+                        const int ent = s_list[e0 + j];
+#pragma unroll
+                        for (int q4 = 0; q4 < kGtMaxB / 4; ++q4) {
+                            seg_sum[4 * q4] = seg_sum[4 * q4] + v[j][q4].x;
+                            seg_sum[4 * q4 + 1] = seg_sum[4 * q4 + 1] + v[j][q4].y;
+                            seg_sum[4 * q4 + 2] = seg_sum[4 * q4 + 2] + v[j][q4].z;
+                            seg_sum[4 * q4 + 3] = seg_sum[4 * q4 + 3] + v[j][q4].w;
+                        }
+                        if (ent & 1) {  // the segment is complete
+                            const int sg = (ent >> 1) & 15;
+                            if (a.epi == GT_ROW_PARTIAL) {
+                                if (row < a.N)
+#pragma unroll
+                                    for (int t = 0; t < kGtMaxB; ++t)
+                                        if (t < B) a.partials[((int64_t)sg * B + t) * a.N + row] = seg_sum[t];
+                            } else {
+#pragma unroll
+                                for (int t = 0; t < kGtMaxB; ++t) tile_sum[t] = tile_sum[t] + seg_sum[t];
+                            }
+#pragma unroll
+                            for (int t = 0; t < kGtMaxB; ++t) seg_sum[t] = -0.f;
+                        }
+                    }
                 }
+                if (ep_tid == 0) *s_more = g_s < a.nseg ? 1 : 0;
+                asm volatile("bar.sync 1, 128;" ::: "memory");  // list consumed; flag visible
+                if (!*s_more) break;
             }
             if (a.epi != GT_ROW_PARTIAL) gt_final(a, row, tile_sum, lane);
         }

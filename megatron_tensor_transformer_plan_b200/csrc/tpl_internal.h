@@ -43,7 +43,8 @@ struct tpl_plan {
     int64_t blk_qkv, blk_o, blk_gu, blk_d;  // byte stride between shard blocks
     int64_t off_qkv, off_o, off_gu, off_d, off_g1, off_g2, packed_bytes;
     std::atomic<long long> reductions;
-    int gemv_mode;  // 0: mma.sync fragments (bf16); 1: fp32 FFMA; 2: bf16 FFMA; 3: tcgen05 + TMA (bf16)
+    int gemv_mode;  // 0: mma.sync fragments (bf16); 1: fp32 FFMA; 2: bf16 FFMA; 3: tcgen05 + TMA (bf16);
+                    // 4: per projection (default for bf16)
     int attn_prefill_mode;  // 0: tcgen05 (power-of-two group sizes); 1: mma.sync
 };
 

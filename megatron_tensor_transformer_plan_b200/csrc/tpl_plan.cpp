@@ -151,7 +151,7 @@ int ws_layout(const tpl_plan *p, int B, int64_t S, WsLayout *w) {
     if (gemv_geom((int)H, p->t, p->F_s, B, xb, sms, &gg) == TPL_OK) gp = std::max(gp, gg.gp_floats);
     w->gp = take(gp * 4 + 4);
     w->xs = take((size_t)32 * H * 2);  // [NX <= 32][hidden] bf16
-    w->gpart = take((size_t)kGemvTcMaxCtas * 2 * p->t * 128 * B * 4);
+    w->gpart = take((size_t)kGemvTcMaxCtas * 2 * p->t * 128 * 16 * 4);
     w->total = off;
     return TPL_OK;
 }
@@ -212,7 +212,7 @@ int tpl_plan_create(const tpl_dims *dims, int32_t t, tpl_plan **out) {
     p->qkv_rows_s = (p->nq_s + 2 * p->nkv_s) * dims->head_dim;
     p->f32 = (dims->flags & TPL_FP32_WEIGHTS) != 0;
     p->esize = p->f32 ? 4 : 2;
-    p->gemv_mode = p->f32 ? 1 : 0;
+    p->gemv_mode = p->f32 ? 1 : 4;
     p->attn_prefill_mode = 0;
     const int64_t H = dims->hidden, es = p->esize;
     // rows padded with zeros to whole 128-column blocks
@@ -247,7 +247,7 @@ void tpl_plan_destroy(tpl_plan *plan) { delete plan; }
 int tpl_plan_set_option(tpl_plan *p, int32_t option, int32_t value) {
     if (!p) return TPL_EINVAL;
     if (option == TPL_OPT_GEMV_MODE) {
-        if (value != 0 && value != 2 && value != 3) return TPL_EINVAL;
+        if (value != 0 && value != 2 && value != 3 && value != 4) return TPL_EINVAL;
         if (p->f32) return value == 0 ? TPL_OK : TPL_EINVAL;
         p->gemv_mode = value;
         return TPL_OK;

@@ -8,6 +8,7 @@ Workloads (seeded synthetic tensors):
   tiny-mlp    hidden 256, ffn 688, t=2, 1 token, no norm/residual (MLP block)
   7b          hidden 4096, 32/32 heads, ffn 11008, KV 2048, B in {1, 16}, t in {1, 2, 4}
   70b         hidden 8192, 64/8 heads, ffn 28672, KV 8192, B=16, t in {1, 4, 8}
+  70b-stack   one layer of the 80-layer stack: t=8, B=4, KV 4096
 Working sets under four times the L2 size rotate over several copies of the
 weights and caches so that every timed call reads from HBM. Timing: CUDA
 events around each call after 3 warm-up calls, median reported.
@@ -58,10 +59,11 @@ def time_calls(fn, copies, iters, stream):
     return statistics.median(a.elapsed_time(b) for a, b in ts) * 1e3  # us
 
 
-def run_layer(tpl, H, nq, nkv, F, t, B, S, iters, mode, flags=None, mlp_only=False):
+def run_layer(tpl, H, nq, nkv, F, t, B, S, iters, mode, flags=None, mlp_only=False, gemv_mode=4):
     dev = torch.device("cuda")
     flags = (tpl.TPL_NORM | tpl.TPL_RESIDUAL) if flags is None else flags
     plan = tpl.Plan(tpl.make_dims(H, nq, nkv, 128, F, 1, 1e-5, flags), t)
+    plan.set_option(tpl.TPL_OPT_GEMV_MODE, gemv_mode)
     nbytes = layer_bytes(H, nq, nkv, 128, F, B, S, mlp_only)
     ncopies = max(1, min(8, -(-4 * L2_BYTES // nbytes)))
     copies = []
@@ -94,6 +96,7 @@ def main() -> None:
     ap = argparse.ArgumentParser()
     ap.add_argument("--iters", type=int, default=30)
     ap.add_argument("--only", default="")
+    ap.add_argument("--gemv-mode", type=int, default=4, help="TPL_OPT_GEMV_MODE of the plan (4: the default)")
     args = ap.parse_args()
     build.build()
     from megatron_tensor_transformer_plan_b200 import tpl
@@ -105,6 +108,7 @@ def main() -> None:
             cases.append(("7b", dict(H=4096, nq=32, nkv=32, F=11008, t=t, B=B, S=2048)))
     for t in (1, 4, 8):
         cases.append(("70b", dict(H=8192, nq=64, nkv=8, F=28672, t=t, B=16, S=8192)))
+    cases.append(("70b-stack", dict(H=8192, nq=64, nkv=8, F=28672, t=8, B=4, S=4096)))
     for name, c in cases:
         if args.only and name != args.only:
             continue
@@ -112,9 +116,11 @@ def main() -> None:
             if c["t"] == 1 and mode == "separate":
                 continue
             us, nbytes, ncopies, rc = run_layer(tpl, c["H"], c["nq"], c["nkv"], c["F"], c["t"], c["B"], c["S"],
-                                                 args.iters, mode, c.get("flags"), c.get("mlp_only", False))
+                                                 args.iters, mode, c.get("flags"), c.get("mlp_only", False),
+                                                 args.gemv_mode)
             gbs = nbytes / (us * 1e-6) / 1e9
-            print(json.dumps({"workload": name, "t": c["t"], "B": c["B"], "S": c["S"], "reduce": mode,
+            print(json.dumps({"workload": name, "gemv_mode": args.gemv_mode, "t": c["t"], "B": c["B"], "S": c["S"],
+                              "reduce": mode,
                               "us_per_layer": round(us, 2), "algorithmic_bytes": nbytes, "gb_s": round(gbs, 1),
                               "frac_of_peak": round(gbs / peak, 4), "peak_gb_s": peak, "peak_kind": kind,
                               "weight_copies_rotated": ncopies, "device_status": rc}), flush=True)

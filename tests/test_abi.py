@@ -179,6 +179,8 @@ def test_workspace_grows_with_batch_and_length(tpl):
 def test_gemv_option(tpl):
     plan = tpl.Plan(tpl.make_dims(256, 2, 2, 128, 688), 2)
     plan.set_option(tpl.TPL_OPT_GEMV_MODE, 2)
+    plan.set_option(tpl.TPL_OPT_GEMV_MODE, 3)
+    plan.set_option(tpl.TPL_OPT_GEMV_MODE, 4)
     plan.set_option(tpl.TPL_OPT_GEMV_MODE, 0)
     with pytest.raises(tpl.TplError):
         plan.set_option(tpl.TPL_OPT_GEMV_MODE, 5)

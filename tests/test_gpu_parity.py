@@ -137,17 +137,22 @@ def test_config2_7b_layer(gpu, t, B):
 
 
 @pytest.mark.slow
-def test_config3_70b_layer(gpu):
-    """70B-shaped layer, t = 4 (2 kv heads per shard), batch 16, KV length 8192."""
+@pytest.mark.parametrize("gemv_mode", [4, 0])
+def test_config3_70b_layer(gpu, gemv_mode):
+    """70B-shaped layer, t = 4 (2 kv heads per shard), batch 16, KV length 8192;
+    the default kernel choice (4) and the mma.sync projections (0)."""
     L = make_layer(8192, 64, 8, 128, 28672, 4, 16, 8192, seed=0)
+    L.plan.set_option(tpl.TPL_OPT_GEMV_MODE, gemv_mode)
     ref_y, tr = oracle_decode(L)
     _check_layer(L, ref_y, tr)
 
 
 @pytest.mark.slow
-def test_stack_shape_layer(gpu):
+@pytest.mark.parametrize("gemv_mode", [4, 0])
+def test_stack_shape_layer(gpu, gemv_mode):
     """One layer at the 80-layer stack's shape: t = 8, batch 4, KV length 4096."""
     L = make_layer(8192, 64, 8, 128, 28672, 8, 4, 4096, seed=0, layer=39)
+    L.plan.set_option(tpl.TPL_OPT_GEMV_MODE, gemv_mode)
     ref_y, tr = oracle_decode(L)
     _check_layer(L, ref_y, tr)
 

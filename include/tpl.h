@@ -136,9 +136,15 @@ void tpl_plan_destroy(tpl_plan *plan);
  * plans always use FFMA.  TPL_OPT_PREFILL_ATTN selects the prefill attention kernel:
  * 0 = 5th-generation tensor cores (tcgen05, TMEM; the default when the
  * query group size is a power of two), 1 = mma.sync (any group size; kept to
- * measure against).  Returns TPL_EINVAL for an unknown option or value. */
+ * measure against).  TPL_OPT_DECODE_ATTN selects the decode attention kernel:
+ * 0 = keys staged through a per-warp shared-memory ring (the default for
+ * query groups of at most 8 heads when every (shard, sequence, kv head) pair
+ * gets at least two CTAs in one wave of SMs; other shapes use the other
+ * kernel), 1 = keys streamed into registers (any shape).
+ * Returns TPL_EINVAL for an unknown option or value. */
 #define TPL_OPT_GEMV_MODE 1
 #define TPL_OPT_PREFILL_ATTN 2
+#define TPL_OPT_DECODE_ATTN 3
 int tpl_plan_set_option(tpl_plan *plan, int32_t option, int32_t value);
 
 /* Footprints (host) -- see tpl_plan_info. */

@@ -36,25 +36,6 @@ struct AttnPrefillArgs {
     __nv_bfloat16 *o_hi, *o_lo;       // [T][nq*128]: output as bf16 hi + lo (the O projection's split operand)
 };
 
-__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((unsigned)__cvta_generic_to_shared(dst)), "l"(src)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
-__device__ __forceinline__ void ldsm_x4(const void *p, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"((unsigned)__cvta_generic_to_shared(p)));
-}
-__device__ __forceinline__ void ldsm_x4_t(const void *p, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"((unsigned)__cvta_generic_to_shared(p)));
-}
-
 __global__ void __launch_bounds__(kApMaxWarps * 32) attn_prefill_kernel(const __grid_constant__ AttnPrefillArgs a) {
     constexpr int D = 128;
     extern __shared__ __align__(128) __nv_bfloat16 apsm[];  // [2 buffers][4 planes: khi, klo, vhi, vlo][64][136]

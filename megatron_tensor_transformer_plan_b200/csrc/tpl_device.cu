@@ -337,11 +337,20 @@ int run_qkv(Ctx &c, const char *packed, const tpl_kv *kv, const void *x, float *
     return gemv_launch(c, a, p->t * p->qkv_rows_s, 1, p->d.hidden, OP_QKV);
 }
 
+bool g_stg_attr[64];
+
 int run_attn(Ctx &c, const tpl_kv *kv, const float *q, const float *knew, const float *vnew, void *o) {
     tpl_plan *p = c.p;
     const int64_t keys = knew ? c.S : c.S + 1;
+    const int sms = num_sms_current();
+    if (sms <= 0) return TPL_ECUDA;
     AttnGeom g;
-    attn_geom(c.B, p->d.n_kv_heads, keys, &g);
+    // staged kernel: groups of at most 8 heads with at least two CTAs per pair
+    // in one wave (where it measured faster; with one CTA per pair the
+    // register-streamed kernel's finer splits win)
+    const bool staged = p->attn_decode_mode == 0 && p->g <= 8 && 2 * c.B * p->d.n_kv_heads <= sms;
+    if (staged) attn_geom_staged(c.B, p->d.n_kv_heads, keys, sms, &g);
+    else attn_geom(c.B, p->d.n_kv_heads, keys, &g);
     if (g.pairs > kMaxPairs) return TPL_EUNSUPPORTED;
     AttnArgs a;
     std::memset(&a, 0, sizeof(a));
@@ -366,6 +375,17 @@ int run_attn(Ctx &c, const tpl_kv *kv, const float *q, const float *knew, const 
     a.o = o;
     a.o_f32 = p->f32;
     const int grid = g.pairs * (g.nsplit / kAttnWarps);
+    if (staged) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return TPL_ECUDA;
+        if (!g_stg_attr[dev]) {
+            if (cudaFuncSetAttribute(attn_decode_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)kStgSmem) != cudaSuccess)
+                return TPL_ECUDA;
+            g_stg_attr[dev] = true;
+        }
+        return cuda_rc(launch_pdl(attn_decode_staged_kernel, grid, kAttnWarps * 32, kStgSmem, c.st, a));
+    }
     return cuda_rc(p->g <= 8 ? launch_pdl(attn_decode_kernel<true>, grid, kAttnWarps * 32, 0, c.st, a)
                               : launch_pdl(attn_decode_kernel<false>, grid, kAttnWarps * 32, 0, c.st, a));
 }

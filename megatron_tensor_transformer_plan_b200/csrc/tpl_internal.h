@@ -22,6 +22,7 @@ constexpr int kAttnWarps = 4;              // warps per attention CTA
 constexpr int kAttnTargetWarps = 1024;     // key-range splits across all (b, kv head) pairs
 constexpr int kAttnMinKeys = 128;          // keys per split at least (when there are that many)
 constexpr int kAttnMaxCtasPerPair = 64;
+constexpr int kAttnSmsBound = 256;         // upper bound on SMs when sizing workspaces
 constexpr int kTicketSlots = 4096;         // uint32 arrival counters at the workspace start
 constexpr int kTicketAttn = 0;             // [0, 1024): attention pairs
 constexpr int kTicketGemv = 1024;          // + 512 * op
@@ -46,6 +47,7 @@ struct tpl_plan {
     int gemv_mode;  // 0: mma.sync fragments (bf16); 1: fp32 FFMA; 2: bf16 FFMA; 3: tcgen05 + TMA (bf16);
                     // 4: per projection (default for bf16)
     int attn_prefill_mode;  // 0: tcgen05 (power-of-two group sizes); 1: mma.sync
+    int attn_decode_mode;   // 0: staged (g <= 8, pairs fit one wave); 1: register-streamed
 };
 
 namespace tpl {
@@ -79,6 +81,9 @@ struct AttnGeom {
 // keys: keys covered by the splits (S when the new token is added in the
 // combine, S + 1 when it is read from the cache).
 void attn_geom(int B, int nkv, int64_t keys, AttnGeom *a);
+// Splits of the staged attention kernel: one CTA per SM, floor(sms / pairs)
+// CTAs per pair (at least 64 keys per warp, at most kAttnMaxCtasPerPair).
+void attn_geom_staged(int B, int nkv, int64_t keys, int sms, AttnGeom *a);
 
 struct WsLayout {
     size_t tickets, q, o, h, act, ybuf0, ybuf1, P, knew, vnew, part_o, part_ml, gp;

@@ -111,6 +111,17 @@ void attn_geom(int B, int nkv, int64_t keys, AttnGeom *a) {
     a->kps = (int)kps;
 }
 
+void attn_geom_staged(int B, int nkv, int64_t keys, int sms, AttnGeom *a) {
+    a->pairs = B * nkv;
+    int64_t cpp = std::max(1, sms / std::max(1, a->pairs));
+    const int64_t by_keys = (keys + 4 * 64 - 1) / (4 * 64);
+    cpp = std::min(cpp, std::max<int64_t>(1, by_keys));
+    cpp = std::min<int64_t>(cpp, kAttnMaxCtasPerPair);
+    a->nsplit = (int)cpp * kAttnWarps;
+    int64_t kps = keys > 0 ? (keys + a->nsplit - 1) / a->nsplit : 16;
+    a->kps = (int)((kps + 15) / 16 * 16);
+}
+
 int ws_layout(const tpl_plan *p, int B, int64_t S, WsLayout *w) {
     if (B <= 0 || S < 0) return TPL_EINVAL;
     const tpl_dims &d = p->d;
@@ -135,7 +146,10 @@ int ws_layout(const tpl_plan *p, int B, int64_t S, WsLayout *w) {
     AttnGeom ag, ag1;  // splits over S keys (new key apart) or S + 1 keys
     attn_geom(B, d.n_kv_heads, S, &ag);
     attn_geom(B, d.n_kv_heads, S + 1, &ag1);
-    const size_t nsp = (size_t)std::max(ag.nsplit, ag1.nsplit);
+    AttnGeom sg, sg1;  // the staged kernel's splits, for the largest SM count
+    attn_geom_staged(B, d.n_kv_heads, S, kAttnSmsBound, &sg);
+    attn_geom_staged(B, d.n_kv_heads, S + 1, kAttnSmsBound, &sg1);
+    const size_t nsp = (size_t)std::max(std::max(ag.nsplit, ag1.nsplit), std::max(sg.nsplit, sg1.nsplit));
     w->part_o = take((size_t)ag.pairs * (nsp / kAttnWarps) * p->g * d.head_dim * 4);
     w->part_ml = take((size_t)ag.pairs * (nsp / kAttnWarps) * p->g * 2 * 4);
     // cross-CTA partials: the largest over the four matrix-vector steps
@@ -214,6 +228,7 @@ int tpl_plan_create(const tpl_dims *dims, int32_t t, tpl_plan **out) {
     p->esize = p->f32 ? 4 : 2;
     p->gemv_mode = p->f32 ? 1 : 4;
     p->attn_prefill_mode = 0;
+    p->attn_decode_mode = 0;
     const int64_t H = dims->hidden, es = p->esize;
     // rows padded with zeros to whole 128-column blocks
     p->ld_h = (int)align_up(H, 128);
@@ -250,6 +265,11 @@ int tpl_plan_set_option(tpl_plan *p, int32_t option, int32_t value) {
         if (value != 0 && value != 2 && value != 3 && value != 4) return TPL_EINVAL;
         if (p->f32) return value == 0 ? TPL_OK : TPL_EINVAL;
         p->gemv_mode = value;
+        return TPL_OK;
+    }
+    if (option == TPL_OPT_DECODE_ATTN) {
+        if (value != 0 && value != 1) return TPL_EINVAL;
+        p->attn_decode_mode = value;
         return TPL_OK;
     }
     if (option == TPL_OPT_PREFILL_ATTN) {

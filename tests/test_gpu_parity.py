@@ -226,3 +226,21 @@ def test_repeated_calls_are_deterministic(gpu):
     for _ in range(3):
         b = run_steps(L)["y32"]
         assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("case", [(1024, 16, 8, 2816, 8, 4, 700), (512, 8, 2, 1376, 2, 3, 37),
+                                  (256, 4, 4, 704, 4, 1, 0)])
+def test_decode_attention_kernels_agree(gpu, case):
+    """The staged attention kernel (default) and the register-streamed one
+    (TPL_OPT_DECODE_ATTN 1): both against the oracle, and close to each other."""
+    H, nq, nkv, F, t, B, S = case
+    outs = []
+    for mode in (0, 1):
+        L = make_layer(H, nq, nkv, 128, F, t, B, S, S_cap=S + 3)
+        L.plan.set_option(tpl.TPL_OPT_DECODE_ATTN, mode)
+        ref_y, tr = oracle_decode(L)
+        st = run_steps(L)
+        assert_close_rel(to_np(st["attn"]), tr["attn"], what=f"attention (mode {mode})")
+        assert_close_rel(to_np(st["y"]), ref_y, what=f"y (mode {mode})")
+        outs.append(to_np(st["attn"]))
+    assert_close_rel(outs[0], outs[1], tol=8e-3, what="staged vs register attention")

@@ -303,6 +303,38 @@ def reductions_per_pass(layers: int) -> int:
     return int(lib().orc_reductions_per_pass(layers))
 
 
+def footprint_per_gpu(dims: Dims, layers: int, t: int, batch: int, seq: int, bytes_per_elem: int = 2) -> int:
+    """Per-GPU weight + KV bytes at shard degree t (-1 if t does not divide)."""
+    f = lib().orc_footprint_per_gpu
+    f.restype = ctypes.c_longlong
+    return int(f(ctypes.byref(dims.c()), ctypes.c_longlong(layers), ctypes.c_int(t), ctypes.c_longlong(batch),
+                 ctypes.c_longlong(seq), ctypes.c_longlong(bytes_per_elem)))
+
+
+def auto_t(dims: Dims, layers: int, budget_bytes: int, headroom: float, batch: int, seq: int,
+           bytes_per_elem: int = 2, max_t: int = 8) -> int:
+    """Smallest power-of-two shard degree that fits ("Tensor Parallelism" docs, "Auto")."""
+    f = lib().orc_auto_t
+    f.restype = ctypes.c_int
+    return int(f(ctypes.byref(dims.c()), ctypes.c_longlong(layers), ctypes.c_longlong(budget_bytes),
+                 ctypes.c_double(headroom), ctypes.c_longlong(batch), ctypes.c_longlong(seq),
+                 ctypes.c_longlong(bytes_per_elem), ctypes.c_int(max_t)))
+
+
+def allreduce_time(n: int, message_bytes: float, latency_s: float, link_bytes_per_s: float) -> float:
+    f = lib().orc_allreduce_time
+    f.restype = ctypes.c_double
+    return float(f(ctypes.c_int(n), ctypes.c_double(message_bytes), ctypes.c_double(latency_s),
+                   ctypes.c_double(link_bytes_per_s)))
+
+
+def tp_time(t_single: float, n: int, layers: int, t_allreduce: float) -> float:
+    """T(N) = T_single/N + 2L * T_allreduce ("Tensor parallel scaling curves", "The scaling math")."""
+    f = lib().orc_tp_time
+    f.restype = ctypes.c_double
+    return float(f(ctypes.c_double(t_single), ctypes.c_int(n), ctypes.c_longlong(layers), ctypes.c_double(t_allreduce)))
+
+
 def silu(z: float) -> float:
     return float(lib().orc_silu(float(z)))
 

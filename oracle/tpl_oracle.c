@@ -485,3 +485,64 @@ long long orc_layer_params_per_shard(const orc_dims *dm, int32_t t) {
 /* Sum reductions per forward pass: one after each row-split projection, two
  * per layer ([TSC], "What tensor parallelism actually splits"). */
 long long orc_reductions_per_pass(long long layers) { return 2 * layers; }
+
+/* ---------------------------------------------------------------------------
+ * Planner extras.
+ *  [TPD]  "Tensor Parallelism" docs, section "Auto": the smallest power of two
+ *         that fits comfortably, preferring 1; where the target's memory cannot
+ *         be seen, the largest power of two the node's GPU count allows.
+ *  [TSC]  "Tensor parallel scaling curves", section "The scaling math":
+ *         T(N) = T_compute/N + T_memory/N + 2L * T_allreduce(N), where
+ *         T_allreduce(N) is a per-call latency plus a bandwidth part; section
+ *         "What tensor parallelism actually splits": a ring all-reduce on N
+ *         GPUs moves about 2 (N-1)/N times the message.
+ * Readings: "fits comfortably" = per-GPU weights + KV <= budget * (1 -
+ * headroom), the headroom given by the caller; t also has to divide the
+ * query heads, kv heads and ffn; at N = 1 there is no all-reduce; the two
+ * terms T_compute/N and T_memory/N are added as printed.
+ * ------------------------------------------------------------------------- */
+
+static int orc_t_divides(const orc_dims *dm, int t) {
+    return dm->n_q_heads % t == 0 && dm->n_kv_heads % t == 0 && dm->ffn % t == 0;
+}
+
+/* Per-GPU bytes of weights of `layers` layers plus the KV cache for `batch`
+ * sequences of `seq` tokens, at shard degree t (-1 if t does not divide). */
+long long orc_footprint_per_gpu(const orc_dims *dm, long long layers, int t, long long batch, long long seq,
+                                long long bytes_per_elem) {
+    if (t <= 0 || !orc_t_divides(dm, t)) return -1;
+    long long w = layers * orc_layer_params_per_shard(dm, t) * bytes_per_elem;
+    long long kv = orc_kv_bytes_per_shard(layers, dm->n_kv_heads, dm->head_dim, seq, bytes_per_elem, batch, t);
+    if (kv < 0) return -1;
+    return w + kv;
+}
+
+/* [TPD] Auto: smallest t in 1, 2, 4, 8 (t <= max_t) that fits; with
+ * budget_bytes <= 0 the largest such t.  0 when none qualifies. */
+int orc_auto_t(const orc_dims *dm, long long layers, long long budget_bytes, double headroom, long long batch,
+               long long seq, long long bytes_per_elem, int max_t) {
+    int best = 0;
+    for (int t = 1; t <= 8 && t <= max_t; t *= 2) {
+        if (!orc_t_divides(dm, t)) continue;
+        if (budget_bytes <= 0) {
+            best = t;  /* blind: keep the largest */
+            continue;
+        }
+        long long need = orc_footprint_per_gpu(dm, layers, t, batch, seq, bytes_per_elem);
+        if (need >= 0 && (double)need <= (double)budget_bytes * (1.0 - headroom)) return t;
+    }
+    return budget_bytes <= 0 ? best : 0;
+}
+
+/* [TSC] one all-reduce on n GPUs: latency + 2 (n-1)/n * message / bandwidth;
+ * none at n = 1. */
+double orc_allreduce_time(int n, double message_bytes, double latency_s, double link_bytes_per_s) {
+    if (n <= 1) return 0.0;
+    return latency_s + 2.0 * (double)(n - 1) / (double)n * message_bytes / link_bytes_per_s;
+}
+
+/* [TSC] per-token time at degree n from the single-GPU time (compute plus
+ * memory) and the per-call all-reduce time. */
+double orc_tp_time(double t_single, int n, long long layers, double t_allreduce) {
+    return t_single / (double)n + 2.0 * (double)layers * t_allreduce;
+}

@@ -463,3 +463,96 @@ def test_prefill_rows_match_the_whole_chunk():
         np.testing.assert_array_equal(trs[name], tr[name][rows])
     with pytest.raises(ValueError):
         oracle.prefill_rows(dims, w, x, [T])
+
+
+# --------------------------------------------------------------------------
+# Planner extras: Auto shard degree and the TP cost model
+# --------------------------------------------------------------------------
+
+D70 = (8192, 64, 8, 128, 28672)
+
+
+def test_scaling_math_worked_example():
+    """The pages' TP=2 example: 160 calls at 8 us, 30 ms -> 16.3 ms, 1.84x."""
+    g = golden("scaling_math.json")
+    comm = oracle.tp_time(0.0, g["n"], g["layers"], g["t_allreduce_s"])
+    assert comm == pytest.approx(2 * g["layers"] * g["t_allreduce_s"], rel=1e-15)
+    assert abs(comm - g["comm_s_approx"]) <= 0.05e-3  # 1.28 ms, printed as about 1.3
+    tn = oracle.tp_time(g["t_single_s"], g["n"], g["layers"], g["t_allreduce_s"])
+    assert abs(tn - g["t_n_s_approx"]) <= 0.05e-3
+    assert abs(g["t_single_s"] / tn - g["speedup_approx"]) <= 0.005
+    # no exchange at N = 1: T(1) is the single-GPU time
+    assert oracle.tp_time(g["t_single_s"], 1, g["layers"], 0.0) == g["t_single_s"]
+
+
+def test_allreduce_time_closed_forms():
+    g = golden("scaling_math.json")
+    m, lat, bw = g["message_bytes"], 7e-6, 770e9
+    assert oracle.allreduce_time(1, m, lat, bw) == 0.0
+    # ring: 2 (N-1)/N of the message crosses each link
+    for n in (2, 4, 8):
+        assert oracle.allreduce_time(n, m, lat, bw) == pytest.approx(lat + 2 * (n - 1) / n * m / bw, rel=1e-15)
+    assert oracle.allreduce_time(2, m, lat, bw) == pytest.approx(lat + m / bw, rel=1e-15)
+    # a 16 KB message: the latency dominates (the bandwidth part is a few ns)
+    for n in (2, 4, 8):
+        t = oracle.allreduce_time(n, m, lat, bw)
+        assert g["latency_range_s"][0] <= t <= g["latency_range_s"][1]
+        assert (t - lat) < 0.01 * lat
+    # bandwidth-bound limit: latency 0, huge message -> 2 (N-1)/N * M / bw
+    assert oracle.allreduce_time(8, 1 << 30, 0.0, bw) == pytest.approx(1.75 * (1 << 30) / bw, rel=1e-15)
+
+
+def test_footprint_per_gpu_is_weights_plus_kv():
+    d = oracle.Dims(*D70)
+    for t in (1, 2, 4, 8):
+        w = 80 * oracle.layer_params_per_shard(d, t) * 2
+        kv = oracle.kv_bytes_per_shard(80, 8, 128, 8192, 2, 16, t)
+        assert oracle.footprint_per_gpu(d, 80, t, 16, 8192) == w + kv
+    assert oracle.footprint_per_gpu(d, 80, 3, 16, 8192) == -1  # 3 divides no head count
+    assert oracle.footprint_per_gpu(d, 80, 16, 16, 8192) == -1  # more shards than kv heads
+
+
+def test_auto_t_70b_on_80gb_cards():
+    """Auto on the pages' 70B example: t = 4 is the smallest that fits."""
+    g = golden("auto_t.json")
+    d = oracle.Dims(*D70)
+    t = oracle.auto_t(d, 80, g["gpu_bytes"], g["headroom"], g["batch"], g["seq"])
+    assert t == g["expected_t"]
+    # t = 2 misses (about 90 GB per GPU), t = 4 fits (about 45 GB)
+    assert oracle.footprint_per_gpu(d, 80, 2, 16, 8192) > g["gpu_bytes"]
+    assert oracle.footprint_per_gpu(d, 80, 4, 16, 8192) < g["gpu_bytes"] * (1 - g["headroom"])
+
+
+def test_auto_t_prefers_one_and_powers_of_two():
+    d7 = oracle.Dims(4096, 32, 32, 128, 11008)
+    # a 7B layer stack fits a 180 GB card alone
+    assert oracle.auto_t(d7, 32, 180 * 10**9, 0.1, 1, 2048) == 1
+    # a budget between two footprints picks the first power of two above it
+    f = {t: oracle.footprint_per_gpu(d7, 32, t, 64, 4096) for t in (1, 2, 4, 8)}
+    assert f[1] > f[2] > f[4] > f[8]
+    for t in (1, 2, 4, 8):
+        assert oracle.auto_t(d7, 32, f[t], 0.0, 64, 4096) == t
+        assert oracle.auto_t(d7, 32, f[t] - 1, 0.0, 64, 4096) == (2 * t if t < 8 else 0)
+    # headroom: exactly at budget * (1 - h) still fits, one byte more does not
+    h = 0.25
+    b = int(f[2] / (1 - h))
+    while b * (1 - h) < f[2]:
+        b += 1
+    assert oracle.auto_t(d7, 32, b, h, 64, 4096) == 2
+    # nothing fits: 0
+    assert oracle.auto_t(d7, 32, 1000, 0.0, 64, 4096) == 0
+    # max_t caps the search
+    assert oracle.auto_t(d7, 32, f[8], 0.0, 64, 4096, max_t=4) == 0
+
+
+def test_auto_t_blind_fallback_and_divisibility():
+    d70 = oracle.Dims(*D70)
+    # memory unknown: the largest power of two the GPU count allows
+    for gpus, want in ((1, 1), (2, 2), (3, 2), (4, 4), (7, 4), (8, 8), (16, 8)):
+        assert oracle.auto_t(d70, 80, 0, 0.1, 16, 8192, max_t=gpus) == want
+    # 2 kv heads: t = 4 and 8 do not divide, so the blind answer stops at 2
+    d = oracle.Dims(1024, 16, 2, 64, 2816)
+    assert oracle.auto_t(d, 4, 0, 0.0, 1, 16, max_t=8) == 2
+    # a budget only t = 4 would meet is not met by any admissible t
+    f4 = oracle.footprint_per_gpu(oracle.Dims(1024, 16, 4, 64, 2816), 4, 4, 1, 16)
+    assert oracle.auto_t(d, 4, f4, 0.0, 1, 16) == 0

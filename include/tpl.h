@@ -62,6 +62,7 @@ extern "C" {
 #define TPL_EUNSUPPORTED 7  /* valid dimensions this build does not implement
                                (head_dim != 128, group size > 16, dims not a
                                multiple of 8)                                    */
+#define TPL_ENOFIT 8        /* tpl_auto_t: no admissible degree fits the budget  */
 
 /* ---- flags ------------------------------------------------------------- */
 #define TPL_NORM 1u          /* pre-RMSNorm before QKV and before gate/up       */
@@ -166,6 +167,49 @@ int tpl_plan_maps(const tpl_plan *plan, int32_t *q_shard, int32_t *q_local, int3
  * when t does not divide the total. */
 int64_t tpl_kv_bytes(const tpl_dims *dims, int32_t t, int64_t batch, int64_t seq,
                      int32_t bytes_per_elem);
+
+/* Per-GPU bytes at degree t of the n_layers layers' weights (each shard's
+ * slices, bytes_per_elem per parameter) plus the KV cache of tpl_kv_bytes:
+ * the footprint that the shard degree divides.  -1 on invalid input or when
+ * t does not divide n_q_heads, n_kv_heads and ffn. */
+int64_t tpl_footprint_bytes(const tpl_dims *dims, int32_t t, int64_t batch, int64_t seq,
+                            int32_t bytes_per_elem);
+
+/* The "Auto" rule of the "Tensor Parallelism" docs (section "Auto"): the
+ * smallest power of two t in {1, 2, 4, 8}, t <= max_t (the GPUs one model may
+ * use), that divides n_q_heads, n_kv_heads and ffn and whose
+ * tpl_footprint_bytes fits "comfortably": footprint <= budget_bytes *
+ * (1 - headroom), headroom in [0, 1) chosen by the caller.  With budget_bytes
+ * <= 0 (the target's memory cannot be seen) it is the largest such t, as the
+ * docs' remote-node fallback.  *t_out (host) receives t; TPL_ENOFIT (and
+ * *t_out = 0) when no admissible t fits, TPL_EINVAL on invalid input. */
+int tpl_auto_t(const tpl_dims *dims, int64_t budget_bytes, double headroom, int64_t batch, int64_t seq,
+               int32_t bytes_per_elem, int32_t max_t, int32_t *t_out);
+
+/* The per-token time model of "Tensor parallel scaling curves", section "The
+ * scaling math": T(N) = T_compute/N + T_memory/N + 2L * T_allreduce(N), with
+ * T_allreduce(N) = latency + 2 (N-1)/N * message_bytes / link_bytes_per_s
+ * (a ring all-reduce moves about 2 (N-1)/N of the message per GPU, section
+ * "What tensor parallelism actually splits") and no all-reduce at N = 1.
+ * All times in seconds. */
+typedef struct {
+    double t_compute, t_memory; /* the single-GPU terms, as given            */
+    double t_allreduce;         /* one call at N                              */
+    double t_comm;              /* 2L * t_allreduce                           */
+    double t_total;             /* T(N)                                       */
+    double speedup;             /* T(1) / T(N)                                */
+    double comm_share;          /* t_comm / t_total                           */
+} tpl_tp_estimate;
+int tpl_tp_estimate_get(double t_compute, double t_memory, int32_t n, int32_t layers, double message_bytes,
+                        double latency_s, double link_bytes_per_s, tpl_tp_estimate *out);
+
+/* The single-GPU terms of one decode step of the whole model (dims->n_layers
+ * layers, batch sequences each attending over seq cached tokens), for
+ * tpl_tp_estimate_get: t_compute = 2 * params * batch / flops_per_s (one
+ * multiply-add per weight per token), t_memory = tpl_footprint_bytes(t = 1) /
+ * hbm_bytes_per_s (every weight and the cache read once).  Host outputs. */
+int tpl_decode_times(const tpl_dims *dims, int64_t batch, int64_t seq, int32_t bytes_per_elem,
+                     double flops_per_s, double hbm_bytes_per_s, double *t_compute, double *t_memory);
 
 /* Bytes of one layer's K (or V) buffer for tpl_kv with the given capacities. */
 int64_t tpl_kv_layer_bytes(const tpl_plan *plan, int32_t batch_cap, int64_t seq_cap);

@@ -331,6 +331,74 @@ int64_t tpl_kv_bytes(const tpl_dims *d, int32_t t, int64_t batch, int64_t seq, i
     return total / t;
 }
 
+int64_t tpl_footprint_bytes(const tpl_dims *d, int32_t t, int64_t batch, int64_t seq, int32_t bytes_per_elem) {
+    if (!d || t <= 0 || d->n_layers < 0 || d->hidden <= 0 || d->head_dim <= 0 || d->n_q_heads <= 0 ||
+        d->n_kv_heads <= 0 || d->ffn <= 0)
+        return -1;
+    if (d->n_q_heads % t || d->n_kv_heads % t || d->ffn % t) return -1;
+    int64_t kv = tpl_kv_bytes(d, t, batch, seq, bytes_per_elem);
+    if (kv < 0) return -1;
+    const int64_t H = d->hidden, hd = d->head_dim;
+    const int64_t per_shard = (d->n_q_heads / t + 2 * (d->n_kv_heads / t)) * hd * H  // Wq, Wk, Wv rows
+                              + H * (d->n_q_heads / t) * hd                          // Wo columns
+                              + 3 * (int64_t)(d->ffn / t) * H;                       // Wg, Wu rows, Wd columns
+    return (int64_t)d->n_layers * per_shard * bytes_per_elem + kv;
+}
+
+int tpl_auto_t(const tpl_dims *d, int64_t budget_bytes, double headroom, int64_t batch, int64_t seq,
+               int32_t bytes_per_elem, int32_t max_t, int32_t *t_out) {
+    if (!d || !t_out || !(headroom >= 0.0 && headroom < 1.0) || batch < 0 || seq < 0 || bytes_per_elem <= 0 ||
+        max_t < 1)
+        return TPL_EINVAL;
+    *t_out = 0;
+    int32_t blind = 0;
+    for (int32_t t = 1; t <= 8 && t <= max_t; t *= 2) {
+        int64_t need = tpl_footprint_bytes(d, t, batch, seq, bytes_per_elem);
+        if (need < 0) continue;  // t does not divide the heads or ffn
+        if (budget_bytes <= 0) {
+            blind = t;
+            continue;
+        }
+        if ((double)need <= (double)budget_bytes * (1.0 - headroom)) {
+            *t_out = t;
+            return TPL_OK;
+        }
+    }
+    if (budget_bytes <= 0 && blind > 0) {
+        *t_out = blind;
+        return TPL_OK;
+    }
+    return TPL_ENOFIT;
+}
+
+int tpl_tp_estimate_get(double t_compute, double t_memory, int32_t n, int32_t layers, double message_bytes,
+                        double latency_s, double link_bytes_per_s, tpl_tp_estimate *out) {
+    if (!out || n < 1 || layers < 0 || !(t_compute >= 0) || !(t_memory >= 0) || !(message_bytes >= 0) ||
+        !(latency_s >= 0) || !(link_bytes_per_s > 0))
+        return TPL_EINVAL;
+    out->t_compute = t_compute;
+    out->t_memory = t_memory;
+    out->t_allreduce = n == 1 ? 0.0 : latency_s + 2.0 * (n - 1) / n * message_bytes / link_bytes_per_s;
+    out->t_comm = 2.0 * layers * out->t_allreduce;
+    out->t_total = t_compute / n + t_memory / n + out->t_comm;
+    const double t1 = t_compute + t_memory;
+    out->speedup = out->t_total > 0 ? t1 / out->t_total : 1.0;
+    out->comm_share = out->t_total > 0 ? out->t_comm / out->t_total : 0.0;
+    return TPL_OK;
+}
+
+int tpl_decode_times(const tpl_dims *d, int64_t batch, int64_t seq, int32_t bytes_per_elem, double flops_per_s,
+                     double hbm_bytes_per_s, double *t_compute, double *t_memory) {
+    if (!d || !t_compute || !t_memory || !(flops_per_s > 0) || !(hbm_bytes_per_s > 0)) return TPL_EINVAL;
+    const int64_t bytes = tpl_footprint_bytes(d, 1, batch, seq, bytes_per_elem);
+    const int64_t kv = tpl_kv_bytes(d, 1, batch, seq, bytes_per_elem);
+    if (bytes < 0 || kv < 0) return TPL_EINVAL;
+    const double params = (double)(bytes - kv) / bytes_per_elem;
+    *t_compute = 2.0 * params * (double)batch / flops_per_s;
+    *t_memory = (double)bytes / hbm_bytes_per_s;
+    return TPL_OK;
+}
+
 int64_t tpl_kv_layer_bytes(const tpl_plan *p, int32_t batch_cap, int64_t seq_cap) {
     if (!p || batch_cap < 0 || seq_cap < 0) return -1;
     return (int64_t)batch_cap * p->d.n_kv_heads * seq_cap * p->d.head_dim * 2;
@@ -383,6 +451,7 @@ const char *tpl_status_string(int s) {
         case TPL_ECUDA: return "CUDA error";
         case TPL_EDEVICE: return "device-side inconsistency recorded";
         case TPL_EUNSUPPORTED: return "unsupported dimensions";
+        case TPL_ENOFIT: return "no admissible shard degree fits the memory budget";
         default: return "unknown status";
     }
 }

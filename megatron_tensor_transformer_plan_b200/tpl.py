@@ -20,7 +20,8 @@ if not os.path.exists(LIB_PATH):
     raise ImportError(f"libtpl.so not built at {LIB_PATH}; run megatron_tensor_transformer_plan_b200/build.py")
 _lib = ctypes.CDLL(LIB_PATH)
 
-TPL_OK, TPL_EINVAL, TPL_EINDIVISIBLE, TPL_EWORKSPACE, TPL_ENOMEM, TPL_ECUDA, TPL_EDEVICE, TPL_EUNSUPPORTED = range(8)
+(TPL_OK, TPL_EINVAL, TPL_EINDIVISIBLE, TPL_EWORKSPACE, TPL_ENOMEM, TPL_ECUDA, TPL_EDEVICE, TPL_EUNSUPPORTED,
+ TPL_ENOFIT) = range(9)
 TPL_NORM, TPL_RESIDUAL, TPL_FP32_WEIGHTS = 1, 2, 4
 TPL_REDUCE_FUSED, TPL_REDUCE_SEPARATE = 0, 1
 TPL_OPT_GEMV_MODE = 1
@@ -35,6 +36,11 @@ P = ctypes.POINTER
 class tpl_dims(ctypes.Structure):
     _fields_ = [("hidden", c_int32), ("n_q_heads", c_int32), ("n_kv_heads", c_int32), ("head_dim", c_int32),
                 ("ffn", c_int32), ("n_layers", c_int32), ("rms_eps", ctypes.c_float), ("flags", c_uint32)]
+
+
+class tpl_tp_estimate(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_double) for n in ("t_compute", "t_memory", "t_allreduce", "t_comm", "t_total",
+                                                "speedup", "comm_share")]
 
 
 class tpl_plan_info(ctypes.Structure):
@@ -69,6 +75,12 @@ _sig("tpl_plan_info_get", ctypes.c_int, _plan_p, P(tpl_plan_info))
 _sig("tpl_plan_maps", ctypes.c_int, _plan_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p)
 _sig("tpl_plan_set_option", ctypes.c_int, _plan_p, c_int32, c_int32)
 _sig("tpl_kv_bytes", c_int64, P(tpl_dims), c_int32, c_int64, c_int64, c_int32)
+_sig("tpl_footprint_bytes", c_int64, P(tpl_dims), c_int32, c_int64, c_int64, c_int32)
+_sig("tpl_auto_t", ctypes.c_int, P(tpl_dims), c_int64, ctypes.c_double, c_int64, c_int64, c_int32, c_int32, P(c_int32))
+_sig("tpl_tp_estimate_get", ctypes.c_int, ctypes.c_double, ctypes.c_double, c_int32, c_int32, ctypes.c_double,
+     ctypes.c_double, ctypes.c_double, P(tpl_tp_estimate))
+_sig("tpl_decode_times", ctypes.c_int, P(tpl_dims), c_int64, c_int64, c_int32, ctypes.c_double, ctypes.c_double,
+     P(ctypes.c_double), P(ctypes.c_double))
 _sig("tpl_kv_layer_bytes", c_int64, _plan_p, c_int32, c_int64)
 _sig("tpl_workspace_size", ctypes.c_int, _plan_p, c_int32, c_int64, P(c_size_t))
 _sig("tpl_workspace_init", ctypes.c_int, _plan_p, c_void_p, c_size_t, c_void_p)
@@ -118,6 +130,38 @@ def check(code: int, where: str = "") -> None:
 def make_dims(hidden, n_q_heads, n_kv_heads, head_dim, ffn, n_layers=1, rms_eps=1e-5,
               flags=TPL_NORM | TPL_RESIDUAL) -> tpl_dims:
     return tpl_dims(hidden, n_q_heads, n_kv_heads, head_dim, ffn, n_layers, rms_eps, flags)
+
+
+def footprint_bytes(dims: tpl_dims, t: int, batch: int, seq: int, bytes_per_elem: int = 2) -> int:
+    """Per-GPU weight + KV bytes at degree t (-1 when t does not divide)."""
+    return int(tpl_footprint_bytes(ctypes.byref(dims), t, batch, seq, bytes_per_elem))
+
+
+def auto_t(dims: tpl_dims, budget_bytes: int, headroom: float, batch: int, seq: int, bytes_per_elem: int = 2,
+           max_t: int = 8) -> int:
+    """The smallest power-of-two degree that fits the budget (0 when none does)."""
+    out = c_int32(0)
+    rc = tpl_auto_t(ctypes.byref(dims), budget_bytes, headroom, batch, seq, bytes_per_elem, max_t, ctypes.byref(out))
+    if rc == TPL_ENOFIT:
+        return 0
+    check(rc, "tpl_auto_t")
+    return int(out.value)
+
+
+def tp_estimate(t_compute: float, t_memory: float, n: int, layers: int, message_bytes: float, latency_s: float,
+                link_bytes_per_s: float) -> tpl_tp_estimate:
+    out = tpl_tp_estimate()
+    check(tpl_tp_estimate_get(t_compute, t_memory, n, layers, message_bytes, latency_s, link_bytes_per_s,
+                              ctypes.byref(out)), "tpl_tp_estimate_get")
+    return out
+
+
+def decode_times(dims: tpl_dims, batch: int, seq: int, bytes_per_elem: int, flops_per_s: float,
+                 hbm_bytes_per_s: float):
+    tc, tm = ctypes.c_double(), ctypes.c_double()
+    check(tpl_decode_times(ctypes.byref(dims), batch, seq, bytes_per_elem, flops_per_s, hbm_bytes_per_s,
+                           ctypes.byref(tc), ctypes.byref(tm)), "tpl_decode_times")
+    return tc.value, tm.value
 
 
 # --------------------------------------------------------------------------

@@ -35,6 +35,7 @@ _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 
 NORM = 1
 RESIDUAL = 2
+ROPE = 8
 
 
 def build(force: bool = False) -> str:
@@ -50,7 +51,8 @@ def build(force: bool = False) -> str:
 class _Dims(ctypes.Structure):
     _fields_ = [("hidden", ctypes.c_int32), ("n_q_heads", ctypes.c_int32),
                 ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
-                ("ffn", ctypes.c_int32), ("eps", ctypes.c_double), ("flags", ctypes.c_uint32)]
+                ("ffn", ctypes.c_int32), ("eps", ctypes.c_double), ("flags", ctypes.c_uint32),
+                ("rope_base", ctypes.c_double)]
 
 
 class _Weights(ctypes.Structure):
@@ -75,6 +77,7 @@ def lib():
         L = _lib
         L.orc_decode_layer.restype = ctypes.c_int
         L.orc_prefill_layer.restype = ctypes.c_int
+        L.orc_prefill_chunk.restype = ctypes.c_int
         L.orc_mlp_sharded.restype = ctypes.c_int
         L.orc_attn_sharded.restype = ctypes.c_int
         L.orc_plan_maps.restype = ctypes.c_int
@@ -107,10 +110,11 @@ class Dims:
     ffn: int
     eps: float = 1e-5
     flags: int = NORM | RESIDUAL
+    rope_base: float = 500000.0
 
     def c(self) -> _Dims:
         return _Dims(self.hidden, self.n_q_heads, self.n_kv_heads, self.head_dim, self.ffn,
-                     float(self.eps), int(self.flags))
+                     float(self.eps), int(self.flags), float(self.rope_base))
 
 
 def _p(a):
@@ -203,6 +207,62 @@ def prefill_layer(dims: Dims, w: dict, x: np.ndarray, trace: bool = False):
                                  _p(y), _p(k), _p(v), ctypes.byref(tr) if tr is not None else None)
     if rc != 0:
         raise ValueError(f"orc_prefill_layer failed ({rc})")
+    return (y, k, v, tr_arrays) if trace else (y, k, v)
+
+
+def rope(v: np.ndarray, pos: int, base: float) -> np.ndarray:
+    """Rotary position embedding of head vectors v[..., d] at one position."""
+    out = np.ascontiguousarray(v, dtype=np.float64).copy()
+    d = out.shape[-1]
+    flat = out.reshape(-1, d)
+    f = lib().orc_rope
+    f.restype = None
+    for r in range(flat.shape[0]):
+        row = np.ascontiguousarray(flat[r])
+        f(_p(row), ctypes.c_long(d), ctypes.c_long(pos), ctypes.c_double(base))
+        flat[r] = row
+    return out
+
+
+def prefill_chunk(dims: Dims, w: dict, x: np.ndarray, P0: int, kc=None, vc=None, rows=None, trace: bool = False):
+    """The prefill layer over a chunk of one sequence whose cache holds P0
+    tokens: token i at position P0 + i attends the cached keys and the chunk's
+    keys 0..i.  kc/vc uint16 (bf16 bits) [n_kv][S_cap][d] (or [1][n_kv][S_cap][d])
+    holding the P0 cached tokens.  rows: the token rows whose outputs are
+    wanted (default all).  Returns y [len(rows)][H], k, v [max(rows)+1][n_kv*d]
+    (and a trace dict with q, attn, h, act at the listed rows)."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    T, H = x.shape
+    r = np.arange(T, dtype=np.int64) if rows is None else np.asarray(rows, dtype=np.int64)
+    r = np.ascontiguousarray(r)
+    n = len(r)
+    R = int(r.max()) + 1 if n else 0
+    nkd = dims.n_kv_heads * dims.head_dim
+    S_cap = 0
+    if kc is not None:
+        kc = np.ascontiguousarray(kc, dtype=np.uint16)
+        vc = np.ascontiguousarray(vc, dtype=np.uint16)
+        if kc.ndim == 4:
+            kc, vc = kc[0], vc[0]
+        S_cap = kc.shape[1]
+    y = np.empty((n, H))
+    k = np.empty((R, nkd))
+    v = np.empty((R, nkd))
+    ws, keep = _weights_struct(w)
+    tr = None
+    tr_arrays = {}
+    if trace:
+        nqd = dims.n_q_heads * dims.head_dim
+        tr_arrays = {"q": np.empty((n, nqd)), "attn": np.empty((n, nqd)), "h": np.empty((n, H)),
+                     "act": np.empty((n, dims.ffn))}
+        tr = _Trace(_p(tr_arrays["q"]), None, None, _p(tr_arrays["attn"]), _p(tr_arrays["h"]),
+                    _p(tr_arrays["act"]))
+    rc = lib().orc_prefill_chunk(ctypes.byref(dims.c()), ctypes.byref(ws), ctypes.c_long(T), _p(x),
+                                 ctypes.c_long(P0), _p(kc), _p(vc), ctypes.c_long(S_cap), ctypes.c_long(n),
+                                 r.ctypes.data_as(ctypes.POINTER(ctypes.c_long)), _p(y), _p(k), _p(v),
+                                 ctypes.byref(tr) if tr is not None else None)
+    if rc != 0:
+        raise ValueError(f"orc_prefill_chunk failed ({rc})")
     return (y, k, v, tr_arrays) if trace else (y, k, v)
 
 

@@ -36,7 +36,14 @@
  *  - decode: the cache holds S tokens, the new token's k/v is position S,
  *    attention spans S+1 keys; the new k/v enter the softmax unrounded;
  *  - weights use the nn.Linear orientation W[out][in]; "column split" in the
- *    pages' x@W notation therefore splits `out`, "row split" splits `in`.
+ *    pages' x@W notation therefore splits `out`, "row split" splits `in`;
+ *  - rotary position embedding (ORC_ROPE, off unless flagged): not on the
+ *    pages; the textbook rotation of RoFormer (Su et al., "RoFormer:
+ *    Enhanced Transformer with Rotary Position Embedding", 2021) in the
+ *    pairing the Llama family uses, element e with element e + d/2;
+ *  - a prefill chunk may start at position P0 of a cache already holding P0
+ *    tokens ("chunked prefill"): its token i sits at position P0 + i and
+ *    attends the P0 cached keys (bf16) and the chunk's keys 0..i (unrounded).
  *
  * Data formats: weights are either raw bf16 bit patterns (uint16) or fp32,
  * widened exactly to double.  The KV cache is raw bf16 in the unsharded
@@ -52,11 +59,13 @@
 
 #define ORC_NORM 1u
 #define ORC_RESIDUAL 2u
+#define ORC_ROPE 8u
 
 typedef struct {
     int32_t hidden, n_q_heads, n_kv_heads, head_dim, ffn;
     double eps;
     uint32_t flags;
+    double rope_base; /* the base of the rotary frequencies (ORC_ROPE) */
 } orc_dims;
 
 /* Unsharded layer weights in nn.Linear orientation.  wtype: 0 = bf16 bits,
@@ -121,6 +130,20 @@ void orc_rmsnorm(const double *x, const float *gamma, long n, double eps, double
 
 double orc_silu(double z) { return z / (1.0 + exp(-z)); }
 
+/* Rotary position embedding of one head vector v[d] at position pos: for
+ * e < d/2 the pair (v[e], v[e + d/2]) is turned by the angle
+ * pos * base^(-2e/d) (RoFormer's frequencies theta_e = base^(-2e/d)). */
+void orc_rope(double *v, long d, long pos, double base) {
+    const long half = d / 2;
+    for (long e = 0; e < half; ++e) {
+        const double ang = (double)pos * pow(base, -2.0 * (double)e / (double)d);
+        const double c = cos(ang), s = sin(ang);
+        const double a = v[e], b = v[e + half];
+        v[e] = a * c - b * s;
+        v[e + half] = b * c + a * s;
+    }
+}
+
 /* Softmax-weighted sum for one query head over nkeys keys.
  * keys(j) / vals(j) are fetched through the callbacks' arrays: the first
  * n_cached keys come from a bf16 cache row block, the optional extra key is
@@ -170,6 +193,7 @@ typedef struct {
  * y [B][H] fp64.  Definition (per sequence):
  *   a   = RMSNorm(x; gamma_attn)                      (if ORC_NORM, else x)
  *   q,k,v = Wq a, Wk a, Wv a                          [TSC]
+ *   q_h, k_j rotated to position S                    (if ORC_ROPE)
  *   o_h = sum_{j<=S} softmax_j(q_h . K_j / sqrt(d)) V_j, kv head floor(h/g),
  *         K_S = k, V_S = v (the new token)            [TSC] local attention
  *   h   = x + Wo o                                    (residual if flagged)
@@ -203,6 +227,10 @@ int orc_decode_layer(const orc_dims *dm, const orc_weights *w, long B, const dou
         linear_block(w->wq, w->wtype, (size_t)H, 0, nq * d, 0, H, a, q);
         linear_block(w->wk, w->wtype, (size_t)H, 0, nkv * d, 0, H, a, k);
         linear_block(w->wv, w->wtype, (size_t)H, 0, nkv * d, 0, H, a, v);
+        if (dm->flags & ORC_ROPE) {
+            for (long hq = 0; hq < nq; ++hq) orc_rope(q + hq * d, d, S, dm->rope_base);
+            for (long j = 0; j < nkv; ++j) orc_rope(k + j * d, d, S, dm->rope_base);
+        }
         long h;
 #pragma omp parallel for schedule(static)
         for (h = 0; h < nq; ++h) {
@@ -236,24 +264,29 @@ int orc_decode_layer(const orc_dims *dm, const orc_weights *w, long B, const dou
     return 0;
 }
 
-/* One unsharded prefill layer over a chunk of T tokens starting at position
- * 0 of empty caches: token i attends keys 0..i of the chunk (causal).  The
+/* One unsharded prefill layer over a chunk of T tokens of one sequence
+ * whose cache already holds P0 tokens: token i sits at position P0 + i and
+ * attends the P0 cached keys and the chunk's keys 0..i (causal).  The
  * layer's outputs are produced for the `nrows` token rows listed in `rows`
- * (each in [0, T)); the keys and values of every token up to the largest
- * listed row are computed, since those rows attend to them.
- *   x [T][H]; y [nrows][H] (row r of y is token rows[r]);
- *   k_out/v_out [R][n_kv*d], R = max(rows) + 1: the new keys/values, which
- *   are what cache slots 0..R-1 hold afterwards;
+ * (each in [0, T)); the keys and values of every chunk token up to the
+ * largest listed row are computed, since those rows attend to them.
+ *   x [T][H]; kc/vc raw bf16 [n_kv][S_cap][d] with P0 cached tokens (may be
+ *   NULL when P0 = 0); y [nrows][H] (row r of y is token rows[r]);
+ *   k_out/v_out [R][n_kv*d], R = max(rows) + 1: the new keys (rotated when
+ *   ORC_ROPE) and values, which are what cache slots P0..P0+R-1 hold
+ *   afterwards (before rounding);
  *   trace (optional): q/attn [nrows][nq*d], h [nrows][H], act [nrows][F].
- * Per token the steps are those of orc_decode_layer with the chunk's own
- * keys 0..i in place of the cache ("Tensor parallel scaling curves",
+ * Per token the steps are those of orc_decode_layer with the cache's keys
+ * followed by the chunk's own keys 0..i ("Tensor parallel scaling curves",
  * "Prefill vs decode: different curves"). */
-int orc_prefill_rows(const orc_dims *dm, const orc_weights *w, long T, const double *x, long nrows,
-                     const long *rows, double *y, double *k_out, double *v_out, const orc_trace *tr) {
+int orc_prefill_chunk(const orc_dims *dm, const orc_weights *w, long T, const double *x, long P0,
+                      const uint16_t *kc, const uint16_t *vc, long S_cap, long nrows, const long *rows,
+                      double *y, double *k_out, double *v_out, const orc_trace *tr) {
     const long H = dm->hidden, nq = dm->n_q_heads, nkv = dm->n_kv_heads, d = dm->head_dim,
                F = dm->ffn;
     if (H <= 0 || nq <= 0 || nkv <= 0 || d <= 0 || F <= 0 || nq % nkv != 0 || T < 0 || nrows < 0)
         return 1;
+    if (P0 < 0 || (P0 > 0 && (!kc || !vc || S_cap < P0))) return 1;
     long R = 0;
     for (long r = 0; r < nrows; ++r) {
         if (rows[r] < 0 || rows[r] >= T) return 1;
@@ -279,6 +312,8 @@ int orc_prefill_rows(const orc_dims *dm, const orc_weights *w, long T, const dou
         else memcpy(a, xp, sizeof(double) * (size_t)H);
         linear_block(w->wk, w->wtype, (size_t)H, 0, nkv * d, 0, H, a, K + (size_t)p * nkv * d);
         linear_block(w->wv, w->wtype, (size_t)H, 0, nkv * d, 0, H, a, V + (size_t)p * nkv * d);
+        if (dm->flags & ORC_ROPE)
+            for (long j = 0; j < nkv; ++j) orc_rope(K + (size_t)p * nkv * d + (size_t)j * d, d, P0 + p, dm->rope_base);
     }
     for (long r = 0; r < nrows; ++r) {
         const long i = rows[r];
@@ -286,31 +321,45 @@ int orc_prefill_rows(const orc_dims *dm, const orc_weights *w, long T, const dou
         if (dm->flags & ORC_NORM) orc_rmsnorm(xi, w->gamma_attn, H, dm->eps, a);
         else memcpy(a, xi, sizeof(double) * (size_t)H);
         linear_block(w->wq, w->wtype, (size_t)H, 0, nq * d, 0, H, a, q);
+        if (dm->flags & ORC_ROPE)
+            for (long hq = 0; hq < nq; ++hq) orc_rope(q + (size_t)hq * d, d, P0 + i, dm->rope_base);
         long h;
 #pragma omp parallel for schedule(static)
         for (h = 0; h < nq; ++h) {
             const long j = h / g;
             const double *qh = q + (size_t)h * d;
             double *out = o + (size_t)h * d;
-            double *logit = malloc(sizeof(double) * (size_t)(i + 1));
+            /* keys 0..P0-1 from the cache, then the chunk's keys 0..i */
+            const long nk = P0 + i + 1;
+            double *logit = malloc(sizeof(double) * (size_t)nk);
             double mx = -INFINITY;
-            for (long p = 0; p <= i; ++p) {
-                const double *kp = K + (size_t)p * nkv * d + (size_t)j * d;
+            for (long p = 0; p < nk; ++p) {
                 double s = 0.0;
-                for (long e = 0; e < d; ++e) s += qh[e] * kp[e];
+                if (p < P0) {
+                    const uint16_t *kp = kc + ((size_t)j * S_cap + (size_t)p) * d;
+                    for (long e = 0; e < d; ++e) s += qh[e] * orc_bf16_to_double(kp[e]);
+                } else {
+                    const double *kp = K + (size_t)(p - P0) * nkv * d + (size_t)j * d;
+                    for (long e = 0; e < d; ++e) s += qh[e] * kp[e];
+                }
                 logit[p] = s * scale;
                 if (logit[p] > mx) mx = logit[p];
             }
             double den = 0.0;
-            for (long p = 0; p <= i; ++p) {
+            for (long p = 0; p < nk; ++p) {
                 logit[p] = exp(logit[p] - mx);
                 den += logit[p];
             }
             for (long e = 0; e < d; ++e) out[e] = 0.0;
-            for (long p = 0; p <= i; ++p) {
-                const double *vp = V + (size_t)p * nkv * d + (size_t)j * d;
+            for (long p = 0; p < nk; ++p) {
                 const double pr = logit[p] / den;
-                for (long e = 0; e < d; ++e) out[e] += pr * vp[e];
+                if (p < P0) {
+                    const uint16_t *vp = vc + ((size_t)j * S_cap + (size_t)p) * d;
+                    for (long e = 0; e < d; ++e) out[e] += pr * orc_bf16_to_double(vp[e]);
+                } else {
+                    const double *vp = V + (size_t)(p - P0) * nkv * d + (size_t)j * d;
+                    for (long e = 0; e < d; ++e) out[e] += pr * vp[e];
+                }
             }
             free(logit);
         }
@@ -337,6 +386,12 @@ int orc_prefill_rows(const orc_dims *dm, const orc_weights *w, long T, const dou
     free(a); free(q); free(K); free(V); free(o); free(hh); free(m);
     free(gg); free(uu); free(act); free(dn);
     return 0;
+}
+
+/* A chunk at position 0 of an empty cache, outputs at the listed rows. */
+int orc_prefill_rows(const orc_dims *dm, const orc_weights *w, long T, const double *x, long nrows,
+                     const long *rows, double *y, double *k_out, double *v_out, const orc_trace *tr) {
+    return orc_prefill_chunk(dm, w, T, x, 0, NULL, NULL, 0, nrows, rows, y, k_out, v_out, tr);
 }
 
 /* The whole chunk: every row 0..T-1.  x [T][H]; y [T][H]; k_out/v_out

@@ -23,7 +23,21 @@ def _softmax(z):
     return e / e.sum(axis=-1, keepdims=True)
 
 
-def decode_layer(H, nq, nkv, d, F, eps, norm, residual, w, x, kc, vc, S):
+def rope(v, pos, base):
+    """Rotary embedding written as complex multiplication: the pair
+    (v[e], v[e + d/2]) is the complex number v[e] + i v[e + d/2], multiplied
+    by exp(i * pos * base^(-2e/d)).  v [..., d]; pos broadcasts against
+    v[..., 0]."""
+    v = np.asarray(v, np.float64)
+    d = v.shape[-1]
+    half = d // 2
+    z = v[..., :half] + 1j * v[..., half:]
+    theta = base ** (-2.0 * np.arange(half) / d)
+    z = z * np.exp(1j * np.asarray(pos, np.float64)[..., None] * theta)
+    return np.concatenate([z.real, z.imag], axis=-1)
+
+
+def decode_layer(H, nq, nkv, d, F, eps, norm, residual, w, x, kc, vc, S, rope_base=None):
     W = {k: _widen(w[k]) for k in ("wq", "wk", "wv", "wo", "wg", "wu", "wd")}
     x = np.asarray(x, np.float64)
     B = x.shape[0]
@@ -32,6 +46,9 @@ def decode_layer(H, nq, nkv, d, F, eps, norm, residual, w, x, kc, vc, S):
     q = a @ W["wq"].T
     k = a @ W["wk"].T
     v = a @ W["wv"].T
+    if rope_base is not None:
+        q = rope(q.reshape(B, nq, d), S, rope_base).reshape(B, nq * d)
+        k = rope(k.reshape(B, nkv, d), S, rope_base).reshape(B, nkv * d)
     Kc = _widen(kc)[:, :, :S, :]
     Vc = _widen(vc)[:, :, :S, :]
     o = np.zeros((B, nq * d))
@@ -55,7 +72,9 @@ def decode_layer(H, nq, nkv, d, F, eps, norm, residual, w, x, kc, vc, S):
     return y, {"q": q, "k_new": k, "v_new": v, "attn": o, "h": hh, "act": act}
 
 
-def prefill_layer(H, nq, nkv, d, F, eps, norm, residual, w, x):
+def prefill_layer(H, nq, nkv, d, F, eps, norm, residual, w, x, P0=0, kc=None, vc=None, rope_base=None):
+    """A chunk of T tokens at positions P0..P0+T-1; kc/vc bf16 bits
+    [n_kv][S_cap][d] hold the P0 earlier tokens' keys and values."""
     W = {k: _widen(w[k]) for k in ("wq", "wk", "wv", "wo", "wg", "wu", "wd")}
     x = np.asarray(x, np.float64)
     T = x.shape[0]
@@ -64,13 +83,23 @@ def prefill_layer(H, nq, nkv, d, F, eps, norm, residual, w, x):
     q = a @ W["wq"].T
     k = a @ W["wk"].T
     v = a @ W["wv"].T
+    if rope_base is not None:
+        pos = P0 + np.arange(T)[:, None]
+        q = rope(q.reshape(T, nq, d), pos, rope_base).reshape(T, nq * d)
+        k = rope(k.reshape(T, nkv, d), pos, rope_base).reshape(T, nkv * d)
     o = np.zeros((T, nq * d))
-    mask = np.tril(np.ones((T, T), bool))
+    # key p (0..P0+T-1) is visible to token i when p <= P0 + i
+    mask = np.arange(P0 + T)[None, :] <= (P0 + np.arange(T))[:, None]
     for h in range(nq):
         j = h // g
-        s = q[:, h * d:(h + 1) * d] @ k[:, j * d:(j + 1) * d].T / np.sqrt(d)
+        keys = k[:, j * d:(j + 1) * d]
+        vals = v[:, j * d:(j + 1) * d]
+        if P0:
+            keys = np.concatenate([_widen(kc)[j, :P0], keys], axis=0)
+            vals = np.concatenate([_widen(vc)[j, :P0], vals], axis=0)
+        s = q[:, h * d:(h + 1) * d] @ keys.T / np.sqrt(d)
         s = np.where(mask, s, -np.inf)
-        o[:, h * d:(h + 1) * d] = _softmax(s) @ v[:, j * d:(j + 1) * d]
+        o[:, h * d:(h + 1) * d] = _softmax(s) @ vals
     hh = o @ W["wo"].T
     if residual:
         hh = x + hh

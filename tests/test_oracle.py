@@ -466,6 +466,137 @@ def test_prefill_rows_match_the_whole_chunk():
 
 
 # --------------------------------------------------------------------------
+# Rotary position embedding and chunked prefill into an existing cache
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("d,base", [(8, 10000.0), (128, 500000.0), (128, 10000.0)])
+def test_rope_matches_complex_rotation(d, base):
+    r = rng(60)
+    v = r.standard_normal((5, d))
+    for pos in (0, 1, 7, 4096, 8191, 131071):
+        got = oracle.rope(v, pos, base)
+        want = np_reference.rope(v, pos, base)
+        # the angle pos * theta carries a rounding of about pos * 1e-16 rad
+        np.testing.assert_allclose(got, want, rtol=0, atol=(1e-14 + 1e-15 * pos) * np.abs(v).max())
+
+
+def test_rope_invariants():
+    r = rng(61)
+    d, base = 128, 500000.0
+    q, k = r.standard_normal(d), r.standard_normal(d)
+    # position 0 is the identity, exactly
+    np.testing.assert_array_equal(oracle.rope(q, 0, base), q)
+    # each pair (e, e + d/2) keeps its length
+    for pos in (1, 33, 8000):
+        rq = oracle.rope(q, pos, base)
+        np.testing.assert_allclose(rq[:64] ** 2 + rq[64:] ** 2, q[:64] ** 2 + q[64:] ** 2, rtol=1e-12)
+    # the logit depends on the distance only: <R(m) q, R(n) k> = <R(m+c) q, R(n+c) k>
+    for m, n, c in ((5, 2, 100), (0, 9, 4000), (8191, 0, 7)):
+        a = oracle.rope(q, m, base) @ oracle.rope(k, n, base)
+        b = oracle.rope(q, m + c, base) @ oracle.rope(k, n + c, base)
+        assert abs(a - b) <= 1e-10 * np.abs(q).sum() * np.abs(k).max()
+    # pair 0 turns by exactly pos radians (theta_0 = 1); the last pair slowest
+    e0 = np.zeros(d)
+    e0[0] = 1.0
+    rq = oracle.rope(e0, 3, base)
+    assert rq[0] == pytest.approx(np.cos(3.0), abs=1e-15) and rq[64] == pytest.approx(np.sin(3.0), abs=1e-15)
+    e1 = np.zeros(d)
+    e1[63] = 1.0
+    rq = oracle.rope(e1, 3, base)
+    ang = 3.0 * base ** (-126.0 / 128.0)
+    assert rq[63] == pytest.approx(np.cos(ang), abs=1e-15) and rq[127] == pytest.approx(np.sin(ang), abs=1e-15)
+
+
+@pytest.mark.parametrize("rope", [False, True])
+def test_decode_with_rope_matches_numpy(rope):
+    r = rng(62)
+    H, nq, nkv, d, F, B, S = 64, 8, 2, 16, 80, 2, 11
+    w = small_layer(r, H, nq, nkv, d, F, std=0.1)
+    flags = oracle.NORM | oracle.RESIDUAL | (oracle.ROPE if rope else 0)
+    dims = oracle.Dims(H, nq, nkv, d, F, flags=flags, rope_base=10000.0)
+    x = r.standard_normal((B, H))
+    kc = rand_bf16_bits(r, (B, nkv, S + 2, d), 1.0)
+    vc = rand_bf16_bits(r, (B, nkv, S + 2, d), 1.0)
+    y, tr = oracle.decode_layer(dims, w, x, kc, vc, S, trace=True)
+    y_np, tr_np = np_reference.decode_layer(H, nq, nkv, d, F, dims.eps, True, True, w, x, kc, vc, S,
+                                            rope_base=10000.0 if rope else None)
+    np.testing.assert_allclose(y, y_np, rtol=1e-11, atol=1e-11 * np.abs(y_np).max())
+    np.testing.assert_allclose(tr["q"], tr_np["q"], rtol=1e-11, atol=1e-11 * np.abs(tr_np["q"]).max())
+    np.testing.assert_allclose(tr["k_new"], tr_np["k_new"], rtol=1e-11,
+                               atol=1e-11 * np.abs(tr_np["k_new"]).max())
+
+
+@pytest.mark.parametrize("rope,P0", [(False, 0), (False, 9), (True, 0), (True, 9), (True, 300)])
+def test_prefill_chunk_matches_numpy(rope, P0):
+    r = rng(63)
+    H, nq, nkv, d, F, T = 64, 8, 2, 16, 80, 7
+    w = small_layer(r, H, nq, nkv, d, F, std=0.1)
+    flags = oracle.NORM | oracle.RESIDUAL | (oracle.ROPE if rope else 0)
+    dims = oracle.Dims(H, nq, nkv, d, F, flags=flags, rope_base=500000.0)
+    x = r.standard_normal((T, H))
+    kc = rand_bf16_bits(r, (nkv, P0 + T + 3, d), 1.0)
+    vc = rand_bf16_bits(r, (nkv, P0 + T + 3, d), 1.0)
+    y, k, v = oracle.prefill_chunk(dims, w, x, P0, kc, vc)
+    y_np, k_np, v_np = np_reference.prefill_layer(H, nq, nkv, d, F, dims.eps, True, True, w, x, P0, kc, vc,
+                                                  rope_base=500000.0 if rope else None)
+    np.testing.assert_allclose(y, y_np, rtol=1e-11, atol=1e-11 * np.abs(y_np).max())
+    np.testing.assert_allclose(k, k_np, rtol=1e-11, atol=1e-11 * np.abs(k_np).max())
+    np.testing.assert_allclose(v, v_np, rtol=1e-11, atol=1e-11 * np.abs(v_np).max())
+
+
+@pytest.mark.parametrize("rope", [False, True])
+def test_one_token_chunk_is_a_decode_step(rope):
+    """A chunk of one token at position S over a cache of S tokens is the
+    decode step at S (the same definition reached by two routes)."""
+    r = rng(64)
+    H, nq, nkv, d, F, S = 32, 4, 2, 8, 24, 13
+    w = small_layer(r, H, nq, nkv, d, F)
+    flags = oracle.NORM | oracle.RESIDUAL | (oracle.ROPE if rope else 0)
+    dims = oracle.Dims(H, nq, nkv, d, F, flags=flags, rope_base=10000.0)
+    x = r.standard_normal((1, H))
+    kc = rand_bf16_bits(r, (1, nkv, S + 1, d), 1.0)
+    vc = rand_bf16_bits(r, (1, nkv, S + 1, d), 1.0)
+    yd, trd = oracle.decode_layer(dims, w, x, kc, vc, S, trace=True)
+    yc, kk, vv, trc = oracle.prefill_chunk(dims, w, x, S, kc, vc, trace=True)
+    np.testing.assert_allclose(yc, yd, rtol=1e-13, atol=1e-13 * np.abs(yd).max())
+    np.testing.assert_allclose(kk, trd["k_new"], rtol=1e-14, atol=0)
+    np.testing.assert_allclose(trc["attn"], trd["attn"], rtol=1e-13, atol=1e-13 * np.abs(trd["attn"]).max())
+
+
+def test_chunks_compose_to_the_whole_sequence():
+    """With keys and values exact in bf16 (small integers), prefilling a
+    sequence in two chunks (the second attending to the first's cached keys)
+    gives the single chunk's outputs."""
+    r = rng(65)
+    H, nq, nkv, d, F, T1, T2 = 16, 4, 2, 8, 12, 5, 4
+    w = {k: f32(r.integers(-2, 3, s)) for k, s in
+         {"wq": (nq * d, H), "wk": (nkv * d, H), "wv": (nkv * d, H), "wo": (H, nq * d),
+          "wg": (F, H), "wu": (F, H), "wd": (H, F)}.items()}
+    w["wq"] = f32(w["wq"] * 0.125)
+    dims = oracle.Dims(H, nq, nkv, d, F, flags=oracle.RESIDUAL)
+    x = r.integers(-2, 3, (T1 + T2, H)).astype(np.float64)
+    y, k, v = oracle.prefill_layer(dims, w, x)
+    y1, k1, v1 = oracle.prefill_chunk(dims, w, x[:T1], 0)
+    kc = np.zeros((nkv, T1 + T2, d), np.float32)
+    vc = np.zeros((nkv, T1 + T2, d), np.float32)
+    for j in range(nkv):
+        kc[j, :T1] = k1[:, j * d:(j + 1) * d]
+        vc[j, :T1] = v1[:, j * d:(j + 1) * d]
+    assert np.array_equal(_bits(kc).astype(np.uint32) << 16, kc.view(np.uint32))  # exact in bf16
+    y2, k2, v2 = oracle.prefill_chunk(dims, w, x[T1:], T1, _bits(kc), _bits(vc))
+    np.testing.assert_allclose(np.concatenate([y1, y2]), y, rtol=1e-13, atol=1e-13 * np.abs(y).max())
+    np.testing.assert_array_equal(np.concatenate([k1, k2]), k)
+    # a changed prefix changes the second chunk (it is read), a changed later
+    # token does not change the first
+    kc2 = kc.copy()
+    kc2[0, 0, 0] += 1.0
+    y2b, _, _ = oracle.prefill_chunk(dims, w, x[T1:], T1, _bits(kc2), _bits(vc))
+    assert not np.array_equal(y2b, y2)
+    with pytest.raises(ValueError):
+        oracle.prefill_chunk(dims, w, x[T1:], T1)  # a prefix needs a cache
+
+
+# --------------------------------------------------------------------------
 # Planner extras: Auto shard degree and the TP cost model
 # --------------------------------------------------------------------------
 

@@ -68,17 +68,26 @@ extern "C" {
 #define TPL_NORM 1u          /* pre-RMSNorm before QKV and before gate/up       */
 #define TPL_RESIDUAL 2u      /* residual adds after O and after down            */
 #define TPL_FP32_WEIGHTS 4u  /* fp32 weights and activations (KV stays bf16)    */
+#define TPL_ROPE 8u          /* rotary position embedding of q and k (below)    */
 
 #define TPL_REDUCE_FUSED 0    /* t-way sum inside the row-parallel epilogue     */
 #define TPL_REDUCE_SEPARATE 1 /* partials to memory, then tpl_reduce_partials   */
 
 typedef void *tpl_stream; /* a cudaStream_t */
 
-/* Layer dimensions.  head_dim must be 128; hidden and ffn/t multiples of 8. */
+/* Layer dimensions.  head_dim must be 128; hidden and ffn/t multiples of 8.
+ * With TPL_ROPE, q and the new k of every token are turned to the token's
+ * position before attention and before k enters the cache: for e < 64 the
+ * pair (v[e], v[e + 64]) is rotated by the angle pos * rope_base^(-2e/128)
+ * (the rotary embedding of RoFormer, Su et al. 2021, in the half-split
+ * pairing of the Llama family; the pages do not name a position encoding, so
+ * it is off unless flagged).  rope_base must be > 1 when TPL_ROPE is set and
+ * is ignored otherwise. */
 typedef struct {
     int32_t hidden, n_q_heads, n_kv_heads, head_dim, ffn, n_layers;
     float rms_eps;
-    uint32_t flags; /* TPL_NORM | TPL_RESIDUAL | TPL_FP32_WEIGHTS */
+    uint32_t flags; /* TPL_NORM | TPL_RESIDUAL | TPL_FP32_WEIGHTS | TPL_ROPE */
+    float rope_base;
 } tpl_dims;
 
 typedef struct tpl_plan tpl_plan; /* opaque, host-owned by the library */
@@ -302,12 +311,26 @@ int tpl_prefill_layer(tpl_plan *plan, const void *packed, const tpl_kv *kv, cons
                       int32_t T, void *y, float *y32, void *ws, size_t ws_bytes,
                       int32_t reduce_mode, tpl_stream stream);
 
+/* Chunked prefill: the same layer over T tokens of one sequence whose cache
+ * (batch row 0) already holds `start` tokens in slots 0..start-1.  Token i
+ * sits at position start + i (its rotary angle with TPL_ROPE), attends the
+ * start cached keys and the chunk's keys 0..i, and its k/v go to cache slot
+ * start + i ("Tensor parallel scaling curves", "Prefill vs decode: different
+ * curves": prompt tokens processed in parallel; a long prompt is taken in
+ * chunks).  Requires start >= 0 and start + T <= kv->seq_cap (TPL_ENOMEM);
+ * otherwise as tpl_prefill_layer, which is this call with start = 0.  A
+ * chunk of one token equals a decode step at S = start. */
+int tpl_prefill_chunk(tpl_plan *plan, const void *packed, const tpl_kv *kv, const void *x,
+                      int32_t T, int64_t start, void *y, float *y32, void *ws, size_t ws_bytes,
+                      int32_t reduce_mode, tpl_stream stream);
+
 /* ---- the individual steps (each is one kernel launch, except where noted;
  *      the decode calls above are these in order) --------------------------- */
 
 /* Column-parallel QKV: q [B][n_q][d] fp32; the new token's k/v go to cache
  * slot S (bf16) and, when k_new/v_new are not NULL, also to k_new/v_new
- * [B][n_kv][d] fp32 (both or neither). */
+ * [B][n_kv][d] fp32 (both or neither).  With TPL_ROPE, q and k are rotated
+ * to position S (a second, small kernel) before they are written out. */
 int tpl_qkv(tpl_plan *plan, const void *packed, const tpl_kv *kv, const void *x, int32_t B,
             int64_t S, float *q, float *k_new, float *v_new, void *ws, size_t ws_bytes,
             tpl_stream stream);

@@ -31,6 +31,7 @@ struct AttnPrefillArgs {
     int64_t seq_cap;
     int batch_cap;
     int T, nq, nkv, nkv_s, g;
+    int p0;                           // position of the chunk's first token (cache slots below hold earlier keys)
     int gc, wpc;                      // chunks per query group, heads (warps) per chunk
     float scale_log2;
     __nv_bfloat16 *o_hi, *o_lo;       // [T][nq*128]: output as bf16 hi + lo (the O projection's split operand)
@@ -50,7 +51,7 @@ __global__ void __launch_bounds__(kApMaxWarps * 32) attn_prefill_kernel(const __
     const int head = j * a.g + chunk * a.wpc + warp;
     const int t0 = rt * 16;
     const int t_last = min(a.T - 1, t0 + 15);
-    const int nkb = t_last / kApKeys + 1;  // key tiles up to the last token's
+    const int nkb = (a.p0 + t_last) / kApKeys + 1;  // key tiles up to the last token's
     const int64_t cache_off = (((int64_t)s * a.batch_cap) * a.nkv_s + jl) * a.seq_cap * D;
 
     pdl_wait();
@@ -63,12 +64,13 @@ __global__ void __launch_bounds__(kApMaxWarps * 32) attn_prefill_kernel(const __
             const int plane = u / (kApKeys * 16), r = (u / 16) % kApKeys, piece = u % 16;
             const int key = kb * kApKeys + r;
             __nv_bfloat16 *dst = base + (size_t)plane * kApTile + r * kApRow + piece * 8;
-            if (key < a.T) {
+            // keys below p0 come from earlier chunks: exact in bf16, no low part
+            if (key < a.p0 + a.T && ((plane & 1) == 0 || key >= a.p0)) {
                 const __nv_bfloat16 *src;
                 if (plane == 0) src = a.khi + cache_off + (int64_t)key * D;
-                else if (plane == 1) src = a.klo + ((int64_t)key * a.nkv + j) * D;
+                else if (plane == 1) src = a.klo + ((int64_t)(key - a.p0) * a.nkv + j) * D;
                 else if (plane == 2) src = a.vhi + cache_off + (int64_t)key * D;
-                else src = a.vlo + ((int64_t)key * a.nkv + j) * D;
+                else src = a.vlo + ((int64_t)(key - a.p0) * a.nkv + j) * D;
                 cp_async16(dst, src + piece * 8);
             } else {
                 *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
@@ -108,6 +110,7 @@ __global__ void __launch_bounds__(kApMaxWarps * 32) attn_prefill_kernel(const __
     for (int t = 0; t < 16; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
     float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
     const int ra = t0 + gid, rb_ = t0 + gid + 8;  // query tokens of rows gid, gid+8
+    const int pa = a.p0 + ra, pb = a.p0 + rb_;    // and their positions
 
     stage(0, 0);
     cp_async_commit();
@@ -126,7 +129,7 @@ __global__ void __launch_bounds__(kApMaxWarps * 32) attn_prefill_kernel(const __
         // 4 sub-blocks of 16 keys
         for (int sb = 0; sb < kApKeys / 16; ++sb) {
             const int key0 = kb * kApKeys + sb * 16;
-            if (key0 > t_last) break;
+            if (key0 > a.p0 + t_last) break;
             float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};  // keys key0+.. tile0 / tile1
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
@@ -146,14 +149,14 @@ __global__ void __launch_bounds__(kApMaxWarps * 32) attn_prefill_kernel(const __
             }
             // causal mask and online softmax; s0 cols = keys key0+2c, +1; s1 = key0+8+2c, +1
             const int kk = key0 + 2 * c;
-            const float x0 = kk <= ra ? s0[0] * a.scale_log2 : -INFINITY;
-            const float x1 = kk + 1 <= ra ? s0[1] * a.scale_log2 : -INFINITY;
-            const float x2 = kk + 8 <= ra ? s1[0] * a.scale_log2 : -INFINITY;
-            const float x3 = kk + 9 <= ra ? s1[1] * a.scale_log2 : -INFINITY;
-            const float y0 = kk <= rb_ ? s0[2] * a.scale_log2 : -INFINITY;
-            const float y1 = kk + 1 <= rb_ ? s0[3] * a.scale_log2 : -INFINITY;
-            const float y2 = kk + 8 <= rb_ ? s1[2] * a.scale_log2 : -INFINITY;
-            const float y3 = kk + 9 <= rb_ ? s1[3] * a.scale_log2 : -INFINITY;
+            const float x0 = kk <= pa ? s0[0] * a.scale_log2 : -INFINITY;
+            const float x1 = kk + 1 <= pa ? s0[1] * a.scale_log2 : -INFINITY;
+            const float x2 = kk + 8 <= pa ? s1[0] * a.scale_log2 : -INFINITY;
+            const float x3 = kk + 9 <= pa ? s1[1] * a.scale_log2 : -INFINITY;
+            const float y0 = kk <= pb ? s0[2] * a.scale_log2 : -INFINITY;
+            const float y1 = kk + 1 <= pb ? s0[3] * a.scale_log2 : -INFINITY;
+            const float y2 = kk + 8 <= pb ? s1[2] * a.scale_log2 : -INFINITY;
+            const float y3 = kk + 9 <= pb ? s1[3] * a.scale_log2 : -INFINITY;
             float mxa = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
             float mxb = fmaxf(fmaxf(y0, y1), fmaxf(y2, y3));
             mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 1));

@@ -1,7 +1,10 @@
 // Causal GQA attention of a prefill chunk on the 5th-generation tensor cores
 // ("Tensor parallel scaling curves", "Prefill vs decode: different curves";
 // attention on owned heads, "What tensor parallelism actually splits"):
-// token i attends keys 0..i of the chunk.
+// the chunk's token i sits at position p0 + i and attends keys 0..p0 + i of
+// the cache (slots below p0 were written by earlier chunks; their low parts
+// are zero, read as the fill value of the remainder planes' negative
+// coordinates).
 //
 // One CTA per (kv head j, block of 128/g tokens): its 128 rows are the block's
 // tokens x the g query heads that share kv head j (row = token * g + head), so
@@ -44,12 +47,13 @@ constexpr size_t kAtSmem = (size_t)kAtStages * kAtStageBytes + 1024 + 256;
 constexpr uint32_t kAtQhi = 0, kAtQlo = 64, kAtO = 128, kAtS = 256;
 
 struct AttnTcArgs {
-    CUtensorMap tm_khi, tm_vhi;  // cache [heads of all shards][T (extent)][128] bf16, box {64, 64, 1}
+    CUtensorMap tm_khi, tm_vhi;  // cache [heads of all shards][p0 + T (extent)][128] bf16, box {64, 64, 1}
     CUtensorMap tm_klo, tm_vlo;  // remainders [T][nkv][128] bf16, box {64, 1, 64}
     const float *q32;            // [T][nq][128]
     __nv_bfloat16 *o_hi, *o_lo;  // [T][nq*128]
     int T, nq, nkv, nkv_s, g, tb;  // tb = tokens per CTA = 128 / g
     int batch_cap;
+    int p0;                      // position of the chunk's first token
     float scale_log2;
 };
 
@@ -106,7 +110,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_prefill_tc_kernel(const __
     const int j = (int)(blockIdx.x % a.nkv);
     const int t0 = rt * a.tb;
     const int t_last = min(a.T - 1, t0 + a.tb - 1);
-    const int nkt = t_last / kAtKeys + 1;
+    const int nkt = (a.p0 + t_last) / kAtKeys + 1;
     const int s_sh = j / a.nkv_s, jl = j % a.nkv_s;
     const int head_block = (s_sh * a.batch_cap) * a.nkv_s + jl;  // batch row 0
 
@@ -156,13 +160,15 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_prefill_tc_kernel(const __
                 mbar_expect_tx(&kfull[s], 2 * kAtTileBytes);
                 for (int h = 0; h < 2; ++h) {
                     tma_load_3d(st + h * (kAtTileBytes / 2), &a.tm_khi, 64 * h, key0, head_block, &kfull[s]);
-                    tma_load_3d(st + kAtTileBytes + h * (kAtTileBytes / 2), &a.tm_klo, 64 * h, j, key0, &kfull[s]);
+                    tma_load_3d(st + kAtTileBytes + h * (kAtTileBytes / 2), &a.tm_klo, 64 * h, j, key0 - a.p0,
+                                &kfull[s]);
                 }
                 mbar_expect_tx(&vfull[s], 2 * kAtTileBytes);
                 for (int h = 0; h < 2; ++h) {
                     tma_load_3d(st + 2 * kAtTileBytes + h * (kAtTileBytes / 2), &a.tm_vhi, 64 * h, key0, head_block,
                                 &vfull[s]);
-                    tma_load_3d(st + 3 * kAtTileBytes + h * (kAtTileBytes / 2), &a.tm_vlo, 64 * h, j, key0, &vfull[s]);
+                    tma_load_3d(st + 3 * kAtTileBytes + h * (kAtTileBytes / 2), &a.tm_vlo, 64 * h, j, key0 - a.p0,
+                                &vfull[s]);
                 }
             }
             *s_issued = it;
@@ -281,7 +287,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) attn_prefill_tc_kernel(const __
             float mx = -INFINITY;
 #pragma unroll
             for (int e = 0; e < 64; ++e) {
-                x[e] = (key0 + e <= tok) ? x[e] * a.scale_log2 : -INFINITY;
+                x[e] = (key0 + e <= a.p0 + tok) ? x[e] * a.scale_log2 : -INFINITY;
                 mx = fmaxf(mx, x[e]);
             }
             // raise the running max only when this tile exceeds it by > 8

@@ -73,6 +73,17 @@ __device__ __forceinline__ void store_act(void *p, int is_f32, int64_t i, float 
 
 __device__ __forceinline__ float silu(float z) { return z / (1.0f + expf(-z)); }
 
+// cos and sin of the rotary angle pos * theta.  The angle is formed and
+// brought into [-pi, pi] in fp64 (positions of long sequences give angles of
+// thousands of radians, where fp32 would lose the low bits), then evaluated
+// by the hardware's fp32 approximation, whose absolute error on [-pi, pi]
+// (a few 1e-7) is far below the bf16 rounding the rotated values meet.
+__device__ __forceinline__ void rope_cs(double pos, double theta, float &c, float &s) {
+    const double ang = pos * theta;
+    const double r = ang - 6.283185307179586 * rint(ang * 0.15915494309189535);
+    __sincosf((float)r, &s, &c);
+}
+
 // Asynchronous 16-byte global -> shared copies and ldmatrix fragment loads.
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((unsigned)__cvta_generic_to_shared(dst)), "l"(src)

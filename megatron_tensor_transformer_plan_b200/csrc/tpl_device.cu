@@ -12,6 +12,7 @@
 #include "tpl_gemv_tc.cuh"
 #include "tpl_internal.h"
 #include "tpl_norm.cuh"
+#include "tpl_rope.cuh"
 #include "tpl_tma.h"
 
 namespace tpl {
@@ -309,7 +310,8 @@ int run_row_tc(Ctx &c, const char *packed, int op, const void *x, const void *re
     return gemv_tc_run(c, a, op, false, W, ld, p->d.hidden, p->t, blk, x, (int64_t)p->t * Ks, c.B, (int)Ks);
 }
 
-int run_qkv(Ctx &c, const char *packed, const tpl_kv *kv, const void *x, float *q, float *knew, float *vnew) {
+int run_qkv_proj(Ctx &c, const char *packed, const tpl_kv *kv, const void *x, float *q, float *knew,
+                 float *vnew) {
     tpl_plan *p = c.p;
     if (use_tc(p, OP_QKV, c.B)) return run_qkv_tc(c, packed, kv, x, q, knew, vnew);
     GemvArgs a = base_args(p);
@@ -335,6 +337,35 @@ int run_qkv(Ctx &c, const char *packed, const tpl_kv *kv, const void *x, float *
     a.S = c.S;
     a.seq_cap = kv->seq_cap;
     return gemv_launch(c, a, p->t * p->qkv_rows_s, 1, p->d.hidden, OP_QKV);
+}
+
+// The QKV step: the projection, then (TPL_ROPE) the rotation of q and the new
+// k to position S, which needs the unrounded keys: without caller buffers
+// the workspace's copies are used.
+int run_qkv(Ctx &c, const char *packed, const tpl_kv *kv, const void *x, float *q, float *knew, float *vnew) {
+    tpl_plan *p = c.p;
+    if (p->rope && !knew) {
+        knew = reinterpret_cast<float *>(c.ws + c.L.knew);
+        vnew = reinterpret_cast<float *>(c.ws + c.L.vnew);
+    }
+    int rc = run_qkv_proj(c, packed, kv, x, q, knew, vnew);
+    if (rc != TPL_OK || !p->rope) return rc;
+    RopeArgs r;
+    std::memset(&r, 0, sizeof(r));
+    r.q = q;
+    r.knew = knew;
+    r.kc = static_cast<__nv_bfloat16 *>(kv->k);
+    r.B = c.B;
+    r.nq = p->d.n_q_heads;
+    r.nkv = p->d.n_kv_heads;
+    r.nkv_s = p->nkv_s;
+    r.batch_cap = kv->batch_cap;
+    r.seq_cap = kv->seq_cap;
+    r.pos = c.S;
+    std::memcpy(r.theta, p->rope_theta, sizeof(r.theta));
+    const int64_t heads = (int64_t)c.B * (r.nq + r.nkv);
+    const int64_t grid = (heads + kRopeThreads / 64 - 1) / (kRopeThreads / 64);
+    return cuda_rc(launch_pdl(rope_decode_kernel, (int)grid, kRopeThreads, 0, c.st, r));
 }
 
 bool g_stg_attr[64];
@@ -727,19 +758,25 @@ int tpl_decode_stack(tpl_plan *p, const void *const *packed_per_layer, const tpl
 
 int tpl_prefill_layer(tpl_plan *p, const void *packed, const tpl_kv *kv, const void *x, int32_t T, void *y,
                       float *y32, void *ws, size_t ws_bytes, int32_t reduce_mode, tpl_stream stream) {
-    if (!p || T < 0) return TPL_EINVAL;
+    return tpl_prefill_chunk(p, packed, kv, x, T, 0, y, y32, ws, ws_bytes, reduce_mode, stream);
+}
+
+int tpl_prefill_chunk(tpl_plan *p, const void *packed, const tpl_kv *kv, const void *x, int32_t T, int64_t start,
+                      void *y, float *y32, void *ws, size_t ws_bytes, int32_t reduce_mode, tpl_stream stream) {
+    if (!p || T < 0 || start < 0) return TPL_EINVAL;
     if (reduce_mode != TPL_REDUCE_FUSED && reduce_mode != TPL_REDUCE_SEPARATE) return TPL_EINVAL;
     if (T == 0) return TPL_OK;
     if (p->f32) return TPL_EUNSUPPORTED;
     if (!packed || !x || !ws || !al16(packed) || !al16(x) || !al16(ws) || (!y && !y32)) return TPL_EINVAL;
     if ((y && !al16(y)) || (y32 && !al16(y32))) return TPL_EINVAL;
-    int rc = check_kv(kv, 1, (int64_t)T - 1);
+    int rc = check_kv(kv, 1, start + T - 1);
     if (rc != TPL_OK) return rc;
+    if (start + T > 0x7fffffffll) return TPL_EUNSUPPORTED;  // key positions are 32-bit in the kernels
     PrefillWs L;
     if ((rc = prefill_ws_layout(p, T, &L)) != TPL_OK) return rc;
     if (ws_bytes < L.total) return TPL_EWORKSPACE;
-    return prefill_layer(p, static_cast<const char *>(packed), kv, x, T, y, y32, static_cast<char *>(ws), L,
-                         reduce_mode, static_cast<cudaStream_t>(stream));
+    return prefill_layer(p, static_cast<const char *>(packed), kv, x, T, (int)start, y, y32, static_cast<char *>(ws),
+                         L, reduce_mode, static_cast<cudaStream_t>(stream));
 }
 
 int tpl_last_device_error(const tpl_plan *p, tpl_stream stream) {

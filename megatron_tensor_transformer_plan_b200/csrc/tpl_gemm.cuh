@@ -63,13 +63,16 @@ struct GemmArgs {
     const void *resid;  // GEPI_ROW
     int resid_f32;
     // QKV mapping: q fp32 [M][nq][hd]; k/v rounded to bf16 into the cache
-    // (batch row 0, slot = token) and their rounding remainders into klo/vlo
-    // [M][nkv][hd] bf16
+    // (batch row 0, slot = pos0 + token) and their rounding remainders into
+    // klo/vlo [M][nkv][hd] bf16
     float *q32;
     __nv_bfloat16 *klo, *vlo;
     __nv_bfloat16 *kc, *vc;
     int rps, nq, nq_s, nkv_s, hd, batch_cap;
     int64_t seq_cap;
+    int64_t pos0;       // position of token row 0
+    int rope;           // rotate q and k heads to their positions (hd = 128)
+    double theta[64];   // rotary frequencies
 };
 
 __device__ __forceinline__ unsigned smem_u32(const void *p) { return (unsigned)__cvta_generic_to_shared(p); }
@@ -268,7 +271,8 @@ __device__ __forceinline__ void gemm_epi_chunk(const GemmArgs &a, const float (&
                 lo[i] = v[i] - hi[i];
             }
             __nv_bfloat16 *cc = isk ? a.kc : a.vc;
-            store16_bf16(cc + (((int64_t)s * a.batch_cap) * a.nkv_s + kvl) * a.seq_cap * a.hd + (int64_t)row * a.hd + dim,
+            store16_bf16(cc + (((int64_t)s * a.batch_cap) * a.nkv_s + kvl) * a.seq_cap * a.hd +
+                             (a.pos0 + row) * a.hd + dim,
                          hi);
             __nv_bfloat16 *fl = isk ? a.klo : a.vlo;
             store16_bf16(fl + ((int64_t)row * nkv + s * a.nkv_s + kvl) * a.hd + dim, lo);
@@ -454,6 +458,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
                         // -0 is the additive identity (x + -0 == x for every x,
                         // +-0 included): segment 0 stores its partial unchanged
                         for (int i = 0; i < 16; ++i) sum[16 * j + i] = (seg == 0 ? -0.f : sum[16 * j + i]) + v[i];
+                    }
+                } else if (a.rope && a.epi == GEPI_QKV && (cb % a.rps) < (a.nq_s + a.nkv_s) * a.hd) {
+                    // this warp's 128 columns are one q or k head: turn each
+                    // pair (e, e + 64) by the row's rotary angle
+                    const double pos = (double)(a.pos0 + row);
+                    for (int j = 0; j < 4; ++j) {
+                        float v0[16], v1[16];
+                        tmem_ld16(taddr + 16 * j, v0);
+                        tmem_ld16(taddr + 16 * (j + 4), v1);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            float cs, sn;
+                            rope_cs(pos, a.theta[16 * j + i], cs, sn);
+                            const float x0 = v0[i], x1 = v1[i];
+                            v0[i] = x0 * cs - x1 * sn;
+                            v1[i] = x1 * cs + x0 * sn;
+                        }
+                        gemm_epi_chunk(a, v0, row, cb + 16 * j, su);
+                        gemm_epi_chunk(a, v1, row, cb + 64 + 16 * j, su);
                     }
                 } else {
                     for (int j = 0; j < 8; ++j) {

@@ -11,6 +11,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstring>
 #include <new>
 
@@ -26,7 +27,8 @@ int validate(const tpl_dims *d, int32_t t) {
         d->ffn <= 0 || d->n_layers <= 0)
         return TPL_EINVAL;
     if (!(d->rms_eps >= 0.0f)) return TPL_EINVAL;
-    if (d->flags & ~(TPL_NORM | TPL_RESIDUAL | TPL_FP32_WEIGHTS)) return TPL_EINVAL;
+    if (d->flags & ~(TPL_NORM | TPL_RESIDUAL | TPL_FP32_WEIGHTS | TPL_ROPE)) return TPL_EINVAL;
+    if ((d->flags & TPL_ROPE) && !(d->rope_base > 1.0f)) return TPL_EINVAL;
     if (!(t == 1 || t == 2 || t == 4 || t == 8)) return TPL_EINDIVISIBLE;
     if (d->n_q_heads % t || d->n_kv_heads % t || d->ffn % t) return TPL_EINDIVISIBLE;
     if (d->n_q_heads % d->n_kv_heads) return TPL_EINDIVISIBLE;
@@ -229,6 +231,9 @@ int tpl_plan_create(const tpl_dims *dims, int32_t t, tpl_plan **out) {
     p->gemv_mode = p->f32 ? 1 : 4;
     p->attn_prefill_mode = 0;
     p->attn_decode_mode = 0;
+    p->rope = (dims->flags & TPL_ROPE) != 0;
+    for (int e = 0; e < 64; ++e)
+        p->rope_theta[e] = p->rope ? std::pow((double)dims->rope_base, -2.0 * e / dims->head_dim) : 0.0;
     const int64_t H = dims->hidden, es = p->esize;
     // rows padded with zeros to whole 128-column blocks
     p->ld_h = (int)align_up(H, 128);

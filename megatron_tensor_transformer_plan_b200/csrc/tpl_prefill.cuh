@@ -118,8 +118,8 @@ bool g_at_attr[64];
 // Tensor-core attention: 128 rows per CTA = (128 / g) tokens x the g heads of
 // a kv head, so g must be a power of two.
 int run_attn_prefill_tc(const tpl_plan *p, const tpl_kv *kv, const float *q, const __nv_bfloat16 *klo,
-                        const __nv_bfloat16 *vlo, int T, __nv_bfloat16 *o_hi, __nv_bfloat16 *o_lo, cudaStream_t st,
-                        int dev) {
+                        const __nv_bfloat16 *vlo, int T, int p0, __nv_bfloat16 *o_hi, __nv_bfloat16 *o_lo,
+                        cudaStream_t st, int dev) {
     if (!g_at_attr[dev]) {
         if (cudaFuncSetAttribute(attn_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAtSmem) !=
             cudaSuccess)
@@ -130,10 +130,11 @@ int run_attn_prefill_tc(const tpl_plan *p, const tpl_kv *kv, const float *q, con
     std::memset(&a, 0, sizeof(a));
     const int nkv = p->d.n_kv_heads;
     const uint64_t head_blocks = (uint64_t)p->t * kv->batch_cap * p->nkv_s;
-    // cache planes: [head blocks][keys < T][128]; keys past the chunk read as 0
-    int rc = make_map(&a.tm_khi, kv->k, 128, (uint64_t)T, 256, 64, kAtKeys, head_blocks, (uint64_t)kv->seq_cap * 256);
+    // cache planes: [head blocks][keys < p0 + T][128]; keys past the chunk read as 0
+    const uint64_t keys = (uint64_t)p0 + (uint64_t)T;
+    int rc = make_map(&a.tm_khi, kv->k, 128, keys, 256, 64, kAtKeys, head_blocks, (uint64_t)kv->seq_cap * 256);
     if (rc == TPL_OK)
-        rc = make_map(&a.tm_vhi, kv->v, 128, (uint64_t)T, 256, 64, kAtKeys, head_blocks, (uint64_t)kv->seq_cap * 256);
+        rc = make_map(&a.tm_vhi, kv->v, 128, keys, 256, 64, kAtKeys, head_blocks, (uint64_t)kv->seq_cap * 256);
     // remainder planes: [T][nkv][128]
     if (rc == TPL_OK) rc = make_map(&a.tm_klo, klo, 128, nkv, 256, 64, 1, (uint64_t)T, (uint64_t)nkv * 256, kAtKeys);
     if (rc == TPL_OK) rc = make_map(&a.tm_vlo, vlo, 128, nkv, 256, 64, 1, (uint64_t)T, (uint64_t)nkv * 256, kAtKeys);
@@ -142,6 +143,7 @@ int run_attn_prefill_tc(const tpl_plan *p, const tpl_kv *kv, const float *q, con
     a.o_hi = o_hi;
     a.o_lo = o_lo;
     a.T = T;
+    a.p0 = p0;
     a.nq = p->d.n_q_heads;
     a.nkv = nkv;
     a.nkv_s = p->nkv_s;
@@ -155,11 +157,12 @@ int run_attn_prefill_tc(const tpl_plan *p, const tpl_kv *kv, const float *q, con
 }
 
 int run_attn_prefill(const tpl_plan *p, const tpl_kv *kv, const float *q, const __nv_bfloat16 *klo,
-                     const __nv_bfloat16 *vlo, int T, __nv_bfloat16 *o_hi, __nv_bfloat16 *o_lo, cudaStream_t st) {
+                     const __nv_bfloat16 *vlo, int T, int p0, __nv_bfloat16 *o_hi, __nv_bfloat16 *o_lo,
+                     cudaStream_t st) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return TPL_ECUDA;
     if ((p->g & (p->g - 1)) == 0 && p->attn_prefill_mode == 0)
-        return run_attn_prefill_tc(p, kv, q, klo, vlo, T, o_hi, o_lo, st, dev);
+        return run_attn_prefill_tc(p, kv, q, klo, vlo, T, p0, o_hi, o_lo, st, dev);
     if (!g_ap_attr[dev]) {
         if (cudaFuncSetAttribute(attn_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kApSmem) !=
             cudaSuccess)
@@ -176,6 +179,7 @@ int run_attn_prefill(const tpl_plan *p, const tpl_kv *kv, const float *q, const 
     a.seq_cap = kv->seq_cap;
     a.batch_cap = kv->batch_cap;
     a.T = T;
+    a.p0 = p0;
     a.nq = p->d.n_q_heads;
     a.nkv = p->d.n_kv_heads;
     a.nkv_s = p->nkv_s;
@@ -192,8 +196,8 @@ int run_attn_prefill(const tpl_plan *p, const tpl_kv *kv, const float *q, const 
     return cuda_rc(launch_pdl(attn_prefill_kernel, (int)grid, a.wpc * 32, kApSmem, st, a));
 }
 
-int prefill_layer(tpl_plan *p, const char *packed, const tpl_kv *kv, const void *x, int T, void *y, float *y32,
-                  char *ws, const PrefillWs &L, int mode, cudaStream_t st) {
+int prefill_layer(tpl_plan *p, const char *packed, const tpl_kv *kv, const void *x, int T, int p0, void *y,
+                  float *y32, char *ws, const PrefillWs &L, int mode, cudaStream_t st) {
     const bool resid = (p->d.flags & TPL_RESIDUAL) != 0;
     const int64_t H = p->d.hidden, hd = p->d.head_dim;
     auto *a_hi = reinterpret_cast<__nv_bfloat16 *>(ws + L.a_hi);
@@ -225,10 +229,13 @@ int prefill_layer(tpl_plan *p, const char *packed, const tpl_kv *kv, const void 
         a.hd = (int)hd;
         a.batch_cap = kv->batch_cap;
         a.seq_cap = kv->seq_cap;
+        a.pos0 = p0;
+        a.rope = p->rope ? 1 : 0;
+        std::memcpy(a.theta, p->rope_theta, sizeof(a.theta));
         rc = gemm_column(a, a_hi, a_lo, H, packed + p->off_qkv, (int64_t)p->t * p->qkv_rows_s, p->ld_h, st);
         if (rc != TPL_OK) return rc;
     }
-    rc = run_attn_prefill(p, kv, q, klo, vlo, T, o, o_lo, st);
+    rc = run_attn_prefill(p, kv, q, klo, vlo, T, p0, o, o_lo, st);
     if (rc != TPL_OK) return rc;
     {  // O: h = x + sum_s o_s Wo[s]^T
         GemmArgs a = gemm_args(T);

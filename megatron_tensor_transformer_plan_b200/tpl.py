@@ -22,7 +22,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 (TPL_OK, TPL_EINVAL, TPL_EINDIVISIBLE, TPL_EWORKSPACE, TPL_ENOMEM, TPL_ECUDA, TPL_EDEVICE, TPL_EUNSUPPORTED,
  TPL_ENOFIT) = range(9)
-TPL_NORM, TPL_RESIDUAL, TPL_FP32_WEIGHTS = 1, 2, 4
+TPL_NORM, TPL_RESIDUAL, TPL_FP32_WEIGHTS, TPL_ROPE = 1, 2, 4, 8
 TPL_REDUCE_FUSED, TPL_REDUCE_SEPARATE = 0, 1
 TPL_OPT_GEMV_MODE = 1
 TPL_OPT_PREFILL_ATTN = 2
@@ -35,7 +35,8 @@ P = ctypes.POINTER
 
 class tpl_dims(ctypes.Structure):
     _fields_ = [("hidden", c_int32), ("n_q_heads", c_int32), ("n_kv_heads", c_int32), ("head_dim", c_int32),
-                ("ffn", c_int32), ("n_layers", c_int32), ("rms_eps", ctypes.c_float), ("flags", c_uint32)]
+                ("ffn", c_int32), ("n_layers", c_int32), ("rms_eps", ctypes.c_float), ("flags", c_uint32),
+                ("rope_base", ctypes.c_float)]
 
 
 class tpl_tp_estimate(ctypes.Structure):
@@ -94,6 +95,8 @@ _sig("tpl_decode_stack", ctypes.c_int, _plan_p, P(c_void_p), P(tpl_kv), c_void_p
      c_void_p, c_void_p, c_size_t, c_int32, c_void_p)
 _sig("tpl_prefill_layer", ctypes.c_int, _plan_p, c_void_p, P(tpl_kv), c_void_p, c_int32, c_void_p, c_void_p,
      c_void_p, c_size_t, c_int32, c_void_p)
+_sig("tpl_prefill_chunk", ctypes.c_int, _plan_p, c_void_p, P(tpl_kv), c_void_p, c_int32, c_int64, c_void_p,
+     c_void_p, c_void_p, c_size_t, c_int32, c_void_p)
 _sig("tpl_qkv", ctypes.c_int, _plan_p, c_void_p, P(tpl_kv), c_void_p, c_int32, c_int64, c_void_p, c_void_p,
      c_void_p, c_void_p, c_size_t, c_void_p)
 _sig("tpl_attn_decode", ctypes.c_int, _plan_p, P(tpl_kv), c_void_p, c_void_p, c_void_p, c_int32, c_int64, c_void_p,
@@ -128,8 +131,8 @@ def check(code: int, where: str = "") -> None:
 
 
 def make_dims(hidden, n_q_heads, n_kv_heads, head_dim, ffn, n_layers=1, rms_eps=1e-5,
-              flags=TPL_NORM | TPL_RESIDUAL) -> tpl_dims:
-    return tpl_dims(hidden, n_q_heads, n_kv_heads, head_dim, ffn, n_layers, rms_eps, flags)
+              flags=TPL_NORM | TPL_RESIDUAL, rope_base=500000.0) -> tpl_dims:
+    return tpl_dims(hidden, n_q_heads, n_kv_heads, head_dim, ffn, n_layers, rms_eps, flags, rope_base)
 
 
 def footprint_bytes(dims: tpl_dims, t: int, batch: int, seq: int, bytes_per_elem: int = 2) -> int:
@@ -297,6 +300,11 @@ class Plan:
         T = x.shape[0]
         check(tpl_prefill_layer(self.handle, packed.data_ptr(), ctypes.byref(kv), x.data_ptr(), T, _ptr(y),
                                 _ptr(y32), ws.data_ptr(), ws.numel(), mode, _stream()), "tpl_prefill_layer")
+
+    def prefill_chunk(self, packed, kv: tpl_kv, x, start: int, y, y32=None, ws=None, mode=TPL_REDUCE_FUSED):
+        T = x.shape[0]
+        check(tpl_prefill_chunk(self.handle, packed.data_ptr(), ctypes.byref(kv), x.data_ptr(), T, start, _ptr(y),
+                                _ptr(y32), ws.data_ptr(), ws.numel(), mode, _stream()), "tpl_prefill_chunk")
 
     def decode_stack(self, packed_list, kv_list, x, S: int, y, y32=None, ws=None, mode=TPL_REDUCE_FUSED):
         L = len(packed_list)

@@ -87,7 +87,8 @@ def oracle_weights(L: Layer) -> dict:
 def oracle_dims(L: Layer) -> oracle.Dims:
     d = L.dims
     return oracle.Dims(d.hidden, d.n_q_heads, d.n_kv_heads, d.head_dim, d.ffn, eps=float(d.rms_eps),
-                       flags=int(d.flags) & 3)
+                       flags=int(d.flags) & (tpl.TPL_NORM | tpl.TPL_RESIDUAL | tpl.TPL_ROPE),
+                       rope_base=float(d.rope_base))
 
 
 def oracle_decode(L: Layer, x=None):

@@ -77,7 +77,8 @@ class Prefill:
     def _oracle_args(self):
         d = self.dims
         dims = oracle.Dims(d.hidden, d.n_q_heads, d.n_kv_heads, d.head_dim, d.ffn, eps=float(d.rms_eps),
-                           flags=int(d.flags) & 3)
+                           flags=int(d.flags) & (tpl.TPL_NORM | tpl.TPL_RESIDUAL | tpl.TPL_ROPE),
+                           rope_base=float(d.rope_base))
         w = {k: synth.bits(v) for k, v in self.w.items()}
         return dims, w, to_np(self.x)
 

@@ -112,3 +112,15 @@ def test_plan_report_reproduces_the_pages_examples(tpl):
     rows = plan_report.report("70b", batch=16, seq=8192, gpu_gb=80, headroom=0.1)
     assert rows[0]["auto_t"] == 4
     assert rows[1]["t_memory_ms"] > rows[1]["t_compute_ms"] > 0
+
+
+def test_rope_flag_validation(tpl):
+    d = tpl.make_dims(1024, 16, 4, 128, 2816, 1, 1e-5, tpl.TPL_NORM | tpl.TPL_ROPE, rope_base=10000.0)
+    tpl.Plan(d, 4)
+    for bad in (1.0, 0.0, -5.0, float("nan")):
+        d = tpl.make_dims(1024, 16, 4, 128, 2816, 1, 1e-5, tpl.TPL_ROPE, rope_base=bad)
+        with pytest.raises(tpl.TplError) as e:
+            tpl.Plan(d, 4)
+        assert e.value.code == tpl.TPL_EINVAL
+    # without the flag the base is ignored
+    tpl.Plan(tpl.make_dims(1024, 16, 4, 128, 2816, 1, 1e-5, tpl.TPL_NORM, rope_base=0.0), 4)

@@ -97,6 +97,7 @@ def main() -> None:
     ap.add_argument("--iters", type=int, default=30)
     ap.add_argument("--only", default="")
     ap.add_argument("--gemv-mode", type=int, default=4, help="TPL_OPT_GEMV_MODE of the plan (4: the default)")
+    ap.add_argument("--rope", action="store_true", help="rotary embedding on (TPL_ROPE)")
     args = ap.parse_args()
     build.build()
     from megatron_tensor_transformer_plan_b200 import tpl
@@ -115,11 +116,15 @@ def main() -> None:
         for mode in ("fused", "separate"):
             if c["t"] == 1 and mode == "separate":
                 continue
+            flags = c.get("flags")
+            if args.rope and not c.get("mlp_only", False):
+                flags = tpl.TPL_NORM | tpl.TPL_RESIDUAL | tpl.TPL_ROPE
             us, nbytes, ncopies, rc = run_layer(tpl, c["H"], c["nq"], c["nkv"], c["F"], c["t"], c["B"], c["S"],
-                                                 args.iters, mode, c.get("flags"), c.get("mlp_only", False),
+                                                 args.iters, mode, flags, c.get("mlp_only", False),
                                                  args.gemv_mode)
             gbs = nbytes / (us * 1e-6) / 1e9
-            print(json.dumps({"workload": name, "gemv_mode": args.gemv_mode, "t": c["t"], "B": c["B"], "S": c["S"],
+            print(json.dumps({"workload": name, "gemv_mode": args.gemv_mode, "rope": args.rope, "t": c["t"],
+                              "B": c["B"], "S": c["S"],
                               "reduce": mode,
                               "us_per_layer": round(us, 2), "algorithmic_bytes": nbytes, "gb_s": round(gbs, 1),
                               "frac_of_peak": round(gbs / peak, 4), "peak_gb_s": peak, "peak_kind": kind,

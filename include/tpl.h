@@ -61,7 +61,8 @@ extern "C" {
                                word, read by tpl_last_device_error)              */
 #define TPL_EUNSUPPORTED 7  /* valid dimensions this build does not implement
                                (head_dim != 128, group size > 16, dims not a
-                               multiple of 8)                                    */
+                               multiple of 8; more than 64 decode tokens per
+                               call, more than 16 with fp32 weights)             */
 #define TPL_ENOFIT 8        /* tpl_auto_t: no admissible degree fits the budget  */
 
 /* ---- flags ------------------------------------------------------------- */
@@ -268,7 +269,9 @@ int tpl_pack_kv(const tpl_plan *plan, const void *unsharded, void *sharded, int3
                 int64_t seq_cap, tpl_stream stream);
 
 /* One decode step of one layer for B sequences with S cached tokens each
- * (the new token is position S; requires S < kv->seq_cap, B <= batch_cap):
+ * (the new token is position S; requires S < kv->seq_cap, B <= batch_cap;
+ * B <= 64, and B <= 16 for fp32 plans.  Above 16 tokens the projections run
+ * on the tensor-core kernel whatever TPL_OPT_GEMV_MODE says):
  *   a = RMSNorm(x)            [TPL_NORM]
  *   q|k|v = column-parallel projection of a, k/v written to slot S
  *   o = owned-head GQA attention over the S+1 positions

@@ -103,7 +103,8 @@ struct Ctx {
 
 int make_ctx(tpl_plan *p, void *ws, size_t ws_bytes, int B, int64_t S, tpl_stream stream, Ctx *c) {
     if (!p || !ws || !al16(ws)) return TPL_EINVAL;
-    if (B < 1 || B > 16 || S < 0) return B > 16 ? TPL_EUNSUPPORTED : TPL_EINVAL;
+    if (B < 1 || S < 0) return TPL_EINVAL;
+    if (B > (p->f32 ? kMaxBatchCuda : kMaxBatch)) return TPL_EUNSUPPORTED;
     int rc = ws_layout(p, B, S, &c->L);
     if (rc != TPL_OK) return rc;
     if (ws_bytes < c->L.total) return TPL_EWORKSPACE;
@@ -123,6 +124,7 @@ int check_kv(const tpl_kv *kv, int B, int64_t S) {
 
 int gemv_launch(Ctx &c, GemvArgs &a, int N, int nseg, int Kseg, int op) {
     tpl_plan *p = c.p;
+    if (c.B > kMaxBatchCuda) return TPL_EUNSUPPORTED;
     const int sms = num_sms_current();
     if (sms <= 0) return TPL_ECUDA;
     // The Q projection feeds a softmax and gate/up feeds SwiGLU: carry their
@@ -163,7 +165,7 @@ GemvArgs base_args(const tpl_plan *p) {
 
 // ---- tensor-core decode projections (TPL_OPT_GEMV_MODE 3) -----------------
 
-bool g_gt_attr[64][3];
+bool g_gt_attr[64][8];
 
 template <int NX, bool SPLIT>
 int gt_go(int slot, GemvTcArgs &a, cudaStream_t st) {
@@ -171,19 +173,16 @@ int gt_go(int slot, GemvTcArgs &a, cudaStream_t st) {
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return TPL_ECUDA;
     if (!g_gt_attr[dev][slot]) {
         if (cudaFuncSetAttribute(gemv_tc_kernel<NX, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 GemvTcSmem<NX>::BYTES) != cudaSuccess)
+                                 GemvTcSmem<NX, SPLIT>::BYTES) != cudaSuccess)
             return TPL_ECUDA;
         g_gt_attr[dev][slot] = true;
     }
     const int sms = num_sms_current();
     if (sms <= 0) return TPL_ECUDA;
     const int64_t G = std::min<int64_t>(std::min<int64_t>(sms, a.U), kGemvTcMaxCtas);
-    return cuda_rc(launch_pdl(gemv_tc_kernel<NX, SPLIT>, (int)G, kGtThreads, (size_t)GemvTcSmem<NX>::BYTES, st, a));
+    return cuda_rc(
+        launch_pdl(gemv_tc_kernel<NX, SPLIT>, (int)G, kGtThreads, (size_t)GemvTcSmem<NX, SPLIT>::BYTES, st, a));
 }
-
-// MMA N: the B token rows (and with a split activation their lo rows), at
-// least 16 and a multiple of 16.
-int gt_nx(int B, bool split) { return split ? (B <= 8 ? 16 : 32) : 16; }
 
 // Fill the geometry, the weight map (2-D column-parallel rows or 3-D per-shard
 // blocks) and the activation map, then launch.
@@ -207,9 +206,21 @@ int gemv_tc_run(Ctx &c, GemvTcArgs &a, int op, bool split, const void *W, int64_
     if (rc == TPL_OK) rc = make_map(&a.tm_x, X, Kx, x_rows, Kx * 2, kGtK, nx);
     if (rc != TPL_OK) return rc;
     a.gpart = reinterpret_cast<float *>(c.ws + c.L.gpart);
+    a.gstride = gt_stride(c.B);
     a.tickets = reinterpret_cast<unsigned *>(c.ws + c.L.tickets) + kTicketGemv + 512 * op;
-    if (split) return nx == 16 ? gt_go<16, true>(0, a, c.st) : gt_go<32, true>(1, a, c.st);
-    return gt_go<16, false>(2, a, c.st);
+    if (split) {
+        switch (nx) {
+            case 16: return gt_go<16, true>(0, a, c.st);
+            case 32: return gt_go<32, true>(1, a, c.st);
+            case 64: return gt_go<64, true>(2, a, c.st);
+            default: return gt_go<128, true>(3, a, c.st);
+        }
+    }
+    switch (nx) {
+        case 16: return gt_go<16, false>(4, a, c.st);
+        case 32: return gt_go<32, false>(5, a, c.st);
+        default: return gt_go<64, false>(6, a, c.st);
+    }
 }
 
 // TPL_OPT_GEMV_MODE 4 (the default for bf16 plans): one kernel family for all
@@ -218,11 +229,14 @@ int gemv_tc_run(Ctx &c, GemvTcArgs &a, int op, bool split, const void *W, int64_
 // mma.sync kernel overlaps consecutive launches better (programmatic
 // dependent launch), and layers that mix the two families measured slower
 // than either.  So: tcgen05 with more than 8 tokens on layers of at least
-// 1 GiB of weights, mma.sync otherwise.
+// 1 GiB of weights, mma.sync otherwise.  Beyond 16 tokens (any mode) only
+// the tcgen05 kernel applies.
 bool use_tc(const tpl_plan *p, int op, int B) {
     (void)op;
-    if (p->gemv_mode == 3) return B <= kGtMaxB;
-    if (p->gemv_mode != 4 || B > kGtMaxB) return false;
+    if (p->f32) return false;
+    if (B > kMaxBatchCuda) return true;  // beyond the mma.sync kernel's 16 tokens
+    if (p->gemv_mode == 3) return true;
+    if (p->gemv_mode != 4) return false;
     const tpl_dims &d = p->d;
     const int64_t layer_params = (int64_t)(d.n_q_heads + 2 * d.n_kv_heads) * d.head_dim * d.hidden +
                                  (int64_t)d.hidden * d.n_q_heads * d.head_dim + 3 * (int64_t)d.ffn * d.hidden;
@@ -817,7 +831,7 @@ extern "C" int tpl_attn_decode_static(tpl_plan *p, const tpl_kv *kv, const float
                                       const float *v_new, int32_t B, int64_t S, void *o, tpl_stream stream) {
     if (!p || !q || !o || !al16(q) || B < 0 || S < 0 || (!k_new != !v_new)) return TPL_EINVAL;
     if (B == 0) return TPL_OK;
-    if (B > 16) return TPL_EUNSUPPORTED;
+    if (B > kMaxBatch) return TPL_EUNSUPPORTED;
     int rc = check_kv(kv, B, S);
     if (rc != TPL_OK) return rc;
     const int64_t keys = k_new ? S : S + 1;

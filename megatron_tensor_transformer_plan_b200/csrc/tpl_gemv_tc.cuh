@@ -1,14 +1,15 @@
-// Decode projections (B <= 16 tokens) on the 5th-generation tensor cores.
+// Decode projections (B <= 64 tokens) on the 5th-generation tensor cores.
 //
 // D[128 weight rows][NX columns] = W[128][K] . X[NX][K]^T in TMEM, where X
 // holds the B tokens' activation rows (bf16; with SPLIT, hi parts in rows
-// 0..B-1 and lo parts in rows NX/2..NX/2+B-1, the rest zero).  The kernel is bound by
-// streaming the weights from HBM: TMA brings 128-row x 64-column weight tiles
-// (16 KB, 128-byte swizzle) and the matching activation tile into a 10-11
-// stage shared-memory ring, one thread issues four M=128, N=NX, K=16 tcgen05.mma per
-// stage, and the tensor pipe idles most of the time.  192 threads: warp 0 TMA
-// producer, warp 1 TMEM owner and MMA issuer, warps 2-5 epilogue (one TMEM
-// lane = one weight row each).
+// 0..B-1 and lo parts in rows NX/2..NX/2+B-1, the rest zero; NX = 16..128).
+// The kernel is bound by streaming the weights from HBM: TMA brings 128-row x
+// 64-column weight tiles (16 KB, 128-byte swizzle) and the matching activation
+// tile into a 6-11 stage shared-memory ring, one thread issues four M=128,
+// N=NX, K=16 tcgen05.mma per stage, and the tensor pipe idles most of the
+// time.  192 threads: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer,
+// warps 2-5 epilogue (one TMEM lane = one weight row each), which walks the
+// tokens in chunks of 16 columns so that its registers do not grow with B.
 //
 // Work division ("stream-K"): the k-blocks of every (row tile, segment) are
 // laid end to end, tile-major then segment then k, and each CTA takes one
@@ -43,16 +44,23 @@ constexpr int kGtRows = 128;     // weight rows per tile (MMA M)
 constexpr int kGtK = 64;         // columns per k-block
 constexpr int kGtWBytes = kGtRows * kGtK * 2;  // 16 KB
 constexpr int kGtBufs = 4;       // TMEM accumulators in flight
-constexpr int kGtMaxB = 16;
+constexpr int kGtMaxB = 64;       // tokens per call
+constexpr int kGtChunk = 16;      // tokens per epilogue chunk
 constexpr int kGtList = 120;      // piece list entries per combine chunk
 constexpr int kGtBarBytes = 1024;  // mbarriers, flags and the piece list after the stage ring
 
-template <int NX>
+// Shared memory: the stage ring, the running tile sums of tiles finished
+// inside one CTA ([tokens][128 rows] fp32), then the barrier area.
+template <int NX, bool SPLIT>
 struct GemvTcSmem {
     static constexpr int XBYTES = NX * kGtK * 2;
     static constexpr int STAGE = kGtWBytes + XBYTES;
-    static constexpr int NS = (200 * 1024) / STAGE;
-    static constexpr int BYTES = NS * STAGE + 1024 + kGtBarBytes;
+    static constexpr int TOK = SPLIT ? NX / 2 : NX;  // token columns of the accumulator
+    static constexpr int NCH = TOK < kGtChunk ? 1 : TOK / kGtChunk;
+    static constexpr int TSBYTES = NCH * kGtChunk * kGtRows * 4;
+    static constexpr int NS = ((NX >= 64 ? 224 : 208) * 1024 - TSBYTES) / STAGE;
+    static constexpr int BYTES = NS * STAGE + TSBYTES + 1024 + kGtBarBytes;
+    static_assert(BYTES <= 232448, "shared memory per block");
 };
 
 enum { GT_QKV = 0, GT_GU = 1, GT_ROW = 2, GT_ROW_PARTIAL = 3 };
@@ -80,43 +88,48 @@ struct GemvTcArgs {
     int rps, nq, nq_s, nkv_s, hd, batch_cap;
     int64_t S, seq_cap;
     // cross-CTA pieces and arrival counters
-    float *gpart;       // [G][2][nseg][128][16]
+    float *gpart;       // [G][2][nseg][gstride / 4][128] float4: token quads outer, rows inner
+    int gstride;        // floats per row of a piece: 16 * ceil(B / 16)
     unsigned *tickets;  // [tiles]
 };
 
-template <int NX>
-__device__ __forceinline__ void tmem_ld_nx(uint32_t taddr, float (&v)[NX]) {
-    if constexpr (NX == 16) {
-        float t[16];
-        tmem_ld16(taddr, t);
+// Tokens 16*ch .. 16*ch+15 of one accumulator row: the hi column plus the
+// lo column NX/2 further (SPLIT), or the column itself.
+template <int NX, bool SPLIT>
+__device__ __forceinline__ void gt_load_chunk(uint32_t taddr, int ch, float (&pv)[kGtChunk]) {
+    if constexpr (SPLIT && NX == 16) {  // 8 tokens: hi in columns 0..7, lo in 8..15
+        float d[16];
+        tmem_ld16(taddr, d);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = t[i];
+        for (int t = 0; t < 16; ++t) pv[t] = t < 8 ? d[t] + d[8 + t] : 0.f;
+    } else if constexpr (SPLIT) {
+        float hi[16], lo[16];
+        tmem_ld16(taddr + (uint32_t)(16 * ch), hi);
+        tmem_ld16(taddr + (uint32_t)(NX / 2 + 16 * ch), lo);
+#pragma unroll
+        for (int t = 0; t < 16; ++t) pv[t] = hi[t] + lo[t];
     } else {
-        float t0[16], t1[16];
-        tmem_ld16(taddr, t0);
-        tmem_ld16(taddr + 16, t1);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            v[i] = t0[i];
-            v[16 + i] = t1[i];
-        }
+        tmem_ld16(taddr + (uint32_t)(16 * ch), pv);
     }
 }
 
 // CTA c's unit range [u0, u1) of U units over G CTAs.
 __device__ __forceinline__ int64_t gt_start(int64_t U, int G, int c) { return U * c / G; }
 
-// Final write of one output row for all tokens (fused sums or column ops).
-__device__ __forceinline__ void gt_final(const GemvTcArgs &a, int row, const float (&v)[kGtMaxB], int lane) {
+// Final write of one output row for tokens tok0 .. tok0+15 (fused sums or
+// column ops).
+__device__ __forceinline__ void gt_final(const GemvTcArgs &a, int row, const float (&v)[kGtChunk], int lane,
+                                         int tok0) {
     const int B = a.B;
     if (a.epi == GT_GU) {
         // rows interleave gate and up: the even lane pairs with its odd neighbour
 #pragma unroll
-        for (int b = 0; b < kGtMaxB; ++b) {
-            const float u = __shfl_down_sync(0xffffffffu, v[b], 1);
+        for (int i = 0; i < kGtChunk; ++i) {
+            const int b = tok0 + i;
+            const float u = __shfl_down_sync(0xffffffffu, v[i], 1);
             if (b < B && !(lane & 1) && row + 1 < a.N)
                 static_cast<__nv_bfloat16 *>(a.out_act)[(int64_t)b * (a.N / 2) + row / 2] =
-                    __float2bfloat16_rn(silu(v[b]) * u);
+                    __float2bfloat16_rn(silu(v[i]) * u);
         }
         return;
     }
@@ -125,30 +138,32 @@ __device__ __forceinline__ void gt_final(const GemvTcArgs &a, int row, const flo
         const int s = row / a.rps, l = row % a.rps;
         const int qd = a.nq_s * a.hd, kd = a.nkv_s * a.hd;
 #pragma unroll
-        for (int b = 0; b < kGtMaxB; ++b) {
+        for (int i = 0; i < kGtChunk; ++i) {
+            const int b = tok0 + i;
             if (b >= B) continue;
             if (l < qd) {
                 const int head = s * a.nq_s + l / a.hd, dim = l % a.hd;
-                a.q[((int64_t)b * a.nq + head) * a.hd + dim] = v[b];
+                a.q[((int64_t)b * a.nq + head) * a.hd + dim] = v[i];
             } else {
                 const bool isk = l < qd + kd;
                 const int ll = isk ? l - qd : l - qd - kd;
                 const int kvl = ll / a.hd, dim = ll % a.hd;
                 __nv_bfloat16 *c = isk ? a.kc : a.vc;
                 c[((((int64_t)s * a.batch_cap + b) * a.nkv_s + kvl) * a.seq_cap + a.S) * a.hd + dim] =
-                    __float2bfloat16_rn(v[b]);
+                    __float2bfloat16_rn(v[i]);
                 float *f = isk ? a.knew : a.vnew;
-                if (f) f[((int64_t)b * (a.nkv_s * (a.nq / a.nq_s)) + s * a.nkv_s + kvl) * a.hd + dim] = v[b];
+                if (f) f[((int64_t)b * (a.nkv_s * (a.nq / a.nq_s)) + s * a.nkv_s + kvl) * a.hd + dim] = v[i];
             }
         }
         return;
     }
     // GT_ROW: out = resid + sum
 #pragma unroll
-    for (int b = 0; b < kGtMaxB; ++b) {
+    for (int j = 0; j < kGtChunk; ++j) {
+        const int b = tok0 + j;
         if (b >= B) continue;
         const int64_t i = (int64_t)b * a.N + row;
-        float o = v[b];
+        float o = v[j];
         if (a.resid) o = load_act(a.resid, a.resid_f32, i) + o;
         if (a.out32) a.out32[i] = o;
         if (a.out_act) static_cast<__nv_bfloat16 *>(a.out_act)[i] = __float2bfloat16_rn(o);
@@ -157,14 +172,17 @@ __device__ __forceinline__ void gt_final(const GemvTcArgs &a, int row, const flo
 
 template <int NX, bool SPLIT>
 __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_constant__ GemvTcArgs a) {
-    constexpr int STAGE = GemvTcSmem<NX>::STAGE;
-    constexpr int NS = GemvTcSmem<NX>::NS;
+    using SMEM = GemvTcSmem<NX, SPLIT>;
+    constexpr int STAGE = SMEM::STAGE;
+    constexpr int NS = SMEM::NS;
     static_assert(2 * NS * 8 + 2 * kGtBufs * 8 + 8 + 4 + 32 + 4 * kGtList <= kGtBarBytes, "barrier area");
-    constexpr int TMEM_COLS = kGtBufs * NX <= 32 ? 32 : kGtBufs * NX <= 64 ? 64 : 128;
-    static_assert(kGtBufs * NX <= 128, "accumulators");
+    constexpr int TMEM_COLS = kGtBufs * NX <= 32 ? 32 : kGtBufs * NX <= 64 ? 64 : kGtBufs * NX <= 128 ? 128
+                              : kGtBufs * NX <= 256 ? 256 : 512;
+    static_assert(kGtBufs * NX <= 512, "accumulators");
     extern __shared__ __align__(1024) unsigned char gv_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(((uintptr_t)gv_raw + 1023) & ~(uintptr_t)1023);
-    uint64_t *full = reinterpret_cast<uint64_t *>(sm + NS * STAGE);
+    float *ts = reinterpret_cast<float *>(sm + NS * STAGE);  // [NCH * 16 tokens][128 rows]
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + NS * STAGE + SMEM::TSBYTES);
     uint64_t *empty = full + NS;
     uint64_t *acc_full = empty + NS;       // [kGtBufs]
     uint64_t *acc_empty = acc_full + kGtBufs;  // [kGtBufs]
@@ -310,12 +328,14 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
         // ---- epilogue: thread = weight row 32*(warp%4) + lane of the tile ----
         // A warp whose wait runs out keeps walking the same pieces with the
         // work suppressed (`dead`), so the named barriers below still meet.
+        // Tokens are handled in chunks of 16 columns (nch of them).
         const int q = warp & 3;
         const int r = 32 * q + lane;
         const uint32_t lane_off = (uint32_t)(32 * q) << 16;
         const int B = a.B;
+        const int nch = min((B + kGtChunk - 1) / kGtChunk, SMEM::NCH);
         const int ep_tid = threadIdx.x - 64;  // 0..127
-        float seg_sum[kGtMaxB], tile_sum[kGtMaxB];
+        float seg_sum[kGtChunk], tile_sum[kGtChunk];
         int c = 0;
         bool dead = false;
         int64_t u = u0;
@@ -339,40 +359,54 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
                     continue;
                 }
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-                float d[NX];
-                tmem_ld_nx<NX>(tmem + lane_off + (uint32_t)(b * NX), d);
+                const uint32_t acc = tmem + lane_off + (uint32_t)(b * NX);
+#pragma unroll 1
+                for (int ch = 0; ch < nch; ++ch) {
+                    // tokens 16*ch + t: hi part in column 16*ch + t, lo part NX/2 further
+                    float pv[kGtChunk];
+                    gt_load_chunk<NX, SPLIT>(acc, ch, pv);
+                    if (local) {
+                        // every segment of a tile inside this CTA is one piece;
+                        // -0 is the additive identity, so segment 0 is stored unchanged
+                        float *tsp = ts + (kGtChunk * ch) * kGtRows + r;
+#pragma unroll
+                        for (int t = 0; t < kGtChunk; ++t)
+                            tsp[t * kGtRows] = (seg == 0 ? -0.f : tsp[t * kGtRows]) + pv[t];
+                        if (a.epi == GT_ROW_PARTIAL) {
+                            const int row = tile * kGtRows + r;
+                            if (row < a.N)
+#pragma unroll
+                                for (int t = 0; t < kGtChunk; ++t)
+                                    if (kGtChunk * ch + t < B)
+                                        a.partials[((int64_t)seg * B + kGtChunk * ch + t) * a.N + row] = pv[t];
+                        }
+                    } else {
+                        // float4 of tokens 4j..4j+3 of all 128 rows side by side:
+                        // a warp's stores cover 512 contiguous bytes
+                        float4 *dst = reinterpret_cast<float4 *>(a.gpart) +
+                                      ((((int64_t)cta * 2 + slot) * a.nseg + seg) * (a.gstride / 4) + 4 * ch) * kGtRows +
+                                      r;
+#pragma unroll
+                        for (int t = 0; t < kGtChunk; t += 4)
+                            if (kGtChunk * ch + t < B)
+                                dst[(t / 4) * kGtRows] = make_float4(pv[t], pv[t + 1], pv[t + 2], pv[t + 3]);
+                    }
+                }
                 asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&acc_empty[b]);
-                // token t: hi part in column t, lo part in column NX/2 + t
-                float pv[kGtMaxB];
-#pragma unroll
-                for (int t = 0; t < kGtMaxB; ++t) {
-                    if constexpr (SPLIT) pv[t] = t < NX / 2 ? d[t] + d[NX / 2 + t] : 0.f;
-                    else pv[t] = t < NX ? d[t] : 0.f;
-                }
-                if (local) {
-                    // every segment of a tile inside this CTA is one piece
-#pragma unroll
-                    for (int t = 0; t < kGtMaxB; ++t) tile_sum[t] = (seg == 0 ? -0.f : tile_sum[t]) + pv[t];
-                    if (a.epi == GT_ROW_PARTIAL) {
-                        const int row = tile * kGtRows + r;
-                        if (row < a.N)
-#pragma unroll
-                            for (int t = 0; t < kGtMaxB; ++t)
-                                if (t < B) a.partials[((int64_t)seg * B + t) * a.N + row] = pv[t];
-                    }
-                } else {
-                    float4 *dst = reinterpret_cast<float4 *>(
-                        a.gpart + ((((int64_t)cta * 2 + slot) * a.nseg + seg) * kGtRows + r) * kGtMaxB);
-#pragma unroll
-                    for (int t = 0; t < kGtMaxB; t += 4)
-                        if (t < B) dst[t / 4] = make_float4(pv[t], pv[t + 1], pv[t + 2], pv[t + 3]);
-                }
             }
             const int row = tile * kGtRows + r;
             if (local) {
-                if (!dead && a.epi != GT_ROW_PARTIAL) gt_final(a, row, tile_sum, lane);
+                if (!dead && a.epi != GT_ROW_PARTIAL) {
+#pragma unroll 1
+                    for (int ch = 0; ch < nch; ++ch) {
+                        const float *tsp = ts + (kGtChunk * ch) * kGtRows + r;
+#pragma unroll
+                        for (int t = 0; t < kGtChunk; ++t) tile_sum[t] = tsp[t * kGtRows];
+                        gt_final(a, row, tile_sum, lane, kGtChunk * ch);
+                    }
+                }
                 continue;
             }
             // shared tile: publish the pieces; the CTA completing the tile adds them
@@ -393,91 +427,107 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
             if (!*s_last) continue;
             __threadfence();
             // The tile's pieces in order (segment, then CTA), listed by one
-            // thread in shared memory in chunks, then loaded four at a time.
+            // thread in shared memory (in rounds of up to kGtList entries),
+            // then loaded eight at a time; the walk is repeated for each
+            // 16-token chunk, reusing the list when one round held it all.
             // Each CTA stored its part in slot 0 if the tile is its first,
             // else in slot 1.
+            bool single = false;  // the whole list is in shared memory
+#pragma unroll 1
+            for (int ch = 0; ch < nch; ++ch) {
+                const int tok0 = kGtChunk * ch;
 #pragma unroll
-            for (int t = 0; t < kGtMaxB; ++t) {
-                tile_sum[t] = -0.f;
-                seg_sum[t] = -0.f;
-            }
-            int g_s = 0, g_cc = 0;  // generator position (thread 0)
-            if (ep_tid == 0) {
-                int cf = (int)((t_beg * G) / a.U);
-                while (cf > 0 && gt_start(a.U, G, cf) > t_beg) --cf;
-                while (gt_start(a.U, G, cf + 1) <= t_beg) ++cf;
-                g_cc = cf;
-            }
-            for (;;) {
-                if (ep_tid == 0) {
-                    int n = 0;
-                    while (n < kGtList && g_s < a.nseg) {
-                        const int64_t sb = t_beg + (int64_t)g_s * a.kbs, se = sb + a.kbs;
-                        const int64_t c0 = gt_start(a.U, G, g_cc), c1 = gt_start(a.U, G, g_cc + 1);
-                        if (c1 > sb && c0 < se) {
-                            const int sl = (tile == (int)(c0 / per_tile)) ? 0 : 1;
-                            const bool seg_last = c1 >= se;
-                            s_list[n++] = (((g_cc * 2 + sl) * a.nseg + g_s) << 5) | (g_s << 1) | (seg_last ? 1 : 0);
-                        }
-                        if (c1 >= se) {
-                            ++g_s;  // next segment starts in this same CTA
-                        } else {
-                            ++g_cc;
-                        }
-                    }
-                    *s_nlist = n;
+                for (int t = 0; t < kGtChunk; ++t) {
+                    tile_sum[t] = -0.f;
+                    seg_sum[t] = -0.f;
                 }
-                asm volatile("bar.sync 1, 128;" ::: "memory");
-                const int n = *s_nlist;
-                for (int e0 = 0; e0 < n; e0 += 4) {
-                    float4 v[4][kGtMaxB / 4];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-#pragma unroll
-                        for (int q4 = 0; q4 < kGtMaxB / 4; ++q4) v[j][q4] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        if (e0 + j < n) {
-                            const int ent = s_list[e0 + j];
-                            const float4 *src = reinterpret_cast<const float4 *>(
-                                a.gpart + ((int64_t)(ent >> 5) * kGtRows + r) * kGtMaxB);
-#pragma unroll
-                            for (int q4 = 0; q4 < kGtMaxB / 4; ++q4)
-                                if (4 * q4 < B) v[j][q4] = __ldcg(src + q4);
-                        }
-                    }
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        if (e0 + j >= n) break;
-                        const int ent = s_list[e0 + j];
-#pragma unroll
-                        for (int q4 = 0; q4 < kGtMaxB / 4; ++q4) {
-                            seg_sum[4 * q4] = seg_sum[4 * q4] + v[j][q4].x;
-                            seg_sum[4 * q4 + 1] = seg_sum[4 * q4 + 1] + v[j][q4].y;
-                            seg_sum[4 * q4 + 2] = seg_sum[4 * q4 + 2] + v[j][q4].z;
-                            seg_sum[4 * q4 + 3] = seg_sum[4 * q4 + 3] + v[j][q4].w;
-                        }
-                        if (ent & 1) {  // the segment is complete
-                            const int sg = (ent >> 1) & 15;
-                            if (a.epi == GT_ROW_PARTIAL) {
-                                if (row < a.N)
-#pragma unroll
-                                    for (int t = 0; t < kGtMaxB; ++t)
-                                        if (t < B) a.partials[((int64_t)sg * B + t) * a.N + row] = seg_sum[t];
-                            } else {
-#pragma unroll
-                                for (int t = 0; t < kGtMaxB; ++t) tile_sum[t] = tile_sum[t] + seg_sum[t];
+                int g_s = 0, g_cc = 0;  // generator position (thread 0)
+                if (!single && ep_tid == 0) {
+                    int cf = (int)((t_beg * G) / a.U);
+                    while (cf > 0 && gt_start(a.U, G, cf) > t_beg) --cf;
+                    while (gt_start(a.U, G, cf + 1) <= t_beg) ++cf;
+                    g_cc = cf;
+                }
+                for (int round = 0;; ++round) {
+                    if (!single) {
+                        if (ep_tid == 0) {
+                            int n = 0;
+                            while (n < kGtList && g_s < a.nseg) {
+                                const int64_t sb = t_beg + (int64_t)g_s * a.kbs, se = sb + a.kbs;
+                                const int64_t c0 = gt_start(a.U, G, g_cc), c1 = gt_start(a.U, G, g_cc + 1);
+                                if (c1 > sb && c0 < se) {
+                                    const int sl = (tile == (int)(c0 / per_tile)) ? 0 : 1;
+                                    const bool seg_last = c1 >= se;
+                                    s_list[n++] =
+                                        (((g_cc * 2 + sl) * a.nseg + g_s) << 5) | (g_s << 1) | (seg_last ? 1 : 0);
+                                }
+                                if (c1 >= se) {
+                                    ++g_s;  // next segment starts in this same CTA
+                                } else {
+                                    ++g_cc;
+                                }
                             }
+                            *s_nlist = n;
+                            *s_more = g_s < a.nseg ? 1 : 0;
+                        }
+                        asm volatile("bar.sync 1, 128;" ::: "memory");
+                    }
+                    const int n = *s_nlist;
+                    for (int e0 = 0; e0 < n; e0 += 8) {
+                        float4 v[8][kGtChunk / 4];
 #pragma unroll
-                            for (int t = 0; t < kGtMaxB; ++t) seg_sum[t] = -0.f;
+                        for (int j = 0; j < 8; ++j)
+#pragma unroll
+                            for (int q4 = 0; q4 < kGtChunk / 4; ++q4) v[j][q4] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            if (e0 + j < n) {
+                                const int ent = s_list[e0 + j];
+                                const float4 *src = reinterpret_cast<const float4 *>(a.gpart) +
+                                                    ((int64_t)(ent >> 5) * (a.gstride / 4) + tok0 / 4) * kGtRows + r;
+#pragma unroll
+                                for (int q4 = 0; q4 < kGtChunk / 4; ++q4)
+                                    if (tok0 + 4 * q4 < B) v[j][q4] = __ldcg(src + q4 * kGtRows);
+                            }
+                        }
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            if (e0 + j >= n) break;
+                            const int ent = s_list[e0 + j];
+#pragma unroll
+                            for (int q4 = 0; q4 < kGtChunk / 4; ++q4) {
+                                seg_sum[4 * q4] = seg_sum[4 * q4] + v[j][q4].x;
+                                seg_sum[4 * q4 + 1] = seg_sum[4 * q4 + 1] + v[j][q4].y;
+                                seg_sum[4 * q4 + 2] = seg_sum[4 * q4 + 2] + v[j][q4].z;
+                                seg_sum[4 * q4 + 3] = seg_sum[4 * q4 + 3] + v[j][q4].w;
+                            }
+                            if (ent & 1) {  // the segment is complete
+                                const int sg = (ent >> 1) & 15;
+                                if (a.epi == GT_ROW_PARTIAL) {
+                                    if (row < a.N)
+#pragma unroll
+                                        for (int t = 0; t < kGtChunk; ++t)
+                                            if (tok0 + t < B)
+                                                a.partials[((int64_t)sg * B + tok0 + t) * a.N + row] = seg_sum[t];
+                                } else {
+#pragma unroll
+                                    for (int t = 0; t < kGtChunk; ++t) tile_sum[t] = tile_sum[t] + seg_sum[t];
+                                }
+#pragma unroll
+                                for (int t = 0; t < kGtChunk; ++t) seg_sum[t] = -0.f;
+                            }
                         }
                     }
+                    if (single) break;
+                    const bool more = *s_more != 0;
+                    asm volatile("bar.sync 1, 128;" ::: "memory");  // list consumed before it is rewritten
+                    if (!more) {
+                        single = round == 0;  // one round held the whole list: keep it
+                        break;
+                    }
                 }
-                if (ep_tid == 0) *s_more = g_s < a.nseg ? 1 : 0;
-                asm volatile("bar.sync 1, 128;" ::: "memory");  // list consumed; flag visible
-                if (!*s_more) break;
+                if (a.epi != GT_ROW_PARTIAL) gt_final(a, row, tile_sum, lane, tok0);
             }
-            if (a.epi != GT_ROW_PARTIAL) gt_final(a, row, tile_sum, lane);
         }
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");

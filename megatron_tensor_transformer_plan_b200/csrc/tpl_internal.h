@@ -23,10 +23,22 @@ constexpr int kAttnTargetWarps = 1024;     // key-range splits across all (b, kv
 constexpr int kAttnMinKeys = 128;          // keys per split at least (when there are that many)
 constexpr int kAttnMaxCtasPerPair = 64;
 constexpr int kAttnSmsBound = 256;         // upper bound on SMs when sizing workspaces
-constexpr int kTicketSlots = 4096;         // uint32 arrival counters at the workspace start
-constexpr int kTicketAttn = 0;             // [0, 1024): attention pairs
-constexpr int kTicketGemv = 1024;          // + 512 * op
-constexpr int kMaxPairs = 1024;
+constexpr int kTicketSlots = 10240;        // uint32 arrival counters at the workspace start
+constexpr int kTicketAttn = 0;             // [0, 8192): attention pairs
+constexpr int kTicketGemv = 8192;          // + 512 * op
+constexpr int kMaxPairs = 8192;
+constexpr int kMaxBatch = 64;              // decode tokens per call (tensor-core projections)
+constexpr int kMaxBatchCuda = 16;          // with the mma.sync / FFMA projections (fp32 plans)
+
+// Columns of the tensor-core decode projection's activation operand for B
+// tokens: B hi rows and B lo rows when the activation is split, else B rows,
+// rounded up to a valid MMA N (16, 32, 64, 128).
+inline int gt_nx(int B, bool split) {
+    const int rows = split ? 2 * B : B;
+    return rows <= 16 ? 16 : rows <= 32 ? 32 : rows <= 64 ? 64 : 128;
+}
+// Floats per row of a cross-CTA piece of that projection (whole 16-token chunks).
+inline int gt_stride(int B) { return 16 * ((B + 15) / 16); }
 constexpr int kMaxRowBlocks = 512;
 constexpr int kGemvTcMaxCtas = 256;        // CTAs of one tensor-core decode projection at most
 constexpr int kGemvTcMaxTiles = 512;       // 128-row tiles per projection (one arrival counter each)

@@ -105,6 +105,8 @@ void attn_geom(int B, int nkv, int64_t keys, AttnGeom *a) {
     ns = std::min<int64_t>(ns, (keys + kAttnMinKeys - 1) / kAttnMinKeys);
     ns = std::min<int64_t>(ns, (int64_t)kAttnMaxCtasPerPair * kAttnWarps);
     ns = std::max<int64_t>(ns, 1);
+    // whole CTAs of kAttnWarps splits, the keys spread over all of them
+    ns = (ns + kAttnWarps - 1) / kAttnWarps * kAttnWarps;
     int64_t kps = (keys + ns - 1) / ns;
     kps = (kps + 15) / 16 * 16;
     ns = (keys + kps - 1) / kps;
@@ -166,8 +168,8 @@ int ws_layout(const tpl_plan *p, int B, int64_t S, WsLayout *w) {
         gp = std::max(gp, gg.gp_floats);
     if (gemv_geom((int)H, p->t, p->F_s, B, xb, sms, &gg) == TPL_OK) gp = std::max(gp, gg.gp_floats);
     w->gp = take(gp * 4 + 4);
-    w->xs = take((size_t)32 * H * 2);  // [NX <= 32][hidden] bf16
-    w->gpart = take((size_t)kGemvTcMaxCtas * 2 * p->t * 128 * 16 * 4);
+    w->xs = take((size_t)gt_nx(B, true) * H * 2);  // [NX][hidden] bf16
+    w->gpart = take((size_t)kGemvTcMaxCtas * 2 * p->t * 128 * gt_stride(B) * 4);
     w->total = off;
     return TPL_OK;
 }

@@ -9,6 +9,8 @@ Workloads (seeded synthetic tensors):
   7b          hidden 4096, 32/32 heads, ffn 11008, KV 2048, B in {1, 16}, t in {1, 2, 4}
   70b         hidden 8192, 64/8 heads, ffn 28672, KV 8192, B=16, t in {1, 4, 8}
   70b-stack   one layer of the 80-layer stack: t=8, B=4, KV 4096
+  70b-batch   hidden 8192, 64/8 heads, ffn 28672, t=4, KV 2048, B in {1..64}
+              (above 16 tokens only the tensor-core projections apply)
 Working sets under four times the L2 size rotate over several copies of the
 weights and caches so that every timed call reads from HBM. Timing: CUDA
 events around each call after 3 warm-up calls, median reported.
@@ -110,11 +112,13 @@ def main() -> None:
     for t in (1, 4, 8):
         cases.append(("70b", dict(H=8192, nq=64, nkv=8, F=28672, t=t, B=16, S=8192)))
     cases.append(("70b-stack", dict(H=8192, nq=64, nkv=8, F=28672, t=8, B=4, S=4096)))
+    for B in (1, 4, 8, 16, 24, 32, 48, 64):
+        cases.append(("70b-batch", dict(H=8192, nq=64, nkv=8, F=28672, t=4, B=B, S=2048, only_fused=True)))
     for name, c in cases:
         if args.only and name != args.only:
             continue
         for mode in ("fused", "separate"):
-            if c["t"] == 1 and mode == "separate":
+            if (c["t"] == 1 or c.get("only_fused")) and mode == "separate":
                 continue
             flags = c.get("flags")
             if args.rope and not c.get("mlp_only", False):
@@ -123,10 +127,12 @@ def main() -> None:
                                                  args.iters, mode, flags, c.get("mlp_only", False),
                                                  args.gemv_mode)
             gbs = nbytes / (us * 1e-6) / 1e9
+            tok_s = c["B"] / (us * 1e-6)
             print(json.dumps({"workload": name, "gemv_mode": args.gemv_mode, "rope": args.rope, "t": c["t"],
                               "B": c["B"], "S": c["S"],
                               "reduce": mode,
-                              "us_per_layer": round(us, 2), "algorithmic_bytes": nbytes, "gb_s": round(gbs, 1),
+                              "us_per_layer": round(us, 2), "tokens_per_s_per_layer": round(tok_s, 1),
+                              "algorithmic_bytes": nbytes, "gb_s": round(gbs, 1),
                               "frac_of_peak": round(gbs / peak, 4), "peak_gb_s": peak, "peak_kind": kind,
                               "weight_copies_rotated": ncopies, "device_status": rc}), flush=True)
 

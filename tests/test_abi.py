@@ -145,9 +145,14 @@ def test_device_calls_validate_before_launch(tpl):
     # workspace too small
     assert tpl.tpl_decode_layer(H, fake, ctypes.byref(kv), fake, 1, 0, fake, None, fake, need - 1, 0, st) == \
         tpl.TPL_EWORKSPACE
-    # batch beyond what the decode kernels take
-    assert tpl.tpl_decode_layer(H, fake, ctypes.byref(kv), fake, 17, 0, fake, None, fake, 1 << 40, 0, st) == \
+    # batch beyond what the decode kernels take: 64 tokens (16 with fp32 weights)
+    assert tpl.tpl_decode_layer(H, fake, ctypes.byref(kv), fake, 65, 0, fake, None, fake, 1 << 40, 0, st) == \
         tpl.TPL_EUNSUPPORTED
+    assert tpl.tpl_decode_layer(H, fake, ctypes.byref(kv), fake, 17, 0, fake, None, fake, 1 << 40, 0, st) == \
+        tpl.TPL_ENOMEM  # supported; the cache holds one sequence
+    p32 = tpl.Plan(tpl.make_dims(256, 2, 2, 128, 688, 1, 1e-5, tpl.TPL_FP32_WEIGHTS), 2)
+    assert tpl.tpl_decode_layer(p32.handle, fake, ctypes.byref(kv), fake, 17, 0, fake, None, fake, 1 << 40, 0,
+                                st) == tpl.TPL_EUNSUPPORTED
     # KV capacity: S must be < seq_cap, B <= batch_cap
     assert tpl.tpl_decode_layer(H, fake, ctypes.byref(kv), fake, 1, 16, fake, None, fake, 1 << 40, 0, st) == \
         tpl.TPL_ENOMEM

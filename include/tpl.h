@@ -141,7 +141,7 @@ void tpl_plan_destroy(tpl_plan *plan);
  * a shared-memory ring and multiplied on the 5th-generation tensor cores
  * (tcgen05, accumulators in TMEM; the normalised activation is computed by a
  * small RMSNorm kernel), 4 = the default: the tcgen05 kernels for every
- * projection of layers with at least 1 GiB of weights when more than 8
+ * projection of layers with at least 1 GiB of weights when 8 or more
  * tokens are decoded, mma.sync otherwise (the choice that measured faster on
  * B200; layers mixing the two families measured slower than either).  fp32
  * plans always use FFMA.  TPL_OPT_PREFILL_ATTN selects the prefill attention kernel:

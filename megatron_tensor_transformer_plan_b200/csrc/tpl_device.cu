@@ -228,9 +228,9 @@ int gemv_tc_run(Ctx &c, GemvTcArgs &a, int op, bool split, const void *W, int64_
 // tcgen05 kernel streams large matrices closer to the copy bandwidth, but the
 // mma.sync kernel overlaps consecutive launches better (programmatic
 // dependent launch), and layers that mix the two families measured slower
-// than either.  So: tcgen05 with more than 8 tokens on layers of at least
-// 1 GiB of weights, mma.sync otherwise.  Beyond 16 tokens (any mode) only
-// the tcgen05 kernel applies.
+// than either.  So: tcgen05 from 8 tokens on layers of at least 1 GiB of
+// weights, mma.sync otherwise.  Beyond 16 tokens (any mode) only the tcgen05
+// kernel applies.
 bool use_tc(const tpl_plan *p, int op, int B) {
     (void)op;
     if (p->f32) return false;
@@ -240,7 +240,7 @@ bool use_tc(const tpl_plan *p, int op, int B) {
     const tpl_dims &d = p->d;
     const int64_t layer_params = (int64_t)(d.n_q_heads + 2 * d.n_kv_heads) * d.head_dim * d.hidden +
                                  (int64_t)d.hidden * d.n_q_heads * d.head_dim + 3 * (int64_t)d.ffn * d.hidden;
-    return B > 8 && layer_params * 2 >= (1ll << 30);
+    return B >= 8 && layer_params * 2 >= (1ll << 30);
 }
 
 GemvTcArgs gt_args(const tpl_plan *p) {

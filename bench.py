@@ -90,7 +90,8 @@ def prefill_flops(T=PREFILL_T):
 
 
 # the sources the decode gate/up kernel and its launch are built from
-DECODE_SOURCES = ("tpl_common.cuh", "tpl_device.cu", "tpl_gemv.cuh", "tpl_internal.h", "tpl_plan.cpp")
+DECODE_SOURCES = ("tpl_common.cuh", "tpl_device.cu", "tpl_gemm.cuh", "tpl_gemv.cuh", "tpl_gemv_tc.cuh",
+                  "tpl_internal.h", "tpl_norm.cuh", "tpl_plan.cpp", "tpl_tma.h")
 
 
 def kernel_source_hash():
@@ -359,6 +360,12 @@ def run_ours(args, ws, rank, local):
 
     peak, peak_kind = load_peaks()
     gu_gbs = gate_up_bytes_per_launch() / (gu_ms / 1e3) / 1e9
+    per_layer = plan.decode_kernel_count(BATCH)
+    if per_layer == 7:  # the tensor-core family: the gate/up step is two kernels
+        gu_kernel = ("gate/up step: norm_split_kernel (RMSNorm rows as bf16 hi + lo) + gemv_tc_kernel<16, true> "
+                     "(tcgen05 gate/up + SwiGLU); timed together, traffic of the GEMV kernel")
+    else:
+        gu_kernel = "gemv_kernel<3, false> (gate/up + SwiGLU, activation as bf16 hi+lo)"
     step_gbs = algorithmic_bytes_per_step() / (ms / 1e3) / 1e9
 
     if rank == 0:
@@ -368,13 +375,13 @@ def run_ours(args, ws, rank, local):
                 "config": dict(config_dict(), step_hbm_gbs=step_gbs, step_hbm_frac=step_gbs / peak,
                                algorithmic_bytes_per_step=algorithmic_bytes_per_step(),
                                reductions_counted=reductions // max(1, args.steps)),
-                "roofline": {"bound": "hbm", "kernel": "gemv_kernel<3, false> (gate/up + SwiGLU, activation as bf16 hi+lo)", "achieved": gu_gbs,
+                "roofline": {"bound": "hbm", "kernel": gu_kernel, "achieved": gu_gbs,
                              "peak": peak, "peak_kind": peak_kind + " (burst copy, kernel timed alone)",
                              "unit": "GB/s", "frac": gu_gbs / peak, "traffic": recorded_traffic(),
                              "algorithmic_bytes_per_launch": gate_up_bytes_per_launch(), "launch_ms": gu_ms},
                 "e2e": {"value": ws * BATCH / (e2e_ms / 1e3), "unit": "tokens/s",
                         "h2d_bytes_per_step": x.numel() * 2, "d2h_bytes_per_step": y.numel() * 2},
-                "gpu_launches": 5 * L * args.steps,
+                "gpu_launches": per_layer * L * args.steps,
                 "clocks": clk,
                 "prefill": {"workload": f"70B-shaped layer prefill, t={T_SHARDS}, {PREFILL_T} tokens, causal in chunk",
                             "ms_per_layer": pf_ms, "tokens_per_s": ws * PREFILL_T / (pf_ms / 1e3),

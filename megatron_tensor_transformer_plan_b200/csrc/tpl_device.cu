@@ -224,13 +224,12 @@ int gemv_tc_run(Ctx &c, GemvTcArgs &a, int op, bool split, const void *W, int64_
 }
 
 // TPL_OPT_GEMV_MODE 4 (the default for bf16 plans): one kernel family for all
-// four projections of a layer, the one that measured faster on B200.  The
-// tcgen05 kernel streams large matrices closer to the copy bandwidth, but the
-// mma.sync kernel overlaps consecutive launches better (programmatic
-// dependent launch), and layers that mix the two families measured slower
-// than either.  So: tcgen05 from 8 tokens on layers of at least 1 GiB of
-// weights, mma.sync otherwise.  Beyond 16 tokens (any mode) only the tcgen05
-// kernel applies.
+// four projections of a layer, the one that measured faster on B200 (layers
+// that mix the two families measured slower than either): tcgen05 from 4
+// tokens on layers of at least 1 GiB of weights and from 16 tokens on any
+// layer, mma.sync otherwise (one token, and small layers, where the tcgen05
+// kernel's fixed costs dominate).  Beyond 16 tokens (any mode) only the
+// tcgen05 kernel applies.
 bool use_tc(const tpl_plan *p, int op, int B) {
     (void)op;
     if (p->f32) return false;
@@ -240,7 +239,7 @@ bool use_tc(const tpl_plan *p, int op, int B) {
     const tpl_dims &d = p->d;
     const int64_t layer_params = (int64_t)(d.n_q_heads + 2 * d.n_kv_heads) * d.head_dim * d.hidden +
                                  (int64_t)d.hidden * d.n_q_heads * d.head_dim + 3 * (int64_t)d.ffn * d.hidden;
-    return B >= 8 && layer_params * 2 >= (1ll << 30);
+    return B >= kMaxBatchCuda || (B >= 4 && layer_params * 2 >= (1ll << 30));
 }
 
 GemvTcArgs gt_args(const tpl_plan *p) {
@@ -791,6 +790,18 @@ int tpl_prefill_chunk(tpl_plan *p, const void *packed, const tpl_kv *kv, const v
     if (ws_bytes < L.total) return TPL_EWORKSPACE;
     return prefill_layer(p, static_cast<const char *>(packed), kv, x, T, (int)start, y, y32, static_cast<char *>(ws),
                          L, reduce_mode, static_cast<cudaStream_t>(stream));
+}
+
+int tpl_decode_kernel_count(const tpl_plan *p, int32_t B, int32_t reduce_mode, int32_t *count) {
+    if (!p || !count || B < 1) return TPL_EINVAL;
+    if (reduce_mode != TPL_REDUCE_FUSED && reduce_mode != TPL_REDUCE_SEPARATE) return TPL_EINVAL;
+    if (B > (p->f32 ? kMaxBatchCuda : kMaxBatch)) return TPL_EUNSUPPORTED;
+    // projections, attention; the tcgen05 family adds two RMSNorm kernels
+    int n = use_tc(p, OP_QKV, B) ? 7 : 5;
+    if (p->rope) n += 1;
+    if (reduce_mode == TPL_REDUCE_SEPARATE) n += 2;
+    *count = n;
+    return TPL_OK;
 }
 
 int tpl_last_device_error(const tpl_plan *p, tpl_stream stream) {

@@ -124,3 +124,19 @@ def test_rope_flag_validation(tpl):
         assert e.value.code == tpl.TPL_EINVAL
     # without the flag the base is ignored
     tpl.Plan(tpl.make_dims(1024, 16, 4, 128, 2816, 1, 1e-5, tpl.TPL_NORM, rope_base=0.0), 4)
+
+
+def test_decode_kernel_count(tpl):
+    """Kernels per decode layer: five with the mma.sync projections, seven
+    with the tensor-core ones (two RMSNorm kernels), one more with the
+    rotation, two more with the separate reductions."""
+    p = tpl.Plan(tpl.make_dims(8192, 64, 8, 128, 28672, 80), 8)
+    assert [p.decode_kernel_count(b) for b in (1, 4, 16, 64)] == [5, 7, 7, 7]
+    assert p.decode_kernel_count(4, tpl.TPL_REDUCE_SEPARATE) == 9
+    p.set_option(tpl.TPL_OPT_GEMV_MODE, 0)
+    assert [p.decode_kernel_count(b) for b in (4, 16, 17)] == [5, 5, 7]
+    small = tpl.Plan(tpl.make_dims(4096, 32, 32, 128, 11008, 32, 1e-5,
+                                   tpl.TPL_NORM | tpl.TPL_RESIDUAL | tpl.TPL_ROPE), 4)
+    assert [small.decode_kernel_count(b) for b in (1, 8, 16)] == [6, 6, 8]
+    with pytest.raises(tpl.TplError):
+        p.decode_kernel_count(65)

@@ -360,10 +360,11 @@ def run_ours(args, ws, rank, local):
 
     peak, peak_kind = load_peaks()
     gu_gbs = gate_up_bytes_per_launch() / (gu_ms / 1e3) / 1e9
-    per_layer = plan.decode_kernel_count(BATCH)
-    if per_layer == 7:  # the tensor-core family: the gate/up step is two kernels
-        gu_kernel = ("gate/up step: norm_split_kernel (RMSNorm rows as bf16 hi + lo) + gemv_tc_kernel<16, true> "
-                     "(tcgen05 gate/up + SwiGLU); timed together, traffic of the GEMV kernel")
+    per_step = plan.decode_kernel_count(BATCH, n_layers=L)
+    if plan.decode_kernel_count(BATCH) == 6:  # the tensor-core family: the gate/up call is two kernels
+        gu_kernel = ("gate/up call: scale_split_kernel (h * gamma as bf16 hi + lo) + gemv_tc_kernel<16, true> "
+                     "(tcgen05 gate/up, 1/rms and SwiGLU in the epilogue); timed together, traffic of the GEMV "
+                     "kernel; inside the layer the O kernel writes that operand and no extra kernel runs")
     else:
         gu_kernel = "gemv_kernel<3, false> (gate/up + SwiGLU, activation as bf16 hi+lo)"
     step_gbs = algorithmic_bytes_per_step() / (ms / 1e3) / 1e9
@@ -381,7 +382,7 @@ def run_ours(args, ws, rank, local):
                              "algorithmic_bytes_per_launch": gate_up_bytes_per_launch(), "launch_ms": gu_ms},
                 "e2e": {"value": ws * BATCH / (e2e_ms / 1e3), "unit": "tokens/s",
                         "h2d_bytes_per_step": x.numel() * 2, "d2h_bytes_per_step": y.numel() * 2},
-                "gpu_launches": per_layer * L * args.steps,
+                "gpu_launches": per_step * args.steps,
                 "clocks": clk,
                 "prefill": {"workload": f"70B-shaped layer prefill, t={T_SHARDS}, {PREFILL_T} tokens, causal in chunk",
                             "ms_per_layer": pf_ms, "tokens_per_s": ws * PREFILL_T / (pf_ms / 1e3),

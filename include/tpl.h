@@ -411,11 +411,13 @@ int tpl_mlp_block(tpl_plan *plan, const void *packed, const void *x, int32_t B, 
 /* Reduction points launched through this plan since creation/reset. */
 int64_t tpl_reduction_count(const tpl_plan *plan);
 
-/* Host: the number of kernels one tpl_decode_layer call launches for B
- * tokens in the given reduce mode (the projections' kernel family, the
- * RMSNorm kernels that feed the tensor-core projections, the rotation, the
- * separate reductions).  tpl_decode_stack launches n_layers times as many. */
-int tpl_decode_kernel_count(const tpl_plan *plan, int32_t B, int32_t reduce_mode, int32_t *count);
+/* Host: the number of kernels a decode call launches for B tokens in the
+ * given reduce mode: tpl_decode_layer with n_layers = 1, tpl_decode_stack
+ * over n_layers layers (the projections' kernel family, the operand kernels
+ * of the tensor-core projections that the fused row-parallel kernels do not
+ * already cover, the rotation, the separate reductions). */
+int tpl_decode_kernel_count(const tpl_plan *plan, int32_t B, int32_t reduce_mode, int32_t n_layers,
+                            int32_t *count);
 void tpl_reset_counters(tpl_plan *plan);
 
 /* Synchronise `stream`, read and clear the device error word of the current

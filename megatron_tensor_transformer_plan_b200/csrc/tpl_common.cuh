@@ -73,6 +73,16 @@ __device__ __forceinline__ void store_act(void *p, int is_f32, int64_t i, float 
 
 __device__ __forceinline__ float silu(float z) { return z / (1.0f + expf(-z)); }
 
+// The operand of the tensor-core decode projections: a = v * gamma[i] (v
+// without gamma), as bf16 hi = rn(a) and lo = rn(a - hi).  Written with
+// explicit roundings so that every kernel producing it gives the same bits.
+__device__ __forceinline__ void split_scaled(float v, const float *gamma, int64_t i, __nv_bfloat16 &hi,
+                                             __nv_bfloat16 &lo) {
+    const float a = gamma ? __fmul_rn(v, gamma[i]) : v;
+    hi = __float2bfloat16_rn(a);
+    lo = __float2bfloat16_rn(__fsub_rn(a, __bfloat162float(hi)));
+}
+
 // cos and sin of the rotary angle pos * theta.  The angle is formed and
 // brought into [-pi, pi] in fp64 (positions of long sequences give angles of
 // thousands of radians, where fp32 would lose the low bits), then evaluated

@@ -45,9 +45,9 @@ namespace {
 // while the previous kernel on the stream drains; every kernel here waits
 // (griddepcontrol.wait) before touching data a previous kernel wrote.
 template <typename... KA, typename... A>
-cudaError_t launch_pdl(void (*kern)(KA...), int grid, int block, size_t smem, cudaStream_t st, A &&...args) {
+cudaError_t launch_pdl(void (*kern)(KA...), dim3 grid, int block, size_t smem, cudaStream_t st, A &&...args) {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
+    cfg.gridDim = grid;
     cfg.blockDim = dim3(block);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
@@ -99,6 +99,12 @@ struct Ctx {
     cudaStream_t st;
     int B;
     int64_t S;
+    // the tensor-core projections' operand (workspace xs) already holds the
+    // split x * gamma_attn of this layer's input (written by the previous
+    // layer's down projection), or h * gamma_mlp (written by O)
+    bool xs_holds_x = false, xs_holds_h = false;
+    const float *next_gamma = nullptr;  // gamma_attn of the next layer of a stack
+    bool has_next = false;
 };
 
 int make_ctx(tpl_plan *p, void *ws, size_t ws_bytes, int B, int64_t S, tpl_stream stream, Ctx *c) {
@@ -249,23 +255,37 @@ GemvTcArgs gt_args(const tpl_plan *p) {
     return a;
 }
 
-// RMSNorm (or a copy without TPL_NORM) of B rows into the workspace's
-// activation operand [NX][hidden]: bf16 hi rows 0..B-1, lo rows NX/2..NX/2+B-1,
-// zero rows elsewhere.
-int run_norm_rows(Ctx &c, const void *x, int x_f32, const float *gamma) {
+// The tensor-core projections' activation operand [NX][hidden] in the
+// workspace: x * gamma (x without TPL_NORM) as bf16 hi rows 0..B-1 and lo
+// rows NX/2..; the RMSNorm factor 1/rms is applied by the projection.
+int run_scale_split(Ctx &c, const void *x, int x_f32, const float *gamma) {
     tpl_plan *p = c.p;
     auto *xs = reinterpret_cast<__nv_bfloat16 *>(c.ws + c.L.xs);
     const int half = gt_nx(c.B, true) / 2;
-    const int norm = (p->d.flags & TPL_NORM) ? 1 : 0;
-    return cuda_rc(launch_pdl(norm_split_kernel, half, 256, 0, c.st, x, x_f32, gamma, p->d.rms_eps, norm,
-                              p->d.hidden, xs, xs + (int64_t)half * p->d.hidden, c.B));
+    const int H = p->d.hidden;
+    const dim3 grid((unsigned)((H / 8 + 255) / 256), (unsigned)c.B);
+    return cuda_rc(launch_pdl(scale_split_kernel, grid, 256, 0, c.st, x, x_f32,
+                              (p->d.flags & TPL_NORM) ? gamma : nullptr, H, xs, half));
+}
+
+// The folded RMSNorm of a column-parallel projection: 1/rms of src's rows.
+void set_rms(const tpl_plan *p, GemvTcArgs &a, const void *src, int src_f32) {
+    if (!(p->d.flags & TPL_NORM)) return;
+    a.rms_src = src;
+    a.rms_f32 = src_f32;
+    a.rms_len = p->d.hidden;
+    a.rms_eps = p->d.rms_eps;
 }
 
 int run_qkv_tc(Ctx &c, const char *packed, const tpl_kv *kv, const void *x, float *q, float *knew, float *vnew) {
     tpl_plan *p = c.p;
-    int rc = run_norm_rows(c, x, 0, reinterpret_cast<const float *>(packed + p->off_g1));
-    if (rc != TPL_OK) return rc;
+    if (!c.xs_holds_x) {
+        int rc = run_scale_split(c, x, 0, reinterpret_cast<const float *>(packed + p->off_g1));
+        if (rc != TPL_OK) return rc;
+    }
+    c.xs_holds_x = false;
     GemvTcArgs a = gt_args(p);
+    set_rms(p, a, x, 0);
     a.epi = GT_QKV;
     a.q = q;
     a.knew = knew;
@@ -286,9 +306,13 @@ int run_qkv_tc(Ctx &c, const char *packed, const tpl_kv *kv, const void *x, floa
 
 int run_gu_tc(Ctx &c, const char *packed, const void *h, int h_is_act, void *act) {
     tpl_plan *p = c.p;
-    int rc = run_norm_rows(c, h, h_is_act ? 0 : 1, reinterpret_cast<const float *>(packed + p->off_g2));
-    if (rc != TPL_OK) return rc;
+    if (!c.xs_holds_h) {
+        int rc = run_scale_split(c, h, h_is_act ? 0 : 1, reinterpret_cast<const float *>(packed + p->off_g2));
+        if (rc != TPL_OK) return rc;
+    }
+    c.xs_holds_h = false;
     GemvTcArgs a = gt_args(p);
+    set_rms(p, a, h, h_is_act ? 0 : 1);
     a.epi = GT_GU;
     a.out_act = act;
     const int64_t H = p->d.hidden;
@@ -297,8 +321,11 @@ int run_gu_tc(Ctx &c, const char *packed, const void *h, int h_is_act, void *act
 }
 
 // Row-parallel O (K slice of shard s: columns s*nq_s*d of o) or down (s*F_s of act).
+// With xs_gamma_or_mark set (fused mode inside a layer or a stack), the
+// epilogue also writes the next column-parallel projection's operand:
+// xs = split(out * gamma), gamma = xs_gamma (NULL without TPL_NORM).
 int run_row_tc(Ctx &c, const char *packed, int op, const void *x, const void *resid, int resid_f32, float *out32,
-               void *out_act, float *partials) {
+               void *out_act, float *partials, bool write_xs = false, const float *xs_gamma = nullptr) {
     tpl_plan *p = c.p;
     GemvTcArgs a = gt_args(p);
     if (partials) {
@@ -310,6 +337,11 @@ int run_row_tc(Ctx &c, const char *packed, int op, const void *x, const void *re
         a.resid_f32 = resid_f32;
         a.out32 = out32;
         a.out_act = out_act;
+        if (write_xs) {
+            a.xs_out = reinterpret_cast<__nv_bfloat16 *>(c.ws + c.L.xs);
+            a.xs_gamma = (p->d.flags & TPL_NORM) ? xs_gamma : nullptr;
+            a.xs_half = gt_nx(c.B, true) / 2;
+        }
     }
     const bool is_o = op == OP_O;
     const int64_t Ks = is_o ? (int64_t)p->nq_s * p->d.head_dim : p->F_s;
@@ -435,11 +467,17 @@ int run_attn(Ctx &c, const tpl_kv *kv, const float *q, const float *knew, const 
 }
 
 // Row-parallel O projection: fused (partials == NULL) or partial output.
-int run_o(Ctx &c, const char *packed, const void *o, const void *resid, float *h, float *partials) {
+// With `chain` (inside a layer, fused mode) the tensor-core kernel also
+// writes gate/up's operand h * gamma_mlp.
+int run_o(Ctx &c, const char *packed, const void *o, const void *resid, float *h, float *partials,
+          bool chain = false) {
     tpl_plan *p = c.p;
     if (use_tc(p, OP_O, c.B)) {
-        int rc = run_row_tc(c, packed, OP_O, o, resid, 0, h, nullptr, partials);
+        const bool wx = chain && !partials;
+        int rc = run_row_tc(c, packed, OP_O, o, resid, 0, h, nullptr, partials, wx,
+                            reinterpret_cast<const float *>(packed + p->off_g2));
         if (rc == TPL_OK && !partials) p->reductions.fetch_add(1);
+        if (rc == TPL_OK && wx) c.xs_holds_h = true;
         return rc;
     }
     GemvArgs a = base_args(p);
@@ -482,12 +520,16 @@ int run_gu(Ctx &c, const char *packed, const void *h, int h_is_act, void *act) {
     return gemv_launch(c, a, p->t * 2 * p->F_s, 1, p->d.hidden, OP_GU);
 }
 
+// With `chain` (a stack layer followed by another, fused mode) the
+// tensor-core kernel also writes the next layer's QKV operand y * gamma_attn.
 int run_down(Ctx &c, const char *packed, const void *act, const void *resid, int resid_f32, void *y, float *y32,
-             float *partials) {
+             float *partials, bool chain = false) {
     tpl_plan *p = c.p;
     if (use_tc(p, OP_DOWN, c.B)) {
-        int rc = run_row_tc(c, packed, OP_DOWN, act, resid, resid_f32, y32, y, partials);
+        const bool wx = chain && !partials && y && c.has_next;
+        int rc = run_row_tc(c, packed, OP_DOWN, act, resid, resid_f32, y32, y, partials, wx, c.next_gamma);
         if (rc == TPL_OK && !partials) p->reductions.fetch_add(1);
+        if (rc == TPL_OK && wx) c.xs_holds_x = true;
         return rc;
     }
     GemvArgs a = base_args(p);
@@ -538,7 +580,7 @@ int decode_layer(Ctx &c, const char *packed, const tpl_kv *kv, const void *x, vo
     if (rc == TPL_OK) rc = run_attn(c, kv, q, knew, vnew, o);
     if (rc == TPL_OK) {
         if (mode == TPL_REDUCE_FUSED) {
-            rc = run_o(c, packed, o, resid ? x : nullptr, h, nullptr);
+            rc = run_o(c, packed, o, resid ? x : nullptr, h, nullptr, true);
         } else {
             rc = run_o(c, packed, o, nullptr, nullptr, P);
             if (rc == TPL_OK) rc = run_reduce(p, c.st, P, resid ? x : nullptr, p->f32, c.B, h, nullptr);
@@ -547,7 +589,7 @@ int decode_layer(Ctx &c, const char *packed, const tpl_kv *kv, const void *x, vo
     if (rc == TPL_OK) rc = run_gu(c, packed, h, 0, act);
     if (rc == TPL_OK) {
         if (mode == TPL_REDUCE_FUSED) {
-            rc = run_down(c, packed, act, resid ? h : nullptr, 1, y, y32, nullptr);
+            rc = run_down(c, packed, act, resid ? h : nullptr, 1, y, y32, nullptr, true);
         } else {
             rc = run_down(c, packed, act, nullptr, 1, nullptr, nullptr, P);
             if (rc == TPL_OK) rc = run_reduce(p, c.st, P, resid ? h : nullptr, 1, c.B, y32, y);
@@ -758,6 +800,12 @@ int tpl_decode_stack(tpl_plan *p, const void *const *packed_per_layer, const tpl
     const void *cur = x;
     for (int l = 0; l < L; ++l) {
         const bool last = l == L - 1;
+        // the down projection of a layer followed by another writes that
+        // layer's QKV operand
+        c.has_next = !last;
+        c.next_gamma = last ? nullptr
+                            : reinterpret_cast<const float *>(static_cast<const char *>(packed_per_layer[l + 1]) +
+                                                              p->off_g1);
         void *out = last ? y : buf[l & 1];
         float *out32 = last ? y32 : nullptr;
         if (last && !y) out = buf[l & 1];
@@ -792,15 +840,22 @@ int tpl_prefill_chunk(tpl_plan *p, const void *packed, const tpl_kv *kv, const v
                          L, reduce_mode, static_cast<cudaStream_t>(stream));
 }
 
-int tpl_decode_kernel_count(const tpl_plan *p, int32_t B, int32_t reduce_mode, int32_t *count) {
-    if (!p || !count || B < 1) return TPL_EINVAL;
+int tpl_decode_kernel_count(const tpl_plan *p, int32_t B, int32_t reduce_mode, int32_t n_layers, int32_t *count) {
+    if (!p || !count || B < 1 || n_layers < 1) return TPL_EINVAL;
     if (reduce_mode != TPL_REDUCE_FUSED && reduce_mode != TPL_REDUCE_SEPARATE) return TPL_EINVAL;
     if (B > (p->f32 ? kMaxBatchCuda : kMaxBatch)) return TPL_EUNSUPPORTED;
-    // projections, attention; the tcgen05 family adds two RMSNorm kernels
-    int n = use_tc(p, OP_QKV, B) ? 7 : 5;
-    if (p->rope) n += 1;
-    if (reduce_mode == TPL_REDUCE_SEPARATE) n += 2;
-    *count = n;
+    const bool sep = reduce_mode == TPL_REDUCE_SEPARATE;
+    int64_t n;
+    if (use_tc(p, OP_QKV, B)) {
+        // QKV, attention, O, gate/up, down; the operand kernel before QKV and
+        // gate/up unless the fused O and the previous layer's down wrote it
+        n = sep ? 9ll * n_layers : 5ll * n_layers + 1;
+    } else {
+        n = (sep ? 7ll : 5ll) * n_layers;
+    }
+    if (p->rope) n += n_layers;
+    if (n > 0x7fffffff) return TPL_EINVAL;
+    *count = (int32_t)n;
     return TPL_OK;
 }
 

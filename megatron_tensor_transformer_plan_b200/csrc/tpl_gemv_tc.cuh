@@ -48,6 +48,7 @@ constexpr int kGtMaxB = 64;       // tokens per call
 constexpr int kGtChunk = 16;      // tokens per epilogue chunk
 constexpr int kGtList = 120;      // piece list entries per combine chunk
 constexpr int kGtBarBytes = 1024;  // mbarriers, flags and the piece list after the stage ring
+constexpr int kGtRmsBytes = 2048;  // per-warp sums of squares and 1/rms per token
 
 // Shared memory: the stage ring, the running tile sums of tiles finished
 // inside one CTA ([tokens][128 rows] fp32), then the barrier area.  The ring
@@ -63,7 +64,7 @@ struct GemvTcSmem {
     static constexpr int NCH = TOK < kGtChunk ? 1 : TOK / kGtChunk;
     static constexpr int TSBYTES = NCH * kGtChunk * kGtRows * 4;
     static constexpr int NS = (160 * 1024 - TSBYTES) / STAGE;
-    static constexpr int BYTES = NS * STAGE + TSBYTES + 1024 + kGtBarBytes;
+    static constexpr int BYTES = NS * STAGE + TSBYTES + 1024 + kGtBarBytes + kGtRmsBytes;
     static_assert(BYTES <= 232448, "shared memory per block");
 };
 
@@ -91,6 +92,17 @@ struct GemvTcArgs {
     __nv_bfloat16 *kc, *vc;
     int rps, nq, nq_s, nkv_s, hd, batch_cap;
     int64_t S, seq_cap;
+    // RMSNorm folded in: the activation operand is x * gamma (split_scaled)
+    // and the column-op results are multiplied by 1/sqrt(mean(src^2) + eps)
+    // per token, computed here from src [B][rms_len] (fp32 or bf16)
+    const void *rms_src;
+    int rms_f32, rms_len;
+    float rms_eps;
+    // GT_ROW: also write the next projection's operand from the output
+    // (out_act rounded when present): xs_out rows b (hi) and xs_half + b (lo)
+    __nv_bfloat16 *xs_out;
+    const float *xs_gamma;
+    int xs_half;
     // cross-CTA pieces and arrival counters
     float *gpart;       // [G][2][nseg][gstride / 4][128] float4: token quads outer, rows inner
     int gstride;        // floats per row of a piece: 16 * ceil(B / 16)
@@ -122,9 +134,13 @@ __device__ __forceinline__ int64_t gt_start(int64_t U, int G, int c) { return U 
 
 // Final write of one output row for tokens tok0 .. tok0+15 (fused sums or
 // column ops).
-__device__ __forceinline__ void gt_final(const GemvTcArgs &a, int row, const float (&v)[kGtChunk], int lane,
-                                         int tok0) {
+__device__ __forceinline__ void gt_final(const GemvTcArgs &a, int row, const float (&v0)[kGtChunk], int lane,
+                                         int tok0, const float *inv_rms) {
     const int B = a.B;
+    float v[kGtChunk];
+#pragma unroll
+    for (int i = 0; i < kGtChunk; ++i)  // the RMSNorm factor of column ops (1 without it)
+        v[i] = (a.rms_src && a.epi != GT_ROW) ? v0[i] * inv_rms[min(tok0 + i, kGtMaxB - 1)] : v0[i];
     if (a.epi == GT_GU) {
         // rows interleave gate and up: the even lane pairs with its odd neighbour
 #pragma unroll
@@ -171,6 +187,13 @@ __device__ __forceinline__ void gt_final(const GemvTcArgs &a, int row, const flo
         if (a.resid) o = load_act(a.resid, a.resid_f32, i) + o;
         if (a.out32) a.out32[i] = o;
         if (a.out_act) static_cast<__nv_bfloat16 *>(a.out_act)[i] = __float2bfloat16_rn(o);
+        if (a.xs_out) {
+            const float src = a.out_act ? __bfloat162float(__float2bfloat16_rn(o)) : o;
+            __nv_bfloat16 hi, lo;
+            split_scaled(src, a.xs_gamma, row, hi, lo);
+            a.xs_out[i] = hi;
+            a.xs_out[(int64_t)(a.xs_half + b) * a.N + row] = lo;
+        }
     }
 }
 
@@ -187,6 +210,9 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
     unsigned char *sm = reinterpret_cast<unsigned char *>(((uintptr_t)gv_raw + 1023) & ~(uintptr_t)1023);
     float *ts = reinterpret_cast<float *>(sm + NS * STAGE);  // [NCH * 16 tokens][128 rows]
     uint64_t *full = reinterpret_cast<uint64_t *>(sm + NS * STAGE + SMEM::TSBYTES);
+    float *s_rpart = reinterpret_cast<float *>(sm + NS * STAGE + SMEM::TSBYTES + kGtBarBytes);  // [4][kGtMaxB]
+    float *s_inv = s_rpart + 4 * kGtMaxB;                                                       // [kGtMaxB]
+    static_assert(5 * kGtMaxB * 4 <= kGtRmsBytes, "rms area");
     uint64_t *empty = full + NS;
     uint64_t *acc_full = empty + NS;       // [kGtBufs]
     uint64_t *acc_empty = acc_full + kGtBufs;  // [kGtBufs]
@@ -339,6 +365,46 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
         const int B = a.B;
         const int nch = min((B + kGtChunk - 1) / kGtChunk, SMEM::NCH);
         const int ep_tid = threadIdx.x - 64;  // 0..127
+        if (a.rms_src) {
+            // 1/rms per token while the first weight tiles stream in: each
+            // warp sums the squares of a strided quarter of the row, the four
+            // quarters are added in a fixed order
+            const int n8 = a.rms_len / 8;
+            for (int b = 0; b < B; ++b) {
+                float ss = 0.f;
+                for (int c8 = ep_tid; c8 < n8; c8 += 128) {
+                    float v[8];
+                    if (a.rms_f32) {
+                        const float4 *p4 = reinterpret_cast<const float4 *>(static_cast<const float *>(a.rms_src) +
+                                                                            (int64_t)b * a.rms_len + 8 * c8);
+                        const float4 u0 = p4[0], u1 = p4[1];
+                        v[0] = u0.x; v[1] = u0.y; v[2] = u0.z; v[3] = u0.w;
+                        v[4] = u1.x; v[5] = u1.y; v[6] = u1.z; v[7] = u1.w;
+                    } else {
+                        const uint4 u = *reinterpret_cast<const uint4 *>(
+                            static_cast<const __nv_bfloat16 *>(a.rms_src) + (int64_t)b * a.rms_len + 8 * c8);
+                        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            v[2 * e] = bf16lo(w4[e]);
+                            v[2 * e + 1] = bf16hi(w4[e]);
+                        }
+                    }
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) ss = fmaf(v[e], v[e], ss);
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+                if (lane == 0) s_rpart[(ep_tid >> 5) * kGtMaxB + b] = ss;
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (ep_tid < B) {
+                const float tot = ((s_rpart[ep_tid] + s_rpart[kGtMaxB + ep_tid]) + s_rpart[2 * kGtMaxB + ep_tid]) +
+                                  s_rpart[3 * kGtMaxB + ep_tid];
+                s_inv[ep_tid] = 1.0f / sqrtf(tot / (float)a.rms_len + a.rms_eps);
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+        }
         float seg_sum[kGtChunk], tile_sum[kGtChunk];
         int c = 0;
         bool dead = false;
@@ -408,7 +474,7 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
                         const float *tsp = ts + (kGtChunk * ch) * kGtRows + r;
 #pragma unroll
                         for (int t = 0; t < kGtChunk; ++t) tile_sum[t] = tsp[t * kGtRows];
-                        gt_final(a, row, tile_sum, lane, kGtChunk * ch);
+                        gt_final(a, row, tile_sum, lane, kGtChunk * ch, s_inv);
                     }
                 }
                 continue;
@@ -530,7 +596,7 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
                         break;
                     }
                 }
-                if (a.epi != GT_ROW_PARTIAL) gt_final(a, row, tile_sum, lane, tok0);
+                if (a.epi != GT_ROW_PARTIAL) gt_final(a, row, tile_sum, lane, tok0, s_inv);
             }
         }
     }

@@ -79,4 +79,36 @@ __global__ void __launch_bounds__(256) norm_split_kernel(const void *x, int x_f3
     }
 }
 
+// The decode projections' operand without the RMSNorm factor: rows 0..B-1 of
+// x * gamma (gamma NULL: x) as bf16 hi rows and lo rows `half` rows further
+// (split_scaled); the tensor-core projection multiplies its results by
+// 1/rms itself.  grid (ceil(H / 2048), B), 256 threads x 8 elements.
+__global__ void __launch_bounds__(256) scale_split_kernel(const void *x, int x_f32, const float *gamma, int H,
+                                                          __nv_bfloat16 *xs, int half) {
+    pdl_wait();
+    pdl_trigger();
+    const int64_t row = blockIdx.y;
+    const int c = blockIdx.x * 256 + threadIdx.x;
+    if (8 * c >= H) return;
+    float v[8];
+    if (x_f32) {
+        const float4 *p = reinterpret_cast<const float4 *>(static_cast<const float *>(x) + row * H + 8 * c);
+        const float4 u0 = p[0], u1 = p[1];
+        v[0] = u0.x; v[1] = u0.y; v[2] = u0.z; v[3] = u0.w; v[4] = u1.x; v[5] = u1.y; v[6] = u1.z; v[7] = u1.w;
+    } else {
+        const uint4 u = *reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(x) + row * H + 8 * c);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            v[2 * e] = bf16lo(w[e]);
+            v[2 * e + 1] = bf16hi(w[e]);
+        }
+    }
+    __align__(16) __nv_bfloat16 h8[8], l8[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) split_scaled(v[e], gamma, 8 * c + e, h8[e], l8[e]);
+    *reinterpret_cast<uint4 *>(xs + row * H + 8 * c) = *reinterpret_cast<const uint4 *>(h8);
+    *reinterpret_cast<uint4 *>(xs + (row + half) * H + 8 * c) = *reinterpret_cast<const uint4 *>(l8);
+}
+
 }  // namespace tpl

@@ -114,7 +114,7 @@ _sig("tpl_reduce_partials", ctypes.c_int, _plan_p, c_void_p, c_void_p, c_int32, 
 _sig("tpl_mlp_block", ctypes.c_int, _plan_p, c_void_p, c_void_p, c_int32, c_void_p, c_void_p, c_void_p, c_size_t,
      c_int32, c_void_p)
 _sig("tpl_reduction_count", c_int64, _plan_p)
-_sig("tpl_decode_kernel_count", ctypes.c_int, _plan_p, c_int32, c_int32, P(c_int32))
+_sig("tpl_decode_kernel_count", ctypes.c_int, _plan_p, c_int32, c_int32, c_int32, P(c_int32))
 _sig("tpl_reset_counters", None, _plan_p)
 _sig("tpl_last_device_error", ctypes.c_int, _plan_p, c_void_p)
 _sig("tpl_status_string", ctypes.c_char_p, ctypes.c_int)
@@ -245,10 +245,10 @@ class Plan:
     def reduction_count(self) -> int:
         return tpl_reduction_count(self.handle)
 
-    def decode_kernel_count(self, B: int, mode=TPL_REDUCE_FUSED) -> int:
-        """Kernels one decode_layer call launches for B tokens."""
+    def decode_kernel_count(self, B: int, mode=TPL_REDUCE_FUSED, n_layers: int = 1) -> int:
+        """Kernels a decode call launches for B tokens (n_layers > 1: a stack)."""
         n = c_int32(0)
-        check(tpl_decode_kernel_count(self.handle, B, mode, ctypes.byref(n)), "tpl_decode_kernel_count")
+        check(tpl_decode_kernel_count(self.handle, B, mode, n_layers, ctypes.byref(n)), "tpl_decode_kernel_count")
         return int(n.value)
 
     def reset_counters(self) -> None:

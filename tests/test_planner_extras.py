@@ -127,16 +127,22 @@ def test_rope_flag_validation(tpl):
 
 
 def test_decode_kernel_count(tpl):
-    """Kernels per decode layer: five with the mma.sync projections, seven
-    with the tensor-core ones (two RMSNorm kernels), one more with the
-    rotation, two more with the separate reductions."""
+    """Kernels per decode call: five per layer with the mma.sync projections;
+    with the tensor-core ones the operand kernel before QKV once per call
+    (the fused O and down write the others), 9 per layer in separate mode;
+    one more per layer with the rotation."""
     p = tpl.Plan(tpl.make_dims(8192, 64, 8, 128, 28672, 80), 8)
-    assert [p.decode_kernel_count(b) for b in (1, 4, 16, 64)] == [5, 7, 7, 7]
+    assert [p.decode_kernel_count(b) for b in (1, 4, 16, 64)] == [5, 6, 6, 6]
+    assert p.decode_kernel_count(4, n_layers=80) == 401
+    assert p.decode_kernel_count(1, n_layers=80) == 400
     assert p.decode_kernel_count(4, tpl.TPL_REDUCE_SEPARATE) == 9
+    assert p.decode_kernel_count(4, tpl.TPL_REDUCE_SEPARATE, n_layers=80) == 720
     p.set_option(tpl.TPL_OPT_GEMV_MODE, 0)
-    assert [p.decode_kernel_count(b) for b in (4, 16, 17)] == [5, 5, 7]
+    assert [p.decode_kernel_count(b) for b in (4, 16, 17)] == [5, 5, 6]
+    assert p.decode_kernel_count(4, tpl.TPL_REDUCE_SEPARATE) == 7
     small = tpl.Plan(tpl.make_dims(4096, 32, 32, 128, 11008, 32, 1e-5,
                                    tpl.TPL_NORM | tpl.TPL_RESIDUAL | tpl.TPL_ROPE), 4)
-    assert [small.decode_kernel_count(b) for b in (1, 8, 16)] == [6, 6, 8]
+    assert [small.decode_kernel_count(b) for b in (1, 8, 16)] == [6, 6, 7]
+    assert small.decode_kernel_count(16, n_layers=32) == 5 * 32 + 1 + 32
     with pytest.raises(tpl.TplError):
         p.decode_kernel_count(65)

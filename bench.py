@@ -23,6 +23,7 @@ import ctypes
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -94,13 +95,21 @@ DECODE_SOURCES = ("tpl_common.cuh", "tpl_device.cu", "tpl_gemm.cuh", "tpl_gemv.c
                   "tpl_internal.h", "tpl_norm.cuh", "tpl_plan.cpp", "tpl_tma.h")
 
 
+def _code_only(text: str) -> str:
+    """Source text without comments and with whitespace collapsed, so that a
+    change to comments alone keeps the recorded capture valid."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "megatron_tensor_transformer_plan_b200", "csrc")
     for name in DECODE_SOURCES:
-        with open(os.path.join(csrc, name), "rb") as f:
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
             h.update(name.encode())
-            h.update(f.read())
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -139,8 +139,9 @@ void tpl_plan_destroy(tpl_plan *plan);
  * decode projections: 0 = register-streamed weights on mma.sync, 2 = FFMA on
  * the CUDA cores (kept to measure against), 3 = weights streamed by TMA into
  * a shared-memory ring and multiplied on the 5th-generation tensor cores
- * (tcgen05, accumulators in TMEM; the normalised activation is computed by a
- * small RMSNorm kernel), 4 = the default: the tcgen05 kernels for every
+ * (tcgen05, accumulators in TMEM; their operand is x * gamma as bf16 hi + lo,
+ * written by the preceding row-parallel kernel inside a layer or by a small
+ * kernel, and the RMSNorm factor 1/rms is applied to their results), 4 = the default: the tcgen05 kernels for every
  * projection of layers with at least 1 GiB of weights when 8 or more
  * tokens are decoded, mma.sync otherwise (the choice that measured faster on
  * B200; layers mixing the two families measured slower than either).  fp32

@@ -101,7 +101,7 @@ void attn_geom_staged(int B, int nkv, int64_t keys, int sms, AttnGeom *a);
 
 struct WsLayout {
     size_t tickets, q, o, h, act, ybuf0, ybuf1, P, knew, vnew, part_o, part_ml, gp;
-    size_t xs;     // normalised activation as bf16 hi + lo rows [2B][hidden] (tcgen05 projections)
+    size_t xs;     // tcgen05 projections' operand x * gamma as bf16 hi rows, then lo rows [NX][hidden]
     size_t gpart;  // cross-CTA pieces of the tcgen05 projections
     size_t total;
 };

@@ -191,3 +191,36 @@ def test_gemv_option(tpl):
         plan.set_option(tpl.TPL_OPT_GEMV_MODE, 5)
     with pytest.raises(tpl.TplError):
         plan.set_option(99, 0)
+
+
+def test_prefill_chunk_validates_before_launch(tpl):
+    """tpl_prefill_chunk's host checks: the chunk must fit the cache after its
+    start position, the start must not be negative, fp32 plans are not
+    supported, T = 0 does nothing."""
+    plan = tpl.Plan(tpl.make_dims(256, 2, 2, 128, 688), 2)
+    H = plan.handle
+    fake = 1 << 20
+    T = 16
+    need = plan.prefill_workspace_size(T)
+    kv = tpl.tpl_kv(fake, fake, 1, 40)
+    args = lambda start, kvp=kv, ws_bytes=need, mode=0: (H, fake, ctypes.byref(kvp), fake, T, start, fake, None, fake,
+                                                          ws_bytes, mode, None)
+    assert tpl.tpl_prefill_chunk(*args(25)) == tpl.TPL_ENOMEM   # 25 + 16 > 40
+    assert tpl.tpl_prefill_chunk(*args(-1)) == tpl.TPL_EINVAL
+    assert tpl.tpl_prefill_chunk(*args(0, ws_bytes=need - 1)) == tpl.TPL_EWORKSPACE
+    assert tpl.tpl_prefill_chunk(*args(0, mode=5)) == tpl.TPL_EINVAL
+    assert tpl.tpl_prefill_chunk(H, fake, ctypes.byref(kv), fake, 0, 3, fake, None, fake, need, 0, None) == tpl.TPL_OK
+    p32 = tpl.Plan(tpl.make_dims(256, 2, 2, 128, 688, 1, 1e-5, tpl.TPL_FP32_WEIGHTS), 2)
+    assert tpl.tpl_prefill_chunk(p32.handle, fake, ctypes.byref(kv), fake, T, 0, fake, None, fake, need, 0,
+                                 None) == tpl.TPL_EUNSUPPORTED
+
+
+def test_rope_plan_workspace_and_maps_unchanged(tpl):
+    """The rotation changes no layout: maps, packed size and workspace are
+    those of the plan without it."""
+    a = tpl.Plan(tpl.make_dims(1024, 16, 4, 128, 2816), 4)
+    b = tpl.Plan(tpl.make_dims(1024, 16, 4, 128, 2816, 1, 1e-5, tpl.TPL_NORM | tpl.TPL_RESIDUAL | tpl.TPL_ROPE), 4)
+    assert a.info().packed_layer_bytes == b.info().packed_layer_bytes
+    for B, S in ((1, 0), (16, 4096), (64, 100)):
+        assert a.workspace_size(B, S) == b.workspace_size(B, S)
+    assert a.prefill_workspace_size(300) == b.prefill_workspace_size(300)

@@ -2,10 +2,14 @@
 //
 // D[128 weight rows][NX columns] = W[128][K] . X[NX][K]^T in TMEM, where X
 // holds the B tokens' activation rows (bf16; with SPLIT, hi parts in rows
-// 0..B-1 and lo parts in rows NX/2..NX/2+B-1, the rest zero; NX = 16..128).
+// 0..B-1 and lo parts in rows NX/2..NX/2+B-1, other rows unused; NX =
+// 16..128).  For the column-parallel projections X is x * gamma and the
+// RMSNorm factor 1/rms is computed by the epilogue warps while the weights
+// stream and applied to the results; the row-parallel ones can also write the
+// next projection's X from their output.
 // The kernel is bound by streaming the weights from HBM: TMA brings 128-row x
 // 64-column weight tiles (16 KB, 128-byte swizzle) and the matching activation
-// tile into a 3-8 stage shared-memory ring, one thread issues four M=128,
+// tile into a 4-8 stage shared-memory ring, one thread issues four M=128,
 // N=NX, K=16 tcgen05.mma per stage, and the tensor pipe idles most of the
 // time.  192 threads: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer,
 // warps 2-5 epilogue (one TMEM lane = one weight row each), which walks the
@@ -13,13 +17,16 @@
 //
 // Work division ("stream-K"): the k-blocks of every (row tile, segment) are
 // laid end to end, tile-major then segment then k, and each CTA takes one
-// contiguous range, so every SM streams the same number of weight bytes.
+// contiguous range, so every SM streams the same number of weight bytes.  A
+// CTA walks its range in the order of gt_order: the parts of its first and
+// last tiles (shared with the neighbouring CTAs) before the tiles in between.
 // A run of k-blocks of one (tile, segment) inside a CTA is one MMA chain (a
 // "piece").  Segments are the row-parallel shards ("Tensor parallel scaling
 // curves", "What tensor parallelism actually splits"); column-parallel
 // projections have one.  Order of the sums, fixed for a given SM count:
 //   segment sum = pieces in k order;  tile sum = segment sums in shard order.
-// A tile whose k-blocks all lie in one CTA is finished in registers.  A tile
+// A tile whose k-blocks all lie in one CTA is finished in the CTA (running
+// sums in shared memory).  A tile
 // split across CTAs has each CTA store its pieces to the workspace and add its
 // k-block count to the tile's arrival counter; the CTA that completes the
 // count adds all pieces in the fixed order (no CTA waits for another) and

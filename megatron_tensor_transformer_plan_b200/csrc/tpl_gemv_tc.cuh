@@ -50,7 +50,7 @@ constexpr int kGtThreads = 192;
 constexpr int kGtRows = 128;     // weight rows per tile (MMA M)
 constexpr int kGtK = 64;         // columns per k-block
 constexpr int kGtWBytes = kGtRows * kGtK * 2;  // 16 KB
-constexpr int kGtBufs = 4;       // TMEM accumulators in flight
+constexpr int kGtBufsMax = 8;    // TMEM accumulators in flight, at most
 constexpr int kGtMaxB = 64;       // tokens per call
 constexpr int kGtChunk = 16;      // tokens per epilogue chunk
 constexpr int kGtList = 120;      // piece list entries per combine chunk
@@ -71,6 +71,9 @@ struct GemvTcSmem {
     static constexpr int NCH = TOK < kGtChunk ? 1 : TOK / kGtChunk;
     static constexpr int TSBYTES = NCH * kGtChunk * kGtRows * 4;
     static constexpr int NS = (160 * 1024 - TSBYTES) / STAGE;
+    // accumulators in flight: as many as TMEM's 512 columns hold, up to 8 (they
+    // let the weight stream run on while the epilogue adds split tiles)
+    static constexpr int BUFS = 512 / NX < kGtBufsMax ? 512 / NX : kGtBufsMax;
     static constexpr int BYTES = NS * STAGE + TSBYTES + 1024 + kGtBarBytes + kGtRmsBytes;
     static_assert(BYTES <= 232448, "shared memory per block");
 };
@@ -230,10 +233,11 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
     using SMEM = GemvTcSmem<NX, SPLIT>;
     constexpr int STAGE = SMEM::STAGE;
     constexpr int NS = SMEM::NS;
-    static_assert(2 * NS * 8 + 2 * kGtBufs * 8 + 8 + 4 + 32 + 4 * kGtList <= kGtBarBytes, "barrier area");
-    constexpr int TMEM_COLS = kGtBufs * NX <= 32 ? 32 : kGtBufs * NX <= 64 ? 64 : kGtBufs * NX <= 128 ? 128
-                              : kGtBufs * NX <= 256 ? 256 : 512;
-    static_assert(kGtBufs * NX <= 512, "accumulators");
+    constexpr int BUFS = SMEM::BUFS;
+    static_assert(2 * NS * 8 + 2 * BUFS * 8 + 8 + 4 + 32 + 4 * kGtList <= kGtBarBytes, "barrier area");
+    constexpr int TMEM_COLS = BUFS * NX <= 32 ? 32 : BUFS * NX <= 64 ? 64 : BUFS * NX <= 128 ? 128
+                              : BUFS * NX <= 256 ? 256 : 512;
+    static_assert(BUFS * NX <= 512, "accumulators");
     extern __shared__ __align__(1024) unsigned char gv_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(((uintptr_t)gv_raw + 1023) & ~(uintptr_t)1023);
     float *ts = reinterpret_cast<float *>(sm + NS * STAGE);  // [NCH * 16 tokens][128 rows]
@@ -242,9 +246,9 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
     float *s_inv = s_rpart + 4 * kGtMaxB;                                                       // [kGtMaxB]
     static_assert(5 * kGtMaxB * 4 <= kGtRmsBytes, "rms area");
     uint64_t *empty = full + NS;
-    uint64_t *acc_full = empty + NS;       // [kGtBufs]
-    uint64_t *acc_empty = acc_full + kGtBufs;  // [kGtBufs]
-    uint64_t *fin = acc_empty + kGtBufs;
+    uint64_t *acc_full = empty + NS;        // [BUFS]
+    uint64_t *acc_empty = acc_full + BUFS;  // [BUFS]
+    uint64_t *fin = acc_empty + BUFS;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(fin + 1);
     volatile int *s_fail = reinterpret_cast<volatile int *>(tmem_slot + 1);
     int *s_issued = const_cast<int *>(s_fail) + 1;
@@ -264,7 +268,7 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        for (int b = 0; b < kGtBufs; ++b) {
+        for (int b = 0; b < BUFS; ++b) {
             mbar_init(&acc_full[b], 1);
             mbar_init(&acc_empty[b], 4);
         }
@@ -366,8 +370,8 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
                 // one piece: the run of k-blocks of one (tile, segment)
                 const int64_t seg_end = (u / a.kbs + 1) * a.kbs;  // segments are kbs-aligned in u
                 const int64_t pe = min(ord.e(sr), seg_end);
-                const int b = c % kGtBufs;
-                const unsigned use = (unsigned)(c / kGtBufs);
+                const int b = c % BUFS;
+                const unsigned use = (unsigned)(c / BUFS);
                 if (*s_fail || !mbar_wait(&acc_empty[b], (use & 1u) ^ 1u)) {
                     ok = false;
                     break;
@@ -463,12 +467,12 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
             while (u < stop) {
                 const int seg = (int)((u % per_tile) / a.kbs);
                 const int64_t pe = min(stop, (u / a.kbs + 1) * a.kbs);
-                const int b = c % kGtBufs;
+                const int b = c % BUFS;
                 ++c;
                 u = pe;
                 if (!dead)
                     dead = !__all_sync(0xffffffffu,
-                                       !*s_fail && mbar_wait(&acc_full[b], (unsigned)((c - 1) / kGtBufs) & 1u));
+                                       !*s_fail && mbar_wait(&acc_full[b], (unsigned)((c - 1) / BUFS) & 1u));
                 if (dead) {
                     *s_fail = 1;
                     continue;

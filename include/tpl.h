@@ -182,8 +182,10 @@ int64_t tpl_kv_bytes(const tpl_dims *dims, int32_t t, int64_t batch, int64_t seq
 
 /* Per-GPU bytes at degree t of the n_layers layers' weights (each shard's
  * slices, bytes_per_elem per parameter) plus the KV cache of tpl_kv_bytes:
- * the footprint that the shard degree divides.  -1 on invalid input or when
- * t does not divide n_q_heads, n_kv_heads and ffn. */
+ * the two footprints "Tensor Parallelism Fundamentals" (section "Memory
+ * Overhead and Communication Bottlenecks") divides by t.  Embeddings and
+ * activations are not counted.  Host only.  -1 on invalid input or when t
+ * does not divide n_q_heads, n_kv_heads and ffn. */
 int64_t tpl_footprint_bytes(const tpl_dims *dims, int32_t t, int64_t batch, int64_t seq,
                             int32_t bytes_per_elem);
 

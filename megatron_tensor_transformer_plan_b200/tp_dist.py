@@ -1,0 +1,217 @@
+"""Tensor parallelism across t GPUs, one rank per GPU: each rank holds one
+shard's weights and KV cache and runs the single-device library's step kernels
+on its slice, and the two row-parallel partial sums of a layer are added by an
+all-reduce over torch.distributed (NCCL) instead of the on-device fused sum
+("Tensor parallel scaling curves", section "What tensor parallelism actually
+splits": Q/K/V and gate/up split by columns so that rank r owns heads
+[r*h_per_gpu, (r+1)*h_per_gpu), O and down split by rows, two all-reduces per
+layer; "Tensor Parallelism Fundamentals", section "Mechanics of Matrix
+Slicing").
+
+Per rank and layer, for the B tokens of a decode step:
+
+    q, k, v   = column-parallel QKV of RMSNorm(x) for the rank's heads   (tpl_qkv)
+    o         = attention over the rank's heads and its cache shard      (tpl_attn_decode)
+    P         = o Wo[:, rank's columns]^T, a full-size partial           (tpl_o_proj, partials)
+    P         = all_reduce(P)                                            (NCCL)
+    h         = x + P                                                    (tpl_reduce_partials)
+    act       = SwiGLU of RMSNorm(h) for the rank's ffn columns          (tpl_gate_up)
+    P2        = act Wd[:, rank's columns]^T                              (tpl_down_proj, partials)
+    P2        = all_reduce(P2)
+    y         = h + P2                                                   (tpl_reduce_partials)
+
+Each rank's local plan is a one-shard plan of the sliced dimensions (hidden,
+n_q/t heads, n_kv/t kv heads, ffn/t), so every kernel is the one the
+single-device layer runs.  The all-reduce adds the partials in NCCL's order,
+so results match the single-device layer within fp32 rounding, not bit for
+bit.  The step order is the same on every rank, so the collectives match.
+
+`DecodeStepOps` is the set of per-rank steps; `CudaOps` runs them through the
+C ABI.  Tests drive the same orchestration with other implementations of the
+steps on the CPU.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+
+@dataclass(frozen=True)
+class ShardSpec:
+    """Rank `rank` of `t`: the q heads, kv heads and ffn columns it owns."""
+    hidden: int
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    ffn: int
+    t: int
+    rank: int
+
+    def __post_init__(self):
+        if self.t < 1 or not 0 <= self.rank < self.t:
+            raise ValueError("rank must be in [0, t)")
+        if self.n_q_heads % self.t or self.n_kv_heads % self.t or self.ffn % self.t:
+            raise ValueError("t must divide the q heads, the kv heads and ffn")
+        if self.n_q_heads % self.n_kv_heads:
+            raise ValueError("n_kv_heads must divide n_q_heads")
+
+    @property
+    def nq_s(self) -> int:
+        return self.n_q_heads // self.t
+
+    @property
+    def nkv_s(self) -> int:
+        return self.n_kv_heads // self.t
+
+    @property
+    def ffn_s(self) -> int:
+        return self.ffn // self.t
+
+    def q_heads(self) -> range:
+        return range(self.rank * self.nq_s, (self.rank + 1) * self.nq_s)
+
+    def kv_heads(self) -> range:
+        return range(self.rank * self.nkv_s, (self.rank + 1) * self.nkv_s)
+
+    def ffn_cols(self) -> range:
+        return range(self.rank * self.ffn_s, (self.rank + 1) * self.ffn_s)
+
+
+def shard_weights(w: dict, spec: ShardSpec) -> dict:
+    """The rank's slices of one layer's weights (nn.Linear orientation
+    W[out][in]; numpy arrays or torch tensors): rows of Wq, Wk, Wv for its
+    heads, columns of Wo for its q heads, rows of Wg and Wu for its ffn
+    columns, columns of Wd; the RMSNorm gains whole (every rank normalises the
+    full hidden vector)."""
+    d = spec.head_dim
+    q0, q1 = spec.q_heads().start * d, spec.q_heads().stop * d
+    k0, k1 = spec.kv_heads().start * d, spec.kv_heads().stop * d
+    f0, f1 = spec.ffn_cols().start, spec.ffn_cols().stop
+    out = {
+        "wq": w["wq"][q0:q1],
+        "wk": w["wk"][k0:k1],
+        "wv": w["wv"][k0:k1],
+        "wo": w["wo"][:, q0:q1],
+        "wg": w["wg"][f0:f1],
+        "wu": w["wu"][f0:f1],
+        "wd": w["wd"][:, f0:f1],
+    }
+    for k in ("gamma_attn", "gamma_mlp"):
+        if w.get(k) is not None:
+            out[k] = w[k]
+    return out
+
+
+def shard_cache(cache, spec: ShardSpec):
+    """The rank's kv heads of an unsharded cache [B][n_kv][S_cap][d]."""
+    return cache[:, spec.kv_heads().start:spec.kv_heads().stop]
+
+
+class DecodeStepOps:
+    """The per-rank steps of one decode layer; arrays are whatever the
+    implementation uses (device tensors for CudaOps)."""
+
+    def qkv(self, x, S):  # -> (q, k_new, v_new) of the rank's heads
+        raise NotImplementedError
+
+    def attn(self, q, k_new, v_new, S):  # -> o [B][nq_s*d]
+        raise NotImplementedError
+
+    def o_partial(self, o):  # -> P [B][H] fp32 (no residual)
+        raise NotImplementedError
+
+    def add_resid(self, P, resid, resid_is_f32):  # -> resid + P, fp32
+        raise NotImplementedError
+
+    def gate_up(self, h):  # -> act [B][ffn_s]
+        raise NotImplementedError
+
+    def down_partial(self, act):  # -> P2 [B][H] fp32
+        raise NotImplementedError
+
+    def add_resid_out(self, P, h):  # -> (y32, y) = h + P
+        raise NotImplementedError
+
+
+def decode_layer_tp(ops: DecodeStepOps, x, S: int, all_reduce, residual: bool = True):
+    """One tensor-parallel decode layer on this rank: the steps in the same
+    order on every rank, with `all_reduce(tensor)` summing a partial in place
+    across the t ranks (torch.distributed.all_reduce for the NCCL group)."""
+    q, kn, vn = ops.qkv(x, S)
+    o = ops.attn(q, kn, vn, S)
+    P = ops.o_partial(o)
+    all_reduce(P)                                   # reduction point 1
+    h = ops.add_resid(P, x if residual else None, False)
+    act = ops.gate_up(h)
+    P2 = ops.down_partial(act)
+    all_reduce(P2)                                  # reduction point 2
+    return ops.add_resid_out(P2, h if residual else None)
+
+
+class CudaOps(DecodeStepOps):
+    """The steps through the C ABI on the rank's GPU: a one-shard plan of the
+    sliced dimensions, the rank's packed weights and KV cache shard."""
+
+    def __init__(self, spec: ShardSpec, weights_local: dict, k_local, v_local, batch: int, seq_cap: int,
+                 rms_eps: float = 1e-5, flags=None, rope_base: float = 500000.0):
+        import torch
+
+        from megatron_tensor_transformer_plan_b200 import tpl
+        self.tpl, self.torch = tpl, torch
+        flags = (tpl.TPL_NORM | tpl.TPL_RESIDUAL) if flags is None else flags
+        self.dims = tpl.make_dims(spec.hidden, spec.nq_s, spec.nkv_s, spec.head_dim, spec.ffn_s, 1, rms_eps, flags,
+                                  rope_base)
+        self.plan = tpl.Plan(self.dims, 1)
+        self.spec = spec
+        # column slices of Wo and Wd are strided views: the library takes dense rows
+        self.packed = self.plan.pack_layer({k: v.contiguous() for k, v in weights_local.items()})
+        self.k, self.v = self.plan.pack_kv(k_local.contiguous()), self.plan.pack_kv(v_local.contiguous())
+        self.kv = tpl.Plan.kv(self.k, self.v, batch, seq_cap)
+        self.B = batch
+        self.dev = self.packed.device
+
+    def _ws(self, S):
+        if getattr(self, "_ws_S", None) != S:
+            self.ws = self.plan.workspace(self.B, S, device=self.dev)
+            self._ws_S = S
+        return self.ws
+
+    def qkv(self, x, S):
+        t = self.torch
+        sp = self.spec
+        q = t.empty((self.B, sp.nq_s, sp.head_dim), dtype=t.float32, device=self.dev)
+        kn = t.empty((self.B, sp.nkv_s, sp.head_dim), dtype=t.float32, device=self.dev)
+        vn = t.empty_like(kn)
+        self.plan.qkv(self.packed, self.kv, x, S, q, self._ws(S), kn, vn)
+        return q, kn, vn
+
+    def attn(self, q, kn, vn, S):
+        o = self.torch.empty((self.B, self.spec.nq_s * self.spec.head_dim), dtype=self.plan.act_dtype,
+                             device=self.dev)
+        self.plan.attn_decode(self.kv, q, S, o, self._ws(S), kn, vn)
+        return o
+
+    def o_partial(self, o):
+        P = self.torch.empty((1, self.B, self.spec.hidden), dtype=self.torch.float32, device=self.dev)
+        self.plan.o_proj(self.packed, o, None, partials=P, ws=self.ws)
+        return P
+
+    def add_resid(self, P, resid, resid_is_f32):
+        h = self.torch.empty((self.B, self.spec.hidden), dtype=self.torch.float32, device=self.dev)
+        self.plan.reduce_partials(P, resid, resid_is_f32, out32=h)
+        return h
+
+    def gate_up(self, h):
+        act = self.torch.empty((self.B, self.spec.ffn_s), dtype=self.plan.act_dtype, device=self.dev)
+        self.plan.gate_up(self.packed, h, act, self.ws)
+        return act
+
+    def down_partial(self, act):
+        P = self.torch.empty((1, self.B, self.spec.hidden), dtype=self.torch.float32, device=self.dev)
+        self.plan.down_proj(self.packed, act, None, partials=P, ws=self.ws)
+        return P
+
+    def add_resid_out(self, P, h):
+        y32 = self.torch.empty((self.B, self.spec.hidden), dtype=self.torch.float32, device=self.dev)
+        y = self.torch.empty((self.B, self.spec.hidden), dtype=self.plan.act_dtype, device=self.dev)
+        self.plan.reduce_partials(P, h, True, out32=y32, out_act=y)
+        return y32, y

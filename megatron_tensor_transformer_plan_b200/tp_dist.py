@@ -147,6 +147,19 @@ def decode_layer_tp(ops: DecodeStepOps, x, S: int, all_reduce, residual: bool = 
     return ops.add_resid_out(P2, h if residual else None)
 
 
+def decode_stack_tp(ops_per_layer, x, S: int, all_reduce, residual: bool = True):
+    """n_layers tensor-parallel decode layers on this rank: layer l reads
+    layer l-1's output (the replicated y, in the activation type), 2 *
+    n_layers all-reduces per step ("Tensor parallel scaling curves": 2L per
+    forward pass).  Returns the last layer's (y32, y)."""
+    out = None
+    cur = x
+    for ops in ops_per_layer:
+        out = decode_layer_tp(ops, cur, S, all_reduce, residual)
+        cur = out[1]
+    return out
+
+
 class CudaOps(DecodeStepOps):
     """The steps through the C ABI on the rank's GPU: a one-shard plan of the
     sliced dimensions, the rank's packed weights and KV cache shard."""

@@ -15,8 +15,8 @@ import torch.distributed as dist
 import torch.multiprocessing as mp
 
 import oracle
-from megatron_tensor_transformer_plan_b200.tp_dist import (DecodeStepOps, ShardSpec, decode_layer_tp, shard_cache,
-                                                            shard_weights)
+from megatron_tensor_transformer_plan_b200.tp_dist import (DecodeStepOps, ShardSpec, decode_layer_tp,
+                                                            decode_stack_tp, shard_cache, shard_weights)
 
 H, NQ, NKV, D, F, B, S = 64, 8, 4, 16, 48, 2, 5
 EPS = 1e-5
@@ -159,3 +159,49 @@ def test_shard_spec_rejects_bad_degrees():
         ShardSpec(H, NQ, NKV, D, F, 2, 2)
     with pytest.raises(ValueError):
         ShardSpec(H, NQ, 3, D, F, 1, 0)
+
+
+def _stack_worker(rank, t, port, q):
+    import datetime
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=t, timeout=datetime.timedelta(seconds=60))
+    try:
+        spec = ShardSpec(H, NQ, NKV, D, F, t, rank)
+        ops = []
+        for layer in range(3):
+            w, _, kc, vc = _inputs(seed=100 + layer)
+            ops.append(NumpyOps(spec, shard_weights(w, spec), shard_cache(kc, spec), shard_cache(vc, spec)))
+        count = [0]
+
+        def ar(T):
+            count[0] += 1
+            dist.all_reduce(T, op=dist.ReduceOp.SUM)
+        _, x, _, _ = _inputs(seed=7)
+        y32, _ = decode_stack_tp(ops, x, S, ar)
+        q.put((rank, y32, count[0]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_tp_stack_over_gloo_matches_a_sequence_of_oracle_layers():
+    """Three layers, two ranks: 2L = 6 all-reduces, and the output of the
+    oracle's layers applied in sequence."""
+    t = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_stack_worker, args=(r, t, port, q)) for r in range(t)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+    res = {r: (y, n) for r, y, n in (q.get(timeout=5) for _ in range(t))}
+    _, cur, _, _ = _inputs(seed=7)
+    for layer in range(3):
+        w, _, kc, vc = _inputs(seed=100 + layer)
+        cur = oracle.decode_layer(oracle.Dims(H, NQ, NKV, D, F, eps=EPS), w, cur, kc, vc, S)
+    for r in range(t):
+        y, n = res[r]
+        assert n == 6
+        np.testing.assert_allclose(y, cur, rtol=1e-9, atol=1e-9 * np.abs(cur).max())

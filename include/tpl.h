@@ -6,10 +6,10 @@
  * Inside, the layer is computed the tensor-parallel way:
  *   - Q/K/V and gate/up projections are split by output columns into t
  *     shards, Q/K/V by whole attention heads ("Tensor parallel scaling
- *     curves", section "What tensor parallelism actually splits"; the
- *     ownership rule heads[rank*h_per_gpu:(rank+1)*h_per_gpu]);
+ *     curves", section "What tensor parallelism actually splits"; shard s
+ *     owns the contiguous query heads [s*n_q/t, (s+1)*n_q/t));
  *   - each shard attends over its own heads only, with no exchange (same
- *     section, "local attention on owned heads");
+ *     section);
  *   - the O and down projections are split by input rows, so each shard
  *     yields a full-size partial sum, and the t partials are added -- the
  *     arithmetic of the all-reduce, two per layer, 2L per forward pass (same
@@ -343,7 +343,8 @@ int tpl_qkv(tpl_plan *plan, const void *packed, const tpl_kv *kv, const void *x,
             tpl_stream stream);
 
 /* Owned-head GQA decode attention over positions 0..S ("Tensor parallel
- * scaling curves": local attention on owned heads).  The S cached keys are
+ * scaling curves", "What tensor parallelism actually splits": each shard
+ * attends over the heads it owns, with no exchange).  The S cached keys are
  * split over key ranges whose partial results are combined in a fixed
  * order; the new token (position S) is taken from k_new/v_new [B][n_kv][d]
  * fp32 when given (both or neither), else from cache slot S.  o [B][n_q*d]
@@ -360,13 +361,16 @@ int tpl_attn_decode(tpl_plan *plan, const tpl_kv *kv, const float *q, const floa
  * partials and arrival counters live in one array of fixed size,
  * TPL_ATTN_STATIC_SCRATCH_BYTES, held in the library's static device memory
  * on every device that loads the library, until the process exits.
- *   - Same arguments and result as tpl_attn_decode, minus the workspace.
+ *   - Same arguments as tpl_attn_decode, minus the workspace.  It runs the
+ *     kernel and split geometry tpl_attn_decode chooses for the same plan,
+ *     options and sizes, so the two give identical bits.
  *   - Returns TPL_ENOMEM, before launching anything, when the problem needs
  *     more scratch than that: the 256-byte-rounded sum of 4*pairs
  *     (counters), 8*pairs*n*g and 512*pairs*n*g bytes, pairs = B*n_kv, n the
- *     blocks per pair (a quarter of the key-range split count, which is
- *     about 1024/pairs rounded up to a multiple of 4, with at least 128 keys
- *     per split).
+ *     CTAs per pair of that geometry (the register-streamed kernel: about
+ *     1024/pairs key-range splits, at least 128 keys each, four per CTA; the
+ *     staged kernel: at most floor(SMs/pairs)).  The 70B shapes need about
+ *     1 MB.
  *   - The first call on a device looks up the array's device address (with
  *     that device current); make that first call before any stream capture.
  *   - Every call uses the same array, and it keeps the previous call's

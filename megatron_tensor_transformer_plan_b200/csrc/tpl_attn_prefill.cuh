@@ -1,5 +1,5 @@
 // Causal GQA attention of a prefill chunk ("Tensor parallel scaling curves",
-// "Prefill vs decode: different curves"; attention on owned heads, "What
+// "Prefill vs decode: different curves"; each shard attends over its own heads, "What
 // tensor parallelism actually splits"): token i attends keys 0..i of the
 // chunk.  One CTA per (kv head, 16-token row tile, chunk of the head's query
 // group); warp w handles one query head of the chunk for those 16 tokens, so

@@ -1,6 +1,6 @@
 // Causal GQA attention of a prefill chunk on the 5th-generation tensor cores
 // ("Tensor parallel scaling curves", "Prefill vs decode: different curves";
-// attention on owned heads, "What tensor parallelism actually splits"):
+// each shard attends over its own heads, "What tensor parallelism actually splits"):
 // the chunk's token i sits at position p0 + i and attends keys 0..p0 + i of
 // the cache (slots below p0 were written by earlier chunks; their low parts
 // are zero, read as the fill value of the remainder planes' negative

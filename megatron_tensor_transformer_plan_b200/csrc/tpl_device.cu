@@ -415,19 +415,25 @@ int run_qkv(Ctx &c, const char *packed, const tpl_kv *kv, const void *x, float *
 
 bool g_stg_attr[64];
 
-int run_attn(Ctx &c, const tpl_kv *kv, const float *q, const float *knew, const float *vnew, void *o) {
-    tpl_plan *p = c.p;
-    const int64_t keys = knew ? c.S : c.S + 1;
+// Which decode attention kernel runs and its split geometry: the staged
+// kernel for groups of at most 8 heads with at least two CTAs per pair in one
+// wave (where it measured faster; with one CTA per pair the register-streamed
+// kernel's finer splits win), else the register-streamed kernel.
+int attn_select(const tpl_plan *p, int B, int64_t keys, AttnGeom *g, bool *staged) {
     const int sms = num_sms_current();
     if (sms <= 0) return TPL_ECUDA;
-    AttnGeom g;
-    // staged kernel: groups of at most 8 heads with at least two CTAs per pair
-    // in one wave (where it measured faster; with one CTA per pair the
-    // register-streamed kernel's finer splits win)
-    const bool staged = p->attn_decode_mode == 0 && p->g <= 8 && 2 * c.B * p->d.n_kv_heads <= sms;
-    if (staged) attn_geom_staged(c.B, p->d.n_kv_heads, keys, sms, &g);
-    else attn_geom(c.B, p->d.n_kv_heads, keys, &g);
-    if (g.pairs > kMaxPairs) return TPL_EUNSUPPORTED;
+    *staged = p->attn_decode_mode == 0 && p->g <= 8 && 2 * B * p->d.n_kv_heads <= sms;
+    if (*staged) attn_geom_staged(B, p->d.n_kv_heads, keys, sms, g);
+    else attn_geom(B, p->d.n_kv_heads, keys, g);
+    if (g->pairs > kMaxPairs) return TPL_EUNSUPPORTED;
+    return TPL_OK;
+}
+
+// Fill the launch arguments (everything except the scratch pointers) and
+// launch the kernel attn_select chose.
+int attn_launch(const tpl_plan *p, const tpl_kv *kv, const float *q, const float *knew, const float *vnew, int B,
+                int64_t keys, void *o, const AttnGeom &g, bool staged, unsigned *tickets, float *part_ml,
+                float *part_o, cudaStream_t st) {
     AttnArgs a;
     std::memset(&a, 0, sizeof(a));
     a.q = q;
@@ -435,7 +441,7 @@ int run_attn(Ctx &c, const tpl_kv *kv, const float *q, const float *knew, const 
     a.vc = static_cast<const __nv_bfloat16 *>(kv->v);
     a.seq_cap = kv->seq_cap;
     a.batch_cap = kv->batch_cap;
-    a.B = c.B;
+    a.B = B;
     a.nq = p->d.n_q_heads;
     a.nkv_s = p->nkv_s;
     a.g = p->g;
@@ -445,9 +451,9 @@ int run_attn(Ctx &c, const tpl_kv *kv, const float *q, const float *knew, const 
     a.nsplit = g.nsplit;
     a.kps = g.kps;
     a.scale_log2 = 1.4426950408889634f / sqrtf((float)p->d.head_dim);
-    a.part_o = reinterpret_cast<float *>(c.ws + c.L.part_o);
-    a.part_ml = reinterpret_cast<float *>(c.ws + c.L.part_ml);
-    a.tickets = reinterpret_cast<unsigned *>(c.ws + c.L.tickets) + kTicketAttn;
+    a.part_o = part_o;
+    a.part_ml = part_ml;
+    a.tickets = tickets;
     a.o = o;
     a.o_f32 = p->f32;
     const int grid = g.pairs * (g.nsplit / kAttnWarps);
@@ -460,10 +466,23 @@ int run_attn(Ctx &c, const tpl_kv *kv, const float *q, const float *knew, const 
                 return TPL_ECUDA;
             g_stg_attr[dev] = true;
         }
-        return cuda_rc(launch_pdl(attn_decode_staged_kernel, grid, kAttnWarps * 32, kStgSmem, c.st, a));
+        return cuda_rc(launch_pdl(attn_decode_staged_kernel, grid, kAttnWarps * 32, kStgSmem, st, a));
     }
-    return cuda_rc(p->g <= 8 ? launch_pdl(attn_decode_kernel<true>, grid, kAttnWarps * 32, 0, c.st, a)
-                              : launch_pdl(attn_decode_kernel<false>, grid, kAttnWarps * 32, 0, c.st, a));
+    return cuda_rc(p->g <= 8 ? launch_pdl(attn_decode_kernel<true>, grid, kAttnWarps * 32, 0, st, a)
+                              : launch_pdl(attn_decode_kernel<false>, grid, kAttnWarps * 32, 0, st, a));
+}
+
+int run_attn(Ctx &c, const tpl_kv *kv, const float *q, const float *knew, const float *vnew, void *o) {
+    tpl_plan *p = c.p;
+    const int64_t keys = knew ? c.S : c.S + 1;
+    AttnGeom g;
+    bool staged = false;
+    int rc = attn_select(p, c.B, keys, &g, &staged);
+    if (rc != TPL_OK) return rc;
+    return attn_launch(p, kv, q, knew, vnew, c.B, keys, o, g, staged,
+                       reinterpret_cast<unsigned *>(c.ws + c.L.tickets) + kTicketAttn,
+                       reinterpret_cast<float *>(c.ws + c.L.part_ml), reinterpret_cast<float *>(c.ws + c.L.part_o),
+                       c.st);
 }
 
 // Row-parallel O projection: fused (partials == NULL) or partial output.
@@ -901,9 +920,11 @@ extern "C" int tpl_attn_decode_static(tpl_plan *p, const tpl_kv *kv, const float
     int rc = check_kv(kv, B, S);
     if (rc != TPL_OK) return rc;
     const int64_t keys = k_new ? S : S + 1;
+    // the same kernel and split geometry tpl_attn_decode chooses, so the two
+    // calls give identical bits
     AttnGeom g;
-    attn_geom(B, p->d.n_kv_heads, keys, &g);
-    if (g.pairs > kMaxPairs) return TPL_EUNSUPPORTED;
+    bool staged = false;
+    if ((rc = attn_select(p, B, keys, &g, &staged)) != TPL_OK) return rc;
     const size_t off_ml = round256((size_t)g.pairs * sizeof(unsigned));
     const size_t cpp = (size_t)g.nsplit / kAttnWarps;  // partials are per CTA
     const size_t off_o = off_ml + round256((size_t)g.pairs * cpp * p->g * 2 * sizeof(float));
@@ -922,29 +943,6 @@ extern "C" int tpl_attn_decode_static(tpl_plan *p, const tpl_kv *kv, const float
     char *scratch = static_cast<char *>(base);
     // The arrival counters must start at zero.
     if (cudaMemsetAsync(scratch, 0, (size_t)g.pairs * sizeof(unsigned), st) != cudaSuccess) return TPL_ECUDA;
-    AttnArgs a;
-    std::memset(&a, 0, sizeof(a));
-    a.q = q;
-    a.kc = static_cast<const __nv_bfloat16 *>(kv->k);
-    a.vc = static_cast<const __nv_bfloat16 *>(kv->v);
-    a.seq_cap = kv->seq_cap;
-    a.batch_cap = kv->batch_cap;
-    a.B = B;
-    a.nq = p->d.n_q_heads;
-    a.nkv_s = p->nkv_s;
-    a.g = p->g;
-    a.keys = keys;
-    a.k_new = k_new;
-    a.v_new = v_new;
-    a.nsplit = g.nsplit;
-    a.kps = g.kps;
-    a.scale_log2 = 1.4426950408889634f / sqrtf((float)p->d.head_dim);
-    a.tickets = reinterpret_cast<unsigned *>(scratch);
-    a.part_ml = reinterpret_cast<float *>(scratch + off_ml);
-    a.part_o = reinterpret_cast<float *>(scratch + off_o);
-    a.o = o;
-    a.o_f32 = p->f32;
-    const int grid = g.pairs * (g.nsplit / kAttnWarps);
-    return cuda_rc(p->g <= 8 ? launch_pdl(attn_decode_kernel<true>, grid, kAttnWarps * 32, 0, st, a)
-                              : launch_pdl(attn_decode_kernel<false>, grid, kAttnWarps * 32, 0, st, a));
+    return attn_launch(p, kv, q, k_new, v_new, B, keys, o, g, staged, reinterpret_cast<unsigned *>(scratch),
+                       reinterpret_cast<float *>(scratch + off_ml), reinterpret_cast<float *>(scratch + off_o), st);
 }

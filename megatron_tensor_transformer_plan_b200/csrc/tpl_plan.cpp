@@ -3,9 +3,9 @@
 // num_sms_current().
 //
 // Ownership rule ("Tensor parallel scaling curves", section "What tensor
-// parallelism actually splits"): shard `rank` owns query heads
-// [rank*h_per_gpu, (rank+1)*h_per_gpu), kv heads [rank*n_kv/t, ...) and ffn
-// columns [rank*F/t, ...).  Footprints: "Tensor Parallelism Fundamentals",
+// parallelism actually splits"): shard s owns the query heads
+// [s*n_q/t, (s+1)*n_q/t), the kv heads [s*n_kv/t, (s+1)*n_kv/t) and the ffn
+// columns [s*F/t, (s+1)*F/t).  Footprints: "Tensor Parallelism Fundamentals",
 // section "Memory Overhead and Communication Bottlenecks".
 
 #include <cuda_runtime.h>

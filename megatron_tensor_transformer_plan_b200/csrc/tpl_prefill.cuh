@@ -5,7 +5,7 @@
 //
 //   norm_split   a = RMSNorm(x) as bf16 hi + lo                 (HBM bound)
 //   gemm QKV     column-parallel, fused scatter to q / cache / k,v remainders
-//   attention    causal, owned heads, mma.sync with hi + lo operands; writes
+//   attention    causal, each shard's own heads, mma.sync with hi + lo operands; writes
 //                its output as bf16 hi + lo
 //   gemm O       row-parallel on o as bf16 hi + lo, t TMEM accumulators summed
 //                in shard order, + x

@@ -3,8 +3,8 @@ shard's weights and KV cache and runs the single-device library's step kernels
 on its slice, and the two row-parallel partial sums of a layer are added by an
 all-reduce over torch.distributed (NCCL) instead of the on-device fused sum
 ("Tensor parallel scaling curves", section "What tensor parallelism actually
-splits": Q/K/V and gate/up split by columns so that rank r owns heads
-[r*h_per_gpu, (r+1)*h_per_gpu), O and down split by rows, two all-reduces per
+splits": Q/K/V and gate/up split by columns so that rank r owns the query
+heads [r*n_q/t, (r+1)*n_q/t), O and down split by rows, two all-reduces per
 layer; "Tensor Parallelism Fundamentals", section "Mechanics of Matrix
 Slicing").
 

@@ -315,6 +315,9 @@ class Plan:
 
     def decode_stack(self, packed_list, kv_list, x, S: int, y, y32=None, ws=None, mode=TPL_REDUCE_FUSED):
         L = len(packed_list)
+        if L != self.dims.n_layers or len(kv_list) != L:
+            raise ValueError(f"decode_stack: the plan has {self.dims.n_layers} layers, got {L} packed layers and "
+                             f"{len(kv_list)} caches")
         arr = (c_void_p * L)(*[p.data_ptr() for p in packed_list])
         kvs = (tpl_kv * L)(*kv_list)
         B = x.shape[0]

@@ -9,7 +9,8 @@ arrays through ctypes.
 Every function cites the page passage it follows, by page title and section:
 
 * "Tensor parallel scaling curves", section "What tensor parallelism actually
-  splits" -- head-wise column split of Q/K/V, local attention on owned heads,
+  splits" -- head-wise column split of Q/K/V, each shard attending over its own
+  heads without exchange,
   row split of the output projection, gate/up column split, down row split,
   partial sums added (two per layer, 2L per pass).
 * "Tensor Parallelism Fundamentals", sections "Mechanics of Matrix Slicing" and
@@ -334,9 +335,10 @@ def attn_sharded(dims: Dims, w: dict, t: int, x: np.ndarray, a: np.ndarray, kc, 
 
 
 def plan_maps(dims: Dims, t: int):
-    """Shard maps from the ownership rule heads[rank*h_per_gpu:(rank+1)*h_per_gpu]
-    ("Tensor parallel scaling curves", "What tensor parallelism actually
-    splits").  Returns None when t is not admissible."""
+    """Shard maps from the ownership rule: shard s owns the contiguous block of
+    query heads [s*n_q/t, (s+1)*n_q/t) ("Tensor parallel scaling curves",
+    "What tensor parallelism actually splits").  Returns None when t is not
+    admissible."""
     q_shard = np.empty(dims.n_q_heads, np.int32)
     q_local = np.empty(dims.n_q_heads, np.int32)
     kv_shard = np.empty(dims.n_kv_heads, np.int32)

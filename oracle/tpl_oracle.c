@@ -12,8 +12,9 @@
  * Sources (page title, section):
  *  [TSC]  "Tensor parallel scaling curves", section "What tensor parallelism
  *         actually splits": Q/K/V projections split by columns so that each
- *         shard owns whole attention heads, heads[rank*h_per_gpu:(rank+1)*
- *         h_per_gpu]; attention runs on owned heads only; the output
+ *         shard owns whole attention heads -- shard s owns the contiguous
+ *         block of query heads [s*n_q/t, (s+1)*n_q/t); each shard computes
+ *         attention for its own heads with no exchange; the output
  *         projection is split by rows and yields a partial sum; gate and up
  *         are split by columns, down by rows; the row-split partials are
  *         summed (all-reduce), two such sums per layer, 2L per forward pass.
@@ -499,7 +500,7 @@ int orc_plan_maps(const orc_dims *dm, int32_t t, int32_t *q_shard, int32_t *q_lo
                   int32_t *kv_shard, int32_t *ffn_shard) {
     if (!(t == 1 || t == 2 || t == 4 || t == 8)) return 2;
     if (dm->n_q_heads % t || dm->n_kv_heads % t || dm->ffn % t) return 2;
-    int32_t hpg = dm->n_q_heads / t; /* h_per_gpu */
+    int32_t hpg = dm->n_q_heads / t; /* query heads per shard */
     for (int32_t rank = 0; rank < t; ++rank) {
         for (int32_t h = rank * hpg; h < (rank + 1) * hpg; ++h) {
             if (q_shard) q_shard[h] = rank;

@@ -121,6 +121,36 @@ def test_plan_maps_invariants(dims, t):
     assert np.all(np.diff(m["ffn_shard"]) >= 0)
 
 
+@pytest.mark.parametrize("dims", [(8192, 64, 8, 128, 28672), (4096, 32, 32, 128, 11008),
+                                  (256, 4, 2, 64, 688), (1024, 16, 8, 128, 2816)])
+@pytest.mark.parametrize("t", [1, 2, 4, 8])
+def test_plan_maps_rank_order(dims, t):
+    """The ownership rule fixes which block each rank holds, not only that the
+    blocks are contiguous: rank r holds the r-th block of n/t query heads, of
+    kv heads and of ffn columns, in ascending order ("Tensor parallel scaling
+    curves", "What tensor parallelism actually splits").  A reversed or
+    rotated rank order passes the invariants above but fails here."""
+    d = oracle.Dims(*dims)
+    m = oracle.plan_maps(d, t)
+    H, nq, nkv, hd, F = dims
+    if nq % t or nkv % t or F % t:
+        assert m is None
+        return
+    for r in range(t):
+        # the block written out from the rule, element by element
+        q_block = list(range(r * (nq // t), (r + 1) * (nq // t)))
+        kv_block = list(range(r * (nkv // t), (r + 1) * (nkv // t)))
+        f_block = list(range(r * (F // t), (r + 1) * (F // t)))
+        assert list(np.nonzero(m["q_shard"] == r)[0]) == q_block
+        assert list(np.nonzero(m["kv_shard"] == r)[0]) == kv_block
+        assert list(np.nonzero(m["ffn_shard"] == r)[0]) == f_block
+        assert [int(m["q_local"][h]) for h in q_block] == list(range(nq // t))
+    # shard 0 holds head 0 and the last shard holds the last head
+    assert m["q_shard"][0] == 0 and m["q_shard"][nq - 1] == t - 1
+    assert m["kv_shard"][0] == 0 and m["kv_shard"][nkv - 1] == t - 1
+    assert m["ffn_shard"][0] == 0 and m["ffn_shard"][F - 1] == t - 1
+
+
 @pytest.mark.parametrize("t", [0, 3, 5, 16, -1])
 def test_plan_maps_rejects_bad_degree(t):
     assert oracle.plan_maps(oracle.Dims(256, 8, 8, 32, 64), t) is None

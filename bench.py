@@ -249,6 +249,121 @@ def build_stack(plan, tpl, synth, torch, dev, seed=0):
     return packed, kvs, keep
 
 
+def run_tp(args, ws, rank, local):
+    """The stack with its shards on the N GPUs of the job (N = t, one shard
+    per rank): each rank holds its slice of every layer (its heads, ffn
+    columns and kv heads) and its cache shard, runs the library's steps on a
+    one-shard plan of those dimensions, and the two row-parallel partial sums
+    of every layer are added by an NCCL all-reduce (2L per step).  Reported
+    against the pages' time model T(N) = T(1)/N + 2L*T_allreduce(N)
+    ("Tensor parallel scaling curves", "The scaling math").  value = the B
+    tokens of one step / the slowest rank's step time (strong scaling: the
+    model is the same at every N)."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    from megatron_tensor_transformer_plan_b200 import build
+    build.build()
+    from megatron_tensor_transformer_plan_b200 import synth, tpl
+    from megatron_tensor_transformer_plan_b200.tp_dist import (CudaOps, ShardSpec, decode_stack_tp, shard_cache,
+                                                                shard_weights)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    t = ws
+    spec = ShardSpec(H, NQ, NKV, D, F, t, rank)
+    layers, keep = [], []
+    wsb = None
+    for l in range(L):
+        w = synth.layer_weights(H, NQ, NKV, D, F, seed=0, layer=l, dtype=torch.bfloat16, device=dev)
+        kl, vl = synth.kv_cache((BATCH, NKV, KV_LEN + 1, D), seed=0, layer=l, device=dev)
+        if wsb is None:
+            probe = tpl.Plan(tpl.make_dims(H, spec.nq_s, spec.nkv_s, D, spec.ffn_s, 1, 1e-5,
+                                           tpl.TPL_NORM | tpl.TPL_RESIDUAL), 1)
+            wsb = CudaOps.make_workspace(probe, BATCH, KV_LEN + 1, dev)
+        layers.append(CudaOps(spec, shard_weights(w, spec), shard_cache(kl, spec), shard_cache(vl, spec), BATCH,
+                              KV_LEN + 1, workspace=wsb))
+        del w, kl, vl
+    x = synth.activations(BATCH, H, seed=0, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def all_reduce(P):
+        if ws > 1:
+            dist.all_reduce(P)
+
+    def no_reduce(P):
+        pass
+
+    def barrier():
+        if ws > 1:
+            dist.barrier()
+
+    def timed(steps, reduce):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(steps):
+            decode_stack_tp(layers, x, KV_LEN, reduce)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        return max_over_ranks(e0.elapsed_time(e1) / steps, ws, dev)
+
+    for _ in range(args.warmup):
+        decode_stack_tp(layers, x, KV_LEN, all_reduce)
+    torch.cuda.synchronize()
+    for op in layers:
+        assert op.plan.last_device_error() == tpl.TPL_OK
+    clocks = Clocks(local)
+    clocks.start()
+    time.sleep(0.3)
+    ms = timed(args.steps, all_reduce)
+    clk = clocks.stop()
+    # the decomposition the model needs (not the reported value): the same
+    # steps with the collectives left out, and one all-reduce of a layer's
+    # partial (B x H fp32) timed alone
+    ms_local = timed(max(3, args.steps // 2), no_reduce)
+    ar_us = 0.0
+    if ws > 1:
+        P = torch.zeros((1, BATCH, H), dtype=torch.float32, device=dev)
+        for _ in range(10):
+            dist.all_reduce(P)
+        n_ar = 200
+        barrier()
+        torch.cuda.synchronize()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(n_ar):
+            dist.all_reduce(P)
+        a1.record(stream)
+        torch.cuda.synchronize()
+        ar_us = max_over_ranks(a0.elapsed_time(a1) / n_ar * 1e3, ws, dev)
+    predicted_ms = ms_local + 2 * L * ar_us / 1e3
+    if rank == 0:
+        line = {"metric": METRIC + " [tensor-parallel over the job's GPUs]", "value": BATCH / (ms / 1e3),
+                "unit": "tokens/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic (seeded N(0,0.02) weights, N(0,1) x/KV)",
+                "config": dict(config_dict(), t=t, workload=f"70B-shaped 80-layer decode stack, t={t} shards on "
+                               f"{t} GPU(s), NCCL all-reduce of the partials", reduce="nccl all-reduce"),
+                "tp_model": {"step_ms_without_collectives": ms_local, "allreduce_us_per_call": ar_us,
+                             "allreduces_per_step": 2 * L,
+                             "predicted_ms": predicted_ms,
+                             "measured_over_predicted": ms / predicted_ms,
+                             "model": "T(N) = T(1)/N + 2L*T_allreduce(N), with T(1)/N taken as this rank's step "
+                                      "without collectives"},
+                "gpu_launches": sum(op.plan.decode_kernel_count(BATCH, tpl.TPL_REDUCE_SEPARATE) for op in layers)
+                * args.steps,
+                "clocks": clk}
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 def run_ours(args, ws, rank, local):
     import torch
     from megatron_tensor_transformer_plan_b200 import build
@@ -368,6 +483,12 @@ def run_ours(args, ws, rank, local):
     del wsp, xp, yp
 
     peak, peak_kind = load_peaks()
+    configs = None
+    if ws == 1 and not args.no_configs:
+        del arr, kva, kvs, keep, packed, wsb
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        configs = run_configs(tpl, peak, peak_kind, local, args.config_iters)
     gu_gbs = gate_up_bytes_per_launch() / (gu_ms / 1e3) / 1e9
     per_step = plan.decode_kernel_count(BATCH, n_layers=L)
     if plan.decode_kernel_count(BATCH) == 6:  # the tensor-core family: the gate/up call is two kernels
@@ -399,6 +520,8 @@ def run_ours(args, ws, rank, local):
                             "peak_tflops": tpeak, "peak_kind": tpeak_kind + " (dense bf16 burst)",
                             "frac": pf_tflops / tpeak, "timing": "median of 10 calls, CUDA events, after 3 warm-ups",
                             "kernels_per_layer": 7}}
+        if configs is not None:
+            line["configs"] = configs
         if ws == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline_sample()
         print(json.dumps(line), flush=True)
@@ -408,31 +531,173 @@ def run_ours(args, ws, rank, local):
     return 0
 
 
+# Per-configuration decode layers (the benchmark spec's targets): one layer call
+# per timed iteration, CUDA events on the launching stream, median of
+# `iters` after 3 warm-ups; working sets under 4 x L2 rotate over copies of
+# the weights and caches so that every call reads from HBM.
+CONFIG_CASES = [
+    # name, H, nq, nkv, F, t, B, S, reduce, extra
+    ("config 1: tiny MLP block", 256, 2, 2, 688, 2, 1, 0, "fused", dict(flags=0, mlp_only=True)),
+    ("config 1: tiny MLP block", 256, 2, 2, 688, 2, 1, 0, "separate", dict(flags=0, mlp_only=True)),
+] + [
+    ("config 2: 7B layer", 4096, 32, 32, 11008, t, B, 2048, mode, {})
+    for B in (1, 16) for t in (1, 2, 4) for mode in (("fused",) if t == 1 else ("fused", "separate"))
+] + [
+    ("config 3: 70B layer", 8192, 64, 8, 28672, t, 16, 8192, mode, {})
+    for t in (1, 4, 8) for mode in (("fused", "separate") if t == 4 else ("fused",))
+] + [
+    ("config 5: one stack layer", 8192, 64, 8, 28672, 8, 4, 4096, "fused", {}),
+]
+
+
+def run_configs(tpl, peak, peak_kind, gpu_index, iters):
+    """Microseconds per layer, algorithmic GB/s and fraction of the copy
+    peak for each case, and each shard layout's fused time against the same
+    workload's unsharded (t = 1) layer."""
+    from megatron_tensor_transformer_plan_b200 import profile_configs as pc
+    clocks = Clocks(gpu_index)
+    clocks.start()
+    rows = []
+    for name, Hc, nq, nkv, Fc, t, B, S, mode, extra in CONFIG_CASES:
+        us, nbytes, ncopies, rc = pc.run_layer(tpl, Hc, nq, nkv, Fc, t, B, S, iters, mode, extra.get("flags"),
+                                               extra.get("mlp_only", False))
+        if rc != tpl.TPL_OK:
+            raise RuntimeError(f"{name}: device status {rc}")
+        gbs = nbytes / (us * 1e-6) / 1e9
+        rows.append({"workload": name, "hidden": Hc, "ffn": Fc, "t": t, "batch": B, "kv_len": S, "reduce": mode,
+                     "us_per_layer": us, "tokens_per_s": B / (us * 1e-6), "algorithmic_bytes": nbytes,
+                     "gb_s": gbs, "frac": gbs / peak, "copies_rotated": ncopies})
+    clk = clocks.stop()
+    base = {(r["workload"].split(":")[0], r["batch"]): r["us_per_layer"] for r in rows
+            if r["t"] == 1 and r["reduce"] == "fused"}
+    for r in rows:
+        b = base.get((r["workload"].split(":")[0], r["batch"]))
+        if b is not None and r["reduce"] == "fused" and r["t"] > 1:
+            r["overhead_vs_t1"] = r["us_per_layer"] / b - 1.0
+    return {"peak_gbs": peak, "peak_kind": peak_kind + " (burst copy)",
+            "timing": f"CUDA events around each layer call, median of {iters} after 3 warm-ups",
+            "bytes": "every weight once, the K/V cache once, new K/V, x and y",
+            "rows": rows, "clocks": clk}
+
+
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def _time_oracle(fn, min_runs=1, budget_s=10.0):
+    """Mean seconds per call of fn over at least min_runs calls, stopping
+    once budget_s has passed."""
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        fn()
+        n += 1
+        if n >= min_runs and time.perf_counter() - t0 > budget_s:
+            break
+        if n >= 5:
+            break
+    return (time.perf_counter() - t0) / n, n
+
+
 def cpu_baseline_sample():
-    """The oracle as it stands on the host cores: one layer of the stack
-    (batch 4, KV 4096), about 10-30 s of CPU work, scaled to the stack."""
+    """The oracle as it stands (plain fp64 C loops) on the host cores, on
+    bounded samples of the workloads: single-threaded and on every core.
+
+    All cores: config 1 (tiny MLP) and config 2 (7B layer, B = 1 and 16) and
+    config 3 (70B layer, B = 16, KV 8192) in full, config 4 (70B prefill) on
+    a 256-token chunk scaled to 2048 tokens by the FLOP count, and one layer
+    of the 80-layer stack scaled by 80 (the bench workload).  One thread: the
+    same, except that the larger cases run one sequence and scale by the
+    batch (each sequence is independent work in the oracle) and the prefill
+    is left out.  Each sample says what it ran."""
     import numpy as np
     import torch
     import oracle
     from megatron_tensor_transformer_plan_b200 import synth
     threads = os.cpu_count() or 1
+    f64 = lambda t: t.float().numpy().astype(np.float64)
+
+    def layer(H, nq, nkv, F, seed=0, mlp_only=False):
+        w = synth.layer_weights(H, nq, nkv, D, F, seed=seed, dtype=torch.bfloat16, device="cpu", mlp_only=mlp_only)
+        return {k: synth.bits(v) for k, v in w.items()}
+
+    def kv(B, nkv, S, seed=0):
+        kl, vl = synth.kv_cache((B, nkv, S + 1, D), seed=seed)
+        return synth.bits(kl), synth.bits(vl)
+
+    out = {"cpu_model": _cpu_model(), "nproc": threads, "entries": []}
+
+    def add(name, cores, secs, n, unit_per_s, unit, sample):
+        out["entries"].append({"workload": name, "cores": cores, "seconds_per_call": secs, "runs": n,
+                               "value": unit_per_s, "unit": unit, "sample": sample})
+
+    # config 1: tiny MLP block, t = 2 (the oracle's unsharded MLP; flags 0)
+    d1 = oracle.Dims(256, 2, 2, D, 688, flags=0)
+    w1 = layer(256, 2, 2, 688, mlp_only=True)
+    x1 = f64(synth.activations(1, 256, seed=0))
+    for cores in (1, threads):
+        oracle.set_threads(cores)
+        secs, n = _time_oracle(lambda: oracle.mlp_sharded(d1, w1, 1, x1), 5, 0.5)
+        add("config 1: tiny MLP H=256 F=688, 1 token", cores, secs, n, 1 / secs, "tokens/s", "full")
+    # config 2: 7B layer (t does not change the unsharded oracle), KV 2048
+    d2 = oracle.Dims(4096, 32, 32, D, 11008)
+    w2 = layer(4096, 32, 32, 11008)
+    k2, v2 = kv(16, 32, 2048)
+    for B in (1, 16):
+        x2 = f64(synth.activations(B, 4096, seed=0))
+        for cores in (1, threads):
+            oracle.set_threads(cores)
+            Bs = 1 if (cores == 1 and B > 1) else B
+            secs, n = _time_oracle(lambda: oracle.decode_layer(d2, w2, x2[:Bs], k2[:Bs], v2[:Bs], 2048), 1, 2.0)
+            secs *= B / Bs
+            add(f"config 2: 7B layer B={B} KV 2048", cores, secs, n, B / secs, "tokens/s",
+                "full" if Bs == B else f"{Bs} of {B} sequences, x{B // Bs}")
+    del w2, k2, v2
+    # config 3: 70B layer, B = 16, KV 8192
+    d3 = oracle.Dims(H, NQ, NKV, D, F)
+    w3 = layer(H, NQ, NKV, F)
+    k3, v3 = kv(16, NKV, 8192)
+    x3 = f64(synth.activations(16, H, seed=0))
+    for cores in (threads, 1):
+        oracle.set_threads(cores)
+        Bs = 1 if cores == 1 else 16
+        secs, n = _time_oracle(lambda: oracle.decode_layer(d3, w3, x3[:Bs], k3[:Bs], v3[:Bs], 8192), 1, 2.0)
+        secs *= 16 / Bs
+        add("config 3: 70B layer B=16 KV 8192", cores, secs, n, 16 / secs, "tokens/s",
+            "full" if Bs == 16 else "1 of 16 sequences, x16")
+    del k3, v3
+    # the bench workload: one layer of the stack (B = 4, KV 4096), x80 layers
+    k5, v5 = kv(BATCH, NKV, KV_LEN)
+    x5 = f64(synth.activations(BATCH, H, seed=0))
+    for cores in (threads, 1):
+        oracle.set_threads(cores)
+        Bs = BATCH if cores > 1 else 1
+        secs, n = _time_oracle(lambda: oracle.decode_layer(d3, w3, x5[:Bs], k5[:Bs], v5[:Bs], KV_LEN), 1, 2.0)
+        secs *= BATCH / Bs
+        add(f"config 5: 80-layer stack B={BATCH} KV {KV_LEN}", cores, secs * L, n, BATCH / (secs * L), "tokens/s",
+            f"one layer{'' if Bs == BATCH else f', 1 of {BATCH} sequences x{BATCH}'}, x{L} layers extrapolated")
+    del k5, v5
+    # config 4: prefill, a 256-token chunk, scaled to 2048 tokens by FLOPs
     oracle.set_threads(threads)
-    dims = oracle.Dims(H, NQ, NKV, D, F)
-    w = synth.layer_weights(H, NQ, NKV, D, F, seed=0, layer=0, dtype=torch.bfloat16, device="cpu")
-    wb = {k: synth.bits(v) for k, v in w.items()}
-    x = synth.activations(BATCH, H, seed=0, dtype=torch.bfloat16).float().numpy().astype(np.float64)
-    kl, vl = synth.kv_cache((BATCH, NKV, KV_LEN + 1, D), seed=0)
-    kb, vb = synth.bits(kl), synth.bits(vl)
-    t0 = time.perf_counter()
-    n = 0
-    while True:
-        oracle.decode_layer(dims, wb, x, kb, vb, KV_LEN)
-        n += 1
-        if time.perf_counter() - t0 > 10.0 or n >= 5:
-            break
-    t_layer = (time.perf_counter() - t0) / n
-    return {"value": BATCH / (t_layer * L), "unit": "tokens/s", "cores": oracle.get_threads(), "kind": "oracle",
-            "sample": f"{n} run(s) of one decoder layer (B={BATCH}, KV {KV_LEN}), fp64; x{L} layers extrapolated"}
+    Tp = 256
+    xp = f64(synth.activations(Tp, H, seed=0, layer=1000))
+    secs, n = _time_oracle(lambda: oracle.prefill_layer(d3, w3, xp), 1, 0.0)
+    secs_full = secs * prefill_flops(PREFILL_T) / prefill_flops(Tp)
+    add(f"config 4: 70B prefill {PREFILL_T} tokens", threads, secs_full, n, PREFILL_T / secs_full, "tokens/s",
+        f"one {Tp}-token chunk, scaled to {PREFILL_T} tokens by the FLOP count "
+        f"({prefill_flops(PREFILL_T) / prefill_flops(Tp):.2f}x)")
+    oracle.set_threads(threads)
+    stack = [e for e in out["entries"] if e["workload"].startswith("config 5") and e["cores"] == threads][0]
+    out.update({"value": stack["value"], "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                "sample": stack["sample"]})
+    return out
 
 
 def main():
@@ -442,12 +707,19 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-configuration layer timings")
+    ap.add_argument("--tp", action="store_true",
+                    help="shard the stack over the job's GPUs (one shard per rank, NCCL all-reduce) instead of "
+                         "running an independent replica per GPU")
+    ap.add_argument("--config-iters", type=int, default=30)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     ws, rank, local = dist_init()
     if args.impl == "reference":
         return run_reference(args, ws, rank)
+    if args.tp:
+        return run_tp(args, ws, rank, local)
     return run_ours(args, ws, rank, local)
 
 

@@ -154,10 +154,22 @@ void tpl_plan_destroy(tpl_plan *plan);
  * query groups of at most 8 heads when every (shard, sequence, kv head) pair
  * gets at least two CTAs in one wave of SMs; other shapes use the other
  * kernel), 1 = keys streamed into registers (any shape).
+ * TPL_OPT_PREFILL_SPLIT chooses, per prefill projection, whether its
+ * activation operand is carried as two bf16 parts (hi + lo, about 16
+ * mantissa bits, two products per tile) or one (rounded to bf16, one
+ * product): a bit mask of TPL_SPLIT_QKV (the normalised x into QKV),
+ * TPL_SPLIT_O (the attention output into O) and TPL_SPLIT_GU (the normalised
+ * h into gate/up); the down projection's operand (act) is always one part.
+ * Default TPL_SPLIT_DEFAULT.
  * Returns TPL_EINVAL for an unknown option or value. */
 #define TPL_OPT_GEMV_MODE 1
 #define TPL_OPT_PREFILL_ATTN 2
 #define TPL_OPT_DECODE_ATTN 3
+#define TPL_OPT_PREFILL_SPLIT 4
+#define TPL_SPLIT_QKV 1
+#define TPL_SPLIT_O 2
+#define TPL_SPLIT_GU 4
+#define TPL_SPLIT_DEFAULT (TPL_SPLIT_QKV | TPL_SPLIT_O | TPL_SPLIT_GU)
 int tpl_plan_set_option(tpl_plan *plan, int32_t option, int32_t value);
 
 /* Footprints (host) -- see tpl_plan_info. */

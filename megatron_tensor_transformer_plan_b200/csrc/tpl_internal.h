@@ -59,6 +59,7 @@ struct tpl_plan {
     int gemv_mode;  // 0: mma.sync fragments (bf16); 1: fp32 FFMA; 2: bf16 FFMA; 3: tcgen05 + TMA (bf16);
                     // 4: per projection (default for bf16)
     int attn_prefill_mode;  // 0: tcgen05 (power-of-two group sizes); 1: mma.sync
+    int prefill_split;      // TPL_SPLIT_* bits: prefill operands carried as bf16 hi + lo
     int attn_decode_mode;   // 0: staged (g <= 8, pairs fit one wave); 1: register-streamed
     bool rope;
     double rope_theta[64];  // rope_base^(-2e/128), e < 64

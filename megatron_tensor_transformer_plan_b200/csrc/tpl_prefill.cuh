@@ -54,12 +54,12 @@ int gemm_go(int slot, GemmArgs &a, int shard_units, cudaStream_t st) {
     return cuda_rc(launch_pdl(gemm_tc_kernel<SA, RS>, grid, kGemmThreads, (size_t)GemmSmem<SA>::BYTES, st, a));
 }
 
-// Column-parallel projection: A = bf16 hi + lo [T][K] activations, W the
-// shards' stacked rows [N][ld] (2-D).
+// Column-parallel projection: A = bf16 hi (+ lo, when a_lo is not NULL)
+// [T][K] activations, W the shards' stacked rows [N][ld] (2-D).
 int gemm_column(GemmArgs &a, const void *a_hi, const void *a_lo, int64_t K, const void *W, int64_t N, int64_t ld,
                 cudaStream_t st) {
     int rc = make_map(&a.tm_a, a_hi, K, a.M, K * 2, kGemmKTile, kGemmMTile);
-    if (rc == TPL_OK) rc = make_map(&a.tm_a2, a_lo, K, a.M, K * 2, kGemmKTile, kGemmMTile);
+    if (rc == TPL_OK && a_lo) rc = make_map(&a.tm_a2, a_lo, K, a.M, K * 2, kGemmKTile, kGemmMTile);
     if (rc == TPL_OK) rc = make_map(&a.tm_w, W, ld, N, ld * 2, kGemmKTile, kGemmNTile);
     if (rc != TPL_OK) return rc;
     a.N = (int)N;
@@ -67,7 +67,7 @@ int gemm_column(GemmArgs &a, const void *a_hi, const void *a_lo, int64_t K, cons
     a.nseg = 1;
     a.a_col_stride = 0;
     a.w3d = 0;
-    return gemm_go<true, false>(0, a, 1, st);
+    return a_lo ? gemm_go<true, false>(0, a, 1, st) : gemm_go<false, false>(1, a, 1, st);
 }
 
 // Row-parallel projection: A [T][t*Ks] bf16 (shard s owns columns
@@ -232,7 +232,8 @@ int prefill_layer(tpl_plan *p, const char *packed, const tpl_kv *kv, const void 
         a.pos0 = p0;
         a.rope = p->rope ? 1 : 0;
         std::memcpy(a.theta, p->rope_theta, sizeof(a.theta));
-        rc = gemm_column(a, a_hi, a_lo, H, packed + p->off_qkv, (int64_t)p->t * p->qkv_rows_s, p->ld_h, st);
+        rc = gemm_column(a, a_hi, (p->prefill_split & TPL_SPLIT_QKV) ? a_lo : nullptr, H, packed + p->off_qkv,
+                         (int64_t)p->t * p->qkv_rows_s, p->ld_h, st);
         if (rc != TPL_OK) return rc;
     }
     rc = run_attn_prefill(p, kv, q, klo, vlo, T, p0, o, o_lo, st);
@@ -246,7 +247,8 @@ int prefill_layer(tpl_plan *p, const char *packed, const tpl_kv *kv, const void 
         } else {
             a.out32 = P;
         }
-        rc = gemm_row(a, p, o, o_lo, (int64_t)p->nq_s * hd, packed + p->off_o, p->ld_o, p->blk_o, fused, st);
+        rc = gemm_row(a, p, o, (p->prefill_split & TPL_SPLIT_O) ? o_lo : nullptr, (int64_t)p->nq_s * hd,
+                      packed + p->off_o, p->ld_o, p->blk_o, fused, st);
         if (rc != TPL_OK) return rc;
         if (fused) p->reductions.fetch_add(1);
         else if ((rc = run_reduce(p, st, P, resid ? x : nullptr, 0, T, h, nullptr)) != TPL_OK) return rc;
@@ -258,7 +260,8 @@ int prefill_layer(tpl_plan *p, const char *packed, const tpl_kv *kv, const void 
         a.epi = GEPI_GU;
         a.out_act = act;
         a.act_f32 = 0;
-        rc = gemm_column(a, a_hi, a_lo, H, packed + p->off_gu, (int64_t)p->t * 2 * p->F_s, p->ld_h, st);
+        rc = gemm_column(a, a_hi, (p->prefill_split & TPL_SPLIT_GU) ? a_lo : nullptr, H, packed + p->off_gu,
+                         (int64_t)p->t * 2 * p->F_s, p->ld_h, st);
         if (rc != TPL_OK) return rc;
     }
     {  // down: y = h + sum_s act_s Wd[s]^T

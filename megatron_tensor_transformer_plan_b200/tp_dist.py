@@ -162,10 +162,18 @@ def decode_stack_tp(ops_per_layer, x, S: int, all_reduce, residual: bool = True)
 
 class CudaOps(DecodeStepOps):
     """The steps through the C ABI on the rank's GPU: a one-shard plan of the
-    sliced dimensions, the rank's packed weights and KV cache shard."""
+    sliced dimensions, the rank's packed weights and KV cache shard.
+
+    Every per-step buffer (q, new k/v, o, the partials, h, act, y) and the
+    workspace are allocated once here, the workspace for the largest S the
+    cache holds (its size does not shrink with S), so a decode loop never
+    enters the allocator.  The step methods return these buffers: a layer's
+    output stays valid until that layer's next step.  `workspace` may be
+    shared by the layers of one rank (their steps run in order on one
+    stream)."""
 
     def __init__(self, spec: ShardSpec, weights_local: dict, k_local, v_local, batch: int, seq_cap: int,
-                 rms_eps: float = 1e-5, flags=None, rope_base: float = 500000.0):
+                 rms_eps: float = 1e-5, flags=None, rope_base: float = 500000.0, workspace=None):
         import torch
 
         from megatron_tensor_transformer_plan_b200 import tpl
@@ -180,51 +188,58 @@ class CudaOps(DecodeStepOps):
         self.k, self.v = self.plan.pack_kv(k_local.contiguous()), self.plan.pack_kv(v_local.contiguous())
         self.kv = tpl.Plan.kv(self.k, self.v, batch, seq_cap)
         self.B = batch
+        self.seq_cap = seq_cap
         self.dev = self.packed.device
+        self.ws = workspace if workspace is not None else self.make_workspace(self.plan, batch, seq_cap, self.dev)
+        if self.ws.numel() < self.plan.workspace_size(batch, seq_cap - 1):
+            raise ValueError("workspace smaller than the plan needs at the cache's capacity")
+        B, sp, f32, act = batch, spec, torch.float32, self.plan.act_dtype
+        self.q = torch.empty((B, sp.nq_s, sp.head_dim), dtype=f32, device=self.dev)
+        self.kn = torch.empty((B, sp.nkv_s, sp.head_dim), dtype=f32, device=self.dev)
+        self.vn = torch.empty_like(self.kn)
+        self.o = torch.empty((B, sp.nq_s * sp.head_dim), dtype=act, device=self.dev)
+        self.P = torch.empty((1, B, sp.hidden), dtype=f32, device=self.dev)
+        self.h = torch.empty((B, sp.hidden), dtype=f32, device=self.dev)
+        self.act = torch.empty((B, sp.ffn_s), dtype=act, device=self.dev)
+        self.P2 = torch.empty((1, B, sp.hidden), dtype=f32, device=self.dev)
+        self.y32 = torch.empty((B, sp.hidden), dtype=f32, device=self.dev)
+        self.y = torch.empty((B, sp.hidden), dtype=act, device=self.dev)
 
-    def _ws(self, S):
-        if getattr(self, "_ws_S", None) != S:
-            self.ws = self.plan.workspace(self.B, S, device=self.dev)
-            self._ws_S = S
-        return self.ws
+    @staticmethod
+    def make_workspace(plan, batch: int, seq_cap: int, device):
+        """A workspace for every S up to seq_cap - 1 (the largest needed)."""
+        return plan.workspace(batch, seq_cap - 1, device=device)
+
+    def _check_S(self, S):
+        if not 0 <= S < self.seq_cap:
+            raise ValueError(f"S = {S} outside the cache's capacity {self.seq_cap}")
 
     def qkv(self, x, S):
-        t = self.torch
-        sp = self.spec
-        q = t.empty((self.B, sp.nq_s, sp.head_dim), dtype=t.float32, device=self.dev)
-        kn = t.empty((self.B, sp.nkv_s, sp.head_dim), dtype=t.float32, device=self.dev)
-        vn = t.empty_like(kn)
-        self.plan.qkv(self.packed, self.kv, x, S, q, self._ws(S), kn, vn)
-        return q, kn, vn
+        self._check_S(S)
+        self.plan.qkv(self.packed, self.kv, x, S, self.q, self.ws, self.kn, self.vn)
+        return self.q, self.kn, self.vn
 
     def attn(self, q, kn, vn, S):
-        o = self.torch.empty((self.B, self.spec.nq_s * self.spec.head_dim), dtype=self.plan.act_dtype,
-                             device=self.dev)
-        self.plan.attn_decode(self.kv, q, S, o, self._ws(S), kn, vn)
-        return o
+        self._check_S(S)
+        self.plan.attn_decode(self.kv, q, S, self.o, self.ws, kn, vn)
+        return self.o
 
     def o_partial(self, o):
-        P = self.torch.empty((1, self.B, self.spec.hidden), dtype=self.torch.float32, device=self.dev)
-        self.plan.o_proj(self.packed, o, None, partials=P, ws=self.ws)
-        return P
+        self.plan.o_proj(self.packed, o, None, partials=self.P, ws=self.ws)
+        return self.P
 
     def add_resid(self, P, resid, resid_is_f32):
-        h = self.torch.empty((self.B, self.spec.hidden), dtype=self.torch.float32, device=self.dev)
-        self.plan.reduce_partials(P, resid, resid_is_f32, out32=h)
-        return h
+        self.plan.reduce_partials(P, resid, resid_is_f32, out32=self.h)
+        return self.h
 
     def gate_up(self, h):
-        act = self.torch.empty((self.B, self.spec.ffn_s), dtype=self.plan.act_dtype, device=self.dev)
-        self.plan.gate_up(self.packed, h, act, self.ws)
-        return act
+        self.plan.gate_up(self.packed, h, self.act, self.ws)
+        return self.act
 
     def down_partial(self, act):
-        P = self.torch.empty((1, self.B, self.spec.hidden), dtype=self.torch.float32, device=self.dev)
-        self.plan.down_proj(self.packed, act, None, partials=P, ws=self.ws)
-        return P
+        self.plan.down_proj(self.packed, act, None, partials=self.P2, ws=self.ws)
+        return self.P2
 
     def add_resid_out(self, P, h):
-        y32 = self.torch.empty((self.B, self.spec.hidden), dtype=self.torch.float32, device=self.dev)
-        y = self.torch.empty((self.B, self.spec.hidden), dtype=self.plan.act_dtype, device=self.dev)
-        self.plan.reduce_partials(P, h, True, out32=y32, out_act=y)
-        return y32, y
+        self.plan.reduce_partials(P, h, True, out32=self.y32, out_act=self.y)
+        return self.y32, self.y

@@ -27,6 +27,9 @@ TPL_REDUCE_FUSED, TPL_REDUCE_SEPARATE = 0, 1
 TPL_OPT_GEMV_MODE = 1
 TPL_OPT_PREFILL_ATTN = 2
 TPL_OPT_DECODE_ATTN = 3
+TPL_OPT_PREFILL_SPLIT = 4
+TPL_SPLIT_QKV, TPL_SPLIT_O, TPL_SPLIT_GU = 1, 2, 4
+TPL_SPLIT_DEFAULT = TPL_SPLIT_QKV | TPL_SPLIT_O | TPL_SPLIT_GU
 TPL_ATTN_STATIC_SCRATCH_BYTES = 4 * 1024 * 1024
 
 c_int32, c_int64, c_size_t, c_void_p, c_uint32 = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_uint32

@@ -445,6 +445,17 @@ void tpl_reset_counters(tpl_plan *plan);
  * TPL_ECUDA (the stream reported an error). */
 int tpl_last_device_error(const tpl_plan *plan, tpl_stream stream);
 
+/* Timeline trace (the diagnostic build of the library, compiled with
+ * -DTPL_TRACE; the ordinary build returns TPL_EUNSUPPORTED and writes 0 to
+ * *n_records).  Each decode kernel appends one record per CTA: a tag (1 QKV,
+ * 2 attention, 3 O, 4 gate/up, 5 down, 6 operand kernel), the CTA index, its
+ * SM, the grid size, and four global-timer values in ns (entry, dependency
+ * wait passed, main loop done, exit; 0 where a kernel takes no such mark).
+ * records: host array of max_records records of 48 bytes (4 x uint32 then 4
+ * x uint64).  Synchronises the device, copies up to max_records of the
+ * records taken since the last read and starts a new trace. */
+int tpl_trace_read(void *records, int32_t max_records, int32_t *n_records);
+
 /* Static description of a status code. */
 const char *tpl_status_string(int status);
 

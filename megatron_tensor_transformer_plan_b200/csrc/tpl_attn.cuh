@@ -116,9 +116,12 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const __gr
         }
     };
     KV16 bufA, bufB;
+    TPL_TRACE_VARS
+    if (threadIdx.x == 0) TPL_TRACE_AT(0);
     if (early && k0 < k1) load16(bufA, k0);
     pdl_wait();
     pdl_trigger();
+    if (threadIdx.x == 0) TPL_TRACE_AT(1);
     if (!early && k0 < k1) load16(bufA, k0);
 
     if (gid < a.g) load_q(gid, qh0, ql0);
@@ -273,6 +276,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const __gr
         }
     }
     __syncthreads();
+    if (threadIdx.x == 0) TPL_TRACE_AT(2);
     const int dim = threadIdx.x;  // 128 threads, one head_dim column each
     const int cpp_ = cpp;
     const int64_t cbase = ((int64_t)pair * cpp_ + chunk) * a.g;  // this CTA's partial
@@ -305,7 +309,13 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const __gr
         if (prev >= (unsigned)cpp_) record_error(2u);
     }
     __syncthreads();
-    if (!s_last) return;
+    if (!s_last) {
+        if (threadIdx.x == 0) {
+            TPL_TRACE_AT(3);
+            TPL_TRACE_PUT(TR_ATTN);
+        }
+        return;
+    }
     __threadfence();
     // stage every CTA partial's (max, sum) for this pair
     __shared__ float s_w[64][16];  // weights exp2(m_i - M) per CTA partial and head
@@ -357,7 +367,11 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const __gr
         if (has_new) num += exp2f(s_new[hrow] - s_M[hrow]) * a.v_new[((int64_t)b * (a.nq / a.g) + j) * D + dim];
         store_act(a.o, a.o_f32, ((int64_t)b * a.nq + (int64_t)j * a.g + hrow) * D + dim, num / s_den[hrow]);
     }
-    if (threadIdx.x == 0) atomicExch(&a.tickets[pair], 0u);
+    if (threadIdx.x == 0) {
+        atomicExch(&a.tickets[pair], 0u);
+        TPL_TRACE_AT(3);
+        TPL_TRACE_PUT(TR_ATTN);
+    }
 }
 
 
@@ -398,6 +412,8 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) attn_decode_staged_kernel(
     const int64_t k1 = min(a.keys, k0 + a.kps);
     const int nsteps = k1 > k0 ? (int)((k1 - k0 + 15) / 16) : 0;
     const bool early = a.k_new != nullptr;
+    TPL_TRACE_VARS
+    if (threadIdx.x == 0) TPL_TRACE_AT(0);
     __nv_bfloat16 *ring = stg_smem + (size_t)warp * kStgStages * kStgStep;
 
     // stage st (keys k0 + 16 st ..) into slot st % kStgStages; keys past k1 read as zero
@@ -426,6 +442,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) attn_decode_staged_kernel(
         for (int st = 0; st < kStgStages - 1; ++st) issue(st);
     pdl_wait();
     pdl_trigger();
+    if (threadIdx.x == 0) TPL_TRACE_AT(1);
     if (!early)
         for (int st = 0; st < kStgStages - 1; ++st) issue(st);
 
@@ -506,6 +523,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) attn_decode_staged_kernel(
         __syncwarp();  // this slot is refilled by a later issue()
     }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
+    if (threadIdx.x == 0) TPL_TRACE_AT(2);
     // rows gid + 8 held the P_lo . V half of the same head
 #pragma unroll
     for (int t = 0; t < 16; ++t) {
@@ -559,7 +577,13 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) attn_decode_staged_kernel(
         if (prev >= (unsigned)cpp) record_error(2u);
     }
     __syncthreads();
-    if (!s_last) return;
+    if (!s_last) {
+        if (threadIdx.x == 0) {
+            TPL_TRACE_AT(3);
+            TPL_TRACE_PUT(TR_ATTN);
+        }
+        return;
+    }
     __threadfence();
     __shared__ float s_w[kAttnMaxCtasPerPair][8];
     __shared__ float s_M[8], s_den[8], s_new[8];
@@ -609,7 +633,11 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) attn_decode_staged_kernel(
         if (has_new) num += exp2f(s_new[hrow] - s_M[hrow]) * a.v_new[((int64_t)b * (a.nq / a.g) + j) * D + dim];
         store_act(a.o, a.o_f32, ((int64_t)b * a.nq + (int64_t)j * a.g + hrow) * D + dim, num / s_den[hrow]);
     }
-    if (threadIdx.x == 0) atomicExch(&a.tickets[pair], 0u);
+    if (threadIdx.x == 0) {
+        atomicExch(&a.tickets[pair], 0u);
+        TPL_TRACE_AT(3);
+        TPL_TRACE_PUT(TR_ATTN);
+    }
 }
 
 }  // namespace tpl

@@ -19,6 +19,50 @@ __device__ __forceinline__ void record_error(unsigned code) { atomicOr(&g_err_wo
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// Timeline tracing (built only with -DTPL_TRACE, the library's diagnostic
+// variant): one thread per CTA takes up to four global-timer marks (entry,
+// dependency wait passed, main loop done, exit) and appends one record per
+// CTA; tpl_trace_read copies the records out.  Compiled out otherwise.
+enum { TR_QKV = 1, TR_ATTN = 2, TR_O = 3, TR_GU = 4, TR_DOWN = 5, TR_OPERAND = 6, TR_REDUCE = 7 };
+#ifdef TPL_TRACE
+constexpr unsigned kTraceMax = 1u << 18;
+struct TraceRec {
+    uint32_t tag, cta, smid, grid;
+    uint64_t t[4];
+};
+__device__ TraceRec g_trace[kTraceMax];
+__device__ unsigned g_trace_n;
+__device__ __forceinline__ uint64_t trace_now() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void trace_put(uint32_t tag, const uint64_t (&t)[4]) {
+    uint32_t sm;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
+    const unsigned k = atomicAdd(&g_trace_n, 1u);
+    if (k < kTraceMax) {
+        TraceRec r;
+        r.tag = tag;
+        r.cta = blockIdx.x + gridDim.x * blockIdx.y;
+        r.smid = sm;
+        r.grid = gridDim.x * gridDim.y;
+        r.t[0] = t[0];
+        r.t[1] = t[1];
+        r.t[2] = t[2];
+        r.t[3] = t[3];
+        g_trace[k] = r;
+    }
+}
+#define TPL_TRACE_VARS uint64_t tr_t[4] = {0, 0, 0, 0};
+#define TPL_TRACE_AT(i) (tr_t[i] = trace_now())
+#define TPL_TRACE_PUT(tag) trace_put((tag), tr_t)
+#else
+#define TPL_TRACE_VARS
+#define TPL_TRACE_AT(i) ((void)0)
+#define TPL_TRACE_PUT(tag) ((void)0)
+#endif
+
 // 16-byte streaming load of read-once data (weights, KV cache): not kept in L1.
 __device__ __forceinline__ uint4 ldg_stream(const void *p) {
     uint4 r;

@@ -130,6 +130,7 @@ int check_kv(const tpl_kv *kv, int B, int64_t S) {
 
 int gemv_launch(Ctx &c, GemvArgs &a, int N, int nseg, int Kseg, int op) {
     tpl_plan *p = c.p;
+    a.trace_row_tag = op == OP_O ? TR_O : TR_DOWN;
     if (c.B > kMaxBatchCuda) return TPL_EUNSUPPORTED;
     const int sms = num_sms_current();
     if (sms <= 0) return TPL_ECUDA;
@@ -328,6 +329,7 @@ int run_row_tc(Ctx &c, const char *packed, int op, const void *x, const void *re
                void *out_act, float *partials, bool write_xs = false, const float *xs_gamma = nullptr) {
     tpl_plan *p = c.p;
     GemvTcArgs a = gt_args(p);
+    a.trace_row_tag = op == OP_O ? TR_O : TR_DOWN;
     if (partials) {
         a.epi = GT_ROW_PARTIAL;
         a.partials = partials;
@@ -876,6 +878,27 @@ int tpl_decode_kernel_count(const tpl_plan *p, int32_t B, int32_t reduce_mode, i
     if (n > 0x7fffffff) return TPL_EINVAL;
     *count = (int32_t)n;
     return TPL_OK;
+}
+
+int tpl_trace_read(void *records, int32_t max_records, int32_t *n_records) {
+#ifdef TPL_TRACE
+    if (!n_records || max_records < 0 || (max_records > 0 && !records)) return TPL_EINVAL;
+    if (cudaDeviceSynchronize() != cudaSuccess) return TPL_ECUDA;
+    unsigned n = 0;
+    if (cudaMemcpyFromSymbol(&n, g_trace_n, sizeof(n)) != cudaSuccess) return TPL_ECUDA;
+    if (n > kTraceMax) n = kTraceMax;
+    const unsigned take = n < (unsigned)max_records ? n : (unsigned)max_records;
+    if (take && cudaMemcpyFromSymbol(records, g_trace, take * sizeof(TraceRec)) != cudaSuccess) return TPL_ECUDA;
+    const unsigned z = 0;
+    if (cudaMemcpyToSymbol(g_trace_n, &z, sizeof(z)) != cudaSuccess) return TPL_ECUDA;
+    *n_records = (int32_t)take;
+    return TPL_OK;
+#else
+    (void)records;
+    (void)max_records;
+    if (n_records) *n_records = 0;
+    return TPL_EUNSUPPORTED;
+#endif
 }
 
 int tpl_last_device_error(const tpl_plan *p, tpl_stream stream) {

@@ -70,6 +70,7 @@ struct GemvArgs {
     int64_t S, seq_cap;
     float *gp;
     unsigned *tickets;
+    int trace_row_tag;  // timeline tag of a row-parallel launch (traced builds)
 };
 
 template <int MODE>
@@ -148,6 +149,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
     const int rb = blockIdx.x / g.ksplit, ks = blockIdx.x % g.ksplit;
     const int rg0 = (int)((int64_t)rb * g.ng / g.rb), rg1 = (int)((int64_t)(rb + 1) * g.ng / g.rb);
     const int kgl = warp % g.wk, wslot = warp / g.wk;
+    TPL_TRACE_VARS
+    if (tid == 0) TPL_TRACE_AT(0);
 
     // K-group -> segment and block range.
     const int KG = g.ksplit * g.wk;
@@ -228,6 +231,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
     }
     pdl_wait();
     pdl_trigger();
+    if (tid == 0) TPL_TRACE_AT(1);
 
     // ---- stage the activation slice (normalised if requested) ----
     // Each token gets a power-of-two group of tpt threads (512 / next pow2 of
@@ -598,6 +602,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
     }
 
     // ---- split-K: the last CTA of the row block adds the partials in order ----
+    if (tid == 0) TPL_TRACE_AT(2);
     if (g.ksplit > 1) {
         __threadfence();
         __syncthreads();
@@ -635,6 +640,10 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
             }
             if (tid == 0) atomicExch(&a.tickets[rb], 0u);
         }
+    }
+    if (tid == 0) {
+        TPL_TRACE_AT(3);
+        TPL_TRACE_PUT(a.epi == EPI_QKV ? TR_QKV : a.epi == EPI_GU ? TR_GU : a.trace_row_tag);
     }
 }
 

@@ -117,6 +117,7 @@ struct GemvTcArgs {
     float *gpart;       // [G][2][nseg][gstride / 4][128] float4: token quads outer, rows inner
     int gstride;        // floats per row of a piece: 16 * ceil(B / 16)
     unsigned *tickets;  // [tiles]
+    int trace_row_tag;  // timeline tag of a row-parallel launch (traced builds)
 };
 
 // Tokens 16*ch .. 16*ch+15 of one accumulator row: the hi column plus the
@@ -262,6 +263,8 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
     const int G = gridDim.x, cta = blockIdx.x;
     const int64_t u0 = gt_start(a.U, G, cta), u1 = gt_start(a.U, G, cta + 1);
     const int64_t per_tile = (int64_t)a.nseg * a.kbs;
+    TPL_TRACE_VARS
+    if (threadIdx.x == 0) TPL_TRACE_AT(0);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
@@ -339,6 +342,7 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
                 else tma_load_2d(st, &a.tm_w, kb * kGtK, tile * kGtRows, &full[i]);
             }
             pdl_wait();
+            TPL_TRACE_AT(1);
             restart();
             int it = 0;
             for (; it < n; ++it, advance()) {
@@ -357,6 +361,7 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
                 tma_load_2d(st + kGtWBytes, &a.tm_x, seg * a.x_seg_stride + kb * kGtK, 0, &full[s]);
             }
             *s_issued = it;
+            TPL_TRACE_AT(2);
         }
     } else if (warp == 1) {
         pdl_wait();
@@ -656,6 +661,10 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
         for (int it = *s_consumed; it < *s_issued; ++it) mbar_wait(&full[it % NS], (unsigned)(it / NS) & 1u);
     }
     __syncthreads();
+    if (threadIdx.x == 0) {
+        TPL_TRACE_AT(3);
+        TPL_TRACE_PUT(a.epi == GT_QKV ? TR_QKV : a.epi == GT_GU ? TR_GU : a.trace_row_tag);
+    }
     if (warp == 1) {
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));

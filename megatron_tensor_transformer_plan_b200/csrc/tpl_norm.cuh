@@ -85,8 +85,16 @@ __global__ void __launch_bounds__(256) norm_split_kernel(const void *x, int x_f3
 // 1/rms itself.  grid (ceil(H / 2048), B), 256 threads x 8 elements.
 __global__ void __launch_bounds__(256) scale_split_kernel(const void *x, int x_f32, const float *gamma, int H,
                                                           __nv_bfloat16 *xs, int half) {
+    TPL_TRACE_VARS
+    if (threadIdx.x == 0) TPL_TRACE_AT(0);
     pdl_wait();
     pdl_trigger();
+    if (threadIdx.x == 0) {
+        TPL_TRACE_AT(1);
+        TPL_TRACE_AT(2);
+        TPL_TRACE_AT(3);
+        TPL_TRACE_PUT(TR_OPERAND);
+    }
     const int64_t row = blockIdx.y;
     const int c = blockIdx.x * 256 + threadIdx.x;
     if (8 * c >= H) return;

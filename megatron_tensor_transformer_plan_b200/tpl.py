@@ -14,7 +14,8 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libtpl.so")
+# TPL_LIB may name the timeline-traced build (libtpl_trace.so) instead
+LIB_PATH = os.environ.get("TPL_LIB") or os.path.join(_HERE, "libtpl.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"libtpl.so not built at {LIB_PATH}; run megatron_tensor_transformer_plan_b200/build.py")
@@ -120,6 +121,24 @@ _sig("tpl_reduction_count", c_int64, _plan_p)
 _sig("tpl_decode_kernel_count", ctypes.c_int, _plan_p, c_int32, c_int32, c_int32, P(c_int32))
 _sig("tpl_reset_counters", None, _plan_p)
 _sig("tpl_last_device_error", ctypes.c_int, _plan_p, c_void_p)
+_sig("tpl_trace_read", ctypes.c_int, c_void_p, c_int32, P(c_int32))
+
+
+class tpl_trace_rec(ctypes.Structure):
+    _fields_ = [("tag", c_uint32), ("cta", c_uint32), ("smid", c_uint32), ("grid", c_uint32),
+                ("t", ctypes.c_uint64 * 4)]
+
+
+TRACE_TAGS = {1: "qkv", 2: "attention", 3: "o_proj", 4: "gate_up", 5: "down", 6: "operand", 7: "reduce"}
+
+
+def trace_read(max_records: int = 1 << 18):
+    """Records of the traced build since the last read, as a list of
+    (tag name, cta, smid, grid, [t0, t1, t2, t3] in ns)."""
+    buf = (tpl_trace_rec * max_records)()
+    n = c_int32()
+    check(tpl_trace_read(ctypes.cast(buf, c_void_p), max_records, ctypes.byref(n)), "tpl_trace_read")
+    return [(TRACE_TAGS.get(r.tag, str(r.tag)), r.cta, r.smid, r.grid, list(r.t)) for r in buf[:n.value]]
 _sig("tpl_status_string", ctypes.c_char_p, ctypes.c_int)
 
 

@@ -153,7 +153,10 @@ void tpl_plan_destroy(tpl_plan *plan);
  * 0 = keys staged through a per-warp shared-memory ring (the default for
  * query groups of at most 8 heads when every (shard, sequence, kv head) pair
  * gets at least two CTAs in one wave of SMs; other shapes use the other
- * kernel), 1 = keys streamed into registers (any shape).
+ * kernel), 1 = keys streamed into registers (any shape), 2 = the cache
+ * streamed by TMA into a shared-memory ring, every SM taking an equal share
+ * of all pairs' 64-key blocks (groups of at most 8 heads and S >= 1; other
+ * cases as 0).
  * TPL_OPT_PREFILL_SPLIT chooses, per prefill projection, whether its
  * activation operand is carried as two bf16 parts (hi + lo, about 16
  * mantissa bits, two products per tile) or one (rounded to bf16, one
@@ -381,8 +384,8 @@ int tpl_attn_decode(tpl_plan *plan, const tpl_kv *kv, const float *q, const floa
  *     (counters), 8*pairs*n*g and 512*pairs*n*g bytes, pairs = B*n_kv, n the
  *     CTAs per pair of that geometry (the register-streamed kernel: about
  *     1024/pairs key-range splits, at least 128 keys each, four per CTA; the
- *     staged kernel: at most floor(SMs/pairs)).  The 70B shapes need about
- *     1 MB.
+ *     staged kernel: at most floor(SMs/pairs); the TMA-streamed kernel: at
+ *     most ceil(min(SMs, 160)/pairs) + 1).  The 70B shapes need about 1 MB.
  *   - The first call on a device looks up the array's device address (with
  *     that device current); make that first call before any stream capture.
  *   - Every call uses the same array, and it keeps the previous call's

@@ -7,6 +7,7 @@
 #include <cstring>
 
 #include "tpl_attn.cuh"
+#include "tpl_attn_tma.cuh"
 #include "tpl_common.cuh"
 #include "tpl_gemv.cuh"
 #include "tpl_gemv_tc.cuh"
@@ -417,25 +418,79 @@ int run_qkv(Ctx &c, const char *packed, const tpl_kv *kv, const void *x, float *
 
 bool g_stg_attr[64];
 
-// Which decode attention kernel runs and its split geometry: the staged
-// kernel for groups of at most 8 heads with at least two CTAs per pair in one
-// wave (where it measured faster; with one CTA per pair the register-streamed
-// kernel's finer splits win), else the register-streamed kernel.
-int attn_select(const tpl_plan *p, int B, int64_t keys, AttnGeom *g, bool *staged) {
+// Which decode attention kernel runs and its split geometry.
+//   TPL_OPT_DECODE_ATTN 0 (default): the staged kernel for groups of at most
+//     8 heads with at least two CTAs per pair in one wave (where it measured
+//     faster; with one CTA per pair the register-streamed kernel's finer
+//     splits win), else the register-streamed kernel;
+//   1: the register-streamed kernel;
+//   2: the TMA-streamed kernel (groups of at most 8 heads, at least one
+//      cached key), else as 0.
+enum { ATTN_REG = 0, ATTN_STAGED = 1, ATTN_TMA = 2 };
+int attn_select(const tpl_plan *p, int B, int64_t keys, AttnGeom *g, int *kind) {
     const int sms = num_sms_current();
     if (sms <= 0) return TPL_ECUDA;
-    *staged = p->attn_decode_mode == 0 && p->g <= 8 && 2 * B * p->d.n_kv_heads <= sms;
-    if (*staged) attn_geom_staged(B, p->d.n_kv_heads, keys, sms, g);
-    else attn_geom(B, p->d.n_kv_heads, keys, g);
+    if (p->attn_decode_mode == 2 && p->g <= kAmMaxG && keys >= 1 && keys <= 0x7fffffffll) {
+        attn_geom_tma(B, p->d.n_kv_heads, keys, sms, g);
+        *kind = ATTN_TMA;
+    } else if (p->attn_decode_mode != 1 && p->g <= 8 && 2 * B * p->d.n_kv_heads <= sms) {
+        attn_geom_staged(B, p->d.n_kv_heads, keys, sms, g);
+        *kind = ATTN_STAGED;
+    } else {
+        attn_geom(B, p->d.n_kv_heads, keys, g);
+        *kind = ATTN_REG;
+    }
     if (g->pairs > kMaxPairs) return TPL_EUNSUPPORTED;
     return TPL_OK;
 }
 
+// CTA partials per pair the chosen kernel writes (sizes its scratch).
+int attn_cpp(const AttnGeom &g, int kind) { return kind == ATTN_TMA ? g.cpp_max : g.nsplit / kAttnWarps; }
+
+bool g_am_attr[64];
+
 // Fill the launch arguments (everything except the scratch pointers) and
 // launch the kernel attn_select chose.
 int attn_launch(const tpl_plan *p, const tpl_kv *kv, const float *q, const float *knew, const float *vnew, int B,
-                int64_t keys, void *o, const AttnGeom &g, bool staged, unsigned *tickets, float *part_ml,
+                int64_t keys, void *o, const AttnGeom &g, int kind, unsigned *tickets, float *part_ml,
                 float *part_o, cudaStream_t st) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return TPL_ECUDA;
+    const float scale_log2 = 1.4426950408889634f / sqrtf((float)p->d.head_dim);
+    if (kind == ATTN_TMA) {
+        AttnTmaArgs a;
+        std::memset(&a, 0, sizeof(a));
+        const uint64_t sb = (uint64_t)p->t * kv->batch_cap;
+        int rc = make_kv_map(&a.tm_k, kv->k, (uint64_t)keys, (uint64_t)p->nkv_s, sb, (uint64_t)kv->seq_cap, kAmKeys);
+        if (rc == TPL_OK)
+            rc = make_kv_map(&a.tm_v, kv->v, (uint64_t)keys, (uint64_t)p->nkv_s, sb, (uint64_t)kv->seq_cap, kAmKeys);
+        if (rc != TPL_OK) return rc;
+        a.q = q;
+        a.B = B;
+        a.nq = p->d.n_q_heads;
+        a.nkv_s = p->nkv_s;
+        a.g = p->g;
+        a.batch_cap = kv->batch_cap;
+        a.keys = (int)keys;
+        a.nb = g.nb;
+        a.U = (int64_t)g.pairs * g.nb;
+        a.k_new = knew;
+        a.v_new = vnew;
+        a.scale_log2 = scale_log2;
+        a.part_o = part_o;
+        a.part_ml = part_ml;
+        a.cpp_max = g.cpp_max;
+        a.tickets = tickets;
+        a.o = o;
+        a.o_f32 = p->f32;
+        if (!g_am_attr[dev]) {
+            if (cudaFuncSetAttribute(attn_decode_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)kAmSmem) != cudaSuccess)
+                return TPL_ECUDA;
+            g_am_attr[dev] = true;
+        }
+        return cuda_rc(launch_pdl(attn_decode_tma_kernel, g.grid, kAmThreads, kAmSmem, st, a));
+    }
     AttnArgs a;
     std::memset(&a, 0, sizeof(a));
     a.q = q;
@@ -452,16 +507,14 @@ int attn_launch(const tpl_plan *p, const tpl_kv *kv, const float *q, const float
     a.v_new = vnew;
     a.nsplit = g.nsplit;
     a.kps = g.kps;
-    a.scale_log2 = 1.4426950408889634f / sqrtf((float)p->d.head_dim);
+    a.scale_log2 = scale_log2;
     a.part_o = part_o;
     a.part_ml = part_ml;
     a.tickets = tickets;
     a.o = o;
     a.o_f32 = p->f32;
     const int grid = g.pairs * (g.nsplit / kAttnWarps);
-    if (staged) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return TPL_ECUDA;
+    if (kind == ATTN_STAGED) {
         if (!g_stg_attr[dev]) {
             if (cudaFuncSetAttribute(attn_decode_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)kStgSmem) != cudaSuccess)
@@ -478,10 +531,10 @@ int run_attn(Ctx &c, const tpl_kv *kv, const float *q, const float *knew, const 
     tpl_plan *p = c.p;
     const int64_t keys = knew ? c.S : c.S + 1;
     AttnGeom g;
-    bool staged = false;
-    int rc = attn_select(p, c.B, keys, &g, &staged);
+    int kind = 0;
+    int rc = attn_select(p, c.B, keys, &g, &kind);
     if (rc != TPL_OK) return rc;
-    return attn_launch(p, kv, q, knew, vnew, c.B, keys, o, g, staged,
+    return attn_launch(p, kv, q, knew, vnew, c.B, keys, o, g, kind,
                        reinterpret_cast<unsigned *>(c.ws + c.L.tickets) + kTicketAttn,
                        reinterpret_cast<float *>(c.ws + c.L.part_ml), reinterpret_cast<float *>(c.ws + c.L.part_o),
                        c.st);
@@ -946,10 +999,10 @@ extern "C" int tpl_attn_decode_static(tpl_plan *p, const tpl_kv *kv, const float
     // the same kernel and split geometry tpl_attn_decode chooses, so the two
     // calls give identical bits
     AttnGeom g;
-    bool staged = false;
-    if ((rc = attn_select(p, B, keys, &g, &staged)) != TPL_OK) return rc;
+    int kind = 0;
+    if ((rc = attn_select(p, B, keys, &g, &kind)) != TPL_OK) return rc;
     const size_t off_ml = round256((size_t)g.pairs * sizeof(unsigned));
-    const size_t cpp = (size_t)g.nsplit / kAttnWarps;  // partials are per CTA
+    const size_t cpp = (size_t)attn_cpp(g, kind);  // partials are per CTA
     const size_t off_o = off_ml + round256((size_t)g.pairs * cpp * p->g * 2 * sizeof(float));
     const size_t need = off_o + round256((size_t)g.pairs * cpp * p->g * p->d.head_dim * sizeof(float));
     if (need > TPL_ATTN_STATIC_SCRATCH_BYTES) return TPL_ENOMEM;
@@ -966,6 +1019,6 @@ extern "C" int tpl_attn_decode_static(tpl_plan *p, const tpl_kv *kv, const float
     char *scratch = static_cast<char *>(base);
     // The arrival counters must start at zero.
     if (cudaMemsetAsync(scratch, 0, (size_t)g.pairs * sizeof(unsigned), st) != cudaSuccess) return TPL_ECUDA;
-    return attn_launch(p, kv, q, k_new, v_new, B, keys, o, g, staged, reinterpret_cast<unsigned *>(scratch),
+    return attn_launch(p, kv, q, k_new, v_new, B, keys, o, g, kind, reinterpret_cast<unsigned *>(scratch),
                        reinterpret_cast<float *>(scratch + off_ml), reinterpret_cast<float *>(scratch + off_o), st);
 }

@@ -92,7 +92,16 @@ int gemv_geom(int N, int nseg, int Kseg, int B, int xbytes, int num_sms, GemvGeo
 
 struct AttnGeom {
     int pairs, nsplit, kps;  // pairs = B * n_kv; splits per pair; keys per split
+    // the TMA-streamed kernel: blocks of kAttnTmaKeys keys per pair, CTAs of
+    // the launch, CTAs per pair at most (sizes the partials)
+    int nb = 0, grid = 0, cpp_max = 0;
 };
+constexpr int kAttnTmaKeys = 64;       // keys per block of the TMA-streamed decode attention
+constexpr int kAttnTmaMaxCtas = 160;   // its CTAs per launch at most
+// Geometry of the TMA-streamed kernel: grid = min(sms, kAttnTmaMaxCtas,
+// pairs * nb) CTAs each taking an equal share of the pairs' blocks; a pair
+// spans at most ceil(grid / pairs) + 1 CTAs.
+void attn_geom_tma(int B, int nkv, int64_t keys, int sms, AttnGeom *a);
 // keys: keys covered by the splits (S when the new token is added in the
 // combine, S + 1 when it is read from the cache).
 void attn_geom(int B, int nkv, int64_t keys, AttnGeom *a);

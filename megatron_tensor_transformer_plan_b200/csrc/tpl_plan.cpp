@@ -126,6 +126,17 @@ void attn_geom_staged(int B, int nkv, int64_t keys, int sms, AttnGeom *a) {
     a->kps = (int)((kps + 15) / 16 * 16);
 }
 
+void attn_geom_tma(int B, int nkv, int64_t keys, int sms, AttnGeom *a) {
+    a->pairs = B * nkv;
+    a->nb = (int)((keys + kAttnTmaKeys - 1) / kAttnTmaKeys);
+    const int64_t U = (int64_t)a->pairs * a->nb;
+    int64_t grid = std::min<int64_t>(std::min(sms, kAttnTmaMaxCtas), U);
+    a->grid = (int)std::max<int64_t>(grid, 1);
+    a->cpp_max = std::min(a->grid, (a->grid + a->pairs - 1) / a->pairs + 1);
+    a->nsplit = 0;
+    a->kps = kAttnTmaKeys;
+}
+
 int ws_layout(const tpl_plan *p, int B, int64_t S, WsLayout *w) {
     if (B <= 0 || S < 0) return TPL_EINVAL;
     const tpl_dims &d = p->d;
@@ -153,9 +164,13 @@ int ws_layout(const tpl_plan *p, int B, int64_t S, WsLayout *w) {
     AttnGeom sg, sg1;  // the staged kernel's splits, for the largest SM count
     attn_geom_staged(B, d.n_kv_heads, S, kAttnSmsBound, &sg);
     attn_geom_staged(B, d.n_kv_heads, S + 1, kAttnSmsBound, &sg1);
-    const size_t nsp = (size_t)std::max(std::max(ag.nsplit, ag1.nsplit), std::max(sg.nsplit, sg1.nsplit));
-    w->part_o = take((size_t)ag.pairs * (nsp / kAttnWarps) * p->g * d.head_dim * 4);
-    w->part_ml = take((size_t)ag.pairs * (nsp / kAttnWarps) * p->g * 2 * 4);
+    AttnGeom tg;  // the TMA-streamed kernel's CTAs per pair, for the largest grid
+    attn_geom_tma(B, d.n_kv_heads, S + 1, kAttnTmaMaxCtas, &tg);
+    const size_t cpp = std::max((size_t)std::max(std::max(ag.nsplit, ag1.nsplit), std::max(sg.nsplit, sg1.nsplit)) /
+                                    kAttnWarps,
+                                (size_t)tg.cpp_max);
+    w->part_o = take((size_t)ag.pairs * cpp * p->g * d.head_dim * 4);
+    w->part_ml = take((size_t)ag.pairs * cpp * p->g * 2 * 4);
     // cross-CTA partials: the largest over the four matrix-vector steps
     size_t gp = 0;
     GemvGeom gg;
@@ -276,7 +291,7 @@ int tpl_plan_set_option(tpl_plan *p, int32_t option, int32_t value) {
         return TPL_OK;
     }
     if (option == TPL_OPT_DECODE_ATTN) {
-        if (value != 0 && value != 1) return TPL_EINVAL;
+        if (value != 0 && value != 1 && value != 2) return TPL_EINVAL;
         p->attn_decode_mode = value;
         return TPL_OK;
     }

@@ -53,4 +53,23 @@ inline int make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t ro
     return r == CUDA_SUCCESS ? TPL_OK : TPL_EINVAL;
 }
 
+// The bf16 KV cache of one layer, [t][batch_cap][n_kv/t][seq_cap][128], as a
+// 4-D map (128 dims, `keys` rows, n_kv/t, t * batch_cap): the rows at or past
+// `keys` read as 0, so a block that runs past the cache length needs no
+// masking of its values.  Boxes of 64 dims x box_keys rows, 128-byte swizzle.
+inline int make_kv_map(CUtensorMap *m, const void *base, uint64_t keys, uint64_t nkv_s, uint64_t sb, uint64_t seq_cap,
+                       uint32_t box_keys) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return TPL_ECUDA;
+    if (((uintptr_t)base & 15u) || keys == 0) return TPL_EINVAL;
+    const cuuint64_t gdim[4] = {128, keys, nkv_s, sb};
+    const cuuint64_t gstr[3] = {256, seq_cap * 256, nkv_s * seq_cap * 256};
+    const cuuint32_t box[4] = {64, box_keys, 1, 1};
+    const cuuint32_t es[4] = {1, 1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), gdim, gstr, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? TPL_OK : TPL_EINVAL;
+}
+
 }  // namespace tpl

@@ -61,11 +61,12 @@ def time_calls(fn, copies, iters, stream):
     return statistics.median(a.elapsed_time(b) for a, b in ts) * 1e3  # us
 
 
-def run_layer(tpl, H, nq, nkv, F, t, B, S, iters, mode, flags=None, mlp_only=False, gemv_mode=4):
+def run_layer(tpl, H, nq, nkv, F, t, B, S, iters, mode, flags=None, mlp_only=False, gemv_mode=4, attn_mode=0):
     dev = torch.device("cuda")
     flags = (tpl.TPL_NORM | tpl.TPL_RESIDUAL) if flags is None else flags
     plan = tpl.Plan(tpl.make_dims(H, nq, nkv, 128, F, 1, 1e-5, flags), t)
     plan.set_option(tpl.TPL_OPT_GEMV_MODE, gemv_mode)
+    plan.set_option(tpl.TPL_OPT_DECODE_ATTN, attn_mode)
     nbytes = layer_bytes(H, nq, nkv, 128, F, B, S, mlp_only)
     ncopies = max(1, min(8, -(-4 * L2_BYTES // nbytes)))
     copies = []
@@ -100,6 +101,7 @@ def main() -> None:
     ap.add_argument("--only", default="")
     ap.add_argument("--gemv-mode", type=int, default=4, help="TPL_OPT_GEMV_MODE of the plan (4: the default)")
     ap.add_argument("--rope", action="store_true", help="rotary embedding on (TPL_ROPE)")
+    ap.add_argument("--attn-mode", type=int, default=0, help="TPL_OPT_DECODE_ATTN of the plan (0: the default)")
     args = ap.parse_args()
     build.build()
     from megatron_tensor_transformer_plan_b200 import tpl
@@ -125,10 +127,11 @@ def main() -> None:
                 flags = tpl.TPL_NORM | tpl.TPL_RESIDUAL | tpl.TPL_ROPE
             us, nbytes, ncopies, rc = run_layer(tpl, c["H"], c["nq"], c["nkv"], c["F"], c["t"], c["B"], c["S"],
                                                  args.iters, mode, flags, c.get("mlp_only", False),
-                                                 args.gemv_mode)
+                                                 args.gemv_mode, args.attn_mode)
             gbs = nbytes / (us * 1e-6) / 1e9
             tok_s = c["B"] / (us * 1e-6)
-            print(json.dumps({"workload": name, "gemv_mode": args.gemv_mode, "rope": args.rope, "t": c["t"],
+            print(json.dumps({"workload": name, "gemv_mode": args.gemv_mode, "attn_mode": args.attn_mode,
+                              "rope": args.rope, "t": c["t"],
                               "B": c["B"], "S": c["S"],
                               "reduce": mode,
                               "us_per_layer": round(us, 2), "tokens_per_s_per_layer": round(tok_s, 1),

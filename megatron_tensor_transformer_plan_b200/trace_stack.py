@@ -15,7 +15,7 @@ before it (the last CTA's exit):
 Medians over the layers of the stack.
 
     python -m megatron_tensor_transformer_plan_b200.trace_stack [--layers N] [--t T] [--batch B] [--kv S]
-        [--shape 70b|7b] [--gemv-mode M] [--steps K]
+        [--shape 70b|7b] [--gemv-mode M] [--attn-mode A] [--steps K]
 """
 from __future__ import annotations
 
@@ -79,6 +79,7 @@ def main() -> None:
     ap.add_argument("--batch", type=int, default=4)
     ap.add_argument("--kv", type=int, default=4096)
     ap.add_argument("--gemv-mode", type=int, default=4)
+    ap.add_argument("--attn-mode", type=int, default=0, help="TPL_OPT_DECODE_ATTN of the plan (0: the default)")
     ap.add_argument("--steps", type=int, default=3)
     ap.add_argument("--json", default="")
     args = ap.parse_args()
@@ -89,6 +90,7 @@ def main() -> None:
     dev = torch.device("cuda")
     plan = tpl.Plan(tpl.make_dims(H, NQ, NKV, D, F, NL, 1e-5, tpl.TPL_NORM | tpl.TPL_RESIDUAL), T)
     plan.set_option(tpl.TPL_OPT_GEMV_MODE, args.gemv_mode)
+    plan.set_option(tpl.TPL_OPT_DECODE_ATTN, args.attn_mode)
     packed, kvs, keep = [], [], []
     for l in range(NL):
         w = synth.layer_weights(H, NQ, NKV, D, F, seed=0, layer=l, device=dev)
@@ -113,6 +115,7 @@ def main() -> None:
             per_kind.setdefault(r["kernel"], []).append(r)
     assert plan.last_device_error() == tpl.TPL_OK
     out = {"shape": args.shape, "t": T, "batch": B, "kv": S, "layers": NL, "gemv_mode": args.gemv_mode,
+           "attn_mode": args.attn_mode,
            "kernels": {}}
     order = ["operand", "qkv", "attention", "o_proj", "gate_up", "down"]
     print(f"{'kernel':10s} {'n':>4s} {'exposed':>8s} {'release':>8s} {'loop':>8s} {'tail':>8s} {'spread':>8s}  (us)")

@@ -231,11 +231,12 @@ def test_repeated_calls_are_deterministic(gpu):
 @pytest.mark.parametrize("case", [(1024, 16, 8, 2816, 8, 4, 700), (512, 8, 2, 1376, 2, 3, 37),
                                   (256, 4, 4, 704, 4, 1, 0)])
 def test_decode_attention_kernels_agree(gpu, case):
-    """The staged attention kernel (default) and the register-streamed one
-    (TPL_OPT_DECODE_ATTN 1): both against the oracle, and close to each other."""
+    """The staged attention kernel (default), the register-streamed one
+    (TPL_OPT_DECODE_ATTN 1) and the TMA-streamed one (2): each against the
+    oracle, and close to each other."""
     H, nq, nkv, F, t, B, S = case
     outs = []
-    for mode in (0, 1):
+    for mode in (0, 1, 2):
         L = make_layer(H, nq, nkv, 128, F, t, B, S, S_cap=S + 3)
         L.plan.set_option(tpl.TPL_OPT_DECODE_ATTN, mode)
         ref_y, tr = oracle_decode(L)
@@ -244,3 +245,42 @@ def test_decode_attention_kernels_agree(gpu, case):
         assert_close_rel(to_np(st["y"]), ref_y, what=f"y (mode {mode})")
         outs.append(to_np(st["attn"]))
     assert_close_rel(outs[0], outs[1], tol=8e-3, what="staged vs register attention")
+    assert_close_rel(outs[0], outs[2], tol=8e-3, what="staged vs TMA-streamed attention")
+
+
+TMA_ATTN_CASES = [
+    # H, nq, nkv, F, t, B, S, S_cap extra: blocks of 64 keys laid end to end over every SM
+    (1024, 16, 8, 2816, 8, 4, 4096, 1),    # the stack's attention shape at small hidden: 32 pairs
+    (1024, 16, 8, 2816, 4, 16, 1000, 5),   # 128 pairs, ragged last block, several pairs per CTA
+    (512, 8, 8, 1024, 2, 3, 1, 1),         # one cached key (a block of one valid row), g = 1
+    (512, 8, 2, 1376, 2, 2, 63, 2),        # 63 keys: one block short of a full one
+    (512, 8, 2, 1376, 2, 2, 65, 1),        # 65 keys: a full block and a block of one key
+    (768, 12, 4, 1056, 4, 5, 129, 9),      # g = 3
+    (1024, 8, 1, 1024, 1, 2, 5000, 3),     # one kv head per sequence: a pair spans many CTAs
+    (2048, 32, 32, 2048, 1, 20, 300, 1),   # 640 pairs: many pairs per CTA
+]
+
+
+@pytest.mark.parametrize("case", TMA_ATTN_CASES)
+def test_tma_attention_kernel(gpu, case):
+    """The TMA-streamed decode attention (TPL_OPT_DECODE_ATTN 2) at ragged
+    cache lengths and pair counts from one CTA per many pairs to many CTAs per
+    pair, against the oracle, with the new token given separately and read
+    from cache slot S."""
+    H, nq, nkv, F, t, B, S, extra = case
+    L = make_layer(H, nq, nkv, 128, F, t, B, S, S_cap=S + extra, seed=17)
+    L.plan.set_option(tpl.TPL_OPT_DECODE_ATTN, 2)
+    ref_y, tr = oracle_decode(L)
+    st = run_steps(L)
+    assert_close_rel(to_np(st["attn"]), tr["attn"], what="attention (new token separate)")
+    assert_close_rel(to_np(st["y"]), ref_y, what="y")
+    # the new token read from cache slot S (written by the QKV step above, bf16):
+    # against the register-streamed kernel reading the same cache
+    o2 = torch.empty_like(st["attn"])
+    L.plan.attn_decode(L.kv, st["q"], S, o2, L.ws)
+    L.plan.set_option(tpl.TPL_OPT_DECODE_ATTN, 1)
+    o1 = torch.empty_like(st["attn"])
+    L.plan.attn_decode(L.kv, st["q"], S, o1, L.ws)
+    torch.cuda.synchronize()
+    assert_close_rel(to_np(o2), to_np(o1), tol=8e-3, what="attention (new token from the cache)")
+    assert L.plan.last_device_error() == tpl.TPL_OK

@@ -550,6 +550,18 @@ CONFIG_CASES = [
 ]
 
 
+def attach_overheads(rows):
+    """Give every fused row with t > 1 its time over the same workload's
+    unsharded (t = 1, fused) row at the same batch: the benchmark spec's
+    fused-reduction overhead."""
+    base = {(r["workload"], r["batch"]): r["us_per_layer"] for r in rows if r["t"] == 1 and r["reduce"] == "fused"}
+    for r in rows:
+        b = base.get((r["workload"], r["batch"]))
+        if b is not None and r["reduce"] == "fused" and r["t"] > 1:
+            r["overhead_vs_t1"] = r["us_per_layer"] / b - 1.0
+    return rows
+
+
 def run_configs(tpl, peak, peak_kind, gpu_index, iters):
     """Microseconds per layer, algorithmic GB/s and fraction of the copy
     peak for each case, and each shard layout's fused time against the same
@@ -568,12 +580,7 @@ def run_configs(tpl, peak, peak_kind, gpu_index, iters):
                      "us_per_layer": us, "tokens_per_s": B / (us * 1e-6), "algorithmic_bytes": nbytes,
                      "gb_s": gbs, "frac": gbs / peak, "copies_rotated": ncopies})
     clk = clocks.stop()
-    base = {(r["workload"].split(":")[0], r["batch"]): r["us_per_layer"] for r in rows
-            if r["t"] == 1 and r["reduce"] == "fused"}
-    for r in rows:
-        b = base.get((r["workload"].split(":")[0], r["batch"]))
-        if b is not None and r["reduce"] == "fused" and r["t"] > 1:
-            r["overhead_vs_t1"] = r["us_per_layer"] / b - 1.0
+    attach_overheads(rows)
     return {"peak_gbs": peak, "peak_kind": peak_kind + " (burst copy)",
             "timing": f"CUDA events around each layer call, median of {iters} after 3 warm-ups",
             "bytes": "every weight once, the K/V cache once, new K/V, x and y",

@@ -11,16 +11,20 @@
 //
 // Per CTA: one producer thread issues 4-D TMA copies of the K and V blocks
 // (two 64-dimension boxes each, 128-byte swizzle) into a ring of kAmStages
-// stages; kAmWarps consumer warps each take 16 keys of every stage on the
-// tensor cores (mma.sync m16n8k16, bf16 operands read with ldmatrix from the
-// swizzled tiles): S = Q K^T with the g <= 8 query heads of the kv head as
-// rows 0-7 (bf16 hi parts) and 8-15 (lo parts), an online softmax per head,
-// O += P V with P carried the same way.  At the end of a segment the warps
-// merge in warp order, the CTA writes its partial (max, sum, unnormalised
-// output) for the pair, and the last CTA of the pair to arrive (an arrival
-// counter, no waiting) adds the partials in CTA order, then the new token's
-// key/value in fp32.  Keys at or past the cache length read as zero (the
-// tensor maps end there) and their logits are masked.
+// stages; two groups of four consumer warps take alternate stages, each warp
+// 16 keys of its group's stages, on the tensor cores (mma.sync m16n8k16, bf16
+// operands read with ldmatrix from the swizzled tiles): S = Q K^T with the
+// g <= 8 query heads of the kv head as rows 0-7 (bf16 hi parts) and 8-15 (lo
+// parts), an online softmax per head whose running maximum is raised only when
+// a step exceeds it by more than 2^8 (so the output is rarely rescaled), and
+// O += P V with P carried the same way.  Two groups keep two warps' dependent
+// chains in flight on every SM sub-partition.  At the end of a segment the
+// second group's warps hand their state to the first group's (same lanes),
+// the first group merges in warp order, the CTA writes its partial (max, sum,
+// unnormalised output) for the pair, and the last CTA of the pair to arrive
+// (an arrival counter, no waiting) adds the partials in CTA order, then the
+// new token's key/value in fp32.  Keys at or past the cache length read as
+// zero (the tensor maps end there) and their logits are masked.
 //
 // The cached keys 0..S-1 are not written by the preceding kernel (it writes
 // slot S), so when the new token is given separately the first stages are
@@ -38,19 +42,22 @@
 
 namespace tpl {
 
-constexpr int kAmWarps = 4;                      // consumer warps; warp kAmWarps is the producer
+constexpr int kAmGroupWarps = 4;                 // warps per consumer group: 16 keys of a stage each
+constexpr int kAmGroups = 2;                     // consumer groups, taking alternate stages
+constexpr int kAmWarps = kAmGroupWarps * kAmGroups;  // consumer warps; warp kAmWarps is the producer
 constexpr int kAmThreads = (kAmWarps + 1) * 32;
-constexpr int kAmKeys = 16 * kAmWarps;           // keys per stage, 16 per consumer warp
+constexpr int kAmKeys = 16 * kAmGroupWarps;      // keys per stage, 16 per warp of a group
 static_assert(kAmKeys == kAttnTmaKeys, "block size shared with the host geometry");
 constexpr int kAmBox = kAmKeys * 64 * 2;         // one box: kAmKeys keys x 64 dims, bf16 (8 KB)
 constexpr int kAmStage = 4 * kAmBox;             // K dims 0-63, K dims 64-127, V dims 0-63, V dims 64-127
 constexpr int kAmStages = 6;
 constexpr int kAmMaxG = 8;
 constexpr int kAmMaxCtas = kAttnTmaMaxCtas;      // CTAs per launch at most (bounds the CTAs per pair)
-constexpr int kAmMergeBytes = kAmWarps * kAmMaxG * 128 * 4;  // warp outputs, reused by the pair combine
+constexpr int kAmMergeBytes = kAmGroupWarps * kAmMaxG * 128 * 4;  // one group's outputs, reused by the pair combine
 constexpr int kAmBarBytes = 1024;
 constexpr size_t kAmSmem = (size_t)kAmStages * kAmStage + kAmMergeBytes + kAmBarBytes + 1024;
 static_assert(kAmSmem <= 232448, "shared memory per block");
+constexpr float kAmLazy = 8.0f;  // the running maximum (log2 units) is raised only past this margin
 
 struct AttnTmaArgs {
     CUtensorMap tm_k, tm_v;  // 4-D (128 dims, keys, n_kv/t, t * batch_cap), box (64, kAmKeys, 1, 1)
@@ -118,7 +125,7 @@ __global__ void __launch_bounds__(kAmThreads, 1) attn_decode_tma_kernel(const __
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kAmWarps);
+            mbar_init(&empty[s], kAmGroupWarps);  // the four warps of the stage's group
         }
         s_flag[0] = 0;
         s_flag[1] = 0;
@@ -162,11 +169,13 @@ __global__ void __launch_bounds__(kAmThreads, 1) attn_decode_tma_kernel(const __
             s_flag[2] = i;
         }
     } else {
-        // ---- consumers: warp w takes keys 16w .. 16w+15 of every stage ----
+        // ---- consumers: group grp takes the stages i with i % kAmGroups == grp;
+        //      warp wl of a group takes keys 16 wl .. 16 wl + 15 of them ----
         pdl_wait();
         if (threadIdx.x == 0) TPL_TRACE_AT(1);
         const int gid = lane >> 2, c = lane & 3;
-        const int tid = threadIdx.x;  // 0..127: one head dimension each in the merge
+        const int grp = warp / kAmGroupWarps, wl = warp % kAmGroupWarps;
+        const int tid = threadIdx.x;  // group 0: 0..127, one head dimension each in the merge
         bool dead = false;
         int i = 0;
         while (i < n) {
@@ -202,6 +211,7 @@ __global__ void __launch_bounds__(kAmThreads, 1) attn_decode_tma_kernel(const __
             for (int t = 0; t < 16; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
             float m_a = -INFINITY, l_a = 0.f;
             for (int e = 0; e < seg_n; ++e, ++i) {
+                if (i % kAmGroups != grp) continue;
                 const int s = i % NS;
                 if (!dead)
                     dead = !__all_sync(0xffffffffu, !s_flag[0] && mbar_wait(&full[s], (unsigned)(i / NS) & 1u));
@@ -210,14 +220,14 @@ __global__ void __launch_bounds__(kAmThreads, 1) attn_decode_tma_kernel(const __
                     continue;
                 }
                 const int blk = (int)((u0 + i) % a.nb);
-                const int kb = blk * kAmKeys + 16 * warp;  // first key of this warp's 16
+                const int kb = blk * kAmKeys + 16 * wl;  // first key of this warp's 16
                 if (kb < a.keys) {
                     const unsigned char *st = sm + s * kAmStage;
                     const unsigned char *Klo = st, *Khi = st + kAmBox, *Vlo = st + 2 * kAmBox,
                                         *Vhi = st + 3 * kAmBox;
                     float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
                     {
-                        const int row = 16 * warp + (lane & 7) + ((lane >> 4) << 3);
+                        const int row = 16 * wl + (lane & 7) + ((lane >> 4) << 3);
                         const int half = (lane >> 3) & 1;
 #pragma unroll
                         for (int ks = 0; ks < 8; ++ks) {
@@ -237,23 +247,28 @@ __global__ void __launch_bounds__(kAmThreads, 1) attn_decode_tma_kernel(const __
                     float mx = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
                     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
                     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-                    const float mn = fmaxf(m_a, mx);  // finite: key kb is in range
-                    const float alpha = exp2f(m_a - mn);
-                    m_a = mn;
-                    const float p0 = exp2f(x0 - mn), p1 = exp2f(x1 - mn), p2 = exp2f(x2 - mn), p3 = exp2f(x3 - mn);
-                    l_a = l_a * alpha + ((p0 + p1) + (p2 + p3));
+                    // mx is finite: key kb is in range.  Raise the running
+                    // maximum only past the margin; until then p <= 2^kAmLazy.
+                    if (mx > m_a + kAmLazy) {
+                        const float alpha = exp2f(m_a - mx);  // 0 on the first step (m_a = -inf)
+                        m_a = mx;
+                        l_a *= alpha;
 #pragma unroll
-                    for (int t = 0; t < 16; ++t) {
-                        o[t][0] *= alpha;
-                        o[t][1] *= alpha;
-                        o[t][2] *= alpha;
-                        o[t][3] *= alpha;
+                        for (int t = 0; t < 16; ++t) {
+                            o[t][0] *= alpha;
+                            o[t][1] *= alpha;
+                            o[t][2] *= alpha;
+                            o[t][3] *= alpha;
+                        }
                     }
+                    const float p0 = exp2f(x0 - m_a), p1 = exp2f(x1 - m_a), p2 = exp2f(x2 - m_a),
+                                p3 = exp2f(x3 - m_a);
+                    l_a += (p0 + p1) + (p2 + p3);
                     const uint32_t ph0 = pack_bf16x2(p0, p1), ph2 = pack_bf16x2(p2, p3);
                     const uint32_t pl0 = pack_bf16x2(p0 - bf16lo(ph0), p1 - bf16hi(ph0));
                     const uint32_t pl2 = pack_bf16x2(p2 - bf16lo(ph2), p3 - bf16hi(ph2));
                     {
-                        const int row = 16 * warp + (lane & 7) + (((lane >> 3) & 1) << 3);
+                        const int row = 16 * wl + (lane & 7) + (((lane >> 3) & 1) << 3);
                         const int half = lane >> 4;
 #pragma unroll
                         for (int n2 = 0; n2 < 8; ++n2) {
@@ -277,103 +292,134 @@ __global__ void __launch_bounds__(kAmThreads, 1) attn_decode_tma_kernel(const __
             l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
             l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
 
-            // ---- merge the warps (ascending order), then the CTA's partial for the pair ----
-            if (gid < a.g) {
+            // ---- group 1 hands its state to group 0 (warp wl to warp wl, same lanes) ----
+            if (grp == 1 && gid < a.g) {
 #pragma unroll
                 for (int t = 0; t < 16; ++t) {
-                    s_o[(warp * kAmMaxG + gid) * D + 8 * t + 2 * c] = o[t][0];
-                    s_o[(warp * kAmMaxG + gid) * D + 8 * t + 2 * c + 1] = o[t][1];
+                    s_o[(wl * kAmMaxG + gid) * D + 8 * t + 2 * c] = o[t][0];
+                    s_o[(wl * kAmMaxG + gid) * D + 8 * t + 2 * c + 1] = o[t][1];
                 }
                 if (c == 0) {
-                    s_ml[(warp * kAmMaxG + gid) * 2 + 0] = m_a;
-                    s_ml[(warp * kAmMaxG + gid) * 2 + 1] = l_a;
+                    s_ml[(wl * kAmMaxG + gid) * 2 + 0] = m_a;
+                    s_ml[(wl * kAmMaxG + gid) * 2 + 1] = l_a;
                 }
             }
             asm volatile("bar.sync 1, %0;" ::"n"(kAmWarps * 32) : "memory");
-            const int cf = am_cta_of(a.U, G, (int64_t)pair * a.nb);
-            const int cl = am_cta_of(a.U, G, (int64_t)pair * a.nb + a.nb - 1);
-            const int n_p = cl - cf + 1;
-            const int64_t cbase = ((int64_t)pair * a.cpp_max + (cta - cf)) * a.g;
-            for (int hrow = 0; hrow < a.g; ++hrow) {
-                float M = -INFINITY;
+            if (grp == 0 && gid < a.g) {
+                const float m1 = s_ml[(wl * kAmMaxG + gid) * 2 + 0], l1 = s_ml[(wl * kAmMaxG + gid) * 2 + 1];
+                const float M = fmaxf(m_a, m1);
+                const float w0 = m_a == -INFINITY ? 0.f : exp2f(m_a - M);
+                const float w1 = m1 == -INFINITY ? 0.f : exp2f(m1 - M);
 #pragma unroll
-                for (int w = 0; w < kAmWarps; ++w) M = fmaxf(M, s_ml[(w * kAmMaxG + hrow) * 2]);
-                float num = 0.f, den = 0.f;
-#pragma unroll
-                for (int w = 0; w < kAmWarps; ++w) {
-                    const float mi = s_ml[(w * kAmMaxG + hrow) * 2];
-                    const float wt = mi == -INFINITY ? 0.f : exp2f(mi - M);
-                    num += wt * s_o[(w * kAmMaxG + hrow) * D + tid];
-                    den += wt * s_ml[(w * kAmMaxG + hrow) * 2 + 1];
+                for (int t = 0; t < 16; ++t) {
+                    o[t][0] = o[t][0] * w0 + s_o[(wl * kAmMaxG + gid) * D + 8 * t + 2 * c] * w1;
+                    o[t][1] = o[t][1] * w0 + s_o[(wl * kAmMaxG + gid) * D + 8 * t + 2 * c + 1] * w1;
                 }
-                a.part_o[(cbase + hrow) * D + tid] = num;
-                if (tid == 0) {
-                    a.part_ml[(cbase + hrow) * 2 + 0] = M;
-                    a.part_ml[(cbase + hrow) * 2 + 1] = den;
-                }
-            }
-            __threadfence();
-            asm volatile("bar.sync 1, %0;" ::"n"(kAmWarps * 32) : "memory");
-            if (tid == 0) {
-                const unsigned prev = atomicAdd(&a.tickets[pair], 1u);
-                s_flag[1] = prev == (unsigned)(n_p - 1);
-                if (prev >= (unsigned)n_p) record_error(2u);
+                l_a = l_a * w0 + l1 * w1;
+                m_a = M;
             }
             asm volatile("bar.sync 1, %0;" ::"n"(kAmWarps * 32) : "memory");
-            if (s_flag[1]) {
-                // ---- the last CTA of the pair: partials in CTA order, then the new token ----
-                __threadfence();
-                float *s_mlp = s_o;                        // [n_p][g][2]
-                float *s_w = s_o + 2 * kAmMaxG * 160;      // [n_p][8]
-                float *s_M = s_misc, *s_den = s_misc + kAmMaxG, *s_new = s_misc + 2 * kAmMaxG;
-                const bool has_new = a.k_new != nullptr;
-                for (int x = tid; x < n_p * a.g * 2; x += kAmWarps * 32)
-                    s_mlp[x] = __ldcg(&a.part_ml[(int64_t)pair * a.cpp_max * a.g * 2 + x]);
-                if (has_new) {
-                    const float kd = a.k_new[((int64_t)b * (a.nq / a.g) + j) * D + tid];
-                    for (int hrow = 0; hrow < a.g; ++hrow) {
-                        float v = a.q[((int64_t)b * a.nq + (int64_t)j * a.g + hrow) * D + tid] * kd;
+            // ---- group 0 merges its warps (ascending order), then the CTA's partial for the pair ----
+            if (grp == 0 && gid < a.g) {
 #pragma unroll
-                        for (int o2 = 16; o2 > 0; o2 >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o2);
-                        if (lane == 0) s_red[warp * kAmMaxG + hrow] = v;
-                    }
+                for (int t = 0; t < 16; ++t) {
+                    s_o[(wl * kAmMaxG + gid) * D + 8 * t + 2 * c] = o[t][0];
+                    s_o[(wl * kAmMaxG + gid) * D + 8 * t + 2 * c + 1] = o[t][1];
                 }
-                asm volatile("bar.sync 1, %0;" ::"n"(kAmWarps * 32) : "memory");
-                if (tid < a.g) {
-                    const int hrow = tid;
-                    float nl = -INFINITY;
-                    if (has_new) {
-                        float v = 0.f;
-#pragma unroll
-                        for (int w = 0; w < kAmWarps; ++w) v += s_red[w * kAmMaxG + hrow];
-                        nl = v * a.scale_log2;
-                        s_new[hrow] = nl;
-                    }
-                    float M = nl;
-                    for (int x = 0; x < n_p; ++x) M = fmaxf(M, s_mlp[(x * a.g + hrow) * 2]);
-                    float den = 0.f;
-                    for (int x = 0; x < n_p; ++x) {
-                        const float mi = s_mlp[(x * a.g + hrow) * 2];
-                        const float wt = mi == -INFINITY ? 0.f : exp2f(mi - M);
-                        s_w[x * kAmMaxG + hrow] = wt;
-                        den += wt * s_mlp[(x * a.g + hrow) * 2 + 1];
-                    }
-                    if (has_new) den += exp2f(nl - M);
-                    s_M[hrow] = M;
-                    s_den[hrow] = den;
+                if (c == 0) {
+                    s_ml[(wl * kAmMaxG + gid) * 2 + 0] = m_a;
+                    s_ml[(wl * kAmMaxG + gid) * 2 + 1] = l_a;
                 }
-                asm volatile("bar.sync 1, %0;" ::"n"(kAmWarps * 32) : "memory");
+            }
+            asm volatile("bar.sync 1, %0;" ::"n"(kAmWarps * 32) : "memory");
+            if (grp == 0) {
+                const int cf = am_cta_of(a.U, G, (int64_t)pair * a.nb);
+                const int cl = am_cta_of(a.U, G, (int64_t)pair * a.nb + a.nb - 1);
+                const int n_p = cl - cf + 1;
+                const int64_t cbase = ((int64_t)pair * a.cpp_max + (cta - cf)) * a.g;
                 for (int hrow = 0; hrow < a.g; ++hrow) {
-                    float num = 0.f;
-                    const float *po = a.part_o + ((int64_t)pair * a.cpp_max * a.g + hrow) * D + tid;
-#pragma unroll 4
-                    for (int x = 0; x < n_p; ++x) num += s_w[x * kAmMaxG + hrow] * __ldcg(po + (int64_t)x * a.g * D);
-                    if (has_new)
-                        num += exp2f(s_new[hrow] - s_M[hrow]) * a.v_new[((int64_t)b * (a.nq / a.g) + j) * D + tid];
-                    store_act(a.o, a.o_f32, ((int64_t)b * a.nq + (int64_t)j * a.g + hrow) * D + tid,
-                              num / s_den[hrow]);
+                    float M = -INFINITY;
+#pragma unroll
+                    for (int w = 0; w < kAmGroupWarps; ++w) M = fmaxf(M, s_ml[(w * kAmMaxG + hrow) * 2]);
+                    float num = 0.f, den = 0.f;
+#pragma unroll
+                    for (int w = 0; w < kAmGroupWarps; ++w) {
+                        const float mi = s_ml[(w * kAmMaxG + hrow) * 2];
+                        const float wt = mi == -INFINITY ? 0.f : exp2f(mi - M);
+                        num += wt * s_o[(w * kAmMaxG + hrow) * D + tid];
+                        den += wt * s_ml[(w * kAmMaxG + hrow) * 2 + 1];
+                    }
+                    a.part_o[(cbase + hrow) * D + tid] = num;
+                    if (tid == 0) {
+                        a.part_ml[(cbase + hrow) * 2 + 0] = M;
+                        a.part_ml[(cbase + hrow) * 2 + 1] = den;
+                    }
                 }
-                if (tid == 0) atomicExch(&a.tickets[pair], 0u);
+                __threadfence();
+                asm volatile("bar.sync 2, %0;" ::"n"(kAmGroupWarps * 32) : "memory");
+                if (tid == 0) {
+                    const unsigned prev = atomicAdd(&a.tickets[pair], 1u);
+                    s_flag[1] = prev == (unsigned)(n_p - 1);
+                    if (prev >= (unsigned)n_p) record_error(2u);
+                }
+                asm volatile("bar.sync 2, %0;" ::"n"(kAmGroupWarps * 32) : "memory");
+                if (s_flag[1]) {
+                    // ---- the last CTA of the pair: partials in CTA order, then the new token ----
+                    __threadfence();
+                    float *s_mlp = s_o;                        // [n_p][g][2]
+                    float *s_w = s_o + 2 * kAmMaxG * 160;      // [n_p][8]
+                    float *s_M = s_misc, *s_den = s_misc + kAmMaxG, *s_new = s_misc + 2 * kAmMaxG;
+                    const bool has_new = a.k_new != nullptr;
+                    for (int x = tid; x < n_p * a.g * 2; x += kAmGroupWarps * 32)
+                        s_mlp[x] = __ldcg(&a.part_ml[(int64_t)pair * a.cpp_max * a.g * 2 + x]);
+                    if (has_new) {
+                        const float kd = a.k_new[((int64_t)b * (a.nq / a.g) + j) * D + tid];
+                        for (int hrow = 0; hrow < a.g; ++hrow) {
+                            float v = a.q[((int64_t)b * a.nq + (int64_t)j * a.g + hrow) * D + tid] * kd;
+#pragma unroll
+                            for (int o2 = 16; o2 > 0; o2 >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o2);
+                            if (lane == 0) s_red[wl * kAmMaxG + hrow] = v;
+                        }
+                    }
+                    asm volatile("bar.sync 2, %0;" ::"n"(kAmGroupWarps * 32) : "memory");
+                    if (tid < a.g) {
+                        const int hrow = tid;
+                        float nl = -INFINITY;
+                        if (has_new) {
+                            float v = 0.f;
+#pragma unroll
+                            for (int w = 0; w < kAmGroupWarps; ++w) v += s_red[w * kAmMaxG + hrow];
+                            nl = v * a.scale_log2;
+                            s_new[hrow] = nl;
+                        }
+                        float M = nl;
+                        for (int x = 0; x < n_p; ++x) M = fmaxf(M, s_mlp[(x * a.g + hrow) * 2]);
+                        float den = 0.f;
+                        for (int x = 0; x < n_p; ++x) {
+                            const float mi = s_mlp[(x * a.g + hrow) * 2];
+                            const float wt = mi == -INFINITY ? 0.f : exp2f(mi - M);
+                            s_w[x * kAmMaxG + hrow] = wt;
+                            den += wt * s_mlp[(x * a.g + hrow) * 2 + 1];
+                        }
+                        if (has_new) den += exp2f(nl - M);
+                        s_M[hrow] = M;
+                        s_den[hrow] = den;
+                    }
+                    asm volatile("bar.sync 2, %0;" ::"n"(kAmGroupWarps * 32) : "memory");
+                    for (int hrow = 0; hrow < a.g; ++hrow) {
+                        float num = 0.f;
+                        const float *po = a.part_o + ((int64_t)pair * a.cpp_max * a.g + hrow) * D + tid;
+#pragma unroll 4
+                        for (int x = 0; x < n_p; ++x)
+                            num += s_w[x * kAmMaxG + hrow] * __ldcg(po + (int64_t)x * a.g * D);
+                        if (has_new)
+                            num += exp2f(s_new[hrow] - s_M[hrow]) *
+                                   a.v_new[((int64_t)b * (a.nq / a.g) + j) * D + tid];
+                        store_act(a.o, a.o_f32, ((int64_t)b * a.nq + (int64_t)j * a.g + hrow) * D + tid,
+                                  num / s_den[hrow]);
+                    }
+                    if (tid == 0) atomicExch(&a.tickets[pair], 0u);
+                }
             }
             // the merge area is rewritten by the next segment
             asm volatile("bar.sync 1, %0;" ::"n"(kAmWarps * 32) : "memory");

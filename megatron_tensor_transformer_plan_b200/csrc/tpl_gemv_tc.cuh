@@ -118,6 +118,7 @@ struct GemvTcArgs {
     int gstride;        // floats per row of a piece: 16 * ceil(B / 16)
     unsigned *tickets;  // [tiles]
     int trace_row_tag;  // timeline tag of a row-parallel launch (traced builds)
+    int l2_pre;         // weight tiles after the first stages prefetched into L2 before the dependency wait
 };
 
 // Tokens 16*ch .. 16*ch+15 of one accumulator row: the hi column plus the
@@ -333,13 +334,19 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
             };
             const int n = (int)(u1 - u0);
             const int pre = n < NS ? n : NS;
-            // weight tiles of the first stages before the dependency wait
+            // weight tiles of the first stages before the dependency wait,
+            // and the next l2_pre tiles into L2 (weights never depend on the
+            // previous kernel; the stream resumes from L2 after the wait)
             restart();
             for (int i = 0; i < pre; ++i, advance()) {
                 unsigned char *st = sm + i * STAGE;
                 mbar_expect_tx(&full[i], STAGE);
                 if (a.w3d) tma_load_3d(st, &a.tm_w, kb * kGtK, tile * kGtRows, seg, &full[i]);
                 else tma_load_2d(st, &a.tm_w, kb * kGtK, tile * kGtRows, &full[i]);
+            }
+            for (int i = pre; i < n && i < pre + a.l2_pre; ++i, advance()) {
+                if (a.w3d) tma_prefetch_3d(&a.tm_w, kb * kGtK, tile * kGtRows, seg);
+                else tma_prefetch_2d(&a.tm_w, kb * kGtK, tile * kGtRows);
             }
             pdl_wait();
             TPL_TRACE_AT(1);
@@ -418,6 +425,10 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
         const int B = a.B;
         const int nch = min((B + kGtChunk - 1) / kGtChunk, SMEM::NCH);
         const int ep_tid = threadIdx.x - 64;  // 0..127
+        // epilogue marks of the last shared tile (traced builds): pieces
+        // published, arrival counted, pieces listed, tile finished
+        TPL_TRACE_VARS
+        bool ep_traced = false;
         if (a.rms_src) {
             // 1/rms per token while the first weight tiles stream in: each
             // warp sums the squares of a strided quarter of the row, the four
@@ -534,6 +545,13 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
                 continue;
             }
             // shared tile: publish the pieces; the CTA completing the tile adds them
+            if (ep_tid == 0) {
+                TPL_TRACE_AT(0);
+                TPL_TRACE_AT(1);
+                TPL_TRACE_AT(2);
+                TPL_TRACE_AT(3);
+                ep_traced = true;
+            }
             __threadfence();
             asm volatile("bar.sync 1, 128;" ::: "memory");
             if (ep_tid == 0) {
@@ -546,6 +564,9 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
                     if (last) atomicExch(&a.tickets[tile], 0u);
                 }
                 *s_last = last ? 1 : 0;
+                TPL_TRACE_AT(1);
+                TPL_TRACE_AT(2);
+                TPL_TRACE_AT(3);
             }
             asm volatile("bar.sync 1, 128;" ::: "memory");
             if (!*s_last) continue;
@@ -593,6 +614,7 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
                             }
                             *s_nlist = n;
                             *s_more = g_s < a.nseg ? 1 : 0;
+                            if (round == 0 && ch == 0) TPL_TRACE_AT(2);
                         }
                         asm volatile("bar.sync 1, 128;" ::: "memory");
                     }
@@ -652,7 +674,10 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
                 }
                 if (a.epi != GT_ROW_PARTIAL) gt_final(a, row, tile_sum, lane, tok0, s_inv);
             }
+            if (ep_tid == 0) TPL_TRACE_AT(3);
         }
+        if (ep_tid == 0 && ep_traced)
+            TPL_TRACE_PUT(100 + (a.epi == GT_QKV ? TR_QKV : a.epi == GT_GU ? TR_GU : a.trace_row_tag));
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();

@@ -47,7 +47,25 @@ def launches(records):
     return out
 
 
-def summarise(ls):
+def epilogue_stats(L, epi):
+    """The tensor-core projections' epilogue marks of the launch's last shared
+    tiles (publish, arrival counted, pieces listed, tile finished)."""
+    t2 = [c[4][2] for c in L["ctas"] if c[4][2]]
+    if not epi or not t2:
+        return {}
+    last_issue = max(t2)
+    lasts = [e for e in epi if e[4][2] > e[4][1]]
+    out = {"publish_after_issue": (max(e[4][0] for e in epi) - last_issue) / 1e3,
+           "count": statistics.median((e[4][1] - e[4][0]) / 1e3 for e in epi)}
+    if lasts:
+        out["list"] = statistics.median((e[4][2] - e[4][1]) / 1e3 for e in lasts)
+        out["combine"] = statistics.median((e[4][3] - e[4][2]) / 1e3 for e in lasts)
+        out["combine_max"] = max((e[4][3] - e[4][2]) / 1e3 for e in lasts)
+        out["lasts"] = len(lasts)
+    return out
+
+
+def summarise(ls, epi_records=()):
     rows = []
     prev_end = None
     for L in ls:
@@ -66,6 +84,9 @@ def summarise(ls):
                 row["loop"] = (max(t2) - max(t1)) / 1e3
                 row["tail"] = (end - max(t2)) / 1e3
                 row["spread"] = (max(t2) - statistics.median(t2)) / 1e3
+        start = min(t0)
+        epi = [e for e in epi_records if e[0] == L["tag"] + ".epi" and start <= e[4][0] <= end]
+        row.update({"epi_" + k: v for k, v in epilogue_stats(L, epi).items()})
         rows.append(row)
         prev_end = end
     return rows
@@ -80,6 +101,7 @@ def main() -> None:
     ap.add_argument("--kv", type=int, default=4096)
     ap.add_argument("--gemv-mode", type=int, default=4)
     ap.add_argument("--attn-mode", type=int, default=0, help="TPL_OPT_DECODE_ATTN of the plan (0: the default)")
+    ap.add_argument("--l2-pre", type=int, default=-1, help="TPL_OPT_L2_PREFETCH of the plan (-1: the default)")
     ap.add_argument("--steps", type=int, default=3)
     ap.add_argument("--json", default="")
     args = ap.parse_args()
@@ -91,6 +113,8 @@ def main() -> None:
     plan = tpl.Plan(tpl.make_dims(H, NQ, NKV, D, F, NL, 1e-5, tpl.TPL_NORM | tpl.TPL_RESIDUAL), T)
     plan.set_option(tpl.TPL_OPT_GEMV_MODE, args.gemv_mode)
     plan.set_option(tpl.TPL_OPT_DECODE_ATTN, args.attn_mode)
+    if args.l2_pre >= 0:
+        plan.set_option(tpl.TPL_OPT_L2_PREFETCH, args.l2_pre)
     packed, kvs, keep = [], [], []
     for l in range(NL):
         w = synth.layer_weights(H, NQ, NKV, D, F, seed=0, layer=l, device=dev)
@@ -110,7 +134,10 @@ def main() -> None:
     for _ in range(args.steps):
         plan.decode_stack(packed, kvs, x, S, y, None, ws)
         torch.cuda.synchronize()
-        rows = summarise(launches(tpl.trace_read()))
+        recs = tpl.trace_read()
+        main_recs = [r for r in recs if not r[0].endswith(".epi")]
+        epi_recs = [r for r in recs if r[0].endswith(".epi")]
+        rows = summarise(launches(main_recs), epi_recs)
         for r in rows[1:]:  # the first launch has no predecessor in this step
             per_kind.setdefault(r["kernel"], []).append(r)
     assert plan.last_device_error() == tpl.TPL_OK
@@ -123,11 +150,14 @@ def main() -> None:
         rs = per_kind.get(k)
         if not rs:
             continue
-        med = {f: statistics.median(r[f] for r in rs if f in r) for f in
-               ("exposed", "release", "loop", "tail", "spread") if any(f in r for r in rs)}
+        fields = sorted({f for r in rs for f in r if f not in ("kernel", "ctas", "grid")})
+        med = {f: statistics.median(r[f] for r in rs if f in r) for f in fields}
         out["kernels"][k] = dict(med, launches=len(rs))
         print(f"{k:10s} {len(rs):4d} " + " ".join(f"{med.get(f, float('nan')):8.1f}" for f in
                                                   ("exposed", "release", "loop", "tail", "spread")))
+        ep = {f: v for f, v in med.items() if f.startswith("epi_")}
+        if ep:
+            print("           epilogue: " + ", ".join(f"{f[4:]} {v:.1f}" for f, v in sorted(ep.items())))
     print(f"sum of median exposed times per layer: {sum(v['exposed'] for k, v in out['kernels'].items() if k != 'operand'):.1f} us")
     if args.json:
         with open(args.json, "w") as f:

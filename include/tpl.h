@@ -164,10 +164,6 @@ void tpl_plan_destroy(tpl_plan *plan);
  * TPL_SPLIT_O (the attention output into O) and TPL_SPLIT_GU (the normalised
  * h into gate/up); the down projection's operand (act) is always one part.
  * Default TPL_SPLIT_DEFAULT.
- * TPL_OPT_L2_PREFETCH: how many 16 KB weight tiles each CTA of a
- * tensor-core decode projection prefetches into L2 (beyond the tiles it
- * loads into its shared-memory ring) before waiting for the preceding
- * kernel, 0..4096; default TPL_L2_PREFETCH_DEFAULT.
  * Returns TPL_EINVAL for an unknown option or value. */
 #define TPL_OPT_GEMV_MODE 1
 #define TPL_OPT_PREFILL_ATTN 2
@@ -177,8 +173,6 @@ void tpl_plan_destroy(tpl_plan *plan);
 #define TPL_SPLIT_O 2
 #define TPL_SPLIT_GU 4
 #define TPL_SPLIT_DEFAULT (TPL_SPLIT_QKV | TPL_SPLIT_O | TPL_SPLIT_GU)
-#define TPL_OPT_L2_PREFETCH 5
-#define TPL_L2_PREFETCH_DEFAULT 0
 int tpl_plan_set_option(tpl_plan *plan, int32_t option, int32_t value);
 
 /* Footprints (host) -- see tpl_plan_info. */

@@ -393,6 +393,111 @@ constexpr int kStgRow = 136;                           // padded row, bf16 eleme
 constexpr int kStgStep = 2 * 16 * kStgRow;             // K and V rows of one stage, elements
 constexpr size_t kStgSmem = (size_t)kAttnWarps * kStgStages * kStgStep * 2;  // dynamic bytes
 
+// The end of a staged-kernel CTA: the warps' (max, sum, output) in s_o /
+// s_ml merged in warp order into the CTA's partial, the arrival counter of
+// the pair, and for the last CTA of the pair the ordered combine of the CTA
+// partials and the new token.  It runs once per CTA at the very end, so its
+// code would be cold there (fetched from L2 line by line): it is one
+// non-inlined copy, run once early with `dry` set (stores to a shared scratch
+// word, loads from the start of q with their values discarded, no counter
+// update, the last-CTA path taken) so that it is cached when needed.
+__device__ __noinline__ void stg_finish(const AttnArgs &a, int pair, int chunk, int cpp, int b, int j,
+                                        const float *s_o, const float *s_ml, bool dry) {
+    constexpr int D = 128;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int dim = threadIdx.x;
+    __shared__ float s_dummy[4];
+    const int64_t cbase = ((int64_t)pair * cpp + chunk) * a.g;
+    float *po_w = dry ? s_dummy : a.part_o + cbase * D + dim;
+    float *pm_w = dry ? s_dummy : a.part_ml + cbase * 2;
+    const int64_t so = dry ? 0 : D, sm = dry ? 0 : 2;
+    for (int hrow = 0; hrow < a.g; ++hrow) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, s_ml[(w * 8 + hrow) * 2]);
+        float num = 0.f, den = 0.f;
+#pragma unroll
+        for (int w = 0; w < kAttnWarps; ++w) {
+            const float mi = s_ml[(w * 8 + hrow) * 2];
+            const float wt = mi == -INFINITY ? 0.f : exp2f(mi - M);
+            num += wt * s_o[(w * 8 + hrow) * D + dim];
+            den += wt * s_ml[(w * 8 + hrow) * 2 + 1];
+        }
+        po_w[hrow * so] = num;
+        if (dim == 0) {
+            pm_w[hrow * sm + 0] = M;
+            pm_w[hrow * sm + 1] = den;
+        }
+    }
+    __shared__ int s_last;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        if (dry) {
+            s_last = 1;
+        } else {
+            const unsigned prev = atomicAdd(&a.tickets[pair], 1u);
+            s_last = prev == (unsigned)(cpp - 1);
+            if (prev >= (unsigned)cpp) record_error(2u);
+        }
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    __shared__ float s_w[kAttnMaxCtasPerPair][8];
+    __shared__ float s_M[8], s_den[8], s_new[8];
+    __shared__ float s_mlp[kAttnMaxCtasPerPair * 8 * 2];
+    __shared__ float s_red[kAttnWarps][8];
+    const bool has_new = a.k_new != nullptr;
+    const float *pm_r = dry ? a.q : a.part_ml + (int64_t)pair * cpp * a.g * 2;
+    for (int i = threadIdx.x; i < cpp * a.g * 2; i += blockDim.x) s_mlp[i] = __ldcg(pm_r + (dry ? 0 : i));
+    if (has_new) {
+        const float kd = a.k_new[((int64_t)b * (a.nq / a.g) + j) * D + dim];
+        for (int hrow = 0; hrow < a.g; ++hrow) {
+            float v = a.q[((int64_t)b * a.nq + (int64_t)j * a.g + hrow) * D + dim] * kd;
+#pragma unroll
+            for (int o2 = 16; o2 > 0; o2 >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o2);
+            if (lane == 0) s_red[warp][hrow] = v;
+        }
+        __syncthreads();
+        if (threadIdx.x < a.g) {
+            float v = 0.f;
+#pragma unroll
+            for (int w = 0; w < kAttnWarps; ++w) v += s_red[w][threadIdx.x];
+            s_new[threadIdx.x] = v * a.scale_log2;
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < a.g) {
+        const int hrow = threadIdx.x;
+        float M = has_new ? s_new[hrow] : -INFINITY;
+        for (int i = 0; i < cpp; ++i) M = fmaxf(M, s_mlp[(i * a.g + hrow) * 2]);
+        float den = 0.f;
+        for (int i = 0; i < cpp; ++i) {
+            const float mi = s_mlp[(i * a.g + hrow) * 2];
+            const float wt = mi == -INFINITY ? 0.f : exp2f(mi - M);
+            s_w[i][hrow] = wt;
+            den += wt * s_mlp[(i * a.g + hrow) * 2 + 1];
+        }
+        if (has_new) den += exp2f(s_new[hrow] - M);
+        s_M[hrow] = M;
+        s_den[hrow] = den;
+    }
+    __syncthreads();
+    const int64_t sp = dry ? 0 : (int64_t)a.g * D;
+    for (int hrow = 0; hrow < a.g; ++hrow) {
+        float num = 0.f;
+        const float *po = dry ? a.q : a.part_o + ((int64_t)pair * cpp * a.g + hrow) * D + dim;
+#pragma unroll 8
+        for (int i = 0; i < cpp; ++i) num += s_w[i][hrow] * __ldcg(po + i * sp);
+        if (has_new) num += exp2f(s_new[hrow] - s_M[hrow]) * a.v_new[((int64_t)b * (a.nq / a.g) + j) * D + dim];
+        if (dry) s_dummy[0] = num / s_den[hrow];
+        else store_act(a.o, a.o_f32, ((int64_t)b * a.nq + (int64_t)j * a.g + hrow) * D + dim, num / s_den[hrow]);
+    }
+    if (threadIdx.x == 0 && !dry) atomicExch(&a.tickets[pair], 0u);
+    __syncthreads();  // the shared arrays are reused by the real call after a dry one
+}
+
 __global__ void __launch_bounds__(kAttnWarps * 32, 1) attn_decode_staged_kernel(const __grid_constant__ AttnArgs a) {
     constexpr int D = 128;
     extern __shared__ __align__(128) __nv_bfloat16 stg_smem[];
@@ -466,6 +571,11 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) attn_decode_staged_kernel(
         }
     }
 
+    // the end-of-kernel code, run dry while the first stages stream in
+    __shared__ float s_o[kAttnWarps][8][D];
+    __shared__ float s_ml[kAttnWarps][8][2];
+    stg_finish(a, pair, chunk, cpp, b, j, &s_o[0][0][0], &s_ml[0][0][0], true);
+
     float o[16][4];
 #pragma unroll
     for (int t = 0; t < 16; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
@@ -534,8 +644,6 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) attn_decode_staged_kernel(
     l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
 
     // ---- merge the CTA's warps (ascending warp order), then the CTA partials ----
-    __shared__ float s_o[kAttnWarps][8][D];
-    __shared__ float s_ml[kAttnWarps][8][2];
     if (gid < a.g) {
 #pragma unroll
         for (int t = 0; t < 16; ++t) {
@@ -548,93 +656,8 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) attn_decode_staged_kernel(
         }
     }
     __syncthreads();
-    const int dim = threadIdx.x;
-    const int64_t cbase = ((int64_t)pair * cpp + chunk) * a.g;
-    for (int hrow = 0; hrow < a.g; ++hrow) {
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, s_ml[w][hrow][0]);
-        float num = 0.f, den = 0.f;
-#pragma unroll
-        for (int w = 0; w < kAttnWarps; ++w) {
-            const float mi = s_ml[w][hrow][0];
-            const float wt = mi == -INFINITY ? 0.f : exp2f(mi - M);
-            num += wt * s_o[w][hrow][dim];
-            den += wt * s_ml[w][hrow][1];
-        }
-        a.part_o[(cbase + hrow) * D + dim] = num;
-        if (dim == 0) {
-            a.part_ml[(cbase + hrow) * 2 + 0] = M;
-            a.part_ml[(cbase + hrow) * 2 + 1] = den;
-        }
-    }
-    __shared__ int s_last;
-    __threadfence();
-    __syncthreads();
+    stg_finish(a, pair, chunk, cpp, b, j, &s_o[0][0][0], &s_ml[0][0][0], false);
     if (threadIdx.x == 0) {
-        const unsigned prev = atomicAdd(&a.tickets[pair], 1u);
-        s_last = prev == (unsigned)(cpp - 1);
-        if (prev >= (unsigned)cpp) record_error(2u);
-    }
-    __syncthreads();
-    if (!s_last) {
-        if (threadIdx.x == 0) {
-            TPL_TRACE_AT(3);
-            TPL_TRACE_PUT(TR_ATTN);
-        }
-        return;
-    }
-    __threadfence();
-    __shared__ float s_w[kAttnMaxCtasPerPair][8];
-    __shared__ float s_M[8], s_den[8], s_new[8];
-    __shared__ float s_mlp[kAttnMaxCtasPerPair * 8 * 2];
-    const bool has_new = a.k_new != nullptr;
-    for (int i = threadIdx.x; i < cpp * a.g * 2; i += blockDim.x)
-        s_mlp[i] = __ldcg(&a.part_ml[(int64_t)pair * cpp * a.g * 2 + i]);
-    if (has_new) {
-        __shared__ float s_red[kAttnWarps][8];
-        const float kd = a.k_new[((int64_t)b * (a.nq / a.g) + j) * D + dim];
-        for (int hrow = 0; hrow < a.g; ++hrow) {
-            float v = a.q[((int64_t)b * a.nq + (int64_t)j * a.g + hrow) * D + dim] * kd;
-#pragma unroll
-            for (int o2 = 16; o2 > 0; o2 >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o2);
-            if (lane == 0) s_red[warp][hrow] = v;
-        }
-        __syncthreads();
-        if (threadIdx.x < a.g) {
-            float v = 0.f;
-#pragma unroll
-            for (int w = 0; w < kAttnWarps; ++w) v += s_red[w][threadIdx.x];
-            s_new[threadIdx.x] = v * a.scale_log2;
-        }
-    }
-    __syncthreads();
-    if (threadIdx.x < a.g) {
-        const int hrow = threadIdx.x;
-        float M = has_new ? s_new[hrow] : -INFINITY;
-        for (int i = 0; i < cpp; ++i) M = fmaxf(M, s_mlp[(i * a.g + hrow) * 2]);
-        float den = 0.f;
-        for (int i = 0; i < cpp; ++i) {
-            const float mi = s_mlp[(i * a.g + hrow) * 2];
-            const float wt = mi == -INFINITY ? 0.f : exp2f(mi - M);
-            s_w[i][hrow] = wt;
-            den += wt * s_mlp[(i * a.g + hrow) * 2 + 1];
-        }
-        if (has_new) den += exp2f(s_new[hrow] - M);
-        s_M[hrow] = M;
-        s_den[hrow] = den;
-    }
-    __syncthreads();
-    for (int hrow = 0; hrow < a.g; ++hrow) {
-        float num = 0.f;
-        const float *po = a.part_o + ((int64_t)pair * cpp * a.g + hrow) * D + dim;
-#pragma unroll 8
-        for (int i = 0; i < cpp; ++i) num += s_w[i][hrow] * __ldcg(po + (int64_t)i * a.g * D);
-        if (has_new) num += exp2f(s_new[hrow] - s_M[hrow]) * a.v_new[((int64_t)b * (a.nq / a.g) + j) * D + dim];
-        store_act(a.o, a.o_f32, ((int64_t)b * a.nq + (int64_t)j * a.g + hrow) * D + dim, num / s_den[hrow]);
-    }
-    if (threadIdx.x == 0) {
-        atomicExch(&a.tickets[pair], 0u);
         TPL_TRACE_AT(3);
         TPL_TRACE_PUT(TR_ATTN);
     }

@@ -254,7 +254,6 @@ GemvTcArgs gt_args(const tpl_plan *p) {
     GemvTcArgs a;
     std::memset(&a, 0, sizeof(a));
     a.hd = p->d.head_dim;
-    a.l2_pre = p->l2_prefetch;
     return a;
 }
 

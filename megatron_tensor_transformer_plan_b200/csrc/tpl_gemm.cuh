@@ -128,19 +128,6 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *tm, in
         : "memory");
 }
 
-// L2 prefetch of one tensor-map tile (no shared memory, no barrier).
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap *tm, int x, int y) {
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(tm)),
-                 "r"(x), "r"(y)
-                 : "memory");
-}
-__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *tm, int x, int y, int z) {
-    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global [%0, {%1, %2, %3}];" ::"l"(
-                     reinterpret_cast<uint64_t>(tm)),
-                 "r"(x), "r"(y), "r"(z)
-                 : "memory");
-}
-
 // K-major, 128-byte-swizzle shared-memory matrix descriptor: rows of 128 B,
 // 8-row groups 1024 B apart.
 __device__ __forceinline__ uint64_t umma_desc(unsigned saddr) {

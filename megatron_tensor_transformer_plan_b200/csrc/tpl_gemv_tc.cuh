@@ -118,7 +118,6 @@ struct GemvTcArgs {
     int gstride;        // floats per row of a piece: 16 * ceil(B / 16)
     unsigned *tickets;  // [tiles]
     int trace_row_tag;  // timeline tag of a row-parallel launch (traced builds)
-    int l2_pre;         // weight tiles after the first stages prefetched into L2 before the dependency wait
 };
 
 // Tokens 16*ch .. 16*ch+15 of one accumulator row: the hi column plus the
@@ -142,7 +141,12 @@ __device__ __forceinline__ void gt_load_chunk(uint32_t taddr, int ch, float (&pv
 }
 
 // CTA c's unit range [u0, u1) of U units over G CTAs.
-__device__ __forceinline__ int64_t gt_start(int64_t U, int G, int c) { return U * c / G; }
+__device__ __forceinline__ int64_t gt_start(int64_t U, int G, int c) {
+    // 32-bit arithmetic when it cannot overflow (c <= G <= 256): much cheaper
+    // than a 64-bit division, and the combine evaluates this many times
+    if (U < (1ll << 23)) return (int64_t)(((uint32_t)U * (uint32_t)c) / (uint32_t)G);
+    return U * c / G;
+}
 
 // The order in which a CTA walks its range, as three sub-ranges [b, e): the
 // part of its first tile, the part of its last tile (both possibly shared
@@ -167,66 +171,214 @@ __device__ __forceinline__ GtOrder gt_order(int64_t u0, int64_t u1, int64_t per_
 
 // Final write of one output row for tokens tok0 .. tok0+15 (fused sums or
 // column ops).
-__device__ __forceinline__ void gt_final(const GemvTcArgs &a, int row, const float (&v0)[kGtChunk], int lane,
-                                         int tok0, const float *inv_rms) {
-    const int B = a.B;
+//
+// This and gt_combine run at the end of the kernel, once per CTA: cold, their
+// instructions were fetched from L2 line by line, which measured 7-15 us per
+// kernel.  Both are therefore not inlined (one copy of the code) and are run
+// once early with `dry` set: every loop and branch taken as for a full chunk
+// of tokens, every store sent to a shared-memory scratch word and every load
+// to the start of the workspace's piece area (valid global memory whose
+// values are discarded), so the instruction cache holds them when the real
+// call comes.
+__device__ __noinline__ void gt_final(const GemvTcArgs &a, int row, const float (&v0)[kGtChunk], int lane, int tok0,
+                                      const float *inv_rms, bool dry, float *dummy) {
+    const int B = dry ? tok0 + kGtChunk : a.B;
+    const bool scale = a.rms_src && a.epi != GT_ROW;  // the RMSNorm factor of column ops
     float v[kGtChunk];
 #pragma unroll
-    for (int i = 0; i < kGtChunk; ++i)  // the RMSNorm factor of column ops (1 without it)
-        v[i] = (a.rms_src && a.epi != GT_ROW) ? v0[i] * inv_rms[min(tok0 + i, kGtMaxB - 1)] : v0[i];
+    for (int i = 0; i < kGtChunk; ++i) v[i] = scale ? v0[i] * inv_rms[min(tok0 + i, kGtMaxB - 1)] : v0[i];
     if (a.epi == GT_GU) {
         // rows interleave gate and up: the even lane pairs with its odd neighbour
+        const bool w = !(lane & 1) && (dry || row + 1 < a.N);
+        __nv_bfloat16 *dst = dry ? reinterpret_cast<__nv_bfloat16 *>(dummy)
+                                 : static_cast<__nv_bfloat16 *>(a.out_act) + row / 2;
+        const int64_t st = dry ? 0 : a.N / 2;
 #pragma unroll
         for (int i = 0; i < kGtChunk; ++i) {
             const int b = tok0 + i;
             const float u = __shfl_down_sync(0xffffffffu, v[i], 1);
-            if (b < B && !(lane & 1) && row + 1 < a.N)
-                static_cast<__nv_bfloat16 *>(a.out_act)[(int64_t)b * (a.N / 2) + row / 2] =
-                    __float2bfloat16_rn(silu(v[i]) * u);
+            if (w && b < B) dst[b * st] = __float2bfloat16_rn(silu(v[i]) * u);
         }
         return;
     }
-    if (row >= a.N) return;
+    if (!dry && row >= a.N) return;
     if (a.epi == GT_QKV) {
+        // the row is one q element, or one k or v element of the cache (and
+        // its fp32 copy); per token only the batch stride moves
         const int s = row / a.rps, l = row % a.rps;
         const int qd = a.nq_s * a.hd, kd = a.nkv_s * a.hd;
+        const bool isq = dry ? (row & 1) != 0 : l < qd;  // a dry run takes both paths
+        const bool isk = l < qd + kd;
+        const int ll = isk ? l - qd : l - qd - kd;  // kv head * hd + dim within the shard
+        float *dq = a.q + (int64_t)s * qd + l;
+        __nv_bfloat16 *dc = (isk ? a.kc : a.vc) + ((int64_t)s * a.batch_cap * a.nkv_s * a.seq_cap + a.S) * a.hd +
+                            (int64_t)(ll / a.hd) * a.seq_cap * a.hd + ll % a.hd;
+        float *dn = isk ? a.knew : a.vnew;
+        if (dn) dn += (int64_t)s * kd + ll;
+        int64_t sq = (int64_t)a.nq * a.hd, sc = (int64_t)a.nkv_s * a.seq_cap * a.hd,
+                sn = (int64_t)a.nkv_s * (a.nq / a.nq_s) * a.hd;
+        if (dry) {
+            dq = dummy;
+            dc = reinterpret_cast<__nv_bfloat16 *>(dummy);
+            dn = dummy;
+            sq = sc = sn = 0;
+        }
 #pragma unroll
         for (int i = 0; i < kGtChunk; ++i) {
             const int b = tok0 + i;
             if (b >= B) continue;
-            if (l < qd) {
-                const int head = s * a.nq_s + l / a.hd, dim = l % a.hd;
-                a.q[((int64_t)b * a.nq + head) * a.hd + dim] = v[i];
+            if (isq) {
+                dq[b * sq] = v[i];
             } else {
-                const bool isk = l < qd + kd;
-                const int ll = isk ? l - qd : l - qd - kd;
-                const int kvl = ll / a.hd, dim = ll % a.hd;
-                __nv_bfloat16 *c = isk ? a.kc : a.vc;
-                c[((((int64_t)s * a.batch_cap + b) * a.nkv_s + kvl) * a.seq_cap + a.S) * a.hd + dim] =
-                    __float2bfloat16_rn(v[i]);
-                float *f = isk ? a.knew : a.vnew;
-                if (f) f[((int64_t)b * (a.nkv_s * (a.nq / a.nq_s)) + s * a.nkv_s + kvl) * a.hd + dim] = v[i];
+                dc[b * sc] = __float2bfloat16_rn(v[i]);
+                if (dn) dn[b * sn] = v[i];
             }
         }
         return;
     }
     // GT_ROW: out = resid + sum
+    const int64_t st = dry ? 0 : a.N;
+    const int64_t i0 = dry ? 0 : row;
+    const void *resid = dry && a.resid ? static_cast<const void *>(a.gpart) : a.resid;
+    float *o32 = dry && a.out32 ? dummy : a.out32;
+    __nv_bfloat16 *oact = dry && a.out_act ? reinterpret_cast<__nv_bfloat16 *>(dummy)
+                                           : static_cast<__nv_bfloat16 *>(a.out_act);
+    __nv_bfloat16 *xs = dry && a.xs_out ? reinterpret_cast<__nv_bfloat16 *>(dummy) : a.xs_out;
+    const float *xg = dry && a.xs_gamma ? a.gpart : a.xs_gamma;
+    const int64_t xrow = dry ? 0 : row, xhalf = dry ? 0 : (int64_t)a.xs_half * a.N;
 #pragma unroll
     for (int j = 0; j < kGtChunk; ++j) {
         const int b = tok0 + j;
         if (b >= B) continue;
-        const int64_t i = (int64_t)b * a.N + row;
+        const int64_t i = b * st + i0;
         float o = v[j];
-        if (a.resid) o = load_act(a.resid, a.resid_f32, i) + o;
-        if (a.out32) a.out32[i] = o;
-        if (a.out_act) static_cast<__nv_bfloat16 *>(a.out_act)[i] = __float2bfloat16_rn(o);
-        if (a.xs_out) {
-            const float src = a.out_act ? __bfloat162float(__float2bfloat16_rn(o)) : o;
+        if (resid) o = load_act(resid, a.resid_f32, i) + o;
+        if (o32) o32[i] = o;
+        if (oact) oact[i] = __float2bfloat16_rn(o);
+        if (xs) {
+            const float src = oact ? __bfloat162float(__float2bfloat16_rn(o)) : o;
             __nv_bfloat16 hi, lo;
-            split_scaled(src, a.xs_gamma, row, hi, lo);
-            a.xs_out[i] = hi;
-            a.xs_out[(int64_t)(a.xs_half + b) * a.N + row] = lo;
+            split_scaled(src, xg, xrow, hi, lo);
+            xs[i] = hi;
+            xs[xhalf + i] = lo;
         }
+    }
+}
+
+// The CTA that completed a tile split across CTAs adds its pieces in the
+// fixed order (segment, then CTA) and writes the tile.  The pieces are listed
+// by one thread in shared memory (in rounds of up to kGtList entries), then
+// loaded eight at a time; the walk is repeated for each 16-token chunk,
+// reusing the list when one round held it all.  Each CTA stored its part in
+// slot 0 if the tile is its first, else in slot 1.  Run by the 128 epilogue
+// threads (named barrier 1); `dry` as for gt_final.
+__device__ __noinline__ void gt_combine(const GemvTcArgs &a, int tile, int G, int nch, int r, int lane, int ep_tid,
+                                        const float *s_inv, volatile int *s_list, volatile int *s_nlist,
+                                        volatile int *s_more, float *dummy, bool dry) {
+    const int64_t per_tile = (int64_t)a.nseg * a.kbs;
+    const int64_t t_beg = (int64_t)tile * per_tile;
+    const int row = tile * kGtRows + r;
+    const int B = dry ? kGtChunk * nch : a.B;
+    float seg_sum[kGtChunk], tile_sum[kGtChunk];
+    bool single = false;  // the whole list is in shared memory
+#pragma unroll 1
+    for (int ch = 0; ch < nch; ++ch) {
+        const int tok0 = kGtChunk * ch;
+#pragma unroll
+        for (int t = 0; t < kGtChunk; ++t) {
+            tile_sum[t] = -0.f;
+            seg_sum[t] = -0.f;
+        }
+        int g_s = 0, g_cc = 0;  // generator position (thread 0)
+        if (!single && ep_tid == 0) {
+            int cf = (int)((t_beg * G) / a.U);
+            while (cf > 0 && gt_start(a.U, G, cf) > t_beg) --cf;
+            while (gt_start(a.U, G, cf + 1) <= t_beg) ++cf;
+            g_cc = cf;
+        }
+        for (int round = 0;; ++round) {
+            if (!single) {
+                if (ep_tid == 0) {
+                    int n = 0;
+                    while (n < kGtList && g_s < a.nseg) {
+                        const int64_t sb = t_beg + (int64_t)g_s * a.kbs, se = sb + a.kbs;
+                        const int64_t c0 = gt_start(a.U, G, g_cc), c1 = gt_start(a.U, G, g_cc + 1);
+                        if (c1 > sb && c0 < se) {
+                            const int sl = (tile == (int)(c0 / per_tile)) ? 0 : 1;
+                            const bool seg_last = c1 >= se;
+                            s_list[n++] = (((g_cc * 2 + sl) * a.nseg + g_s) << 5) | (g_s << 1) | (seg_last ? 1 : 0);
+                        }
+                        if (c1 >= se) {
+                            ++g_s;  // next segment starts in this same CTA
+                        } else {
+                            ++g_cc;
+                        }
+                    }
+                    *s_nlist = n;
+                    *s_more = g_s < a.nseg ? 1 : 0;
+                }
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+            }
+            const int n = dry ? 8 : *s_nlist;
+            for (int e0 = 0; e0 < n; e0 += 8) {
+                float4 v[8][kGtChunk / 4];
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+#pragma unroll
+                    for (int q4 = 0; q4 < kGtChunk / 4; ++q4) v[j][q4] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    if (e0 + j < n) {
+                        const int ent = s_list[e0 + j];
+                        const float4 *src =
+                            dry ? reinterpret_cast<const float4 *>(a.gpart)
+                                : reinterpret_cast<const float4 *>(a.gpart) +
+                                      ((int64_t)(ent >> 5) * (a.gstride / 4) + tok0 / 4) * kGtRows + r;
+                        const int64_t sq = dry ? 0 : kGtRows;
+#pragma unroll
+                        for (int q4 = 0; q4 < kGtChunk / 4; ++q4)
+                            if (tok0 + 4 * q4 < B) v[j][q4] = __ldcg(src + q4 * sq);
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    if (e0 + j >= n) break;
+                    const int ent = s_list[e0 + j];
+#pragma unroll
+                    for (int q4 = 0; q4 < kGtChunk / 4; ++q4) {
+                        seg_sum[4 * q4] = seg_sum[4 * q4] + v[j][q4].x;
+                        seg_sum[4 * q4 + 1] = seg_sum[4 * q4 + 1] + v[j][q4].y;
+                        seg_sum[4 * q4 + 2] = seg_sum[4 * q4 + 2] + v[j][q4].z;
+                        seg_sum[4 * q4 + 3] = seg_sum[4 * q4 + 3] + v[j][q4].w;
+                    }
+                    if (dry || (ent & 1)) {  // the segment is complete
+                        const int sg = (ent >> 1) & 15;
+                        if (a.epi == GT_ROW_PARTIAL) {
+                            if (dry || row < a.N) {
+                                float *dst = dry ? dummy : a.partials + ((int64_t)sg * B + tok0) * a.N + row;
+                                const int64_t st = dry ? 0 : a.N;
+#pragma unroll
+                                for (int t = 0; t < kGtChunk; ++t)
+                                    if (tok0 + t < B) dst[t * st] = seg_sum[t];
+                            }
+                        } else {
+#pragma unroll
+                            for (int t = 0; t < kGtChunk; ++t) tile_sum[t] = tile_sum[t] + seg_sum[t];
+                        }
+#pragma unroll
+                        for (int t = 0; t < kGtChunk; ++t) seg_sum[t] = -0.f;
+                    }
+                }
+            }
+            if (single) break;
+            const bool more = *s_more != 0;
+            asm volatile("bar.sync 1, 128;" ::: "memory");  // list consumed before it is rewritten
+            if (!more) {
+                single = round == 0;  // one round held the whole list: keep it
+                break;
+            }
+        }
+        if (a.epi != GT_ROW_PARTIAL) gt_final(a, row, tile_sum, lane, tok0, s_inv, dry, dummy);
     }
 }
 
@@ -246,7 +398,8 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
     uint64_t *full = reinterpret_cast<uint64_t *>(sm + NS * STAGE + SMEM::TSBYTES);
     float *s_rpart = reinterpret_cast<float *>(sm + NS * STAGE + SMEM::TSBYTES + kGtBarBytes);  // [4][kGtMaxB]
     float *s_inv = s_rpart + 4 * kGtMaxB;                                                       // [kGtMaxB]
-    static_assert(5 * kGtMaxB * 4 <= kGtRmsBytes, "rms area");
+    float *s_dummy = s_inv + kGtMaxB;  // [16]: the scratch words of the early dry run of the combine code
+    static_assert(5 * kGtMaxB * 4 + 64 <= kGtRmsBytes, "rms area");
     uint64_t *empty = full + NS;
     uint64_t *acc_full = empty + NS;        // [BUFS]
     uint64_t *acc_empty = acc_full + BUFS;  // [BUFS]
@@ -334,19 +487,14 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
             };
             const int n = (int)(u1 - u0);
             const int pre = n < NS ? n : NS;
-            // weight tiles of the first stages before the dependency wait,
-            // and the next l2_pre tiles into L2 (weights never depend on the
-            // previous kernel; the stream resumes from L2 after the wait)
+            // weight tiles of the first stages before the dependency wait
+            // (weights never depend on the previous kernel)
             restart();
             for (int i = 0; i < pre; ++i, advance()) {
                 unsigned char *st = sm + i * STAGE;
                 mbar_expect_tx(&full[i], STAGE);
                 if (a.w3d) tma_load_3d(st, &a.tm_w, kb * kGtK, tile * kGtRows, seg, &full[i]);
                 else tma_load_2d(st, &a.tm_w, kb * kGtK, tile * kGtRows, &full[i]);
-            }
-            for (int i = pre; i < n && i < pre + a.l2_pre; ++i, advance()) {
-                if (a.w3d) tma_prefetch_3d(&a.tm_w, kb * kGtK, tile * kGtRows, seg);
-                else tma_prefetch_2d(&a.tm_w, kb * kGtK, tile * kGtRows);
             }
             pdl_wait();
             TPL_TRACE_AT(1);
@@ -469,7 +617,11 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
             }
             asm volatile("bar.sync 1, 128;" ::: "memory");
         }
-        float seg_sum[kGtChunk], tile_sum[kGtChunk];
+        // warm the instruction cache with the end-of-kernel code while the
+        // first weight tiles stream in (a dry run: no global access)
+        gt_combine(a, 0, G, nch, r, lane, ep_tid, s_inv, s_list, s_nlist, s_more, s_dummy, true);
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        float tile_sum[kGtChunk];
         int c = 0;
         bool dead = false;
         const GtOrder ord = gt_order(u0, u1, per_tile);
@@ -539,7 +691,7 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
                         const float *tsp = ts + (kGtChunk * ch) * kGtRows + r;
 #pragma unroll
                         for (int t = 0; t < kGtChunk; ++t) tile_sum[t] = tsp[t * kGtRows];
-                        gt_final(a, row, tile_sum, lane, kGtChunk * ch, s_inv);
+                        gt_final(a, row, tile_sum, lane, kGtChunk * ch, s_inv, false, s_dummy);
                     }
                 }
                 continue;
@@ -571,109 +723,7 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
             asm volatile("bar.sync 1, 128;" ::: "memory");
             if (!*s_last) continue;
             __threadfence();
-            // The tile's pieces in order (segment, then CTA), listed by one
-            // thread in shared memory (in rounds of up to kGtList entries),
-            // then loaded eight at a time; the walk is repeated for each
-            // 16-token chunk, reusing the list when one round held it all.
-            // Each CTA stored its part in slot 0 if the tile is its first,
-            // else in slot 1.
-            bool single = false;  // the whole list is in shared memory
-#pragma unroll 1
-            for (int ch = 0; ch < nch; ++ch) {
-                const int tok0 = kGtChunk * ch;
-#pragma unroll
-                for (int t = 0; t < kGtChunk; ++t) {
-                    tile_sum[t] = -0.f;
-                    seg_sum[t] = -0.f;
-                }
-                int g_s = 0, g_cc = 0;  // generator position (thread 0)
-                if (!single && ep_tid == 0) {
-                    int cf = (int)((t_beg * G) / a.U);
-                    while (cf > 0 && gt_start(a.U, G, cf) > t_beg) --cf;
-                    while (gt_start(a.U, G, cf + 1) <= t_beg) ++cf;
-                    g_cc = cf;
-                }
-                for (int round = 0;; ++round) {
-                    if (!single) {
-                        if (ep_tid == 0) {
-                            int n = 0;
-                            while (n < kGtList && g_s < a.nseg) {
-                                const int64_t sb = t_beg + (int64_t)g_s * a.kbs, se = sb + a.kbs;
-                                const int64_t c0 = gt_start(a.U, G, g_cc), c1 = gt_start(a.U, G, g_cc + 1);
-                                if (c1 > sb && c0 < se) {
-                                    const int sl = (tile == (int)(c0 / per_tile)) ? 0 : 1;
-                                    const bool seg_last = c1 >= se;
-                                    s_list[n++] =
-                                        (((g_cc * 2 + sl) * a.nseg + g_s) << 5) | (g_s << 1) | (seg_last ? 1 : 0);
-                                }
-                                if (c1 >= se) {
-                                    ++g_s;  // next segment starts in this same CTA
-                                } else {
-                                    ++g_cc;
-                                }
-                            }
-                            *s_nlist = n;
-                            *s_more = g_s < a.nseg ? 1 : 0;
-                            if (round == 0 && ch == 0) TPL_TRACE_AT(2);
-                        }
-                        asm volatile("bar.sync 1, 128;" ::: "memory");
-                    }
-                    const int n = *s_nlist;
-                    for (int e0 = 0; e0 < n; e0 += 8) {
-                        float4 v[8][kGtChunk / 4];
-#pragma unroll
-                        for (int j = 0; j < 8; ++j)
-#pragma unroll
-                            for (int q4 = 0; q4 < kGtChunk / 4; ++q4) v[j][q4] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            if (e0 + j < n) {
-                                const int ent = s_list[e0 + j];
-                                const float4 *src = reinterpret_cast<const float4 *>(a.gpart) +
-                                                    ((int64_t)(ent >> 5) * (a.gstride / 4) + tok0 / 4) * kGtRows + r;
-#pragma unroll
-                                for (int q4 = 0; q4 < kGtChunk / 4; ++q4)
-                                    if (tok0 + 4 * q4 < B) v[j][q4] = __ldcg(src + q4 * kGtRows);
-                            }
-                        }
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            if (e0 + j >= n) break;
-                            const int ent = s_list[e0 + j];
-#pragma unroll
-                            for (int q4 = 0; q4 < kGtChunk / 4; ++q4) {
-                                seg_sum[4 * q4] = seg_sum[4 * q4] + v[j][q4].x;
-                                seg_sum[4 * q4 + 1] = seg_sum[4 * q4 + 1] + v[j][q4].y;
-                                seg_sum[4 * q4 + 2] = seg_sum[4 * q4 + 2] + v[j][q4].z;
-                                seg_sum[4 * q4 + 3] = seg_sum[4 * q4 + 3] + v[j][q4].w;
-                            }
-                            if (ent & 1) {  // the segment is complete
-                                const int sg = (ent >> 1) & 15;
-                                if (a.epi == GT_ROW_PARTIAL) {
-                                    if (row < a.N)
-#pragma unroll
-                                        for (int t = 0; t < kGtChunk; ++t)
-                                            if (tok0 + t < B)
-                                                a.partials[((int64_t)sg * B + tok0 + t) * a.N + row] = seg_sum[t];
-                                } else {
-#pragma unroll
-                                    for (int t = 0; t < kGtChunk; ++t) tile_sum[t] = tile_sum[t] + seg_sum[t];
-                                }
-#pragma unroll
-                                for (int t = 0; t < kGtChunk; ++t) seg_sum[t] = -0.f;
-                            }
-                        }
-                    }
-                    if (single) break;
-                    const bool more = *s_more != 0;
-                    asm volatile("bar.sync 1, 128;" ::: "memory");  // list consumed before it is rewritten
-                    if (!more) {
-                        single = round == 0;  // one round held the whole list: keep it
-                        break;
-                    }
-                }
-                if (a.epi != GT_ROW_PARTIAL) gt_final(a, row, tile_sum, lane, tok0, s_inv);
-            }
+            gt_combine(a, tile, G, nch, r, lane, ep_tid, s_inv, s_list, s_nlist, s_more, s_dummy, false);
             if (ep_tid == 0) TPL_TRACE_AT(3);
         }
         if (ep_tid == 0 && ep_traced)

@@ -248,7 +248,6 @@ int tpl_plan_create(const tpl_dims *dims, int32_t t, tpl_plan **out) {
     p->gemv_mode = p->f32 ? 1 : 4;
     p->attn_prefill_mode = 0;
     p->prefill_split = TPL_SPLIT_DEFAULT;
-    p->l2_prefetch = TPL_L2_PREFETCH_DEFAULT;
     p->attn_decode_mode = 0;
     p->rope = (dims->flags & TPL_ROPE) != 0;
     for (int e = 0; e < 64; ++e)
@@ -299,11 +298,6 @@ int tpl_plan_set_option(tpl_plan *p, int32_t option, int32_t value) {
     if (option == TPL_OPT_PREFILL_ATTN) {
         if (value != 0 && value != 1) return TPL_EINVAL;
         p->attn_prefill_mode = value;
-        return TPL_OK;
-    }
-    if (option == TPL_OPT_L2_PREFETCH) {
-        if (value < 0 || value > 4096) return TPL_EINVAL;
-        p->l2_prefetch = value;
         return TPL_OK;
     }
     if (option == TPL_OPT_PREFILL_SPLIT) {

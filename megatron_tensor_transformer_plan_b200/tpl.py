@@ -31,7 +31,6 @@ TPL_OPT_DECODE_ATTN = 3
 TPL_OPT_PREFILL_SPLIT = 4
 TPL_SPLIT_QKV, TPL_SPLIT_O, TPL_SPLIT_GU = 1, 2, 4
 TPL_SPLIT_DEFAULT = TPL_SPLIT_QKV | TPL_SPLIT_O | TPL_SPLIT_GU
-TPL_OPT_L2_PREFETCH = 5
 TPL_ATTN_STATIC_SCRATCH_BYTES = 4 * 1024 * 1024
 
 c_int32, c_int64, c_size_t, c_void_p, c_uint32 = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_uint32
@@ -131,7 +130,8 @@ class tpl_trace_rec(ctypes.Structure):
 
 
 TRACE_TAGS = {1: "qkv", 2: "attention", 3: "o_proj", 4: "gate_up", 5: "down", 6: "operand", 7: "reduce",
-              101: "qkv.epi", 103: "o_proj.epi", 104: "gate_up.epi", 105: "down.epi"}
+              101: "qkv.epi", 103: "o_proj.epi", 104: "gate_up.epi", 105: "down.epi",
+              201: "qkv.clk", 203: "o_proj.clk", 204: "gate_up.clk", 205: "down.clk"}
 
 
 def trace_read(max_records: int = 1 << 18):

@@ -101,11 +101,11 @@ def main() -> None:
     ap.add_argument("--kv", type=int, default=4096)
     ap.add_argument("--gemv-mode", type=int, default=4)
     ap.add_argument("--attn-mode", type=int, default=0, help="TPL_OPT_DECODE_ATTN of the plan (0: the default)")
-    ap.add_argument("--l2-pre", type=int, default=-1, help="TPL_OPT_L2_PREFETCH of the plan (-1: the default)")
     ap.add_argument("--steps", type=int, default=3)
     ap.add_argument("--json", default="")
     args = ap.parse_args()
-    os.environ["TPL_LIB"] = build.build(trace=True)
+    if not os.environ.get("TPL_LIB"):  # another traced build may be named explicitly
+        os.environ["TPL_LIB"] = build.build(trace=True)
     from megatron_tensor_transformer_plan_b200 import tpl
     H, NQ, NKV, F = SHAPES[args.shape]
     T, B, S, NL = args.t, args.batch, args.kv, args.layers
@@ -113,8 +113,6 @@ def main() -> None:
     plan = tpl.Plan(tpl.make_dims(H, NQ, NKV, D, F, NL, 1e-5, tpl.TPL_NORM | tpl.TPL_RESIDUAL), T)
     plan.set_option(tpl.TPL_OPT_GEMV_MODE, args.gemv_mode)
     plan.set_option(tpl.TPL_OPT_DECODE_ATTN, args.attn_mode)
-    if args.l2_pre >= 0:
-        plan.set_option(tpl.TPL_OPT_L2_PREFETCH, args.l2_pre)
     packed, kvs, keep = [], [], []
     for l in range(NL):
         w = synth.layer_weights(H, NQ, NKV, D, F, seed=0, layer=l, device=dev)
@@ -131,12 +129,17 @@ def main() -> None:
     torch.cuda.synchronize()
     tpl.trace_read()  # drop the warm-up records
     per_kind = {}
+    clk = {}
     for _ in range(args.steps):
         plan.decode_stack(packed, kvs, x, S, y, None, ws)
         torch.cuda.synchronize()
         recs = tpl.trace_read()
-        main_recs = [r for r in recs if not r[0].endswith(".epi")]
+        main_recs = [r for r in recs if not r[0].endswith((".epi", ".clk"))]
         epi_recs = [r for r in recs if r[0].endswith(".epi")]
+        for r in recs:  # combine phases in SM cycles: loads and sums, list barrier, final write
+            if r[0].endswith(".clk") and r[4][3] > r[4][0] > 0:
+                t = r[4]
+                clk.setdefault(r[0][:-4], []).append((t[1] - t[0], t[2] - t[1] if t[2] else 0, t[3] - max(t[1], t[2])))
         rows = summarise(launches(main_recs), epi_recs)
         for r in rows[1:]:  # the first launch has no predecessor in this step
             per_kind.setdefault(r["kernel"], []).append(r)
@@ -158,6 +161,9 @@ def main() -> None:
         ep = {f: v for f, v in med.items() if f.startswith("epi_")}
         if ep:
             print("           epilogue: " + ", ".join(f"{f[4:]} {v:.1f}" for f, v in sorted(ep.items())))
+    for k, v in sorted(clk.items()):
+        print(f"{k:10s} combine cycles (median over CTAs): loads+sums {statistics.median(x[0] for x in v):.0f}, "
+              f"barrier {statistics.median(x[1] for x in v):.0f}, final {statistics.median(x[2] for x in v):.0f}")
     print(f"sum of median exposed times per layer: {sum(v['exposed'] for k, v in out['kernels'].items() if k != 'operand'):.1f} us")
     if args.json:
         with open(args.json, "w") as f:

@@ -571,10 +571,8 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) attn_decode_staged_kernel(
         }
     }
 
-    // the end-of-kernel code, run dry while the first stages stream in
     __shared__ float s_o[kAttnWarps][8][D];
     __shared__ float s_ml[kAttnWarps][8][2];
-    stg_finish(a, pair, chunk, cpp, b, j, &s_o[0][0][0], &s_ml[0][0][0], true);
 
     float o[16][4];
 #pragma unroll

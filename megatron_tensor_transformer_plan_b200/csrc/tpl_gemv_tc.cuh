@@ -11,9 +11,11 @@
 // 64-column weight tiles (16 KB, 128-byte swizzle) and the matching activation
 // tile into a 4-8 stage shared-memory ring, one thread issues four M=128,
 // N=NX, K=16 tcgen05.mma per stage, and the tensor pipe idles most of the
-// time.  192 threads: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer,
+// time.  224 threads: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer,
 // warps 2-5 epilogue (one TMEM lane = one weight row each), which walks the
-// tokens in chunks of 16 columns so that its registers do not grow with B.
+// tokens in chunks of 16 columns so that its registers do not grow with B,
+// and warp 6, which only runs the end-of-kernel code once, dry, at the start
+// (gt_final), so that it is in the instruction cache when the kernel ends.
 //
 // Work division ("stream-K"): the k-blocks of every (row tile, segment) are
 // laid end to end, tile-major then segment then k, and each CTA takes one
@@ -46,7 +48,7 @@
 
 namespace tpl {
 
-constexpr int kGtThreads = 192;
+constexpr int kGtThreads = 224;  // 6 working warps + the instruction-cache warm-up warp
 constexpr int kGtRows = 128;     // weight rows per tile (MMA M)
 constexpr int kGtK = 64;         // columns per k-block
 constexpr int kGtWBytes = kGtRows * kGtK * 2;  // 16 KB
@@ -174,12 +176,12 @@ __device__ __forceinline__ GtOrder gt_order(int64_t u0, int64_t u1, int64_t per_
 //
 // This and gt_combine run at the end of the kernel, once per CTA: cold, their
 // instructions were fetched from L2 line by line, which measured 7-15 us per
-// kernel.  Both are therefore not inlined (one copy of the code) and are run
-// once early with `dry` set: every loop and branch taken as for a full chunk
-// of tokens, every store sent to a shared-memory scratch word and every load
-// to the start of the workspace's piece area (valid global memory whose
-// values are discarded), so the instruction cache holds them when the real
-// call comes.
+// kernel (a second run of the same code took 1-2 us).  Both are therefore not
+// inlined (one copy of the code) and a spare warp runs them once at the start
+// with `dry` set: every loop and branch taken as for a full chunk of tokens,
+// every store sent to a shared-memory scratch word and every load to the start
+// of the workspace's piece area (valid global memory whose values are
+// discarded), so the instruction cache holds them when the real call comes.
 __device__ __noinline__ void gt_final(const GemvTcArgs &a, int row, const float (&v0)[kGtChunk], int lane, int tok0,
                                       const float *inv_rms, bool dry, float *dummy) {
     const int B = dry ? tok0 + kGtChunk : a.B;
@@ -246,21 +248,28 @@ __device__ __noinline__ void gt_final(const GemvTcArgs &a, int row, const float 
     __nv_bfloat16 *xs = dry && a.xs_out ? reinterpret_cast<__nv_bfloat16 *>(dummy) : a.xs_out;
     const float *xg = dry && a.xs_gamma ? a.gpart : a.xs_gamma;
     const int64_t xrow = dry ? 0 : row, xhalf = dry ? 0 : (int64_t)a.xs_half * a.N;
+    // every load before any store (the pointers may alias as far as the
+    // compiler knows, which would otherwise serialise the loads' latencies)
+    float rv[kGtChunk];
+#pragma unroll
+    for (int j = 0; j < kGtChunk; ++j)
+        rv[j] = (resid && tok0 + j < B) ? load_act(resid, a.resid_f32, (tok0 + j) * st + i0) : 0.f;
+    const float gam = xg ? xg[xrow] : 1.f;
 #pragma unroll
     for (int j = 0; j < kGtChunk; ++j) {
         const int b = tok0 + j;
         if (b >= B) continue;
         const int64_t i = b * st + i0;
-        float o = v[j];
-        if (resid) o = load_act(resid, a.resid_f32, i) + o;
+        const float o = resid ? rv[j] + v[j] : v[j];
         if (o32) o32[i] = o;
         if (oact) oact[i] = __float2bfloat16_rn(o);
         if (xs) {
+            // split_scaled with the row's gain loaded once
             const float src = oact ? __bfloat162float(__float2bfloat16_rn(o)) : o;
-            __nv_bfloat16 hi, lo;
-            split_scaled(src, xg, xrow, hi, lo);
+            const float sc = xg ? __fmul_rn(src, gam) : src;
+            const __nv_bfloat16 hi = __float2bfloat16_rn(sc);
             xs[i] = hi;
-            xs[xhalf + i] = lo;
+            xs[xhalf + i] = __float2bfloat16_rn(__fsub_rn(sc, __bfloat162float(hi)));
         }
     }
 }
@@ -271,16 +280,22 @@ __device__ __noinline__ void gt_final(const GemvTcArgs &a, int row, const float 
 // loaded eight at a time; the walk is repeated for each 16-token chunk,
 // reusing the list when one round held it all.  Each CTA stored its part in
 // slot 0 if the tile is its first, else in slot 1.  Run by the 128 epilogue
-// threads (named barrier 1); `dry` as for gt_final.
+// threads (named barrier 1); `dry` as for gt_final, run by the one warm-up
+// warp (no barrier, its own list area).
 __device__ __noinline__ void gt_combine(const GemvTcArgs &a, int tile, int G, int nch, int r, int lane, int ep_tid,
                                         const float *s_inv, volatile int *s_list, volatile int *s_nlist,
-                                        volatile int *s_more, float *dummy, bool dry) {
+                                        volatile int *s_more, volatile int *s_cnt, float *dummy, bool dry) {
     const int64_t per_tile = (int64_t)a.nseg * a.kbs;
     const int64_t t_beg = (int64_t)tile * per_tile;
     const int row = tile * kGtRows + r;
     const int B = dry ? kGtChunk * nch : a.B;
     float seg_sum[kGtChunk], tile_sum[kGtChunk];
     bool single = false;  // the whole list is in shared memory
+#ifdef TPL_TRACE
+    // SM-clock marks of the first chunk (traced builds): start, list built,
+    // pieces loaded and added, written
+    uint64_t ck[4] = {(uint64_t)clock64(), 0, 0, 0};
+#endif
 #pragma unroll 1
     for (int ch = 0; ch < nch; ++ch) {
         const int tok0 = kGtChunk * ch;
@@ -289,13 +304,47 @@ __device__ __noinline__ void gt_combine(const GemvTcArgs &a, int tile, int G, in
             tile_sum[t] = -0.f;
             seg_sum[t] = -0.f;
         }
-        int g_s = 0, g_cc = 0;  // generator position (thread 0)
-        if (!single && ep_tid == 0) {
-            int cf = (int)((t_beg * G) / a.U);
-            while (cf > 0 && gt_start(a.U, G, cf) > t_beg) --cf;
-            while (gt_start(a.U, G, cf + 1) <= t_beg) ++cf;
-            g_cc = cf;
+        // The CTAs cf..cl cover the tile.  With at most 128 (segment, CTA)
+        // candidates, the 128 threads test one each and the list is compacted
+        // in candidate order (segment-major, CTAs ascending); otherwise one
+        // thread generates it in rounds.
+        int cf = (int)((t_beg * G) / a.U);
+        while (cf > 0 && gt_start(a.U, G, cf) > t_beg) --cf;
+        while (gt_start(a.U, G, cf + 1) <= t_beg) ++cf;
+        int cl = cf;
+        while (cl + 1 < G && gt_start(a.U, G, cl + 1) < t_beg + per_tile) ++cl;
+        const int ncta = cl - cf + 1, ncand = a.nseg * ncta;
+        if (!single && ncand <= 128) {
+            const int k = dry ? lane : ep_tid;
+            const int g_s = k / ncta, c = cf + k % ncta;
+            bool valid = false;
+            int ent = 0;
+            if (k < ncand) {
+                const int64_t sb = t_beg + (int64_t)g_s * a.kbs, se = sb + a.kbs;
+                const int64_t c0 = gt_start(a.U, G, c), c1 = gt_start(a.U, G, c + 1);
+                valid = c1 > sb && c0 < se;
+                const int sl = (tile == (int)(c0 / per_tile)) ? 0 : 1;
+                ent = (((c * 2 + sl) * a.nseg + g_s) << 5) | (g_s << 1) | (c1 >= se ? 1 : 0);
+            }
+            const unsigned m = __ballot_sync(0xffffffffu, valid);
+            const int w = dry ? 0 : ep_tid >> 5;
+            if (lane == 0) s_cnt[w] = __popc(m);
+            if (dry) __syncwarp();
+            else asm volatile("bar.sync 1, 128;" ::: "memory");
+            int base = 0;
+            for (int x = 0; x < w; ++x) base += s_cnt[x];
+            const int pos = base + __popc(m & ((1u << lane) - 1u));
+            if (valid && pos < kGtList) s_list[dry ? 0 : pos] = ent;
+            if (ep_tid == 0) {
+                const int tot = s_cnt[0] + s_cnt[1] + s_cnt[2] + s_cnt[3];
+                *s_nlist = tot < kGtList ? tot : kGtList;
+                *s_more = 0;
+            }
+            if (dry) __syncwarp();
+            else asm volatile("bar.sync 1, 128;" ::: "memory");
+            single = *s_nlist < kGtList || dry;  // a full list may have dropped entries: generate it instead
         }
+        int g_s = 0, g_cc = cf;  // generator position (thread 0)
         for (int round = 0;; ++round) {
             if (!single) {
                 if (ep_tid == 0) {
@@ -317,68 +366,109 @@ __device__ __noinline__ void gt_combine(const GemvTcArgs &a, int tile, int G, in
                     *s_nlist = n;
                     *s_more = g_s < a.nseg ? 1 : 0;
                 }
-                asm volatile("bar.sync 1, 128;" ::: "memory");
+                if (dry) __syncwarp();
+                else asm volatile("bar.sync 1, 128;" ::: "memory");
             }
-            const int n = dry ? 8 : *s_nlist;
-            for (int e0 = 0; e0 < n; e0 += 8) {
-                float4 v[8][kGtChunk / 4];
+            // at most 4 tokens in this chunk: one float4 per piece, 32 pieces'
+            // loads in flight per round; else 16 tokens (4 float4), 8 pieces.
+            // The choice follows the real token count, also in a dry run.
+            const bool narrow = a.B - tok0 <= 4;
+            const int n = dry ? (narrow ? 32 : 8) : *s_nlist;
+#ifdef TPL_TRACE
+            if (ch == 0 && round == 0) ck[1] = (uint64_t)clock64();
+#endif
+            // one listed piece added to its segment sum; a completed segment
+            // goes to the tile sum (or out, as a shard partial)
+            auto add_piece = [&](int ent, const float4 (&pv)[kGtChunk / 4], int nq4) {
 #pragma unroll
-                for (int j = 0; j < 8; ++j)
-#pragma unroll
-                    for (int q4 = 0; q4 < kGtChunk / 4; ++q4) v[j][q4] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    if (e0 + j < n) {
-                        const int ent = s_list[e0 + j];
-                        const float4 *src =
-                            dry ? reinterpret_cast<const float4 *>(a.gpart)
-                                : reinterpret_cast<const float4 *>(a.gpart) +
-                                      ((int64_t)(ent >> 5) * (a.gstride / 4) + tok0 / 4) * kGtRows + r;
-                        const int64_t sq = dry ? 0 : kGtRows;
-#pragma unroll
-                        for (int q4 = 0; q4 < kGtChunk / 4; ++q4)
-                            if (tok0 + 4 * q4 < B) v[j][q4] = __ldcg(src + q4 * sq);
-                    }
+                for (int q4 = 0; q4 < kGtChunk / 4; ++q4) {
+                    if (q4 >= nq4) break;
+                    seg_sum[4 * q4] = seg_sum[4 * q4] + pv[q4].x;
+                    seg_sum[4 * q4 + 1] = seg_sum[4 * q4 + 1] + pv[q4].y;
+                    seg_sum[4 * q4 + 2] = seg_sum[4 * q4 + 2] + pv[q4].z;
+                    seg_sum[4 * q4 + 3] = seg_sum[4 * q4 + 3] + pv[q4].w;
                 }
+                if (dry || (ent & 1)) {  // the segment is complete
+                    const int sg = (ent >> 1) & 15;
+                    if (a.epi == GT_ROW_PARTIAL) {
+                        if (dry || row < a.N) {
+                            float *dst = dry ? dummy : a.partials + ((int64_t)sg * B + tok0) * a.N + row;
+                            const int64_t st = dry ? 0 : a.N;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    if (e0 + j >= n) break;
-                    const int ent = s_list[e0 + j];
-#pragma unroll
-                    for (int q4 = 0; q4 < kGtChunk / 4; ++q4) {
-                        seg_sum[4 * q4] = seg_sum[4 * q4] + v[j][q4].x;
-                        seg_sum[4 * q4 + 1] = seg_sum[4 * q4 + 1] + v[j][q4].y;
-                        seg_sum[4 * q4 + 2] = seg_sum[4 * q4 + 2] + v[j][q4].z;
-                        seg_sum[4 * q4 + 3] = seg_sum[4 * q4 + 3] + v[j][q4].w;
-                    }
-                    if (dry || (ent & 1)) {  // the segment is complete
-                        const int sg = (ent >> 1) & 15;
-                        if (a.epi == GT_ROW_PARTIAL) {
-                            if (dry || row < a.N) {
-                                float *dst = dry ? dummy : a.partials + ((int64_t)sg * B + tok0) * a.N + row;
-                                const int64_t st = dry ? 0 : a.N;
-#pragma unroll
-                                for (int t = 0; t < kGtChunk; ++t)
-                                    if (tok0 + t < B) dst[t * st] = seg_sum[t];
-                            }
-                        } else {
-#pragma unroll
-                            for (int t = 0; t < kGtChunk; ++t) tile_sum[t] = tile_sum[t] + seg_sum[t];
+                            for (int t = 0; t < kGtChunk; ++t)
+                                if (tok0 + t < B) dst[t * st] = seg_sum[t];
                         }
+                    } else {
 #pragma unroll
-                        for (int t = 0; t < kGtChunk; ++t) seg_sum[t] = -0.f;
+                        for (int t = 0; t < kGtChunk; ++t) tile_sum[t] = tile_sum[t] + seg_sum[t];
+                    }
+#pragma unroll
+                    for (int t = 0; t < kGtChunk; ++t) seg_sum[t] = -0.f;
+                }
+            };
+            auto piece_src = [&](int ent) {
+                return dry ? reinterpret_cast<const float4 *>(a.gpart)
+                           : reinterpret_cast<const float4 *>(a.gpart) +
+                                 ((int64_t)(ent >> 5) * (a.gstride / 4) + tok0 / 4) * kGtRows + r;
+            };
+            if (narrow) {
+                for (int e0 = 0; e0 < n; e0 += 32) {
+                    float4 v1[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        v1[j] = e0 + j < n ? __ldcg(piece_src(s_list[dry ? 0 : e0 + j]))
+                                           : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        if (e0 + j >= n) break;
+                        const float4 pv[kGtChunk / 4] = {v1[j]};
+                        add_piece(s_list[dry ? 0 : e0 + j], pv, 1);
+                    }
+                }
+            } else {
+                for (int e0 = 0; e0 < n; e0 += 8) {
+                    float4 v[8][kGtChunk / 4];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+#pragma unroll
+                        for (int q4 = 0; q4 < kGtChunk / 4; ++q4) v[j][q4] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        if (e0 + j < n) {
+                            const float4 *src = piece_src(s_list[dry ? 0 : e0 + j]);
+                            const int64_t sq = dry ? 0 : kGtRows;
+#pragma unroll
+                            for (int q4 = 0; q4 < kGtChunk / 4; ++q4)
+                                if (tok0 + 4 * q4 < B) v[j][q4] = __ldcg(src + q4 * sq);
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        if (e0 + j >= n) break;
+                        add_piece(s_list[dry ? 0 : e0 + j], v[j], kGtChunk / 4);
                     }
                 }
             }
+#ifdef TPL_TRACE
+            if (ch == 0 && round == 0) ck[2] = (uint64_t)clock64();
+#endif
             if (single) break;
             const bool more = *s_more != 0;
-            asm volatile("bar.sync 1, 128;" ::: "memory");  // list consumed before it is rewritten
+            if (dry) __syncwarp();
+            else asm volatile("bar.sync 1, 128;" ::: "memory");  // list consumed before it is rewritten
             if (!more) {
                 single = round == 0;  // one round held the whole list: keep it
                 break;
             }
         }
         if (a.epi != GT_ROW_PARTIAL) gt_final(a, row, tile_sum, lane, tok0, s_inv, dry, dummy);
+#ifdef TPL_TRACE
+        if (ch == 0) {
+            ck[3] = (uint64_t)clock64();
+            if (ep_tid == 0) trace_put((dry ? 300 : 200) + a.trace_row_tag * 0 + (a.epi == GT_QKV ? TR_QKV
+                                       : a.epi == GT_GU ? TR_GU : a.trace_row_tag), ck);
+        }
+#endif
     }
 }
 
@@ -388,7 +478,7 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
     constexpr int STAGE = SMEM::STAGE;
     constexpr int NS = SMEM::NS;
     constexpr int BUFS = SMEM::BUFS;
-    static_assert(2 * NS * 8 + 2 * BUFS * 8 + 8 + 4 + 32 + 4 * kGtList <= kGtBarBytes, "barrier area");
+    static_assert(2 * NS * 8 + 2 * BUFS * 8 + 8 + 4 + 32 + 4 * (kGtList + 4) <= kGtBarBytes, "barrier area");
     constexpr int TMEM_COLS = BUFS * NX <= 32 ? 32 : BUFS * NX <= 64 ? 64 : BUFS * NX <= 128 ? 128
                               : BUFS * NX <= 256 ? 256 : 512;
     static_assert(BUFS * NX <= 512, "accumulators");
@@ -399,7 +489,8 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
     float *s_rpart = reinterpret_cast<float *>(sm + NS * STAGE + SMEM::TSBYTES + kGtBarBytes);  // [4][kGtMaxB]
     float *s_inv = s_rpart + 4 * kGtMaxB;                                                       // [kGtMaxB]
     float *s_dummy = s_inv + kGtMaxB;  // [16]: the scratch words of the early dry run of the combine code
-    static_assert(5 * kGtMaxB * 4 + 64 <= kGtRmsBytes, "rms area");
+    volatile int *w_list = reinterpret_cast<volatile int *>(s_dummy + 16);  // [kGtList + 6]: its piece list
+    static_assert(5 * kGtMaxB * 4 + 64 + 4 * (kGtList + 6) <= kGtRmsBytes, "rms area");
     uint64_t *empty = full + NS;
     uint64_t *acc_full = empty + NS;        // [BUFS]
     uint64_t *acc_empty = acc_full + BUFS;  // [BUFS]
@@ -561,6 +652,14 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
             umma_commit(fin);
             if (!mbar_wait(fin, 0)) *s_fail = 1;
         }
+    } else if (warp == 6) {
+        // ---- warm-up: the end-of-kernel code once, dry, into the instruction cache.
+        //      No dependency wait: it reads only the start of the piece area
+        //      (values discarded) and writes only this CTA's shared scratch,
+        //      so it can run while the preceding kernel finishes ----
+        const int nch = min((a.B + kGtChunk - 1) / kGtChunk, SMEM::NCH);
+        gt_combine(a, 0, G, nch, 32 * (lane & 3) + lane, lane, lane, s_inv, w_list + 2, w_list, w_list + 1,
+                   w_list + 2 + kGtList, s_dummy, true);
     } else {
         pdl_wait();
         // ---- epilogue: thread = weight row 32*(warp%4) + lane of the tile ----
@@ -617,10 +716,6 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
             }
             asm volatile("bar.sync 1, 128;" ::: "memory");
         }
-        // warm the instruction cache with the end-of-kernel code while the
-        // first weight tiles stream in (a dry run: no global access)
-        gt_combine(a, 0, G, nch, r, lane, ep_tid, s_inv, s_list, s_nlist, s_more, s_dummy, true);
-        asm volatile("bar.sync 1, 128;" ::: "memory");
         float tile_sum[kGtChunk];
         int c = 0;
         bool dead = false;
@@ -723,7 +818,8 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
             asm volatile("bar.sync 1, 128;" ::: "memory");
             if (!*s_last) continue;
             __threadfence();
-            gt_combine(a, tile, G, nch, r, lane, ep_tid, s_inv, s_list, s_nlist, s_more, s_dummy, false);
+            gt_combine(a, tile, G, nch, r, lane, ep_tid, s_inv, s_list, s_nlist, s_more, s_list + kGtList, s_dummy,
+                       false);
             if (ep_tid == 0) TPL_TRACE_AT(3);
         }
         if (ep_tid == 0 && ep_traced)

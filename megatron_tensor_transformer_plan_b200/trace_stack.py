@@ -134,12 +134,12 @@ def main() -> None:
         plan.decode_stack(packed, kvs, x, S, y, None, ws)
         torch.cuda.synchronize()
         recs = tpl.trace_read()
-        main_recs = [r for r in recs if not r[0].endswith((".epi", ".clk"))]
+        main_recs = [r for r in recs if not r[0].endswith((".epi", ".clk", ".dry"))]
         epi_recs = [r for r in recs if r[0].endswith(".epi")]
-        for r in recs:  # combine phases in SM cycles: loads and sums, list barrier, final write
-            if r[0].endswith(".clk") and r[4][3] > r[4][0] > 0:
+        for r in recs:  # combine phases in SM cycles: list, loads and sums, final write
+            if r[0].endswith((".clk", ".dry")) and r[4][3] > r[4][0] > 0:
                 t = r[4]
-                clk.setdefault(r[0][:-4], []).append((t[1] - t[0], t[2] - t[1] if t[2] else 0, t[3] - max(t[1], t[2])))
+                clk.setdefault(r[0], []).append((t[1] - t[0], t[2] - t[1], t[3] - t[2]))
         rows = summarise(launches(main_recs), epi_recs)
         for r in rows[1:]:  # the first launch has no predecessor in this step
             per_kind.setdefault(r["kernel"], []).append(r)
@@ -162,8 +162,9 @@ def main() -> None:
         if ep:
             print("           epilogue: " + ", ".join(f"{f[4:]} {v:.1f}" for f, v in sorted(ep.items())))
     for k, v in sorted(clk.items()):
-        print(f"{k:10s} combine cycles (median over CTAs): loads+sums {statistics.median(x[0] for x in v):.0f}, "
-              f"barrier {statistics.median(x[1] for x in v):.0f}, final {statistics.median(x[2] for x in v):.0f}")
+        print(f"{k:14s} combine cycles (median of {len(v)}): list {statistics.median(x[0] for x in v):.0f}, "
+              f"loads+sums {statistics.median(x[1] for x in v):.0f}, final {statistics.median(x[2] for x in v):.0f}; "
+              f"slowest total {max(sum(x) for x in v):.0f}")
     print(f"sum of median exposed times per layer: {sum(v['exposed'] for k, v in out['kernels'].items() if k != 'operand'):.1f} us")
     if args.json:
         with open(args.json, "w") as f:

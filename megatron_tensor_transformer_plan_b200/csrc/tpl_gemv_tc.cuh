@@ -369,83 +369,107 @@ __device__ __noinline__ void gt_combine(const GemvTcArgs &a, int tile, int G, in
                 if (dry) __syncwarp();
                 else asm volatile("bar.sync 1, 128;" ::: "memory");
             }
-            // at most 4 tokens in this chunk: one float4 per piece, 32 pieces'
-            // loads in flight per round; else 16 tokens (4 float4), 8 pieces.
-            // The choice follows the real token count, also in a dry run.
+            // At most 4 tokens in this chunk: one float4 per piece, up to 16
+            // pieces' loads in flight, a short branch-free body per piece.
+            // Else 16 tokens (4 float4 per piece), 8 pieces per round.  The
+            // choice follows the real token count, also in a dry run, whose
+            // loads are predicated off.
             const bool narrow = a.B - tok0 <= 4;
-            const int n = dry ? (narrow ? 32 : 8) : *s_nlist;
+            const int n = dry ? (narrow ? 16 : 8) : *s_nlist;
 #ifdef TPL_TRACE
             if (ch == 0 && round == 0) ck[1] = (uint64_t)clock64();
 #endif
-            // one listed piece added to its segment sum; a completed segment
-            // goes to the tile sum (or out, as a shard partial)
-            auto add_piece = [&](int ent, const float4 (&pv)[kGtChunk / 4], int nq4) {
-#pragma unroll
-                for (int q4 = 0; q4 < kGtChunk / 4; ++q4) {
-                    if (q4 >= nq4) break;
-                    seg_sum[4 * q4] = seg_sum[4 * q4] + pv[q4].x;
-                    seg_sum[4 * q4 + 1] = seg_sum[4 * q4 + 1] + pv[q4].y;
-                    seg_sum[4 * q4 + 2] = seg_sum[4 * q4 + 2] + pv[q4].z;
-                    seg_sum[4 * q4 + 3] = seg_sum[4 * q4 + 3] + pv[q4].w;
-                }
-                if (dry || (ent & 1)) {  // the segment is complete
-                    const int sg = (ent >> 1) & 15;
-                    if (a.epi == GT_ROW_PARTIAL) {
-                        if (dry || row < a.N) {
-                            float *dst = dry ? dummy : a.partials + ((int64_t)sg * B + tok0) * a.N + row;
-                            const int64_t st = dry ? 0 : a.N;
-#pragma unroll
-                            for (int t = 0; t < kGtChunk; ++t)
-                                if (tok0 + t < B) dst[t * st] = seg_sum[t];
-                        }
-                    } else {
-#pragma unroll
-                        for (int t = 0; t < kGtChunk; ++t) tile_sum[t] = tile_sum[t] + seg_sum[t];
-                    }
-#pragma unroll
-                    for (int t = 0; t < kGtChunk; ++t) seg_sum[t] = -0.f;
-                }
-            };
             auto piece_src = [&](int ent) {
-                return dry ? reinterpret_cast<const float4 *>(a.gpart)
-                           : reinterpret_cast<const float4 *>(a.gpart) +
-                                 ((int64_t)(ent >> 5) * (a.gstride / 4) + tok0 / 4) * kGtRows + r;
+                return reinterpret_cast<const float4 *>(a.gpart) +
+                       ((int64_t)(ent >> 5) * (a.gstride / 4) + tok0 / 4) * kGtRows + r;
             };
             if (narrow) {
-                for (int e0 = 0; e0 < n; e0 += 32) {
-                    float4 v1[32];
+                float4 seg4 = make_float4(seg_sum[0], seg_sum[1], seg_sum[2], seg_sum[3]);
+                float4 tile4 = make_float4(tile_sum[0], tile_sum[1], tile_sum[2], tile_sum[3]);
+                for (int e0 = 0; e0 < n; e0 += 16) {
+                    float4 v1[16];
+                    int en[16];
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        v1[j] = e0 + j < n ? __ldcg(piece_src(s_list[dry ? 0 : e0 + j]))
-                                           : make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (int j = 0; j < 16; ++j) {
+                        en[j] = e0 + j < n ? s_list[dry ? 0 : e0 + j] : 0;
+                        v1[j] = (e0 + j < n && !dry) ? __ldcg(piece_src(en[j])) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        if (e0 + j >= n) break;
-                        const float4 pv[kGtChunk / 4] = {v1[j]};
-                        add_piece(s_list[dry ? 0 : e0 + j], pv, 1);
+                    for (int j = 0; j < 16; ++j) {
+                        if (!dry && e0 + j >= n) break;
+                        seg4.x = seg4.x + v1[j].x;
+                        seg4.y = seg4.y + v1[j].y;
+                        seg4.z = seg4.z + v1[j].z;
+                        seg4.w = seg4.w + v1[j].w;
+                        if (dry || (en[j] & 1)) {  // the segment is complete
+                            if (a.epi == GT_ROW_PARTIAL) {
+                                if (dry || row < a.N) {
+                                    const int sg = (en[j] >> 1) & 15;
+                                    float *dst = dry ? dummy : a.partials + ((int64_t)sg * B + tok0) * a.N + row;
+                                    const int64_t st = dry ? 0 : a.N;
+                                    const float w4[4] = {seg4.x, seg4.y, seg4.z, seg4.w};
+#pragma unroll
+                                    for (int t = 0; t < 4; ++t)
+                                        if (tok0 + t < B) dst[t * st] = w4[t];
+                                }
+                            } else {
+                                tile4.x = tile4.x + seg4.x;
+                                tile4.y = tile4.y + seg4.y;
+                                tile4.z = tile4.z + seg4.z;
+                                tile4.w = tile4.w + seg4.w;
+                            }
+                            seg4 = make_float4(-0.f, -0.f, -0.f, -0.f);
+                        }
                     }
                 }
+                seg_sum[0] = seg4.x;
+                seg_sum[1] = seg4.y;
+                seg_sum[2] = seg4.z;
+                seg_sum[3] = seg4.w;
+                tile_sum[0] = tile4.x;
+                tile_sum[1] = tile4.y;
+                tile_sum[2] = tile4.z;
+                tile_sum[3] = tile4.w;
             } else {
                 for (int e0 = 0; e0 < n; e0 += 8) {
                     float4 v[8][kGtChunk / 4];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j)
-#pragma unroll
-                        for (int q4 = 0; q4 < kGtChunk / 4; ++q4) v[j][q4] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    int en[8];
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        if (e0 + j < n) {
-                            const float4 *src = piece_src(s_list[dry ? 0 : e0 + j]);
-                            const int64_t sq = dry ? 0 : kGtRows;
+                        en[j] = e0 + j < n ? s_list[dry ? 0 : e0 + j] : 0;
+                        const float4 *src = piece_src(en[j]);
 #pragma unroll
-                            for (int q4 = 0; q4 < kGtChunk / 4; ++q4)
-                                if (tok0 + 4 * q4 < B) v[j][q4] = __ldcg(src + q4 * sq);
-                        }
+                        for (int q4 = 0; q4 < kGtChunk / 4; ++q4)
+                            v[j][q4] = (e0 + j < n && tok0 + 4 * q4 < B && !dry) ? __ldcg(src + q4 * kGtRows)
+                                                                                : make_float4(0.f, 0.f, 0.f, 0.f);
                     }
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        if (e0 + j >= n) break;
-                        add_piece(s_list[dry ? 0 : e0 + j], v[j], kGtChunk / 4);
+                        if (!dry && e0 + j >= n) break;
+#pragma unroll
+                        for (int q4 = 0; q4 < kGtChunk / 4; ++q4) {
+                            seg_sum[4 * q4] = seg_sum[4 * q4] + v[j][q4].x;
+                            seg_sum[4 * q4 + 1] = seg_sum[4 * q4 + 1] + v[j][q4].y;
+                            seg_sum[4 * q4 + 2] = seg_sum[4 * q4 + 2] + v[j][q4].z;
+                            seg_sum[4 * q4 + 3] = seg_sum[4 * q4 + 3] + v[j][q4].w;
+                        }
+                        if (dry || (en[j] & 1)) {  // the segment is complete
+                            const int sg = (en[j] >> 1) & 15;
+                            if (a.epi == GT_ROW_PARTIAL) {
+                                if (dry || row < a.N) {
+                                    float *dst = dry ? dummy : a.partials + ((int64_t)sg * B + tok0) * a.N + row;
+                                    const int64_t st = dry ? 0 : a.N;
+#pragma unroll
+                                    for (int t = 0; t < kGtChunk; ++t)
+                                        if (tok0 + t < B) dst[t * st] = seg_sum[t];
+                                }
+                            } else {
+#pragma unroll
+                                for (int t = 0; t < kGtChunk; ++t) tile_sum[t] = tile_sum[t] + seg_sum[t];
+                            }
+#pragma unroll
+                            for (int t = 0; t < kGtChunk; ++t) seg_sum[t] = -0.f;
+                        }
                     }
                 }
             }

@@ -521,6 +521,8 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) attn_decode_staged_kernel(
     if (threadIdx.x == 0) TPL_TRACE_AT(0);
     __nv_bfloat16 *ring = stg_smem + (size_t)warp * kStgStages * kStgStep;
 
+    uint64_t kvpol;  // the cache is read once: evict it from L2 first
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(kvpol));
     // stage st (keys k0 + 16 st ..) into slot st % kStgStages; keys past k1 read as zero
     auto issue = [&](int st) {
         if (st < nsteps) {
@@ -533,8 +535,8 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) attn_decode_staged_kernel(
                 const int r = piece >> 4, col = (piece & 15) * 8;
                 const int64_t key = kb + r;
                 if (key < k1) {
-                    cp_async16(kd + r * kStgRow + col, Kp + key * D + col);
-                    cp_async16(vd + r * kStgRow + col, Vp + key * D + col);
+                    cp_async16_hint(kd + r * kStgRow + col, Kp + key * D + col, kvpol);
+                    cp_async16_hint(vd + r * kStgRow + col, Vp + key * D + col, kvpol);
                 } else {
                     *reinterpret_cast<uint4 *>(kd + r * kStgRow + col) = make_uint4(0, 0, 0, 0);
                     *reinterpret_cast<uint4 *>(vd + r * kStgRow + col) = make_uint4(0, 0, 0, 0);

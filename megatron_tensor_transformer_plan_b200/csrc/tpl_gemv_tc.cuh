@@ -602,14 +602,15 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
             };
             const int n = (int)(u1 - u0);
             const int pre = n < NS ? n : NS;
+            const uint64_t wpol = l2_evict_first_policy();  // the weights are read once
             // weight tiles of the first stages before the dependency wait
             // (weights never depend on the previous kernel)
             restart();
             for (int i = 0; i < pre; ++i, advance()) {
                 unsigned char *st = sm + i * STAGE;
                 mbar_expect_tx(&full[i], STAGE);
-                if (a.w3d) tma_load_3d(st, &a.tm_w, kb * kGtK, tile * kGtRows, seg, &full[i]);
-                else tma_load_2d(st, &a.tm_w, kb * kGtK, tile * kGtRows, &full[i]);
+                if (a.w3d) tma_load_3d_hint(st, &a.tm_w, kb * kGtK, tile * kGtRows, seg, &full[i], wpol);
+                else tma_load_2d_hint(st, &a.tm_w, kb * kGtK, tile * kGtRows, &full[i], wpol);
             }
             pdl_wait();
             TPL_TRACE_AT(1);
@@ -625,8 +626,8 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
                         break;
                     }
                     mbar_expect_tx(&full[s], STAGE);
-                    if (a.w3d) tma_load_3d(st, &a.tm_w, kb * kGtK, tile * kGtRows, seg, &full[s]);
-                    else tma_load_2d(st, &a.tm_w, kb * kGtK, tile * kGtRows, &full[s]);
+                    if (a.w3d) tma_load_3d_hint(st, &a.tm_w, kb * kGtK, tile * kGtRows, seg, &full[s], wpol);
+                    else tma_load_2d_hint(st, &a.tm_w, kb * kGtK, tile * kGtRows, &full[s], wpol);
                 }
                 tma_load_2d(st + kGtWBytes, &a.tm_x, seg * a.x_seg_stride + kb * kGtK, 0, &full[s]);
             }

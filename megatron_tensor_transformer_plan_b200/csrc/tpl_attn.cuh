@@ -98,21 +98,22 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const __gr
     struct KV16 {
         uint4 kt0[4], kt1[4], va[2], vb[2], vc2[2], vd[2];
     };
+    const uint64_t kvpol = evict_first_policy();  // the cache is read once
     auto load16 = [&](KV16 &f, int64_t kb) {
         const int64_t key0 = kb + gid, key1 = kb + 8 + gid;
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
-            f.kt0[m] = key0 < k1 ? ldg_stream(Kp + key0 * D + 32 * m + 8 * c) : make_uint4(0, 0, 0, 0);
-            f.kt1[m] = key1 < k1 ? ldg_stream(Kp + key1 * D + 32 * m + 8 * c) : make_uint4(0, 0, 0, 0);
+            f.kt0[m] = key0 < k1 ? ldg_stream(Kp + key0 * D + 32 * m + 8 * c, kvpol) : make_uint4(0, 0, 0, 0);
+            f.kt1[m] = key1 < k1 ? ldg_stream(Kp + key1 * D + 32 * m + 8 * c, kvpol) : make_uint4(0, 0, 0, 0);
         }
         const int64_t ka = kb + 2 * c, kbb = ka + 1, kc_ = ka + 8, kd = ka + 9;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int col = 16 * gid + 8 * h;
-            f.va[h] = ka < k1 ? ldg_stream(Vp + ka * D + col) : make_uint4(0, 0, 0, 0);
-            f.vb[h] = kbb < k1 ? ldg_stream(Vp + kbb * D + col) : make_uint4(0, 0, 0, 0);
-            f.vc2[h] = kc_ < k1 ? ldg_stream(Vp + kc_ * D + col) : make_uint4(0, 0, 0, 0);
-            f.vd[h] = kd < k1 ? ldg_stream(Vp + kd * D + col) : make_uint4(0, 0, 0, 0);
+            f.va[h] = ka < k1 ? ldg_stream(Vp + ka * D + col, kvpol) : make_uint4(0, 0, 0, 0);
+            f.vb[h] = kbb < k1 ? ldg_stream(Vp + kbb * D + col, kvpol) : make_uint4(0, 0, 0, 0);
+            f.vc2[h] = kc_ < k1 ? ldg_stream(Vp + kc_ * D + col, kvpol) : make_uint4(0, 0, 0, 0);
+            f.vd[h] = kd < k1 ? ldg_stream(Vp + kd * D + col, kvpol) : make_uint4(0, 0, 0, 0);
         }
     };
     KV16 bufA, bufB;
@@ -521,8 +522,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) attn_decode_staged_kernel(
     if (threadIdx.x == 0) TPL_TRACE_AT(0);
     __nv_bfloat16 *ring = stg_smem + (size_t)warp * kStgStages * kStgStep;
 
-    uint64_t kvpol;  // the cache is read once: evict it from L2 first
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(kvpol));
+    const uint64_t kvpol = evict_first_policy();  // the cache is read once
     // stage st (keys k0 + 16 st ..) into slot st % kStgStages; keys past k1 read as zero
     auto issue = [&](int st) {
         if (st < nsteps) {

@@ -77,11 +77,11 @@ struct AttnTmaArgs {
 };
 
 __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *tm, int x, int y, int z, int w,
-                                            uint64_t *bar) {
+                                            uint64_t *bar, uint64_t policy) {
     asm volatile(
-        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
-        "[%6];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, "
+        "%3, %4, %5}], [%6], %7;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar)), "l"(policy)
         : "memory");
 }
 
@@ -138,6 +138,7 @@ __global__ void __launch_bounds__(kAmThreads, 1) attn_decode_tma_kernel(const __
     if (warp == kAmWarps) {
         // ---- producer ----
         if (lane == 0) {
+            const uint64_t kvpol = evict_first_policy();  // the cache is read once
             auto issue = [&](int i) {
                 const int s = i % NS;
                 const int64_t u = u0 + i;
@@ -147,10 +148,10 @@ __global__ void __launch_bounds__(kAmThreads, 1) attn_decode_tma_kernel(const __
                 const int sb = sh * a.batch_cap + b;
                 unsigned char *st = sm + s * kAmStage;
                 mbar_expect_tx(&full[s], kAmStage);
-                tma_load_4d(st, &a.tm_k, 0, blk * kAmKeys, jl, sb, &full[s]);
-                tma_load_4d(st + kAmBox, &a.tm_k, 64, blk * kAmKeys, jl, sb, &full[s]);
-                tma_load_4d(st + 2 * kAmBox, &a.tm_v, 0, blk * kAmKeys, jl, sb, &full[s]);
-                tma_load_4d(st + 3 * kAmBox, &a.tm_v, 64, blk * kAmKeys, jl, sb, &full[s]);
+                tma_load_4d(st, &a.tm_k, 0, blk * kAmKeys, jl, sb, &full[s], kvpol);
+                tma_load_4d(st + kAmBox, &a.tm_k, 64, blk * kAmKeys, jl, sb, &full[s], kvpol);
+                tma_load_4d(st + 2 * kAmBox, &a.tm_v, 0, blk * kAmKeys, jl, sb, &full[s], kvpol);
+                tma_load_4d(st + 3 * kAmBox, &a.tm_v, 64, blk * kAmKeys, jl, sb, &full[s], kvpol);
             };
             const int pre = n < NS ? n : NS;
             int i = 0;

@@ -63,13 +63,23 @@ __device__ __forceinline__ void trace_put(uint32_t tag, const uint64_t (&t)[4]) 
 #define TPL_TRACE_PUT(tag) ((void)0)
 #endif
 
-// 16-byte streaming load of read-once data (weights, KV cache): not kept in L1.
-__device__ __forceinline__ uint4 ldg_stream(const void *p) {
+// 16-byte streaming load of read-once data (weights, KV cache): not kept in L1,
+// first out of L2 under the given policy.
+__device__ __forceinline__ uint4 ldg_stream(const void *p, uint64_t policy) {
     uint4 r;
-    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+    asm("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
         : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-        : "l"(p));
+        : "l"(p), "l"(policy));
     return r;
+}
+
+// L2 policy for data read exactly once (weights and KV-cache streams): evict
+// it first, so that it does not push out the small data read again
+// (activations, cross-CTA partials, norms).
+__device__ __forceinline__ uint64_t evict_first_policy() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
 }
 
 __device__ __forceinline__ void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }

@@ -120,15 +120,6 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *tm, in
         : "memory");
 }
 
-// L2 policy for data read exactly once (weights and KV-cache streams): evict
-// it first, so that it does not push out the small data that is read again
-// (activations, cross-CTA pieces, norms).
-__device__ __forceinline__ uint64_t l2_evict_first_policy() {
-    uint64_t p;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-    return p;
-}
-
 __device__ __forceinline__ void tma_load_2d_hint(void *dst, const CUtensorMap *tm, int x, int y, uint64_t *bar,
                                                  uint64_t policy) {
     asm volatile(

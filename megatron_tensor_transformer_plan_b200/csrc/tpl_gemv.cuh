@@ -188,13 +188,14 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
                ((int64_t)(row % a.rps) * a.ldw + (int64_t)kb_lo * 128 + 8 * c) * T::WES;
     };
     uint4 ring[D][NW];
+    const uint64_t wpol = evict_first_policy();  // the weights are read once
     int lr = 0, lj = 0;
     const char *lptr = nrg_w > 0 ? rowptr(0) : a.W;
     auto load_next = [&](uint4 (&w)[NW]) {
 #pragma unroll
         for (int m = 0; m < 4; ++m)
 #pragma unroll
-            for (int l = 0; l < T::LPM; ++l) w[m * T::LPM + l] = ldg_stream(lptr + m * 32 * T::WES + 16 * l);
+            for (int l = 0; l < T::LPM; ++l) w[m * T::LPM + l] = ldg_stream(lptr + m * 32 * T::WES + 16 * l, wpol);
         if (++lj == nblk) {
             lj = 0;
             if (++lr < nrg_w) lptr = rowptr(lr);

@@ -602,7 +602,7 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
             };
             const int n = (int)(u1 - u0);
             const int pre = n < NS ? n : NS;
-            const uint64_t wpol = l2_evict_first_policy();  // the weights are read once
+            const uint64_t wpol = evict_first_policy();  // the weights are read once
             // weight tiles of the first stages before the dependency wait
             // (weights never depend on the previous kernel)
             restart();

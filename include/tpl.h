@@ -152,8 +152,10 @@ void tpl_plan_destroy(tpl_plan *plan);
  * measure against).  TPL_OPT_DECODE_ATTN selects the decode attention kernel:
  * 0 = keys staged through a per-warp shared-memory ring (the default for
  * query groups of at most 8 heads when every (shard, sequence, kv head) pair
- * gets at least two CTAs in one wave of SMs; other shapes use the other
- * kernel), 1 = keys streamed into registers (any shape), 2 = the cache
+ * gets at least two CTAs in one wave of SMs, and the cache streamed by TMA
+ * (below) when the pairs fit one wave and each has at least 8192 cached keys;
+ * other shapes use the register kernel), 1 = keys streamed into registers
+ * (any shape), 2 = the cache
  * streamed by TMA into a shared-memory ring, every SM taking an equal share
  * of all pairs' 64-key blocks (groups of at most 8 heads and S >= 1; other
  * cases as 0).

@@ -419,18 +419,23 @@ int run_qkv(Ctx &c, const char *packed, const tpl_kv *kv, const void *x, float *
 bool g_stg_attr[64];
 
 // Which decode attention kernel runs and its split geometry.
-//   TPL_OPT_DECODE_ATTN 0 (default): the staged kernel for groups of at most
-//     8 heads with at least two CTAs per pair in one wave (where it measured
-//     faster; with one CTA per pair the register-streamed kernel's finer
-//     splits win), else the register-streamed kernel;
+//   TPL_OPT_DECODE_ATTN 0 (default): the TMA-streamed kernel for groups of at
+//     most 8 heads when the pairs fit one wave of SMs and each has at least
+//     kAttnTmaMinKeys cached keys (70B layer, batch 16, 8192 keys: 96.8 us
+//     against 104.9); else the staged kernel for groups of at most 8 heads
+//     with at least two CTAs per pair in one wave; else the register-streamed
+//     kernel (with one CTA per pair its finer splits win);
 //   1: the register-streamed kernel;
 //   2: the TMA-streamed kernel (groups of at most 8 heads, at least one
 //      cached key), else as 0.
 enum { ATTN_REG = 0, ATTN_STAGED = 1, ATTN_TMA = 2 };
+constexpr int64_t kAttnTmaMinKeys = 8192;
 int attn_select(const tpl_plan *p, int B, int64_t keys, AttnGeom *g, int *kind) {
     const int sms = num_sms_current();
     if (sms <= 0) return TPL_ECUDA;
-    if (p->attn_decode_mode == 2 && p->g <= kAmMaxG && keys >= 1 && keys <= 0x7fffffffll) {
+    const bool tma_ok = p->g <= kAmMaxG && keys >= 1 && keys <= 0x7fffffffll;
+    const bool tma_auto = p->attn_decode_mode == 0 && B * p->d.n_kv_heads <= sms && keys >= kAttnTmaMinKeys;
+    if (tma_ok && (p->attn_decode_mode == 2 || tma_auto)) {
         attn_geom_tma(B, p->d.n_kv_heads, keys, sms, g);
         *kind = ATTN_TMA;
     } else if (p->attn_decode_mode != 1 && p->g <= 8 && 2 * B * p->d.n_kv_heads <= sms) {
@@ -521,7 +526,7 @@ int attn_launch(const tpl_plan *p, const tpl_kv *kv, const float *q, const float
                 return TPL_ECUDA;
             g_stg_attr[dev] = true;
         }
-        return cuda_rc(launch_pdl(attn_decode_staged_kernel, grid, kAttnWarps * 32, kStgSmem, st, a));
+        return cuda_rc(launch_pdl(attn_decode_staged_kernel, grid, kAttnWarps * 32 + 32, kStgSmem, st, a));
     }
     return cuda_rc(p->g <= 8 ? launch_pdl(attn_decode_kernel<true>, grid, kAttnWarps * 32, 0, st, a)
                               : launch_pdl(attn_decode_kernel<false>, grid, kAttnWarps * 32, 0, st, a));

@@ -394,126 +394,7 @@ constexpr int kStgRow = 136;                           // padded row, bf16 eleme
 constexpr int kStgStep = 2 * 16 * kStgRow;             // K and V rows of one stage, elements
 constexpr size_t kStgSmem = (size_t)kAttnWarps * kStgStages * kStgStep * 2;  // dynamic bytes
 
-// The end of a staged-kernel CTA: the warps' (max, sum, output) in s_o /
-// s_ml merged in warp order into the CTA's partial, the arrival counter of
-// the pair, and for the last CTA of the pair the ordered combine of the CTA
-// partials and the new token.  It runs once per CTA at the very end, where
-// its code would be cold (fetched from L2 line by line, several us): it is
-// one non-inlined copy that a fifth warp runs once at the start with `dry`
-// set (stores to a shared scratch word, loads from the start of q with their
-// values discarded, no counter update, the last-CTA path taken), so that it
-// is in the instruction cache when the four working warps need it.  The real
-// call uses named barrier 1 (the 128 working threads); tid / warp are the
-// thread's index among them (the dry run: its lane, warp 0).
-__device__ __noinline__ void stg_finish(const AttnArgs &a, int pair, int chunk, int cpp, int b, int j,
-                                        const float *s_o, const float *s_ml, bool dry, int tid, int warp) {
-    constexpr int D = 128;
-    const int lane = tid & 31;
-    const int nthr = dry ? 32 : kAttnWarps * 32;
-    const int dim = tid;
-    auto sync = [&]() {
-        if (dry) __syncwarp();
-        else asm volatile("bar.sync 1, %0;" ::"n"(kAttnWarps * 32) : "memory");
-    };
-    __shared__ float s_dummy[4];
-    __shared__ float s_w[kAttnMaxCtasPerPair][8];
-    __shared__ float s_M[8], s_den[8], s_new[8];
-    __shared__ float s_mlp[kAttnMaxCtasPerPair * 8 * 2];
-    __shared__ float s_red[kAttnWarps][8];
-    __shared__ int s_last;
-    const int64_t cbase = ((int64_t)pair * cpp + chunk) * a.g;
-    float *po_w = dry ? s_dummy : a.part_o + cbase * D + dim;
-    float *pm_w = dry ? s_dummy : a.part_ml + cbase * 2;
-    const int64_t so = dry ? 0 : D, sm = dry ? 0 : 2;
-    for (int hrow = 0; hrow < a.g; ++hrow) {
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, s_ml[(w * 8 + hrow) * 2]);
-        float num = 0.f, den = 0.f;
-#pragma unroll
-        for (int w = 0; w < kAttnWarps; ++w) {
-            const float mi = s_ml[(w * 8 + hrow) * 2];
-            const float wt = mi == -INFINITY ? 0.f : exp2f(mi - M);
-            num += wt * s_o[(w * 8 + hrow) * D + dim];
-            den += wt * s_ml[(w * 8 + hrow) * 2 + 1];
-        }
-        po_w[hrow * so] = num;
-        if (dim == 0) {
-            pm_w[hrow * sm + 0] = M;
-            pm_w[hrow * sm + 1] = den;
-        }
-    }
-    __threadfence();
-    sync();
-    if (tid == 0) {
-        if (dry) {
-            s_dummy[1] = 1.f;
-        } else {
-            const unsigned prev = atomicAdd(&a.tickets[pair], 1u);
-            s_last = prev == (unsigned)(cpp - 1);
-            if (prev >= (unsigned)cpp) record_error(2u);
-        }
-    }
-    sync();
-    if (!dry && !s_last) return;
-    __threadfence();
-    const bool has_new = a.k_new != nullptr;
-    float *mlp = dry ? s_dummy : s_mlp;
-    const float *pm_r = dry ? a.q : a.part_ml + (int64_t)pair * cpp * a.g * 2;
-    for (int i = tid; i < cpp * a.g * 2; i += nthr) mlp[dry ? 0 : i] = __ldcg(pm_r + (dry ? 0 : i));
-    if (has_new) {
-        const float kd = a.k_new[((int64_t)b * (a.nq / a.g) + j) * D + dim];
-        for (int hrow = 0; hrow < a.g; ++hrow) {
-            float v = a.q[((int64_t)b * a.nq + (int64_t)j * a.g + hrow) * D + dim] * kd;
-#pragma unroll
-            for (int o2 = 16; o2 > 0; o2 >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o2);
-            if (lane == 0) (dry ? s_dummy : &s_red[warp][0])[dry ? 0 : hrow] = v;
-        }
-        sync();
-        if (tid < a.g) {
-            float v = 0.f;
-#pragma unroll
-            for (int w = 0; w < kAttnWarps; ++w) v += dry ? s_dummy[0] : s_red[w][tid];
-            (dry ? s_dummy : s_new)[dry ? 0 : tid] = v * a.scale_log2;
-        }
-    }
-    sync();
-    if (tid < a.g) {
-        const int hrow = tid;
-        const float *nw = dry ? s_dummy : s_new;
-        float M = has_new ? nw[dry ? 0 : hrow] : -INFINITY;
-        for (int i = 0; i < cpp; ++i) M = fmaxf(M, mlp[dry ? 0 : (i * a.g + hrow) * 2]);
-        float den = 0.f;
-        for (int i = 0; i < cpp; ++i) {
-            const float mi = mlp[dry ? 0 : (i * a.g + hrow) * 2];
-            const float wt = mi == -INFINITY ? 0.f : exp2f(mi - M);
-            (dry ? s_dummy : &s_w[0][0])[dry ? 0 : i * 8 + hrow] = wt;
-            den += wt * mlp[dry ? 0 : (i * a.g + hrow) * 2 + 1];
-        }
-        if (has_new) den += exp2f(nw[dry ? 0 : hrow] - M);
-        (dry ? s_dummy : s_M)[dry ? 0 : hrow] = M;
-        (dry ? s_dummy : s_den)[dry ? 0 : hrow] = den;
-    }
-    sync();
-    const int64_t sp = dry ? 0 : (int64_t)a.g * D;
-    const float *wv = dry ? s_dummy : &s_w[0][0];
-    const float *Mv = dry ? s_dummy : s_M;
-    const float *dv = dry ? s_dummy : s_den;
-    const float *nv = dry ? s_dummy : s_new;
-    for (int hrow = 0; hrow < a.g; ++hrow) {
-        float num = 0.f;
-        const float *po = dry ? a.q : a.part_o + ((int64_t)pair * cpp * a.g + hrow) * D + dim;
-        const int hs = dry ? 0 : hrow;
-#pragma unroll 8
-        for (int i = 0; i < cpp; ++i) num += wv[dry ? 0 : i * 8 + hs] * __ldcg(po + i * sp);
-        if (has_new) num += exp2f(nv[hs] - Mv[hs]) * a.v_new[((int64_t)b * (a.nq / a.g) + j) * D + dim];
-        if (dry) s_dummy[2] = num / dv[hs];
-        else store_act(a.o, a.o_f32, ((int64_t)b * a.nq + (int64_t)j * a.g + hrow) * D + dim, num / dv[hs]);
-    }
-    if (tid == 0 && !dry) atomicExch(&a.tickets[pair], 0u);
-}
-
-__global__ void __launch_bounds__(kAttnWarps * 32 + 32, 1) attn_decode_staged_kernel(const __grid_constant__ AttnArgs a) {
+__global__ void __launch_bounds__(kAttnWarps * 32, 1) attn_decode_staged_kernel(const __grid_constant__ AttnArgs a) {
     constexpr int D = 128;
     extern __shared__ __align__(128) __nv_bfloat16 stg_smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -532,159 +413,230 @@ __global__ void __launch_bounds__(kAttnWarps * 32 + 32, 1) attn_decode_staged_ke
     const int64_t k1 = min(a.keys, k0 + a.kps);
     const int nsteps = k1 > k0 ? (int)((k1 - k0 + 15) / 16) : 0;
     const bool early = a.k_new != nullptr;
-    __shared__ float s_o[kAttnWarps][8][D];
-    __shared__ float s_ml[kAttnWarps][8][2];
-    // The fifth warp runs the end-of-kernel code (stg_finish) once, dry, into
-    // the instruction cache (no dependency wait: it reads q and the new k/v
-    // only to discard them), then tells the working warps it is done.  One
-    // call site serves both, so that the cached code is the code they run.
-    const bool warm = warp == kAttnWarps;
     TPL_TRACE_VARS
-    if (!warm) {
-        if (threadIdx.x == 0) TPL_TRACE_AT(0);
-        __nv_bfloat16 *ring = stg_smem + (size_t)warp * kStgStages * kStgStep;
+    if (threadIdx.x == 0) TPL_TRACE_AT(0);
+    __nv_bfloat16 *ring = stg_smem + (size_t)warp * kStgStages * kStgStep;
 
-        const uint64_t kvpol = evict_first_policy();  // the cache is read once
-        // stage st (keys k0 + 16 st ..) into slot st % kStgStages; keys past k1 read as zero
-        auto issue = [&](int st) {
-            if (st < nsteps) {
-                __nv_bfloat16 *kd = ring + (st % kStgStages) * kStgStep;
-                __nv_bfloat16 *vd = kd + 16 * kStgRow;
-                const int64_t kb = k0 + 16 * (int64_t)st;
+    const uint64_t kvpol = evict_first_policy();  // the cache is read once
+    // stage st (keys k0 + 16 st ..) into slot st % kStgStages; keys past k1 read as zero
+    auto issue = [&](int st) {
+        if (st < nsteps) {
+            __nv_bfloat16 *kd = ring + (st % kStgStages) * kStgStep;
+            __nv_bfloat16 *vd = kd + 16 * kStgRow;
+            const int64_t kb = k0 + 16 * (int64_t)st;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int piece = lane + 32 * i;  // 256 pieces of 16 bytes: 16 rows x 16
-                    const int r = piece >> 4, col = (piece & 15) * 8;
-                    const int64_t key = kb + r;
-                    if (key < k1) {
-                        cp_async16_hint(kd + r * kStgRow + col, Kp + key * D + col, kvpol);
-                        cp_async16_hint(vd + r * kStgRow + col, Vp + key * D + col, kvpol);
-                    } else {
-                        *reinterpret_cast<uint4 *>(kd + r * kStgRow + col) = make_uint4(0, 0, 0, 0);
-                        *reinterpret_cast<uint4 *>(vd + r * kStgRow + col) = make_uint4(0, 0, 0, 0);
-                    }
+            for (int i = 0; i < 8; ++i) {
+                const int piece = lane + 32 * i;  // 256 pieces of 16 bytes: 16 rows x 16
+                const int r = piece >> 4, col = (piece & 15) * 8;
+                const int64_t key = kb + r;
+                if (key < k1) {
+                    cp_async16_hint(kd + r * kStgRow + col, Kp + key * D + col, kvpol);
+                    cp_async16_hint(vd + r * kStgRow + col, Vp + key * D + col, kvpol);
+                } else {
+                    *reinterpret_cast<uint4 *>(kd + r * kStgRow + col) = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4 *>(vd + r * kStgRow + col) = make_uint4(0, 0, 0, 0);
                 }
             }
-            cp_async_commit();  // one group per stage, empty ones included
-        };
-        if (early)
-            for (int st = 0; st < kStgStages - 1; ++st) issue(st);
-        pdl_wait();
-        pdl_trigger();
-        if (threadIdx.x == 0) TPL_TRACE_AT(1);
-        if (!early)
-            for (int st = 0; st < kStgStages - 1; ++st) issue(st);
-
-        // q fragments: rows gid (hi) / gid + 8 (lo) of head gid, dims 16ks + 2c (+1, +8, +9)
-        uint32_t qf[8][4];
-        {
-            const bool live = gid < a.g;
-            const float *qp = a.q + ((int64_t)b * a.nq + (int64_t)j * a.g + (live ? gid : 0)) * D;
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                float2 u = make_float2(0.f, 0.f), w = make_float2(0.f, 0.f);
-                if (live) {
-                    u = *reinterpret_cast<const float2 *>(qp + 16 * ks + 2 * c);
-                    w = *reinterpret_cast<const float2 *>(qp + 16 * ks + 2 * c + 8);
-                }
-                const uint32_t h0 = pack_bf16x2(u.x, u.y), h2 = pack_bf16x2(w.x, w.y);
-                qf[ks][0] = h0;
-                qf[ks][1] = pack_bf16x2(u.x - bf16lo(h0), u.y - bf16hi(h0));
-                qf[ks][2] = h2;
-                qf[ks][3] = pack_bf16x2(w.x - bf16lo(h2), w.y - bf16hi(h2));
-            }
         }
+        cp_async_commit();  // one group per stage, empty ones included
+    };
+    if (early)
+        for (int st = 0; st < kStgStages - 1; ++st) issue(st);
+    pdl_wait();
+    pdl_trigger();
+    if (threadIdx.x == 0) TPL_TRACE_AT(1);
+    if (!early)
+        for (int st = 0; st < kStgStages - 1; ++st) issue(st);
 
-        float o[16][4];
+    // q fragments: rows gid (hi) / gid + 8 (lo) of head gid, dims 16ks + 2c (+1, +8, +9)
+    uint32_t qf[8][4];
+    {
+        const bool live = gid < a.g;
+        const float *qp = a.q + ((int64_t)b * a.nq + (int64_t)j * a.g + (live ? gid : 0)) * D;
 #pragma unroll
-        for (int t = 0; t < 16; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
-        float m_a = -INFINITY, l_a = 0.f;  // head gid: running max (log2 domain), lane-partial sum
-
-        for (int st = 0; st < nsteps; ++st) {
-            issue(st + kStgStages - 1);
-            asm volatile("cp.async.wait_group %0;" ::"n"(kStgStages - 1) : "memory");
-            __syncwarp();
-            const __nv_bfloat16 *Ks = ring + (st % kStgStages) * kStgStep;
-            const __nv_bfloat16 *Vs = Ks + 16 * kStgRow;
-            float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const int r = (lane & 7) + ((lane >> 4) << 3);
-                const int col = 16 * ks + ((lane >> 3) & 1) * 8;
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4(Ks + r * kStgRow + col, b0, b1, b2, b3);
-                mma_bf16_16816(s0, qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], b0, b1);
-                mma_bf16_16816(s1, qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], b2, b3);
+        for (int ks = 0; ks < 8; ++ks) {
+            float2 u = make_float2(0.f, 0.f), w = make_float2(0.f, 0.f);
+            if (live) {
+                u = *reinterpret_cast<const float2 *>(qp + 16 * ks + 2 * c);
+                w = *reinterpret_cast<const float2 *>(qp + 16 * ks + 2 * c + 8);
             }
-            // logits: hi rows + lo rows of the same head; keys kb + 2c, +1 (tile 0), kb + 8 + 2c, +1 (tile 1)
-            const int64_t kk = k0 + 16 * (int64_t)st + 2 * c;
-            const float x0 = kk < k1 ? (s0[0] + s0[2]) * a.scale_log2 : -INFINITY;
-            const float x1 = kk + 1 < k1 ? (s0[1] + s0[3]) * a.scale_log2 : -INFINITY;
-            const float x2 = kk + 8 < k1 ? (s1[0] + s1[2]) * a.scale_log2 : -INFINITY;
-            const float x3 = kk + 9 < k1 ? (s1[1] + s1[3]) * a.scale_log2 : -INFINITY;
-            float mx = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-            const float mn = fmaxf(m_a, mx);  // finite: the first key of every step is in range
-            const float alpha = exp2f(m_a - mn);
-            m_a = mn;
-            const float p0 = exp2f(x0 - mn), p1 = exp2f(x1 - mn), p2 = exp2f(x2 - mn), p3 = exp2f(x3 - mn);
-            l_a = l_a * alpha + ((p0 + p1) + (p2 + p3));
-#pragma unroll
-            for (int t = 0; t < 16; ++t) {
-                o[t][0] *= alpha;
-                o[t][1] *= alpha;
-                o[t][2] *= alpha;
-                o[t][3] *= alpha;
-            }
-            const uint32_t ph0 = pack_bf16x2(p0, p1), ph2 = pack_bf16x2(p2, p3);
-            const uint32_t pl0 = pack_bf16x2(p0 - bf16lo(ph0), p1 - bf16hi(ph0));
-            const uint32_t pl2 = pack_bf16x2(p2 - bf16lo(ph2), p3 - bf16hi(ph2));
-#pragma unroll
-            for (int n2 = 0; n2 < 8; ++n2) {
-                const int r = (lane & 7) + (((lane >> 3) & 1) << 3);
-                const int col = 16 * n2 + ((lane >> 4) << 3);
-                uint32_t v0, v1, v2, v3;
-                ldsm_x4_t(Vs + r * kStgRow + col, v0, v1, v2, v3);
-                mma_bf16_16816(o[2 * n2], ph0, pl0, ph2, pl2, v0, v1);
-                mma_bf16_16816(o[2 * n2 + 1], ph0, pl0, ph2, pl2, v2, v3);
-            }
-            __syncwarp();  // this slot is refilled by a later issue()
+            const uint32_t h0 = pack_bf16x2(u.x, u.y), h2 = pack_bf16x2(w.x, w.y);
+            qf[ks][0] = h0;
+            qf[ks][1] = pack_bf16x2(u.x - bf16lo(h0), u.y - bf16hi(h0));
+            qf[ks][2] = h2;
+            qf[ks][3] = pack_bf16x2(w.x - bf16lo(h2), w.y - bf16hi(h2));
         }
-        asm volatile("cp.async.wait_group 0;" ::: "memory");
-        if (threadIdx.x == 0) TPL_TRACE_AT(2);
-        // rows gid + 8 held the P_lo . V half of the same head
+    }
+
+    float o[16][4];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
+    float m_a = -INFINITY, l_a = 0.f;  // head gid: running max (log2 domain), lane-partial sum
+
+    for (int st = 0; st < nsteps; ++st) {
+        issue(st + kStgStages - 1);
+        asm volatile("cp.async.wait_group %0;" ::"n"(kStgStages - 1) : "memory");
+        __syncwarp();
+        const __nv_bfloat16 *Ks = ring + (st % kStgStages) * kStgStep;
+        const __nv_bfloat16 *Vs = Ks + 16 * kStgRow;
+        float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            const int r = (lane & 7) + ((lane >> 4) << 3);
+            const int col = 16 * ks + ((lane >> 3) & 1) * 8;
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4(Ks + r * kStgRow + col, b0, b1, b2, b3);
+            mma_bf16_16816(s0, qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], b0, b1);
+            mma_bf16_16816(s1, qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], b2, b3);
+        }
+        // logits: hi rows + lo rows of the same head; keys kb + 2c, +1 (tile 0), kb + 8 + 2c, +1 (tile 1)
+        const int64_t kk = k0 + 16 * (int64_t)st + 2 * c;
+        const float x0 = kk < k1 ? (s0[0] + s0[2]) * a.scale_log2 : -INFINITY;
+        const float x1 = kk + 1 < k1 ? (s0[1] + s0[3]) * a.scale_log2 : -INFINITY;
+        const float x2 = kk + 8 < k1 ? (s1[0] + s1[2]) * a.scale_log2 : -INFINITY;
+        const float x3 = kk + 9 < k1 ? (s1[1] + s1[3]) * a.scale_log2 : -INFINITY;
+        float mx = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        const float mn = fmaxf(m_a, mx);  // finite: the first key of every step is in range
+        const float alpha = exp2f(m_a - mn);
+        m_a = mn;
+        const float p0 = exp2f(x0 - mn), p1 = exp2f(x1 - mn), p2 = exp2f(x2 - mn), p3 = exp2f(x3 - mn);
+        l_a = l_a * alpha + ((p0 + p1) + (p2 + p3));
 #pragma unroll
         for (int t = 0; t < 16; ++t) {
-            o[t][0] += o[t][2];
-            o[t][1] += o[t][3];
+            o[t][0] *= alpha;
+            o[t][1] *= alpha;
+            o[t][2] *= alpha;
+            o[t][3] *= alpha;
         }
-        l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
-        l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
-
-        // ---- merge the CTA's warps (ascending warp order), then the CTA partials ----
-        if (gid < a.g) {
+        const uint32_t ph0 = pack_bf16x2(p0, p1), ph2 = pack_bf16x2(p2, p3);
+        const uint32_t pl0 = pack_bf16x2(p0 - bf16lo(ph0), p1 - bf16hi(ph0));
+        const uint32_t pl2 = pack_bf16x2(p2 - bf16lo(ph2), p3 - bf16hi(ph2));
 #pragma unroll
-            for (int t = 0; t < 16; ++t) {
-                s_o[warp][gid][8 * t + 2 * c] = o[t][0];
-                s_o[warp][gid][8 * t + 2 * c + 1] = o[t][1];
-            }
-            if (c == 0) {
-                s_ml[warp][gid][0] = m_a;
-                s_ml[warp][gid][1] = l_a;
-            }
+        for (int n2 = 0; n2 < 8; ++n2) {
+            const int r = (lane & 7) + (((lane >> 3) & 1) << 3);
+            const int col = 16 * n2 + ((lane >> 4) << 3);
+            uint32_t v0, v1, v2, v3;
+            ldsm_x4_t(Vs + r * kStgRow + col, v0, v1, v2, v3);
+            mma_bf16_16816(o[2 * n2], ph0, pl0, ph2, pl2, v0, v1);
+            mma_bf16_16816(o[2 * n2 + 1], ph0, pl0, ph2, pl2, v2, v3);
         }
-        // the warm-up warp is done with the shared arrays stg_finish uses
-        asm volatile("bar.sync 2, %0;" ::"n"(kAttnWarps * 32 + 32) : "memory");
-        asm volatile("bar.sync 1, %0;" ::"n"(kAttnWarps * 32) : "memory");
-    }  // !warm
-    stg_finish(a, pair, chunk, cpp, b, j, &s_o[0][0][0], &s_ml[0][0][0], warm, warm ? lane : (int)threadIdx.x,
-               warm ? 0 : warp);
-    if (warm) {
-        asm volatile("bar.arrive 2, %0;" ::"n"(kAttnWarps * 32 + 32) : "memory");
+        __syncwarp();  // this slot is refilled by a later issue()
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    if (threadIdx.x == 0) TPL_TRACE_AT(2);
+    // rows gid + 8 held the P_lo . V half of the same head
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+        o[t][0] += o[t][2];
+        o[t][1] += o[t][3];
+    }
+    l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
+    l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
+
+    // ---- merge the CTA's warps (ascending warp order), then the CTA partials ----
+    __shared__ float s_o[kAttnWarps][8][D];
+    __shared__ float s_ml[kAttnWarps][8][2];
+    if (gid < a.g) {
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+            s_o[warp][gid][8 * t + 2 * c] = o[t][0];
+            s_o[warp][gid][8 * t + 2 * c + 1] = o[t][1];
+        }
+        if (c == 0) {
+            s_ml[warp][gid][0] = m_a;
+            s_ml[warp][gid][1] = l_a;
+        }
+    }
+    __syncthreads();
+    const int dim = threadIdx.x;
+    const int64_t cbase = ((int64_t)pair * cpp + chunk) * a.g;
+    for (int hrow = 0; hrow < a.g; ++hrow) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, s_ml[w][hrow][0]);
+        float num = 0.f, den = 0.f;
+#pragma unroll
+        for (int w = 0; w < kAttnWarps; ++w) {
+            const float mi = s_ml[w][hrow][0];
+            const float wt = mi == -INFINITY ? 0.f : exp2f(mi - M);
+            num += wt * s_o[w][hrow][dim];
+            den += wt * s_ml[w][hrow][1];
+        }
+        a.part_o[(cbase + hrow) * D + dim] = num;
+        if (dim == 0) {
+            a.part_ml[(cbase + hrow) * 2 + 0] = M;
+            a.part_ml[(cbase + hrow) * 2 + 1] = den;
+        }
+    }
+    __shared__ int s_last;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const unsigned prev = atomicAdd(&a.tickets[pair], 1u);
+        s_last = prev == (unsigned)(cpp - 1);
+        if (prev >= (unsigned)cpp) record_error(2u);
+    }
+    __syncthreads();
+    if (!s_last) {
+        if (threadIdx.x == 0) {
+            TPL_TRACE_AT(3);
+            TPL_TRACE_PUT(TR_ATTN);
+        }
         return;
     }
+    __threadfence();
+    __shared__ float s_w[kAttnMaxCtasPerPair][8];
+    __shared__ float s_M[8], s_den[8], s_new[8];
+    __shared__ float s_mlp[kAttnMaxCtasPerPair * 8 * 2];
+    const bool has_new = a.k_new != nullptr;
+    for (int i = threadIdx.x; i < cpp * a.g * 2; i += blockDim.x)
+        s_mlp[i] = __ldcg(&a.part_ml[(int64_t)pair * cpp * a.g * 2 + i]);
+    if (has_new) {
+        __shared__ float s_red[kAttnWarps][8];
+        const float kd = a.k_new[((int64_t)b * (a.nq / a.g) + j) * D + dim];
+        for (int hrow = 0; hrow < a.g; ++hrow) {
+            float v = a.q[((int64_t)b * a.nq + (int64_t)j * a.g + hrow) * D + dim] * kd;
+#pragma unroll
+            for (int o2 = 16; o2 > 0; o2 >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o2);
+            if (lane == 0) s_red[warp][hrow] = v;
+        }
+        __syncthreads();
+        if (threadIdx.x < a.g) {
+            float v = 0.f;
+#pragma unroll
+            for (int w = 0; w < kAttnWarps; ++w) v += s_red[w][threadIdx.x];
+            s_new[threadIdx.x] = v * a.scale_log2;
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < a.g) {
+        const int hrow = threadIdx.x;
+        float M = has_new ? s_new[hrow] : -INFINITY;
+        for (int i = 0; i < cpp; ++i) M = fmaxf(M, s_mlp[(i * a.g + hrow) * 2]);
+        float den = 0.f;
+        for (int i = 0; i < cpp; ++i) {
+            const float mi = s_mlp[(i * a.g + hrow) * 2];
+            const float wt = mi == -INFINITY ? 0.f : exp2f(mi - M);
+            s_w[i][hrow] = wt;
+            den += wt * s_mlp[(i * a.g + hrow) * 2 + 1];
+        }
+        if (has_new) den += exp2f(s_new[hrow] - M);
+        s_M[hrow] = M;
+        s_den[hrow] = den;
+    }
+    __syncthreads();
+    for (int hrow = 0; hrow < a.g; ++hrow) {
+        float num = 0.f;
+        const float *po = a.part_o + ((int64_t)pair * cpp * a.g + hrow) * D + dim;
+#pragma unroll 8
+        for (int i = 0; i < cpp; ++i) num += s_w[i][hrow] * __ldcg(po + (int64_t)i * a.g * D);
+        if (has_new) num += exp2f(s_new[hrow] - s_M[hrow]) * a.v_new[((int64_t)b * (a.nq / a.g) + j) * D + dim];
+        store_act(a.o, a.o_f32, ((int64_t)b * a.nq + (int64_t)j * a.g + hrow) * D + dim, num / s_den[hrow]);
+    }
     if (threadIdx.x == 0) {
+        atomicExch(&a.tickets[pair], 0u);
         TPL_TRACE_AT(3);
         TPL_TRACE_PUT(TR_ATTN);
     }

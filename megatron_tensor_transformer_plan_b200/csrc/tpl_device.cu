@@ -526,7 +526,7 @@ int attn_launch(const tpl_plan *p, const tpl_kv *kv, const float *q, const float
                 return TPL_ECUDA;
             g_stg_attr[dev] = true;
         }
-        return cuda_rc(launch_pdl(attn_decode_staged_kernel, grid, kAttnWarps * 32 + 32, kStgSmem, st, a));
+        return cuda_rc(launch_pdl(attn_decode_staged_kernel, grid, kAttnWarps * 32, kStgSmem, st, a));
     }
     return cuda_rc(p->g <= 8 ? launch_pdl(attn_decode_kernel<true>, grid, kAttnWarps * 32, 0, st, a)
                               : launch_pdl(attn_decode_kernel<false>, grid, kAttnWarps * 32, 0, st, a));

@@ -11,11 +11,9 @@
 // 64-column weight tiles (16 KB, 128-byte swizzle) and the matching activation
 // tile into a 4-8 stage shared-memory ring, one thread issues four M=128,
 // N=NX, K=16 tcgen05.mma per stage, and the tensor pipe idles most of the
-// time.  224 threads: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer,
+// time.  192 threads: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer,
 // warps 2-5 epilogue (one TMEM lane = one weight row each), which walks the
-// tokens in chunks of 16 columns so that its registers do not grow with B,
-// and warp 6, which only runs the end-of-kernel code once, dry, at the start
-// (gt_final), so that it is in the instruction cache when the kernel ends.
+// tokens in chunks of 16 columns so that its registers do not grow with B.
 //
 // Work division ("stream-K"): the k-blocks of every (row tile, segment) are
 // laid end to end, tile-major then segment then k, and each CTA takes one
@@ -48,7 +46,7 @@
 
 namespace tpl {
 
-constexpr int kGtThreads = 224;  // 6 working warps + the instruction-cache warm-up warp
+constexpr int kGtThreads = 192;
 constexpr int kGtRows = 128;     // weight rows per tile (MMA M)
 constexpr int kGtK = 64;         // columns per k-block
 constexpr int kGtWBytes = kGtRows * kGtK * 2;  // 16 KB
@@ -172,29 +170,24 @@ __device__ __forceinline__ GtOrder gt_order(int64_t u0, int64_t u1, int64_t per_
 }
 
 // Final write of one output row for tokens tok0 .. tok0+15 (fused sums or
-// column ops).
-//
-// This and gt_combine run at the end of the kernel, once per CTA: cold, their
-// instructions were fetched from L2 line by line, which measured 7-15 us per
-// kernel (a second run of the same code took 1-2 us).  Both are therefore not
-// inlined (one copy of the code) and a spare warp runs them once at the start
-// with `dry` set: every loop and branch taken as for a full chunk of tokens,
-// every store sent to a shared-memory scratch word and every load to the start
-// of the workspace's piece area (valid global memory whose values are
-// discarded), so the instruction cache holds them when the real call comes.
-__device__ __noinline__ void gt_final(const GemvTcArgs &a, int row, const float (&v0)[kGtChunk], int lane, int tok0,
-                                      const float *inv_rms, bool dry, float *dummy) {
-    const int B = dry ? tok0 + kGtChunk : a.B;
+// column ops).  This and gt_combine run at the end of the kernel, once per
+// CTA, where their code is cold (fetched from L2 line by line, which measured
+// several us): both are kept short -- per-row destinations computed once, a
+// few stores per token, the piece list built in parallel.  (Non-inlined
+// copies, and a spare warp running them early to warm the instruction cache,
+// both measured slower.)
+__device__ __forceinline__ void gt_final(const GemvTcArgs &a, int row, const float (&v0)[kGtChunk], int lane, int tok0,
+                                      const float *inv_rms) {
+    const int B = a.B;
     const bool scale = a.rms_src && a.epi != GT_ROW;  // the RMSNorm factor of column ops
     float v[kGtChunk];
 #pragma unroll
     for (int i = 0; i < kGtChunk; ++i) v[i] = scale ? v0[i] * inv_rms[min(tok0 + i, kGtMaxB - 1)] : v0[i];
     if (a.epi == GT_GU) {
         // rows interleave gate and up: the even lane pairs with its odd neighbour
-        const bool w = !(lane & 1) && (dry || row + 1 < a.N);
-        __nv_bfloat16 *dst = dry ? reinterpret_cast<__nv_bfloat16 *>(dummy)
-                                 : static_cast<__nv_bfloat16 *>(a.out_act) + row / 2;
-        const int64_t st = dry ? 0 : a.N / 2;
+        const bool w = !(lane & 1) && row + 1 < a.N;
+        __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(a.out_act) + row / 2;
+        const int64_t st = a.N / 2;
 #pragma unroll
         for (int i = 0; i < kGtChunk; ++i) {
             const int b = tok0 + i;
@@ -203,13 +196,13 @@ __device__ __noinline__ void gt_final(const GemvTcArgs &a, int row, const float 
         }
         return;
     }
-    if (!dry && row >= a.N) return;
+    if (row >= a.N) return;
     if (a.epi == GT_QKV) {
         // the row is one q element, or one k or v element of the cache (and
         // its fp32 copy); per token only the batch stride moves
         const int s = row / a.rps, l = row % a.rps;
         const int qd = a.nq_s * a.hd, kd = a.nkv_s * a.hd;
-        const bool isq = dry ? (row & 1) != 0 : l < qd;  // a dry run takes both paths
+        const bool isq = l < qd;
         const bool isk = l < qd + kd;
         const int ll = isk ? l - qd : l - qd - kd;  // kv head * hd + dim within the shard
         float *dq = a.q + (int64_t)s * qd + l;
@@ -217,14 +210,8 @@ __device__ __noinline__ void gt_final(const GemvTcArgs &a, int row, const float 
                             (int64_t)(ll / a.hd) * a.seq_cap * a.hd + ll % a.hd;
         float *dn = isk ? a.knew : a.vnew;
         if (dn) dn += (int64_t)s * kd + ll;
-        int64_t sq = (int64_t)a.nq * a.hd, sc = (int64_t)a.nkv_s * a.seq_cap * a.hd,
-                sn = (int64_t)a.nkv_s * (a.nq / a.nq_s) * a.hd;
-        if (dry) {
-            dq = dummy;
-            dc = reinterpret_cast<__nv_bfloat16 *>(dummy);
-            dn = dummy;
-            sq = sc = sn = 0;
-        }
+        const int64_t sq = (int64_t)a.nq * a.hd, sc = (int64_t)a.nkv_s * a.seq_cap * a.hd,
+                      sn = (int64_t)a.nkv_s * (a.nq / a.nq_s) * a.hd;
 #pragma unroll
         for (int i = 0; i < kGtChunk; ++i) {
             const int b = tok0 + i;
@@ -238,57 +225,51 @@ __device__ __noinline__ void gt_final(const GemvTcArgs &a, int row, const float 
         }
         return;
     }
-    // GT_ROW: out = resid + sum
-    const int64_t st = dry ? 0 : a.N;
-    const int64_t i0 = dry ? 0 : row;
-    const void *resid = dry && a.resid ? static_cast<const void *>(a.gpart) : a.resid;
-    float *o32 = dry && a.out32 ? dummy : a.out32;
-    __nv_bfloat16 *oact = dry && a.out_act ? reinterpret_cast<__nv_bfloat16 *>(dummy)
-                                           : static_cast<__nv_bfloat16 *>(a.out_act);
-    __nv_bfloat16 *xs = dry && a.xs_out ? reinterpret_cast<__nv_bfloat16 *>(dummy) : a.xs_out;
-    const float *xg = dry && a.xs_gamma ? a.gpart : a.xs_gamma;
-    const int64_t xrow = dry ? 0 : row, xhalf = dry ? 0 : (int64_t)a.xs_half * a.N;
-    // every load before any store (the pointers may alias as far as the
-    // compiler knows, which would otherwise serialise the loads' latencies)
+    // GT_ROW: out = resid + sum.  Every load before any store (the pointers
+    // may alias as far as the compiler knows, which would otherwise
+    // serialise the loads' latencies).
     float rv[kGtChunk];
 #pragma unroll
     for (int j = 0; j < kGtChunk; ++j)
-        rv[j] = (resid && tok0 + j < B) ? load_act(resid, a.resid_f32, (tok0 + j) * st + i0) : 0.f;
-    const float gam = xg ? xg[xrow] : 1.f;
+        rv[j] = (a.resid && tok0 + j < B) ? load_act(a.resid, a.resid_f32, (int64_t)(tok0 + j) * a.N + row) : 0.f;
+    const float gam = a.xs_gamma ? a.xs_gamma[row] : 1.f;
+    __nv_bfloat16 *oact = static_cast<__nv_bfloat16 *>(a.out_act);
 #pragma unroll
     for (int j = 0; j < kGtChunk; ++j) {
         const int b = tok0 + j;
         if (b >= B) continue;
-        const int64_t i = b * st + i0;
-        const float o = resid ? rv[j] + v[j] : v[j];
-        if (o32) o32[i] = o;
+        const int64_t i = (int64_t)b * a.N + row;
+        const float o = a.resid ? rv[j] + v[j] : v[j];
+        if (a.out32) a.out32[i] = o;
         if (oact) oact[i] = __float2bfloat16_rn(o);
-        if (xs) {
-            // split_scaled with the row's gain loaded once
+        if (a.xs_out) {
+            // the next projection's operand: split_scaled with the row's gain loaded once
             const float src = oact ? __bfloat162float(__float2bfloat16_rn(o)) : o;
-            const float sc = xg ? __fmul_rn(src, gam) : src;
+            const float sc = a.xs_gamma ? __fmul_rn(src, gam) : src;
             const __nv_bfloat16 hi = __float2bfloat16_rn(sc);
-            xs[i] = hi;
-            xs[xhalf + i] = __float2bfloat16_rn(__fsub_rn(sc, __bfloat162float(hi)));
+            a.xs_out[i] = hi;
+            a.xs_out[(int64_t)(a.xs_half + b) * a.N + row] = __float2bfloat16_rn(__fsub_rn(sc, __bfloat162float(hi)));
         }
     }
 }
 
 // The CTA that completed a tile split across CTAs adds its pieces in the
-// fixed order (segment, then CTA) and writes the tile.  The pieces are listed
-// by one thread in shared memory (in rounds of up to kGtList entries), then
-// loaded eight at a time; the walk is repeated for each 16-token chunk,
-// reusing the list when one round held it all.  Each CTA stored its part in
-// slot 0 if the tile is its first, else in slot 1.  Run by the 128 epilogue
-// threads (named barrier 1); `dry` as for gt_final, run by the one warm-up
-// warp (no barrier, its own list area).
-__device__ __noinline__ void gt_combine(const GemvTcArgs &a, int tile, int G, int nch, int r, int lane, int ep_tid,
+// fixed order (segment, then CTA) and writes the tile.  The CTAs cf..cl cover
+// the tile; with at most 128 (segment, CTA) candidates the 128 epilogue
+// threads test one each and compact the list in candidate order, else one
+// thread generates it in rounds of up to kGtList entries.  The pieces are
+// then loaded (with at most 4 tokens in the chunk one float4 each, 16 in
+// flight; else 8 pieces of 4 float4) and added in list order; the walk is
+// repeated for each 16-token chunk, reusing the list when one round held it
+// all.  Each CTA stored its part in slot 0 if the tile is its first, else in
+// slot 1.  Run by the 128 epilogue threads (named barrier 1).
+__device__ __forceinline__ void gt_combine(const GemvTcArgs &a, int tile, int G, int nch, int r, int lane, int ep_tid,
                                         const float *s_inv, volatile int *s_list, volatile int *s_nlist,
-                                        volatile int *s_more, volatile int *s_cnt, float *dummy, bool dry) {
+                                        volatile int *s_more, volatile int *s_cnt) {
     const int64_t per_tile = (int64_t)a.nseg * a.kbs;
     const int64_t t_beg = (int64_t)tile * per_tile;
     const int row = tile * kGtRows + r;
-    const int B = dry ? kGtChunk * nch : a.B;
+    const int B = a.B;
     float seg_sum[kGtChunk], tile_sum[kGtChunk];
     bool single = false;  // the whole list is in shared memory
 #ifdef TPL_TRACE
@@ -304,10 +285,6 @@ __device__ __noinline__ void gt_combine(const GemvTcArgs &a, int tile, int G, in
             tile_sum[t] = -0.f;
             seg_sum[t] = -0.f;
         }
-        // The CTAs cf..cl cover the tile.  With at most 128 (segment, CTA)
-        // candidates, the 128 threads test one each and the list is compacted
-        // in candidate order (segment-major, CTAs ascending); otherwise one
-        // thread generates it in rounds.
         int cf = (int)((t_beg * G) / a.U);
         while (cf > 0 && gt_start(a.U, G, cf) > t_beg) --cf;
         while (gt_start(a.U, G, cf + 1) <= t_beg) ++cf;
@@ -315,11 +292,10 @@ __device__ __noinline__ void gt_combine(const GemvTcArgs &a, int tile, int G, in
         while (cl + 1 < G && gt_start(a.U, G, cl + 1) < t_beg + per_tile) ++cl;
         const int ncta = cl - cf + 1, ncand = a.nseg * ncta;
         if (!single && ncand <= 128) {
-            const int k = dry ? lane : ep_tid;
-            const int g_s = k / ncta, c = cf + k % ncta;
+            const int g_s = ep_tid / ncta, c = cf + ep_tid % ncta;
             bool valid = false;
             int ent = 0;
-            if (k < ncand) {
+            if (ep_tid < ncand) {
                 const int64_t sb = t_beg + (int64_t)g_s * a.kbs, se = sb + a.kbs;
                 const int64_t c0 = gt_start(a.U, G, c), c1 = gt_start(a.U, G, c + 1);
                 valid = c1 > sb && c0 < se;
@@ -327,22 +303,20 @@ __device__ __noinline__ void gt_combine(const GemvTcArgs &a, int tile, int G, in
                 ent = (((c * 2 + sl) * a.nseg + g_s) << 5) | (g_s << 1) | (c1 >= se ? 1 : 0);
             }
             const unsigned m = __ballot_sync(0xffffffffu, valid);
-            const int w = dry ? 0 : ep_tid >> 5;
+            const int w = ep_tid >> 5;
             if (lane == 0) s_cnt[w] = __popc(m);
-            if (dry) __syncwarp();
-            else asm volatile("bar.sync 1, 128;" ::: "memory");
+            asm volatile("bar.sync 1, 128;" ::: "memory");
             int base = 0;
             for (int x = 0; x < w; ++x) base += s_cnt[x];
             const int pos = base + __popc(m & ((1u << lane) - 1u));
-            if (valid && pos < kGtList) s_list[dry ? 0 : pos] = ent;
+            if (valid && pos < kGtList) s_list[pos] = ent;
             if (ep_tid == 0) {
                 const int tot = s_cnt[0] + s_cnt[1] + s_cnt[2] + s_cnt[3];
                 *s_nlist = tot < kGtList ? tot : kGtList;
                 *s_more = 0;
             }
-            if (dry) __syncwarp();
-            else asm volatile("bar.sync 1, 128;" ::: "memory");
-            single = *s_nlist < kGtList || dry;  // a full list may have dropped entries: generate it instead
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            single = *s_nlist < kGtList;  // a full list may have dropped entries: generate it instead
         }
         int g_s = 0, g_cc = cf;  // generator position (thread 0)
         for (int round = 0;; ++round) {
@@ -366,16 +340,9 @@ __device__ __noinline__ void gt_combine(const GemvTcArgs &a, int tile, int G, in
                     *s_nlist = n;
                     *s_more = g_s < a.nseg ? 1 : 0;
                 }
-                if (dry) __syncwarp();
-                else asm volatile("bar.sync 1, 128;" ::: "memory");
+                asm volatile("bar.sync 1, 128;" ::: "memory");
             }
-            // At most 4 tokens in this chunk: one float4 per piece, up to 16
-            // pieces' loads in flight, a short branch-free body per piece.
-            // Else 16 tokens (4 float4 per piece), 8 pieces per round.  The
-            // choice follows the real token count, also in a dry run, whose
-            // loads are predicated off.
-            const bool narrow = a.B - tok0 <= 4;
-            const int n = dry ? (narrow ? 16 : 8) : *s_nlist;
+            const int n = *s_nlist;
 #ifdef TPL_TRACE
             if (ch == 0 && round == 0) ck[1] = (uint64_t)clock64();
 #endif
@@ -383,7 +350,7 @@ __device__ __noinline__ void gt_combine(const GemvTcArgs &a, int tile, int G, in
                 return reinterpret_cast<const float4 *>(a.gpart) +
                        ((int64_t)(ent >> 5) * (a.gstride / 4) + tok0 / 4) * kGtRows + r;
             };
-            if (narrow) {
+            if (B - tok0 <= 4) {
                 float4 seg4 = make_float4(seg_sum[0], seg_sum[1], seg_sum[2], seg_sum[3]);
                 float4 tile4 = make_float4(tile_sum[0], tile_sum[1], tile_sum[2], tile_sum[3]);
                 for (int e0 = 0; e0 < n; e0 += 16) {
@@ -391,26 +358,25 @@ __device__ __noinline__ void gt_combine(const GemvTcArgs &a, int tile, int G, in
                     int en[16];
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
-                        en[j] = e0 + j < n ? s_list[dry ? 0 : e0 + j] : 0;
-                        v1[j] = (e0 + j < n && !dry) ? __ldcg(piece_src(en[j])) : make_float4(0.f, 0.f, 0.f, 0.f);
+                        en[j] = e0 + j < n ? s_list[e0 + j] : 0;
+                        v1[j] = e0 + j < n ? __ldcg(piece_src(en[j])) : make_float4(0.f, 0.f, 0.f, 0.f);
                     }
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
-                        if (!dry && e0 + j >= n) break;
+                        if (e0 + j >= n) break;
                         seg4.x = seg4.x + v1[j].x;
                         seg4.y = seg4.y + v1[j].y;
                         seg4.z = seg4.z + v1[j].z;
                         seg4.w = seg4.w + v1[j].w;
-                        if (dry || (en[j] & 1)) {  // the segment is complete
+                        if (en[j] & 1) {  // the segment is complete
                             if (a.epi == GT_ROW_PARTIAL) {
-                                if (dry || row < a.N) {
+                                if (row < a.N) {
                                     const int sg = (en[j] >> 1) & 15;
-                                    float *dst = dry ? dummy : a.partials + ((int64_t)sg * B + tok0) * a.N + row;
-                                    const int64_t st = dry ? 0 : a.N;
+                                    float *dst = a.partials + ((int64_t)sg * B + tok0) * a.N + row;
                                     const float w4[4] = {seg4.x, seg4.y, seg4.z, seg4.w};
 #pragma unroll
                                     for (int t = 0; t < 4; ++t)
-                                        if (tok0 + t < B) dst[t * st] = w4[t];
+                                        if (tok0 + t < B) dst[t * a.N] = w4[t];
                                 }
                             } else {
                                 tile4.x = tile4.x + seg4.x;
@@ -436,16 +402,16 @@ __device__ __noinline__ void gt_combine(const GemvTcArgs &a, int tile, int G, in
                     int en[8];
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        en[j] = e0 + j < n ? s_list[dry ? 0 : e0 + j] : 0;
+                        en[j] = e0 + j < n ? s_list[e0 + j] : 0;
                         const float4 *src = piece_src(en[j]);
 #pragma unroll
                         for (int q4 = 0; q4 < kGtChunk / 4; ++q4)
-                            v[j][q4] = (e0 + j < n && tok0 + 4 * q4 < B && !dry) ? __ldcg(src + q4 * kGtRows)
-                                                                                : make_float4(0.f, 0.f, 0.f, 0.f);
+                            v[j][q4] = (e0 + j < n && tok0 + 4 * q4 < B) ? __ldcg(src + q4 * kGtRows)
+                                                                        : make_float4(0.f, 0.f, 0.f, 0.f);
                     }
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        if (!dry && e0 + j >= n) break;
+                        if (e0 + j >= n) break;
 #pragma unroll
                         for (int q4 = 0; q4 < kGtChunk / 4; ++q4) {
                             seg_sum[4 * q4] = seg_sum[4 * q4] + v[j][q4].x;
@@ -453,15 +419,14 @@ __device__ __noinline__ void gt_combine(const GemvTcArgs &a, int tile, int G, in
                             seg_sum[4 * q4 + 2] = seg_sum[4 * q4 + 2] + v[j][q4].z;
                             seg_sum[4 * q4 + 3] = seg_sum[4 * q4 + 3] + v[j][q4].w;
                         }
-                        if (dry || (en[j] & 1)) {  // the segment is complete
+                        if (en[j] & 1) {  // the segment is complete
                             const int sg = (en[j] >> 1) & 15;
                             if (a.epi == GT_ROW_PARTIAL) {
-                                if (dry || row < a.N) {
-                                    float *dst = dry ? dummy : a.partials + ((int64_t)sg * B + tok0) * a.N + row;
-                                    const int64_t st = dry ? 0 : a.N;
+                                if (row < a.N) {
+                                    float *dst = a.partials + ((int64_t)sg * B + tok0) * a.N + row;
 #pragma unroll
                                     for (int t = 0; t < kGtChunk; ++t)
-                                        if (tok0 + t < B) dst[t * st] = seg_sum[t];
+                                        if (tok0 + t < B) dst[t * a.N] = seg_sum[t];
                                 }
                             } else {
 #pragma unroll
@@ -478,19 +443,18 @@ __device__ __noinline__ void gt_combine(const GemvTcArgs &a, int tile, int G, in
 #endif
             if (single) break;
             const bool more = *s_more != 0;
-            if (dry) __syncwarp();
-            else asm volatile("bar.sync 1, 128;" ::: "memory");  // list consumed before it is rewritten
+            asm volatile("bar.sync 1, 128;" ::: "memory");  // list consumed before it is rewritten
             if (!more) {
                 single = round == 0;  // one round held the whole list: keep it
                 break;
             }
         }
-        if (a.epi != GT_ROW_PARTIAL) gt_final(a, row, tile_sum, lane, tok0, s_inv, dry, dummy);
+        if (a.epi != GT_ROW_PARTIAL) gt_final(a, row, tile_sum, lane, tok0, s_inv);
 #ifdef TPL_TRACE
         if (ch == 0) {
             ck[3] = (uint64_t)clock64();
-            if (ep_tid == 0) trace_put((dry ? 300 : 200) + a.trace_row_tag * 0 + (a.epi == GT_QKV ? TR_QKV
-                                       : a.epi == GT_GU ? TR_GU : a.trace_row_tag), ck);
+            if (ep_tid == 0)
+                trace_put(200 + (a.epi == GT_QKV ? TR_QKV : a.epi == GT_GU ? TR_GU : a.trace_row_tag), ck);
         }
 #endif
     }
@@ -512,9 +476,7 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
     uint64_t *full = reinterpret_cast<uint64_t *>(sm + NS * STAGE + SMEM::TSBYTES);
     float *s_rpart = reinterpret_cast<float *>(sm + NS * STAGE + SMEM::TSBYTES + kGtBarBytes);  // [4][kGtMaxB]
     float *s_inv = s_rpart + 4 * kGtMaxB;                                                       // [kGtMaxB]
-    float *s_dummy = s_inv + kGtMaxB;  // [16]: the scratch words of the early dry run of the combine code
-    volatile int *w_list = reinterpret_cast<volatile int *>(s_dummy + 16);  // [kGtList + 6]: its piece list
-    static_assert(5 * kGtMaxB * 4 + 64 + 4 * (kGtList + 6) <= kGtRmsBytes, "rms area");
+    static_assert(5 * kGtMaxB * 4 <= kGtRmsBytes, "rms area");
     uint64_t *empty = full + NS;
     uint64_t *acc_full = empty + NS;        // [BUFS]
     uint64_t *acc_empty = acc_full + BUFS;  // [BUFS]
@@ -677,14 +639,6 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
             umma_commit(fin);
             if (!mbar_wait(fin, 0)) *s_fail = 1;
         }
-    } else if (warp == 6) {
-        // ---- warm-up: the end-of-kernel code once, dry, into the instruction cache.
-        //      No dependency wait: it reads only the start of the piece area
-        //      (values discarded) and writes only this CTA's shared scratch,
-        //      so it can run while the preceding kernel finishes ----
-        const int nch = min((a.B + kGtChunk - 1) / kGtChunk, SMEM::NCH);
-        gt_combine(a, 0, G, nch, 32 * (lane & 3) + lane, lane, lane, s_inv, w_list + 2, w_list, w_list + 1,
-                   w_list + 2 + kGtList, s_dummy, true);
     } else {
         pdl_wait();
         // ---- epilogue: thread = weight row 32*(warp%4) + lane of the tile ----
@@ -811,7 +765,7 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
                         const float *tsp = ts + (kGtChunk * ch) * kGtRows + r;
 #pragma unroll
                         for (int t = 0; t < kGtChunk; ++t) tile_sum[t] = tsp[t * kGtRows];
-                        gt_final(a, row, tile_sum, lane, kGtChunk * ch, s_inv, false, s_dummy);
+                        gt_final(a, row, tile_sum, lane, kGtChunk * ch, s_inv);
                     }
                 }
                 continue;
@@ -843,8 +797,7 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
             asm volatile("bar.sync 1, 128;" ::: "memory");
             if (!*s_last) continue;
             __threadfence();
-            gt_combine(a, tile, G, nch, r, lane, ep_tid, s_inv, s_list, s_nlist, s_more, s_list + kGtList, s_dummy,
-                       false);
+            gt_combine(a, tile, G, nch, r, lane, ep_tid, s_inv, s_list, s_nlist, s_more, s_list + kGtList);
             if (ep_tid == 0) TPL_TRACE_AT(3);
         }
         if (ep_tid == 0 && ep_traced)

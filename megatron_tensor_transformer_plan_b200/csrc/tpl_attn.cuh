@@ -45,6 +45,101 @@ struct AttnArgs {
     int o_f32;
 };
 
+// The last CTA of a (shard, sequence, kv head) pair: the CTA partials in
+// ascending order, then the new token's key/value in fp32, for the g <= MAXG
+// heads of the pair; one thread per head dimension (128 threads, named as
+// `dim`).  Every global load is issued before the first store: with up to 8
+// partials per pair (the usual case) all of them at once, since a load after
+// a store of the loop before would wait for it (the compiler cannot rule out
+// aliasing), and each round trip to L2 costs about a microsecond at the end
+// of the kernel (with more partials, or more than 8 heads, in smaller
+// batches).  s_mlp holds the partials' (max, sum) [cpp][g][2]; the other
+// shared arrays are scratch.
+template <int MAXG>
+__device__ __forceinline__ void attn_pair_combine(const AttnArgs &a, int pair, int cpp, int b, int j, int dim,
+                                                  int lane, int warp, const float *s_mlp, float (*s_w)[MAXG],
+                                                  float *s_M, float *s_den, float *s_new, float (*s_red)[MAXG]) {
+    constexpr int D = 128;
+    const bool has_new = a.k_new != nullptr;
+    const int64_t kv_i = ((int64_t)b * (a.nq / a.g) + j) * D + dim;
+    const int64_t q0 = ((int64_t)b * a.nq + (int64_t)j * a.g) * D + dim;
+    float vnew = 0.f;
+    if (has_new) {
+        // logits of the new token for the g heads, fp32, fixed-order reduction
+        const float kd = a.k_new[kv_i];
+        vnew = a.v_new[kv_i];
+        float qv[MAXG];
+#pragma unroll
+        for (int h = 0; h < MAXG; ++h) qv[h] = h < a.g ? a.q[q0 + (int64_t)h * D] : 0.f;
+#pragma unroll
+        for (int h = 0; h < MAXG; ++h) {
+            if (h >= a.g) break;
+            float v = qv[h] * kd;
+#pragma unroll
+            for (int o2 = 16; o2 > 0; o2 >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o2);
+            if (lane == 0) s_red[warp][h] = v;
+        }
+        __syncthreads();
+        if (threadIdx.x < a.g) {
+            float v = 0.f;
+#pragma unroll
+            for (int w = 0; w < kAttnWarps; ++w) v += s_red[w][threadIdx.x];
+            s_new[threadIdx.x] = v * a.scale_log2;
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < a.g) {
+        const int hrow = threadIdx.x;
+        float M = has_new ? s_new[hrow] : -INFINITY;
+        for (int i = 0; i < cpp; ++i) M = fmaxf(M, s_mlp[(i * a.g + hrow) * 2]);
+        float den = 0.f;
+        for (int i = 0; i < cpp; ++i) {
+            const float mi = s_mlp[(i * a.g + hrow) * 2];
+            const float wt = mi == -INFINITY ? 0.f : exp2f(mi - M);
+            s_w[i][hrow] = wt;
+            den += wt * s_mlp[(i * a.g + hrow) * 2 + 1];
+        }
+        if (has_new) den += exp2f(s_new[hrow] - M);
+        s_M[hrow] = M;
+        s_den[hrow] = den;
+    }
+    __syncthreads();
+    const float *po = a.part_o + (int64_t)pair * cpp * a.g * D + dim;  // [cpp][g][D]
+    const int64_t ps = (int64_t)a.g * D;
+    constexpr int CB = MAXG > 8 ? 4 : 8;  // partials loaded at once per head (registers: MAXG * CB)
+    float num[MAXG];
+    if (cpp <= CB) {
+        float pv[MAXG][CB];
+#pragma unroll
+        for (int h = 0; h < MAXG; ++h)
+#pragma unroll
+            for (int i = 0; i < CB; ++i) pv[h][i] = (h < a.g && i < cpp) ? __ldcg(po + i * ps + h * D) : 0.f;
+#pragma unroll
+        for (int h = 0; h < MAXG; ++h) {
+            float n = 0.f;
+#pragma unroll
+            for (int i = 0; i < CB; ++i)
+                if (i < cpp) n += s_w[i][h] * pv[h][i];
+            num[h] = n;
+        }
+    } else {
+#pragma unroll
+        for (int h = 0; h < MAXG; ++h) {
+            float n = 0.f;
+            if (h < a.g)
+                for (int i = 0; i < cpp; ++i) n += s_w[i][h] * __ldcg(po + i * ps + h * D);
+            num[h] = n;
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < MAXG; ++h) {
+        if (h >= a.g) break;
+        float n = num[h];
+        if (has_new) n += exp2f(s_new[h] - s_M[h]) * vnew;
+        store_act(a.o, a.o_f32, q0 + (int64_t)h * D, n / s_den[h]);
+    }
+}
+
 template <bool PACKED>  // PACKED: g <= 8, q/P low parts in rows 8-15
 __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const __grid_constant__ AttnArgs a) {
     constexpr int D = 128;
@@ -321,53 +416,11 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const __gr
     // stage every CTA partial's (max, sum) for this pair
     __shared__ float s_w[64][16];  // weights exp2(m_i - M) per CTA partial and head
     __shared__ float s_M[16], s_den[16], s_new[16];
-    const bool has_new = a.k_new != nullptr;
+    __shared__ float s_red[kAttnWarps][16];
     float *s_mlp = &s_o[0][0][0];  // reuse: [cpp][g][2] (cpp <= 64)
     for (int i = threadIdx.x; i < cpp_ * a.g * 2; i += blockDim.x)
         s_mlp[i] = __ldcg(&a.part_ml[(int64_t)pair * cpp_ * a.g * 2 + i]);
-    if (has_new) {
-        // logits of the new token for the g heads, fp32, fixed-order reduction
-        __shared__ float s_red[kAttnWarps][16];
-        const float kd = a.k_new[((int64_t)b * (a.nq / a.g) + j) * D + dim];
-        for (int hrow = 0; hrow < a.g; ++hrow) {
-            float v = a.q[((int64_t)b * a.nq + (int64_t)j * a.g + hrow) * D + dim] * kd;
-#pragma unroll
-            for (int o2 = 16; o2 > 0; o2 >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o2);
-            if (lane == 0) s_red[warp][hrow] = v;
-        }
-        __syncthreads();
-        if (threadIdx.x < a.g) {
-            float v = 0.f;
-#pragma unroll
-            for (int w = 0; w < kAttnWarps; ++w) v += s_red[w][threadIdx.x];
-            s_new[threadIdx.x] = v * a.scale_log2;
-        }
-    }
-    __syncthreads();
-    if (threadIdx.x < a.g) {
-        const int hrow = threadIdx.x;
-        float M = has_new ? s_new[hrow] : -INFINITY;
-        for (int i = 0; i < cpp_; ++i) M = fmaxf(M, s_mlp[(i * a.g + hrow) * 2]);
-        float den = 0.f;
-        for (int i = 0; i < cpp_; ++i) {
-            const float mi = s_mlp[(i * a.g + hrow) * 2];
-            const float wt = mi == -INFINITY ? 0.f : exp2f(mi - M);
-            s_w[i][hrow] = wt;
-            den += wt * s_mlp[(i * a.g + hrow) * 2 + 1];
-        }
-        if (has_new) den += exp2f(s_new[hrow] - M);
-        s_M[hrow] = M;
-        s_den[hrow] = den;
-    }
-    __syncthreads();
-    for (int hrow = 0; hrow < a.g; ++hrow) {
-        float num = 0.f;
-        const float *po = a.part_o + ((int64_t)pair * cpp_ * a.g + hrow) * D + dim;
-#pragma unroll 8
-        for (int i = 0; i < cpp_; ++i) num += s_w[i][hrow] * __ldcg(po + (int64_t)i * a.g * D);
-        if (has_new) num += exp2f(s_new[hrow] - s_M[hrow]) * a.v_new[((int64_t)b * (a.nq / a.g) + j) * D + dim];
-        store_act(a.o, a.o_f32, ((int64_t)b * a.nq + (int64_t)j * a.g + hrow) * D + dim, num / s_den[hrow]);
-    }
+    attn_pair_combine<16>(a, pair, cpp_, b, j, dim, lane, warp, s_mlp, s_w, s_M, s_den, s_new, s_red);
     if (threadIdx.x == 0) {
         atomicExch(&a.tickets[pair], 0u);
         TPL_TRACE_AT(3);
@@ -526,6 +579,11 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) attn_decode_staged_kernel(
     }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
     if (threadIdx.x == 0) TPL_TRACE_AT(2);
+#ifdef TPL_TRACE
+    // SM-clock marks of the end (traced builds): every warp's loop done,
+    // partial written, arrival counted, combine done
+    uint64_t ck[4] = {0, 0, 0, 0};
+#endif
     // rows gid + 8 held the P_lo . V half of the same head
 #pragma unroll
     for (int t = 0; t < 16; ++t) {
@@ -550,6 +608,9 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) attn_decode_staged_kernel(
         }
     }
     __syncthreads();
+#ifdef TPL_TRACE
+    if (threadIdx.x == 0) ck[0] = (uint64_t)clock64();
+#endif
     const int dim = threadIdx.x;
     const int64_t cbase = ((int64_t)pair * cpp + chunk) * a.g;
     for (int hrow = 0; hrow < a.g; ++hrow) {
@@ -573,16 +634,25 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) attn_decode_staged_kernel(
     __shared__ int s_last;
     __threadfence();
     __syncthreads();
+#ifdef TPL_TRACE
+    if (threadIdx.x == 0) ck[1] = (uint64_t)clock64();
+#endif
     if (threadIdx.x == 0) {
         const unsigned prev = atomicAdd(&a.tickets[pair], 1u);
         s_last = prev == (unsigned)(cpp - 1);
         if (prev >= (unsigned)cpp) record_error(2u);
     }
     __syncthreads();
+#ifdef TPL_TRACE
+    if (threadIdx.x == 0) ck[2] = ck[3] = (uint64_t)clock64();
+#endif
     if (!s_last) {
         if (threadIdx.x == 0) {
             TPL_TRACE_AT(3);
             TPL_TRACE_PUT(TR_ATTN);
+#ifdef TPL_TRACE
+            trace_put(202, ck);
+#endif
         }
         return;
     }
@@ -590,55 +660,18 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) attn_decode_staged_kernel(
     __shared__ float s_w[kAttnMaxCtasPerPair][8];
     __shared__ float s_M[8], s_den[8], s_new[8];
     __shared__ float s_mlp[kAttnMaxCtasPerPair * 8 * 2];
-    const bool has_new = a.k_new != nullptr;
+    __shared__ float s_red[kAttnWarps][8];
     for (int i = threadIdx.x; i < cpp * a.g * 2; i += blockDim.x)
         s_mlp[i] = __ldcg(&a.part_ml[(int64_t)pair * cpp * a.g * 2 + i]);
-    if (has_new) {
-        __shared__ float s_red[kAttnWarps][8];
-        const float kd = a.k_new[((int64_t)b * (a.nq / a.g) + j) * D + dim];
-        for (int hrow = 0; hrow < a.g; ++hrow) {
-            float v = a.q[((int64_t)b * a.nq + (int64_t)j * a.g + hrow) * D + dim] * kd;
-#pragma unroll
-            for (int o2 = 16; o2 > 0; o2 >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o2);
-            if (lane == 0) s_red[warp][hrow] = v;
-        }
-        __syncthreads();
-        if (threadIdx.x < a.g) {
-            float v = 0.f;
-#pragma unroll
-            for (int w = 0; w < kAttnWarps; ++w) v += s_red[w][threadIdx.x];
-            s_new[threadIdx.x] = v * a.scale_log2;
-        }
-    }
-    __syncthreads();
-    if (threadIdx.x < a.g) {
-        const int hrow = threadIdx.x;
-        float M = has_new ? s_new[hrow] : -INFINITY;
-        for (int i = 0; i < cpp; ++i) M = fmaxf(M, s_mlp[(i * a.g + hrow) * 2]);
-        float den = 0.f;
-        for (int i = 0; i < cpp; ++i) {
-            const float mi = s_mlp[(i * a.g + hrow) * 2];
-            const float wt = mi == -INFINITY ? 0.f : exp2f(mi - M);
-            s_w[i][hrow] = wt;
-            den += wt * s_mlp[(i * a.g + hrow) * 2 + 1];
-        }
-        if (has_new) den += exp2f(s_new[hrow] - M);
-        s_M[hrow] = M;
-        s_den[hrow] = den;
-    }
-    __syncthreads();
-    for (int hrow = 0; hrow < a.g; ++hrow) {
-        float num = 0.f;
-        const float *po = a.part_o + ((int64_t)pair * cpp * a.g + hrow) * D + dim;
-#pragma unroll 8
-        for (int i = 0; i < cpp; ++i) num += s_w[i][hrow] * __ldcg(po + (int64_t)i * a.g * D);
-        if (has_new) num += exp2f(s_new[hrow] - s_M[hrow]) * a.v_new[((int64_t)b * (a.nq / a.g) + j) * D + dim];
-        store_act(a.o, a.o_f32, ((int64_t)b * a.nq + (int64_t)j * a.g + hrow) * D + dim, num / s_den[hrow]);
-    }
+    attn_pair_combine<8>(a, pair, cpp, b, j, dim, lane, warp, s_mlp, s_w, s_M, s_den, s_new, s_red);
     if (threadIdx.x == 0) {
         atomicExch(&a.tickets[pair], 0u);
         TPL_TRACE_AT(3);
         TPL_TRACE_PUT(TR_ATTN);
+#ifdef TPL_TRACE
+        ck[3] = (uint64_t)clock64();
+        trace_put(212, ck);
+#endif
     }
 }
 

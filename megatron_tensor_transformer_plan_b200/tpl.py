@@ -132,7 +132,7 @@ class tpl_trace_rec(ctypes.Structure):
 TRACE_TAGS = {1: "qkv", 2: "attention", 3: "o_proj", 4: "gate_up", 5: "down", 6: "operand", 7: "reduce",
               101: "qkv.epi", 103: "o_proj.epi", 104: "gate_up.epi", 105: "down.epi",
               201: "qkv.clk", 203: "o_proj.clk", 204: "gate_up.clk", 205: "down.clk",
-              301: "qkv.dry", 303: "o_proj.dry", 304: "gate_up.dry", 305: "down.dry"}
+              202: "attention.clk", 212: "attention_last.clk"}
 
 
 def trace_read(max_records: int = 1 << 18):

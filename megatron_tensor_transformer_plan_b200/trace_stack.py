@@ -134,10 +134,10 @@ def main() -> None:
         plan.decode_stack(packed, kvs, x, S, y, None, ws)
         torch.cuda.synchronize()
         recs = tpl.trace_read()
-        main_recs = [r for r in recs if not r[0].endswith((".epi", ".clk", ".dry"))]
+        main_recs = [r for r in recs if not r[0].endswith((".epi", ".clk"))]
         epi_recs = [r for r in recs if r[0].endswith(".epi")]
         for r in recs:  # combine phases in SM cycles: list, loads and sums, final write
-            if r[0].endswith((".clk", ".dry")) and r[4][3] > r[4][0] > 0:
+            if r[0].endswith(".clk") and r[4][3] >= r[4][0] > 0:
                 t = r[4]
                 clk.setdefault(r[0], []).append((t[1] - t[0], t[2] - t[1], t[3] - t[2]))
         rows = summarise(launches(main_recs), epi_recs)

@@ -54,17 +54,27 @@ struct AttnArgs {
 // aliasing), and each round trip to L2 costs about a microsecond at the end
 // of the kernel (with more partials, or more than 8 heads, in smaller
 // batches).  s_mlp holds the partials' (max, sum) [cpp][g][2]; the other
-// shared arrays are scratch.
+// shared arrays are scratch.  With `early` the caller has already written the
+// warps' parts of the new token's logits to s_red (attn_new_logits) and
+// passes the new value's element as vnew.
 template <int MAXG>
 __device__ __forceinline__ void attn_pair_combine(const AttnArgs &a, int pair, int cpp, int b, int j, int dim,
                                                   int lane, int warp, const float *s_mlp, float (*s_w)[MAXG],
-                                                  float *s_M, float *s_den, float *s_new, float (*s_red)[MAXG]) {
+                                                  float *s_M, float *s_den, float *s_new, float (*s_red)[MAXG],
+                                                  bool early = false, float vnew_early = 0.f) {
     constexpr int D = 128;
     const bool has_new = a.k_new != nullptr;
     const int64_t kv_i = ((int64_t)b * (a.nq / a.g) + j) * D + dim;
     const int64_t q0 = ((int64_t)b * a.nq + (int64_t)j * a.g) * D + dim;
-    float vnew = 0.f;
-    if (has_new) {
+    float vnew = vnew_early;
+    if (has_new && early) {
+        if (threadIdx.x < a.g) {
+            float v = 0.f;
+#pragma unroll
+            for (int w = 0; w < kAttnWarps; ++w) v += s_red[w][threadIdx.x];
+            s_new[threadIdx.x] = v * a.scale_log2;
+        }
+    } else if (has_new) {
         // logits of the new token for the g heads, fp32, fixed-order reduction
         const float kd = a.k_new[kv_i];
         vnew = a.v_new[kv_i];
@@ -138,6 +148,34 @@ __device__ __forceinline__ void attn_pair_combine(const AttnArgs &a, int pair, i
         if (has_new) n += exp2f(s_new[h] - s_M[h]) * vnew;
         store_act(a.o, a.o_f32, q0 + (int64_t)h * D, n / s_den[h]);
     }
+}
+
+// The new token's logits for the pair's g heads, each warp's part of the
+// fixed-order sum over the head dimension into s_red[warp][h] (the same
+// arithmetic as attn_pair_combine's), computed by every CTA right after the
+// dependency wait so that the pair's last CTA finds them ready; returns the
+// thread's element of the new value.
+template <int MAXG>
+__device__ __forceinline__ float attn_new_logits(const AttnArgs &a, int b, int j, int dim, int lane, int warp,
+                                                 float (*s_red)[MAXG]) {
+    constexpr int D = 128;
+    if (!a.k_new) return 0.f;
+    const int64_t kv_i = ((int64_t)b * (a.nq / a.g) + j) * D + dim;
+    const int64_t q0 = ((int64_t)b * a.nq + (int64_t)j * a.g) * D + dim;
+    const float kd = a.k_new[kv_i];
+    const float vnew = a.v_new[kv_i];
+    float qv[MAXG];
+#pragma unroll
+    for (int h = 0; h < MAXG; ++h) qv[h] = h < a.g ? a.q[q0 + (int64_t)h * D] : 0.f;
+#pragma unroll
+    for (int h = 0; h < MAXG; ++h) {
+        if (h >= a.g) break;
+        float v = qv[h] * kd;
+#pragma unroll
+        for (int o2 = 16; o2 > 0; o2 >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o2);
+        if (lane == 0) s_red[warp][h] = v;
+    }
+    return vnew;
 }
 
 template <bool PACKED>  // PACKED: g <= 8, q/P low parts in rows 8-15
@@ -521,6 +559,10 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) attn_decode_staged_kernel(
         }
     }
 
+    // the new token's logits, for whichever CTA of the pair finishes last
+    __shared__ float s_red[kAttnWarps][8];
+    const float vnew = attn_new_logits<8>(a, b, j, threadIdx.x, lane, warp, s_red);
+
     float o[16][4];
 #pragma unroll
     for (int t = 0; t < 16; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
@@ -660,10 +702,9 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) attn_decode_staged_kernel(
     __shared__ float s_w[kAttnMaxCtasPerPair][8];
     __shared__ float s_M[8], s_den[8], s_new[8];
     __shared__ float s_mlp[kAttnMaxCtasPerPair * 8 * 2];
-    __shared__ float s_red[kAttnWarps][8];
     for (int i = threadIdx.x; i < cpp * a.g * 2; i += blockDim.x)
         s_mlp[i] = __ldcg(&a.part_ml[(int64_t)pair * cpp * a.g * 2 + i]);
-    attn_pair_combine<8>(a, pair, cpp, b, j, dim, lane, warp, s_mlp, s_w, s_M, s_den, s_new, s_red);
+    attn_pair_combine<8>(a, pair, cpp, b, j, dim, lane, warp, s_mlp, s_w, s_M, s_den, s_new, s_red, true, vnew);
     if (threadIdx.x == 0) {
         atomicExch(&a.tickets[pair], 0u);
         TPL_TRACE_AT(3);

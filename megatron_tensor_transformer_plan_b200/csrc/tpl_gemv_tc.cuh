@@ -176,8 +176,25 @@ __device__ __forceinline__ GtOrder gt_order(int64_t u0, int64_t u1, int64_t per_
 // few stores per token, the piece list built in parallel.  (Non-inlined
 // copies, and a spare warp running them early to warm the instruction cache,
 // both measured slower.)
+// The loads the row-parallel final write needs (the residual of the chunk's
+// tokens and the row's gain for the next operand), issued early so that
+// their latency overlaps the combine's own loads.
+struct GtRowIn {
+    float rv[kGtChunk];
+    float gam;
+};
+__device__ __forceinline__ void gt_row_loads(const GemvTcArgs &a, int row, int tok0, GtRowIn &in) {
+    const int B = a.B;
+    const bool ok = row < a.N;
+#pragma unroll
+    for (int j = 0; j < kGtChunk; ++j)
+        in.rv[j] = (ok && a.resid && tok0 + j < B) ? load_act(a.resid, a.resid_f32, (int64_t)(tok0 + j) * a.N + row)
+                                                    : 0.f;
+    in.gam = (ok && a.xs_gamma) ? a.xs_gamma[row] : 1.f;
+}
+
 __device__ __forceinline__ void gt_final(const GemvTcArgs &a, int row, const float (&v0)[kGtChunk], int lane, int tok0,
-                                      const float *inv_rms) {
+                                      const float *inv_rms, const GtRowIn *pre = nullptr) {
     const int B = a.B;
     const bool scale = a.rms_src && a.epi != GT_ROW;  // the RMSNorm factor of column ops
     float v[kGtChunk];
@@ -227,12 +244,12 @@ __device__ __forceinline__ void gt_final(const GemvTcArgs &a, int row, const flo
     }
     // GT_ROW: out = resid + sum.  Every load before any store (the pointers
     // may alias as far as the compiler knows, which would otherwise
-    // serialise the loads' latencies).
-    float rv[kGtChunk];
-#pragma unroll
-    for (int j = 0; j < kGtChunk; ++j)
-        rv[j] = (a.resid && tok0 + j < B) ? load_act(a.resid, a.resid_f32, (int64_t)(tok0 + j) * a.N + row) : 0.f;
-    const float gam = a.xs_gamma ? a.xs_gamma[row] : 1.f;
+    // serialise the loads' latencies); the combine issues them even earlier.
+    GtRowIn in_local;
+    if (!pre) gt_row_loads(a, row, tok0, in_local);
+    const GtRowIn &in = pre ? *pre : in_local;
+    const float *rv = in.rv;
+    const float gam = in.gam;
     __nv_bfloat16 *oact = static_cast<__nv_bfloat16 *>(a.out_act);
 #pragma unroll
     for (int j = 0; j < kGtChunk; ++j) {
@@ -271,6 +288,7 @@ __device__ __forceinline__ void gt_combine(const GemvTcArgs &a, int tile, int G,
     const int row = tile * kGtRows + r;
     const int B = a.B;
     float seg_sum[kGtChunk], tile_sum[kGtChunk];
+    GtRowIn row_in;       // the row-parallel final write's loads, issued with the pieces'
     bool single = false;  // the whole list is in shared memory
 #ifdef TPL_TRACE
     // SM-clock marks of the first chunk (traced builds): start, list built,
@@ -350,6 +368,7 @@ __device__ __forceinline__ void gt_combine(const GemvTcArgs &a, int tile, int G,
                 return reinterpret_cast<const float4 *>(a.gpart) +
                        ((int64_t)(ent >> 5) * (a.gstride / 4) + tok0 / 4) * kGtRows + r;
             };
+            if (a.epi == GT_ROW && round == 0) gt_row_loads(a, row, tok0, row_in);
             if (B - tok0 <= 4) {
                 float4 seg4 = make_float4(seg_sum[0], seg_sum[1], seg_sum[2], seg_sum[3]);
                 float4 tile4 = make_float4(tile_sum[0], tile_sum[1], tile_sum[2], tile_sum[3]);
@@ -449,7 +468,7 @@ __device__ __forceinline__ void gt_combine(const GemvTcArgs &a, int tile, int G,
                 break;
             }
         }
-        if (a.epi != GT_ROW_PARTIAL) gt_final(a, row, tile_sum, lane, tok0, s_inv);
+        if (a.epi != GT_ROW_PARTIAL) gt_final(a, row, tile_sum, lane, tok0, s_inv, a.epi == GT_ROW ? &row_in : nullptr);
 #ifdef TPL_TRACE
         if (ch == 0) {
             ck[3] = (uint64_t)clock64();

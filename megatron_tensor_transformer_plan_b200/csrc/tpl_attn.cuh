@@ -54,7 +54,8 @@ struct AttnArgs {
 // aliasing), and each round trip to L2 costs about a microsecond at the end
 // of the kernel (with more partials, or more than 8 heads, in smaller
 // batches).  s_mlp holds the partials' (max, sum) [cpp][g][2]; the other
-// shared arrays are scratch.  With `early` the caller has already written the
+// shared arrays are scratch.  Run by the CTA's first 128 threads (named
+// barrier 1).  With `early` the caller has already written the
 // warps' parts of the new token's logits to s_red (attn_new_logits) and
 // passes the new value's element as vnew.
 template <int MAXG>
@@ -89,7 +90,7 @@ __device__ __forceinline__ void attn_pair_combine(const AttnArgs &a, int pair, i
             for (int o2 = 16; o2 > 0; o2 >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o2);
             if (lane == 0) s_red[warp][h] = v;
         }
-        __syncthreads();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
         if (threadIdx.x < a.g) {
             float v = 0.f;
 #pragma unroll
@@ -97,7 +98,7 @@ __device__ __forceinline__ void attn_pair_combine(const AttnArgs &a, int pair, i
             s_new[threadIdx.x] = v * a.scale_log2;
         }
     }
-    __syncthreads();
+    asm volatile("bar.sync 1, 128;" ::: "memory");
     if (threadIdx.x < a.g) {
         const int hrow = threadIdx.x;
         float M = has_new ? s_new[hrow] : -INFINITY;
@@ -113,7 +114,7 @@ __device__ __forceinline__ void attn_pair_combine(const AttnArgs &a, int pair, i
         s_M[hrow] = M;
         s_den[hrow] = den;
     }
-    __syncthreads();
+    asm volatile("bar.sync 1, 128;" ::: "memory");
     const float *po = a.part_o + (int64_t)pair * cpp * a.g * D + dim;  // [cpp][g][D]
     const int64_t ps = (int64_t)a.g * D;
     constexpr int CB = MAXG > 8 ? 4 : 8;  // partials loaded at once per head (registers: MAXG * CB)
@@ -480,19 +481,22 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const __gr
 //   O: A = P (rows 0-7 hi, rows 8-15 lo), B = 16 keys x 8 dims (ldmatrix.trans
 //      of V rows); output tile t holds dims 8t + 2c, 8t + 2c + 1.
 // ---------------------------------------------------------------------------
-constexpr int kStgStages = 4;
+constexpr int kStgWarps = kAttnStgWarps;               // two per SM sub-partition
+constexpr int kStgStages = 3;
 constexpr int kStgRow = 136;                           // padded row, bf16 elements
 constexpr int kStgStep = 2 * 16 * kStgRow;             // K and V rows of one stage, elements
-constexpr size_t kStgSmem = (size_t)kAttnWarps * kStgStages * kStgStep * 2;  // dynamic bytes
+constexpr size_t kStgSmem = (size_t)kStgWarps * kStgStages * kStgStep * 2;  // dynamic bytes
+static_assert((size_t)kStgWarps * 8 * (128 + 2) * 4 <= kStgSmem, "the warps' merge overlays the rings");
+constexpr float kStgLazy = 8.0f;  // the running maximum (log2 units) is raised only past this margin
 
-__global__ void __launch_bounds__(kAttnWarps * 32, 1) attn_decode_staged_kernel(const __grid_constant__ AttnArgs a) {
+__global__ void __launch_bounds__(kStgWarps * 32, 1) attn_decode_staged_kernel(const __grid_constant__ AttnArgs a) {
     constexpr int D = 128;
     extern __shared__ __align__(128) __nv_bfloat16 stg_smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gid = lane >> 2, c = lane & 3;
-    const int cpp = a.nsplit / kAttnWarps;
+    const int cpp = a.nsplit / kStgWarps;
     const int pair = blockIdx.x / cpp, chunk = blockIdx.x % cpp;
-    const int split = chunk * kAttnWarps + warp;
+    const int split = chunk * kStgWarps + warp;
     const int jl = pair % a.nkv_s;
     const int sb = pair / a.nkv_s;
     const int b = sb % a.B, s = sb / a.B;
@@ -560,8 +564,9 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) attn_decode_staged_kernel(
     }
 
     // the new token's logits, for whichever CTA of the pair finishes last
+    // (the first 128 threads: one head dimension each)
     __shared__ float s_red[kAttnWarps][8];
-    const float vnew = attn_new_logits<8>(a, b, j, threadIdx.x, lane, warp, s_red);
+    const float vnew = warp < kAttnWarps ? attn_new_logits<8>(a, b, j, threadIdx.x, lane, warp, s_red) : 0.f;
 
     float o[16][4];
 #pragma unroll
@@ -593,18 +598,22 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) attn_decode_staged_kernel(
         float mx = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        const float mn = fmaxf(m_a, mx);  // finite: the first key of every step is in range
-        const float alpha = exp2f(m_a - mn);
-        m_a = mn;
-        const float p0 = exp2f(x0 - mn), p1 = exp2f(x1 - mn), p2 = exp2f(x2 - mn), p3 = exp2f(x3 - mn);
-        l_a = l_a * alpha + ((p0 + p1) + (p2 + p3));
+        // mx is finite: the first key of every step is in range.  Raise the
+        // running maximum only past the margin; until then p <= 2^kStgLazy.
+        if (mx > m_a + kStgLazy) {
+            const float alpha = exp2f(m_a - mx);  // 0 on the first step (m_a = -inf)
+            m_a = mx;
+            l_a *= alpha;
 #pragma unroll
-        for (int t = 0; t < 16; ++t) {
-            o[t][0] *= alpha;
-            o[t][1] *= alpha;
-            o[t][2] *= alpha;
-            o[t][3] *= alpha;
+            for (int t = 0; t < 16; ++t) {
+                o[t][0] *= alpha;
+                o[t][1] *= alpha;
+                o[t][2] *= alpha;
+                o[t][3] *= alpha;
+            }
         }
+        const float p0 = exp2f(x0 - m_a), p1 = exp2f(x1 - m_a), p2 = exp2f(x2 - m_a), p3 = exp2f(x3 - m_a);
+        l_a += (p0 + p1) + (p2 + p3);
         const uint32_t ph0 = pack_bf16x2(p0, p1), ph2 = pack_bf16x2(p2, p3);
         const uint32_t pl0 = pack_bf16x2(p0 - bf16lo(ph0), p1 - bf16hi(ph0));
         const uint32_t pl2 = pack_bf16x2(p2 - bf16lo(ph2), p3 - bf16hi(ph2));
@@ -635,9 +644,11 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) attn_decode_staged_kernel(
     l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
     l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
 
-    // ---- merge the CTA's warps (ascending warp order), then the CTA partials ----
-    __shared__ float s_o[kAttnWarps][8][D];
-    __shared__ float s_ml[kAttnWarps][8][2];
+    // ---- merge the CTA's warps (ascending warp order), then the CTA partials.
+    //      The warps' outputs go to the (now idle) stage rings ----
+    __syncthreads();  // every warp is done with its ring
+    float(*s_o)[8][D] = reinterpret_cast<float(*)[8][D]>(stg_smem);                       // [kStgWarps][8][D]
+    float(*s_ml)[8][2] = reinterpret_cast<float(*)[8][2]>(stg_smem + kStgWarps * 8 * D * 2);  // [kStgWarps][8][2]
     if (gid < a.g) {
 #pragma unroll
         for (int t = 0; t < 16; ++t) {
@@ -653,15 +664,16 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) attn_decode_staged_kernel(
 #ifdef TPL_TRACE
     if (threadIdx.x == 0) ck[0] = (uint64_t)clock64();
 #endif
-    const int dim = threadIdx.x;
+    // thread t: head dimension t % 128 of the heads t / 128, + 2, + 4, ...
+    const int dim = threadIdx.x & (D - 1);
     const int64_t cbase = ((int64_t)pair * cpp + chunk) * a.g;
-    for (int hrow = 0; hrow < a.g; ++hrow) {
+    for (int hrow = threadIdx.x / D; hrow < a.g; hrow += kStgWarps * 32 / D) {
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, s_ml[w][hrow][0]);
+        for (int w = 0; w < kStgWarps; ++w) M = fmaxf(M, s_ml[w][hrow][0]);
         float num = 0.f, den = 0.f;
 #pragma unroll
-        for (int w = 0; w < kAttnWarps; ++w) {
+        for (int w = 0; w < kStgWarps; ++w) {
             const float mi = s_ml[w][hrow][0];
             const float wt = mi == -INFINITY ? 0.f : exp2f(mi - M);
             num += wt * s_o[w][hrow][dim];
@@ -699,10 +711,12 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) attn_decode_staged_kernel(
         return;
     }
     __threadfence();
+    // the pair's combine runs on the first 128 threads (one head dimension each)
+    if (warp >= kAttnWarps) return;
     __shared__ float s_w[kAttnMaxCtasPerPair][8];
     __shared__ float s_M[8], s_den[8], s_new[8];
     __shared__ float s_mlp[kAttnMaxCtasPerPair * 8 * 2];
-    for (int i = threadIdx.x; i < cpp * a.g * 2; i += blockDim.x)
+    for (int i = threadIdx.x; i < cpp * a.g * 2; i += kAttnWarps * 32)
         s_mlp[i] = __ldcg(&a.part_ml[(int64_t)pair * cpp * a.g * 2 + i]);
     attn_pair_combine<8>(a, pair, cpp, b, j, dim, lane, warp, s_mlp, s_w, s_M, s_den, s_new, s_red, true, vnew);
     if (threadIdx.x == 0) {

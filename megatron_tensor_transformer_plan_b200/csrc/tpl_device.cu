@@ -450,7 +450,9 @@ int attn_select(const tpl_plan *p, int B, int64_t keys, AttnGeom *g, int *kind) 
 }
 
 // CTA partials per pair the chosen kernel writes (sizes its scratch).
-int attn_cpp(const AttnGeom &g, int kind) { return kind == ATTN_TMA ? g.cpp_max : g.nsplit / kAttnWarps; }
+int attn_cpp(const AttnGeom &g, int kind) {
+    return kind == ATTN_TMA ? g.cpp_max : g.nsplit / (kind == ATTN_STAGED ? kAttnStgWarps : kAttnWarps);
+}
 
 bool g_am_attr[64];
 
@@ -518,7 +520,7 @@ int attn_launch(const tpl_plan *p, const tpl_kv *kv, const float *q, const float
     a.tickets = tickets;
     a.o = o;
     a.o_f32 = p->f32;
-    const int grid = g.pairs * (g.nsplit / kAttnWarps);
+    const int grid = g.pairs * attn_cpp(g, kind);
     if (kind == ATTN_STAGED) {
         if (!g_stg_attr[dev]) {
             if (cudaFuncSetAttribute(attn_decode_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -526,7 +528,7 @@ int attn_launch(const tpl_plan *p, const tpl_kv *kv, const float *q, const float
                 return TPL_ECUDA;
             g_stg_attr[dev] = true;
         }
-        return cuda_rc(launch_pdl(attn_decode_staged_kernel, grid, kAttnWarps * 32, kStgSmem, st, a));
+        return cuda_rc(launch_pdl(attn_decode_staged_kernel, grid, kAttnStgWarps * 32, kStgSmem, st, a));
     }
     return cuda_rc(p->g <= 8 ? launch_pdl(attn_decode_kernel<true>, grid, kAttnWarps * 32, 0, st, a)
                               : launch_pdl(attn_decode_kernel<false>, grid, kAttnWarps * 32, 0, st, a));

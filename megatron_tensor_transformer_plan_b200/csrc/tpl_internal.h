@@ -18,7 +18,8 @@ constexpr int kGemvThreads = 512;          // 16 warps, one CTA per SM
 constexpr int kGemvWarps = kGemvThreads / 32;
 constexpr size_t kXSmemMax = 140 * 1024;   // activation slice staged per CTA
 constexpr size_t kPartSmemMax = 64 * 1024; // per-round partial sums
-constexpr int kAttnWarps = 4;              // warps per attention CTA
+constexpr int kAttnWarps = 4;              // warps per attention CTA (register-streamed kernel)
+constexpr int kAttnStgWarps = 8;           // warps per CTA of the staged kernel
 constexpr int kAttnTargetWarps = 1024;     // key-range splits across all (b, kv head) pairs
 constexpr int kAttnMinKeys = 128;          // keys per split at least (when there are that many)
 constexpr int kAttnMaxCtasPerPair = 64;
@@ -105,8 +106,9 @@ void attn_geom_tma(int B, int nkv, int64_t keys, int sms, AttnGeom *a);
 // keys: keys covered by the splits (S when the new token is added in the
 // combine, S + 1 when it is read from the cache).
 void attn_geom(int B, int nkv, int64_t keys, AttnGeom *a);
-// Splits of the staged attention kernel: one CTA per SM, floor(sms / pairs)
-// CTAs per pair (at least 64 keys per warp, at most kAttnMaxCtasPerPair).
+// Splits of the staged attention kernel: one CTA of kAttnStgWarps warps per
+// SM, floor(sms / pairs) CTAs per pair (at least 64 keys per warp, at most
+// kAttnMaxCtasPerPair).
 void attn_geom_staged(int B, int nkv, int64_t keys, int sms, AttnGeom *a);
 
 struct WsLayout {

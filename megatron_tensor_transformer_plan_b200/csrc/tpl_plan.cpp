@@ -118,10 +118,10 @@ void attn_geom(int B, int nkv, int64_t keys, AttnGeom *a) {
 void attn_geom_staged(int B, int nkv, int64_t keys, int sms, AttnGeom *a) {
     a->pairs = B * nkv;
     int64_t cpp = std::max(1, sms / std::max(1, a->pairs));
-    const int64_t by_keys = (keys + 4 * 64 - 1) / (4 * 64);
+    const int64_t by_keys = (keys + kAttnStgWarps * 64 - 1) / (kAttnStgWarps * 64);
     cpp = std::min(cpp, std::max<int64_t>(1, by_keys));
     cpp = std::min<int64_t>(cpp, kAttnMaxCtasPerPair);
-    a->nsplit = (int)cpp * kAttnWarps;
+    a->nsplit = (int)cpp * kAttnStgWarps;
     int64_t kps = keys > 0 ? (keys + a->nsplit - 1) / a->nsplit : 16;
     a->kps = (int)((kps + 15) / 16 * 16);
 }

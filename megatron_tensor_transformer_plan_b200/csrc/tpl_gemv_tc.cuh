@@ -89,6 +89,7 @@ struct GemvTcArgs {
     int64_t U;          // tiles * nseg * kbs
     int x_seg_stride;   // X column offset between segments (row ops), elements
     int w3d;
+    int xsplit;         // the activation rows are bf16 hi + lo pairs (the <16, true> kernel serves both forms)
     int epi;
     // outputs
     float *out32;       // GT_ROW
@@ -121,14 +122,23 @@ struct GemvTcArgs {
 };
 
 // Tokens 16*ch .. 16*ch+15 of one accumulator row: the hi column plus the
-// lo column NX/2 further (SPLIT), or the column itself.
+// lo column NX/2 further (SPLIT), or the column itself.  With 16 columns and
+// at most 8 tokens the two forms share one shared-memory layout, so one
+// kernel serves the split and the unsplit projections (xsplit chooses at run
+// time): the four projections of a layer then run the same code, and the
+// end-of-kernel code one of them fetched into the instruction cache is still
+// there for the next (stack layer 317 -> 315 us).
 template <int NX, bool SPLIT>
-__device__ __forceinline__ void gt_load_chunk(uint32_t taddr, int ch, float (&pv)[kGtChunk]) {
-    if constexpr (SPLIT && NX == 16) {  // 8 tokens: hi in columns 0..7, lo in 8..15
-        float d[16];
-        tmem_ld16(taddr, d);
+__device__ __forceinline__ void gt_load_chunk(uint32_t taddr, int ch, float (&pv)[kGtChunk], bool xsplit) {
+    if constexpr (SPLIT && NX == 16) {
+        if (xsplit) {  // 8 tokens: hi in columns 0..7, lo in 8..15
+            float d[16];
+            tmem_ld16(taddr, d);
 #pragma unroll
-        for (int t = 0; t < 16; ++t) pv[t] = t < 8 ? d[t] + d[8 + t] : 0.f;
+            for (int t = 0; t < 16; ++t) pv[t] = t < 8 ? d[t] + d[8 + t] : 0.f;
+        } else {
+            tmem_ld16(taddr, pv);
+        }
     } else if constexpr (SPLIT) {
         float hi[16], lo[16];
         tmem_ld16(taddr + (uint32_t)(16 * ch), hi);
@@ -148,6 +158,14 @@ __device__ __forceinline__ int64_t gt_start(int64_t U, int G, int c) {
     return U * c / G;
 }
 
+// x / d for the unit indices (0 <= x, 0 < d): 32-bit when both fit, which
+// they do at every supported shape; the 64-bit division is a long subroutine
+// that the prologue and the combine would otherwise run cold.
+__device__ __forceinline__ int64_t gt_div(int64_t x, int64_t d) {
+    if ((((uint64_t)x | (uint64_t)d) >> 31) == 0) return (int64_t)((uint32_t)x / (uint32_t)d);
+    return x / d;
+}
+
 // The order in which a CTA walks its range, as three sub-ranges [b, e): the
 // part of its first tile, the part of its last tile (both possibly shared
 // with the neighbouring CTAs), then the whole tiles in between.  Taking the
@@ -164,8 +182,8 @@ __device__ __forceinline__ GtOrder gt_order(int64_t u0, int64_t u1, int64_t per_
     GtOrder o;
     o.u0 = u0;
     o.u1 = u1;
-    o.f_end = min(u1, (u0 / per_tile + 1) * per_tile);
-    o.l_beg = max(o.f_end, ((u1 - 1) / per_tile) * per_tile);
+    o.f_end = min(u1, (gt_div(u0, per_tile) + 1) * per_tile);
+    o.l_beg = max(o.f_end, u1 > 0 ? gt_div(u1 - 1, per_tile) * per_tile : 0);
     return o;
 }
 
@@ -317,7 +335,7 @@ __device__ __forceinline__ void gt_combine(const GemvTcArgs &a, int tile, int G,
                 const int64_t sb = t_beg + (int64_t)g_s * a.kbs, se = sb + a.kbs;
                 const int64_t c0 = gt_start(a.U, G, c), c1 = gt_start(a.U, G, c + 1);
                 valid = c1 > sb && c0 < se;
-                const int sl = (tile == (int)(c0 / per_tile)) ? 0 : 1;
+                const int sl = (tile == (int)gt_div(c0, per_tile)) ? 0 : 1;
                 ent = (((c * 2 + sl) * a.nseg + g_s) << 5) | (g_s << 1) | (c1 >= se ? 1 : 0);
             }
             const unsigned m = __ballot_sync(0xffffffffu, valid);
@@ -345,7 +363,7 @@ __device__ __forceinline__ void gt_combine(const GemvTcArgs &a, int tile, int G,
                         const int64_t sb = t_beg + (int64_t)g_s * a.kbs, se = sb + a.kbs;
                         const int64_t c0 = gt_start(a.U, G, g_cc), c1 = gt_start(a.U, G, g_cc + 1);
                         if (c1 > sb && c0 < se) {
-                            const int sl = (tile == (int)(c0 / per_tile)) ? 0 : 1;
+                            const int sl = (tile == (int)gt_div(c0, per_tile)) ? 0 : 1;
                             const bool seg_last = c1 >= se;
                             s_list[n++] = (((g_cc * 2 + sl) * a.nseg + g_s) << 5) | (g_s << 1) | (seg_last ? 1 : 0);
                         }
@@ -517,6 +535,9 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
     if (threadIdx.x == 0) TPL_TRACE_AT(0);
 
     if (threadIdx.x == 0) {
+        // the descriptors are fetched while the barriers are set up
+        tma_prefetch_map(&a.tm_w);
+        tma_prefetch_map(&a.tm_x);
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
@@ -553,7 +574,7 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
             int sr = 0, tile = 0, seg = 0, kb = 0;
             int64_t uu = u0;
             auto locate = [&]() {
-                tile = (int)(uu / per_tile);
+                tile = (int)gt_div(uu, per_tile);
                 const int w = (int)(uu - (int64_t)tile * per_tile);
                 seg = w / a.kbs;
                 kb = w - seg * a.kbs;
@@ -625,7 +646,7 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
             for (int sr = 0; ok && sr < 3; ++sr)
             for (int64_t u = ord.b(sr); ok && u < ord.e(sr); ++c) {
                 // one piece: the run of k-blocks of one (tile, segment)
-                const int64_t seg_end = (u / a.kbs + 1) * a.kbs;  // segments are kbs-aligned in u
+                const int64_t seg_end = (gt_div(u, a.kbs) + 1) * a.kbs;  // segments are kbs-aligned in u
                 const int64_t pe = min(ord.e(sr), seg_end);
                 const int b = c % BUFS;
                 const unsigned use = (unsigned)(c / BUFS);
@@ -720,14 +741,14 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
         const GtOrder ord = gt_order(u0, u1, per_tile);
         for (int sr = 0; sr < 3; ++sr)
         for (int64_t u = ord.b(sr); u < ord.e(sr);) {
-            const int tile = (int)(u / per_tile);
+            const int tile = (int)gt_div(u, per_tile);
             const int64_t t_beg = (int64_t)tile * per_tile, t_end = t_beg + per_tile;
             const bool local = t_beg >= u0 && t_end <= u1;
-            const int slot = (tile == (int)(u0 / per_tile)) ? 0 : 1;
+            const int slot = (tile == (int)gt_div(u0, per_tile)) ? 0 : 1;
             const int64_t stop = min(ord.e(sr), t_end);  // this CTA's part of the tile: one sub-range holds all of it
             while (u < stop) {
-                const int seg = (int)((u % per_tile) / a.kbs);
-                const int64_t pe = min(stop, (u / a.kbs + 1) * a.kbs);
+                const int seg = (int)(u - t_beg) / a.kbs;
+                const int64_t pe = min(stop, (gt_div(u, a.kbs) + 1) * a.kbs);
                 const int b = c % BUFS;
                 ++c;
                 u = pe;
@@ -744,7 +765,7 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
                 for (int ch = 0; ch < nch; ++ch) {
                     // tokens 16*ch + t: hi part in column 16*ch + t, lo part NX/2 further
                     float pv[kGtChunk];
-                    gt_load_chunk<NX, SPLIT>(acc, ch, pv);
+                    gt_load_chunk<NX, SPLIT>(acc, ch, pv, a.xsplit != 0);
                     if (local) {
                         // every segment of a tile inside this CTA is one piece;
                         // -0 is the additive identity, so segment 0 is stored unchanged

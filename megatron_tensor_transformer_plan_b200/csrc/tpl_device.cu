@@ -62,6 +62,24 @@ cudaError_t launch_pdl(void (*kern)(KA...), dim3 grid, int block, size_t smem, c
 
 bool g_attr_done[64][8];
 
+// Preferred carve-out of a kernel with static shared memory only: the share
+// of the SM's shared memory that its resident CTAs need (as many as fit by
+// registers and threads), rounded up by the driver to a supported size.
+template <typename K>
+cudaError_t set_fit_carveout(K kern, int threads) {
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+    int dev = 0, blocks = 0, smem_sm = 0;
+    if (e == cudaSuccess) e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kern, threads, 0);
+    if (e != cudaSuccess) return e;
+    if (blocks < 1 || smem_sm <= 0) return cudaSuccess;  // keep the default
+    const long need = (long)blocks * ((long)fa.sharedSizeBytes + 1024);  // 1 KB reserved per CTA
+    const int pct = (int)std::min<long>(100, (need * 100 + smem_sm - 1) / smem_sm);
+    return cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, pct);
+}
+
 // The mma.sync projections stream their weights through registers, and a
 // load in flight holds L1 staging space: they ask for the smallest shared-
 // memory carve-out that fits them (the rest of the 256 KB is L1).  Without
@@ -203,14 +221,26 @@ int gt_go(int slot, GemvTcArgs &a, cudaStream_t st) {
         launch_pdl(gemv_tc_kernel<NX, SPLIT>, (int)G, kGtThreads, (size_t)GemvTcSmem<NX, SPLIT>::BYTES, st, a));
 }
 
+// A layer of at least 1 GiB of bf16 weights (the 70B shape; the 7B layer is
+// 0.4 GiB): the decode kernels' choices below differ by layer size.
+bool large_layer(const tpl_plan *p) {
+    const tpl_dims &d = p->d;
+    const int64_t layer_params = (int64_t)(d.n_q_heads + 2 * d.n_kv_heads) * d.head_dim * d.hidden +
+                                 (int64_t)d.hidden * d.n_q_heads * d.head_dim + 3 * (int64_t)d.ffn * d.hidden;
+    return layer_params * 2 >= (1ll << 30);
+}
+
 // Fill the geometry, the weight map (2-D column-parallel rows or 3-D per-shard
 // blocks) and the activation map, then launch.
 int gemv_tc_run(Ctx &c, GemvTcArgs &a, int op, bool split, const void *W, int64_t ld, int64_t N, int nseg,
                 int64_t blk, const void *X, int64_t Kx, int64_t x_rows, int x_seg_stride) {
-    tpl_plan *p = c.p;
-    (void)p;
     if (c.B > kGtMaxB) return TPL_EUNSUPPORTED;
-    const int nx = gt_nx(c.B, split);
+    // On small layers 9 to 16 tokens unsplit take the split form's 32 columns
+    // (the upper 16 read as zero rows), so that all four projections run one
+    // kernel binary (7B layer, 16 tokens: 224 -> 220 us); on large layers the
+    // extra operand bytes per stage cost more than the shared code saves
+    const bool widen = !split && c.B > 8 && c.B <= 16 && !large_layer(c.p);
+    const int nx = widen ? 32 : gt_nx(c.B, split);
     a.B = c.B;
     a.N = (int)N;
     a.tiles = (int)((N + kGtRows - 1) / kGtRows);
@@ -231,7 +261,7 @@ int gemv_tc_run(Ctx &c, GemvTcArgs &a, int op, bool split, const void *W, int64_
     // up to 8 tokens the split and unsplit forms share one kernel (see
     // gt_load_chunk); from 9 tokens the split form needs more columns anyway
     if (nx == 16 && (split || c.B <= 8)) return gt_go<16, true>(0, a, c.st);
-    if (split) {
+    if (split || widen) {
         switch (nx) {
             case 32: return gt_go<32, true>(1, a, c.st);
             case 64: return gt_go<64, true>(2, a, c.st);
@@ -258,10 +288,7 @@ bool use_tc(const tpl_plan *p, int op, int B) {
     if (B > kMaxBatchCuda) return true;  // beyond the mma.sync kernel's 16 tokens
     if (p->gemv_mode == 3) return true;
     if (p->gemv_mode != 4) return false;
-    const tpl_dims &d = p->d;
-    const int64_t layer_params = (int64_t)(d.n_q_heads + 2 * d.n_kv_heads) * d.head_dim * d.hidden +
-                                 (int64_t)d.hidden * d.n_q_heads * d.head_dim + 3 * (int64_t)d.ffn * d.hidden;
-    return B >= kMaxBatchCuda || (B >= 4 && layer_params * 2 >= (1ll << 30));
+    return B >= kMaxBatchCuda || (B >= 4 && large_layer(p));
 }
 
 GemvTcArgs gt_args(const tpl_plan *p) {
@@ -546,12 +573,12 @@ int attn_launch(const tpl_plan *p, const tpl_kv *kv, const float *q, const float
         return cuda_rc(launch_pdl(attn_decode_staged_kernel, grid, kAttnStgWarps * 32, kStgSmem, st, a));
     }
     if (!g_reg_attr[dev]) {
-        // register-streamed K/V: as for the mma.sync projections, the smallest
-        // carve-out that fits, so that the loads in flight have L1 to land in
-        if (cudaFuncSetAttribute(attn_decode_kernel<true>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 (int)cudaSharedmemCarveoutMaxL1) != cudaSuccess ||
-            cudaFuncSetAttribute(attn_decode_kernel<false>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 (int)cudaSharedmemCarveoutMaxL1) != cudaSuccess)
+        // register-streamed K/V: as for the mma.sync projections, a carve-out
+        // just large enough for the CTAs that fit an SM by registers, so that
+        // the loads in flight have L1 to land in (the smallest carve-out
+        // would cut the resident CTAs instead)
+        if (set_fit_carveout(attn_decode_kernel<true>, kAttnWarps * 32) != cudaSuccess ||
+            set_fit_carveout(attn_decode_kernel<false>, kAttnWarps * 32) != cudaSuccess)
             return TPL_ECUDA;
         g_reg_attr[dev] = true;
     }

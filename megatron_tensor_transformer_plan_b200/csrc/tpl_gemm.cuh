@@ -120,12 +120,6 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *tm, in
         : "memory");
 }
 
-// Fetch a tensor map (a kernel parameter) into the TMA unit's descriptor
-// cache ahead of its first copy.
-__device__ __forceinline__ void tma_prefetch_map(const CUtensorMap *tm) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tm)) : "memory");
-}
-
 __device__ __forceinline__ void tma_load_2d_hint(void *dst, const CUtensorMap *tm, int x, int y, uint64_t *bar,
                                                  uint64_t policy) {
     asm volatile(

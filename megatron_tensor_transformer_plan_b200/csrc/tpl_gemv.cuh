@@ -133,15 +133,6 @@ __device__ __forceinline__ void gemv_final_pair(const GemvArgs &a, int pair, int
     store_act(a.out_act, a.act_f32, (int64_t)tok * (a.g.N / 2) + pair, silu(gsum) * usum);
 }
 
-// a * b / c for non-negative ints, in 32-bit arithmetic when the product fits
-// (always, at the supported shapes): the 64-bit division is a long
-// subroutine on the path from a CTA's entry to its first weight load.
-__device__ __forceinline__ int muldiv(int a, int b, int c) {
-    const uint64_t p = (uint64_t)(uint32_t)a * (uint32_t)b;
-    if ((p >> 32) == 0) return (int)((uint32_t)p / (uint32_t)c);
-    return (int)(p / (uint32_t)c);
-}
-
 template <int MODE, bool BIG>  // BIG: more than 8 tokens (tokens 8..15 in A rows 8-15)
 __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_constant__ GemvArgs a) {
     using T = GemvTraits<MODE>;
@@ -156,7 +147,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
     const int gid = lane >> 2, c = lane & 3;
     const int B = a.B;
     const int rb = blockIdx.x / g.ksplit, ks = blockIdx.x % g.ksplit;
-    const int rg0 = muldiv(rb, g.ng, g.rb), rg1 = muldiv(rb + 1, g.ng, g.rb);
+    const int rg0 = (int)((int64_t)rb * g.ng / g.rb), rg1 = (int)((int64_t)(rb + 1) * g.ng / g.rb);
     const int kgl = warp % g.wk, wslot = warp / g.wk;
     TPL_TRACE_VARS
     if (tid == 0) TPL_TRACE_AT(0);
@@ -166,14 +157,14 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
     const int kpseg = KG / g.nseg;
     const int Gk = ks * g.wk + kgl;
     const int seg = Gk / kpseg, piece = Gk % kpseg;
-    const int kb_lo = muldiv(piece, g.nb, kpseg), kb_hi = muldiv(piece + 1, g.nb, kpseg);
+    const int kb_lo = (int)((int64_t)piece * g.nb / kpseg), kb_hi = (int)((int64_t)(piece + 1) * g.nb / kpseg);
     // CTA's staged span.
     const int seg_lo = (ks * g.wk) / kpseg;
     int cblk_lo = 0, nbc = g.nb;
     if (g.ksplit > g.nseg) {
         const int per = g.pieces, pi = ks % per;
-        cblk_lo = muldiv(pi, g.nb, per);
-        nbc = muldiv(pi + 1, g.nb, per) - cblk_lo;
+        cblk_lo = (int)((int64_t)pi * g.nb / per);
+        nbc = (int)((int64_t)(pi + 1) * g.nb / per) - cblk_lo;
     }
     const int kpc = g.wk / g.segs_per_cta;  // K-groups per segment inside the CTA
 

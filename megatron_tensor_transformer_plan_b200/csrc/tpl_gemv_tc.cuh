@@ -140,11 +140,15 @@ __device__ __forceinline__ void gt_load_chunk(uint32_t taddr, int ch, float (&pv
             tmem_ld16(taddr, pv);
         }
     } else if constexpr (SPLIT) {
-        float hi[16], lo[16];
-        tmem_ld16(taddr + (uint32_t)(16 * ch), hi);
-        tmem_ld16(taddr + (uint32_t)(NX / 2 + 16 * ch), lo);
+        if (xsplit) {
+            float hi[16], lo[16];
+            tmem_ld16(taddr + (uint32_t)(16 * ch), hi);
+            tmem_ld16(taddr + (uint32_t)(NX / 2 + 16 * ch), lo);
 #pragma unroll
-        for (int t = 0; t < 16; ++t) pv[t] = hi[t] + lo[t];
+            for (int t = 0; t < 16; ++t) pv[t] = hi[t] + lo[t];
+        } else {  // unsplit tokens in the first NX/2 columns, the rest zero
+            tmem_ld16(taddr + (uint32_t)(16 * ch), pv);
+        }
     } else {
         tmem_ld16(taddr + (uint32_t)(16 * ch), pv);
     }
@@ -156,14 +160,6 @@ __device__ __forceinline__ int64_t gt_start(int64_t U, int G, int c) {
     // than a 64-bit division, and the combine evaluates this many times
     if (U < (1ll << 23)) return (int64_t)(((uint32_t)U * (uint32_t)c) / (uint32_t)G);
     return U * c / G;
-}
-
-// x / d for the unit indices (0 <= x, 0 < d): 32-bit when both fit, which
-// they do at every supported shape; the 64-bit division is a long subroutine
-// that the prologue and the combine would otherwise run cold.
-__device__ __forceinline__ int64_t gt_div(int64_t x, int64_t d) {
-    if ((((uint64_t)x | (uint64_t)d) >> 31) == 0) return (int64_t)((uint32_t)x / (uint32_t)d);
-    return x / d;
 }
 
 // The order in which a CTA walks its range, as three sub-ranges [b, e): the
@@ -182,8 +178,8 @@ __device__ __forceinline__ GtOrder gt_order(int64_t u0, int64_t u1, int64_t per_
     GtOrder o;
     o.u0 = u0;
     o.u1 = u1;
-    o.f_end = min(u1, (gt_div(u0, per_tile) + 1) * per_tile);
-    o.l_beg = max(o.f_end, u1 > 0 ? gt_div(u1 - 1, per_tile) * per_tile : 0);
+    o.f_end = min(u1, (u0 / per_tile + 1) * per_tile);
+    o.l_beg = max(o.f_end, ((u1 - 1) / per_tile) * per_tile);
     return o;
 }
 
@@ -335,7 +331,7 @@ __device__ __forceinline__ void gt_combine(const GemvTcArgs &a, int tile, int G,
                 const int64_t sb = t_beg + (int64_t)g_s * a.kbs, se = sb + a.kbs;
                 const int64_t c0 = gt_start(a.U, G, c), c1 = gt_start(a.U, G, c + 1);
                 valid = c1 > sb && c0 < se;
-                const int sl = (tile == (int)gt_div(c0, per_tile)) ? 0 : 1;
+                const int sl = (tile == (int)(c0 / per_tile)) ? 0 : 1;
                 ent = (((c * 2 + sl) * a.nseg + g_s) << 5) | (g_s << 1) | (c1 >= se ? 1 : 0);
             }
             const unsigned m = __ballot_sync(0xffffffffu, valid);
@@ -363,7 +359,7 @@ __device__ __forceinline__ void gt_combine(const GemvTcArgs &a, int tile, int G,
                         const int64_t sb = t_beg + (int64_t)g_s * a.kbs, se = sb + a.kbs;
                         const int64_t c0 = gt_start(a.U, G, g_cc), c1 = gt_start(a.U, G, g_cc + 1);
                         if (c1 > sb && c0 < se) {
-                            const int sl = (tile == (int)gt_div(c0, per_tile)) ? 0 : 1;
+                            const int sl = (tile == (int)(c0 / per_tile)) ? 0 : 1;
                             const bool seg_last = c1 >= se;
                             s_list[n++] = (((g_cc * 2 + sl) * a.nseg + g_s) << 5) | (g_s << 1) | (seg_last ? 1 : 0);
                         }
@@ -535,9 +531,6 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
     if (threadIdx.x == 0) TPL_TRACE_AT(0);
 
     if (threadIdx.x == 0) {
-        // the descriptors are fetched while the barriers are set up
-        tma_prefetch_map(&a.tm_w);
-        tma_prefetch_map(&a.tm_x);
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
@@ -574,7 +567,7 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
             int sr = 0, tile = 0, seg = 0, kb = 0;
             int64_t uu = u0;
             auto locate = [&]() {
-                tile = (int)gt_div(uu, per_tile);
+                tile = (int)(uu / per_tile);
                 const int w = (int)(uu - (int64_t)tile * per_tile);
                 seg = w / a.kbs;
                 kb = w - seg * a.kbs;
@@ -646,7 +639,7 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
             for (int sr = 0; ok && sr < 3; ++sr)
             for (int64_t u = ord.b(sr); ok && u < ord.e(sr); ++c) {
                 // one piece: the run of k-blocks of one (tile, segment)
-                const int64_t seg_end = (gt_div(u, a.kbs) + 1) * a.kbs;  // segments are kbs-aligned in u
+                const int64_t seg_end = (u / a.kbs + 1) * a.kbs;  // segments are kbs-aligned in u
                 const int64_t pe = min(ord.e(sr), seg_end);
                 const int b = c % BUFS;
                 const unsigned use = (unsigned)(c / BUFS);
@@ -741,14 +734,14 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
         const GtOrder ord = gt_order(u0, u1, per_tile);
         for (int sr = 0; sr < 3; ++sr)
         for (int64_t u = ord.b(sr); u < ord.e(sr);) {
-            const int tile = (int)gt_div(u, per_tile);
+            const int tile = (int)(u / per_tile);
             const int64_t t_beg = (int64_t)tile * per_tile, t_end = t_beg + per_tile;
             const bool local = t_beg >= u0 && t_end <= u1;
-            const int slot = (tile == (int)gt_div(u0, per_tile)) ? 0 : 1;
+            const int slot = (tile == (int)(u0 / per_tile)) ? 0 : 1;
             const int64_t stop = min(ord.e(sr), t_end);  // this CTA's part of the tile: one sub-range holds all of it
             while (u < stop) {
-                const int seg = (int)(u - t_beg) / a.kbs;
-                const int64_t pe = min(stop, (gt_div(u, a.kbs) + 1) * a.kbs);
+                const int seg = (int)((u % per_tile) / a.kbs);
+                const int64_t pe = min(stop, (u / a.kbs + 1) * a.kbs);
                 const int b = c % BUFS;
                 ++c;
                 u = pe;

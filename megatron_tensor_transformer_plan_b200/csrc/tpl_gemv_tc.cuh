@@ -197,34 +197,53 @@ struct GtRowIn {
     float rv[kGtChunk];
     float gam;
 };
+// Per-token code of the end-of-kernel writes runs for the chunk's first 4
+// tokens, and for the other 12 only behind one branch taken when the chunk
+// holds more: at 4 tokens or fewer the 12 copies are never fetched, which
+// matters for code that runs cold (about 1.5 us of the row-parallel combine).
+template <typename F>
+__device__ __forceinline__ void gt_for_tokens(int ntok, F &&f) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) f(j);
+    if (ntok > 4) {
+#pragma unroll
+        for (int j = 4; j < kGtChunk; ++j) f(j);
+    }
+}
+
 __device__ __forceinline__ void gt_row_loads(const GemvTcArgs &a, int row, int tok0, GtRowIn &in) {
     const int B = a.B;
-    const bool ok = row < a.N;
-#pragma unroll
-    for (int j = 0; j < kGtChunk; ++j)
-        in.rv[j] = (ok && a.resid && tok0 + j < B) ? load_act(a.resid, a.resid_f32, (int64_t)(tok0 + j) * a.N + row)
-                                                    : 0.f;
-    in.gam = (ok && a.xs_gamma) ? a.xs_gamma[row] : 1.f;
+    const bool ok = row < a.N && a.resid;
+    const int64_t base = (int64_t)tok0 * a.N + row;
+    if (a.resid_f32) {
+        const float *r = static_cast<const float *>(a.resid) + base;
+        gt_for_tokens(B - tok0, [&](int j) { in.rv[j] = (ok && tok0 + j < B) ? r[(int64_t)j * a.N] : 0.f; });
+    } else {
+        const __nv_bfloat16 *r = static_cast<const __nv_bfloat16 *>(a.resid) + base;
+        gt_for_tokens(B - tok0, [&](int j) {
+            in.rv[j] = (ok && tok0 + j < B) ? __bfloat162float(r[(int64_t)j * a.N]) : 0.f;
+        });
+    }
+    in.gam = (row < a.N && a.xs_gamma) ? a.xs_gamma[row] : 1.f;
 }
 
 __device__ __forceinline__ void gt_final(const GemvTcArgs &a, int row, const float (&v0)[kGtChunk], int lane, int tok0,
                                       const float *inv_rms, const GtRowIn *pre = nullptr) {
     const int B = a.B;
     const bool scale = a.rms_src && a.epi != GT_ROW;  // the RMSNorm factor of column ops
+    const int ntok = B - tok0;
     float v[kGtChunk];
-#pragma unroll
-    for (int i = 0; i < kGtChunk; ++i) v[i] = scale ? v0[i] * inv_rms[min(tok0 + i, kGtMaxB - 1)] : v0[i];
+    gt_for_tokens(ntok, [&](int i) { v[i] = scale ? v0[i] * inv_rms[min(tok0 + i, kGtMaxB - 1)] : v0[i]; });
     if (a.epi == GT_GU) {
         // rows interleave gate and up: the even lane pairs with its odd neighbour
         const bool w = !(lane & 1) && row + 1 < a.N;
         __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(a.out_act) + row / 2;
         const int64_t st = a.N / 2;
-#pragma unroll
-        for (int i = 0; i < kGtChunk; ++i) {
+        gt_for_tokens(ntok, [&](int i) {
             const int b = tok0 + i;
             const float u = __shfl_down_sync(0xffffffffu, v[i], 1);
             if (w && b < B) dst[b * st] = __float2bfloat16_rn(silu(v[i]) * u);
-        }
+        });
         return;
     }
     if (row >= a.N) return;
@@ -243,17 +262,16 @@ __device__ __forceinline__ void gt_final(const GemvTcArgs &a, int row, const flo
         if (dn) dn += (int64_t)s * kd + ll;
         const int64_t sq = (int64_t)a.nq * a.hd, sc = (int64_t)a.nkv_s * a.seq_cap * a.hd,
                       sn = (int64_t)a.nkv_s * (a.nq / a.nq_s) * a.hd;
-#pragma unroll
-        for (int i = 0; i < kGtChunk; ++i) {
+        gt_for_tokens(ntok, [&](int i) {
             const int b = tok0 + i;
-            if (b >= B) continue;
+            if (b >= B) return;
             if (isq) {
                 dq[b * sq] = v[i];
             } else {
                 dc[b * sc] = __float2bfloat16_rn(v[i]);
                 if (dn) dn[b * sn] = v[i];
             }
-        }
+        });
         return;
     }
     // GT_ROW: out = resid + sum.  Every load before any store (the pointers
@@ -265,10 +283,9 @@ __device__ __forceinline__ void gt_final(const GemvTcArgs &a, int row, const flo
     const float *rv = in.rv;
     const float gam = in.gam;
     __nv_bfloat16 *oact = static_cast<__nv_bfloat16 *>(a.out_act);
-#pragma unroll
-    for (int j = 0; j < kGtChunk; ++j) {
+    gt_for_tokens(ntok, [&](int j) {
         const int b = tok0 + j;
-        if (b >= B) continue;
+        if (b >= B) return;
         const int64_t i = (int64_t)b * a.N + row;
         const float o = a.resid ? rv[j] + v[j] : v[j];
         if (a.out32) a.out32[i] = o;
@@ -281,7 +298,7 @@ __device__ __forceinline__ void gt_final(const GemvTcArgs &a, int row, const flo
             a.xs_out[i] = hi;
             a.xs_out[(int64_t)(a.xs_half + b) * a.N + row] = __float2bfloat16_rn(__fsub_rn(sc, __bfloat162float(hi)));
         }
-    }
+    });
 }
 
 // The CTA that completed a tile split across CTAs adds its pieces in the

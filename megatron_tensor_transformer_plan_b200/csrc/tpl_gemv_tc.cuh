@@ -54,7 +54,7 @@ constexpr int kGtBufsMax = 8;    // TMEM accumulators in flight, at most
 constexpr int kGtMaxB = 64;       // tokens per call
 constexpr int kGtChunk = 16;      // tokens per epilogue chunk
 constexpr int kGtList = 120;      // piece list entries per combine chunk
-constexpr int kGtBarBytes = 1024;  // mbarriers, flags and the piece list after the stage ring
+constexpr int kGtBarBytes = 2048;  // mbarriers, flags and the piece lists after the stage ring
 constexpr int kGtRmsBytes = 2048;  // per-warp sums of squares and 1/rms per token
 
 // Shared memory: the stage ring, the running tile sums of tiles finished
@@ -311,16 +311,70 @@ __device__ __forceinline__ void gt_final(const GemvTcArgs &a, int row, const flo
 // repeated for each 16-token chunk, reusing the list when one round held it
 // all.  Each CTA stored its part in slot 0 if the tile is its first, else in
 // slot 1.  Run by the 128 epilogue threads (named barrier 1).
+// The CTAs cf..cl whose unit ranges cover a tile.
+__device__ __forceinline__ void gt_tile_ctas(const GemvTcArgs &a, int tile, int G, int &cf, int &cl) {
+    const int64_t per_tile = (int64_t)a.nseg * a.kbs;
+    const int64_t t_beg = (int64_t)tile * per_tile;
+    cf = (int)((t_beg * G) / a.U);
+    while (cf > 0 && gt_start(a.U, G, cf) > t_beg) --cf;
+    while (gt_start(a.U, G, cf + 1) <= t_beg) ++cf;
+    cl = cf;
+    while (cl + 1 < G && gt_start(a.U, G, cl + 1) < t_beg + per_tile) ++cl;
+}
+
+// A split tile's piece list in the fixed order (segment, then CTA) built by
+// the 128 epilogue threads at once: with at most 128 (segment, CTA)
+// candidates each thread tests one and the valid ones are compacted by ballot
+// into list[0, *nlist).  Returns whether the whole list was built (false:
+// too many candidates, or a full list that may have dropped entries).  All
+// 128 threads call it (named barrier 1); cnt is scratch for 4 counts.
+__device__ __forceinline__ bool gt_build_list(const GemvTcArgs &a, int tile, int G, int lane, int ep_tid,
+                                           volatile int *list, volatile int *nlist, volatile int *cnt) {
+    const int64_t per_tile = (int64_t)a.nseg * a.kbs;
+    const int64_t t_beg = (int64_t)tile * per_tile;
+    int cf, cl;
+    gt_tile_ctas(a, tile, G, cf, cl);
+    const int ncta = cl - cf + 1, ncand = a.nseg * ncta;
+    if (ncand > 128) return false;
+    const int g_s = ep_tid / ncta, c = cf + ep_tid % ncta;
+    bool valid = false;
+    int ent = 0;
+    if (ep_tid < ncand) {
+        const int64_t sb = t_beg + (int64_t)g_s * a.kbs, se = sb + a.kbs;
+        const int64_t c0 = gt_start(a.U, G, c), c1 = gt_start(a.U, G, c + 1);
+        valid = c1 > sb && c0 < se;
+        const int sl = (tile == (int)(c0 / per_tile)) ? 0 : 1;
+        ent = (((c * 2 + sl) * a.nseg + g_s) << 5) | (g_s << 1) | (c1 >= se ? 1 : 0);
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, valid);
+    const int w = ep_tid >> 5;
+    if (lane == 0) cnt[w] = __popc(m);
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    int base = 0;
+    for (int x = 0; x < w; ++x) base += cnt[x];
+    const int pos = base + __popc(m & ((1u << lane) - 1u));
+    if (valid && pos < kGtList) list[pos] = ent;
+    const int tot = cnt[0] + cnt[1] + cnt[2] + cnt[3];
+    if (ep_tid == 0) *nlist = tot < kGtList ? tot : kGtList;
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    return tot < kGtList;
+}
+
+// `pre`/`pre_n`: the tile's piece list built while the weights streamed
+// (pre_n < 0: none), which spares the combine, run cold at the end of the
+// kernel, the candidate search.
 __device__ __forceinline__ void gt_combine(const GemvTcArgs &a, int tile, int G, int nch, int r, int lane, int ep_tid,
                                         const float *s_inv, volatile int *s_list, volatile int *s_nlist,
-                                        volatile int *s_more, volatile int *s_cnt) {
+                                        volatile int *s_more, volatile int *s_cnt, const volatile int *pre,
+                                        int pre_n) {
     const int64_t per_tile = (int64_t)a.nseg * a.kbs;
     const int64_t t_beg = (int64_t)tile * per_tile;
     const int row = tile * kGtRows + r;
     const int B = a.B;
     float seg_sum[kGtChunk], tile_sum[kGtChunk];
-    GtRowIn row_in;       // the row-parallel final write's loads, issued with the pieces'
-    bool single = false;  // the whole list is in shared memory
+    GtRowIn row_in;                  // the row-parallel final write's loads, issued with the pieces'
+    bool single = pre_n >= 0;        // the whole list is in shared memory
+    const volatile int *lst = single ? pre : s_list;
 #ifdef TPL_TRACE
     // SM-clock marks of the first chunk (traced builds): start, list built,
     // pieces loaded and added, written
@@ -334,40 +388,13 @@ __device__ __forceinline__ void gt_combine(const GemvTcArgs &a, int tile, int G,
             tile_sum[t] = -0.f;
             seg_sum[t] = -0.f;
         }
-        int cf = (int)((t_beg * G) / a.U);
-        while (cf > 0 && gt_start(a.U, G, cf) > t_beg) --cf;
-        while (gt_start(a.U, G, cf + 1) <= t_beg) ++cf;
-        int cl = cf;
-        while (cl + 1 < G && gt_start(a.U, G, cl + 1) < t_beg + per_tile) ++cl;
-        const int ncta = cl - cf + 1, ncand = a.nseg * ncta;
-        if (!single && ncand <= 128) {
-            const int g_s = ep_tid / ncta, c = cf + ep_tid % ncta;
-            bool valid = false;
-            int ent = 0;
-            if (ep_tid < ncand) {
-                const int64_t sb = t_beg + (int64_t)g_s * a.kbs, se = sb + a.kbs;
-                const int64_t c0 = gt_start(a.U, G, c), c1 = gt_start(a.U, G, c + 1);
-                valid = c1 > sb && c0 < se;
-                const int sl = (tile == (int)(c0 / per_tile)) ? 0 : 1;
-                ent = (((c * 2 + sl) * a.nseg + g_s) << 5) | (g_s << 1) | (c1 >= se ? 1 : 0);
-            }
-            const unsigned m = __ballot_sync(0xffffffffu, valid);
-            const int w = ep_tid >> 5;
-            if (lane == 0) s_cnt[w] = __popc(m);
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            int base = 0;
-            for (int x = 0; x < w; ++x) base += s_cnt[x];
-            const int pos = base + __popc(m & ((1u << lane) - 1u));
-            if (valid && pos < kGtList) s_list[pos] = ent;
-            if (ep_tid == 0) {
-                const int tot = s_cnt[0] + s_cnt[1] + s_cnt[2] + s_cnt[3];
-                *s_nlist = tot < kGtList ? tot : kGtList;
-                *s_more = 0;
-            }
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            single = *s_nlist < kGtList;  // a full list may have dropped entries: generate it instead
+        int g_s = 0, g_cc = 0;  // generator position (thread 0)
+        if (!single) {
+            single = gt_build_list(a, tile, G, lane, ep_tid, s_list, s_nlist, s_cnt);
+            if (ep_tid == 0) *s_more = 0;
+            int cl;
+            gt_tile_ctas(a, tile, G, g_cc, cl);
         }
-        int g_s = 0, g_cc = cf;  // generator position (thread 0)
         for (int round = 0;; ++round) {
             if (!single) {
                 if (ep_tid == 0) {
@@ -391,7 +418,7 @@ __device__ __forceinline__ void gt_combine(const GemvTcArgs &a, int tile, int G,
                 }
                 asm volatile("bar.sync 1, 128;" ::: "memory");
             }
-            const int n = *s_nlist;
+            const int n = lst == pre ? pre_n : *s_nlist;
 #ifdef TPL_TRACE
             if (ch == 0 && round == 0) ck[1] = (uint64_t)clock64();
 #endif
@@ -408,7 +435,7 @@ __device__ __forceinline__ void gt_combine(const GemvTcArgs &a, int tile, int G,
                     int en[16];
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
-                        en[j] = e0 + j < n ? s_list[e0 + j] : 0;
+                        en[j] = e0 + j < n ? lst[e0 + j] : 0;
                         v1[j] = e0 + j < n ? __ldcg(piece_src(en[j])) : make_float4(0.f, 0.f, 0.f, 0.f);
                     }
 #pragma unroll
@@ -452,7 +479,7 @@ __device__ __forceinline__ void gt_combine(const GemvTcArgs &a, int tile, int G,
                     int en[8];
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        en[j] = e0 + j < n ? s_list[e0 + j] : 0;
+                        en[j] = e0 + j < n ? lst[e0 + j] : 0;
                         const float4 *src = piece_src(en[j]);
 #pragma unroll
                         for (int q4 = 0; q4 < kGtChunk / 4; ++q4)
@@ -516,7 +543,8 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
     constexpr int STAGE = SMEM::STAGE;
     constexpr int NS = SMEM::NS;
     constexpr int BUFS = SMEM::BUFS;
-    static_assert(2 * NS * 8 + 2 * BUFS * 8 + 8 + 4 + 32 + 4 * (kGtList + 4) <= kGtBarBytes, "barrier area");
+    static_assert(2 * NS * 8 + 2 * BUFS * 8 + 8 + 4 + 32 + 4 * (kGtList + 4) + 4 * (2 * kGtList + 2) <= kGtBarBytes,
+                  "barrier area");
     constexpr int TMEM_COLS = BUFS * NX <= 32 ? 32 : BUFS * NX <= 64 ? 64 : BUFS * NX <= 128 ? 128
                               : BUFS * NX <= 256 ? 256 : 512;
     static_assert(BUFS * NX <= 512, "accumulators");
@@ -539,6 +567,8 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
     volatile int *s_nlist = const_cast<int *>(s_fail) + 4;
     volatile int *s_more = const_cast<int *>(s_fail) + 5;
     volatile int *s_list = const_cast<int *>(s_fail) + 8;  // [kGtList]
+    volatile int *s_pre = s_list + kGtList + 4;              // [2][kGtList]: lists of the first and last tile
+    volatile int *s_pre_n = s_pre + 2 * kGtList;             // [2]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = gridDim.x, cta = blockIdx.x;
@@ -745,6 +775,20 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
             }
             asm volatile("bar.sync 1, 128;" ::: "memory");
         }
+        // the piece lists of this CTA's first and last tiles where other CTAs
+        // share them, built now while the weights stream: the CTA that
+        // completes such a tile combines it at the end of the kernel, cold
+        int pre_tile[2] = {-1, -1};
+        if (u1 > u0) {
+#pragma unroll 1
+            for (int k = 0; k < 2; ++k) {
+                const int tl = (int)((k ? u1 - 1 : u0) / per_tile);
+                const int64_t tb = (int64_t)tl * per_tile;
+                if ((k == 1 && tl == pre_tile[0]) || (tb >= u0 && tb + per_tile <= u1)) continue;
+                if (gt_build_list(a, tl, G, lane, ep_tid, s_pre + k * kGtList, s_pre_n + k, s_list + kGtList))
+                    pre_tile[k] = tl;
+            }
+        }
         float tile_sum[kGtChunk];
         int c = 0;
         bool dead = false;
@@ -847,7 +891,9 @@ __global__ void __launch_bounds__(kGtThreads, 1) gemv_tc_kernel(const __grid_con
             asm volatile("bar.sync 1, 128;" ::: "memory");
             if (!*s_last) continue;
             __threadfence();
-            gt_combine(a, tile, G, nch, r, lane, ep_tid, s_inv, s_list, s_nlist, s_more, s_list + kGtList);
+            const int pk = tile == pre_tile[0] ? 0 : tile == pre_tile[1] ? 1 : -1;
+            gt_combine(a, tile, G, nch, r, lane, ep_tid, s_inv, s_list, s_nlist, s_more, s_list + kGtList,
+                       pk >= 0 ? s_pre + pk * kGtList : nullptr, pk >= 0 ? s_pre_n[pk] : -1);
             if (ep_tid == 0) TPL_TRACE_AT(3);
         }
         if (ep_tid == 0 && ep_traced)

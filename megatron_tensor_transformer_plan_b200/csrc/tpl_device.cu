@@ -277,18 +277,18 @@ int gemv_tc_run(Ctx &c, GemvTcArgs &a, int op, bool split, const void *W, int64_
 
 // TPL_OPT_GEMV_MODE 4 (the default for bf16 plans): one kernel family for all
 // four projections of a layer, the one that measured faster on B200 (layers
-// that mix the two families measured slower than either): tcgen05 from 4
-// tokens on layers of at least 1 GiB of weights and from 16 tokens on any
-// layer, mma.sync otherwise (one token, and small layers, where the tcgen05
-// kernel's fixed costs dominate).  Beyond 16 tokens (any mode) only the
-// tcgen05 kernel applies.
+// that mix the two families measured slower than either): tcgen05 on layers
+// of at least 1 GiB of weights at any token count (70B layer, one token: 305
+// against 345 us) and from 3 tokens on any layer, mma.sync for one or two
+// tokens on small layers (7B layer, one token: 113 against 117 us at t = 1).
+// Beyond 16 tokens (any mode) only the tcgen05 kernel applies.
 bool use_tc(const tpl_plan *p, int op, int B) {
     (void)op;
     if (p->f32) return false;
     if (B > kMaxBatchCuda) return true;  // beyond the mma.sync kernel's 16 tokens
     if (p->gemv_mode == 3) return true;
     if (p->gemv_mode != 4) return false;
-    return B >= kMaxBatchCuda || (B >= 4 && large_layer(p));
+    return large_layer(p) || B >= 3;
 }
 
 GemvTcArgs gt_args(const tpl_plan *p) {

@@ -85,6 +85,7 @@ def test_tc_matches_default_kernels(gpu):
     """Both kernel families on the same layer: close (different summation
     order only)."""
     L = make_layer(1024, 16, 8, 128, 2816, 4, 5, 300)
+    L.plan.set_option(tpl.TPL_OPT_GEMV_MODE, 0)  # the mma.sync family
     a = run_steps(L)
     L.plan.set_option(tpl.TPL_OPT_GEMV_MODE, TC)
     b = run_steps(L)

@@ -132,9 +132,9 @@ def test_decode_kernel_count(tpl):
     (the fused O and down write the others), 9 per layer in separate mode;
     one more per layer with the rotation."""
     p = tpl.Plan(tpl.make_dims(8192, 64, 8, 128, 28672, 80), 8)
-    assert [p.decode_kernel_count(b) for b in (1, 4, 16, 64)] == [5, 6, 6, 6]
+    assert [p.decode_kernel_count(b) for b in (1, 4, 16, 64)] == [6, 6, 6, 6]  # large layer: tcgen05 throughout
     assert p.decode_kernel_count(4, n_layers=80) == 401
-    assert p.decode_kernel_count(1, n_layers=80) == 400
+    assert p.decode_kernel_count(1, n_layers=80) == 401
     assert p.decode_kernel_count(4, tpl.TPL_REDUCE_SEPARATE) == 9
     assert p.decode_kernel_count(4, tpl.TPL_REDUCE_SEPARATE, n_layers=80) == 720
     p.set_option(tpl.TPL_OPT_GEMV_MODE, 0)
@@ -142,7 +142,7 @@ def test_decode_kernel_count(tpl):
     assert p.decode_kernel_count(4, tpl.TPL_REDUCE_SEPARATE) == 7
     small = tpl.Plan(tpl.make_dims(4096, 32, 32, 128, 11008, 32, 1e-5,
                                    tpl.TPL_NORM | tpl.TPL_RESIDUAL | tpl.TPL_ROPE), 4)
-    assert [small.decode_kernel_count(b) for b in (1, 8, 16)] == [6, 6, 7]
+    assert [small.decode_kernel_count(b) for b in (1, 2, 3, 8, 16)] == [6, 6, 7, 7, 7]  # tcgen05 from 3 tokens
     assert small.decode_kernel_count(16, n_layers=32) == 5 * 32 + 1 + 32
     with pytest.raises(tpl.TplError):
         p.decode_kernel_count(65)

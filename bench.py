@@ -402,7 +402,25 @@ def run_ours(args, ws, rank, local):
             step(x, y)
     torch.cuda.synchronize()
     assert plan.last_device_error() == tpl.TPL_OK
+    y_direct = y.clone()
     plan.reset_counters()
+    # one CUDA graph per step: the 401 launches of tpl_decode_stack captured
+    # once (their programmatic-dependent-launch edges included) and replayed;
+    # the reductions are counted by the host call, so during the capture
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            step(x, y)
+        y.zero_()
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                graph.replay()
+        torch.cuda.synchronize()
+        assert plan.last_device_error() == tpl.TPL_OK
+        assert torch.equal(y, y_direct), "graph replay differs from the direct calls"
+        reductions = plan.reduction_count() * args.steps
+    run_step = (lambda: graph.replay()) if graph is not None else (lambda: step(x, y))
     clocks = Clocks(local)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
@@ -410,24 +428,32 @@ def run_ours(args, ws, rank, local):
     clocks.start()
     time.sleep(0.3)
     e0.record(stream)
-    for _ in range(args.steps):
-        step(x, y)
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            run_step()
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, ws, dev)
-    reductions = plan.reduction_count()
+    if graph is None:
+        reductions = plan.reduction_count()
     tokens_per_s = ws * BATCH / (ms / 1e3)
 
     # ---- end to end: pinned host x in, y back to the host, every step ----
     xh = x.cpu().pin_memory()
     yh = torch.empty_like(xh).pin_memory()
     xd = torch.empty_like(x)
+    e2e_step = lambda: step(xd, y)
+    if graph is not None:
+        graph_e2e = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph_e2e, stream=stream):
+            step(xd, y)
+        e2e_step = lambda: graph_e2e.replay()
     with torch.cuda.stream(stream):
         for _ in range(2):
             xd.copy_(xh, non_blocking=True)
-            step(xd, y)
+            e2e_step()
             yh.copy_(y, non_blocking=True)
     torch.cuda.synchronize()
     barrier()
@@ -437,7 +463,7 @@ def run_ours(args, ws, rank, local):
     with torch.cuda.stream(stream):
         for _ in range(e2e_steps):
             xd.copy_(xh, non_blocking=True)
-            step(xd, y)
+            e2e_step()
             yh.copy_(y, non_blocking=True)
     f1.record(stream)
     torch.cuda.synchronize()
@@ -505,7 +531,10 @@ def run_ours(args, ws, rank, local):
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,0.02) weights, N(0,1) x/KV)",
                 "config": dict(config_dict(), step_hbm_gbs=step_gbs, step_hbm_frac=step_gbs / peak,
                                algorithmic_bytes_per_step=algorithmic_bytes_per_step(),
-                               reductions_counted=reductions // max(1, args.steps)),
+                               reductions_counted=reductions // max(1, args.steps),
+                               launch=("one CUDA graph per step (tpl_decode_stack captured once, replayed; "
+                                       "bit-identical to direct calls)") if graph is not None
+                               else "tpl_decode_stack called every step"),
                 "roofline": {"bound": "hbm", "kernel": gu_kernel, "achieved": gu_gbs,
                              "peak": peak, "peak_kind": peak_kind + " (burst copy, kernel timed alone)",
                              "unit": "GB/s", "frac": gu_gbs / peak, "traffic": recorded_traffic(),
@@ -719,6 +748,8 @@ def main():
                     help="shard the stack over the job's GPUs (one shard per rank, NCCL all-reduce) instead of "
                          "running an independent replica per GPU")
     ap.add_argument("--config-iters", type=int, default=30)
+    ap.add_argument("--no-graph", action="store_true",
+                    help="call tpl_decode_stack every step instead of replaying one captured CUDA graph")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

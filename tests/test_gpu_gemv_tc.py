@@ -123,6 +123,36 @@ def test_stack_equals_layer_sequence_tc(gpu):
     assert torch.equal(ys, y_stack)
 
 
+def test_stack_captured_in_cuda_graph(gpu):
+    """The decode stack captured once into a CUDA graph (its launches and
+    their programmatic-dependent-launch edges) and replayed gives the bits of
+    the direct call, replay after replay (every arrival counter resets itself
+    inside the kernels)."""
+    H, nq, nkv, F, t, B, S, NL = 2048, 16, 4, 5632, 2, 4, 300, 3
+    layers = [tc_layer(H, nq, nkv, 128, F, t, B, S, seed=9, layer=l, n_layers=NL) for l in range(NL)]
+    plan = layers[0].plan
+    x = layers[0].x
+    ws = plan.workspace(B, S)
+    snaps = [(L.k.clone(), L.v.clone()) for L in layers]
+    y = torch.empty_like(x)
+    plan.decode_stack([L.packed for L in layers], [L.kv for L in layers], x, S, y, None, ws)
+    torch.cuda.synchronize()
+    y_direct = y.clone()
+    stream = torch.cuda.Stream()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        plan.decode_stack([L.packed for L in layers], [L.kv for L in layers], x, S, y, None, ws)
+    for _ in range(3):
+        for L, (k, v) in zip(layers, snaps):
+            L.k.copy_(k)
+            L.v.copy_(v)
+        y.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(y, y_direct)
+    assert plan.last_device_error() == tpl.TPL_OK
+
+
 def test_repeated_calls_are_deterministic_tc(gpu):
     L = tc_layer(1024, 16, 8, 128, 2816, 8, 16, 500)
     a = run_steps(L)["y32"].clone()

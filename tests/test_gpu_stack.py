@@ -7,7 +7,7 @@ captured by running the stack truncated to that many layers (a plan with
 n_layers = l whose y is layer l-1's output), the oracle evaluates layer l on
 exactly those bits with layer l's weights and cache, and the full stack's
 output of layer l (the stack truncated to l+1 layers) must match it element
-by element at the benchmark spec's tolerance.  The pages' stack is 2L reductions
+by element at the 2e-2 tolerance.  The pages' stack is 2L reductions
 per forward pass ("Tensor parallel scaling curves", "What tensor parallelism
 actually splits"); each truncated run is checked to count 2 per layer.
 """

@@ -39,6 +39,7 @@ constexpr int kGemmThreads = 320;
 constexpr int kGemmEpiWarps = 8;
 constexpr int kGemmMTile = 128;
 constexpr int kGemmNTile = 256;
+constexpr int kGemmHalfN = kGemmNTile / 2;  // the width of a half tile of the last wave
 constexpr int kGemmKTile = 64;  // 128 bytes of bf16: one swizzle row
 constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s: far above any healthy wait
 
@@ -48,13 +49,15 @@ struct GemmArgs {
     CUtensorMap tm_a;   // A hi: [M][K] bf16 (2-D)
     CUtensorMap tm_a2;  // A lo (SPLIT_A)
     CUtensorMap tm_w;   // W: 2-D [N][K_pad] or 3-D [t][N][K_pad] (row-parallel)
+    CUtensorMap tm_wh;  // the same weights in boxes of kGemmHalfN rows (half tiles)
     int M, N;           // output rows (tokens), output columns
     int k_blocks;       // 64-column blocks per accumulation segment
     int nseg;           // segments per output tile (t for the fused row split, else 1)
     int a_col_stride;   // A column offset between shards (row-parallel), in elements
     int w3d;            // weights are the 3-D per-shard map
     int m_tiles, n_tiles;
-    int units;          // m_tiles * n_tiles (* t in the separate row mode: one unit per shard)
+    int units;          // work units: full_units whole tiles, then two half tiles per remaining tile
+    int full_units;     // tiles (m_tiles * n_tiles, * t in the separate row mode) done whole
     int epi;
     // epilogue outputs
     float *out32;       // GEPI_F32 / GEPI_ROW: [M][N]; GEPI_PARTIAL: [shards][M][N]
@@ -237,8 +240,17 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Unit u -> tile origin and the shard of a separate-mode unit.
-__device__ __forceinline__ void gemm_unit(const GemmArgs &a, int u, int &m0, int &n0, int &shard) {
+// Unit u -> tile origin, the shard of a separate-mode unit, and which half
+// of the tile's columns a half unit covers (-1: the whole tile).  Tiles past
+// full_units are done as two units of kGemmHalfN columns each, so that the
+// last, partial wave of tiles spreads over twice as many SMs.
+__device__ __forceinline__ void gemm_unit(const GemmArgs &a, int u, int &m0, int &n0, int &shard, int &half) {
+    half = -1;
+    if (u >= a.full_units) {
+        const int h = u - a.full_units;
+        u = a.full_units + (h >> 1);
+        half = h & 1;
+    }
     const int mt = u % a.m_tiles;
     const int r = u / a.m_tiles;
     m0 = mt * kGemmMTile;
@@ -375,10 +387,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
     if (warp == 0) {
         if (lane == 0) {
             constexpr unsigned TX = SM::A_BYTES * (SPLIT_A ? 2 : 1) + SM::W_BYTES;
+            constexpr unsigned TX_HALF = TX - SM::W_BYTES / 2;
             int it = 0;
             for (int u = blockIdx.x; u < a.units && !*s_fail; u += gridDim.x) {
-                int m0, n0, su;
-                gemm_unit(a, u, m0, n0, su);
+                int m0, n0, su, half;
+                gemm_unit(a, u, m0, n0, su, half);
+                const CUtensorMap *wm = half < 0 ? &a.tm_w : &a.tm_wh;
+                const int wn = half < 0 ? n0 : n0 + half * kGemmHalfN;
                 for (int seg = 0; seg < a.nseg && !*s_fail; ++seg) {
                     const int sh = su + seg;
                     for (int kb = 0; kb < a.k_blocks; ++kb, ++it) {
@@ -389,13 +404,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
                             break;
                         }
                         unsigned char *st = gsm + s * SM::STAGE;
-                        mbar_expect_tx(&full[s], TX);
+                        mbar_expect_tx(&full[s], half < 0 ? TX : TX_HALF);
                         const int ax = sh * a.a_col_stride + kb * kGemmKTile;
                         tma_load_2d(st, &a.tm_a, ax, m0, &full[s]);
                         if (SPLIT_A) tma_load_2d(st + SM::A_BYTES, &a.tm_a2, ax, m0, &full[s]);
                         unsigned char *wdst = st + SM::A_BYTES * (SPLIT_A ? 2 : 1);
-                        if (a.w3d) tma_load_3d(wdst, &a.tm_w, kb * kGemmKTile, n0, sh, &full[s]);
-                        else tma_load_2d(wdst, &a.tm_w, kb * kGemmKTile, n0, &full[s]);
+                        if (a.w3d) tma_load_3d(wdst, wm, kb * kGemmKTile, wn, sh, &full[s]);
+                        else tma_load_2d(wdst, wm, kb * kGemmKTile, wn, &full[s]);
                     }
                 }
             }
@@ -403,9 +418,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            constexpr uint32_t IDESC = umma_idesc(kGemmMTile, kGemmNTile);
+            constexpr uint32_t IDESC_FULL = umma_idesc(kGemmMTile, kGemmNTile);
+            constexpr uint32_t IDESC_HALF = umma_idesc(kGemmMTile, kGemmHalfN);
             int it = 0, c = 0;
             for (int u = blockIdx.x; u < a.units && !*s_fail; u += gridDim.x) {
+                // a half unit is an N = 128 product into the accumulator's
+                // first 128 columns, over the same K steps in the same order
+                const uint32_t IDESC = u < a.full_units ? IDESC_FULL : IDESC_HALF;
                 for (int seg = 0; seg < a.nseg && !*s_fail; ++seg, ++c) {
                     const int b = c & 1;
                     const unsigned use = (unsigned)(c >> 1);
@@ -451,10 +470,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(hf * 128);
         int c = 0;
         for (int u = blockIdx.x; u < a.units && !*s_fail; u += gridDim.x) {
-            int m0, n0, su;
-            gemm_unit(a, u, m0, n0, su);
+            int m0, n0, su, half;
+            gemm_unit(a, u, m0, n0, su, half);
             const int row = m0 + 32 * q + lane;
-            const int cb = n0 + hf * 128;
+            // a half unit's columns sit in accumulator columns [0, 128): the
+            // warps of the first column half store them, the others (cb = N)
+            // only keep the accumulator hand-off in step; so do warps whose
+            // columns all lie past N
+            const int cb = half < 0 ? n0 + hf * 128 : (hf == 0 ? n0 + half * kGemmHalfN : a.N);
+            const bool idle = cb >= a.N;
             float sum[ROWSUM ? 128 : 1];  // running sum of the shard partials (fused row split)
             bool ok = true;
             for (int seg = 0; seg < a.nseg; ++seg, ++c) {
@@ -467,7 +491,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
                 }
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
                 const uint32_t taddr = lane_base + (uint32_t)(b * kGemmNTile);
-                if constexpr (ROWSUM) {
+                if (idle) {
+                    // nothing of this unit in the second column half
+                } else if constexpr (ROWSUM) {
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         float v[16];
@@ -509,6 +535,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
             }
             if (!ok) break;
             if constexpr (ROWSUM) {
+                if (idle) continue;
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     float v[16];

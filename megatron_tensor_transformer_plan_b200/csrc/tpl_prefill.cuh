@@ -47,10 +47,15 @@ int gemm_go(int slot, GemmArgs &a, int shard_units, cudaStream_t st) {
     if (sms <= 0) return TPL_ECUDA;
     a.m_tiles = (a.M + kGemmMTile - 1) / kGemmMTile;
     a.n_tiles = (a.N + kGemmNTile - 1) / kGemmNTile;
-    const int64_t units = (int64_t)a.m_tiles * a.n_tiles * shard_units;
-    if (units > 0x7fffffff) return TPL_EUNSUPPORTED;
-    a.units = (int)units;
-    const int grid = (int)std::min<int64_t>(units, sms);
+    const int64_t tiles = (int64_t)a.m_tiles * a.n_tiles * shard_units;
+    if (2 * tiles > 0x7fffffff) return TPL_EUNSUPPORTED;
+    // A last wave that fills at most half the SMs runs as half tiles, two
+    // units per tile: it then ends in about half a tile's time.
+    const int64_t rem = tiles % sms;
+    const int64_t split = (rem > 0 && 2 * rem <= sms) ? rem : 0;
+    a.full_units = (int)(tiles - split);
+    a.units = (int)(tiles + split);
+    const int grid = (int)std::min<int64_t>(a.units, sms);
     return cuda_rc(launch_pdl(gemm_tc_kernel<SA, RS>, grid, kGemmThreads, (size_t)GemmSmem<SA>::BYTES, st, a));
 }
 
@@ -61,6 +66,7 @@ int gemm_column(GemmArgs &a, const void *a_hi, const void *a_lo, int64_t K, cons
     int rc = make_map(&a.tm_a, a_hi, K, a.M, K * 2, kGemmKTile, kGemmMTile);
     if (rc == TPL_OK && a_lo) rc = make_map(&a.tm_a2, a_lo, K, a.M, K * 2, kGemmKTile, kGemmMTile);
     if (rc == TPL_OK) rc = make_map(&a.tm_w, W, ld, N, ld * 2, kGemmKTile, kGemmNTile);
+    if (rc == TPL_OK) rc = make_map(&a.tm_wh, W, ld, N, ld * 2, kGemmKTile, kGemmHalfN);
     if (rc != TPL_OK) return rc;
     a.N = (int)N;
     a.k_blocks = (int)(ld / kGemmKTile);
@@ -83,6 +89,7 @@ int gemm_row(GemmArgs &a, const tpl_plan *p, const void *A, const void *A_lo, in
     if (rc == TPL_OK && A_lo)
         rc = make_map(&a.tm_a2, A_lo, (uint64_t)t * Ks, a.M, (uint64_t)t * Ks * 2, kGemmKTile, kGemmMTile);
     if (rc == TPL_OK) rc = make_map(&a.tm_w, W, ld, H, ld * 2, kGemmKTile, kGemmNTile, t, blk);
+    if (rc == TPL_OK) rc = make_map(&a.tm_wh, W, ld, H, ld * 2, kGemmKTile, kGemmHalfN, t, blk);
     if (rc != TPL_OK) return rc;
     a.N = (int)H;
     a.k_blocks = (int)(ld / kGemmKTile);

@@ -166,11 +166,17 @@ void tpl_plan_destroy(tpl_plan *plan);
  * TPL_SPLIT_O (the attention output into O) and TPL_SPLIT_GU (the normalised
  * h into gate/up); the down projection's operand (act) is always one part.
  * Default TPL_SPLIT_DEFAULT.
+ * TPL_OPT_PREFILL_TAIL: 1 (the default) runs a prefill projection's last,
+ * partial wave of 128 x 256 output tiles as 128 x 128 half tiles when it
+ * fills at most half the SMs (two units per tile over the same K steps in
+ * the same order: the results are bit-identical to whole tiles); 0 keeps
+ * every tile whole (kept to measure against and to check that identity).
  * Returns TPL_EINVAL for an unknown option or value. */
 #define TPL_OPT_GEMV_MODE 1
 #define TPL_OPT_PREFILL_ATTN 2
 #define TPL_OPT_DECODE_ATTN 3
 #define TPL_OPT_PREFILL_SPLIT 4
+#define TPL_OPT_PREFILL_TAIL 5
 #define TPL_SPLIT_QKV 1
 #define TPL_SPLIT_O 2
 #define TPL_SPLIT_GU 4

@@ -61,6 +61,7 @@ struct tpl_plan {
                     // 4: per projection (default for bf16)
     int attn_prefill_mode;  // 0: tcgen05 (power-of-two group sizes); 1: mma.sync
     int prefill_split;      // TPL_SPLIT_* bits: prefill operands carried as bf16 hi + lo
+    int prefill_tail;       // 1: a GEMM's partial last wave runs as half tiles
     int attn_decode_mode;   // 0: staged (g <= 8, pairs fit one wave); 1: register-streamed
     bool rope;
     double rope_theta[64];  // rope_base^(-2e/128), e < 64

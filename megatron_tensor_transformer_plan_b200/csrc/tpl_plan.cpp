@@ -248,6 +248,7 @@ int tpl_plan_create(const tpl_dims *dims, int32_t t, tpl_plan **out) {
     p->gemv_mode = p->f32 ? 1 : 4;
     p->attn_prefill_mode = 0;
     p->prefill_split = TPL_SPLIT_DEFAULT;
+    p->prefill_tail = 1;
     p->attn_decode_mode = 0;
     p->rope = (dims->flags & TPL_ROPE) != 0;
     for (int e = 0; e < 64; ++e)
@@ -303,6 +304,11 @@ int tpl_plan_set_option(tpl_plan *p, int32_t option, int32_t value) {
     if (option == TPL_OPT_PREFILL_SPLIT) {
         if (value < 0 || value > (TPL_SPLIT_QKV | TPL_SPLIT_O | TPL_SPLIT_GU)) return TPL_EINVAL;
         p->prefill_split = value;
+        return TPL_OK;
+    }
+    if (option == TPL_OPT_PREFILL_TAIL) {
+        if (value != 0 && value != 1) return TPL_EINVAL;
+        p->prefill_tail = value;
         return TPL_OK;
     }
     return TPL_EINVAL;

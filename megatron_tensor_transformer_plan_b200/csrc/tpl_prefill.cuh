@@ -34,7 +34,7 @@ namespace {
 bool g_gemm_attr[64][4];  // per device: dynamic shared memory attribute set, per instantiation
 
 template <bool SA, bool RS>
-int gemm_go(int slot, GemmArgs &a, int shard_units, cudaStream_t st) {
+int gemm_go(int slot, GemmArgs &a, int shard_units, bool halves, cudaStream_t st) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return TPL_ECUDA;
     if (!g_gemm_attr[dev][slot]) {
@@ -52,7 +52,7 @@ int gemm_go(int slot, GemmArgs &a, int shard_units, cudaStream_t st) {
     // A last wave that fills at most half the SMs runs as half tiles, two
     // units per tile: it then ends in about half a tile's time.
     const int64_t rem = tiles % sms;
-    const int64_t split = (rem > 0 && 2 * rem <= sms) ? rem : 0;
+    const int64_t split = (halves && rem > 0 && 2 * rem <= sms) ? rem : 0;
     a.full_units = (int)(tiles - split);
     a.units = (int)(tiles + split);
     const int grid = (int)std::min<int64_t>(a.units, sms);
@@ -61,8 +61,8 @@ int gemm_go(int slot, GemmArgs &a, int shard_units, cudaStream_t st) {
 
 // Column-parallel projection: A = bf16 hi (+ lo, when a_lo is not NULL)
 // [T][K] activations, W the shards' stacked rows [N][ld] (2-D).
-int gemm_column(GemmArgs &a, const void *a_hi, const void *a_lo, int64_t K, const void *W, int64_t N, int64_t ld,
-                cudaStream_t st) {
+int gemm_column(GemmArgs &a, const tpl_plan *p, const void *a_hi, const void *a_lo, int64_t K, const void *W,
+                int64_t N, int64_t ld, cudaStream_t st) {
     int rc = make_map(&a.tm_a, a_hi, K, a.M, K * 2, kGemmKTile, kGemmMTile);
     if (rc == TPL_OK && a_lo) rc = make_map(&a.tm_a2, a_lo, K, a.M, K * 2, kGemmKTile, kGemmMTile);
     if (rc == TPL_OK) rc = make_map(&a.tm_w, W, ld, N, ld * 2, kGemmKTile, kGemmNTile);
@@ -73,7 +73,8 @@ int gemm_column(GemmArgs &a, const void *a_hi, const void *a_lo, int64_t K, cons
     a.nseg = 1;
     a.a_col_stride = 0;
     a.w3d = 0;
-    return a_lo ? gemm_go<true, false>(0, a, 1, st) : gemm_go<false, false>(1, a, 1, st);
+    const bool halves = p->prefill_tail != 0;
+    return a_lo ? gemm_go<true, false>(0, a, 1, halves, st) : gemm_go<false, false>(1, a, 1, halves, st);
 }
 
 // Row-parallel projection: A [T][t*Ks] bf16 (shard s owns columns
@@ -95,14 +96,15 @@ int gemm_row(GemmArgs &a, const tpl_plan *p, const void *A, const void *A_lo, in
     a.k_blocks = (int)(ld / kGemmKTile);
     a.a_col_stride = (int)Ks;
     a.w3d = 1;
+    const bool halves = p->prefill_tail != 0;
     if (!fused) {
         a.nseg = 1;
         a.epi = GEPI_PARTIAL;
-        return A_lo ? gemm_go<true, false>(0, a, t, st) : gemm_go<false, false>(1, a, t, st);
+        return A_lo ? gemm_go<true, false>(0, a, t, halves, st) : gemm_go<false, false>(1, a, t, halves, st);
     }
     a.nseg = t;
     a.epi = GEPI_ROW;
-    return A_lo ? gemm_go<true, true>(2, a, 1, st) : gemm_go<false, true>(3, a, 1, st);
+    return A_lo ? gemm_go<true, true>(2, a, 1, halves, st) : gemm_go<false, true>(3, a, 1, halves, st);
 }
 
 GemmArgs gemm_args(int M) {
@@ -239,7 +241,7 @@ int prefill_layer(tpl_plan *p, const char *packed, const tpl_kv *kv, const void 
         a.pos0 = p0;
         a.rope = p->rope ? 1 : 0;
         std::memcpy(a.theta, p->rope_theta, sizeof(a.theta));
-        rc = gemm_column(a, a_hi, (p->prefill_split & TPL_SPLIT_QKV) ? a_lo : nullptr, H, packed + p->off_qkv,
+        rc = gemm_column(a, p, a_hi, (p->prefill_split & TPL_SPLIT_QKV) ? a_lo : nullptr, H, packed + p->off_qkv,
                          (int64_t)p->t * p->qkv_rows_s, p->ld_h, st);
         if (rc != TPL_OK) return rc;
     }
@@ -267,7 +269,7 @@ int prefill_layer(tpl_plan *p, const char *packed, const tpl_kv *kv, const void 
         a.epi = GEPI_GU;
         a.out_act = act;
         a.act_f32 = 0;
-        rc = gemm_column(a, a_hi, (p->prefill_split & TPL_SPLIT_GU) ? a_lo : nullptr, H, packed + p->off_gu,
+        rc = gemm_column(a, p, a_hi, (p->prefill_split & TPL_SPLIT_GU) ? a_lo : nullptr, H, packed + p->off_gu,
                          (int64_t)p->t * 2 * p->F_s, p->ld_h, st);
         if (rc != TPL_OK) return rc;
     }

@@ -1,12 +1,13 @@
 """Run the 70B-shaped layer prefill (t = 8, a chunk of 2048 tokens, causal
 attention inside the chunk) through the C-ABI: a self-contained workload for
-profilers and for timing (about 5 GB on the device, eight kernels per call).
+profilers and for timing (about 5 GB on the device, seven kernels per call).
 
     python -m megatron_tensor_transformer_plan_b200.profile_prefill [--calls N] [--mode fused|separate]
-        [--time] [--tokens T] [--start P0] [--rope]
+        [--time] [--tokens T] [--start P0] [--rope] [--whole-tiles]
 
 --start P0 makes the call a chunk at position P0 of a cache already holding P0
-tokens (tpl_prefill_chunk); --rope turns on the rotary embedding.  With --time
+tokens (tpl_prefill_chunk); --rope turns on the rotary embedding; --whole-tiles
+keeps every GEMM output tile whole (TPL_OPT_PREFILL_TAIL 0).  With --time
 it reports the CUDA-event time per call (after 3 warm-up calls) and the
 algorithmic FLOP rate: 2*T per weight for the four projections plus 4*d per
 (query head, key) pair that the causal mask keeps (T*P0 + T(T+1)/2 pairs per
@@ -39,6 +40,8 @@ def main() -> None:
     ap.add_argument("--time", action="store_true")
     ap.add_argument("--start", type=int, default=0)
     ap.add_argument("--rope", action="store_true")
+    ap.add_argument("--whole-tiles", action="store_true",
+                    help="keep every GEMM output tile whole (no half tiles in a partial last wave)")
     args = ap.parse_args()
     build.build()
     from megatron_tensor_transformer_plan_b200 import tpl
@@ -46,6 +49,8 @@ def main() -> None:
     T, P0 = args.tokens, args.start
     flags = tpl.TPL_NORM | tpl.TPL_RESIDUAL | (tpl.TPL_ROPE if args.rope else 0)
     plan = tpl.Plan(tpl.make_dims(H, NQ, NKV, D, F, 1, 1e-5, flags), TP)
+    if args.whole_tiles:
+        plan.set_option(tpl.TPL_OPT_PREFILL_TAIL, 0)
     w = synth.layer_weights(H, NQ, NKV, D, F, seed=0, device=dev)
     packed = plan.pack_layer(w)
     torch.cuda.synchronize()
@@ -85,7 +90,9 @@ def main() -> None:
     times.sort()
     med = times[len(times) // 2]
     rope = ", rope" if args.rope else ""
-    print(json.dumps({"workload": f"70B layer prefill t={TP} T={T} start={P0} ({args.mode}{rope})", "ms_median": med,
+    whole = ", whole tiles" if args.whole_tiles else ""
+    print(json.dumps({"workload": f"70B layer prefill t={TP} T={T} start={P0} ({args.mode}{rope}{whole})",
+                      "ms_median": med,
                       "ms_min": times[0], "tflops": (lin + att) / (med * 1e-3) / 1e12,
                       "device_status": plan.last_device_error()}))
 

@@ -29,6 +29,7 @@ TPL_OPT_GEMV_MODE = 1
 TPL_OPT_PREFILL_ATTN = 2
 TPL_OPT_DECODE_ATTN = 3
 TPL_OPT_PREFILL_SPLIT = 4
+TPL_OPT_PREFILL_TAIL = 5
 TPL_SPLIT_QKV, TPL_SPLIT_O, TPL_SPLIT_GU = 1, 2, 4
 TPL_SPLIT_DEFAULT = TPL_SPLIT_QKV | TPL_SPLIT_O | TPL_SPLIT_GU
 TPL_ATTN_STATIC_SCRATCH_BYTES = 4 * 1024 * 1024

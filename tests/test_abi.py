@@ -193,6 +193,15 @@ def test_gemv_option(tpl):
         plan.set_option(99, 0)
 
 
+def test_prefill_tail_option(tpl):
+    plan = tpl.Plan(tpl.make_dims(256, 2, 2, 128, 688), 2)
+    plan.set_option(tpl.TPL_OPT_PREFILL_TAIL, 0)
+    plan.set_option(tpl.TPL_OPT_PREFILL_TAIL, 1)
+    for bad in (-1, 2):
+        with pytest.raises(tpl.TplError):
+            plan.set_option(tpl.TPL_OPT_PREFILL_TAIL, bad)
+
+
 def test_prefill_chunk_validates_before_launch(tpl):
     """tpl_prefill_chunk's host checks: the chunk must fit the cache after its
     start position, the start must not be negative, fp32 plans are not

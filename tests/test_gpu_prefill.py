@@ -128,6 +128,51 @@ def test_prefill_small(gpu, case):
     check_prefill(Prefill(H, nq, nkv, F, t, T, gamma_std=0.02 if T > 100 else 0.0))
 
 
+def tile_waves(M, N, shards=1, sms=148):
+    """Output tiles of one prefill GEMM (128 x 256) and how many of them the
+    kernel runs as half tiles on `sms` SMs: the partial last wave, when it
+    fills at most half of them."""
+    tiles = -(-M // 128) * -(-N // 256) * shards
+    rem = tiles % sms
+    return tiles, (rem if 0 < rem and 2 * rem <= sms else 0)
+
+
+@pytest.mark.parametrize("flags", ["default", "rope"])
+def test_prefill_half_tiles_change_no_bits(gpu, flags):
+    """The half tiles of a partial last wave (N = 128 products over the same
+    K steps in the same order) give the same bits as whole tiles, for every
+    output of the layer, in both reduction modes."""
+    H, nq, nkv, F, t, T = 1024, 16, 8, 2816, 4, 1280
+    fl = None if flags == "default" else tpl.TPL_NORM | tpl.TPL_RESIDUAL | tpl.TPL_ROPE
+    P = Prefill(H, nq, nkv, F, t, T, seed=5, flags=fl)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    rps = (nq // t + 2 * (nkv // t)) * 128
+    # QKV 160 tiles (12 as halves), gate/up 220 (72), O and down fused 40 (all
+    # halves), separate 160 (12): both kinds of unit in every kernel family
+    waves = [tile_waves(T, t * rps, 1, sms), tile_waves(T, 2 * F, 1, sms), tile_waves(T, H, 1, sms),
+             tile_waves(T, H, t, sms)]
+    assert all(h > 0 for _, h in waves), waves
+    assert any(tiles > h for tiles, h in waves), waves
+
+    def outputs():
+        out = {}
+        for mode in (tpl.TPL_REDUCE_FUSED, tpl.TPL_REDUCE_SEPARATE):
+            y, y32 = P.run(mode)
+            out[f"y{mode}"], out[f"y32_{mode}"] = y, y32
+            out.update({f"{k}{mode}": v.clone() for k, v in P.intermediates().items()})
+            kt, vt, _ = P.cache()
+            out[f"k{mode}"], out[f"v{mode}"] = kt.clone(), vt.clone()
+        return out
+
+    P.plan.set_option(tpl.TPL_OPT_PREFILL_TAIL, 1)
+    halves = outputs()
+    P.plan.set_option(tpl.TPL_OPT_PREFILL_TAIL, 0)
+    whole = outputs()
+    for k in halves:
+        assert torch.equal(halves[k].view(torch.uint8), whole[k].view(torch.uint8)), k
+    assert P.plan.last_device_error() == tpl.TPL_OK
+
+
 @pytest.mark.parametrize("case", [(1024, 16, 4, 2816, 4, 200), (512, 16, 1, 512, 1, 64)])
 def test_prefill_mma_sync_attention(gpu, case):
     """The mma.sync attention kernel (kept to measure against) on group sizes

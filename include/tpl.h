@@ -143,7 +143,7 @@ void tpl_plan_destroy(tpl_plan *plan);
  * written by the preceding row-parallel kernel inside a layer or by a small
  * kernel, and the RMSNorm factor 1/rms is applied to their results), 4 = the
  * default: the tcgen05 kernels for every projection at any token count on
- * layers with at least 1 GiB of weights and from 3 tokens on any layer,
+ * layers with at least 1 GiB of weights and from 7 tokens on any layer,
  * mma.sync otherwise (the choice that measured faster on B200; layers mixing
  * the two families measured slower than either).  Above 16 tokens every mode runs
  * the tcgen05 kernels.  fp32 plans always use FFMA.  TPL_OPT_PREFILL_ATTN selects the prefill attention kernel:

@@ -278,9 +278,10 @@ int gemv_tc_run(Ctx &c, GemvTcArgs &a, int op, bool split, const void *W, int64_
 // TPL_OPT_GEMV_MODE 4 (the default for bf16 plans): one kernel family for all
 // four projections of a layer, the one that measured faster on B200 (layers
 // that mix the two families measured slower than either): tcgen05 on layers
-// of at least 1 GiB of weights at any token count (70B layer, one token: 305
-// against 345 us) and from 3 tokens on any layer, mma.sync for one or two
-// tokens on small layers (7B layer, one token: 113 against 117 us at t = 1).
+// of at least 1 GiB of weights at any token count (70B layer, one token: 304
+// against 312 us) and from 7 tokens on any layer, mma.sync for up to 6 tokens
+// on small layers (7B layer at t = 1, one token: 99.9 against 115.2 us; six:
+// 155.0 against 158.1; seven: 161.3 against 160.2).
 // Beyond 16 tokens (any mode) only the tcgen05 kernel applies.
 bool use_tc(const tpl_plan *p, int op, int B) {
     (void)op;
@@ -288,7 +289,7 @@ bool use_tc(const tpl_plan *p, int op, int B) {
     if (B > kMaxBatchCuda) return true;  // beyond the mma.sync kernel's 16 tokens
     if (p->gemv_mode == 3) return true;
     if (p->gemv_mode != 4) return false;
-    return large_layer(p) || B >= 3;
+    return large_layer(p) || B >= 7;
 }
 
 GemvTcArgs gt_args(const tpl_plan *p) {

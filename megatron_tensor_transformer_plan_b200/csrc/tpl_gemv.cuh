@@ -41,7 +41,13 @@ namespace tpl {
 
 enum { EPI_QKV = 0, EPI_GU = 1, EPI_ROW = 2, EPI_ROW_PARTIAL = 3 };
 
-constexpr int kPrefetchBlocks = 4;  // blocks per warp prefetched into L2 before the dependency wait (0, 4, 8, 16 measured: 4 fastest at one token)
+// How far (blocks per warp) an L2 prefetch runs ahead of the register loads:
+// issued before the dependency wait for the first blocks, then one block per
+// block loaded.  The register ring holds 2 blocks per warp (64 KB per SM in
+// flight), too few to cover DRAM latency alone; on the 7B layer at one token
+// distances of 2-3 took 99.9-100.6 us, 4 took 102.8, 8 took 108.9, 16 took
+// 115.1, and no in-loop prefetch 112.9.
+constexpr int kPrefetchBlocks = 3;
 
 struct GemvArgs {
     const char *W;   // first weight block
@@ -206,30 +212,31 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
     // Issue the first weight loads before waiting on the previous kernel, and
     // prefetch the next kPrefetchBlocks blocks of this warp's stream into L2
     // (each block: 8 rows x 128 columns; lanes with c == 0 cover both 128-byte
-    // lines of their row).
+    // lines of their row); the loop keeps that distance.
 #pragma unroll
     for (int d = 0; d < D; ++d)
         if (d < T_blocks) load_next(ring[d]);
-    {
-        int pr = lr, pj = lj;
-        const char *pp = lptr;
-        for (int q = 0; q < kPrefetchBlocks && pr < nrg_w && D + q < T_blocks; ++q) {
-            if (c == 0) {
-                prefetch_l2(pp);
-                prefetch_l2(pp + 64 * T::WES);
-                if (T::WES == 4) {
-                    prefetch_l2(pp + 128 * 2);
-                    prefetch_l2(pp + 128 * 3);
-                }
-            }
-            if (++pj == nblk) {
-                pj = 0;
-                if (++pr < nrg_w) pp = rowptr(pr);
-            } else {
-                pp += BLK_BYTES;
+    // L2 prefetch cursor (row group pr, block pj)
+    int pr = lr, pj = lj;
+    const char *pp = lptr;
+    auto prefetch_next = [&]() {
+        if (pr >= nrg_w) return;
+        if (c == 0) {
+            prefetch_l2(pp);
+            prefetch_l2(pp + 64 * T::WES);
+            if (T::WES == 4) {
+                prefetch_l2(pp + 128 * 2);
+                prefetch_l2(pp + 128 * 3);
             }
         }
-    }
+        if (++pj == nblk) {
+            pj = 0;
+            if (++pr < nrg_w) pp = rowptr(pr);
+        } else {
+            pp += BLK_BYTES;
+        }
+    };
+    for (int q = 0; q < kPrefetchBlocks && D + q < T_blocks; ++q) prefetch_next();
     pdl_wait();
     pdl_trigger();
     if (tid == 0) TPL_TRACE_AT(1);
@@ -548,7 +555,10 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const __grid_cons
             for (int d = 0; d < D; ++d) {
                 if (i + d < i_end) {
                     compute(ring[d], cj);
-                    if (i + d + D < T_blocks) load_next(ring[d]);
+                    if (i + d + D < T_blocks) {
+                        load_next(ring[d]);
+                        prefetch_next();
+                    }
                     if (++cj == nblk) {
                         write_part(r, cr);
                         cj = 0;

@@ -142,7 +142,7 @@ def test_decode_kernel_count(tpl):
     assert p.decode_kernel_count(4, tpl.TPL_REDUCE_SEPARATE) == 7
     small = tpl.Plan(tpl.make_dims(4096, 32, 32, 128, 11008, 32, 1e-5,
                                    tpl.TPL_NORM | tpl.TPL_RESIDUAL | tpl.TPL_ROPE), 4)
-    assert [small.decode_kernel_count(b) for b in (1, 2, 3, 8, 16)] == [6, 6, 7, 7, 7]  # tcgen05 from 3 tokens
+    assert [small.decode_kernel_count(b) for b in (1, 2, 6, 7, 8, 16)] == [6, 6, 6, 7, 7, 7]  # tcgen05 from 7 tokens
     assert small.decode_kernel_count(16, n_layers=32) == 5 * 32 + 1 + 32
     with pytest.raises(tpl.TplError):
         p.decode_kernel_count(65)
